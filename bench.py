@@ -1,0 +1,291 @@
+"""Benchmark of the forward NeRF render: one step = ray generation plus the full
+coarse + fine render of one 800x800 frame (64 stratified + 128 inverse-CDF
+samples per ray, 8x256 skip MLP with bf16 weights), all in libnerf's kernels.
+
+Prints one JSON line (rank 0). `--impl reference` times the CPU oracle on the
+same workload instead (a bounded sample of rays per step).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import nerf_inputs as S  # noqa: E402
+
+WORKLOAD = "full"
+METRIC = "rays/sec at 800x800 coarse+fine (64+128 samples/ray)"
+UNIT = "rays/s"
+MLP_FLOP_PER_ROW = 1186816          # algorithmic FLOPs of one 8x256 NeRF MLP evaluation
+
+
+def mlp_flops_per_row(shape):
+    return 2 * sum(n * k for name, n, k in shape.layer_shapes())
+
+
+def config_json(wl, n_gpus, extra=None):
+    c = {"workload": wl.name, "H": wl.H, "W": wl.W, "rays_per_frame": wl.n_rays,
+         "n_coarse": wl.n_coarse, "n_fine": wl.n_fine, "mlp": "8x256 skip@4, bf16 weights",
+         "mlp_rows_per_frame": wl.n_rays * (2 * wl.n_coarse + wl.n_fine),
+         "parallelism": f"rays sharded, {n_gpus} independent frame(s) per step",
+         "l2": "flushed between timed steps (256 MiB write)"}
+    if extra:
+        c.update(extra)
+    return c
+
+
+class ClockSampler:
+    def __init__(self, index):
+        self.proc = None
+        self.index = index
+
+    def __enter__(self):
+        q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={q}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in getattr(self, "lines", []):
+            f = [x.strip() for x in ln.split(",")]
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except (ValueError, IndexError):
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+def cpu_baseline(wl, n_rays_sample, seed=123):
+    """The oracle as it stands, on a bounded seeded sample of the frame's rays."""
+    from oracle import nerf as onerf
+    o, d = onerf.raygen(wl.H, wl.W, wl.focal, wl.c2w())
+    ids = S.ray_subset(wl.n_rays, n_rays_sample, seed)
+    cw, _ = S.nerf_weights(wl.mlp, wl.seed, 0, wl.sigma_scale, wl.precision)
+    fw, _ = S.nerf_weights(wl.mlp, wl.seed, 1, wl.sigma_scale, wl.precision)
+    t0 = time.perf_counter()
+    onerf.render_nerf(wl, o[ids], d[ids], ids, cw, fw)
+    dt = time.perf_counter() - t0
+    return len(ids) / dt, dt, len(ids)
+
+
+def n_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count()
+
+
+def run_reference(args, rank, world):
+    wl = S.WORKLOADS[WORKLOAD]
+    if rank != 0:
+        return
+    per_step = args.ref_rays
+    for _ in range(args.warmup):
+        cpu_baseline(wl, max(8, per_step // 8))
+    times = []
+    for k in range(args.steps):
+        r, dt, n = cpu_baseline(wl, per_step, seed=1000 + k)
+        times.append(dt)
+    rays = per_step * args.steps
+    value = rays / sum(times)
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000 * sum(times) / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": config_json(wl, world, {"sample_rays_per_step": per_step}),
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": n_cores(), "kind": "oracle",
+                             "sample": f"{per_step} seeded rays of the frame per step"},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import neural_radiance_field_b200 as nb
+    from neural_radiance_field_b200 import build as nbuild
+    nbuild.build()
+    torch.cuda.set_device(local_rank)
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    wl = S.WORKLOADS[WORKLOAD]
+    # each rank renders its own camera (weak scaling: one frame per GPU per step)
+    cam = S.look_at_c2w(*S.seeded_camera(wl.seed + 1000 * rank)) if rank else wl.c2w()
+    c2w = cam.ravel().tolist()
+    cw, _ = S.nerf_weights(wl.mlp, wl.seed, 0, wl.sigma_scale, wl.precision)
+    fw, _ = S.nerf_weights(wl.mlp, wl.seed, 1, wl.sigma_scale, wl.precision)
+    cwt = torch.from_numpy(cw).to(torch.bfloat16).cuda()
+    fwt = torch.from_numpy(fw).to(torch.bfloat16).cuda()
+    R = wl.n_rays
+    o = torch.empty(R, 3, device="cuda")
+    d = torch.empty(R, 3, device="cuda")
+    rgb = torch.empty(R, 3, device="cuda")
+    dep = torch.empty(R, device="cuda")
+    acc = torch.empty(R, device="cuda")
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    rnd = nb.Renderer(precision=S.PREC_BF16, max_rays=R, max_samples=wl.n_coarse + wl.n_fine)
+    p = rnd.params(coarse_w=cwt, fine_w=fwt, seed=wl.seed, perturb=1)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        nb.nerf_raygen(wl.H, wl.W, wl.focal, c2w, o, d)
+        rnd.render(o, d, wl.near, wl.far, wl.n_coarse, wl.n_fine, p, rgb, dep, acc)
+
+    for _ in range(args.warmup):
+        flush.fill_(1)
+        step()
+    torch.cuda.synchronize()
+    rnd.sync_status()
+    rnd.timing_enable(True)
+    rnd.timing_read()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local_rank) as clk:
+        for k in range(args.steps):
+            flush.fill_(k & 0xFF)
+            ev[k][0].record(stream)
+            step()
+            ev[k][1].record(stream)
+        torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    step_ms = [a.elapsed_time(b) for a, b in ev]
+    mlp_ms, mlp_launches = rnd.timing_read()
+    rnd.timing_enable(False)
+    rnd.sync_status()
+    tot_ms = sum(step_ms)
+    if dist:
+        t = torch.tensor([tot_ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        tot_ms = float(t.item())
+
+    # end to end through the host-buffer entry point (pinned host memory)
+    oh, dh = o.cpu().pin_memory(), d.cpu().pin_memory()
+    rgbh = torch.empty(R, 3).pin_memory()
+    deph = torch.empty(R).pin_memory()
+    acch = torch.empty(R).pin_memory()
+    e2e_steps = max(1, min(args.steps, 5))
+    rnd.render_host(oh, dh, wl.near, wl.far, wl.n_coarse, wl.n_fine, p, rgbh, deph, acch)
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        rnd.render_host(oh, dh, wl.near, wl.far, wl.n_coarse, wl.n_fine, p, rgbh, deph, acch)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / e2e_steps
+    if dist:
+        t = torch.tensor([e2e_ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+
+    rows = R * (2 * wl.n_coarse + wl.n_fine)
+    flops_launch_avg = MLP_FLOP_PER_ROW * rows / 2          # coarse + fine launches per frame
+    peaks, peak_kind = load_peaks()
+    avg_launch_ms = mlp_ms / max(1, mlp_launches)
+    achieved_tf = flops_launch_avg / (avg_launch_ms * 1e-3) / 1e12
+    peak_tf = peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops"))
+    value = world * R * args.steps / (tot_ms * 1e-3)
+    line = None
+    if rank == 0:
+        cpu = None
+        if world == 1 and not args.no_cpu_baseline:
+            rps, dt, n = cpu_baseline(wl, args.cpu_rays)
+            cpu = {"value": rps, "unit": UNIT, "cores": n_cores(), "kind": "oracle",
+                   "sample": f"{n} seeded rays of the 800x800 frame, full coarse+fine oracle render "
+                             f"({dt:.1f} s)"}
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": tot_ms / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded camera, Xavier-init weights)",
+            "config": config_json(wl, world),
+            "sample_points_per_s": value * (wl.n_coarse + wl.n_fine),
+            "mlp_rows_per_s": world * rows * args.steps / (tot_ms * 1e-3),
+            "roofline": {"bound": "tensor", "kernel": "scene MLP (coarse and fine launches)",
+                         "achieved": achieved_tf, "peak": peak_tf, "unit": "TFLOP/s",
+                         "frac": achieved_tf / peak_tf, "peak_kind": f"bf16 sustained, {peak_kind}",
+                         "traffic": None, "avg_launch_ms": avg_launch_ms,
+                         "flop_per_launch": flops_launch_avg},
+            "cpu_baseline": cpu,
+            "e2e": {"value": world * R / (e2e_ms * 1e-3), "unit": UNIT,
+                    "h2d_bytes_per_step": R * 24, "d2h_bytes_per_step": R * 20},
+            "gpu_launches": args.steps * 9,
+            "clocks": clk.summary(),
+        }
+        print(json.dumps(line), flush=True)
+    rnd.close()
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--cpu-rays", type=int, default=1024)
+    ap.add_argument("--ref-rays", type=int, default=128)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+    else:
+        run_ours(args, rank, world, local_rank)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,222 @@
+/*
+ * nerf.h - C ABI of the B200 forward NeRF renderer (libnerf.so, sm_100a).
+ *
+ * The library renders batches of rays with the method of "Spatial Intelligence -
+ * Part 1: NeRF" (halannhile.github.io): stratified samples on [near, far],
+ * positional encoding gamma(x), gamma(d), the scene MLP F_theta(x, d) -> (c, sigma),
+ * alpha compositing with T_i = exp(-sum_{j<i} sigma_j delta_j), then inverse-CDF
+ * resampling and a fine pass (Sections 1.3, 1.4 and 2.2-2.6 of that page). Two
+ * alternative scene functions march a 128^3 occupancy grid instead: a 16^3 grid
+ * of tiny MLPs (the KiloNeRF page, abstract) and a 3D multiresolution hash grid
+ * with a small MLP (the Instant-NGP notebook, "A shared toolkit" and Experiment 1).
+ *
+ * Conventions for every entry point:
+ *  - Pointers named *_host are host memory; every other buffer pointer is device
+ *    memory on the current CUDA device, owned by the caller, and must stay valid
+ *    until the work enqueued on `stream` has completed.
+ *  - `stream` is a cudaStream_t (NULL = legacy default stream). Calls only
+ *    enqueue work; they never synchronise, except nerf_render_host and
+ *    nerf_sync_status, which say so.
+ *  - Arrays are dense, row-major, fp32 unless stated; [R][3] means R rows of 3.
+ *  - Argument errors are reported synchronously (NERF_ERR_INVALID_ARG) before any
+ *    work is enqueued. Launch errors come back as NERF_ERR_CUDA. Errors that the
+ *    kernels detect set a device flag that nerf_sync_status reports.
+ *  - A context is not thread-safe; use one context per host thread.
+ *  - There is no CPU implementation behind this ABI: without a usable CUDA
+ *    device every call that needs one returns NERF_ERR_CUDA.
+ */
+#ifndef NERF_B200_H
+#define NERF_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define NERF_API __attribute__((visibility("default")))
+#else
+#define NERF_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct nerf_ctx nerf_ctx;
+
+typedef enum {
+  NERF_OK = 0,
+  NERF_ERR_INVALID_ARG = 1,   /* bad pointer, size or mode; nothing was enqueued */
+  NERF_ERR_CUDA = 2,          /* CUDA runtime or launch error */
+  NERF_ERR_UNSUPPORTED = 3,   /* valid request this build does not implement */
+  NERF_ERR_OOM = 4,           /* workspace allocation failed at create time */
+  NERF_ERR_TIMEOUT = 5,       /* a bounded device wait gave up */
+  NERF_ERR_DEVICE_FLAG = 6    /* a kernel reported an out-of-range input */
+} nerf_status;
+
+enum { NERF_MODEL_MLP = 0, NERF_MODEL_KILONERF = 1, NERF_MODEL_HASHGRID = 2 };
+enum { NERF_SIGMA_RELU = 0, NERF_SIGMA_SOFTPLUS = 1 };
+enum { NERF_FP32 = 0, NERF_BF16 = 1 };
+/* Length of the last interval of a ray: 1e10 as in the NeRF page's volume_render
+ * (Section 2.5), or up to `far` (the closed form of T(t) on [t_n, t_f]). */
+enum { NERF_LAST_1E10 = 0, NERF_LAST_TO_FAR = 1 };
+
+/* Fixed at create time. For NERF_MODEL_MLP the network is the NeRF page's
+ * F_theta (Section 2.4): D layers of width W with ReLU, gamma(x) concatenated
+ * after layer `skip` (skip < 0: none), sigma head Linear(W,1), feature layer
+ * Linear(W,W), direction layer Linear(W + 3(1+2 L_dir), W/2) + ReLU, rgb head
+ * Linear(W/2, 3). Supported: (W=256, D=8, skip=4) and (W=64, D in 1..8, no skip),
+ * L_pos = 10, L_dir = 4. precision BF16 selects the tensor-core path (W=256
+ * only); sigma_act and white_bkgd are applied in compositing.
+ * KILONERF and HASHGRID ignore D..precision. max_rays and max_samples size
+ * the context's workspace (max_samples >= n_coarse + n_fine of any render). */
+typedef struct {
+  int model;
+  int D, W, skip, L_pos, L_dir;
+  int sigma_act;
+  int precision;
+  int last_delta_mode;
+  int white_bkgd;
+  int64_t max_rays;
+  int max_samples;
+} nerf_config;
+
+/* Per-render inputs (device pointers unless stated).
+ *  coarse_w, fine_w  NERF_MODEL_MLP: flat parameter blobs, fp32 (precision FP32)
+ *                    or bf16 (precision BF16). Layer order: pts0..pts{D-1},
+ *                    sigma, feature, dir, rgb; each layer is its weight matrix
+ *                    [N_out][K_in] row-major followed by its bias [N_out].
+ *                    fine_w may be NULL when n_fine == 0.
+ *  occupancy         march models: 128^3 occupancy bits over [-1.5, 1.5)^3,
+ *                    uint32[65536]; voxel (ix,iy,iz) is bit (i & 31) of word
+ *                    i >> 5, i = (ix*128 + iy)*128 + iz.
+ *  cell_w            KILONERF: fp32 [4096][3317] per-cell parameters, cell id
+ *                    (cx*16+cy)*16+cz; per cell: W1[32][63] b1[32] W2[32][32]
+ *                    b2[32] w_sigma[32] b_sigma[1] Wc[3][59] bc[3].
+ *  hash_table        HASHGRID: fp16 [6101902][2], all 16 levels concatenated.
+ *  hash_mlp          HASHGRID: fp32 blob d0[64][32] b, d1[64][64] b, sigma[1][64] b,
+ *                    c0[64][80] b, c1[64][64] b, rgb[3][64] b.
+ *  march_step        march models: t_k = near + k * march_step, k < n_coarse.
+ *  ert_T             march models: stop a ray before the first occupied sample
+ *                    with transmittance below ert_T (0 disables).
+ *  seed, perturb     jitter of the stratified samples and the inverse-CDF draws
+ *                    (counter-based SplitMix64); perturb = 0 uses u = 0.5 for the
+ *                    jitter and evenly spaced draws (k + 0.5) / n_fine.
+ */
+typedef struct {
+  const void* coarse_w;
+  const void* fine_w;
+  const uint32_t* occupancy;
+  const float* cell_w;
+  const uint16_t* hash_table;
+  const float* hash_mlp;
+  float march_step;
+  float ert_T;
+  uint64_t seed;
+  int perturb;
+} nerf_params;
+
+/* Create a context: validates `cfg`, allocates the workspace on the current
+ * device (NERF_ERR_OOM on failure). *out is NULL on error. */
+NERF_API nerf_status nerf_create(const nerf_config* cfg, nerf_ctx** out);
+
+/* Free the workspace (synchronises the device first). NULL is a no-op. */
+NERF_API nerf_status nerf_destroy(nerf_ctx* ctx);
+
+/* Message of the last error on this context (or of the last failed create when
+ * ctx is NULL). Owned by the library; valid until the next call. */
+NERF_API const char* nerf_last_error(const nerf_ctx* ctx);
+
+/* Waits for `stream`, then reports launch errors and the device error flag
+ * (clearing it): NERF_OK, NERF_ERR_CUDA, NERF_ERR_TIMEOUT or
+ * NERF_ERR_DEVICE_FLAG. */
+NERF_API nerf_status nerf_sync_status(nerf_ctx* ctx, void* stream);
+
+/* Pinhole rays for an H x W image (NeRF page, Section 2.2, get_rays):
+ * camera-space direction ((i - W/2)/focal, -(j - H/2)/focal, -1) rotated by the
+ * upper 3x3 of c2w (not normalised), origin = c2w translation. Pixel (j, i)
+ * is row j*W + i. c2w_host: 12 floats, row-major [3][4], read during the call.
+ * rays_o, rays_d: [H*W][3]. Evaluated in IEEE fp32 without contraction. */
+NERF_API nerf_status nerf_raygen(int H, int W, float focal, const float* c2w_host,
+                        float* rays_o, float* rays_d, void* stream);
+
+/* Render n_rays rays (NeRF page, Section 2.6 render_rays):
+ *  NERF_MODEL_MLP: n_coarse stratified samples on [near, far] through the coarse
+ *    network; if n_fine > 0, n_fine inverse-CDF draws from the coarse weights of
+ *    the interior samples, the sorted union of n_coarse + n_fine positions
+ *    through the fine network; the output is the last pass. n_coarse must be 64
+ *    when n_fine > 0; n_coarse + n_fine <= max_samples.
+ *  march models: n_coarse fixed-step candidates (march_step), only occupied ones
+ *    evaluated; n_fine must be 0.
+ * Outputs: out_rgb [n_rays][3], out_depth [n_rays] (sum of w_i t_i, in t units),
+ * out_acc [n_rays] (sum of w_i). rays_o, rays_d: [n_rays][3]. 0 < n_rays <=
+ * max_rays, near < far. */
+NERF_API nerf_status nerf_render(nerf_ctx* ctx, const float* rays_o, const float* rays_d,
+                        int64_t n_rays, float near, float far, int n_coarse, int n_fine,
+                        const nerf_params* params, float* out_rgb, float* out_depth,
+                        float* out_acc, void* stream);
+
+/* nerf_render with HOST ray and output buffers (pinned memory recommended):
+ * copies the rays into the context's staging buffers, renders, copies the
+ * results back and synchronises `stream` before returning. */
+NERF_API nerf_status nerf_render_host(nerf_ctx* ctx, const float* rays_o_host, const float* rays_d_host,
+                             int64_t n_rays, float near, float far, int n_coarse, int n_fine,
+                             const nerf_params* params, float* out_rgb_host,
+                             float* out_depth_host, float* out_acc_host, void* stream);
+
+/* Device timing of the scene-network kernels, for benchmarks. While enabled,
+ * every network launch of nerf_render / nerf_test_mlp is bracketed by CUDA
+ * events recorded on the caller's stream (at most 4096 launches between reads;
+ * further launches are not timed). nerf_timing_read waits for the recorded
+ * events, returns the summed kernel time in milliseconds and the number of
+ * timed launches since the previous read, and starts a new count. */
+NERF_API nerf_status nerf_timing_enable(nerf_ctx* ctx, int enable);
+NERF_API nerf_status nerf_timing_read(nerf_ctx* ctx, double* ms, int64_t* launches);
+
+/* ---------------------------------------------------------------------------
+ * Unit entry points: one step of the path each, same conventions as above.
+ * ------------------------------------------------------------------------- */
+
+/* Stratified samples (NeRF page, Section 1.4.2): t_i = near + (i + u_i) * (far -
+ * near)/n in fp32 (step = (far-near)/n, s = i + u, t = near + s*step, each op
+ * rounded) and points x = o + t d (fp32, no contraction). out_t [R][n],
+ * out_x [R][n][3] (may be NULL). */
+NERF_API nerf_status nerf_test_stratified(const float* rays_o, const float* rays_d, int64_t n_rays,
+                                 float near, float far, int n, uint64_t seed, int perturb,
+                                 float* out_t, float* out_x, void* stream);
+
+/* Positional encoding (NeRF page, Section 1.4.1): [x, sin(2^k pi x_c),
+ * cos(2^k pi x_c)], sin and cos blocks coordinate-major. x [P][3], out [P][3+6L]. */
+NERF_API nerf_status nerf_test_pe(const float* x, int64_t n, int L, float* out, void* stream);
+
+/* The context's scene network on arbitrary points x [P][3] seen from directions
+ * d [P][3] (normalised inside): raw output [P][4] = (r, g, b, sigma) before
+ * activations. NERF_MODEL_MLP contexts only; P <= max_rays. */
+NERF_API nerf_status nerf_test_mlp(nerf_ctx* ctx, const void* weights, const float* x, const float* d,
+                          int64_t n, float* out_raw, void* stream);
+
+/* Compositing (NeRF page, Sections 1.3 and 2.5) of raw network outputs
+ * raw [R][S][4] at positions t [R][S] along rays with directions d [R][3]:
+ * delta_i = (t_{i+1} - t_i) ||d||, last interval per last_delta_mode (march_step
+ * * ||d|| when last_delta_mode == 2), sigma = act(raw), c = sigmoid(raw).
+ * Outputs rgb [R][3], depth [R], acc [R], weights [R][S] (may be NULL). */
+NERF_API nerf_status nerf_test_composite(const float* raw, const float* t, const float* rays_d,
+                                int64_t n_rays, int S, float far, int last_delta_mode,
+                                float march_step, int sigma_act, int white_bkgd,
+                                float* out_rgb, float* out_depth, float* out_acc,
+                                float* out_weights, void* stream);
+
+/* Inverse-CDF resampling and merge (NeRF page, Section 2.6 sample_pdf and the
+ * sorted union): bins are the fp32 midpoints of t_c [R][Nc], the pdf is
+ * weights[R][1..Nc-2] + 1e-5, draws u = m 2^-24 (seed, stream 1) or (k+0.5)/Nf.
+ * The CDF is exact: q_i = floor(fl32(w_i + 1e-5) 2^32), bin = #{k : C_k 2^24 <=
+ * m C_total}. out_t_fine [R][Nf] (draw order), out_below [R][Nf] int32 (bin
+ * index, may be NULL), out_t_all [R][Nc+Nf] ascending. Nc = 64, Nf <= 128. */
+NERF_API nerf_status nerf_test_sample_pdf(const float* t_coarse, const float* weights, int64_t n_rays,
+                                 int Nc, int Nf, uint64_t seed, int perturb, float* out_t_fine,
+                                 int32_t* out_below, float* out_t_all, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* NERF_B200_H */

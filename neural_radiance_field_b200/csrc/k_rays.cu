@@ -1,0 +1,142 @@
+// Ray generation, stratified sampling, positional encoding and the per-ray part
+// of the direction layer.
+#include "nerf_internal.cuh"
+
+namespace nerfb {
+
+struct C2W { float m[12]; };
+
+// get_rays of the NeRF page (Section 2.2): one thread per pixel, row-major.
+__global__ void raygen_kernel(int H, int W, float focal, C2W c, float* __restrict__ o,
+                              float* __restrict__ d) {
+  int64_t p = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (p >= (int64_t)H * W) return;
+  int j = (int)(p / W), i = (int)(p % W);
+  float dx = fdiv(fsub((float)i, fmul((float)W, 0.5f)), focal);
+  float dy = -fdiv(fsub((float)j, fmul((float)H, 0.5f)), focal);
+#pragma unroll
+  for (int r = 0; r < 3; ++r) {
+    float v = fadd(fadd(fmul(dx, c.m[r * 4 + 0]), fmul(dy, c.m[r * 4 + 1])),
+                   fmul(-1.0f, c.m[r * 4 + 2]));
+    d[p * 3 + r] = v;
+    o[p * 3 + r] = c.m[r * 4 + 3];
+  }
+}
+
+cudaError_t launch_raygen(int H, int W, float focal, const float* c2w, float* o, float* d,
+                          cudaStream_t st) {
+  C2W c;
+  for (int k = 0; k < 12; ++k) c.m[k] = c2w[k];
+  int64_t n = (int64_t)H * W;
+  raygen_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(H, W, focal, c, o, d);
+  return cudaGetLastError();
+}
+
+__global__ void stratified_kernel(const float* __restrict__ o, const float* __restrict__ d,
+                                  int64_t R, float near, float step, int n, uint64_t key,
+                                  int perturb, float* __restrict__ out_t,
+                                  float* __restrict__ out_x) {
+  int64_t q = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (q >= R * n) return;
+  int64_t r = q / n;
+  int i = (int)(q % n);
+  uint32_t m = perturb ? draw_bits(key, (uint64_t)r, 0, (uint32_t)i) : 0u;
+  float t = stratified_t(near, step, i, m, perturb != 0);
+  out_t[q] = t;
+  if (out_x) {
+#pragma unroll
+    for (int c = 0; c < 3; ++c) out_x[q * 3 + c] = fadd(o[r * 3 + c], fmul(t, d[r * 3 + c]));
+  }
+}
+
+cudaError_t launch_stratified(const float* o, const float* d, int64_t R, float near, float far,
+                              int n, uint64_t key, int perturb, float* out_t, float* out_x,
+                              cudaStream_t st) {
+  float step = (float)(far - near);  // fp32 subtraction of fp32 operands
+  step = step / (float)n;
+  int64_t tot = R * n;
+  stratified_kernel<<<(unsigned)((tot + 255) / 256), 256, 0, st>>>(o, d, R, near, step, n, key,
+                                                                    perturb, out_t, out_x);
+  return cudaGetLastError();
+}
+
+__global__ void pe_kernel(const float* __restrict__ x, int64_t n, int L, float* __restrict__ out) {
+  int dim = 3 + 6 * L;
+  int64_t q = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (q >= n * dim) return;
+  int64_t p = q / dim;
+  int j = (int)(q % dim);
+  float v;
+  if (j < 3) {
+    v = x[p * 3 + j];
+  } else {
+    int jj = (j - 3) % (3 * L);
+    int c = jj / L, k = jj % L;
+    float s, co;
+    pe_sincos(x[p * 3 + c], k, &s, &co);
+    v = (j - 3 < 3 * L) ? s : co;
+  }
+  out[q] = v;
+}
+
+cudaError_t launch_pe(const float* x, int64_t n, int L, float* out, cudaStream_t st) {
+  int64_t tot = n * (3 + 6 * L);
+  pe_kernel<<<(unsigned)((tot + 255) / 256), 256, 0, st>>>(x, n, L, out);
+  return cudaGetLastError();
+}
+
+__device__ __forceinline__ float load_param(const void* blob, int precision, int64_t i) {
+  if (precision == NERF_BF16) return __bfloat162float(((const __nv_bfloat16*)blob)[i]);
+  return ((const float*)blob)[i];
+}
+
+// One block of 256 threads covers 256 / (W/2) rays; thread j of a ray computes
+// output unit j of the direction layer's per-ray part.
+__global__ void dir_bias_kernel(const float* __restrict__ d, int64_t R, const void* blob,
+                                int precision, int W, int L_dir, int64_t w_off, int64_t b_off,
+                                float* __restrict__ out) {
+  const int Wh = W / 2;
+  const int dir_ch = 3 + 6 * L_dir;
+  const int rays_per_block = blockDim.x / Wh;
+  __shared__ float enc[8][32];
+  int local = threadIdx.x / Wh;
+  int j = threadIdx.x % Wh;
+  int64_t r = (int64_t)blockIdx.x * rays_per_block + local;
+  if (r < R && j < dir_ch) {
+    float dx = d[r * 3 + 0], dy = d[r * 3 + 1], dz = d[r * 3 + 2];
+    float inv = 1.0f / sqrtf(dx * dx + dy * dy + dz * dz);
+    float u[3] = {dx * inv, dy * inv, dz * inv};
+    float v;
+    if (j < 3) {
+      v = u[j];
+    } else {
+      int jj = (j - 3) % (3 * L_dir);
+      float s, c;
+      pe_sincos(u[jj / L_dir], jj % L_dir, &s, &c);
+      v = (j - 3 < 3 * L_dir) ? s : c;
+    }
+    enc[local][j] = v;
+  }
+  __syncthreads();
+  if (r >= R) return;
+  const int K = W + dir_ch;
+  float acc = load_param(blob, precision, b_off + j);
+  for (int k = 0; k < dir_ch; ++k)
+    acc = fmaf(load_param(blob, precision, w_off + (int64_t)j * K + W + k), enc[local][k], acc);
+  out[r * Wh + j] = acc;
+}
+
+cudaError_t launch_dir_bias(const float* d, int64_t R, const void* blob, int precision, int W,
+                            int L_dir, int64_t w_off, int64_t b_off, float* out,
+                            cudaStream_t st) {
+  int Wh = W / 2;
+  int rays_per_block = 256 / Wh;
+  if (rays_per_block > 8 || 3 + 6 * L_dir > 32 || 3 + 6 * L_dir > Wh)
+    return cudaErrorInvalidValue;
+  unsigned blocks = (unsigned)((R + rays_per_block - 1) / rays_per_block);
+  dir_bias_kernel<<<blocks, rays_per_block * Wh, 0, st>>>(d, R, blob, precision, W, L_dir, w_off,
+                                                          b_off, out);
+  return cudaGetLastError();
+}
+
+}  // namespace nerfb

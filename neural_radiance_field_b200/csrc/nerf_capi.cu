@@ -1,0 +1,418 @@
+// The C ABI: argument validation, the context's workspace and the order of the
+// kernels of one render (NeRF page, Section 2.6 render_rays).
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <string>
+
+#include "nerf_internal.cuh"
+#include "nerf_ctx.h"
+
+using namespace nerfb;
+
+namespace {
+
+thread_local std::string g_create_error;
+
+nerf_status fail(nerf_ctx* ctx, nerf_status st, const char* fmt, ...) __attribute__((format(printf, 3, 4)));
+nerf_status fail(nerf_ctx* ctx, nerf_status st, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof buf, fmt, ap);
+  va_end(ap);
+  if (ctx) ctx->err = buf; else g_create_error = buf;
+  return st;
+}
+
+nerf_status cuda_fail(nerf_ctx* ctx, cudaError_t e, const char* where) {
+  return fail(ctx, NERF_ERR_CUDA, "%s: %s", where, cudaGetErrorString(e));
+}
+
+#define NERF_CHECK_LAUNCH(ctx, expr)                                  \
+  do {                                                                \
+    cudaError_t e_ = (expr);                                          \
+    if (e_ != cudaSuccess) return cuda_fail((ctx), e_, #expr);        \
+  } while (0)
+
+template <class T>
+cudaError_t dalloc(T** p, size_t count) {
+  *p = nullptr;
+  if (count == 0) return cudaSuccess;
+  return cudaMalloc((void**)p, count * sizeof(T));
+}
+
+int64_t mlp_param_count(int D, int W, int skip, int pos_ch, int dir_ch) {
+  int64_t n = 0;
+  for (int l = 0; l < D; ++l) {
+    int k = l == 0 ? pos_ch : (l == skip + 1 ? W + pos_ch : W);
+    n += (int64_t)W * k + W;
+  }
+  n += W + 1;                                   // sigma
+  n += (int64_t)W * W + W;                      // feature
+  n += (int64_t)(W / 2) * (W + dir_ch) + W / 2; // dir
+  n += 3 * (W / 2) + 3;                         // rgb
+  return n;
+}
+
+// Offsets of the direction layer's weight and bias in the ABI blob.
+void dir_offsets(const nerf_config& c, int64_t* w_off, int64_t* b_off) {
+  const int pos_ch = 3 * (1 + 2 * c.L_pos);
+  int64_t n = 0;
+  for (int l = 0; l < c.D; ++l) {
+    int k = l == 0 ? pos_ch : (l == c.skip + 1 ? c.W + pos_ch : c.W);
+    n += (int64_t)c.W * k + c.W;
+  }
+  n += c.W + 1;
+  n += (int64_t)c.W * c.W + c.W;
+  *w_off = n;
+  *b_off = n + (int64_t)(c.W / 2) * (c.W + 3 * (1 + 2 * c.L_dir));
+}
+
+bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+
+}  // namespace
+
+extern "C" {
+
+const char* nerf_last_error(const nerf_ctx* ctx) {
+  return ctx ? ctx->err.c_str() : g_create_error.c_str();
+}
+
+nerf_status nerf_create(const nerf_config* cfg, nerf_ctx** out) {
+  if (!out) return fail(nullptr, NERF_ERR_INVALID_ARG, "out is NULL");
+  *out = nullptr;
+  if (!cfg) return fail(nullptr, NERF_ERR_INVALID_ARG, "cfg is NULL");
+  const nerf_config c = *cfg;
+  if (c.max_rays <= 0 || c.max_samples <= 0 || c.max_samples > 512)
+    return fail(nullptr, NERF_ERR_INVALID_ARG, "max_rays must be > 0 and 0 < max_samples <= 512");
+  if (c.last_delta_mode != NERF_LAST_1E10 && c.last_delta_mode != NERF_LAST_TO_FAR)
+    return fail(nullptr, NERF_ERR_INVALID_ARG, "last_delta_mode must be 0 or 1");
+  if (c.sigma_act != NERF_SIGMA_RELU && c.sigma_act != NERF_SIGMA_SOFTPLUS)
+    return fail(nullptr, NERF_ERR_INVALID_ARG, "sigma_act must be RELU or SOFTPLUS");
+  if (c.model == NERF_MODEL_MLP) {
+    if (c.L_pos != 10 || c.L_dir != 4)
+      return fail(nullptr, NERF_ERR_UNSUPPORTED, "L_pos must be 10 and L_dir 4");
+    bool big = (c.W == 256 && c.D == 8 && c.skip == 4);
+    bool tiny = (c.W == 64 && c.D >= 1 && c.D <= 8 && c.skip < 0);
+    if (!big && !tiny)
+      return fail(nullptr, NERF_ERR_UNSUPPORTED,
+                  "network must be (W=256, D=8, skip=4) or (W=64, D<=8, no skip)");
+    if (c.precision != NERF_FP32 && c.precision != NERF_BF16)
+      return fail(nullptr, NERF_ERR_INVALID_ARG, "precision must be FP32 or BF16");
+    if (c.precision == NERF_BF16 && !big)
+      return fail(nullptr, NERF_ERR_UNSUPPORTED, "BF16 tensor-core path needs W=256, D=8");
+  } else if (c.model == NERF_MODEL_KILONERF || c.model == NERF_MODEL_HASHGRID) {
+    return fail(nullptr, NERF_ERR_UNSUPPORTED, "march models are not built into this library yet");
+  } else {
+    return fail(nullptr, NERF_ERR_INVALID_ARG, "unknown model %d", c.model);
+  }
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return fail(nullptr, NERF_ERR_CUDA, "no CUDA device: %s", cudaGetErrorString(e));
+
+  nerf_ctx* ctx = new nerf_ctx();
+  ctx->cfg = c;
+  ctx->device = dev;
+  const int pos_ch = 3 * (1 + 2 * c.L_pos), dir_ch = 3 * (1 + 2 * c.L_dir);
+  ctx->plan = plan_fp32(c.D, c.W, c.skip, pos_ch, dir_ch);
+  ctx->n_params = mlp_param_count(c.D, c.W, c.skip, pos_ch, dir_ch);
+  const int64_t R = c.max_rays, S = c.max_samples;
+  bool ok = true;
+  ok &= dalloc(&ctx->packed, (size_t)ctx->plan.total) == cudaSuccess;
+  ok &= dalloc(&ctx->dir_bias, (size_t)(R * (c.W / 2))) == cudaSuccess;
+  ok &= dalloc(&ctx->raw, (size_t)(R * S * 4)) == cudaSuccess;
+  ok &= dalloc(&ctx->t_all, (size_t)(R * S)) == cudaSuccess;
+  ok &= dalloc(&ctx->stage, (size_t)(R * 11)) == cudaSuccess;
+  ok &= dalloc(&ctx->d_flag, 1) == cudaSuccess;
+  if (ok) ok &= cudaMemset(ctx->d_flag, 0, sizeof(unsigned)) == cudaSuccess;
+  if (ok && c.precision == NERF_BF16) ok &= tc_alloc(ctx) == cudaSuccess;
+  if (!ok) {
+    cudaGetLastError();
+    nerf_destroy(ctx);
+    return fail(nullptr, NERF_ERR_OOM, "workspace allocation failed for max_rays=%lld, max_samples=%d",
+                (long long)R, (int)S);
+  }
+  *out = ctx;
+  return NERF_OK;
+}
+
+nerf_status nerf_destroy(nerf_ctx* ctx) {
+  if (!ctx) return NERF_OK;
+  cudaDeviceSynchronize();
+  cudaFree(ctx->packed);
+  cudaFree(ctx->dir_bias);
+  cudaFree(ctx->raw);
+  cudaFree(ctx->t_all);
+  cudaFree(ctx->stage);
+  cudaFree(ctx->d_flag);
+  if (ctx->ev) {
+    for (int i = 0; i < 2 * kMaxTimed; ++i) cudaEventDestroy(ctx->ev[i]);
+    delete[] ctx->ev;
+  }
+  tc_free(ctx);
+  delete ctx;
+  return NERF_OK;
+}
+
+nerf_status nerf_sync_status(nerf_ctx* ctx, void* stream) {
+  if (!ctx) return fail(nullptr, NERF_ERR_INVALID_ARG, "ctx is NULL");
+  cudaStream_t st = (cudaStream_t)stream;
+  cudaError_t e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return cuda_fail(ctx, e, "cudaStreamSynchronize");
+  unsigned flag = 0;
+  e = cudaMemcpy(&flag, ctx->d_flag, sizeof flag, cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(ctx, e, "reading the device flag");
+  if (flag) {
+    cudaMemset(ctx->d_flag, 0, sizeof(unsigned));
+    if (flag & FLAG_TIMEOUT) return fail(ctx, NERF_ERR_TIMEOUT, "a bounded device wait gave up (flag 0x%x)", flag);
+    return fail(ctx, NERF_ERR_DEVICE_FLAG, "a kernel reported an out-of-range input (flag 0x%x)", flag);
+  }
+  return NERF_OK;
+}
+
+nerf_status nerf_raygen(int H, int W, float focal, const float* c2w_host, float* rays_o,
+                        float* rays_d, void* stream) {
+  if (H <= 0 || W <= 0 || !(focal > 0.0f) || !c2w_host || !rays_o || !rays_d)
+    return fail(nullptr, NERF_ERR_INVALID_ARG, "nerf_raygen: bad size, focal or NULL pointer");
+  NERF_CHECK_LAUNCH(nullptr, launch_raygen(H, W, focal, c2w_host, rays_o, rays_d, (cudaStream_t)stream));
+  return NERF_OK;
+}
+
+}  // extern "C"
+
+// --------------------------------------------------------------------------
+// render
+// --------------------------------------------------------------------------
+
+namespace {
+
+struct TimedScope {
+  nerf_ctx* ctx;
+  cudaStream_t st;
+  int slot = -1;
+  TimedScope(nerf_ctx* c, cudaStream_t s) : ctx(c), st(s) {
+    if (ctx->timing && ctx->n_timed < kMaxTimed) {
+      slot = ctx->n_timed++;
+      cudaEventRecord(ctx->ev[2 * slot], st);
+    }
+  }
+  ~TimedScope() {
+    if (slot >= 0) cudaEventRecord(ctx->ev[2 * slot + 1], st);
+  }
+};
+
+// Runs one network (coarse or fine) over R rays with S samples each.
+nerf_status run_network(nerf_ctx* ctx, const void* blob, const float* o, const float* d,
+                        int64_t R, const SampleSpec& ss, float* raw, cudaStream_t st) {
+  const nerf_config& c = ctx->cfg;
+  int64_t w_off, b_off;
+  dir_offsets(c, &w_off, &b_off);
+  NERF_CHECK_LAUNCH(ctx, launch_dir_bias(d, R, blob, c.precision, c.W, c.L_dir, w_off, b_off,
+                                         ctx->dir_bias, st));
+  if (c.precision == NERF_BF16 && ctx->tc_enabled) {
+    NERF_CHECK_LAUNCH(ctx, tc_pack(ctx, blob, st));
+    TimedScope ts(ctx, st);
+    NERF_CHECK_LAUNCH(ctx, tc_run(ctx, o, d, R, ss, raw, st));
+    return NERF_OK;
+  }
+  const int dir_ch = 3 * (1 + 2 * c.L_dir);
+  NERF_CHECK_LAUNCH(ctx, launch_pack_fp32(blob, c.precision, ctx->plan, dir_ch, ctx->packed, st));
+  TimedScope ts(ctx, st);
+  NERF_CHECK_LAUNCH(ctx, launch_mlp_fp32(ctx->plan, ctx->packed, ctx->dir_bias, o, d, R, ss, raw, st));
+  return NERF_OK;
+}
+
+nerf_status check_render_args(nerf_ctx* ctx, const float* o, const float* d, int64_t n_rays,
+                              float near, float far, int n_coarse, int n_fine,
+                              const nerf_params* p, const float* rgb, const float* depth,
+                              const float* acc) {
+  if (!ctx) return fail(nullptr, NERF_ERR_INVALID_ARG, "ctx is NULL");
+  const nerf_config& c = ctx->cfg;
+  if (!o || !d || !p || !rgb || !depth || !acc)
+    return fail(ctx, NERF_ERR_INVALID_ARG, "NULL ray, params or output pointer");
+  if (n_rays <= 0 || n_rays > c.max_rays)
+    return fail(ctx, NERF_ERR_INVALID_ARG, "n_rays=%lld outside (0, max_rays=%lld]",
+                (long long)n_rays, (long long)c.max_rays);
+  if (!(near < far)) return fail(ctx, NERF_ERR_INVALID_ARG, "near must be < far");
+  if (n_coarse <= 0 || n_fine < 0 || n_coarse + n_fine > c.max_samples)
+    return fail(ctx, NERF_ERR_INVALID_ARG, "n_coarse + n_fine must be in (0, max_samples=%d]",
+                c.max_samples);
+  if (c.model == NERF_MODEL_MLP) {
+    if (!p->coarse_w) return fail(ctx, NERF_ERR_INVALID_ARG, "coarse_w is NULL");
+    if (n_fine > 0) {
+      if (!p->fine_w) return fail(ctx, NERF_ERR_INVALID_ARG, "fine_w is NULL with n_fine > 0");
+      if (n_coarse != 64 || n_fine > 128)
+        return fail(ctx, NERF_ERR_UNSUPPORTED, "the fine pass needs n_coarse = 64, n_fine <= 128");
+    }
+    if (c.precision == NERF_BF16 && (!aligned16(p->coarse_w) || (n_fine > 0 && !aligned16(p->fine_w))))
+      return fail(ctx, NERF_ERR_INVALID_ARG, "bf16 weight blobs must be 16-byte aligned");
+  }
+  return NERF_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+nerf_status nerf_render(nerf_ctx* ctx, const float* rays_o, const float* rays_d, int64_t n_rays,
+                        float near, float far, int n_coarse, int n_fine, const nerf_params* params,
+                        float* out_rgb, float* out_depth, float* out_acc, void* stream) {
+  nerf_status s = check_render_args(ctx, rays_o, rays_d, n_rays, near, far, n_coarse, n_fine,
+                                    params, out_rgb, out_depth, out_acc);
+  if (s != NERF_OK) return s;
+  cudaStream_t st = (cudaStream_t)stream;
+  const nerf_config& c = ctx->cfg;
+  const int64_t R = n_rays;
+  const uint64_t key = sm64_mix(params->seed);
+  SampleSpec coarse{};
+  coarse.mode = SAMPLES_STRATIFIED;
+  coarse.S = n_coarse;
+  coarse.near = near;
+  coarse.step = (far - near) / (float)n_coarse;
+  coarse.key = key;
+  coarse.perturb = params->perturb;
+  CompositeSpec cs{c.last_delta_mode, far, 0.0f, c.sigma_act, c.white_bkgd};
+
+  s = run_network(ctx, params->coarse_w, rays_o, rays_d, R, coarse, ctx->raw, st);
+  if (s != NERF_OK) return s;
+  if (n_fine == 0) {
+    NERF_CHECK_LAUNCH(ctx, launch_composite(ctx->raw, coarse, rays_d, R, cs, out_rgb, out_depth,
+                                            out_acc, nullptr, st));
+    return NERF_OK;
+  }
+  NERF_CHECK_LAUNCH(ctx, launch_coarse_resample(ctx->raw, coarse, rays_d, R, cs, n_fine, key,
+                                                params->perturb, ctx->t_all, st));
+  SampleSpec fine{};
+  fine.mode = SAMPLES_GIVEN_T;
+  fine.S = n_coarse + n_fine;
+  fine.t = ctx->t_all;
+  s = run_network(ctx, params->fine_w, rays_o, rays_d, R, fine, ctx->raw, st);
+  if (s != NERF_OK) return s;
+  NERF_CHECK_LAUNCH(ctx, launch_composite(ctx->raw, fine, rays_d, R, cs, out_rgb, out_depth,
+                                          out_acc, nullptr, st));
+  return NERF_OK;
+}
+
+nerf_status nerf_render_host(nerf_ctx* ctx, const float* rays_o_host, const float* rays_d_host,
+                             int64_t n_rays, float near, float far, int n_coarse, int n_fine,
+                             const nerf_params* params, float* out_rgb_host, float* out_depth_host,
+                             float* out_acc_host, void* stream) {
+  nerf_status s = check_render_args(ctx, rays_o_host, rays_d_host, n_rays, near, far, n_coarse,
+                                    n_fine, params, out_rgb_host, out_depth_host, out_acc_host);
+  if (s != NERF_OK) return s;
+  cudaStream_t st = (cudaStream_t)stream;
+  const int64_t R = n_rays;
+  float* o = ctx->stage;
+  float* d = o + R * 3;
+  float* rgb = d + R * 3;
+  float* dep = rgb + R * 3;
+  float* acc = dep + R;
+  NERF_CHECK_LAUNCH(ctx, cudaMemcpyAsync(o, rays_o_host, R * 12, cudaMemcpyHostToDevice, st));
+  NERF_CHECK_LAUNCH(ctx, cudaMemcpyAsync(d, rays_d_host, R * 12, cudaMemcpyHostToDevice, st));
+  s = nerf_render(ctx, o, d, R, near, far, n_coarse, n_fine, params, rgb, dep, acc, stream);
+  if (s != NERF_OK) return s;
+  NERF_CHECK_LAUNCH(ctx, cudaMemcpyAsync(out_rgb_host, rgb, R * 12, cudaMemcpyDeviceToHost, st));
+  NERF_CHECK_LAUNCH(ctx, cudaMemcpyAsync(out_depth_host, dep, R * 4, cudaMemcpyDeviceToHost, st));
+  NERF_CHECK_LAUNCH(ctx, cudaMemcpyAsync(out_acc_host, acc, R * 4, cudaMemcpyDeviceToHost, st));
+  NERF_CHECK_LAUNCH(ctx, cudaStreamSynchronize(st));
+  return NERF_OK;
+}
+
+nerf_status nerf_timing_enable(nerf_ctx* ctx, int enable) {
+  if (!ctx) return fail(nullptr, NERF_ERR_INVALID_ARG, "ctx is NULL");
+  if (enable && !ctx->ev) {
+    ctx->ev = new cudaEvent_t[2 * kMaxTimed]();
+    for (int i = 0; i < 2 * kMaxTimed; ++i) {
+      cudaError_t e = cudaEventCreate(&ctx->ev[i]);
+      if (e != cudaSuccess) return cuda_fail(ctx, e, "cudaEventCreate");
+    }
+  }
+  ctx->timing = enable != 0;
+  ctx->n_timed = 0;
+  return NERF_OK;
+}
+
+nerf_status nerf_timing_read(nerf_ctx* ctx, double* ms, int64_t* launches) {
+  if (!ctx || !ms || !launches) return fail(ctx, NERF_ERR_INVALID_ARG, "NULL argument");
+  double tot = 0.0;
+  for (int i = 0; i < ctx->n_timed; ++i) {
+    cudaError_t e = cudaEventSynchronize(ctx->ev[2 * i + 1]);
+    if (e != cudaSuccess) return cuda_fail(ctx, e, "cudaEventSynchronize");
+    float t = 0.0f;
+    e = cudaEventElapsedTime(&t, ctx->ev[2 * i], ctx->ev[2 * i + 1]);
+    if (e != cudaSuccess) return cuda_fail(ctx, e, "cudaEventElapsedTime");
+    tot += t;
+  }
+  *ms = tot;
+  *launches = ctx->n_timed;
+  ctx->n_timed = 0;
+  return NERF_OK;
+}
+
+// ----------------------------------------------------------------- unit entry points
+
+nerf_status nerf_test_stratified(const float* rays_o, const float* rays_d, int64_t n_rays,
+                                 float near, float far, int n, uint64_t seed, int perturb,
+                                 float* out_t, float* out_x, void* stream) {
+  if (!rays_o || !rays_d || !out_t || n_rays <= 0 || n <= 0 || n > 65536 || !(near < far))
+    return fail(nullptr, NERF_ERR_INVALID_ARG, "nerf_test_stratified: bad argument");
+  NERF_CHECK_LAUNCH(nullptr, launch_stratified(rays_o, rays_d, n_rays, near, far, n, sm64_mix(seed),
+                                               perturb, out_t, out_x, (cudaStream_t)stream));
+  return NERF_OK;
+}
+
+nerf_status nerf_test_pe(const float* x, int64_t n, int L, float* out, void* stream) {
+  if (!x || !out || n <= 0 || L < 1 || L > 16)
+    return fail(nullptr, NERF_ERR_INVALID_ARG, "nerf_test_pe: bad argument");
+  NERF_CHECK_LAUNCH(nullptr, launch_pe(x, n, L, out, (cudaStream_t)stream));
+  return NERF_OK;
+}
+
+nerf_status nerf_test_mlp(nerf_ctx* ctx, const void* weights, const float* x, const float* d,
+                          int64_t n, float* out_raw, void* stream) {
+  if (!ctx) return fail(nullptr, NERF_ERR_INVALID_ARG, "ctx is NULL");
+  if (ctx->cfg.model != NERF_MODEL_MLP)
+    return fail(ctx, NERF_ERR_INVALID_ARG, "nerf_test_mlp needs an MLP context");
+  if (!weights || !x || !d || !out_raw || n <= 0 || n > ctx->cfg.max_rays)
+    return fail(ctx, NERF_ERR_INVALID_ARG, "nerf_test_mlp: bad argument");
+  if (ctx->cfg.precision == NERF_BF16 && !aligned16(weights))
+    return fail(ctx, NERF_ERR_INVALID_ARG, "bf16 weight blobs must be 16-byte aligned");
+  SampleSpec ss{};
+  ss.mode = SAMPLES_GIVEN_X;
+  ss.S = 1;
+  ss.t = x;
+  return run_network(ctx, weights, x, d, n, ss, out_raw, (cudaStream_t)stream);
+}
+
+nerf_status nerf_test_composite(const float* raw, const float* t, const float* rays_d,
+                                int64_t n_rays, int S, float far, int last_delta_mode,
+                                float march_step, int sigma_act, int white_bkgd, float* out_rgb,
+                                float* out_depth, float* out_acc, float* out_weights,
+                                void* stream) {
+  if (!raw || !t || !rays_d || !out_rgb || !out_depth || !out_acc || n_rays <= 0 || S <= 0 ||
+      S > 512 || last_delta_mode < 0 || last_delta_mode > 2 || !aligned16(raw))
+    return fail(nullptr, NERF_ERR_INVALID_ARG, "nerf_test_composite: bad argument");
+  SampleSpec ss{};
+  ss.mode = SAMPLES_GIVEN_T;
+  ss.S = S;
+  ss.t = t;
+  CompositeSpec cs{last_delta_mode, far, march_step, sigma_act, white_bkgd};
+  NERF_CHECK_LAUNCH(nullptr, launch_composite(raw, ss, rays_d, n_rays, cs, out_rgb, out_depth,
+                                              out_acc, out_weights, (cudaStream_t)stream));
+  return NERF_OK;
+}
+
+nerf_status nerf_test_sample_pdf(const float* t_coarse, const float* weights, int64_t n_rays,
+                                 int Nc, int Nf, uint64_t seed, int perturb, float* out_t_fine,
+                                 int32_t* out_below, float* out_t_all, void* stream) {
+  if (!t_coarse || !weights || n_rays <= 0 || Nc != 64 || Nf < 1 || Nf > 128 ||
+      (!out_t_fine && !out_t_all))
+    return fail(nullptr, NERF_ERR_INVALID_ARG, "nerf_test_sample_pdf: bad argument (Nc must be 64, 1 <= Nf <= 128)");
+  NERF_CHECK_LAUNCH(nullptr, launch_sample_pdf(t_coarse, weights, n_rays, Nc, Nf, sm64_mix(seed),
+                                               perturb, out_t_fine, out_below, out_t_all,
+                                               (cudaStream_t)stream));
+  return NERF_OK;
+}
+
+}  // extern "C"

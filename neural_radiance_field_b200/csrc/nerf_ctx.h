@@ -1,0 +1,41 @@
+// The context behind the opaque nerf_ctx handle.
+#pragma once
+
+#include <string>
+
+#include "nerf_internal.cuh"
+
+struct nerf_ctx {
+  nerf_config cfg{};
+  int device = -1;
+  std::string err;
+  int64_t n_params = 0;
+  nerfb::PackedFp32 plan{};
+
+  // workspace (device), sized at create for max_rays x max_samples
+  float* packed = nullptr;     // fp32 packed weights of the network being run
+  float* dir_bias = nullptr;   // [max_rays][W/2]
+  float* raw = nullptr;        // [max_rays * max_samples][4]
+  float* t_all = nullptr;      // [max_rays][max_samples]
+  float* stage = nullptr;      // host-path staging: o, d, rgb [R][3]; depth, acc [R]
+  unsigned* d_flag = nullptr;  // device error flag
+
+  // network-kernel timing (nerf_timing_enable / nerf_timing_read)
+  bool timing = false;
+  int n_timed = 0;
+  cudaEvent_t* ev = nullptr;   // 2 * kMaxTimed events, created on first enable
+
+  // tensor-core (bf16) path
+  bool tc_enabled = false;
+  void* tc_weights = nullptr;  // packed bf16 operand images + fp32 epilogue vectors
+  int num_sms = 0;
+};
+
+namespace nerfb {
+constexpr int kMaxTimed = 4096;
+cudaError_t tc_alloc(nerf_ctx* ctx);
+void tc_free(nerf_ctx* ctx);
+cudaError_t tc_pack(nerf_ctx* ctx, const void* blob, cudaStream_t st);
+cudaError_t tc_run(nerf_ctx* ctx, const float* o, const float* d, int64_t R,
+                   const SampleSpec& ss, float* raw, cudaStream_t st);
+}  // namespace nerfb

@@ -274,7 +274,7 @@ def render_nerf(wl, o, d, ray_ids, coarse_flat, fine_flat=None, seed=None, pertu
     ray_ids = np.asarray(ray_ids, dtype=np.int64)
     R = len(ray_ids)
     res = {k: [] for k in ("rgb", "depth", "acc", "t_c", "w_c", "t_f", "t_all", "below",
-                           "rgb_c", "acc_c")}
+                           "rgb_c", "acc_c", "sigma_last_raw")}
     for s in range(0, R, chunk):
         sl = slice(s, min(R, s + chunk))
         oo, dd, ids = o[sl], d[sl], ray_ids[sl]
@@ -292,6 +292,7 @@ def render_nerf(wl, o, d, ray_ids, coarse_flat, fine_flat=None, seed=None, pertu
         res["rgb_c"].append(rgb_c)
         res["acc_c"].append(acc_c)
         if wl.n_fine == 0:
+            res["sigma_last_raw"].append(raw[:, -1, 3])
             res["rgb"].append(rgb_c)
             res["depth"].append(dep_c)
             res["acc"].append(acc_c)
@@ -312,6 +313,7 @@ def render_nerf(wl, o, d, ray_ids, coarse_flat, fine_flat=None, seed=None, pertu
         col = sigmoid(raw[..., :3])
         delta = deltas(t_all, dn, wl.last_delta, far=wl.far)
         rgb, dep, acc, _ = composite(sig, col, t_all, delta, wl.white_bkgd)
+        res["sigma_last_raw"].append(raw[:, -1, 3])
         res["rgb"].append(rgb)
         res["depth"].append(dep)
         res["acc"].append(acc)

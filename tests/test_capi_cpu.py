@@ -1,0 +1,66 @@
+"""Host-side checks of the C ABI that need no GPU: the library loads, exports
+every entry point that include/nerf.h declares, and rejects bad arguments
+before touching a device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from neural_radiance_field_b200 import _capi
+from neural_radiance_field_b200 import build as nbuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    nbuild.build()
+    return _capi.lib()
+
+
+def header_functions():
+    with open(os.path.join(ROOT, "include", "nerf.h")) as f:
+        text = f.read()
+    return re.findall(r"NERF_API\s+[\w\s\*]+?\b(nerf_\w+)\s*\(", text)
+
+
+def test_header_declares_the_entry_points():
+    names = header_functions()
+    for n in ("nerf_create", "nerf_render", "nerf_destroy", "nerf_render_host", "nerf_raygen"):
+        assert n in names
+    assert set(names) == set(_capi.SIGNATURES), "binding and header disagree"
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in header_functions():
+        assert hasattr(lib, name), name
+
+
+def test_create_rejects_bad_configs_without_a_device(lib):
+    h = ctypes.c_void_p()
+    cfg = _capi.nerf_config(0, 8, 256, 4, 10, 4, 0, 0, 0, 0, 0, 192)      # max_rays = 0
+    assert lib.nerf_create(ctypes.byref(cfg), ctypes.byref(h)) == _capi.NERF_ERR_INVALID_ARG
+    assert h.value is None
+    assert b"max_rays" in lib.nerf_last_error(None)
+    cfg = _capi.nerf_config(0, 8, 128, 4, 10, 4, 0, 0, 0, 0, 16, 192)     # W = 128
+    assert lib.nerf_create(ctypes.byref(cfg), ctypes.byref(h)) == _capi.NERF_ERR_UNSUPPORTED
+    cfg = _capi.nerf_config(0, 4, 64, -1, 10, 4, 0, 1, 0, 0, 16, 192)     # bf16 tiny
+    assert lib.nerf_create(ctypes.byref(cfg), ctypes.byref(h)) == _capi.NERF_ERR_UNSUPPORTED
+    cfg = _capi.nerf_config(7, 8, 256, 4, 10, 4, 0, 0, 0, 0, 16, 192)     # unknown model
+    assert lib.nerf_create(ctypes.byref(cfg), ctypes.byref(h)) == _capi.NERF_ERR_INVALID_ARG
+    assert lib.nerf_create(None, ctypes.byref(h)) == _capi.NERF_ERR_INVALID_ARG
+
+
+def test_unit_entry_points_reject_null_and_bad_sizes(lib):
+    assert lib.nerf_test_pe(None, 4, 10, None, None) == _capi.NERF_ERR_INVALID_ARG
+    fake = ctypes.c_void_p(16)   # never dereferenced: validation fails first
+    assert lib.nerf_test_pe(fake, 0, 10, fake, None) == _capi.NERF_ERR_INVALID_ARG
+    assert lib.nerf_test_sample_pdf(fake, fake, 4, 32, 128, 0, 1, fake, None, None, None) \
+        == _capi.NERF_ERR_INVALID_ARG
+    assert lib.nerf_test_composite(fake, fake, fake, 4, 600, 6.0, 0, 0.0, 0, 0, fake, fake, fake,
+                                   None, None) == _capi.NERF_ERR_INVALID_ARG
+    assert lib.nerf_raygen(0, 4, 1.0, None, fake, fake, None) == _capi.NERF_ERR_INVALID_ARG
+    assert lib.nerf_render(None, fake, fake, 4, 2.0, 6.0, 64, 0, None, fake, fake, fake, None) \
+        == _capi.NERF_ERR_INVALID_ARG
+    assert lib.nerf_destroy(None) == _capi.NERF_OK
