@@ -18,7 +18,7 @@ struct PackSeg {
   int64_t src_off, dst_off;
   int N, K_take, K_pad, stride, transpose;
 };
-struct PackTable { PackSeg s[14]; int n; };
+struct PackTable { PackSeg s[24]; int n; };
 
 __global__ void pack_kernel(const void* __restrict__ src, int precision, PackTable tab,
                             float* __restrict__ dst) {
@@ -87,7 +87,7 @@ cudaError_t launch_pack_fp32(const void* blob, int precision, const PackedFp32& 
   t.s[t.n++] = {so, p.dir_w, W / 2, W, W, W + dir_ch, 1};
   so += (int64_t)(W / 2) * (W + dir_ch) + W / 2;
   // rgb [3][W/2] kept row-major, then its bias
-  if (t.n + 2 > 14) return cudaErrorInvalidValue;
+  if (t.n + 2 > 24) return cudaErrorInvalidValue;
   t.s[t.n++] = {so, p.rgb_w, 3 * (W / 2), 0, 0, 0, 0}; so += 3 * (W / 2);
   t.s[t.n++] = {so, p.rgb_b, 3, 0, 0, 0, 0};
   dim3 grid(64, t.n);
