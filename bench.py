@@ -152,6 +152,9 @@ def run_ours(args, rank, world, local_rank):
         import datetime
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     wl = S.WORKLOADS[WORKLOAD]
+    if args.size:
+        import dataclasses
+        wl = dataclasses.replace(wl, H=args.size, W=args.size, focal=1.25 * args.size)
     # each rank renders its own camera (weak scaling: one frame per GPU per step)
     cam = S.look_at_c2w(*S.seeded_camera(wl.seed + 1000 * rank)) if rank else wl.c2w()
     c2w = cam.ravel().tolist()
@@ -277,6 +280,8 @@ def main():
     ap.add_argument("--cpu-rays", type=int, default=1024)
     ap.add_argument("--ref-rays", type=int, default=128)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--size", type=int, default=0,
+                    help="render an SIZE x SIZE frame instead (profiling runs only)")
     args = ap.parse_args()
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))

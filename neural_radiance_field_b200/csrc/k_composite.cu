@@ -54,14 +54,16 @@ __device__ void composite_ray(const float* __restrict__ raw, const SampleSpec& s
       local += tau[c];
     }
   }
-  // exclusive scan of the lanes' sums
+  // exclusive scan of the lanes' sums (shifted inclusive scan: subtracting a
+  // lane's own sum would cancel catastrophically next to the 1e10 interval)
   float incl = local;
 #pragma unroll
   for (int off = 1; off < 32; off <<= 1) {
     float v = __shfl_up_sync(0xffffffffu, incl, off);
     if (lane >= off) incl += v;
   }
-  float run = incl - local;
+  float run = __shfl_up_sync(0xffffffffu, incl, 1);
+  if (lane == 0) run = 0.0f;
   float r = 0.f, g = 0.f, b = 0.f, dep = 0.f, acc = 0.f;
 #pragma unroll
   for (int c = 0; c < C; ++c) {

@@ -90,52 +90,67 @@ __device__ __forceinline__ float load_param(const void* blob, int precision, int
   return ((const float*)blob)[i];
 }
 
-// One block of 256 threads covers 256 / (W/2) rays; thread j of a ray computes
-// output unit j of the direction layer's per-ray part.
+// Thread j (< W/2) keeps row j of the direction layer's gamma(d) columns in
+// registers; the block walks over groups of RB rays, encodes their unit
+// directions into shared memory and writes RB outputs per thread.
+constexpr int DIR_RB = 8;
+constexpr int DIR_MAXCH = 27;
+
 __global__ void dir_bias_kernel(const float* __restrict__ d, int64_t R, const void* blob,
                                 int precision, int W, int L_dir, int64_t w_off, int64_t b_off,
                                 float* __restrict__ out) {
   const int Wh = W / 2;
   const int dir_ch = 3 + 6 * L_dir;
-  const int rays_per_block = blockDim.x / Wh;
-  __shared__ float enc[8][32];
-  int local = threadIdx.x / Wh;
-  int j = threadIdx.x % Wh;
-  int64_t r = (int64_t)blockIdx.x * rays_per_block + local;
-  if (r < R && j < dir_ch) {
-    float dx = d[r * 3 + 0], dy = d[r * 3 + 1], dz = d[r * 3 + 2];
-    float inv = 1.0f / sqrtf(dx * dx + dy * dy + dz * dz);
-    float u[3] = {dx * inv, dy * inv, dz * inv};
-    float v;
-    if (j < 3) {
-      v = u[j];
-    } else {
-      int jj = (j - 3) % (3 * L_dir);
-      float s, c;
-      pe_sincos(u[jj / L_dir], jj % L_dir, &s, &c);
-      v = (j - 3 < 3 * L_dir) ? s : c;
-    }
-    enc[local][j] = v;
-  }
-  __syncthreads();
-  if (r >= R) return;
+  const int j = threadIdx.x;
+  __shared__ float enc[DIR_RB][32];
   const int K = W + dir_ch;
-  float acc = load_param(blob, precision, b_off + j);
-  for (int k = 0; k < dir_ch; ++k)
-    acc = fmaf(load_param(blob, precision, w_off + (int64_t)j * K + W + k), enc[local][k], acc);
-  out[r * Wh + j] = acc;
+  float w[DIR_MAXCH];
+#pragma unroll
+  for (int k = 0; k < DIR_MAXCH; ++k)
+    w[k] = k < dir_ch ? load_param(blob, precision, w_off + (int64_t)j * K + W + k) : 0.0f;
+  const float b = load_param(blob, precision, b_off + j);
+  for (int64_t r0 = (int64_t)blockIdx.x * DIR_RB; r0 < R; r0 += (int64_t)gridDim.x * DIR_RB) {
+    __syncthreads();
+    for (int q = j; q < DIR_RB * dir_ch; q += Wh) {
+      const int rr = q / dir_ch, k = q % dir_ch;
+      const int64_t r = r0 + rr;
+      float v = 0.0f;
+      if (r < R) {
+        float dx = d[r * 3 + 0], dy = d[r * 3 + 1], dz = d[r * 3 + 2];
+        float inv = 1.0f / sqrtf(dx * dx + dy * dy + dz * dz);
+        float u[3] = {dx * inv, dy * inv, dz * inv};
+        if (k < 3) {
+          v = u[k];
+        } else {
+          int kk = (k - 3) % (3 * L_dir);
+          float s, c;
+          pe_sincos(u[kk / L_dir], kk % L_dir, &s, &c);
+          v = (k - 3 < 3 * L_dir) ? s : c;
+        }
+      }
+      enc[rr][k] = v;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int rr = 0; rr < DIR_RB; ++rr) {
+      const int64_t r = r0 + rr;
+      if (r >= R) break;
+      float acc = b;
+#pragma unroll
+      for (int k = 0; k < DIR_MAXCH; ++k) acc = fmaf(w[k], enc[rr][k], acc);
+      out[r * Wh + j] = acc;
+    }
+  }
 }
 
 cudaError_t launch_dir_bias(const float* d, int64_t R, const void* blob, int precision, int W,
                             int L_dir, int64_t w_off, int64_t b_off, float* out,
                             cudaStream_t st) {
-  int Wh = W / 2;
-  int rays_per_block = 256 / Wh;
-  if (rays_per_block > 8 || 3 + 6 * L_dir > 32 || 3 + 6 * L_dir > Wh)
-    return cudaErrorInvalidValue;
-  unsigned blocks = (unsigned)((R + rays_per_block - 1) / rays_per_block);
-  dir_bias_kernel<<<blocks, rays_per_block * Wh, 0, st>>>(d, R, blob, precision, W, L_dir, w_off,
-                                                          b_off, out);
+  const int Wh = W / 2;
+  if (3 + 6 * L_dir > DIR_MAXCH || Wh < 32 || Wh > 1024) return cudaErrorInvalidValue;
+  int64_t groups = (R + DIR_RB - 1) / DIR_RB;
+  unsigned blocks = (unsigned)(groups < 148 * 16 ? groups : 148 * 16);
+  dir_bias_kernel<<<blocks, Wh, 0, st>>>(d, R, blob, precision, W, L_dir, w_off, b_off, out);
   return cudaGetLastError();
 }
 

@@ -88,6 +88,7 @@ def test_mlp_rows(torch, key):
     ref = onerf.nerf_mlp(shape, p, onerf.positional_encoding(x.astype(np.float64), shape.L_pos),
                          onerf.positional_encoding(onerf.unit(dv), shape.L_dir))
     err = np.abs(out.cpu().numpy() - ref).max()
+    print(f"[mlp_rows {key}] max raw error {err:.3e} (bound {RAW_BOUND[wl.precision]:.1e})")
     assert err <= RAW_BOUND[wl.precision], err
 
 
