@@ -215,6 +215,39 @@ NERF_API nerf_status nerf_test_sample_pdf(const float* t_coarse, const float* we
                                  int Nc, int Nf, uint64_t seed, int perturb, float* out_t_fine,
                                  int32_t* out_below, float* out_t_all, void* stream);
 
+/* Occupancy march (empty-space skipping over the 128^3 grid of nerf_params):
+ * candidates t_k = near + k * step (fp32, k < K <= 512), points x = o + t_k d
+ * (fp32, no contraction); a point is live when it lies in [-1.5, 1.5)^3 and its
+ * voxel (the exact floor of (x + 1.5) * 128 / 3 per axis) is occupied.
+ * out_count [R] int32: live candidates per ray; out_live [R][K] uint8 (may be
+ * NULL): 1 where candidate k is live. */
+NERF_API nerf_status nerf_test_march(const float* rays_o, const float* rays_d, int64_t n_rays,
+                                     float near, float step, int K, const uint32_t* occupancy,
+                                     int32_t* out_count, uint8_t* out_live, void* stream);
+
+/* KiloNeRF routing of points x [P][3] (inside [-1.5, 1.5)^3): out_cell [P]
+ * int32 = (cx*16 + cy)*16 + cz with c = voxel >> 3; out_cell_count [4096] and
+ * out_cell_offset [4097] int32 (exclusive scan); out_order [P] int32 (may be
+ * NULL): point indices grouped by cell (cell-major; order inside a cell
+ * unspecified). */
+NERF_API nerf_status nerf_test_route_cells(const float* x, int64_t n, int32_t* out_cell,
+                                           int32_t* out_cell_count, int32_t* out_cell_offset,
+                                           int32_t* out_order, void* stream);
+
+/* Hash-grid encoding (Instant-NGP notebook, HashGrid2D.encode, extended to 3D):
+ * 16 levels N_l = round(16 b^l), b = (2048/16)^(1/15); T = 2^19 entries per level,
+ * 2 fp16 features per entry (table: nerf_params.hash_table layout); direct
+ * index (ix*(N+1)+iy)*(N+1)+iz while (N+1)^3 <= T, else (ix XOR iy*2654435761
+ * XOR iz*805459861) mod T; trilinear weights of c = fl(fl((x + 1.5)/3) * N).
+ * x [P][3]; out_feat [P][32] (level-major); out_rows [P][16][8] int32 (may be
+ * NULL): global table row of every corner (dx, dy, dz loop order). */
+NERF_API nerf_status nerf_test_hash_encode(const float* x, int64_t n, const uint16_t* hash_table,
+                                           float* out_feat, int32_t* out_rows, void* stream);
+
+/* Real spherical harmonics of bands 0..3 (16 values, index l*l + l + m, no
+ * Condon-Shortley phase) of the unit vectors d/|d|; d [P][3], out [P][16]. */
+NERF_API nerf_status nerf_test_sh(const float* d, int64_t n, float* out, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

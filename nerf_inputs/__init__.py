@@ -261,11 +261,13 @@ class HashGridShape:
     N_max: int = 2048
 
 
-def hashgrid_table(shape: HashGridShape, sizes, seed: int, scale: float):
-    """All levels' feature tables concatenated, fp16 [sum(sizes)][F], U(+-scale)."""
+HASH_ENTRIES = 6101902   # rows of the 16 concatenated level tables of HashGridShape()
+
+
+def hashgrid_table(shape: HashGridShape, n_entries: int, seed: int, scale: float):
+    """All levels' feature tables concatenated, fp16 [n_entries][F], U(+-scale)."""
     rng = np.random.default_rng([seed, 53])
-    total = int(sum(sizes))
-    return rng.uniform(-scale, scale, size=(total, shape.F)).astype(np.float16)
+    return rng.uniform(-scale, scale, size=(int(n_entries), shape.F)).astype(np.float16)
 
 
 HASH_MLP_HIDDEN = 64

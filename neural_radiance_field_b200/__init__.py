@@ -79,6 +79,29 @@ def nerf_test_sample_pdf(t_coarse, weights, n_fine, seed, perturb, out_t_fine=No
         _ptr(out_t_fine), _ptr(out_below), _ptr(out_t_all), _stream(stream)))
 
 
+def nerf_test_march(rays_o, rays_d, near, step, K, occupancy, out_count, out_live=None,
+                    stream=None):
+    _capi.check(_capi.lib().nerf_test_march(
+        _ptr(rays_o), _ptr(rays_d), rays_o.shape[0], float(near), float(step), int(K),
+        _ptr(occupancy), _ptr(out_count), _ptr(out_live), _stream(stream)))
+
+
+def nerf_test_route_cells(x, out_cell, out_cell_count, out_cell_offset, out_order=None,
+                          stream=None):
+    _capi.check(_capi.lib().nerf_test_route_cells(
+        _ptr(x), x.shape[0], _ptr(out_cell), _ptr(out_cell_count), _ptr(out_cell_offset),
+        _ptr(out_order), _stream(stream)))
+
+
+def nerf_test_hash_encode(x, hash_table, out_feat, out_rows=None, stream=None):
+    _capi.check(_capi.lib().nerf_test_hash_encode(
+        _ptr(x), x.shape[0], _ptr(hash_table), _ptr(out_feat), _ptr(out_rows), _stream(stream)))
+
+
+def nerf_test_sh(d, out, stream=None):
+    _capi.check(_capi.lib().nerf_test_sh(_ptr(d), d.shape[0], _ptr(out), _stream(stream)))
+
+
 class Renderer:
     """Owns a nerf_ctx (nerf_create / nerf_destroy)."""
 

@@ -68,6 +68,10 @@ SIGNATURES = {
     "nerf_test_mlp": (_I, [_P, _P, _P, _P, _I64, _P, _P]),
     "nerf_test_composite": (_I, [_P, _P, _P, _I64, _I, _F, _I, _F, _I, _I, _P, _P, _P, _P, _P]),
     "nerf_test_sample_pdf": (_I, [_P, _P, _I64, _I, _I, _U64, _I, _P, _P, _P, _P]),
+    "nerf_test_march": (_I, [_P, _P, _I64, _F, _F, _I, _P, _P, _P, _P]),
+    "nerf_test_route_cells": (_I, [_P, _I64, _P, _P, _P, _P, _P]),
+    "nerf_test_hash_encode": (_I, [_P, _I64, _P, _P, _P, _P]),
+    "nerf_test_sh": (_I, [_P, _I64, _P, _P]),
 }
 
 _lib = None

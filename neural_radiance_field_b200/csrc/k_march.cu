@@ -1,0 +1,606 @@
+// Marching scene functions: occupancy-grid empty-space skipping, the 3D
+// multiresolution hash grid with its small MLP (Instant-NGP notebook, "A shared
+// toolkit" and Experiment 1, in 3D), the KiloNeRF grid of tiny MLPs with a cell
+// router (KiloNeRF page, abstract), and compositing with early termination.
+#include <cmath>
+
+#include "nerf_march.cuh"
+
+namespace nerfb {
+
+// ------------------------------------------------------------------ occupancy
+
+// Voxel of one coordinate by exact comparison with the boundaries b_v = -1.5 +
+// v * 3/128 (exact in fp32): returns -1 outside [-1.5, 1.5).
+__device__ __forceinline__ int voxel_axis(float x) {
+  if (!(x >= -1.5f) || !(x < 1.5f)) return -1;
+  int v = (int)floorf(fmul(fadd(x, 1.5f), 42.666666666666664f));
+  v = v < 0 ? 0 : (v > 127 ? 127 : v);
+  if (x < fsub(fmul((float)v, 0.0234375f), 1.5f)) --v;
+  else if (v < 127 && x >= fsub(fmul((float)(v + 1), 0.0234375f), 1.5f)) ++v;
+  return v;
+}
+
+__device__ __forceinline__ bool occupied_at(const uint32_t* __restrict__ occ, float x0, float x1,
+                                            float x2, int* vox) {
+  const int a = voxel_axis(x0), b = voxel_axis(x1), c = voxel_axis(x2);
+  if (a < 0 || b < 0 || c < 0) return false;
+  const int idx = (a * 128 + b) * 128 + c;
+  if (vox) *vox = idx;
+  return (__ldg(occ + (idx >> 5)) >> (idx & 31)) & 1u;
+}
+
+__device__ __forceinline__ void march_point(const float* o, const float* d, int64_t r, float near,
+                                            float step, int k, float* x, float* t) {
+  *t = fadd(near, fmul((float)k, step));
+#pragma unroll
+  for (int c = 0; c < 3; ++c) x[c] = fadd(o[r * 3 + c], fmul(*t, d[r * 3 + c]));
+}
+
+// Warp per ray: live bitmask (K <= 512 -> 16 words) and live count.
+__global__ void march_mask_kernel(const float* __restrict__ o, const float* __restrict__ d,
+                                  int64_t R, float near, float step, int K,
+                                  const uint32_t* __restrict__ occ, uint32_t* __restrict__ mask,
+                                  int32_t* __restrict__ count, uint8_t* __restrict__ live_u8) {
+  const int lane = threadIdx.x & 31;
+  const int64_t r = (int64_t)blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;
+  if (r >= R) return;
+  int n = 0;
+  for (int w = 0; w < (K + 31) / 32; ++w) {
+    const int k = w * 32 + lane;
+    bool live = false;
+    if (k < K) {
+      float x[3], t;
+      march_point(o, d, r, near, step, k, x, &t);
+      live = occupied_at(occ, x[0], x[1], x[2], nullptr);
+      if (live_u8) live_u8[r * K + k] = live;
+    }
+    const uint32_t m = __ballot_sync(0xffffffffu, live);
+    if (lane == 0 && mask) mask[r * 16 + w] = m;
+    n += __popc(m);
+  }
+  if (lane == 0) count[r] = n;
+}
+
+// Live entries (ray << 9 | k) in ray-major order from the masks and offsets;
+// entries past `cap` are dropped and flagged.
+__global__ void march_emit_kernel(const uint32_t* __restrict__ mask, const int32_t* __restrict__ off,
+                                  int64_t R, int K, uint32_t* __restrict__ live, int64_t cap,
+                                  unsigned* flag) {
+  const int lane = threadIdx.x & 31;
+  const int64_t r = (int64_t)blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;
+  if (r >= R) return;
+  int64_t base = off[r];
+  for (int w = 0; w < (K + 31) / 32; ++w) {
+    const uint32_t m = mask[r * 16 + w];
+    if ((m >> lane) & 1u) {
+      const int64_t pos = base + __popc(m & ((1u << lane) - 1u));
+      if (pos < cap) live[pos] = ((uint32_t)r << 9) | (uint32_t)(w * 32 + lane);
+      else atomicOr(flag, FLAG_BAD_INDEX);
+    }
+    base += __popc(m);
+  }
+}
+
+// ------------------------------------------------------------------ scan
+
+// Exclusive scan of int32 counts (n <= 2048 * 1024) into off[0..n].
+__global__ void scan_block_kernel(const int32_t* __restrict__ in, int64_t n,
+                                  int32_t* __restrict__ out, int32_t* __restrict__ block_sums) {
+  __shared__ int32_t s[1024];
+  const int64_t i = (int64_t)blockIdx.x * 1024 + threadIdx.x;
+  int v = i < n ? in[i] : 0;
+  s[threadIdx.x] = v;
+  __syncthreads();
+  for (int offs = 1; offs < 1024; offs <<= 1) {
+    int a = threadIdx.x >= offs ? s[threadIdx.x - offs] : 0;
+    __syncthreads();
+    s[threadIdx.x] += a;
+    __syncthreads();
+  }
+  if (i < n) out[i] = s[threadIdx.x] - v;
+  if (threadIdx.x == 1023) block_sums[blockIdx.x] = s[1023];
+}
+
+__global__ void scan_sums_kernel(int32_t* __restrict__ sums, int nb, int32_t* __restrict__ total) {
+  __shared__ int32_t s[2048];
+  for (int i = threadIdx.x; i < 2048; i += blockDim.x) s[i] = i < nb ? sums[i] : 0;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int run = 0;
+    for (int i = 0; i < nb; ++i) { int v = s[i]; s[i] = run; run += v; }
+    *total = run;
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < nb; i += blockDim.x) sums[i] = s[i];
+}
+
+__global__ void scan_add_kernel(int32_t* __restrict__ out, int64_t n,
+                                const int32_t* __restrict__ block_sums) {
+  const int64_t i = (int64_t)blockIdx.x * 1024 + threadIdx.x;
+  if (i < n) out[i] += block_sums[blockIdx.x];
+}
+
+cudaError_t exclusive_scan(const int32_t* in, int64_t n, int32_t* out, int32_t* tmp,
+                           cudaStream_t st) {
+  const int64_t nb = (n + 1023) / 1024;
+  if (nb > 2048) return cudaErrorInvalidValue;
+  scan_block_kernel<<<(unsigned)nb, 1024, 0, st>>>(in, n, out, tmp);
+  scan_sums_kernel<<<1, 256, 0, st>>>(tmp, (int)nb, out + n);
+  scan_add_kernel<<<(unsigned)nb, 1024, 0, st>>>(out, n, tmp);
+  return cudaGetLastError();
+}
+
+// ------------------------------------------------------------------ hash grid
+
+__constant__ int c_hres[16];
+__constant__ int c_hoff[16];
+__constant__ int c_hdirect[16];
+
+HashGridInfo hash_grid_info() {
+  HashGridInfo h{};
+  const double b = std::exp((std::log(2048.0) - std::log(16.0)) / 15.0);
+  int64_t off = 0;
+  for (int l = 0; l < 16; ++l) {
+    const double v = 16.0 * std::pow(b, l);
+    // round half to even, as the resolution schedule specifies
+    double fl = std::floor(v);
+    int N = (int)fl;
+    const double frac = v - fl;
+    if (frac > 0.5 || (frac == 0.5 && (N & 1))) N += 1;
+    const int64_t cells = (int64_t)(N + 1) * (N + 1) * (N + 1);
+    h.res[l] = N;
+    h.direct[l] = cells <= (int64_t(1) << 19);
+    h.offset[l] = (int)off;
+    off += h.direct[l] ? cells : (int64_t(1) << 19);
+  }
+  h.entries = off;
+  return h;
+}
+
+cudaError_t upload_hash_grid(const HashGridInfo& h) {
+  cudaError_t e = cudaMemcpyToSymbol(c_hres, h.res, sizeof h.res);
+  if (e == cudaSuccess) e = cudaMemcpyToSymbol(c_hoff, h.offset, sizeof h.offset);
+  if (e == cudaSuccess) e = cudaMemcpyToSymbol(c_hdirect, h.direct, sizeof h.direct);
+  return e;
+}
+
+// Encoding of one point; optionally records the corner rows.
+__device__ __forceinline__ void hash_encode_point(const __half2* __restrict__ table, float x0,
+                                                  float x1, float x2, float* feat,
+                                                  int32_t* rows_out) {
+  const float u0 = fdiv(fadd(x0, 1.5f), 3.0f);
+  const float u1 = fdiv(fadd(x1, 1.5f), 3.0f);
+  const float u2 = fdiv(fadd(x2, 1.5f), 3.0f);
+#pragma unroll 4
+  for (int l = 0; l < 16; ++l) {
+    const int N = c_hres[l];
+    const float fN = (float)N;
+    const float c0 = fmul(u0, fN), c1 = fmul(u1, fN), c2 = fmul(u2, fN);
+    const float f0 = floorf(c0), f1 = floorf(c1), f2 = floorf(c2);
+    const float w0 = fsub(c0, f0), w1 = fsub(c1, f1), w2 = fsub(c2, f2);
+    const int i0 = (int)f0, i1 = (int)f1, i2 = (int)f2;
+    float a0 = 0.f, a1 = 0.f;
+#pragma unroll
+    for (int corner = 0; corner < 8; ++corner) {
+      const int dx = corner >> 2, dy = (corner >> 1) & 1, dz = corner & 1;
+      const int ix = min(max(i0 + dx, 0), N), iy = min(max(i1 + dy, 0), N),
+                iz = min(max(i2 + dz, 0), N);
+      uint32_t idx;
+      if (c_hdirect[l]) {
+        idx = (uint32_t)((ix * (N + 1) + iy) * (N + 1) + iz);
+      } else {
+        idx = ((uint32_t)ix ^ ((uint32_t)iy * 2654435761u) ^ ((uint32_t)iz * 805459861u)) &
+              ((1u << 19) - 1u);
+      }
+      const int row = c_hoff[l] + (int)idx;
+      if (rows_out) rows_out[l * 8 + corner] = row;
+      const float2 f = __half22float2(__ldg(table + row));
+      const float wx = dx ? w0 : 1.0f - w0;
+      const float wy = dy ? w1 : 1.0f - w1;
+      const float wz = dz ? w2 : 1.0f - w2;
+      const float wt = wx * wy * wz;
+      a0 = fmaf(wt, f.x, a0);
+      a1 = fmaf(wt, f.y, a1);
+    }
+    feat[2 * l] = a0;
+    feat[2 * l + 1] = a1;
+  }
+}
+
+__global__ void hash_encode_kernel(const float* __restrict__ x, int64_t n,
+                                   const __half2* __restrict__ table, float* __restrict__ feat,
+                                   int32_t* __restrict__ rows) {
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= n) return;
+  float f[32];
+  hash_encode_point(table, x[i * 3], x[i * 3 + 1], x[i * 3 + 2], f, rows ? rows + i * 128 : nullptr);
+#pragma unroll
+  for (int j = 0; j < 32; ++j) feat[i * 32 + j] = f[j];
+}
+
+// Real SH bands 0..3 of a unit vector, no Condon-Shortley phase; K holds
+// sqrt(2) K_l^m (m > 0) or K_l^0 folded with the Legendre leading factors.
+__device__ __forceinline__ void sh16(float x, float y, float z, const ShConst& K, float* o) {
+  o[0] = K.k[0];
+  o[1] = K.k[1] * y;
+  o[2] = K.k[2] * z;
+  o[3] = K.k[1] * x;
+  o[4] = K.k[4] * x * y;
+  o[5] = K.k[5] * y * z;
+  o[6] = K.k[6] * (3.0f * z * z - 1.0f);
+  o[7] = K.k[5] * x * z;
+  o[8] = K.k[8] * (x * x - y * y);
+  o[9] = K.k[9] * (3.0f * x * x * y - y * y * y);
+  o[10] = K.k[10] * x * y * z;
+  o[11] = K.k[11] * y * (5.0f * z * z - 1.0f);
+  o[12] = K.k[12] * z * (5.0f * z * z - 3.0f);
+  o[13] = K.k[11] * x * (5.0f * z * z - 1.0f);
+  o[14] = K.k[14] * z * (x * x - y * y);
+  o[15] = K.k[9] * (x * x * x - 3.0f * x * y * y);
+}
+
+ShConst sh_constants() {
+  auto fact = [](int n) { double f = 1; for (int i = 2; i <= n; ++i) f *= i; return f; };
+  auto norm = [&](int l, int m) {
+    return std::sqrt((2 * l + 1) / (4.0 * M_PI) * fact(l - m) / fact(l + m));
+  };
+  const double r2 = std::sqrt(2.0);
+  ShConst K{};
+  // P_l^m (no Condon-Shortley phase) times cos/sin(m phi), written in x, y, z:
+  // P_1^1 -> (x, y); P_2^1 = 3z sqrt(1-z^2); P_2^2 = 3(1-z^2); P_2^0 = (3z^2-1)/2;
+  // P_3^0 = z(5z^2-3)/2; P_3^1 = 3/2 (5z^2-1) sqrt(1-z^2); P_3^2 = 15 z (1-z^2);
+  // P_3^3 = 15 (1-z^2)^(3/2); sin(2 phi) terms carry the factor 2 of 2xy.
+  K.k[0] = (float)norm(0, 0);
+  K.k[1] = (float)(r2 * norm(1, 1));
+  K.k[2] = (float)norm(1, 0);
+  K.k[4] = (float)(r2 * norm(2, 2) * 3.0 * 2.0);
+  K.k[5] = (float)(r2 * norm(2, 1) * 3.0);
+  K.k[6] = (float)(norm(2, 0) * 0.5);
+  K.k[8] = (float)(r2 * norm(2, 2) * 3.0);
+  K.k[9] = (float)(r2 * norm(3, 3) * 15.0);
+  K.k[10] = (float)(r2 * norm(3, 2) * 15.0 * 2.0);
+  K.k[11] = (float)(r2 * norm(3, 1) * 1.5);
+  K.k[12] = (float)(norm(3, 0) * 0.5);
+  K.k[14] = (float)(r2 * norm(3, 2) * 15.0);
+  return K;
+}
+
+__global__ void sh_kernel(const float* __restrict__ d, int64_t n, ShConst K,
+                          float* __restrict__ out) {
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= n) return;
+  const float dx = d[i * 3], dy = d[i * 3 + 1], dz = d[i * 3 + 2];
+  const float inv = 1.0f / sqrtf(dx * dx + dy * dy + dz * dz);
+  float o[16];
+  sh16(dx * inv, dy * inv, dz * inv, K, o);
+#pragma unroll
+  for (int j = 0; j < 16; ++j) out[i * 16 + j] = o[j];
+}
+
+// Hash scene function for every live entry: encoding, density MLP, SH colour MLP.
+// Weights (fp32 blob of the ABI, 15,876 floats) are staged in shared memory.
+constexpr int HASH_NW = 15876;
+
+template <int K, int N>
+__device__ __forceinline__ void dense_relu(const float* __restrict__ W, const float* __restrict__ b,
+                                           const float* in, float* out, bool relu) {
+#pragma unroll
+  for (int n = 0; n < N; ++n) {
+    float acc = b[n];
+#pragma unroll
+    for (int k = 0; k < K; ++k) acc = fmaf(W[n * K + k], in[k], acc);
+    out[n] = relu ? fmaxf(acc, 0.0f) : acc;
+  }
+}
+
+__global__ void __launch_bounds__(128)
+hash_eval_kernel(const float* __restrict__ o, const float* __restrict__ d, int64_t r0,
+                 float near, float step, const uint32_t* __restrict__ live,
+                 const int32_t* __restrict__ total, const __half2* __restrict__ table,
+                 const float* __restrict__ mlp, ShConst K, float* __restrict__ out) {
+  extern __shared__ float w[];
+  for (int i = threadIdx.x; i < HASH_NW; i += blockDim.x) w[i] = mlp[i];
+  __syncthreads();
+  const float* d0 = w;            const float* d0b = d0 + 64 * 32;
+  const float* d1 = d0b + 64;     const float* d1b = d1 + 64 * 64;
+  const float* sw = d1b + 64;     const float* sb = sw + 64;
+  const float* c0 = sb + 1;       const float* c0b = c0 + 64 * 80;
+  const float* c1 = c0b + 64;     const float* c1b = c1 + 64 * 64;
+  const float* rw = c1b + 64;     const float* rb = rw + 3 * 64;
+  const int64_t P = *total;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < P;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const uint32_t e = live[i];
+    const int64_t r = r0 + (e >> 9);
+    const int k = (int)(e & 511u);
+    float x[3], t;
+    march_point(o, d, r, near, step, k, x, &t);
+    float in[80], h[64];
+    hash_encode_point(table, x[0], x[1], x[2], in, nullptr);
+    dense_relu<32, 64>(d0, d0b, in, h, true);
+    dense_relu<64, 64>(d1, d1b, h, in, true);          // in[0..63] = h2
+    float sigma = sb[0];
+#pragma unroll
+    for (int j = 0; j < 64; ++j) sigma = fmaf(sw[j], in[j], sigma);
+    sigma = fmaxf(sigma, 0.0f);
+    const float dx = d[r * 3], dy = d[r * 3 + 1], dz = d[r * 3 + 2];
+    const float inv = 1.0f / sqrtf(dx * dx + dy * dy + dz * dz);
+    sh16(dx * inv, dy * inv, dz * inv, K, in + 64);
+    dense_relu<80, 64>(c0, c0b, in, h, true);
+    dense_relu<64, 64>(c1, c1b, h, in, true);
+    float rgb[3];
+    dense_relu<64, 3>(rw, rb, in, rgb, false);
+    float4 v = make_float4(1.0f / (1.0f + expf(-rgb[0])), 1.0f / (1.0f + expf(-rgb[1])),
+                           1.0f / (1.0f + expf(-rgb[2])), sigma);
+    reinterpret_cast<float4*>(out)[i] = v;
+  }
+}
+
+// ------------------------------------------------------------------ KiloNeRF
+
+__global__ void cell_hist_kernel(const float* __restrict__ o, const float* __restrict__ d,
+                                 int64_t r0, float near, float step,
+                                 const uint32_t* __restrict__ live, const int32_t* __restrict__ total,
+                                 int32_t* __restrict__ cell, int32_t* __restrict__ hist) {
+  const int64_t P = *total;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < P;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const uint32_t e = live[i];
+    float x[3], t;
+    march_point(o, d, r0 + (e >> 9), near, step, (int)(e & 511u), x, &t);
+    const int a = voxel_axis(x[0]), b = voxel_axis(x[1]), c = voxel_axis(x[2]);
+    const int id = ((a >> 3) * 16 + (b >> 3)) * 16 + (c >> 3);
+    cell[i] = id;
+    atomicAdd(&hist[id], 1);
+  }
+}
+
+__global__ void cell_hist_points_kernel(const float* __restrict__ x, int64_t n,
+                                        int32_t* __restrict__ cell, int32_t* __restrict__ hist,
+                                        unsigned* flag) {
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= n) return;
+  const int a = voxel_axis(x[i * 3]), b = voxel_axis(x[i * 3 + 1]), c = voxel_axis(x[i * 3 + 2]);
+  if (a < 0 || b < 0 || c < 0) { cell[i] = -1; atomicOr(flag, FLAG_BAD_INDEX); return; }
+  const int id = ((a >> 3) * 16 + (b >> 3)) * 16 + (c >> 3);
+  cell[i] = id;
+  atomicAdd(&hist[id], 1);
+}
+
+__global__ void cell_scatter_kernel(const int32_t* __restrict__ cell, const int32_t* __restrict__ total,
+                                    int64_t n_fixed, const int32_t* __restrict__ cell_off,
+                                    int32_t* __restrict__ fill, int32_t* __restrict__ order) {
+  const int64_t P = total ? (int64_t)*total : n_fixed;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < P;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const int c = cell[i];
+    if (c < 0) continue;
+    const int pos = cell_off[c] + atomicAdd(&fill[c], 1);
+    order[pos] = (int32_t)i;
+  }
+}
+
+constexpr int KILO_NP = 3317;
+
+// Per-cell tiny MLP over the cell-grouped order: consecutive threads mostly
+// share a cell, so their weight loads coalesce into broadcasts.
+__global__ void __launch_bounds__(128)
+kilo_eval_kernel(const float* __restrict__ o, const float* __restrict__ d, int64_t r0, float near,
+                 float step, const uint32_t* __restrict__ live, const int32_t* __restrict__ total,
+                 const int32_t* __restrict__ order, const int32_t* __restrict__ cell,
+                 const float* __restrict__ cell_w, float* __restrict__ out) {
+  const int64_t P = *total;
+  for (int64_t j = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; j < P;
+       j += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t i = order[j];
+    const uint32_t e = live[i];
+    const int64_t r = r0 + (e >> 9);
+    float x[3], t;
+    march_point(o, d, r, near, step, (int)(e & 511u), x, &t);
+    const float* W = cell_w + (int64_t)cell[i] * KILO_NP;
+    const float* W1 = W;           const float* b1 = W1 + 32 * 63;
+    const float* W2 = b1 + 32;     const float* b2 = W2 + 32 * 32;
+    const float* ws = b2 + 32;     const float* bs = ws + 32;
+    const float* Wc = bs + 1;      const float* bc = Wc + 3 * 59;
+    float pe[63];
+    pe[0] = x[0]; pe[1] = x[1]; pe[2] = x[2];
+#pragma unroll
+    for (int c = 0; c < 3; ++c)
+#pragma unroll
+      for (int k = 0; k < 10; ++k) pe_sincos(x[c], k, &pe[3 + c * 10 + k], &pe[33 + c * 10 + k]);
+    float h1[32], h2[59];
+#pragma unroll 4
+    for (int n = 0; n < 32; ++n) {
+      float acc = __ldg(b1 + n);
+#pragma unroll
+      for (int k = 0; k < 63; ++k) acc = fmaf(__ldg(W1 + n * 63 + k), pe[k], acc);
+      h1[n] = fmaxf(acc, 0.0f);
+    }
+#pragma unroll 4
+    for (int n = 0; n < 32; ++n) {
+      float acc = __ldg(b2 + n);
+#pragma unroll
+      for (int k = 0; k < 32; ++k) acc = fmaf(__ldg(W2 + n * 32 + k), h1[k], acc);
+      h2[n] = fmaxf(acc, 0.0f);
+    }
+    float sigma = __ldg(bs);
+#pragma unroll
+    for (int k = 0; k < 32; ++k) sigma = fmaf(__ldg(ws + k), h2[k], sigma);
+    sigma = fmaxf(sigma, 0.0f);
+    const float dx = d[r * 3], dy = d[r * 3 + 1], dz = d[r * 3 + 2];
+    const float inv = 1.0f / sqrtf(dx * dx + dy * dy + dz * dz);
+    const float u[3] = {dx * inv, dy * inv, dz * inv};
+    h2[32] = u[0]; h2[33] = u[1]; h2[34] = u[2];
+#pragma unroll
+    for (int c = 0; c < 3; ++c)
+#pragma unroll
+      for (int k = 0; k < 4; ++k) pe_sincos(u[c], k, &h2[35 + c * 4 + k], &h2[47 + c * 4 + k]);
+    float rgb[3];
+#pragma unroll
+    for (int n = 0; n < 3; ++n) {
+      float acc = __ldg(bc + n);
+#pragma unroll
+      for (int k = 0; k < 59; ++k) acc = fmaf(__ldg(Wc + n * 59 + k), h2[k], acc);
+      rgb[n] = 1.0f / (1.0f + expf(-acc));
+    }
+    reinterpret_cast<float4*>(out)[i] = make_float4(rgb[0], rgb[1], rgb[2], sigma);
+  }
+}
+
+// ------------------------------------------------------------------ compositing
+
+// Warp per ray over its live entries (already activated sigma, rgb); every
+// live sample has delta = step * |d|. Early termination: stop before the first
+// live sample whose transmittance (fp32) is below ert_T.
+__global__ void march_composite_kernel(const float* __restrict__ d, int64_t r0, int64_t R,
+                                       float near, float step, float ert_T,
+                                       const int32_t* __restrict__ off,
+                                       const uint32_t* __restrict__ live,
+                                       const float* __restrict__ val, float* __restrict__ rgb,
+                                       float* __restrict__ depth, float* __restrict__ acc_out) {
+  const int lane = threadIdx.x & 31;
+  const int64_t rl = (int64_t)blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;
+  if (rl >= R) return;
+  const int64_t r = r0 + rl;
+  const float dx = d[r * 3], dy = d[r * 3 + 1], dz = d[r * 3 + 2];
+  const float delta = step * sqrtf(dx * dx + dy * dy + dz * dz);
+  const int64_t b = off[rl], e = off[rl + 1];
+  float S = 0.0f, cr = 0.f, cg = 0.f, cb = 0.f, dep = 0.f, acc = 0.f;
+  bool done = false;
+  for (int64_t s0 = b; s0 < e && !done; s0 += 32) {
+    const int64_t i = s0 + lane;
+    const bool in = i < e;
+    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+    float t = 0.0f;
+    if (in) {
+      v = reinterpret_cast<const float4*>(val)[i];
+      t = fadd(near, fmul((float)(live[i] & 511u), step));
+    }
+    const float tau = in ? v.w * delta : 0.0f;
+    float incl = tau;
+#pragma unroll
+    for (int o2 = 1; o2 < 32; o2 <<= 1) {
+      float q = __shfl_up_sync(0xffffffffu, incl, o2);
+      if (lane >= o2) incl += q;
+    }
+    float excl = __shfl_up_sync(0xffffffffu, incl, 1);
+    if (lane == 0) excl = 0.0f;
+    const float T = expf(-(S + excl));
+    bool keep = in;
+    if (ert_T > 0.0f) {
+      const uint32_t stop = __ballot_sync(0xffffffffu, in && T < ert_T);
+      if (stop) {
+        const int first = __ffs(stop) - 1;
+        keep = in && lane < first;
+        done = true;
+      }
+    }
+    if (keep) {
+      const float w = T * (-expm1f(-tau));
+      cr += w * v.x; cg += w * v.y; cb += w * v.z;
+      dep += w * t;
+      acc += w;
+    }
+    S += __shfl_sync(0xffffffffu, incl, 31);
+  }
+#pragma unroll
+  for (int o2 = 16; o2 > 0; o2 >>= 1) {
+    cr += __shfl_xor_sync(0xffffffffu, cr, o2);
+    cg += __shfl_xor_sync(0xffffffffu, cg, o2);
+    cb += __shfl_xor_sync(0xffffffffu, cb, o2);
+    dep += __shfl_xor_sync(0xffffffffu, dep, o2);
+    acc += __shfl_xor_sync(0xffffffffu, acc, o2);
+  }
+  if (lane == 0) {
+    rgb[r * 3] = cr; rgb[r * 3 + 1] = cg; rgb[r * 3 + 2] = cb;
+    depth[r] = dep;
+    acc_out[r] = acc;
+  }
+}
+
+// ------------------------------------------------------------------ launchers
+
+static unsigned grid_for(int64_t work, int block, int max_blocks) {
+  int64_t b = (work + block - 1) / block;
+  if (b < 1) b = 1;
+  return (unsigned)(b < max_blocks ? b : max_blocks);
+}
+
+cudaError_t launch_march_mask(const float* o, const float* d, int64_t R, float near, float step,
+                              int K, const uint32_t* occ, uint32_t* mask, int32_t* count,
+                              uint8_t* live_u8, cudaStream_t st) {
+  if (K < 1 || K > 512) return cudaErrorInvalidValue;
+  march_mask_kernel<<<(unsigned)((R + 7) / 8), 256, 0, st>>>(o, d, R, near, step, K, occ, mask,
+                                                              count, live_u8);
+  return cudaGetLastError();
+}
+
+cudaError_t march_render_chunk(const MarchArgs& a, cudaStream_t st) {
+  const int64_t R = a.R;
+  cudaError_t e = launch_march_mask(a.o + a.r0 * 3, a.d + a.r0 * 3, R, a.near, a.step, a.K, a.occ,
+                                    a.ws.mask, a.ws.count, nullptr, st);
+  if (e != cudaSuccess) return e;
+  e = exclusive_scan(a.ws.count, R, a.ws.off, a.ws.scan_tmp, st);
+  if (e != cudaSuccess) return e;
+  march_emit_kernel<<<(unsigned)((R + 7) / 8), 256, 0, st>>>(a.ws.mask, a.ws.off, R, a.K,
+                                                             a.ws.live, a.ws.cap, a.flag);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  const int32_t* total = a.ws.off + R;
+  const unsigned g = (unsigned)(a.num_sms * 8);
+  if (a.model == NERF_MODEL_HASHGRID) {
+    hash_eval_kernel<<<g, 128, HASH_NW * sizeof(float), st>>>(
+        a.o, a.d, a.r0, a.near, a.step, a.ws.live, total,
+        reinterpret_cast<const __half2*>(a.hash_table), a.hash_mlp, a.sh, a.ws.val);
+  } else {
+    cudaMemsetAsync(a.ws.cell_hist, 0, 2 * 4096 * sizeof(int32_t), st);
+    cell_hist_kernel<<<g, 256, 0, st>>>(a.o, a.d, a.r0, a.near, a.step, a.ws.live, total,
+                                        a.ws.cell, a.ws.cell_hist);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    e = exclusive_scan(a.ws.cell_hist, 4096, a.ws.cell_off, a.ws.scan_tmp, st);
+    if (e != cudaSuccess) return e;
+    cell_scatter_kernel<<<g, 256, 0, st>>>(a.ws.cell, total, 0, a.ws.cell_off, a.ws.cell_fill,
+                                           a.ws.order);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    kilo_eval_kernel<<<g, 128, 0, st>>>(a.o, a.d, a.r0, a.near, a.step, a.ws.live, total,
+                                        a.ws.order, a.ws.cell, a.cell_w, a.ws.val);
+  }
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  march_composite_kernel<<<(unsigned)((R + 7) / 8), 256, 0, st>>>(
+      a.d, a.r0, R, a.near, a.step, a.ert_T, a.ws.off, a.ws.live, a.ws.val, a.rgb, a.depth, a.acc);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_route_points(const float* x, int64_t n, int32_t* cell, int32_t* hist,
+                                int32_t* off, int32_t* order, int32_t* fill, int32_t* scan_tmp,
+                                unsigned* flag, cudaStream_t st) {
+  cudaMemsetAsync(hist, 0, 4096 * sizeof(int32_t), st);
+  cell_hist_points_kernel<<<grid_for(n, 256, 1 << 20), 256, 0, st>>>(x, n, cell, hist, flag);
+  cudaError_t e = exclusive_scan(hist, 4096, off, scan_tmp, st);
+  if (e != cudaSuccess || !order) return e == cudaSuccess ? cudaGetLastError() : e;
+  cudaMemsetAsync(fill, 0, 4096 * sizeof(int32_t), st);
+  cell_scatter_kernel<<<grid_for(n, 256, 4096), 256, 0, st>>>(cell, nullptr, n, off, fill, order);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_hash_encode(const float* x, int64_t n, const uint16_t* table, float* feat,
+                               int32_t* rows, cudaStream_t st) {
+  hash_encode_kernel<<<(unsigned)((n + 127) / 128), 128, 0, st>>>(
+      x, n, reinterpret_cast<const __half2*>(table), feat, rows);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_sh(const float* d, int64_t n, float* out, cudaStream_t st) {
+  sh_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(d, n, sh_constants(), out);
+  return cudaGetLastError();
+}
+
+cudaError_t march_prepare(cudaStream_t st) {
+  (void)st;
+  cudaError_t e = upload_hash_grid(hash_grid_info());
+  if (e != cudaSuccess) return e;
+  return cudaFuncSetAttribute(hash_eval_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              HASH_NW * (int)sizeof(float));
+}
+
+}  // namespace nerfb

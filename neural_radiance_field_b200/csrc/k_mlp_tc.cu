@@ -33,7 +33,8 @@ constexpr int NSTAGE = 4;
 constexpr int RING_BYTES = 256 * CHUNK_K * 2;       // 16384 per slot
 constexpr int NLAYER = 10;                          // pts0..pts7, feature, dir
 constexpr int NTHREADS = 320;
-constexpr size_t SMEM_BYTES = 2 * ACT_BYTES + NSTAGE * RING_BYTES + 1024;
+constexpr int VEC_BYTES = 2 * 256 * 4;                // staged epilogue vectors
+constexpr size_t SMEM_BYTES = 2 * ACT_BYTES + NSTAGE * RING_BYTES + VEC_BYTES + 256;
 
 // per layer: K chunks, output width, first K-group of the A operand
 __constant__ int c_kchunks[NLAYER] = {2, 8, 8, 8, 8, 10, 8, 8, 8, 8};
@@ -231,11 +232,116 @@ struct Params {
   int64_t n_pairs;
 };
 
+// Issue a 32-column TMEM load; the registers are valid after tmem_wait32.
+__device__ __forceinline__ void tmem_ld32_issue(uint32_t taddr, uint32_t* r) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+}
+
+// Wait for outstanding TMEM loads; the registers are threaded through the asm
+// so that no use of them can be scheduled before the wait.
+__device__ __forceinline__ void tmem_wait32(uint32_t* r) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;"
+               : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]),
+                 "+r"(r[6]), "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]),
+                 "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15]), "+r"(r[16]), "+r"(r[17]),
+                 "+r"(r[18]), "+r"(r[19]), "+r"(r[20]), "+r"(r[21]), "+r"(r[22]), "+r"(r[23]),
+                 "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]), "+r"(r[29]),
+                 "+r"(r[30]), "+r"(r[31])
+               :
+               : "memory");
+}
+
+// Barrier among the 256 epilogue threads only (named barrier 1).
+__device__ __forceinline__ void epilogue_sync() {
+  asm volatile("bar.sync 1, 256;" ::: "memory");
+}
+
+// Same barrier, returning whether any of the 256 threads passed true.
+__device__ __forceinline__ bool epilogue_sync_or(bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.or.pred q, 1, 256, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)v)
+      : "memory");
+  return r != 0;
+}
+
+// One 32-column block of a hidden layer: bias, activation, bf16, store to the
+// next layer's A operand; on the last trunk layer also accumulates sigma.
+template <bool RELU, bool SIGMA>
+__device__ __forceinline__ void epi_block(const uint32_t* u, const float* sb_bias,
+                                          const float* sb_ws, int cb, uint32_t act_base, int r,
+                                          float& sigma) {
+  float v[32];
+#pragma unroll
+  for (int i = 0; i < 32; i += 4) {
+    const float4 b4 = *reinterpret_cast<const float4*>(sb_bias + cb + i);
+    v[i] = __uint_as_float(u[i]) + b4.x;
+    v[i + 1] = __uint_as_float(u[i + 1]) + b4.y;
+    v[i + 2] = __uint_as_float(u[i + 2]) + b4.z;
+    v[i + 3] = __uint_as_float(u[i + 3]) + b4.w;
+  }
+  if (SIGMA) {
+#pragma unroll
+    for (int i = 0; i < 32; i += 4) {
+      const float4 w4 = *reinterpret_cast<const float4*>(sb_ws + cb + i);
+      sigma = fmaf(fmaxf(v[i], 0.f), w4.x, sigma);
+      sigma = fmaf(fmaxf(v[i + 1], 0.f), w4.y, sigma);
+      sigma = fmaf(fmaxf(v[i + 2], 0.f), w4.z, sigma);
+      sigma = fmaf(fmaxf(v[i + 3], 0.f), w4.w, sigma);
+    }
+  }
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const float* p = v + 8 * j;
+    uint32_t w0, w1, w2, w3;
+    if (RELU) {
+      w0 = pack_relu(p[0], p[1]); w1 = pack_relu(p[2], p[3]);
+      w2 = pack_relu(p[4], p[5]); w3 = pack_relu(p[6], p[7]);
+    } else {
+      w0 = pack_plain(p[0], p[1]); w1 = pack_plain(p[2], p[3]);
+      w2 = pack_plain(p[4], p[5]); w3 = pack_plain(p[6], p[7]);
+    }
+    st_shared_v4(act_base + act_off(r, cb + 8 * j), w0, w1, w2, w3);
+  }
+}
+
+template <bool RELU, bool SIGMA>
+__device__ __forceinline__ void epi_layer(uint32_t t_row, const float* sb_bias, const float* sb_ws,
+                                          uint32_t act_base, int r, float& sigma) {
+  uint32_t ua[32], ub[32];
+  tmem_ld32_issue(t_row, ua);
+  tmem_wait32(ua);
+#pragma unroll
+  for (int cb = 0; cb < 256; cb += 64) {
+    tmem_ld32_issue(t_row + cb + 32, ub);
+    epi_block<RELU, SIGMA>(ua, sb_bias, sb_ws, cb, act_base, r, sigma);
+    tmem_wait32(ub);
+    if (cb + 64 < 256) tmem_ld32_issue(t_row + cb + 64, ua);
+    epi_block<RELU, SIGMA>(ub, sb_bias, sb_ws, cb + 32, act_base, r, sigma);
+    if (cb + 64 < 256) tmem_wait32(ua);
+  }
+}
+
 __global__ void __launch_bounds__(NTHREADS, 1) mlp_tc_kernel(Params P) {
   extern __shared__ __align__(1024) uint8_t smem[];
   uint8_t* act = smem;                                   // 2 x ACT_BYTES
   uint8_t* ring = smem + 2 * ACT_BYTES;                  // NSTAGE x RING_BYTES
-  uint64_t* bars = reinterpret_cast<uint64_t*>(ring + NSTAGE * RING_BYTES);
+  float* svec = reinterpret_cast<float*>(ring + NSTAGE * RING_BYTES);   // 2 x 256 fp32
+  uint64_t* bars = reinterpret_cast<uint64_t*>(ring + NSTAGE * RING_BYTES + VEC_BYTES);
   uint64_t* full = bars;                 // [NSTAGE]
   uint64_t* empty = bars + NSTAGE;       // [NSTAGE]
   uint64_t* mma_done = bars + 2 * NSTAGE;     // [2]
@@ -327,12 +433,14 @@ __global__ void __launch_bounds__(NTHREADS, 1) mlp_tc_kernel(Params P) {
     }
   } else {
     // ---------------------------------------------------------- epilogue
-    const int g = (warp - 2) >> 2;                 // tile within the pair
-    const int quarter = warp & 3;                  // TMEM lane quarter of this warp
-    const int r = quarter * 32 + lane;             // row in the tile = TMEM lane
-    uint8_t* my_act = act + g * ACT_BYTES;
-    const uint32_t act_base = smem_u32(my_act);
+    const int et = threadIdx.x - 64;              // 0..255 over both tiles
+    const int g = (warp - 2) >> 2;                // tile within the pair
+    const int quarter = warp & 3;                 // TMEM lane quarter of this warp
+    const int r = quarter * 32 + lane;            // row in the tile = TMEM lane
+    const uint32_t act_base = smem_u32(act + g * ACT_BYTES);
     const uint32_t t_row = tmem + (uint32_t)(g * 256) + ((uint32_t)(quarter * 32) << 16);
+    float* sb0 = svec;          // layer bias / rgb weights rows 0, 1
+    float* sb1 = svec + 256;    // sigma weights / rgb row 2, rgb and sigma biases
     uint32_t ph_md = 0;
     const float* vec = P.vec;
     for (int64_t pr = blockIdx.x; pr < P.n_pairs; pr += gridDim.x) {
@@ -377,65 +485,55 @@ __global__ void __launch_bounds__(NTHREADS, 1) mlp_tc_kernel(Params P) {
 
       float sigma = 0.0f;
       for (int l = 0; l < NLAYER; ++l) {
-        if (!mbar_wait(&mma_done[g], ph_md, ctl)) break;
+        // this layer's epilogue vectors: loaded now, staged after the MMA wait
+        float pre0, pre1 = 0.0f;
+        if (l < 9) {
+          pre0 = __ldg(vec + P.lay.bias[l] + et);
+          if (l == 7) pre1 = __ldg(vec + P.lay.w_sigma + et);
+        } else {
+          pre0 = __ldg(vec + P.lay.w_rgb + et);
+          if (et < 128) pre1 = __ldg(vec + P.lay.w_rgb + 256 + et);
+          else if (et < 131) pre1 = __ldg(vec + P.lay.b_rgb + et - 128);
+          else if (et == 131) pre1 = __ldg(vec + P.lay.b_sigma);
+        }
+        const bool waited = mbar_wait(&mma_done[g], ph_md, ctl);
         ph_md ^= 1;
         tc_fence_after();
-        const float* bias = vec + P.lay.bias[l];
+        // both tiles are done with the previous vectors; all 256 threads agree
+        // on giving up together, so no thread is left behind at a barrier
+        if (epilogue_sync_or(!waited || *abort_flag)) break;
+        sb0[et] = pre0;
+        sb1[et] = pre1;
+        epilogue_sync();
         if (l < 9) {
-          const bool relu = (l != 8);
-#pragma unroll 1
-          for (int cb = 0; cb < 256; cb += 32) {
-            float v[32];
-            tmem_ld32(t_row + cb, v);
-#pragma unroll
-            for (int i = 0; i < 32; i += 4) {
-              const float4 b4 = __ldg(reinterpret_cast<const float4*>(bias + cb + i));
-              v[i] += b4.x; v[i + 1] += b4.y; v[i + 2] += b4.z; v[i + 3] += b4.w;
-            }
-            if (l == 7) {
-#pragma unroll
-              for (int i = 0; i < 32; i += 4) {
-                const float4 w4 = __ldg(reinterpret_cast<const float4*>(vec + P.lay.w_sigma + cb + i));
-                sigma = fmaf(fmaxf(v[i], 0.f), w4.x, sigma);
-                sigma = fmaf(fmaxf(v[i + 1], 0.f), w4.y, sigma);
-                sigma = fmaf(fmaxf(v[i + 2], 0.f), w4.z, sigma);
-                sigma = fmaf(fmaxf(v[i + 3], 0.f), w4.w, sigma);
-              }
-            }
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              const float* p = v + 8 * j;
-              uint32_t w0, w1, w2, w3;
-              if (relu) {
-                w0 = pack_relu(p[0], p[1]); w1 = pack_relu(p[2], p[3]);
-                w2 = pack_relu(p[4], p[5]); w3 = pack_relu(p[6], p[7]);
-              } else {
-                w0 = pack_plain(p[0], p[1]); w1 = pack_plain(p[2], p[3]);
-                w2 = pack_plain(p[4], p[5]); w3 = pack_plain(p[6], p[7]);
-              }
-              st_shared_v4(act_base + act_off(r, cb + 8 * j), w0, w1, w2, w3);
-            }
-          }
+          if (l == 8) epi_layer<false, false>(t_row, sb0, sb1, act_base, r, sigma);
+          else if (l == 7) epi_layer<true, true>(t_row, sb0, sb1, act_base, r, sigma);
+          else epi_layer<true, false>(t_row, sb0, sb1, act_base, r, sigma);
           tc_fence_before();
           fence_async_smem();
           mbar_arrive(&act_ready[g]);
         } else {
           // direction layer: + per-ray bias, ReLU, then the rgb head in fp32
           const float* rb = P.dir_bias + ray * 128;
-          float rgb0 = vec[P.lay.b_rgb], rgb1 = vec[P.lay.b_rgb + 1], rgb2 = vec[P.lay.b_rgb + 2];
-          const float* wr = vec + P.lay.w_rgb;
+          float rgb0 = sb1[128], rgb1 = sb1[129], rgb2 = sb1[130];
+          uint32_t u[32];
 #pragma unroll 1
           for (int cb = 0; cb < 128; cb += 32) {
-            float v[32];
-            tmem_ld32(t_row + cb, v);
+            tmem_ld32_issue(t_row + cb, u);
+            float4 bb[8];
 #pragma unroll
-            for (int i = 0; i < 32; i += 4) {
-              const float4 b4 = __ldg(reinterpret_cast<const float4*>(rb + cb + i));
-              const float h0 = fmaxf(v[i] + b4.x, 0.f), h1 = fmaxf(v[i + 1] + b4.y, 0.f);
-              const float h2 = fmaxf(v[i + 2] + b4.z, 0.f), h3 = fmaxf(v[i + 3] + b4.w, 0.f);
-              const float4 a4 = __ldg(reinterpret_cast<const float4*>(wr + cb + i));
-              const float4 c4 = __ldg(reinterpret_cast<const float4*>(wr + 128 + cb + i));
-              const float4 d4 = __ldg(reinterpret_cast<const float4*>(wr + 256 + cb + i));
+            for (int i = 0; i < 8; ++i) bb[i] = __ldg(reinterpret_cast<const float4*>(rb + cb) + i);
+            tmem_wait32(u);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              const int c = cb + 4 * i;
+              const float h0 = fmaxf(__uint_as_float(u[4 * i]) + bb[i].x, 0.f);
+              const float h1 = fmaxf(__uint_as_float(u[4 * i + 1]) + bb[i].y, 0.f);
+              const float h2 = fmaxf(__uint_as_float(u[4 * i + 2]) + bb[i].z, 0.f);
+              const float h3 = fmaxf(__uint_as_float(u[4 * i + 3]) + bb[i].w, 0.f);
+              const float4 a4 = *reinterpret_cast<const float4*>(sb0 + c);
+              const float4 c4 = *reinterpret_cast<const float4*>(sb0 + 128 + c);
+              const float4 d4 = *reinterpret_cast<const float4*>(sb1 + c);
               rgb0 = fmaf(h0, a4.x, fmaf(h1, a4.y, fmaf(h2, a4.z, fmaf(h3, a4.w, rgb0))));
               rgb1 = fmaf(h0, c4.x, fmaf(h1, c4.y, fmaf(h2, c4.z, fmaf(h3, c4.w, rgb1))));
               rgb2 = fmaf(h0, d4.x, fmaf(h1, d4.y, fmaf(h2, d4.z, fmaf(h3, d4.w, rgb2))));
@@ -444,10 +542,10 @@ __global__ void __launch_bounds__(NTHREADS, 1) mlp_tc_kernel(Params P) {
           tc_fence_before();
           if (valid)
             *reinterpret_cast<float4*>(P.raw + row * 4) =
-                make_float4(rgb0, rgb1, rgb2, sigma + vec[P.lay.b_sigma]);
+                make_float4(rgb0, rgb1, rgb2, sigma + sb1[131]);
         }
       }
-      if (*abort_flag) break;
+      if (epilogue_sync_or(*abort_flag)) break;
     }
   }
 

@@ -71,6 +71,56 @@ void dir_offsets(const nerf_config& c, int64_t* w_off, int64_t* b_off) {
 
 bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
 
+void free_march(nerf_ctx* ctx) {
+  MarchWs& w = ctx->mws;
+  cudaFree(w.mask); cudaFree(w.count); cudaFree(w.off); cudaFree(w.scan_tmp);
+  cudaFree(w.live); cudaFree(w.val); cudaFree(w.cell); cudaFree(w.order);
+  cudaFree(w.cell_hist); cudaFree(w.cell_off);
+  w = MarchWs{};
+}
+
+// Contexts of the march models: rays are processed in chunks of up to 2^19, each
+// with room for every candidate of every ray, so no input can overflow it.
+nerf_status create_march(const nerf_config& c, nerf_ctx** out) {
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return fail(nullptr, NERF_ERR_CUDA, "no CUDA device: %s", cudaGetErrorString(e));
+  nerf_ctx* ctx = new nerf_ctx();
+  ctx->cfg = c;
+  ctx->device = dev;
+  cudaDeviceGetAttribute(&ctx->num_sms, cudaDevAttrMultiProcessorCount, dev);
+  const int64_t chunk = c.max_rays < (int64_t(1) << 19) ? c.max_rays : (int64_t(1) << 19);
+  ctx->chunk_rays = chunk;
+  MarchWs& w = ctx->mws;
+  w.cap = chunk * c.max_samples;
+  bool ok = true;
+  ok &= dalloc(&w.mask, (size_t)(chunk * 16)) == cudaSuccess;
+  ok &= dalloc(&w.count, (size_t)chunk) == cudaSuccess;
+  ok &= dalloc(&w.off, (size_t)(chunk + 1)) == cudaSuccess;
+  ok &= dalloc(&w.scan_tmp, 2048) == cudaSuccess;
+  ok &= dalloc(&w.live, (size_t)w.cap) == cudaSuccess;
+  ok &= dalloc(&w.val, (size_t)(w.cap * 4)) == cudaSuccess;
+  if (c.model == NERF_MODEL_KILONERF) {
+    ok &= dalloc(&w.cell, (size_t)w.cap) == cudaSuccess;
+    ok &= dalloc(&w.order, (size_t)w.cap) == cudaSuccess;
+    ok &= dalloc(&w.cell_hist, 2 * 4096) == cudaSuccess;
+    ok &= dalloc(&w.cell_off, 4097) == cudaSuccess;
+    if (ok) w.cell_fill = w.cell_hist + 4096;
+  }
+  ok &= dalloc(&ctx->stage, (size_t)(c.max_rays * 11)) == cudaSuccess;
+  ok &= dalloc(&ctx->d_flag, 1) == cudaSuccess;
+  if (ok) ok &= cudaMemset(ctx->d_flag, 0, sizeof(unsigned)) == cudaSuccess;
+  if (ok) ok &= march_prepare(nullptr) == cudaSuccess;
+  if (!ok) {
+    cudaGetLastError();
+    nerf_destroy(ctx);
+    return fail(nullptr, NERF_ERR_OOM, "march workspace allocation failed for max_rays=%lld, max_samples=%d",
+                (long long)c.max_rays, c.max_samples);
+  }
+  *out = ctx;
+  return NERF_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -103,7 +153,7 @@ nerf_status nerf_create(const nerf_config* cfg, nerf_ctx** out) {
     if (c.precision == NERF_BF16 && !big)
       return fail(nullptr, NERF_ERR_UNSUPPORTED, "BF16 tensor-core path needs W=256, D=8");
   } else if (c.model == NERF_MODEL_KILONERF || c.model == NERF_MODEL_HASHGRID) {
-    return fail(nullptr, NERF_ERR_UNSUPPORTED, "march models are not built into this library yet");
+    return create_march(c, out);
   } else {
     return fail(nullptr, NERF_ERR_INVALID_ARG, "unknown model %d", c.model);
   }
@@ -146,6 +196,7 @@ nerf_status nerf_destroy(nerf_ctx* ctx) {
   cudaFree(ctx->t_all);
   cudaFree(ctx->stage);
   cudaFree(ctx->d_flag);
+  free_march(ctx);
   if (ctx->ev) {
     for (int i = 0; i < 2 * kMaxTimed; ++i) cudaEventDestroy(ctx->ev[i]);
     delete[] ctx->ev;
@@ -247,6 +298,47 @@ nerf_status check_render_args(nerf_ctx* ctx, const float* o, const float* d, int
     }
     if (c.precision == NERF_BF16 && (!aligned16(p->coarse_w) || (n_fine > 0 && !aligned16(p->fine_w))))
       return fail(ctx, NERF_ERR_INVALID_ARG, "bf16 weight blobs must be 16-byte aligned");
+  } else {
+    if (n_fine != 0) return fail(ctx, NERF_ERR_INVALID_ARG, "march models take n_fine = 0");
+    if (n_coarse > 512) return fail(ctx, NERF_ERR_INVALID_ARG, "march candidates must be <= 512");
+    if (!p->occupancy) return fail(ctx, NERF_ERR_INVALID_ARG, "occupancy grid is NULL");
+    if (!(p->march_step > 0.0f)) return fail(ctx, NERF_ERR_INVALID_ARG, "march_step must be > 0");
+    if (!(p->ert_T >= 0.0f && p->ert_T < 1.0f))
+      return fail(ctx, NERF_ERR_INVALID_ARG, "ert_T must be in [0, 1)");
+    if (c.model == NERF_MODEL_KILONERF && !p->cell_w)
+      return fail(ctx, NERF_ERR_INVALID_ARG, "cell_w is NULL");
+    if (c.model == NERF_MODEL_HASHGRID && (!p->hash_table || !p->hash_mlp || !aligned16(p->hash_mlp)))
+      return fail(ctx, NERF_ERR_INVALID_ARG, "hash_table / hash_mlp NULL or misaligned");
+  }
+  return NERF_OK;
+}
+
+nerf_status render_march(nerf_ctx* ctx, const float* o, const float* d, int64_t R, float near,
+                         int K, const nerf_params* p, float* rgb, float* depth, float* acc,
+                         cudaStream_t st) {
+  MarchArgs a{};
+  a.model = ctx->cfg.model;
+  a.o = o;
+  a.d = d;
+  a.near = near;
+  a.step = p->march_step;
+  a.ert_T = p->ert_T;
+  a.K = K;
+  a.occ = p->occupancy;
+  a.cell_w = p->cell_w;
+  a.hash_table = p->hash_table;
+  a.hash_mlp = p->hash_mlp;
+  a.sh = sh_constants();
+  a.rgb = rgb;
+  a.depth = depth;
+  a.acc = acc;
+  a.flag = ctx->d_flag;
+  a.num_sms = ctx->num_sms;
+  a.ws = ctx->mws;
+  for (int64_t r0 = 0; r0 < R; r0 += ctx->chunk_rays) {
+    a.r0 = r0;
+    a.R = R - r0 < ctx->chunk_rays ? R - r0 : ctx->chunk_rays;
+    NERF_CHECK_LAUNCH(ctx, march_render_chunk(a, st));
   }
   return NERF_OK;
 }
@@ -264,6 +356,9 @@ nerf_status nerf_render(nerf_ctx* ctx, const float* rays_o, const float* rays_d,
   cudaStream_t st = (cudaStream_t)stream;
   const nerf_config& c = ctx->cfg;
   const int64_t R = n_rays;
+  if (c.model != NERF_MODEL_MLP)
+    return render_march(ctx, rays_o, rays_d, R, near, n_coarse, params, out_rgb, out_depth,
+                        out_acc, st);
   const uint64_t key = sm64_mix(params->seed);
   SampleSpec coarse{};
   coarse.mode = SAMPLES_STRATIFIED;
@@ -412,6 +507,59 @@ nerf_status nerf_test_sample_pdf(const float* t_coarse, const float* weights, in
   NERF_CHECK_LAUNCH(nullptr, launch_sample_pdf(t_coarse, weights, n_rays, Nc, Nf, sm64_mix(seed),
                                                perturb, out_t_fine, out_below, out_t_all,
                                                (cudaStream_t)stream));
+  return NERF_OK;
+}
+
+}  // extern "C"
+
+// ----------------------------------------------------------------- march unit entry points
+
+extern "C" {
+
+nerf_status nerf_test_march(const float* rays_o, const float* rays_d, int64_t n_rays, float near,
+                            float step, int K, const uint32_t* occupancy, int32_t* out_count,
+                            uint8_t* out_live, void* stream) {
+  if (!rays_o || !rays_d || !occupancy || !out_count || n_rays <= 0 || K < 1 || K > 512 ||
+      !(step > 0.0f))
+    return fail(nullptr, NERF_ERR_INVALID_ARG, "nerf_test_march: bad argument");
+  NERF_CHECK_LAUNCH(nullptr, launch_march_mask(rays_o, rays_d, n_rays, near, step, K, occupancy,
+                                               nullptr, out_count, out_live, (cudaStream_t)stream));
+  return NERF_OK;
+}
+
+nerf_status nerf_test_route_cells(const float* x, int64_t n, int32_t* out_cell,
+                                  int32_t* out_cell_count, int32_t* out_cell_offset,
+                                  int32_t* out_order, void* stream) {
+  if (!x || !out_cell || !out_cell_count || !out_cell_offset || n <= 0 || n > (int64_t(1) << 30))
+    return fail(nullptr, NERF_ERR_INVALID_ARG, "nerf_test_route_cells: bad argument");
+  cudaStream_t st = (cudaStream_t)stream;
+  int32_t* scratch = nullptr;   // cell fill counters [4096] + scan partials [2048]
+  NERF_CHECK_LAUNCH(nullptr, cudaMallocAsync((void**)&scratch, (4096 + 2048) * sizeof(int32_t), st));
+  unsigned* flag = nullptr;
+  cudaError_t e = cudaMallocAsync((void**)&flag, sizeof(unsigned), st);
+  if (e == cudaSuccess) e = cudaMemsetAsync(flag, 0, sizeof(unsigned), st);
+  if (e == cudaSuccess)
+    e = launch_route_points(x, n, out_cell, out_cell_count, out_cell_offset, out_order, scratch,
+                            scratch + 4096, flag, st);
+  cudaFreeAsync(scratch, st);
+  if (flag) cudaFreeAsync(flag, st);
+  if (e != cudaSuccess) return cuda_fail(nullptr, e, "nerf_test_route_cells");
+  return NERF_OK;
+}
+
+nerf_status nerf_test_hash_encode(const float* x, int64_t n, const uint16_t* hash_table,
+                                  float* out_feat, int32_t* out_rows, void* stream) {
+  if (!x || !hash_table || !out_feat || n <= 0)
+    return fail(nullptr, NERF_ERR_INVALID_ARG, "nerf_test_hash_encode: bad argument");
+  NERF_CHECK_LAUNCH(nullptr, march_prepare(nullptr));
+  NERF_CHECK_LAUNCH(nullptr, launch_hash_encode(x, n, hash_table, out_feat, out_rows,
+                                                (cudaStream_t)stream));
+  return NERF_OK;
+}
+
+nerf_status nerf_test_sh(const float* d, int64_t n, float* out, void* stream) {
+  if (!d || !out || n <= 0) return fail(nullptr, NERF_ERR_INVALID_ARG, "nerf_test_sh: bad argument");
+  NERF_CHECK_LAUNCH(nullptr, launch_sh(d, n, out, (cudaStream_t)stream));
   return NERF_OK;
 }
 

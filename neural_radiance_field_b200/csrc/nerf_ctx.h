@@ -4,6 +4,7 @@
 #include <string>
 
 #include "nerf_internal.cuh"
+#include "nerf_march.cuh"
 
 struct nerf_ctx {
   nerf_config cfg{};
@@ -24,6 +25,10 @@ struct nerf_ctx {
   bool timing = false;
   int n_timed = 0;
   cudaEvent_t* ev = nullptr;   // 2 * kMaxTimed events, created on first enable
+
+  // march models (KILONERF, HASHGRID): ray chunks and their live-entry workspace
+  int64_t chunk_rays = 0;
+  nerfb::MarchWs mws{};
 
   // tensor-core (bf16) path
   bool tc_enabled = false;

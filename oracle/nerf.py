@@ -261,10 +261,24 @@ def sample_pdf(bins, weights, m):
 # --------------------------------------------------------------------------
 
 def render_nerf(wl, o, d, ray_ids, coarse_flat, fine_flat=None, seed=None, perturb=True,
-                chunk=512, return_aux=False):
+                chunk=512, return_aux=False, raw_noise=None):
     """Render rays (o, d fp32 [R,3], global indices ray_ids) with workload `wl`
-    (a synth.Workload). Returns dict with rgb [R,3], depth [R], acc [R] (fp64)
-    and, with return_aux, the intermediates of both passes."""
+    (a nerf_inputs.Workload). Returns dict with rgb [R,3], depth [R], acc [R]
+    (fp64) and, with return_aux, the intermediates of both passes.
+
+    raw_noise = (seed, rel, abs) is a conditioning probe for the tests, never
+    part of the reference result: it perturbs every raw network output as
+    raw * (1 + rel * n1) + abs * n2 with seeded standard normals, to measure how
+    far a ray's result moves when the network is evaluated at a lower working
+    precision (resampling and the page-mode last interval can amplify it)."""
+    noise_rng = np.random.default_rng(raw_noise[0]) if raw_noise else None
+
+    def net(shape, params, oo, dd, t, denc):
+        out = _eval(shape, params, oo, dd, t, denc)
+        if noise_rng is not None:
+            out = (out * (1.0 + raw_noise[1] * noise_rng.standard_normal(out.shape))
+                   + raw_noise[2] * noise_rng.standard_normal(out.shape))
+        return out
     shape = wl.mlp
     seed = wl.seed if seed is None else seed
     pc = split_params(shape, coarse_flat)
@@ -282,7 +296,7 @@ def render_nerf(wl, o, d, ray_ids, coarse_flat, fine_flat=None, seed=None, pertu
         denc = positional_encoding(unit(dd), shape.L_dir)
         # coarse pass
         t_c = stratified_t(wl.near, wl.far, wl.n_coarse, seed, ids, perturb)
-        raw = _eval(shape, pc, oo, dd, t_c, denc)
+        raw = net(shape, pc, oo, dd, t_c, denc)
         sig = sigma_activation(raw[..., 3], wl.sigma_act)
         col = sigmoid(raw[..., :3])
         delta = deltas(t_c, dn, wl.last_delta, far=wl.far)
@@ -308,7 +322,7 @@ def render_nerf(wl, o, d, ray_ids, coarse_flat, fine_flat=None, seed=None, pertu
         t_f, below = sample_pdf(bins, w_c[:, 1:-1], m)
         t_f = t_f.astype(F32)
         t_all = np.sort(np.concatenate([t_c, t_f], axis=-1), axis=-1)
-        raw = _eval(shape, pf, oo, dd, t_all, denc)
+        raw = net(shape, pf, oo, dd, t_all, denc)
         sig = sigma_activation(raw[..., 3], wl.sigma_act)
         col = sigmoid(raw[..., :3])
         delta = deltas(t_all, dn, wl.last_delta, far=wl.far)

@@ -13,10 +13,14 @@ from oracle import nerf as onerf
 # Tolerances (see the design notes, "Parity bar"):
 TOL_FP32 = dict(rgb=1e-4, acc=1e-4, depth_rel=1e-3)      # depth: 1e-3 * (far - near)
 TOL_BF16 = dict(rgb=2e-2, acc=2e-2, depth_far=2e-2)      # depth: 2e-2 * far
-# bounds on the raw network outputs the MLP unit tests enforce; the end-to-end
-# tests treat rays whose last raw density lies within twice this bound of the
-# ReLU kink (the page-mode last interval makes acc jump there) as undetermined
-RAW_BOUND = {S.PREC_FP32: 5e-5, S.PREC_BF16: 2.5e-2}
+# Bounds on the raw network outputs that the MLP unit tests enforce. fp32: a
+# K = 256..320 fp32 dot-product chain, ~K * 2^-24 relative per layer on O(1)
+# values, with margin. bf16: operands and activations rounded to bf16 (2^-9
+# relative) through 10 layers, accumulated with random signs, with margin.
+RAW_BOUND = {S.PREC_FP32: 5e-5, S.PREC_BF16: 5e-3}
+# Working-precision noise for the oracle's conditioning probe (rel, abs): the
+# typical size of the kernel's rounding of a raw output, not a bound on it.
+PROBE_NOISE = {S.PREC_FP32: (0.0, 2e-6), S.PREC_BF16: (2.0 ** -8, 0.0)}
 
 
 def torch_mod():
@@ -73,15 +77,38 @@ def oracle_weights(wl):
     return cw, fw
 
 
+def ray_errors(a, b):
+    return dict(rgb=np.abs(a["rgb"] - b["rgb"]).max(-1), acc=np.abs(a["acc"] - b["acc"]),
+                depth=np.abs(a["depth"] - b["depth"]))
+
+
 def compare(gpu, ref, wl, ids=None, band=None):
-    """Per-ray errors and the set of rays the tolerance applies to."""
+    """Per-ray errors and the rays on which the pages' discontinuity leaves the
+    result undetermined: in page mode (last interval 1e10) a ReLU density whose
+    raw value lies within `band` of 0 at the last sample decides between an
+    opaque and a transparent end of the ray."""
     g = {k: (v[ids] if ids is not None else v) for k, v in gpu.items()}
-    err = dict(rgb=np.abs(g["rgb"] - ref["rgb"]).max(-1), acc=np.abs(g["acc"] - ref["acc"]),
-               depth=np.abs(g["depth"] - ref["depth"]))
+    err = ray_errors(g, ref)
     keep = np.ones(len(err["acc"]), dtype=bool)
     if band is not None and wl.sigma_act == S.SIGMA_RELU and wl.last_delta == S.LAST_DELTA_PAGE:
         keep = np.abs(ref["sigma_last_raw"]) >= band
     return err, keep
+
+
+def conditioned(wl, o_np, d_np, ids, cw, fw, ref, perturb=True):
+    """Rays whose oracle result stays within half the tolerance when every raw
+    network output is perturbed at the kernel's working precision (two seeded
+    draws). Elsewhere the inverse-CDF resampling of a random high-frequency
+    field amplifies rounding beyond the tolerance for any implementation."""
+    rel, ab = PROBE_NOISE[wl.precision]
+    trgb, tacc, tdep = tolerances(wl)
+    ok = np.ones(len(ids), dtype=bool)
+    for s in (101, 202):
+        p = onerf.render_nerf(wl, o_np[ids], d_np[ids], ids, cw, fw, perturb=perturb,
+                              raw_noise=(s, rel, ab))
+        e = ray_errors(p, ref)
+        ok &= (e["rgb"] <= trgb / 2) & (e["acc"] <= tacc / 2) & (e["depth"] <= tdep / 2)
+    return ok
 
 
 def tolerances(wl):

@@ -1,0 +1,188 @@
+"""Parity of the marching scene functions (occupancy march, KiloNeRF cell routing
+and tiny MLPs, hash-grid encoding, SH and hash MLP) with the CPU oracle.
+
+Bit-exact: live candidates (voxel decisions), cell ids, per-cell counts and
+offsets, hash-table rows. Floating point: encodings 1e-5 (fp32 products of fp16
+features), renders 1e-4 rgb/acc and 1e-3 (far - near) depth (fp32 path); rays
+whose early-termination decision lies within 1e-5 of the threshold in the
+oracle are held to 1e-3."""
+import dataclasses
+
+import numpy as np
+import pytest
+
+import nerf_inputs as S
+from oracle import hashgrid as ohash
+from oracle import march as omarch
+from oracle import nerf as onerf
+from oracle import sh as osh
+
+from gpu_cases import rays_for
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def torch():
+    import torch
+    from neural_radiance_field_b200 import build
+    build.build()
+    return torch
+
+
+def _t(torch, a):
+    return torch.from_numpy(np.ascontiguousarray(a)).cuda()
+
+
+@pytest.mark.parametrize("key", ["kilonerf", "hashgrid"])
+def test_march_live_candidates_bit_exact(torch, key):
+    import neural_radiance_field_b200 as nb
+    wl = S.WORKLOADS[key]
+    o, d = rays_for(wl)
+    ids = S.ray_subset(wl.n_rays, 3001, 7)
+    o, d = o[ids].contiguous(), d[ids].contiguous()
+    packed, dense = S.occupancy_grid(wl.seed)
+    R, K = o.shape[0], wl.n_coarse
+    cnt = torch.empty(R, dtype=torch.int32, device="cuda")
+    live = torch.empty(R, K, dtype=torch.uint8, device="cuda")
+    nb.nerf_test_march(o, d, wl.near, wl.march_step, K, _t(torch, packed.view(np.int32)), cnt, live)
+    on, dn = o.cpu().numpy(), d.cpu().numpy()
+    t = onerf.march_t(wl.near, wl.march_step, K)
+    x = on[:, None, :] + t[None, :, None] * dn[:, None, :]
+    ref = omarch.occupied(x.reshape(-1, 3), dense).reshape(R, K)
+    np.testing.assert_array_equal(live.cpu().numpy().astype(bool), ref)
+    np.testing.assert_array_equal(cnt.cpu().numpy(), ref.sum(1))
+    assert ref.any(1).mean() > 0.3           # the blobs are actually hit
+
+
+def test_route_cells_bit_exact(torch):
+    import neural_radiance_field_b200 as nb
+    g = np.random.default_rng(3)
+    x = g.uniform(-1.5, 1.5, size=(50001, 3)).astype(np.float32)
+    edges = (-1.5 + np.arange(128) * 3 / 128).astype(np.float32)
+    x[:1000] = g.choice(edges, size=(1000, 3))             # on voxel and cell boundaries
+    n = x.shape[0]
+    cell = torch.empty(n, dtype=torch.int32, device="cuda")
+    cnt = torch.empty(4096, dtype=torch.int32, device="cuda")
+    off = torch.empty(4097, dtype=torch.int32, device="cuda")
+    order = torch.empty(n, dtype=torch.int32, device="cuda")
+    nb.nerf_test_route_cells(_t(torch, x), cell, cnt, off, order)
+    ref = omarch.cell_id(x)
+    np.testing.assert_array_equal(cell.cpu().numpy(), ref)
+    rc = np.bincount(ref, minlength=4096)
+    np.testing.assert_array_equal(cnt.cpu().numpy(), rc)
+    np.testing.assert_array_equal(off.cpu().numpy(), np.concatenate([[0], np.cumsum(rc)]))
+    # grouping: a permutation whose segments hold exactly each cell's points
+    o_np = order.cpu().numpy()
+    assert np.array_equal(np.sort(o_np), np.arange(n))
+    np.testing.assert_array_equal(ref[o_np], np.repeat(np.arange(4096), rc))
+
+
+def test_hash_encode_rows_exact_and_features(torch):
+    import neural_radiance_field_b200 as nb
+    grid = ohash.HashGrid3D()
+    table = S.hashgrid_table(S.HashGridShape(), grid.n_entries, 5, 1.0)
+    g = np.random.default_rng(4)
+    x = g.uniform(-1.5, 1.5, size=(20011, 3)).astype(np.float32)
+    x[:16] = np.float32(-1.5)                               # lower cube corner
+    x[16:32] = np.nextafter(np.float32(1.5), np.float32(0))  # just inside the upper face
+    n = x.shape[0]
+    feat = torch.empty(n, 32, device="cuda")
+    rows = torch.empty(n, 16, 8, dtype=torch.int32, device="cuda")
+    nb.nerf_test_hash_encode(_t(torch, x), _t(torch, table.view(np.int16)), feat, rows)
+    ref_rows = np.stack([grid.corners(x, l)[0] for l in range(16)], axis=1)
+    np.testing.assert_array_equal(rows.cpu().numpy(), ref_rows)
+    np.testing.assert_allclose(feat.cpu().numpy(), grid.encode(x, table), atol=1e-5)
+
+
+def test_sh_against_oracle(torch):
+    import neural_radiance_field_b200 as nb
+    d = np.random.default_rng(5).normal(size=(4099, 3)).astype(np.float32)
+    d[:3] = [[0, 0, 1], [0, 0, -1], [1, 0, 0]]
+    out = torch.empty(d.shape[0], 16, device="cuda")
+    nb.nerf_test_sh(_t(torch, d), out)
+    np.testing.assert_allclose(out.cpu().numpy(), osh.real_sh(onerf.unit(d)), atol=2e-6)
+
+
+def _render_march(torch, wl, params_kw, o, d):
+    import neural_radiance_field_b200 as nb
+    R = o.shape[0]
+    model = {"kilonerf": nb.NERF_MODEL_KILONERF, "hashgrid": nb.NERF_MODEL_HASHGRID}[wl.model]
+    rnd = nb.Renderer(model=model, max_rays=R, max_samples=wl.n_coarse)
+    rgb = torch.empty(R, 3, device="cuda")
+    dep = torch.empty(R, device="cuda")
+    acc = torch.empty(R, device="cuda")
+    p = rnd.params(march_step=wl.march_step, ert_T=wl.ert_T, **params_kw)
+    rnd.render(o, d, wl.near, wl.far, wl.n_coarse, 0, p, rgb, dep, acc)
+    rnd.sync_status()
+    rnd.close()
+    return dict(rgb=rgb.cpu().numpy(), depth=dep.cpu().numpy(), acc=acc.cpu().numpy())
+
+
+def _check(gpu, ref, ids, wl):
+    err_rgb = np.abs(gpu["rgb"][ids] - ref["rgb"]).max(-1)
+    err_acc = np.abs(gpu["acc"][ids] - ref["acc"])
+    err_dep = np.abs(gpu["depth"][ids] - ref["depth"])
+    near_thr = ref["ert_margin"] < 1e-5
+    tol = np.where(near_thr, 1e-3, 1e-4)
+    # a termination decision taken one sample apart moves depth by at most ert_T * far
+    tdep = 1e-3 * (wl.far - wl.near) + np.where(near_thr, 1e-3 * wl.far, 0.0)
+    print(f"[march e2e {wl.name}] max err rgb {err_rgb.max():.2e} acc {err_acc.max():.2e} "
+          f"depth {err_dep.max():.2e}; near-threshold rays {near_thr.sum()}; "
+          f"live samples/ray {ref['n_live'].mean():.1f}")
+    assert near_thr.mean() < 0.02
+    assert np.all(err_rgb <= tol) and np.all(err_acc <= tol), (err_rgb.max(), err_acc.max())
+    assert np.all(err_dep <= tdep), err_dep.max()
+
+
+def test_e2e_kilonerf_full_frame(torch):
+    wl = S.WORKLOADS["kilonerf"]
+    o, d = rays_for(wl)
+    packed, dense = S.occupancy_grid(wl.seed)
+    cells = S.kilonerf_weights(wl.seed)
+    gpu = _render_march(torch, wl, dict(occupancy=_t(torch, packed.view(np.int32)),
+                                        cell_w=_t(torch, cells)), o, d)
+    ids = S.ray_subset(wl.n_rays, 160, 9)
+    on, dn = o.cpu().numpy()[ids], d.cpu().numpy()[ids]
+    ev = lambda idx, x, du: omarch.kilonerf_eval(cells, omarch.cell_id(x), x, du)
+    ref = omarch.render_march(wl, on, dn, dense, ev)
+    _check(gpu, ref, ids, wl)
+
+
+def test_e2e_hashgrid_full_frame(torch):
+    wl = S.WORKLOADS["hashgrid"]
+    o, d = rays_for(wl)
+    packed, dense = S.occupancy_grid(wl.seed)
+    grid = ohash.HashGrid3D()
+    table = S.hashgrid_table(S.HashGridShape(), grid.n_entries, wl.seed, 1.0)
+    mlp = S.hash_mlp_weights(wl.seed)
+    gpu = _render_march(torch, wl, dict(occupancy=_t(torch, packed.view(np.int32)),
+                                        hash_table=_t(torch, table.view(np.int16)),
+                                        hash_mlp=_t(torch, mlp)), o, d)
+    ids = S.ray_subset(wl.n_rays, 160, 10)
+    on, dn = o.cpu().numpy()[ids], d.cpu().numpy()[ids]
+    ev = lambda idx, x, du: omarch.hash_eval(grid, table, mlp, x, du)
+    ref = omarch.render_march(wl, on, dn, dense, ev)
+    _check(gpu, ref, ids, wl)
+
+
+def test_e2e_march_ragged_small(torch):
+    for key in ("kilonerf", "hashgrid"):
+        wl = dataclasses.replace(S.WORKLOADS[key], H=13, W=17, focal=21.25)
+        o, d = rays_for(wl)
+        packed, dense = S.occupancy_grid(wl.seed)
+        if key == "kilonerf":
+            cells = S.kilonerf_weights(wl.seed)
+            kw = dict(occupancy=_t(torch, packed.view(np.int32)), cell_w=_t(torch, cells))
+            ev = lambda idx, x, du: omarch.kilonerf_eval(cells, omarch.cell_id(x), x, du)
+        else:
+            grid = ohash.HashGrid3D()
+            table = S.hashgrid_table(S.HashGridShape(), grid.n_entries, wl.seed, 1.0)
+            mlp = S.hash_mlp_weights(wl.seed)
+            kw = dict(occupancy=_t(torch, packed.view(np.int32)),
+                      hash_table=_t(torch, table.view(np.int16)), hash_mlp=_t(torch, mlp))
+            ev = lambda idx, x, du: omarch.hash_eval(grid, table, mlp, x, du)
+        gpu = _render_march(torch, wl, kw, o, d)
+        ids = np.arange(wl.n_rays)
+        ref = omarch.render_march(wl, o.cpu().numpy(), d.cpu().numpy(), dense, ev)
+        _check(gpu, ref, ids, wl)
