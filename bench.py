@@ -235,7 +235,11 @@ def run_ours(args, rank, world, local_rank):
     peaks, peak_kind = load_peaks()
     avg_launch_ms = mlp_ms / max(1, mlp_launches)
     achieved_tf = flops_launch_avg / (avg_launch_ms * 1e-3) / 1e12
-    peak_tf = peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops"))
+    # The network kernel holds the top SM clock through a frame (see "clocks"),
+    # so the burst cuBLAS figure is its ceiling; the power-capped sustained figure
+    # is reported beside it.
+    peak_tf = peaks.get("bf16_tflops")
+    peak_sus = peaks.get("bf16_tflops_sustained", peak_tf)
     value = world * R * args.steps / (tot_ms * 1e-3)
     line = None
     if rank == 0:
@@ -255,8 +259,9 @@ def run_ours(args, rank, world, local_rank):
             "mlp_rows_per_s": world * rows * args.steps / (tot_ms * 1e-3),
             "roofline": {"bound": "tensor", "kernel": "scene MLP (coarse and fine launches)",
                          "achieved": achieved_tf, "peak": peak_tf, "unit": "TFLOP/s",
-                         "frac": achieved_tf / peak_tf, "peak_kind": f"bf16 sustained, {peak_kind}",
-                         "traffic": None, "avg_launch_ms": avg_launch_ms,
+                         "frac": achieved_tf / peak_tf, "peak_kind": f"bf16 burst, {peak_kind}",
+                         "frac_of_sustained": achieved_tf / peak_sus,
+                         "traffic": args.traffic_bytes or None, "avg_launch_ms": avg_launch_ms,
                          "flop_per_launch": flops_launch_avg},
             "cpu_baseline": cpu,
             "e2e": {"value": world * R / (e2e_ms * 1e-3), "unit": UNIT,
@@ -280,6 +285,8 @@ def main():
     ap.add_argument("--cpu-rays", type=int, default=1024)
     ap.add_argument("--ref-rays", type=int, default=128)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--traffic-bytes", type=float, default=0.0,
+                    help="DRAM bytes per network launch from an ncu capture of this kernel")
     ap.add_argument("--size", type=int, default=0,
                     help="render an SIZE x SIZE frame instead (profiling runs only)")
     args = ap.parse_args()

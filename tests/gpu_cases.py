@@ -95,20 +95,20 @@ def compare(gpu, ref, wl, ids=None, band=None):
     return err, keep
 
 
-def conditioned(wl, o_np, d_np, ids, cw, fw, ref, perturb=True):
-    """Rays whose oracle result stays within half the tolerance when every raw
-    network output is perturbed at the kernel's working precision (two seeded
-    draws). Elsewhere the inverse-CDF resampling of a random high-frequency
-    field amplifies rounding beyond the tolerance for any implementation."""
+def probe_spread(wl, o_np, d_np, ids, cw, fw, ref, perturb=True, draws=4):
+    """Per ray and output, the largest move of the oracle's own result when every
+    raw network output is perturbed at the kernel's working precision (seeded
+    draws). Where the inverse-CDF resampling of a random high-frequency field
+    amplifies rounding, this spread exceeds the tolerance for any
+    implementation at that precision."""
     rel, ab = PROBE_NOISE[wl.precision]
-    trgb, tacc, tdep = tolerances(wl)
-    ok = np.ones(len(ids), dtype=bool)
-    for s in (101, 202):
+    spread = None
+    for s in range(draws):
         p = onerf.render_nerf(wl, o_np[ids], d_np[ids], ids, cw, fw, perturb=perturb,
-                              raw_noise=(s, rel, ab))
+                              raw_noise=(101 + s, rel, ab))
         e = ray_errors(p, ref)
-        ok &= (e["rgb"] <= trgb / 2) & (e["acc"] <= tacc / 2) & (e["depth"] <= tdep / 2)
-    return ok
+        spread = e if spread is None else {k: np.maximum(spread[k], e[k]) for k in e}
+    return spread
 
 
 def tolerances(wl):

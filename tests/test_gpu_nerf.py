@@ -12,7 +12,7 @@ import nerf_inputs as S
 from oracle import nerf as onerf
 from oracle import rng as orng
 
-from gpu_cases import (RAW_BOUND, compare, conditioned, make_renderer, oracle_render,
+from gpu_cases import (RAW_BOUND, compare, probe_spread, make_renderer, oracle_render,
                        oracle_weights, rays_for, render_gpu, tolerances, weights_tensor)
 
 pytestmark = pytest.mark.gpu
@@ -156,7 +156,11 @@ def test_sample_pdf_bins_exact_and_merge(torch, perturb, Nf):
 def _e2e(torch, wl, n_check, seed_ids, perturb=1, probe=True):
     """Render the whole image on the GPU (the benchmark's launch configuration
     for the 800x800 workload) and compare sampled rays with the oracle.
-    Returns per-ray errors, the rays the tolerance applies to, and the pass mask."""
+
+    Returns per-ray errors, `kink` (page-mode rays whose last raw density is
+    within twice the MLP bound of the ReLU kink: acc jumps there), `strict`
+    (within the tolerance) and `consistent` (within max(tolerance, 3 x the
+    oracle's own spread under working-precision noise))."""
     o, d = rays_for(wl)
     cw, fw = oracle_weights(wl)
     gpu = render_gpu(wl, o, d, weights_tensor(cw, wl.precision),
@@ -166,60 +170,69 @@ def _e2e(torch, wl, n_check, seed_ids, perturb=1, probe=True):
     o_np, d_np = o.cpu().numpy(), d.cpu().numpy()
     ref = oracle_render(wl, o_np, d_np, ids, cw, fw, perturb=bool(perturb))
     err, keep = compare(gpu, ref, wl, ids, band=2 * RAW_BOUND[wl.precision])
-    if probe and wl.n_fine > 0:
-        keep &= conditioned(wl, o_np, d_np, ids, cw, fw, ref, perturb=bool(perturb))
+    kink = ~keep
     trgb, tacc, tdep = tolerances(wl)
-    ok = (err["rgb"] <= trgb) & (err["acc"] <= tacc) & (err["depth"] <= tdep)
-    summary = {k: (float(v[keep].max()) if keep.any() else 0.0, float(v.max())) for k, v in err.items()}
-    print(f"[e2e {wl.name} {wl.H}x{wl.W}] determined {keep.sum()}/{len(keep)}; "
-          f"max err (determined, all): {summary}")
-    return err, keep, ok
+    tol = dict(rgb=trgb, acc=tacc, depth=tdep)
+    strict = np.ones(len(ids), dtype=bool)
+    for k in err:
+        strict &= err[k] <= tol[k]
+    consistent = strict.copy()
+    if probe and wl.n_fine > 0:
+        spread = probe_spread(wl, o_np, d_np, ids, cw, fw, ref, perturb=bool(perturb))
+        consistent = np.ones(len(ids), dtype=bool)
+        for k in err:
+            consistent &= err[k] <= np.maximum(tol[k], 3.0 * spread[k])
+    print(f"[e2e {wl.name} {wl.H}x{wl.W}] rays {len(ids)}: strict {strict.sum()}, "
+          f"kink {kink.sum()}, consistent-or-kink {(consistent | kink).sum()}; max err "
+          f"(off kink): " + ", ".join(f"{k} {err[k][~kink].max():.2e}" for k in err))
+    return err, kink, strict, consistent
 
 
 def test_e2e_tiny_full_image(torch):
     wl = S.WORKLOADS["tiny"]
-    err, keep, ok = _e2e(torch, wl, wl.n_rays, 0)
-    assert keep.all()
-    assert ok.all(), {k: v.max() for k, v in err.items()}
+    err, kink, strict, _ = _e2e(torch, wl, wl.n_rays, 0)
+    assert strict.all(), {k: v.max() for k, v in err.items()}
 
 
 def test_e2e_tiny_variants_ragged(torch):
     for kw in (dict(H=7, W=11), dict(H=1, W=1), dict(H=5, W=9, white_bkgd=1,
                                                         last_delta=S.LAST_DELTA_TO_FAR)):
         wl = dataclasses.replace(S.WORKLOADS["tiny"], **kw)
-        err, keep, ok = _e2e(torch, wl, wl.n_rays, 0)
-        assert ok.all(), (kw, {k: v.max() for k, v in err.items()})
+        err, kink, strict, _ = _e2e(torch, wl, wl.n_rays, 0)
+        assert strict.all(), (kw, {k: v.max() for k, v in err.items()})
+
+
+def _assert_fine_pass(err, kink, strict, consistent, min_strict):
+    """The fine pass resamples a random L=10 field: rays that the inputs do not
+    determine to the tolerance at the working precision are held to the oracle's
+    own spread; the rest to the tolerance."""
+    assert (consistent | kink).all(), {k: v[~(consistent | kink)].max() for k, v in err.items()}
+    assert strict.mean() >= min_strict, strict.mean()
 
 
 def test_e2e_small_fp32_subset(torch):
     wl = S.WORKLOADS["small"]
-    err, keep, ok = _e2e(torch, wl, 384, 1)
-    assert keep.mean() >= 0.8
-    assert ok[keep].all(), {k: v[keep].max() for k, v in err.items()}
+    _assert_fine_pass(*_e2e(torch, wl, 384, 1), min_strict=0.9)
 
 
 def test_e2e_small_fp32_unperturbed_to_far(torch):
     wl = dataclasses.replace(S.WORKLOADS["small"], H=20, W=30, last_delta=S.LAST_DELTA_TO_FAR)
-    err, keep, ok = _e2e(torch, wl, wl.n_rays, 0, perturb=0)
-    assert keep.mean() >= 0.8
-    assert ok[keep].all(), {k: v[keep].max() for k, v in err.items()}
+    _assert_fine_pass(*_e2e(torch, wl, wl.n_rays, 0, perturb=0), min_strict=0.9)
 
 
 def test_e2e_full_bf16_coarse_pass(torch):
     """800x800, bf16 network, coarse pass only: the sample positions are exact on
     both sides, so every ray away from the page-mode kink meets the bar."""
     wl = dataclasses.replace(S.WORKLOADS["full"], n_fine=0)
-    err, keep, ok = _e2e(torch, wl, 512, 4)
-    assert keep.mean() >= 0.8
-    assert ok[keep].all(), {k: v[keep].max() for k, v in err.items()}
+    err, kink, strict, _ = _e2e(torch, wl, 512, 4)
+    assert kink.mean() <= 0.2
+    assert strict[~kink].all(), {k: v[~kink].max() for k, v in err.items()}
 
 
 def test_e2e_full_bf16_sampled(torch):
     """800x800 coarse + fine, bf16 network; sampled rays."""
     wl = S.WORKLOADS["full"]
-    err, keep, ok = _e2e(torch, wl, 256, 3)
-    assert keep.mean() >= 0.7
-    assert ok[keep].all(), {k: v[keep].max() for k, v in err.items()}
+    _assert_fine_pass(*_e2e(torch, wl, 256, 3), min_strict=0.85)
 
 
 def test_render_host_matches_device(torch):
