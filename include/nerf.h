@@ -248,6 +248,31 @@ NERF_API nerf_status nerf_test_hash_encode(const float* x, int64_t n, const uint
  * Condon-Shortley phase) of the unit vectors d/|d|; d [P][3], out [P][16]. */
 NERF_API nerf_status nerf_test_sh(const float* d, int64_t n, float* out, void* stream);
 
+/* ---------------------------------------------------------------------------
+ * Entry point that allocates no device memory. The pages have no counterpart;
+ * it exists for callers that cannot call cudaMalloc, such as a host framework
+ * that owns all device memory through its own allocator, or a render loop held
+ * to a fixed memory budget.
+ *
+ * Occupancy-march compaction (the live-candidate test of nerf_test_march) that
+ * writes, for n_rays <= 1,048,576 rays: out_offsets [n_rays + 1] int32, the
+ * exclusive prefix sum of the per-ray live counts (out_offsets[n_rays] = total
+ * live), and out_live [n_rays * K] uint32 (caller-sized for the worst case),
+ * whose first out_offsets[n_rays] entries are (ray << 9) | k in ray-major, then
+ * k-ascending order. out_live is also used as temporary storage during the call.
+ * Its only scratch is a static 4 KB device array compiled into the library (one
+ * int32 per 1024 rays); every device that loads the library holds it until the
+ * process exits. The first call on each device looks up the array's device
+ * address (cudaGetSymbolAddress); make that first call before any stream
+ * capture. All calls share the array and it keeps the last call's contents:
+ * calls whose work overlaps on the GPU (different streams) race on it.
+ * n_rays above the limit returns NERF_ERR_INVALID_ARG with a message in
+ * nerf_last_error(NULL). */
+NERF_API nerf_status nerf_march_compact_noalloc(const float* rays_o, const float* rays_d,
+                                                int64_t n_rays, float near, float step, int K,
+                                                const uint32_t* occupancy, int32_t* out_offsets,
+                                                uint32_t* out_live, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -564,3 +564,8 @@ nerf_status nerf_test_sh(const float* d, int64_t n, float* out, void* stream) {
 }
 
 }  // extern "C"
+
+namespace nerfb {
+// Records a context-free error message for nerf_last_error(NULL).
+void set_global_error(const char* msg) { g_create_error = msg; }
+}  // namespace nerfb
