@@ -97,6 +97,30 @@ def load_peaks():
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
 
 
+def rank_camera(wl, rank):
+    """Weak scaling: every rank renders one whole frame per step from its own
+    camera (rank 0 renders the workload's camera). Rays never cross ranks."""
+    if rank == 0:
+        return wl.c2w()
+    return S.look_at_c2w(*S.seeded_camera(wl.seed + 1000 * rank))
+
+
+def max_over_ranks(value, dist, device):
+    """Max over ranks of a per-rank device time (the only collective of the
+    benchmark besides barriers; it is outside the timed region)."""
+    if not dist:
+        return float(value)
+    import torch
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_rays_per_s(rays_per_rank_step, world, steps, max_ms):
+    """Whole-job throughput: the rays all ranks rendered over the slowest rank's time."""
+    return world * rays_per_rank_step * steps / (max_ms * 1e-3)
+
+
 def cpu_baseline(wl, n_rays_sample, seed=123):
     """The oracle as it stands, on a bounded seeded sample of the frame's rays."""
     from oracle import nerf as onerf
@@ -155,9 +179,7 @@ def run_ours(args, rank, world, local_rank):
     if args.size:
         import dataclasses
         wl = dataclasses.replace(wl, H=args.size, W=args.size, focal=1.25 * args.size)
-    # each rank renders its own camera (weak scaling: one frame per GPU per step)
-    cam = S.look_at_c2w(*S.seeded_camera(wl.seed + 1000 * rank)) if rank else wl.c2w()
-    c2w = cam.ravel().tolist()
+    c2w = rank_camera(wl, rank).ravel().tolist()
     cw, _ = S.nerf_weights(wl.mlp, wl.seed, 0, wl.sigma_scale, wl.precision)
     fw, _ = S.nerf_weights(wl.mlp, wl.seed, 1, wl.sigma_scale, wl.precision)
     cwt = torch.from_numpy(cw).to(torch.bfloat16).cuda()
@@ -202,11 +224,7 @@ def run_ours(args, rank, world, local_rank):
     mlp_ms, mlp_launches = rnd.timing_read()
     rnd.timing_enable(False)
     rnd.sync_status()
-    tot_ms = sum(step_ms)
-    if dist:
-        t = torch.tensor([tot_ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        tot_ms = float(t.item())
+    tot_ms = max_over_ranks(sum(step_ms), dist, "cuda")
 
     # end to end through the host-buffer entry point (pinned host memory)
     oh, dh = o.cpu().pin_memory(), d.cpu().pin_memory()
@@ -224,11 +242,7 @@ def run_ours(args, rank, world, local_rank):
         rnd.render_host(oh, dh, wl.near, wl.far, wl.n_coarse, wl.n_fine, p, rgbh, deph, acch)
     e1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1) / e2e_steps
-    if dist:
-        t = torch.tensor([e2e_ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, dist, "cuda")
 
     rows = R * (2 * wl.n_coarse + wl.n_fine)
     flops_launch_avg = MLP_FLOP_PER_ROW * rows / 2          # coarse + fine launches per frame
@@ -240,7 +254,7 @@ def run_ours(args, rank, world, local_rank):
     # is reported beside it.
     peak_tf = peaks.get("bf16_tflops")
     peak_sus = peaks.get("bf16_tflops_sustained", peak_tf)
-    value = world * R * args.steps / (tot_ms * 1e-3)
+    value = job_rays_per_s(R, world, args.steps, tot_ms)
     line = None
     if rank == 0:
         cpu = None
@@ -276,6 +290,95 @@ def run_ours(args, rank, world, local_rank):
         dist.destroy_process_group()
 
 
+FP32_PEAK_NOTE = "fp32 FMA: 148 SMs x 128 lanes x 2 FLOP x SM clock"
+
+
+def run_march(args, rank, world, local_rank):
+    """One step = ray generation + a full-frame march render of the KiloNeRF or
+    hash-grid workload (occupancy skipping, scene function, compositing)."""
+    import torch
+    import neural_radiance_field_b200 as nb
+    from neural_radiance_field_b200 import build as nbuild
+    nbuild.build()
+    torch.cuda.set_device(local_rank)
+    wl = S.WORKLOADS[args.workload]
+    c2w = wl.c2w().ravel().tolist()
+    R = wl.n_rays
+    packed, _ = S.occupancy_grid(wl.seed)
+    occ = torch.from_numpy(packed.view(np.int32)).cuda()
+    if wl.model == "kilonerf":
+        model = nb.NERF_MODEL_KILONERF
+        cell_w = torch.from_numpy(S.kilonerf_weights(wl.seed)).cuda()
+        kw = dict(occupancy=occ, cell_w=cell_w)
+        flop_per_point, kname = 2 * 3249, "kilo_eval_kernel (per-cell tiny MLPs)"
+    else:
+        model = nb.NERF_MODEL_HASHGRID
+        table = torch.from_numpy(
+            S.hashgrid_table(S.HashGridShape(), S.HASH_ENTRIES, wl.seed, 1e-4).view(np.int16)).cuda()
+        mlp = torch.from_numpy(S.hash_mlp_weights(wl.seed)).cuda()
+        kw = dict(occupancy=occ, hash_table=table, hash_mlp=mlp)
+        flop_per_point, kname = 2 * 15616, "hash_eval_kernel (encoding + MLPs)"
+    o = torch.empty(R, 3, device="cuda")
+    d = torch.empty(R, 3, device="cuda")
+    rgb = torch.empty(R, 3, device="cuda")
+    dep = torch.empty(R, device="cuda")
+    acc = torch.empty(R, device="cuda")
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    rnd = nb.Renderer(model=model, max_rays=R, max_samples=wl.n_coarse)
+    p = rnd.params(march_step=wl.march_step, ert_T=wl.ert_T, **kw)
+    nb.nerf_raygen(wl.H, wl.W, wl.focal, c2w, o, d)
+    cnt = torch.empty(R, dtype=torch.int32, device="cuda")
+    nb.nerf_test_march(o, d, wl.near, wl.march_step, wl.n_coarse, occ, cnt)
+    live = int(cnt.sum().item())          # occupied candidates (before termination)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        nb.nerf_raygen(wl.H, wl.W, wl.focal, c2w, o, d)
+        rnd.render(o, d, wl.near, wl.far, wl.n_coarse, 0, p, rgb, dep, acc)
+
+    for _ in range(args.warmup):
+        flush.fill_(1)
+        step()
+    torch.cuda.synchronize()
+    rnd.sync_status()
+    rnd.timing_enable(True)
+    rnd.timing_read()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    with ClockSampler(local_rank) as clk:
+        for k in range(args.steps):
+            flush.fill_(k & 0xFF)
+            ev[k][0].record(stream)
+            step()
+            ev[k][1].record(stream)
+        torch.cuda.synchronize()
+    tot_ms = sum(a.elapsed_time(b) for a, b in ev)
+    k_ms, k_launches = rnd.timing_read()
+    rnd.timing_enable(False)
+    rnd.sync_status()
+    clocks = clk.summary()
+    sm_mhz = clocks["sm_mhz"] or 1965.0
+    peak = 148 * 128 * 2 * sm_mhz * 1e6 / 1e12
+    per_frame_k_ms = k_ms / args.steps
+    achieved = live * flop_per_point / (per_frame_k_ms * 1e-3) / 1e12
+    line = {"metric": f"rays/sec, {wl.name} march render", "value": R * args.steps / (tot_ms * 1e-3),
+            "unit": UNIT, "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": tot_ms / args.steps, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": wl.name, "H": wl.H, "W": wl.W, "candidates": wl.n_coarse,
+                       "march_step": wl.march_step, "ert_T": wl.ert_T,
+                       "occupied_candidates_per_frame": live,
+                       "l2": "flushed between timed steps (256 MiB write)"},
+            "sample_points_per_s": live * args.steps / (tot_ms * 1e-3),
+            "roofline": {"bound": "alu", "kernel": kname, "achieved": achieved, "peak": peak,
+                         "unit": "TFLOP/s", "frac": achieved / peak, "peak_kind": FP32_PEAK_NOTE,
+                         "traffic": None, "kernel_ms_per_frame": per_frame_k_ms,
+                         "flop_per_point": flop_per_point},
+            "gpu_launches": None, "clocks": clocks}
+    print(json.dumps(line), flush=True)
+    rnd.close()
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -285,6 +388,8 @@ def main():
     ap.add_argument("--cpu-rays", type=int, default=1024)
     ap.add_argument("--ref-rays", type=int, default=128)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--workload", default=WORKLOAD, choices=[WORKLOAD, "kilonerf", "hashgrid"],
+                    help="the benchmark workload (default) or a march workload (extra lines)")
     ap.add_argument("--traffic-bytes", type=float, default=0.0,
                     help="DRAM bytes per network launch from an ncu capture of this kernel")
     ap.add_argument("--size", type=int, default=0,
@@ -295,6 +400,8 @@ def main():
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     if args.impl == "reference":
         run_reference(args, rank, world)
+    elif args.workload != WORKLOAD:
+        run_march(args, rank, world, local_rank)
     else:
         run_ours(args, rank, world, local_rank)
 

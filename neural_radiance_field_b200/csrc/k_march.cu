@@ -549,6 +549,7 @@ cudaError_t march_render_chunk(const MarchArgs& a, cudaStream_t st) {
   const int32_t* total = a.ws.off + R;
   const unsigned g = (unsigned)(a.num_sms * 8);
   if (a.model == NERF_MODEL_HASHGRID) {
+    if (a.ev_start) cudaEventRecord(a.ev_start, st);
     hash_eval_kernel<<<g, 128, HASH_NW * sizeof(float), st>>>(
         a.o, a.d, a.r0, a.near, a.step, a.ws.live, total,
         reinterpret_cast<const __half2*>(a.hash_table), a.hash_mlp, a.sh, a.ws.val);
@@ -562,9 +563,11 @@ cudaError_t march_render_chunk(const MarchArgs& a, cudaStream_t st) {
     cell_scatter_kernel<<<g, 256, 0, st>>>(a.ws.cell, total, 0, a.ws.cell_off, a.ws.cell_fill,
                                            a.ws.order);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if (a.ev_start) cudaEventRecord(a.ev_start, st);
     kilo_eval_kernel<<<g, 128, 0, st>>>(a.o, a.d, a.r0, a.near, a.step, a.ws.live, total,
                                         a.ws.order, a.ws.cell, a.cell_w, a.ws.val);
   }
+  if (a.ev_stop) cudaEventRecord(a.ev_stop, st);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   march_composite_kernel<<<(unsigned)((R + 7) / 8), 256, 0, st>>>(
       a.d, a.r0, R, a.near, a.step, a.ert_T, a.ws.off, a.ws.live, a.ws.val, a.rgb, a.depth, a.acc);

@@ -338,6 +338,12 @@ nerf_status render_march(nerf_ctx* ctx, const float* o, const float* d, int64_t 
   for (int64_t r0 = 0; r0 < R; r0 += ctx->chunk_rays) {
     a.r0 = r0;
     a.R = R - r0 < ctx->chunk_rays ? R - r0 : ctx->chunk_rays;
+    a.ev_start = a.ev_stop = nullptr;
+    if (ctx->timing && ctx->n_timed < kMaxTimed) {
+      const int slot = ctx->n_timed++;
+      a.ev_start = ctx->ev[2 * slot];
+      a.ev_stop = ctx->ev[2 * slot + 1];
+    }
     NERF_CHECK_LAUNCH(ctx, march_render_chunk(a, st));
   }
   return NERF_OK;

@@ -50,6 +50,8 @@ struct MarchArgs {
   unsigned* flag;
   int num_sms;
   MarchWs ws;
+  cudaEvent_t ev_start = nullptr;   // recorded around the scene-function kernel
+  cudaEvent_t ev_stop = nullptr;    // when timing is enabled
 };
 
 cudaError_t march_prepare(cudaStream_t st);
