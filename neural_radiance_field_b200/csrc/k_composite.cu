@@ -172,24 +172,44 @@ __device__ void resample_ray(ResampleSmem& sm, int64_t ray, int Nf, uint64_t key
     if (t_f) t_f[ray * Nf + k] = t;
     if (below_out) below_out[ray * Nf + k] = below;
   }
+  // pad the draws to 128 with +inf and sort them (bitonic network, 4 keys per lane)
+  for (int k = Nf + lane; k < 128; k += 32) sm.tf[k] = __int_as_float(0x7f800000);
   __syncwarp();
   if (!t_all) return;
+  for (int kb = 2; kb <= 128; kb <<= 1) {
+    for (int j = kb >> 1; j > 0; j >>= 1) {
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int i = lane + 32 * q;
+        const int p = i ^ j;
+        if (p > i) {
+          const float a = sm.tf[i], b = sm.tf[p];
+          const bool up = (i & kb) == 0;
+          if (up ? (a > b) : (a < b)) { sm.tf[i] = b; sm.tf[p] = a; }
+        }
+      }
+      __syncwarp();
+    }
+  }
+  // merge with the 64 sorted coarse positions (coarse first among equal values)
   const int S = 64 + Nf;
   for (int j = lane; j < Nf; j += 32) {
-    float v = sm.tf[j];
-    int pos = 0;
-    for (int i = 0; i < Nf; ++i) {
-      float u = sm.tf[i];
-      pos += (u < v) || (u == v && i < j);
+    const float v = sm.tf[j];
+    int lo = 0, hi = 64;                       // #{c : tc[c] <= v}
+    while (lo < hi) {
+      const int mid = (lo + hi) >> 1;
+      if (sm.tc[mid] <= v) lo = mid + 1; else hi = mid;
     }
-    for (int c = 0; c < 64; ++c) pos += sm.tc[c] <= v;
-    t_all[ray * S + pos] = v;
+    t_all[ray * S + j + lo] = v;
   }
   for (int c = lane; c < 64; c += 32) {
-    float v = sm.tc[c];
-    int pos = c;
-    for (int i = 0; i < Nf; ++i) pos += sm.tf[i] < v;
-    t_all[ray * S + pos] = v;
+    const float v = sm.tc[c];
+    int lo = 0, hi = Nf;                       // #{f : tf[f] < v}
+    while (lo < hi) {
+      const int mid = (lo + hi) >> 1;
+      if (sm.tf[mid] < v) lo = mid + 1; else hi = mid;
+    }
+    t_all[ray * S + c + lo] = v;
   }
 }
 

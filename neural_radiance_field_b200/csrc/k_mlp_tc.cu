@@ -2,21 +2,24 @@
 // sm_100a: tcgen05.mma with fp32 accumulators in tensor memory, weights streamed
 // by the bulk-copy engine, activations kept on chip for the whole network.
 //
-// Persistent kernel, one CTA per SM, 10 warps:
-//   warp 0      issues the MMAs (one elected thread) and owns the TMEM allocation
-//   warp 1      streams the packed weights into a 4-slot shared-memory ring
-//   warps 2-5   epilogue of tile A (128 rows, thread = row = TMEM lane)
-//   warps 6-9   epilogue of tile B
+// Persistent kernel, one CTA per SM, 18 warps:
+//   warp 0       issues the MMAs (one elected thread) and owns the TMEM allocation
+//   warp 1       streams the packed weights into a 4-slot shared-memory ring
+//   warps 2-9    epilogue of tile A: warp w drains TMEM lane quarter (w % 4) of
+//                column half ((w - 2) / 4) % 2, i.e. thread = (row, half)
+//   warps 10-17  epilogue of tile B, same split
 // A CTA works on pairs of 128-row tiles. Every weight chunk that lands in the
 // ring feeds both tiles before its slot is refilled, so each weight byte read
 // from L2 serves 256 rows. Per layer the accumulators of both tiles (2 x 256
 // fp32 columns = all 512 TMEM columns) are drained by the epilogue warps, which
 // add the bias, apply ReLU, round to bf16 and write the next layer's A operand
-// back into shared memory.
+// back into shared memory. Two warps per lane quarter keep twice as many TMEM
+// loads in flight as one would; the drain is latency-bound, not bandwidth-bound.
 //
-// Shared memory (229,376 B): act[2] = per tile 128 rows x 320 bf16 holding
+// Shared memory (231,680 B): act[2] = per tile 128 rows x 320 bf16 holding
 // [h (256) | gamma(x) (63) | 0], so the skip layer reads columns 0..319 and the
-// first layer columns 256..319; ring[4] = weight chunks of K = 32 columns.
+// first layer columns 256..319; ring[4] = weight chunks of K = 32 columns;
+// 2 KB of per-layer epilogue vectors; barriers.
 // Operands use the no-swizzle K-major core-matrix layout: element (r, k) of a
 // block of R rows sits at (k/8)*R*16 + (r/8)*128 + (r%8)*16 + (k%8)*2 bytes.
 #include "nerf_ctx.h"
@@ -32,8 +35,10 @@ constexpr int CHUNK_K = 32;
 constexpr int NSTAGE = 4;
 constexpr int RING_BYTES = 256 * CHUNK_K * 2;       // 16384 per slot
 constexpr int NLAYER = 10;                          // pts0..pts7, feature, dir
-constexpr int NTHREADS = 320;
-constexpr int VEC_BYTES = 2 * 256 * 4;                // staged epilogue vectors
+constexpr int EPI_THREADS = 512;                    // 16 epilogue warps
+constexpr int TILE_THREADS = 256;                   // epilogue threads per tile
+constexpr int NTHREADS = 64 + EPI_THREADS;
+constexpr int VEC_BYTES = 2 * 256 * 4;              // staged epilogue vectors
 constexpr size_t SMEM_BYTES = 2 * ACT_BYTES + NSTAGE * RING_BYTES + VEC_BYTES + 256;
 
 // per layer: K chunks, output width, first K-group of the A operand
@@ -178,23 +183,6 @@ __device__ __forceinline__ void mma_commit(uint64_t* bar) {
                ::"r"(smem_u32(bar)) : "memory");
 }
 
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v) {
-  uint32_t r[32];
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
-      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
-      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
-        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
-        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
-        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-      : "r"(taddr));
-  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-#pragma unroll
-  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
-}
-
 // Two fp32 -> packed bf16x2 with ReLU (lo = first element in memory order).
 __device__ __forceinline__ uint32_t pack_relu(float lo, float hi) {
   uint32_t d;
@@ -260,18 +248,18 @@ __device__ __forceinline__ void tmem_wait32(uint32_t* r) {
                : "memory");
 }
 
-// Barrier among the 256 epilogue threads only (named barrier 1).
-__device__ __forceinline__ void epilogue_sync() {
-  asm volatile("bar.sync 1, 256;" ::: "memory");
+// Named barriers: 1 = all 512 epilogue threads, 2 + g = the 256 threads of tile g.
+__device__ __forceinline__ void named_sync(int id, int count) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 
-// Same barrier, returning whether any of the 256 threads passed true.
+// Barrier over all epilogue threads that returns whether any passed true.
 __device__ __forceinline__ bool epilogue_sync_or(bool v) {
   uint32_t r;
   asm volatile(
       "{\n\t.reg .pred p, q;\n\t"
       "setp.ne.u32 p, %1, 0;\n\t"
-      "bar.red.or.pred q, 1, 256, p;\n\t"
+      "bar.red.or.pred q, 1, 512, p;\n\t"
       "selp.u32 %0, 1, 0, q;\n\t}"
       : "=r"(r)
       : "r"((uint32_t)v)
@@ -280,59 +268,93 @@ __device__ __forceinline__ bool epilogue_sync_or(bool v) {
 }
 
 // One 32-column block of a hidden layer: bias, activation, bf16, store to the
-// next layer's A operand; on the last trunk layer also accumulates sigma.
+// next layer's A operand; on the last trunk layer also accumulates sigma. Works
+// 8 columns at a time so that only the loaded block stays live.
 template <bool RELU, bool SIGMA>
 __device__ __forceinline__ void epi_block(const uint32_t* u, const float* sb_bias,
                                           const float* sb_ws, int cb, uint32_t act_base, int r,
                                           float& sigma) {
-  float v[32];
-#pragma unroll
-  for (int i = 0; i < 32; i += 4) {
-    const float4 b4 = *reinterpret_cast<const float4*>(sb_bias + cb + i);
-    v[i] = __uint_as_float(u[i]) + b4.x;
-    v[i + 1] = __uint_as_float(u[i + 1]) + b4.y;
-    v[i + 2] = __uint_as_float(u[i + 2]) + b4.z;
-    v[i + 3] = __uint_as_float(u[i + 3]) + b4.w;
-  }
-  if (SIGMA) {
-#pragma unroll
-    for (int i = 0; i < 32; i += 4) {
-      const float4 w4 = *reinterpret_cast<const float4*>(sb_ws + cb + i);
-      sigma = fmaf(fmaxf(v[i], 0.f), w4.x, sigma);
-      sigma = fmaf(fmaxf(v[i + 1], 0.f), w4.y, sigma);
-      sigma = fmaf(fmaxf(v[i + 2], 0.f), w4.z, sigma);
-      sigma = fmaf(fmaxf(v[i + 3], 0.f), w4.w, sigma);
-    }
-  }
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
-    const float* p = v + 8 * j;
+    const float4 b0 = *reinterpret_cast<const float4*>(sb_bias + cb + 8 * j);
+    const float4 b1 = *reinterpret_cast<const float4*>(sb_bias + cb + 8 * j + 4);
+    float v[8];
+    v[0] = __uint_as_float(u[8 * j + 0]) + b0.x;
+    v[1] = __uint_as_float(u[8 * j + 1]) + b0.y;
+    v[2] = __uint_as_float(u[8 * j + 2]) + b0.z;
+    v[3] = __uint_as_float(u[8 * j + 3]) + b0.w;
+    v[4] = __uint_as_float(u[8 * j + 4]) + b1.x;
+    v[5] = __uint_as_float(u[8 * j + 5]) + b1.y;
+    v[6] = __uint_as_float(u[8 * j + 6]) + b1.z;
+    v[7] = __uint_as_float(u[8 * j + 7]) + b1.w;
+    if (SIGMA) {
+      const float4 w0 = *reinterpret_cast<const float4*>(sb_ws + cb + 8 * j);
+      const float4 w1 = *reinterpret_cast<const float4*>(sb_ws + cb + 8 * j + 4);
+      sigma = fmaf(fmaxf(v[0], 0.f), w0.x, sigma);
+      sigma = fmaf(fmaxf(v[1], 0.f), w0.y, sigma);
+      sigma = fmaf(fmaxf(v[2], 0.f), w0.z, sigma);
+      sigma = fmaf(fmaxf(v[3], 0.f), w0.w, sigma);
+      sigma = fmaf(fmaxf(v[4], 0.f), w1.x, sigma);
+      sigma = fmaf(fmaxf(v[5], 0.f), w1.y, sigma);
+      sigma = fmaf(fmaxf(v[6], 0.f), w1.z, sigma);
+      sigma = fmaf(fmaxf(v[7], 0.f), w1.w, sigma);
+    }
     uint32_t w0, w1, w2, w3;
     if (RELU) {
-      w0 = pack_relu(p[0], p[1]); w1 = pack_relu(p[2], p[3]);
-      w2 = pack_relu(p[4], p[5]); w3 = pack_relu(p[6], p[7]);
+      w0 = pack_relu(v[0], v[1]); w1 = pack_relu(v[2], v[3]);
+      w2 = pack_relu(v[4], v[5]); w3 = pack_relu(v[6], v[7]);
     } else {
-      w0 = pack_plain(p[0], p[1]); w1 = pack_plain(p[2], p[3]);
-      w2 = pack_plain(p[4], p[5]); w3 = pack_plain(p[6], p[7]);
+      w0 = pack_plain(v[0], v[1]); w1 = pack_plain(v[2], v[3]);
+      w2 = pack_plain(v[4], v[5]); w3 = pack_plain(v[6], v[7]);
     }
     st_shared_v4(act_base + act_off(r, cb + 8 * j), w0, w1, w2, w3);
   }
 }
 
+// 128 columns [c0, c0 + 128) of a 256-wide hidden layer, two TMEM loads in flight.
 template <bool RELU, bool SIGMA>
-__device__ __forceinline__ void epi_layer(uint32_t t_row, const float* sb_bias, const float* sb_ws,
-                                          uint32_t act_base, int r, float& sigma) {
+__device__ __forceinline__ void epi_half(uint32_t t_row, int c0, const float* sb_bias,
+                                         const float* sb_ws, uint32_t act_base, int r,
+                                         float& sigma) {
   uint32_t ua[32], ub[32];
-  tmem_ld32_issue(t_row, ua);
+  tmem_ld32_issue(t_row + c0, ua);
+  tmem_ld32_issue(t_row + c0 + 32, ub);
   tmem_wait32(ua);
-#pragma unroll
-  for (int cb = 0; cb < 256; cb += 64) {
-    tmem_ld32_issue(t_row + cb + 32, ub);
-    epi_block<RELU, SIGMA>(ua, sb_bias, sb_ws, cb, act_base, r, sigma);
-    tmem_wait32(ub);
-    if (cb + 64 < 256) tmem_ld32_issue(t_row + cb + 64, ua);
-    epi_block<RELU, SIGMA>(ub, sb_bias, sb_ws, cb + 32, act_base, r, sigma);
-    if (cb + 64 < 256) tmem_wait32(ua);
+  tmem_wait32(ub);
+  epi_block<RELU, SIGMA>(ua, sb_bias, sb_ws, c0, act_base, r, sigma);
+  tmem_ld32_issue(t_row + c0 + 64, ua);
+  epi_block<RELU, SIGMA>(ub, sb_bias, sb_ws, c0 + 32, act_base, r, sigma);
+  tmem_ld32_issue(t_row + c0 + 96, ub);
+  tmem_wait32(ua);
+  tmem_wait32(ub);
+  epi_block<RELU, SIGMA>(ua, sb_bias, sb_ws, c0 + 64, act_base, r, sigma);
+  epi_block<RELU, SIGMA>(ub, sb_bias, sb_ws, c0 + 96, act_base, r, sigma);
+}
+
+// Positional-encoding value J (0..63) of a point: [x, sin block, cos block, 0],
+// sin and cos blocks coordinate-major (c * 10 + k): sin/cos(pi 2^k x_c).
+template <int J>
+__device__ __forceinline__ float pe_value(float x0, float x1, float x2) {
+  if (J < 3) return J == 0 ? x0 : (J == 1 ? x1 : x2);
+  if (J == 63) return 0.0f;
+  constexpr int jj = J < 33 ? J - 3 : J - 33;
+  constexpr int c = jj / 10, k = jj % 10;
+  const float xc = c == 0 ? x0 : (c == 1 ? x1 : x2);
+  return J < 33 ? sinpif(ldexpf(xc, k)) : cospif(ldexpf(xc, k));
+}
+
+// Columns [32 H, 32 H + 32) of gamma(x), packed to bf16 and stored as the
+// A operand's K-groups 32 + 4H .. 35 + 4H.
+template <int H, int G = 0>
+__device__ __forceinline__ void store_pe(float x0, float x1, float x2, uint32_t act_base, int r) {
+  if constexpr (G < 4) {
+    constexpr int k0 = H * 32 + 8 * G;
+    st_shared_v4(act_base + act_off(r, 256 + k0),
+                 pack_plain(pe_value<k0 + 0>(x0, x1, x2), pe_value<k0 + 1>(x0, x1, x2)),
+                 pack_plain(pe_value<k0 + 2>(x0, x1, x2), pe_value<k0 + 3>(x0, x1, x2)),
+                 pack_plain(pe_value<k0 + 4>(x0, x1, x2), pe_value<k0 + 5>(x0, x1, x2)),
+                 pack_plain(pe_value<k0 + 6>(x0, x1, x2), pe_value<k0 + 7>(x0, x1, x2)));
+    store_pe<H, G + 1>(x0, x1, x2, act_base, r);
   }
 }
 
@@ -356,7 +378,10 @@ __global__ void __launch_bounds__(NTHREADS, 1) mlp_tc_kernel(Params P) {
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < NSTAGE; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
-    for (int g = 0; g < 2; ++g) { mbar_init(&mma_done[g], 1); mbar_init(&act_ready[g], TM); }
+    for (int g = 0; g < 2; ++g) {
+      mbar_init(&mma_done[g], 1);
+      mbar_init(&act_ready[g], TILE_THREADS);
+    }
     mbar_init(final_bar, 1);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -433,14 +458,19 @@ __global__ void __launch_bounds__(NTHREADS, 1) mlp_tc_kernel(Params P) {
     }
   } else {
     // ---------------------------------------------------------- epilogue
-    const int et = threadIdx.x - 64;              // 0..255 over both tiles
-    const int g = (warp - 2) >> 2;                // tile within the pair
+    const int et = threadIdx.x - 64;              // 0..511
+    const int g = et >> 8;                        // tile within the pair
+    const int h = (et >> 7) & 1;                  // column half
     const int quarter = warp & 3;                 // TMEM lane quarter of this warp
     const int r = quarter * 32 + lane;            // row in the tile = TMEM lane
-    const uint32_t act_base = smem_u32(act + g * ACT_BYTES);
+    uint8_t* my_act = act + g * ACT_BYTES;
+    const uint32_t act_base = smem_u32(my_act);
     const uint32_t t_row = tmem + (uint32_t)(g * 256) + ((uint32_t)(quarter * 32) << 16);
     float* sb0 = svec;          // layer bias / rgb weights rows 0, 1
     float* sb1 = svec + 256;    // sigma weights / rgb row 2, rgb and sigma biases
+    // partial (sigma, r, g, b) of the second column half, handed to the first
+    // half through the tile's (then idle) activation buffer
+    float4* xchg = reinterpret_cast<float4*>(my_act);
     uint32_t ph_md = 0;
     const float* vec = P.vec;
     for (int64_t pr = blockIdx.x; pr < P.n_pairs; pr += gridDim.x) {
@@ -465,60 +495,50 @@ __global__ void __launch_bounds__(NTHREADS, 1) mlp_tc_kernel(Params P) {
           for (int c = 0; c < 3; ++c) x[c] = fadd(P.o[ray * 3 + c], fmul(t, P.d[ray * 3 + c]));
         }
       }
-      // gamma(x) -> columns 256..319 (layer -1 "epilogue")
-      {
-        float e[64];
-        e[0] = x[0]; e[1] = x[1]; e[2] = x[2];
-#pragma unroll
-        for (int c = 0; c < 3; ++c)
-#pragma unroll
-          for (int k = 0; k < 10; ++k) pe_sincos(x[c], k, &e[3 + c * 10 + k], &e[33 + c * 10 + k]);
-        e[63] = 0.0f;
-#pragma unroll
-        for (int j = 0; j < 8; ++j)
-          st_shared_v4(act_base + act_off(r, 256 + 8 * j), pack_plain(e[8 * j], e[8 * j + 1]),
-                       pack_plain(e[8 * j + 2], e[8 * j + 3]), pack_plain(e[8 * j + 4], e[8 * j + 5]),
-                       pack_plain(e[8 * j + 6], e[8 * j + 7]));
-      }
+      // gamma(x) -> columns 256..319; this half writes 32 of the 64 columns
+      if (h == 0) store_pe<0>(x[0], x[1], x[2], act_base, r);
+      else store_pe<1>(x[0], x[1], x[2], act_base, r);
       fence_async_smem();
       mbar_arrive(&act_ready[g]);
 
       float sigma = 0.0f;
       for (int l = 0; l < NLAYER; ++l) {
         // this layer's epilogue vectors: loaded now, staged after the MMA wait
-        float pre0, pre1 = 0.0f;
+        float pre;
         if (l < 9) {
-          pre0 = __ldg(vec + P.lay.bias[l] + et);
-          if (l == 7) pre1 = __ldg(vec + P.lay.w_sigma + et);
+          pre = et < 256 ? __ldg(vec + P.lay.bias[l] + et)
+                         : (l == 7 ? __ldg(vec + P.lay.w_sigma + et - 256) : 0.0f);
         } else {
-          pre0 = __ldg(vec + P.lay.w_rgb + et);
-          if (et < 128) pre1 = __ldg(vec + P.lay.w_rgb + 256 + et);
-          else if (et < 131) pre1 = __ldg(vec + P.lay.b_rgb + et - 128);
-          else if (et == 131) pre1 = __ldg(vec + P.lay.b_sigma);
+          const int q2 = et - 256;
+          pre = et < 256 ? __ldg(vec + P.lay.w_rgb + et)
+              : q2 < 128 ? __ldg(vec + P.lay.w_rgb + 256 + q2)
+              : q2 < 131 ? __ldg(vec + P.lay.b_rgb + q2 - 128)
+              : q2 == 131 ? __ldg(vec + P.lay.b_sigma) : 0.0f;
         }
         const bool waited = mbar_wait(&mma_done[g], ph_md, ctl);
         ph_md ^= 1;
         tc_fence_after();
-        // both tiles are done with the previous vectors; all 256 threads agree
-        // on giving up together, so no thread is left behind at a barrier
+        // every epilogue thread is done with the previous vectors; all agree on
+        // giving up together, so no thread is left behind at a barrier
         if (epilogue_sync_or(!waited || *abort_flag)) break;
-        sb0[et] = pre0;
-        sb1[et] = pre1;
-        epilogue_sync();
+        svec[et] = pre;
+        named_sync(1, EPI_THREADS);
         if (l < 9) {
-          if (l == 8) epi_layer<false, false>(t_row, sb0, sb1, act_base, r, sigma);
-          else if (l == 7) epi_layer<true, true>(t_row, sb0, sb1, act_base, r, sigma);
-          else epi_layer<true, false>(t_row, sb0, sb1, act_base, r, sigma);
+          const int c0 = h * 128;
+          if (l == 8) epi_half<false, false>(t_row, c0, sb0, sb1, act_base, r, sigma);
+          else if (l == 7) epi_half<true, true>(t_row, c0, sb0, sb1, act_base, r, sigma);
+          else epi_half<true, false>(t_row, c0, sb0, sb1, act_base, r, sigma);
           tc_fence_before();
           fence_async_smem();
           mbar_arrive(&act_ready[g]);
         } else {
-          // direction layer: + per-ray bias, ReLU, then the rgb head in fp32
+          // direction layer (N = 128): + per-ray bias, ReLU, the rgb head in fp32
+          // on this half's 64 columns; the halves are summed through shared memory
           const float* rb = P.dir_bias + ray * 128;
-          float rgb0 = sb1[128], rgb1 = sb1[129], rgb2 = sb1[130];
-          uint32_t u[32];
+          float rgb0 = 0.f, rgb1 = 0.f, rgb2 = 0.f;
 #pragma unroll 1
-          for (int cb = 0; cb < 128; cb += 32) {
+          for (int cb = h * 64; cb < h * 64 + 64; cb += 32) {
+            uint32_t u[32];
             tmem_ld32_issue(t_row + cb, u);
             float4 bb[8];
 #pragma unroll
@@ -540,9 +560,15 @@ __global__ void __launch_bounds__(NTHREADS, 1) mlp_tc_kernel(Params P) {
             }
           }
           tc_fence_before();
-          if (valid)
+          if (h == 1) xchg[r] = make_float4(sigma, rgb0, rgb1, rgb2);
+          named_sync(2 + g, TILE_THREADS);
+          if (h == 0 && valid) {
+            const float4 o2 = xchg[r];
             *reinterpret_cast<float4*>(P.raw + row * 4) =
-                make_float4(rgb0, rgb1, rgb2, sigma + sb1[131]);
+                make_float4(rgb0 + o2.y + sb1[128], rgb1 + o2.z + sb1[129],
+                            rgb2 + o2.w + sb1[130], sigma + o2.x + sb1[131]);
+          }
+          named_sync(2 + g, TILE_THREADS);
         }
       }
       if (epilogue_sync_or(*abort_flag)) break;
