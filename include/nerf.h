@@ -248,6 +248,17 @@ NERF_API nerf_status nerf_test_hash_encode(const float* x, int64_t n, const uint
  * Condon-Shortley phase) of the unit vectors d/|d|; d [P][3], out [P][16]. */
 NERF_API nerf_status nerf_test_sh(const float* d, int64_t n, float* out, void* stream);
 
+/* Failure detection of the device waits. Every wait of the library's kernels on
+ * a barrier (weight arrival, MMA completion, epilogue hand-off) gives up after a
+ * bound (2 s), sets NERF_ERR_TIMEOUT's flag bit and lets the kernel return, so
+ * the context stays usable and nerf_sync_status reports the timeout. This entry
+ * point runs that same bounded wait, with timeout_us (1..2,000,000), on a
+ * barrier that nothing ever completes: out_flag (device uint32, caller-zeroed)
+ * receives the flag bit (2), out_waited_us (device uint32, may be NULL) the
+ * time waited in microseconds. */
+NERF_API nerf_status nerf_test_bounded_wait(uint32_t timeout_us, uint32_t* out_flag,
+                                            uint32_t* out_waited_us, void* stream);
+
 /* ---------------------------------------------------------------------------
  * Entry point that allocates no device memory. The pages have no counterpart;
  * it exists for callers that cannot call cudaMalloc, such as a host framework

@@ -120,15 +120,17 @@ __device__ __forceinline__ bool mbar_try(uint64_t* bar, uint32_t parity) {
 struct Ctl {
   volatile int* abort;
   unsigned* flag;
+  uint64_t limit_ns;   // wait bound (2 s in the kernels)
 };
+constexpr uint64_t kWaitLimitNs = 2000000000ull;
 
-// Bounded wait: gives up after ~2 s, raises the timeout flag and the CTA abort.
+// Bounded wait: gives up after ctl.limit_ns, raises the timeout flag and the CTA abort.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const Ctl& ctl) {
   if (mbar_try(bar, parity)) return true;
   const uint64_t t0 = globaltimer();
   while (!mbar_try(bar, parity)) {
     if (*ctl.abort) return false;
-    if (globaltimer() - t0 > 2000000000ull) {
+    if (globaltimer() - t0 > ctl.limit_ns) {
       atomicOr(ctl.flag, FLAG_TIMEOUT);
       *ctl.abort = 1;
       return false;
@@ -374,7 +376,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) mlp_tc_kernel(Params P) {
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  Ctl ctl{abort_flag, P.flag};
+  Ctl ctl{abort_flag, P.flag, kWaitLimitNs};
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < NSTAGE; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
@@ -438,7 +440,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) mlp_tc_kernel(Params P) {
       // drain: everything issued so far completes before the CTA frees TMEM
       mma_commit(final_bar);
       uint64_t t0 = globaltimer();
-      while (!mbar_try(final_bar, 0) && globaltimer() - t0 < 2000000000ull) {}
+      while (!mbar_try(final_bar, 0) && globaltimer() - t0 < kWaitLimitNs) {}
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------- weight loader
@@ -583,6 +585,26 @@ __global__ void __launch_bounds__(NTHREADS, 1) mlp_tc_kernel(Params P) {
   }
 }
 
+// A wait that nothing completes, bounded by limit_ns: exercises the timeout
+// path of the kernels' waits (flag bit FLAG_TIMEOUT, no hang, context intact).
+__global__ void bounded_wait_probe_kernel(unsigned* flag, uint64_t limit_ns,
+                                          unsigned* waited_us) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_s;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_s = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    Ctl ctl{&abort_s, flag, limit_ns};
+    const uint64_t t0 = globaltimer();
+    mbar_wait(&bar, 0, ctl);
+    if (waited_us) *waited_us = (unsigned)((globaltimer() - t0) / 1000);
+  }
+}
+
 // ------------------------------------------------------------------ weight packing
 
 struct PackLayer {
@@ -684,6 +706,12 @@ void tc_free(nerf_ctx* ctx) {
   delete s;
   ctx->tc_weights = nullptr;
   ctx->tc_enabled = false;
+}
+
+cudaError_t launch_bounded_wait_probe(uint32_t timeout_us, uint32_t* flag, uint32_t* waited_us,
+                                      cudaStream_t st) {
+  bounded_wait_probe_kernel<<<1, 32, 0, st>>>(flag, (uint64_t)timeout_us * 1000ull, waited_us);
+  return cudaGetLastError();
 }
 
 cudaError_t tc_pack(nerf_ctx* ctx, const void* blob, cudaStream_t st) {

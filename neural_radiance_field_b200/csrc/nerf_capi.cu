@@ -575,3 +575,14 @@ namespace nerfb {
 // Records a context-free error message for nerf_last_error(NULL).
 void set_global_error(const char* msg) { g_create_error = msg; }
 }  // namespace nerfb
+
+extern "C" nerf_status nerf_test_bounded_wait(uint32_t timeout_us, uint32_t* out_flag,
+                                              uint32_t* out_waited_us, void* stream) {
+  if (!out_flag || timeout_us < 1 || timeout_us > 2000000) {
+    nerfb::set_global_error("nerf_test_bounded_wait: bad argument");
+    return NERF_ERR_INVALID_ARG;
+  }
+  cudaError_t e = nerfb::launch_bounded_wait_probe(timeout_us, out_flag, out_waited_us,
+                                                   (cudaStream_t)stream);
+  return e == cudaSuccess ? NERF_OK : NERF_ERR_CUDA;
+}

@@ -41,6 +41,8 @@ constexpr int kMaxTimed = 4096;
 cudaError_t tc_alloc(nerf_ctx* ctx);
 void tc_free(nerf_ctx* ctx);
 cudaError_t tc_pack(nerf_ctx* ctx, const void* blob, cudaStream_t st);
+cudaError_t launch_bounded_wait_probe(uint32_t timeout_us, uint32_t* flag, uint32_t* waited_us,
+                                      cudaStream_t st);
 cudaError_t tc_run(nerf_ctx* ctx, const float* o, const float* d, int64_t R,
                    const SampleSpec& ss, float* raw, cudaStream_t st);
 }  // namespace nerfb
