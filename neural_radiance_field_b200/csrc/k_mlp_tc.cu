@@ -41,10 +41,6 @@ constexpr int NTHREADS = 64 + EPI_THREADS;
 constexpr int VEC_BYTES = 2 * 256 * 4;              // staged epilogue vectors
 constexpr size_t SMEM_BYTES = 2 * ACT_BYTES + NSTAGE * RING_BYTES + VEC_BYTES + 256;
 
-// per layer: K chunks, output width, first K-group of the A operand
-__constant__ int c_kchunks[NLAYER] = {2, 8, 8, 8, 8, 10, 8, 8, 8, 8};
-__constant__ int c_nout[NLAYER] = {256, 256, 256, 256, 256, 256, 256, 256, 256, 128};
-__constant__ int c_kgroup0[NLAYER] = {32, 0, 0, 0, 0, 0, 0, 0, 0, 0};
 
 // Packed weight stream (bf16 chunks in consumption order) and fp32 vectors.
 struct TcLayout {
@@ -360,6 +356,52 @@ __device__ __forceinline__ void store_pe(float x0, float x1, float x2, uint32_t 
   }
 }
 
+// The MMAs of one layer for both tiles of the pair, issued by one thread. The
+// tensor pipe finishes an M = 128, N = 256, K = 16 MMA in 128 cycles, and a
+// single thread's dependent integer work easily takes longer than that, so
+// everything that can be is a compile-time constant (shape, instruction
+// descriptor, descriptor strides) and the operand descriptors advance by adds.
+//   N: output width; KG0: first K-group of the A operand; NCH: K chunks
+template <int N, int KG0, int NCH>
+__device__ __forceinline__ bool mma_layer(uint32_t& q, uint32_t (&ph_act)[2], uint64_t* full,
+                                          uint64_t* empty, uint64_t* mma_done,
+                                          uint64_t* act_ready, uint64_t a_desc, uint64_t b_desc,
+                                          uint32_t tmem, const Ctl& ctl) {
+  if (!mbar_wait(&act_ready[0], ph_act[0], ctl) || !mbar_wait(&act_ready[1], ph_act[1], ctl))
+    return false;
+  ph_act[0] ^= 1;
+  ph_act[1] ^= 1;
+  tc_fence_after();
+  constexpr uint32_t idesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) |
+                             ((uint32_t)(TM >> 4) << 24);
+  // descriptor address steps (bytes >> 4)
+  constexpr uint64_t A_KSTEP = (2 * TM * 16) >> 4;        // K = 16: two K-groups
+  constexpr uint64_t A_CHUNK = (4 * TM * 16) >> 4;        // K = 32
+  constexpr uint64_t A_TILE = ACT_BYTES >> 4;
+  constexpr uint64_t B_KSTEP = (2 * N * 16) >> 4;
+  constexpr uint64_t B_SLOT = RING_BYTES >> 4;
+  // B descriptors of ring slot 0 carry this layer's K-group stride (N * 16 B)
+  const uint64_t b0 = (b_desc & ~(0x3FFFull << 16)) | ((uint64_t)((N * 16) >> 4) << 16);
+  const uint64_t a0 = a_desc + (uint64_t)((KG0 * TM * 16) >> 4);
+#pragma unroll 2
+  for (int c = 0; c < NCH; ++c, ++q) {
+    const uint32_t slot = q & (NSTAGE - 1);
+    if (!mbar_wait(&full[slot], (q / NSTAGE) & 1, ctl)) return false;
+    tc_fence_after();
+    const uint64_t b = b0 + slot * B_SLOT;
+    const uint64_t a = a0 + (uint64_t)c * A_CHUNK;
+    const uint32_t acc = c != 0;
+    mma_bf16(tmem, a, b, idesc, acc);
+    mma_bf16(tmem, a + A_KSTEP, b + B_KSTEP, idesc, 1);
+    mma_bf16(tmem + 256, a + A_TILE, b, idesc, acc);
+    mma_bf16(tmem + 256, a + A_TILE + A_KSTEP, b + B_KSTEP, idesc, 1);
+    mma_commit(&empty[slot]);
+  }
+  mma_commit(&mma_done[0]);
+  mma_commit(&mma_done[1]);
+  return true;
+}
+
 __global__ void __launch_bounds__(NTHREADS, 1) mlp_tc_kernel(Params P) {
   extern __shared__ __align__(1024) uint8_t smem[];
   uint8_t* act = smem;                                   // 2 x ACT_BYTES
@@ -405,37 +447,21 @@ __global__ void __launch_bounds__(NTHREADS, 1) mlp_tc_kernel(Params P) {
     if (lane == 0) {
       uint32_t q = 0, ph_act[2] = {0, 0};
       bool ok = true;
+      const uint64_t a_desc = sdesc(smem_u32(act), TM * 16, 128);
+      const uint64_t b_desc = sdesc(smem_u32(ring), 0, 128);
       for (int64_t pr = blockIdx.x; pr < P.n_pairs && ok; pr += gridDim.x) {
-        for (int l = 0; l < NLAYER && ok; ++l) {
-          ok = mbar_wait(&act_ready[0], ph_act[0], ctl) && mbar_wait(&act_ready[1], ph_act[1], ctl);
-          if (!ok) break;
-          ph_act[0] ^= 1; ph_act[1] ^= 1;
-          tc_fence_after();
-          const int N = c_nout[l];
-          const uint32_t idesc = idesc_bf16(N);
-          const int kg0 = c_kgroup0[l];
-          for (int c = 0; c < c_kchunks[l]; ++c, ++q) {
-            const int slot = q % NSTAGE;
-            if (!mbar_wait(&full[slot], (q / NSTAGE) & 1, ctl)) { ok = false; break; }
-            tc_fence_after();
-            const uint32_t bbase = smem_u32(ring + slot * RING_BYTES);
-#pragma unroll
-            for (int g = 0; g < 2; ++g) {
-              const uint32_t abase = smem_u32(act + g * ACT_BYTES);
-#pragma unroll
-              for (int kk = 0; kk < 2; ++kk) {
-                const int kg = kg0 + c * 4 + kk * 2;
-                uint64_t a = sdesc(abase + kg * (TM * 16), TM * 16, 128);
-                uint64_t b = sdesc(bbase + kk * 2 * (N * 16), N * 16, 128);
-                mma_bf16(tmem + g * 256, a, b, idesc, (c | kk) != 0);
-              }
-            }
-            mma_commit(&empty[slot]);
-          }
-          if (!ok) break;
-          mma_commit(&mma_done[0]);
-          mma_commit(&mma_done[1]);
-        }
+        // layer shapes: pts0 (K = 63 -> 64, from the gamma columns), pts1..4,
+        // pts5 (skip: K = 256 + 64), pts6, pts7, feature, direction (N = 128)
+        ok = mma_layer<256, 32, 2>(q, ph_act, full, empty, mma_done, act_ready, a_desc, b_desc, tmem, ctl) &&
+             mma_layer<256, 0, 8>(q, ph_act, full, empty, mma_done, act_ready, a_desc, b_desc, tmem, ctl) &&
+             mma_layer<256, 0, 8>(q, ph_act, full, empty, mma_done, act_ready, a_desc, b_desc, tmem, ctl) &&
+             mma_layer<256, 0, 8>(q, ph_act, full, empty, mma_done, act_ready, a_desc, b_desc, tmem, ctl) &&
+             mma_layer<256, 0, 8>(q, ph_act, full, empty, mma_done, act_ready, a_desc, b_desc, tmem, ctl) &&
+             mma_layer<256, 0, 10>(q, ph_act, full, empty, mma_done, act_ready, a_desc, b_desc, tmem, ctl) &&
+             mma_layer<256, 0, 8>(q, ph_act, full, empty, mma_done, act_ready, a_desc, b_desc, tmem, ctl) &&
+             mma_layer<256, 0, 8>(q, ph_act, full, empty, mma_done, act_ready, a_desc, b_desc, tmem, ctl) &&
+             mma_layer<256, 0, 8>(q, ph_act, full, empty, mma_done, act_ready, a_desc, b_desc, tmem, ctl) &&
+             mma_layer<128, 0, 8>(q, ph_act, full, empty, mma_done, act_ready, a_desc, b_desc, tmem, ctl);
       }
       // drain: everything issued so far completes before the CTA frees TMEM
       mma_commit(final_bar);
