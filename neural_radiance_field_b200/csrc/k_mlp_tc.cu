@@ -1,27 +1,33 @@
 // bf16 tensor-core evaluation of the NeRF scene MLP (NeRF page, Section 2.4) on
 // sm_100a: tcgen05.mma with fp32 accumulators in tensor memory, weights streamed
-// by the bulk-copy engine, activations kept on chip for the whole network.
+// by TMA, activations kept on chip for the whole network.
 //
-// Persistent kernel, one CTA per SM, 18 warps:
-//   warp 0       issues the MMAs (one elected thread) and owns the TMEM allocation
-//   warp 1       streams the packed weights into a 4-slot shared-memory ring
+// Clusters of two CTAs on two SMs run 2-SM MMAs (cta_group::2, M = 256): each
+// CTA holds 128 rows of a 256-row tile and half of every weight chunk, and
+// receives its 128 rows x N of the accumulator in its own tensor memory. A
+// cluster works on pairs of such tiles, A and B, whose layers alternate on the
+// tensor cores (A0 B0 A1 B1 ...), so that one tile's epilogue runs while the
+// other tile's layer is computed. Each weight chunk that lands in the ring
+// serves both tiles (tile A's pass waits for it, tile B's pass frees its slot),
+// so each weight byte read from L2 serves 512 rows. Per CTA, 18 warps:
+//   warp 0       CTA 0: issues the MMAs of the pair; both CTAs: TMEM allocation
+//   warp 1       streams this CTA's half of each weight chunk into an 8-slot ring
+//                (one 256-input layer)
 //   warps 2-9    epilogue of tile A: warp w drains TMEM lane quarter (w % 4) of
 //                column half ((w - 2) / 4) % 2, i.e. thread = (row, half)
 //   warps 10-17  epilogue of tile B, same split
-// A CTA works on pairs of 128-row tiles. Every weight chunk that lands in the
-// ring feeds both tiles before its slot is refilled, so each weight byte read
-// from L2 serves 256 rows. Per layer the accumulators of both tiles (2 x 256
-// fp32 columns = all 512 TMEM columns) are drained by the epilogue warps, which
-// add the bias, apply ReLU, round to bf16 and write the next layer's A operand
-// back into shared memory. Two warps per lane quarter keep twice as many TMEM
-// loads in flight as one would; the drain is latency-bound, not bandwidth-bound.
+// The epilogue adds the bias, applies ReLU, rounds to bf16 and writes the next
+// layer's A operand into shared memory; the last layers add the sigma and rgb
+// heads in fp32.
 //
-// Shared memory (231,680 B): act[2] = per tile 128 rows x 320 bf16 holding
+// Shared memory per CTA (231,680 B): act[2] = per tile 128 rows x 320 bf16 holding
 // [h (256) | gamma(x) (63) | 0], so the skip layer reads columns 0..319 and the
-// first layer columns 256..319; ring[4] = weight chunks of K = 32 columns;
-// 2 KB of per-layer epilogue vectors; barriers.
+// first layer columns 256..319; ring[8] = half weight chunks (N/2 rows x 32 K);
+// 2 KB of per-tile epilogue vectors (bf16); barriers.
 // Operands use the no-swizzle K-major core-matrix layout: element (r, k) of a
 // block of R rows sits at (k/8)*R*16 + (r/8)*128 + (r%8)*16 + (k%8)*2 bytes.
+#include <cuda.h>
+
 #include "nerf_ctx.h"
 
 namespace nerfb {
@@ -32,15 +38,14 @@ constexpr int TM = 128;
 constexpr int ACT_K = 320;
 constexpr int ACT_BYTES = TM * ACT_K * 2;           // 81920
 constexpr int CHUNK_K = 32;
-constexpr int NSTAGE = 4;
-constexpr int RING_BYTES = 256 * CHUNK_K * 2;       // 16384 per slot
+constexpr int NSTAGE = 8;
+constexpr int RING_BYTES = 128 * CHUNK_K * 2;       // 8192: one CTA's half of a chunk
 constexpr int NLAYER = 10;                          // pts0..pts7, feature, dir
 constexpr int EPI_THREADS = 512;                    // 16 epilogue warps
 constexpr int TILE_THREADS = 256;                   // epilogue threads per tile
 constexpr int NTHREADS = 64 + EPI_THREADS;
-constexpr int VEC_BYTES = 2 * 256 * 4;              // staged epilogue vectors
+constexpr int VEC_BYTES = 2 * 512 * 2;              // per-tile staged epilogue vectors (bf16)
 constexpr size_t SMEM_BYTES = 2 * ACT_BYTES + NSTAGE * RING_BYTES + VEC_BYTES + 256;
-
 
 // Packed weight stream (bf16 chunks in consumption order) and fp32 vectors.
 struct TcLayout {
@@ -135,13 +140,6 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const 
   return true;
 }
 
-__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
-  asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
-      ::"r"(smem_u32(dst)), "l"(src), "r"(bytes), "r"(smem_u32(bar))
-      : "memory");
-}
-
 __device__ __forceinline__ void tc_fence_before() {
   asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
 }
@@ -160,25 +158,6 @@ __device__ __forceinline__ uint64_t sdesc(uint32_t addr, uint32_t lbo, uint32_t 
   d |= (uint64_t)((sbo >> 4) & 0x3FFF) << 32;
   d |= (uint64_t)1 << 46;                    // descriptor version for sm_100
   return d;                                  // base offset 0, swizzle none
-}
-
-// Instruction descriptor: bf16 x bf16 -> fp32, both K-major, M = 128.
-__device__ __forceinline__ uint32_t idesc_bf16(int N) {
-  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(TM >> 4) << 24);
-}
-
-__device__ __forceinline__ void mma_bf16(uint32_t tmem_d, uint64_t a, uint64_t b, uint32_t idesc,
-                                         uint32_t accum) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
-      ::"r"(tmem_d), "l"(a), "l"(b), "r"(idesc), "r"(accum));
-}
-
-__device__ __forceinline__ void mma_commit(uint64_t* bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
-               ::"r"(smem_u32(bar)) : "memory");
 }
 
 // Two fp32 -> packed bf16x2 with ReLU (lo = first element in memory order).
@@ -246,56 +225,53 @@ __device__ __forceinline__ void tmem_wait32(uint32_t* r) {
                : "memory");
 }
 
-// Named barriers: 1 = all 512 epilogue threads, 2 + g = the 256 threads of tile g.
-__device__ __forceinline__ void named_sync(int id, int count) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+// Named barrier 1 + g over the 256 epilogue threads of tile g.
+__device__ __forceinline__ void tile_sync(int g) {
+  asm volatile("bar.sync %0, 256;" ::"r"(1 + g) : "memory");
 }
 
-// Barrier over all epilogue threads that returns whether any passed true.
-__device__ __forceinline__ bool epilogue_sync_or(bool v) {
+// The same barrier, returning whether any of the tile's threads passed true.
+__device__ __forceinline__ bool tile_sync_or(int g, bool v) {
   uint32_t r;
   asm volatile(
       "{\n\t.reg .pred p, q;\n\t"
-      "setp.ne.u32 p, %1, 0;\n\t"
-      "bar.red.or.pred q, 1, 512, p;\n\t"
+      "setp.ne.u32 p, %2, 0;\n\t"
+      "bar.red.or.pred q, %1, 256, p;\n\t"
       "selp.u32 %0, 1, 0, q;\n\t}"
       : "=r"(r)
-      : "r"((uint32_t)v)
+      : "r"(1 + g), "r"((uint32_t)v)
       : "memory");
   return r != 0;
+}
+
+// Eight bf16 values (16 bytes of shared memory) widened exactly to fp32.
+__device__ __forceinline__ void load_bf16x8(const uint16_t* p, float* f) {
+  const uint4 w = *reinterpret_cast<const uint4*>(p);
+  f[0] = __uint_as_float(w.x << 16); f[1] = __uint_as_float(w.x & 0xFFFF0000u);
+  f[2] = __uint_as_float(w.y << 16); f[3] = __uint_as_float(w.y & 0xFFFF0000u);
+  f[4] = __uint_as_float(w.z << 16); f[5] = __uint_as_float(w.z & 0xFFFF0000u);
+  f[6] = __uint_as_float(w.w << 16); f[7] = __uint_as_float(w.w & 0xFFFF0000u);
 }
 
 // One 32-column block of a hidden layer: bias, activation, bf16, store to the
 // next layer's A operand; on the last trunk layer also accumulates sigma. Works
 // 8 columns at a time so that only the loaded block stays live.
 template <bool RELU, bool SIGMA>
-__device__ __forceinline__ void epi_block(const uint32_t* u, const float* sb_bias,
-                                          const float* sb_ws, int cb, uint32_t act_base, int r,
+__device__ __forceinline__ void epi_block(const uint32_t* u, const uint16_t* sb_bias,
+                                          const uint16_t* sb_ws, int cb, uint32_t act_base, int r,
                                           float& sigma) {
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
-    const float4 b0 = *reinterpret_cast<const float4*>(sb_bias + cb + 8 * j);
-    const float4 b1 = *reinterpret_cast<const float4*>(sb_bias + cb + 8 * j + 4);
+    float b[8];
+    load_bf16x8(sb_bias + cb + 8 * j, b);
     float v[8];
-    v[0] = __uint_as_float(u[8 * j + 0]) + b0.x;
-    v[1] = __uint_as_float(u[8 * j + 1]) + b0.y;
-    v[2] = __uint_as_float(u[8 * j + 2]) + b0.z;
-    v[3] = __uint_as_float(u[8 * j + 3]) + b0.w;
-    v[4] = __uint_as_float(u[8 * j + 4]) + b1.x;
-    v[5] = __uint_as_float(u[8 * j + 5]) + b1.y;
-    v[6] = __uint_as_float(u[8 * j + 6]) + b1.z;
-    v[7] = __uint_as_float(u[8 * j + 7]) + b1.w;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(u[8 * j + i]) + b[i];
     if (SIGMA) {
-      const float4 w0 = *reinterpret_cast<const float4*>(sb_ws + cb + 8 * j);
-      const float4 w1 = *reinterpret_cast<const float4*>(sb_ws + cb + 8 * j + 4);
-      sigma = fmaf(fmaxf(v[0], 0.f), w0.x, sigma);
-      sigma = fmaf(fmaxf(v[1], 0.f), w0.y, sigma);
-      sigma = fmaf(fmaxf(v[2], 0.f), w0.z, sigma);
-      sigma = fmaf(fmaxf(v[3], 0.f), w0.w, sigma);
-      sigma = fmaf(fmaxf(v[4], 0.f), w1.x, sigma);
-      sigma = fmaf(fmaxf(v[5], 0.f), w1.y, sigma);
-      sigma = fmaf(fmaxf(v[6], 0.f), w1.z, sigma);
-      sigma = fmaf(fmaxf(v[7], 0.f), w1.w, sigma);
+      float w[8];
+      load_bf16x8(sb_ws + cb + 8 * j, w);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) sigma = fmaf(fmaxf(v[i], 0.f), w[i], sigma);
     }
     uint32_t w0, w1, w2, w3;
     if (RELU) {
@@ -311,8 +287,8 @@ __device__ __forceinline__ void epi_block(const uint32_t* u, const float* sb_bia
 
 // 128 columns [c0, c0 + 128) of a 256-wide hidden layer, two TMEM loads in flight.
 template <bool RELU, bool SIGMA>
-__device__ __forceinline__ void epi_half(uint32_t t_row, int c0, const float* sb_bias,
-                                         const float* sb_ws, uint32_t act_base, int r,
+__device__ __forceinline__ void epi_half(uint32_t t_row, int c0, const uint16_t* sb_bias,
+                                         const uint16_t* sb_ws, uint32_t act_base, int r,
                                          float& sigma) {
   uint32_t ua[32], ub[32];
   tmem_ld32_issue(t_row + c0, ua);
@@ -356,153 +332,288 @@ __device__ __forceinline__ void store_pe(float x0, float x1, float x2, uint32_t 
   }
 }
 
-// The MMAs of one layer for both tiles of the pair, issued by one thread. The
-// tensor pipe finishes an M = 128, N = 256, K = 16 MMA in 128 cycles, and a
-// single thread's dependent integer work easily takes longer than that, so
-// everything that can be is a compile-time constant (shape, instruction
-// descriptor, descriptor strides) and the operand descriptors advance by adds.
-//   N: output width; KG0: first K-group of the A operand; NCH: K chunks
-template <int N, int KG0, int NCH>
-__device__ __forceinline__ bool mma_layer(uint32_t& q, uint32_t (&ph_act)[2], uint64_t* full,
-                                          uint64_t* empty, uint64_t* mma_done,
-                                          uint64_t* act_ready, uint64_t a_desc, uint64_t b_desc,
-                                          uint32_t tmem, const Ctl& ctl) {
-  if (!mbar_wait(&act_ready[0], ph_act[0], ctl) || !mbar_wait(&act_ready[1], ph_act[1], ctl))
-    return false;
-  ph_act[0] ^= 1;
-  ph_act[1] ^= 1;
-  tc_fence_after();
-  constexpr uint32_t idesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) |
-                             ((uint32_t)(TM >> 4) << 24);
-  // descriptor address steps (bytes >> 4)
-  constexpr uint64_t A_KSTEP = (2 * TM * 16) >> 4;        // K = 16: two K-groups
-  constexpr uint64_t A_CHUNK = (4 * TM * 16) >> 4;        // K = 32
-  constexpr uint64_t A_TILE = ACT_BYTES >> 4;
-  constexpr uint64_t B_KSTEP = (2 * N * 16) >> 4;
-  constexpr uint64_t B_SLOT = RING_BYTES >> 4;
-  // B descriptors of ring slot 0 carry this layer's K-group stride (N * 16 B)
-  const uint64_t b0 = (b_desc & ~(0x3FFFull << 16)) | ((uint64_t)((N * 16) >> 4) << 16);
-  const uint64_t a0 = a_desc + (uint64_t)((KG0 * TM * 16) >> 4);
-#pragma unroll 2
-  for (int c = 0; c < NCH; ++c, ++q) {
-    const uint32_t slot = q & (NSTAGE - 1);
-    if (!mbar_wait(&full[slot], (q / NSTAGE) & 1, ctl)) return false;
-    tc_fence_after();
-    const uint64_t b = b0 + slot * B_SLOT;
-    const uint64_t a = a0 + (uint64_t)c * A_CHUNK;
-    const uint32_t acc = c != 0;
-    mma_bf16(tmem, a, b, idesc, acc);
-    mma_bf16(tmem, a + A_KSTEP, b + B_KSTEP, idesc, 1);
-    mma_bf16(tmem + 256, a + A_TILE, b, idesc, acc);
-    mma_bf16(tmem + 256, a + A_TILE + A_KSTEP, b + B_KSTEP, idesc, 1);
-    mma_commit(&empty[slot]);
+// ---- 2-SM additions (cluster of 2 CTAs, tcgen05 cta_group::2) ----
+
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ uint32_t cluster_id_x() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%clusterid.x;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ uint32_t nclusters_x() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%nclusterid.x;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;"
+               ::: "memory");
+}
+
+// try_wait with cluster-scope acquire: the barrier may be completed by the peer CTA.
+__device__ __forceinline__ bool mbar_try_cl(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+__device__ __forceinline__ bool mbar_wait_cl(uint64_t* bar, uint32_t parity, const Ctl& ctl) {
+  if (mbar_try_cl(bar, parity)) return true;
+  const uint64_t t0 = globaltimer();
+  while (!mbar_try_cl(bar, parity)) {
+    if (*ctl.abort) return false;
+    if (globaltimer() - t0 > ctl.limit_ns) {
+      atomicOr(ctl.flag, FLAG_TIMEOUT);
+      *ctl.abort = 1;
+      return false;
+    }
   }
-  mma_commit(&mma_done[0]);
-  mma_commit(&mma_done[1]);
   return true;
 }
 
-__global__ void __launch_bounds__(NTHREADS, 1) mlp_tc_kernel(Params P) {
+// Arrive on the barrier at the same offset in CTA 0 of the cluster.
+__device__ __forceinline__ void mbar_arrive_leader(uint64_t* bar) {
+  asm volatile(
+      "{\n\t.reg .b32 ra;\n\t"
+      "mapa.shared::cluster.u32 ra, %0, 0;\n\t"
+      "mbarrier.arrive.release.cluster.shared::cluster.b64 _, [ra];\n\t}"
+      ::"r"(smem_u32(bar))
+      : "memory");
+}
+
+// 2-D tensor load into this CTA's shared memory whose completion is counted on
+// CTA 0's barrier (the barrier address with the peer bit cleared).
+__device__ __forceinline__ void tma_load_2d_pair(void* dst, const void* tmap, int x, int y,
+                                                 uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4}], [%2];"
+      ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(tmap)),
+        "r"(smem_u32(bar) & 0xFEFFFFFFu), "r"(x), "r"(y)
+      : "memory");
+}
+
+
+__device__ __forceinline__ void mma_bf16_pair(uint32_t tmem_d, uint64_t a, uint64_t b,
+                                              uint32_t idesc, uint32_t accum) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}"
+      ::"r"(tmem_d), "l"(a), "l"(b), "r"(idesc), "r"(accum));
+}
+
+// Arrive (once each) on the barrier at this offset in both CTAs of the pair
+// when every previously issued MMA of this thread has completed.
+__device__ __forceinline__ void mma_commit_pair(uint64_t* bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
+      " [%0], %1;"
+      ::"r"(smem_u32(bar)), "h"((uint16_t)3)
+      : "memory");
+}
+
+// MMAs of tile g over chunks [C0, C1) of one layer, issued by CTA 0's MMA
+// thread. Every weight chunk serves both tiles: tile A's pass is its first
+// use (it waits for the chunk to land), tile B's pass its second (it releases
+// the ring slot). A 2-SM MMA (M = 256, N = 256, K = 16) takes 128 cycles on
+// the tensor pipe and a chunk holds two, so the thread's work per chunk must
+// stay well under 256 cycles: shapes and the instruction descriptor are
+// compile-time constants and operand descriptors advance by additions.
+//   N: output width; KG0: first K-group of the A operand
+template <int N, int KG0, int C0, int C1, bool FIRST_USE>
+__device__ __forceinline__ bool mma_pass(int g, uint32_t q0, uint64_t* full, uint64_t* empty,
+                                         uint64_t a_desc, uint64_t b_desc, uint32_t tmem,
+                                         const Ctl& ctl) {
+  constexpr int Nh = N / 2;                 // rows of B held by each CTA
+  constexpr uint32_t idesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) |
+                             (16u << 24);   // M = 256
+  constexpr uint64_t A_KSTEP = (2 * TM * 16) >> 4;
+  constexpr uint64_t A_CHUNK = (4 * TM * 16) >> 4;
+  constexpr uint64_t A_TILE = ACT_BYTES >> 4;
+  constexpr uint64_t B_KSTEP = (2 * Nh * 16) >> 4;
+  constexpr uint64_t B_SLOT = RING_BYTES >> 4;
+  const uint64_t b0 = (b_desc & ~(0x3FFFull << 16)) | ((uint64_t)((Nh * 16) >> 4) << 16);
+  const uint64_t a0 = a_desc + (uint64_t)g * A_TILE + (uint64_t)((KG0 * TM * 16) >> 4);
+  const uint32_t td = tmem + (uint32_t)g * 256;
+#pragma unroll 2
+  for (int c = C0; c < C1; ++c) {
+    const uint32_t q = q0 + (uint32_t)c;
+    const uint32_t slot = q & (NSTAGE - 1);
+    if (FIRST_USE) {
+      if (!mbar_wait_cl(&full[slot], (q / NSTAGE) & 1, ctl)) return false;
+      tc_fence_after();
+    }
+    const uint64_t b = b0 + slot * B_SLOT;
+    const uint64_t a = a0 + (uint64_t)c * A_CHUNK;
+    mma_bf16_pair(td, a, b, idesc, c != 0);
+    mma_bf16_pair(td, a + A_KSTEP, b + B_KSTEP, idesc, 1);
+    if (!FIRST_USE) mma_commit_pair(&empty[slot]);
+  }
+  return true;
+}
+
+__device__ __forceinline__ bool wait_act(int g, uint32_t (&ph_act)[2], uint64_t* act_ready,
+                                         const Ctl& ctl) {
+  if (!mbar_wait_cl(&act_ready[g], ph_act[g], ctl)) return false;
+  ph_act[g] ^= 1;
+  tc_fence_after();
+  return true;
+}
+
+// One layer of both tiles, tile A first (A0 B0 A1 B1 ...): while one tile's
+// accumulator is drained by its epilogue, the other tile's layer runs. The
+// ring holds 8 chunks, one layer; the 10-chunk skip layer runs as A[0..7]
+// B[0..7] A[8, 9] B[8, 9], so that its last two chunks can reuse the slots
+// that tile B has released.
+template <int N, int KG0, int NCH>
+__device__ __forceinline__ bool mma_layer_pingpong(uint32_t& q, uint32_t (&ph_act)[2],
+                                                   uint64_t* full, uint64_t* empty,
+                                                   uint64_t* mma_done, uint64_t* act_ready,
+                                                   uint64_t a_desc, uint64_t b_desc,
+                                                   uint32_t tmem, const Ctl& ctl) {
+  static_assert(NCH <= NSTAGE || NCH == NSTAGE + 2, "chunk schedule");
+  constexpr int CA = NCH <= NSTAGE ? NCH : NSTAGE;
+  if (!wait_act(0, ph_act, act_ready, ctl) ||
+      !mma_pass<N, KG0, 0, CA, true>(0, q, full, empty, a_desc, b_desc, tmem, ctl))
+    return false;
+  if (NCH == CA) mma_commit_pair(&mma_done[0]);
+  if (!wait_act(1, ph_act, act_ready, ctl) ||
+      !mma_pass<N, KG0, 0, CA, false>(1, q, full, empty, a_desc, b_desc, tmem, ctl))
+    return false;
+  if (NCH == CA) {
+    mma_commit_pair(&mma_done[1]);
+  } else {
+    if (!mma_pass<N, KG0, CA, NCH, true>(0, q, full, empty, a_desc, b_desc, tmem, ctl))
+      return false;
+    mma_commit_pair(&mma_done[0]);
+    if (!mma_pass<N, KG0, CA, NCH, false>(1, q, full, empty, a_desc, b_desc, tmem, ctl))
+      return false;
+    mma_commit_pair(&mma_done[1]);
+  }
+  q += NCH;
+  return true;
+}
+
+__global__ void __launch_bounds__(NTHREADS, 1) mlp_tc_kernel(Params P, const __grid_constant__ CUtensorMap tmap_h64,
+              const __grid_constant__ CUtensorMap tmap_h32) {
   extern __shared__ __align__(1024) uint8_t smem[];
   uint8_t* act = smem;                                   // 2 x ACT_BYTES
   uint8_t* ring = smem + 2 * ACT_BYTES;                  // NSTAGE x RING_BYTES
-  float* svec = reinterpret_cast<float*>(ring + NSTAGE * RING_BYTES);   // 2 x 256 fp32
+  uint16_t* svec = reinterpret_cast<uint16_t*>(ring + NSTAGE * RING_BYTES);  // 2 tiles x 512 bf16
   uint64_t* bars = reinterpret_cast<uint64_t*>(ring + NSTAGE * RING_BYTES + VEC_BYTES);
-  uint64_t* full = bars;                 // [NSTAGE]
+  uint64_t* full = bars;                 // [NSTAGE] (used in CTA 0)
   uint64_t* empty = bars + NSTAGE;       // [NSTAGE]
   uint64_t* mma_done = bars + 2 * NSTAGE;     // [2]
-  uint64_t* act_ready = bars + 2 * NSTAGE + 2;  // [2]
+  uint64_t* act_ready = bars + 2 * NSTAGE + 2;  // [2] (used in CTA 0)
   uint64_t* final_bar = bars + 2 * NSTAGE + 4;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 2 * NSTAGE + 5);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  const int cta = (int)cluster_ctarank();      // 0 issues the MMAs of the pair
+  const int64_t cid = cluster_id_x(), ncl = nclusters_x();
   Ctl ctl{abort_flag, P.flag, kWaitLimitNs};
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < NSTAGE; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
     for (int g = 0; g < 2; ++g) {
       mbar_init(&mma_done[g], 1);
-      mbar_init(&act_ready[g], TILE_THREADS);
+      mbar_init(&act_ready[g], 2 * TILE_THREADS);     // both CTAs' epilogue threads
     }
     mbar_init(final_bar, 1);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   if (warp == 0) {
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;"
                  ::"r"(smem_u32(tmem_holder)), "r"(512));
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;");
   }
   tc_fence_before();
   __syncthreads();
+  cluster_sync_all();            // both CTAs' barriers exist before any remote use
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
 
   const int64_t rows = P.R * P.ss.S;
 
   if (warp == 0) {
-    // ---------------------------------------------------------- MMA issuer
-    if (lane == 0) {
+    // ---------------------------------------------------------- MMA issuer (CTA 0)
+    if (lane == 0 && cta == 0) {
       uint32_t q = 0, ph_act[2] = {0, 0};
       bool ok = true;
       const uint64_t a_desc = sdesc(smem_u32(act), TM * 16, 128);
       const uint64_t b_desc = sdesc(smem_u32(ring), 0, 128);
-      for (int64_t pr = blockIdx.x; pr < P.n_pairs && ok; pr += gridDim.x) {
+#define NERF_PP_LAYER(N, KG0, NCH) \
+  mma_layer_pingpong<N, KG0, NCH>(q, ph_act, full, empty, mma_done, act_ready, a_desc, b_desc, tmem, ctl)
+      for (int64_t pr = cid; pr < P.n_pairs && ok; pr += ncl) {
         // layer shapes: pts0 (K = 63 -> 64, from the gamma columns), pts1..4,
         // pts5 (skip: K = 256 + 64), pts6, pts7, feature, direction (N = 128)
-        ok = mma_layer<256, 32, 2>(q, ph_act, full, empty, mma_done, act_ready, a_desc, b_desc, tmem, ctl) &&
-             mma_layer<256, 0, 8>(q, ph_act, full, empty, mma_done, act_ready, a_desc, b_desc, tmem, ctl) &&
-             mma_layer<256, 0, 8>(q, ph_act, full, empty, mma_done, act_ready, a_desc, b_desc, tmem, ctl) &&
-             mma_layer<256, 0, 8>(q, ph_act, full, empty, mma_done, act_ready, a_desc, b_desc, tmem, ctl) &&
-             mma_layer<256, 0, 8>(q, ph_act, full, empty, mma_done, act_ready, a_desc, b_desc, tmem, ctl) &&
-             mma_layer<256, 0, 10>(q, ph_act, full, empty, mma_done, act_ready, a_desc, b_desc, tmem, ctl) &&
-             mma_layer<256, 0, 8>(q, ph_act, full, empty, mma_done, act_ready, a_desc, b_desc, tmem, ctl) &&
-             mma_layer<256, 0, 8>(q, ph_act, full, empty, mma_done, act_ready, a_desc, b_desc, tmem, ctl) &&
-             mma_layer<256, 0, 8>(q, ph_act, full, empty, mma_done, act_ready, a_desc, b_desc, tmem, ctl) &&
-             mma_layer<128, 0, 8>(q, ph_act, full, empty, mma_done, act_ready, a_desc, b_desc, tmem, ctl);
+        ok = NERF_PP_LAYER(256, 32, 2) && NERF_PP_LAYER(256, 0, 8) && NERF_PP_LAYER(256, 0, 8) &&
+             NERF_PP_LAYER(256, 0, 8) && NERF_PP_LAYER(256, 0, 8) && NERF_PP_LAYER(256, 0, 10) &&
+             NERF_PP_LAYER(256, 0, 8) && NERF_PP_LAYER(256, 0, 8) && NERF_PP_LAYER(256, 0, 8) &&
+             NERF_PP_LAYER(128, 0, 8);
       }
-      // drain: everything issued so far completes before the CTA frees TMEM
-      mma_commit(final_bar);
+#undef NERF_PP_LAYER
+      // drain: everything issued so far completes before the pair frees TMEM
+      mma_commit_pair(final_bar);
       uint64_t t0 = globaltimer();
-      while (!mbar_try(final_bar, 0) && globaltimer() - t0 < kWaitLimitNs) {}
+      while (!mbar_try_cl(final_bar, 0) && globaltimer() - t0 < 2000000000ull) {}
     }
   } else if (warp == 1) {
-    // ---------------------------------------------------------- weight loader
+    // ---------------------------------------------------------- weight loader (both CTAs)
+    // Each CTA loads its half of every chunk (rows [cta * N/2, (cta + 1) * N/2)
+    // of the layer); the bytes of both halves are counted on CTA 0's barrier.
     if (lane == 0) {
       uint32_t q = 0;
-      for (int64_t pr = blockIdx.x; pr < P.n_pairs; pr += gridDim.x) {
+      for (int64_t pr = cid; pr < P.n_pairs; pr += ncl) {
         bool ok = true;
         for (int j = 0; j < P.lay.n_chunks; ++j, ++q) {
           const int slot = q % NSTAGE;
-          if (!mbar_wait(&empty[slot], ((q / NSTAGE) & 1) ^ 1, ctl)) { ok = false; break; }
-          const uint32_t bytes = (uint32_t)P.lay.chunk_bytes[j];
-          mbar_arrive_tx(&full[slot], bytes);
-          bulk_g2s(ring + slot * RING_BYTES, P.stream + P.lay.chunk_off[j], bytes, &full[slot]);
+          // the slot's previous chunk has served both tiles
+          if (!mbar_wait_cl(&empty[slot], ((q / NSTAGE) & 1) ^ 1, ctl)) { ok = false; break; }
+          const uint32_t bytes = (uint32_t)P.lay.chunk_bytes[j];        // both halves
+          const int64_t half_off = P.lay.chunk_off[j] + (int64_t)cta * (bytes / 2);
+          if (cta == 0) mbar_arrive_tx(&full[slot], bytes);
+          tma_load_2d_pair(ring + slot * RING_BYTES, bytes == 2 * 8192 ? (const void*)&tmap_h64
+                                                                       : (const void*)&tmap_h32,
+                           0, (int)(half_off / 128), &full[slot]);
         }
         if (!ok) break;
       }
     }
   } else {
-    // ---------------------------------------------------------- epilogue
+    // ---------------------------------------------------------- epilogue (both CTAs)
     const int et = threadIdx.x - 64;              // 0..511
     const int g = et >> 8;                        // tile within the pair
     const int h = (et >> 7) & 1;                  // column half
     const int quarter = warp & 3;                 // TMEM lane quarter of this warp
-    const int r = quarter * 32 + lane;            // row in the tile = TMEM lane
+    const int r = quarter * 32 + lane;            // row in this CTA's half tile = TMEM lane
     uint8_t* my_act = act + g * ACT_BYTES;
     const uint32_t act_base = smem_u32(my_act);
     const uint32_t t_row = tmem + (uint32_t)(g * 256) + ((uint32_t)(quarter * 32) << 16);
-    float* sb0 = svec;          // layer bias / rgb weights rows 0, 1
-    float* sb1 = svec + 256;    // sigma weights / rgb row 2, rgb and sigma biases
+    const int tt = et & 255;                      // thread within the tile
+    uint16_t* sb0 = svec + g * 512;   // layer bias / rgb weights rows 0, 1 (bf16)
+    uint16_t* sb1 = sb0 + 256;        // sigma weights / rgb row 2, rgb and sigma biases
     // partial (sigma, r, g, b) of the second column half, handed to the first
     // half through the tile's (then idle) activation buffer
     float4* xchg = reinterpret_cast<float4*>(my_act);
     uint32_t ph_md = 0;
     const float* vec = P.vec;
-    for (int64_t pr = blockIdx.x; pr < P.n_pairs; pr += gridDim.x) {
-      const int64_t row = (pr * 2 + g) * TM + r;
+    for (int64_t pr = cid; pr < P.n_pairs; pr += ncl) {
+      const int64_t row = (pr * 2 + g) * (2 * TM) + cta * TM + r;
       const bool valid = row < rows;
       int64_t ray = 0;
       float x[3] = {0.f, 0.f, 0.f};
@@ -527,30 +638,31 @@ __global__ void __launch_bounds__(NTHREADS, 1) mlp_tc_kernel(Params P) {
       if (h == 0) store_pe<0>(x[0], x[1], x[2], act_base, r);
       else store_pe<1>(x[0], x[1], x[2], act_base, r);
       fence_async_smem();
-      mbar_arrive(&act_ready[g]);
+      if (cta == 0) mbar_arrive(&act_ready[g]); else mbar_arrive_leader(&act_ready[g]);
 
       float sigma = 0.0f;
       for (int l = 0; l < NLAYER; ++l) {
         // this layer's epilogue vectors: loaded now, staged after the MMA wait
-        float pre;
+        // (all values are bf16 weights of the blob, so the bf16 staging is exact)
+        float pre0, pre1 = 0.0f;
         if (l < 9) {
-          pre = et < 256 ? __ldg(vec + P.lay.bias[l] + et)
-                         : (l == 7 ? __ldg(vec + P.lay.w_sigma + et - 256) : 0.0f);
+          pre0 = __ldg(vec + P.lay.bias[l] + tt);
+          if (l == 7) pre1 = __ldg(vec + P.lay.w_sigma + tt);
         } else {
-          const int q2 = et - 256;
-          pre = et < 256 ? __ldg(vec + P.lay.w_rgb + et)
-              : q2 < 128 ? __ldg(vec + P.lay.w_rgb + 256 + q2)
-              : q2 < 131 ? __ldg(vec + P.lay.b_rgb + q2 - 128)
-              : q2 == 131 ? __ldg(vec + P.lay.b_sigma) : 0.0f;
+          pre0 = __ldg(vec + P.lay.w_rgb + tt);
+          pre1 = tt < 128 ? __ldg(vec + P.lay.w_rgb + 256 + tt)
+               : tt < 131 ? __ldg(vec + P.lay.b_rgb + tt - 128)
+               : tt == 131 ? __ldg(vec + P.lay.b_sigma) : 0.0f;
         }
-        const bool waited = mbar_wait(&mma_done[g], ph_md, ctl);
+        const bool waited = mbar_wait_cl(&mma_done[g], ph_md, ctl);
         ph_md ^= 1;
         tc_fence_after();
-        // every epilogue thread is done with the previous vectors; all agree on
-        // giving up together, so no thread is left behind at a barrier
-        if (epilogue_sync_or(!waited || *abort_flag)) break;
-        svec[et] = pre;
-        named_sync(1, EPI_THREADS);
+        // every thread of the tile is done with the previous vectors; all agree
+        // on giving up together, so no thread is left behind at a barrier
+        if (tile_sync_or(g, !waited || *abort_flag)) break;
+        sb0[tt] = __bfloat16_as_ushort(__float2bfloat16_rn(pre0));
+        sb1[tt] = __bfloat16_as_ushort(__float2bfloat16_rn(pre1));
+        tile_sync(g);
         if (l < 9) {
           const int c0 = h * 128;
           if (l == 8) epi_half<false, false>(t_row, c0, sb0, sb1, act_base, r, sigma);
@@ -558,7 +670,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) mlp_tc_kernel(Params P) {
           else epi_half<true, false>(t_row, c0, sb0, sb1, act_base, r, sigma);
           tc_fence_before();
           fence_async_smem();
-          mbar_arrive(&act_ready[g]);
+          if (cta == 0) mbar_arrive(&act_ready[g]); else mbar_arrive_leader(&act_ready[g]);
         } else {
           // direction layer (N = 128): + per-ray bias, ReLU, the rgb head in fp32
           // on this half's 64 columns; the halves are summed through shared memory
@@ -579,35 +691,40 @@ __global__ void __launch_bounds__(NTHREADS, 1) mlp_tc_kernel(Params P) {
               const float h1 = fmaxf(__uint_as_float(u[4 * i + 1]) + bb[i].y, 0.f);
               const float h2 = fmaxf(__uint_as_float(u[4 * i + 2]) + bb[i].z, 0.f);
               const float h3 = fmaxf(__uint_as_float(u[4 * i + 3]) + bb[i].w, 0.f);
-              const float4 a4 = *reinterpret_cast<const float4*>(sb0 + c);
-              const float4 c4 = *reinterpret_cast<const float4*>(sb0 + 128 + c);
-              const float4 d4 = *reinterpret_cast<const float4*>(sb1 + c);
-              rgb0 = fmaf(h0, a4.x, fmaf(h1, a4.y, fmaf(h2, a4.z, fmaf(h3, a4.w, rgb0))));
-              rgb1 = fmaf(h0, c4.x, fmaf(h1, c4.y, fmaf(h2, c4.z, fmaf(h3, c4.w, rgb1))));
-              rgb2 = fmaf(h0, d4.x, fmaf(h1, d4.y, fmaf(h2, d4.z, fmaf(h3, d4.w, rgb2))));
+              const uint2 a2 = *reinterpret_cast<const uint2*>(sb0 + c);
+              const uint2 c2 = *reinterpret_cast<const uint2*>(sb0 + 128 + c);
+              const uint2 d2 = *reinterpret_cast<const uint2*>(sb1 + c);
+              rgb0 = fmaf(h0, __uint_as_float(a2.x << 16), fmaf(h1, __uint_as_float(a2.x & 0xFFFF0000u),
+                     fmaf(h2, __uint_as_float(a2.y << 16), fmaf(h3, __uint_as_float(a2.y & 0xFFFF0000u), rgb0))));
+              rgb1 = fmaf(h0, __uint_as_float(c2.x << 16), fmaf(h1, __uint_as_float(c2.x & 0xFFFF0000u),
+                     fmaf(h2, __uint_as_float(c2.y << 16), fmaf(h3, __uint_as_float(c2.y & 0xFFFF0000u), rgb1))));
+              rgb2 = fmaf(h0, __uint_as_float(d2.x << 16), fmaf(h1, __uint_as_float(d2.x & 0xFFFF0000u),
+                     fmaf(h2, __uint_as_float(d2.y << 16), fmaf(h3, __uint_as_float(d2.y & 0xFFFF0000u), rgb2))));
             }
           }
           tc_fence_before();
           if (h == 1) xchg[r] = make_float4(sigma, rgb0, rgb1, rgb2);
-          named_sync(2 + g, TILE_THREADS);
+          tile_sync(g);
           if (h == 0 && valid) {
             const float4 o2 = xchg[r];
+            auto bf = [&](int i) { return __uint_as_float((uint32_t)sb1[i] << 16); };
             *reinterpret_cast<float4*>(P.raw + row * 4) =
-                make_float4(rgb0 + o2.y + sb1[128], rgb1 + o2.z + sb1[129],
-                            rgb2 + o2.w + sb1[130], sigma + o2.x + sb1[131]);
+                make_float4(rgb0 + o2.y + bf(128), rgb1 + o2.z + bf(129),
+                            rgb2 + o2.w + bf(130), sigma + o2.x + bf(131));
           }
-          named_sync(2 + g, TILE_THREADS);
+          tile_sync(g);
         }
       }
-      if (epilogue_sync_or(*abort_flag)) break;
+      if (tile_sync_or(g, *abort_flag)) break;
     }
   }
 
   tc_fence_before();
   __syncthreads();
+  cluster_sync_all();            // the peer's MMAs and loads into this CTA are over
   if (warp == 0) {
     tc_fence_after();
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(512));
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(512));
   }
 }
 
@@ -644,11 +761,15 @@ struct PackPlan {
   int64_t sigma_w, sigma_b, rgb_w, rgb_b;
 };
 
+// Chunk c of a layer holds K columns [32c, 32c + 32) of all N rows as two
+// halves (rows [0, N/2) then [N/2, N)), one per CTA of the pair, each in the
+// no-swizzle K-major core-matrix layout of an N/2-row operand.
 __global__ void tc_pack_kernel(const __nv_bfloat16* __restrict__ blob, PackPlan plan,
                                TcLayout lay, uint8_t* __restrict__ out) {
   const int layer = blockIdx.y;
   const PackLayer& pl = plan.L[layer];
   __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(out);
+  const int Nh = pl.N / 2;
   const int64_t total = (int64_t)pl.n_chunks * CHUNK_K * pl.N;
   for (int64_t q = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; q < total;
        q += (int64_t)gridDim.x * blockDim.x) {
@@ -658,8 +779,9 @@ __global__ void tc_pack_kernel(const __nv_bfloat16* __restrict__ blob, PackPlan 
     const int k = c * CHUNK_K + kl;
     __nv_bfloat16 v = k < pl.K_src ? blob[pl.src_w + (int64_t)n * pl.K_src + k]
                                    : __float2bfloat16(0.0f);
-    const int64_t byte = lay.chunk_off[pl.chunk0 + c] + (kl >> 3) * (pl.N * 16) + (n >> 3) * 128 +
-                         (n & 7) * 16 + (kl & 7) * 2;
+    const int hh = n / Nh, nn = n % Nh;
+    const int64_t byte = lay.chunk_off[pl.chunk0 + c] + (int64_t)hh * (Nh * CHUNK_K * 2) +
+                         (kl >> 3) * (Nh * 16) + (nn >> 3) * 128 + (nn & 7) * 16 + (kl & 7) * 2;
     dst[byte / 2] = v;
   }
   // fp32 vectors (done by the y = 0 slice)
@@ -684,7 +806,34 @@ struct TcState {
   TcLayout lay;
   PackPlan plan;
   uint8_t* buf = nullptr;
+  CUtensorMap tmap_h64;     // the stream as rows of 128 B, boxes of 64 rows (8 KB halves)
+  CUtensorMap tmap_h32;     // boxes of 32 rows (4 KB halves of the direction layer)
+  int max_clusters = 0;     // co-resident CTA pairs of the kernel on this device
 };
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+cudaError_t make_stream_map(CUtensorMap* m, void* base, int64_t bytes, int box_rows) {
+  static EncodeTiledFn encode = nullptr;
+  if (!encode) {
+    cudaDriverEntryPointQueryResult q;
+    void* fn = nullptr;
+    cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q);
+    if (e != cudaSuccess || q != cudaDriverEntryPointSuccess || !fn) return cudaErrorNotSupported;
+    encode = reinterpret_cast<EncodeTiledFn>(fn);
+  }
+  const cuuint64_t dims[2] = {64, (cuuint64_t)(bytes / 128)};
+  const cuuint64_t strides[1] = {128};
+  const cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  CUresult r = encode(m, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, base, dims, strides, box, estr,
+                      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
 
 }  // namespace
 
@@ -713,12 +862,16 @@ cudaError_t tc_alloc(nerf_ctx* ctx) {
   s->plan.rgb_w = off; off += 3 * (W / 2);
   s->plan.rgb_b = off;
   cudaError_t e = cudaMalloc(&s->buf, s->lay.vec_off + s->lay.vec_count * sizeof(float));
-  if (e != cudaSuccess) { delete s; return e; }
+  if (e == cudaSuccess) e = make_stream_map(&s->tmap_h64, s->buf, s->lay.stream_bytes, 64);
+  if (e == cudaSuccess) e = make_stream_map(&s->tmap_h32, s->buf, s->lay.stream_bytes, 32);
+  if (e != cudaSuccess) { cudaFree(s->buf); delete s; return e; }
   int dev = 0;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&ctx->num_sms, cudaDevAttrMultiProcessorCount, dev);
   e = cudaFuncSetAttribute(mlp_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)SMEM_BYTES);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(mlp_tc_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 0);
   if (e != cudaSuccess) { cudaFree(s->buf); delete s; return e; }
   ctx->tc_weights = s;
   ctx->tc_enabled = true;
@@ -742,12 +895,8 @@ cudaError_t launch_bounded_wait_probe(uint32_t timeout_us, uint32_t* flag, uint3
 
 cudaError_t tc_pack(nerf_ctx* ctx, const void* blob, cudaStream_t st) {
   TcState* s = static_cast<TcState*>(ctx->tc_weights);
-  // The dir layer's K columns 0..255 are read with the blob's row stride
-  // (W + dir_ch); the pack kernel indexes rows with K_src, so pass the stride
-  // and clip the packed K range to the first W columns.
-  PackPlan plan = s->plan;
   dim3 grid(128, NLAYER);
-  tc_pack_kernel<<<grid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(blob), plan, s->lay,
+  tc_pack_kernel<<<grid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(blob), s->plan, s->lay,
                                        s->buf);
   return cudaGetLastError();
 }
@@ -767,10 +916,29 @@ cudaError_t tc_run(nerf_ctx* ctx, const float* o, const float* d, int64_t R, con
   P.raw = raw;
   P.flag = ctx->d_flag;
   const int64_t rows = R * ss.S;
-  P.n_pairs = (rows + 2 * TM - 1) / (2 * TM);
-  const int64_t grid = P.n_pairs < ctx->num_sms ? P.n_pairs : ctx->num_sms;
-  mlp_tc_kernel<<<(unsigned)grid, NTHREADS, SMEM_BYTES, st>>>(P);
-  return cudaGetLastError();
+  P.n_pairs = (rows + 4 * TM - 1) / (4 * TM);     // two tiles of 256 rows per CTA pair
+  cudaLaunchConfig_t cfg = {};
+  cfg.blockDim = dim3(NTHREADS);
+  cfg.dynamicSmemBytes = SMEM_BYTES;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (s->max_clusters <= 0) {
+    // persistent grid: as many CTA pairs as can be resident at once
+    cfg.gridDim = dim3((unsigned)ctx->num_sms & ~1u);
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, mlp_tc_kernel, &cfg) != cudaSuccess || n <= 0)
+      n = ctx->num_sms / 2;
+    s->max_clusters = n;
+  }
+  const int64_t clusters = P.n_pairs < s->max_clusters ? P.n_pairs : s->max_clusters;
+  cfg.gridDim = dim3((unsigned)(2 * clusters));
+  return cudaLaunchKernelEx(&cfg, mlp_tc_kernel, P, s->tmap_h64, s->tmap_h32);
 }
 
 }  // namespace nerfb
