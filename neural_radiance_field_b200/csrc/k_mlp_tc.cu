@@ -463,6 +463,18 @@ __device__ __forceinline__ bool mma_pass(int g, uint32_t q0, uint64_t* full, uin
   return true;
 }
 
+// The epilogue's hand-off to the MMA thread: every lane has made its stores
+// visible to the async proxy; after the warp converges, one lane arrives (on
+// CTA 0's barrier, remotely from CTA 1). 256 per-thread arrivals on one
+// barrier would serialize; 8 per CTA do not.
+__device__ __forceinline__ void warp_arrive_act(uint64_t* bar, uint32_t cta, int lane) {
+  __syncwarp();
+  if (lane == 0) {
+    if (cta == 0) mbar_arrive(bar);
+    else mbar_arrive_leader(bar);
+  }
+}
+
 __device__ __forceinline__ bool wait_act(int g, uint32_t (&ph_act)[2], uint64_t* act_ready,
                                          const Ctl& ctl) {
   if (!mbar_wait_cl(&act_ready[g], ph_act[g], ctl)) return false;
@@ -530,7 +542,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) mlp_tc_kernel(Params P, const __g
     for (int s = 0; s < NSTAGE; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
     for (int g = 0; g < 2; ++g) {
       mbar_init(&mma_done[g], 1);
-      mbar_init(&act_ready[g], 2 * TILE_THREADS);     // both CTAs' epilogue threads
+      mbar_init(&act_ready[g], 2 * TILE_THREADS / 32);   // one arrival per epilogue warp
     }
     mbar_init(final_bar, 1);
     *abort_flag = 0;
@@ -638,7 +650,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) mlp_tc_kernel(Params P, const __g
       if (h == 0) store_pe<0>(x[0], x[1], x[2], act_base, r);
       else store_pe<1>(x[0], x[1], x[2], act_base, r);
       fence_async_smem();
-      if (cta == 0) mbar_arrive(&act_ready[g]); else mbar_arrive_leader(&act_ready[g]);
+      warp_arrive_act(&act_ready[g], cta, lane);
 
       float sigma = 0.0f;
       for (int l = 0; l < NLAYER; ++l) {
@@ -670,7 +682,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) mlp_tc_kernel(Params P, const __g
           else epi_half<true, false>(t_row, c0, sb0, sb1, act_base, r, sigma);
           tc_fence_before();
           fence_async_smem();
-          if (cta == 0) mbar_arrive(&act_ready[g]); else mbar_arrive_leader(&act_ready[g]);
+          warp_arrive_act(&act_ready[g], cta, lane);
         } else {
           // direction layer (N = 128): + per-ray bias, ReLU, the rgb head in fp32
           // on this half's 64 columns; the halves are summed through shared memory
