@@ -275,7 +275,9 @@ def run_ours(args, rank, world, local_rank):
                          "achieved": achieved_tf, "peak": peak_tf, "unit": "TFLOP/s",
                          "frac": achieved_tf / peak_tf, "peak_kind": f"bf16 burst, {peak_kind}",
                          "frac_of_sustained": achieved_tf / peak_sus,
-                         "traffic": args.traffic_bytes or None, "avg_launch_ms": avg_launch_ms,
+                         "traffic": args.traffic_bytes or traffic_per_launch(flops_launch_avg),
+                         "traffic_source": "--traffic-bytes" if args.traffic_bytes else TRAFFIC_SOURCE,
+                         "avg_launch_ms": avg_launch_ms,
                          "flop_per_launch": flops_launch_avg},
             "cpu_baseline": cpu,
             "e2e": {"value": world * R / (e2e_ms * 1e-3), "unit": UNIT,
@@ -377,6 +379,20 @@ def run_march(args, rank, world, local_rank):
             "gpu_launches": None, "clocks": clocks}
     print(json.dumps(line), flush=True)
     rnd.close()
+
+
+# DRAM bytes (read + write) per MLP row of the scene-MLP kernel, from the ncu
+# capture summarised in profiles/mlp_tc_kernel_256x256.md: 236.75 MB for the fine
+# launch of a 256x256 frame (12,582,912 rows). The traffic is the raw output
+# and the sample positions, so it grows in proportion to the rows; it is scaled
+# to the launch size here. Re-measure whenever the kernel changes.
+TRAFFIC_B_PER_ROW = 236.75e6 / 12582912
+TRAFFIC_SOURCE = ("ncu dram__bytes_read.sum + dram__bytes_write.sum of the fine launch at "
+                  "256x256, scaled by rows to the average launch")
+
+
+def traffic_per_launch(flops_launch_avg):
+    return TRAFFIC_B_PER_ROW * flops_launch_avg / MLP_FLOP_PER_ROW
 
 
 def main():
