@@ -25,6 +25,7 @@ import nerf_inputs as S  # noqa: E402
 WORKLOAD = "full"
 METRIC = "rays/sec at 800x800 coarse+fine (64+128 samples/ray)"
 UNIT = "rays/s"
+SWEEP_FRAMES = 24                   # the novel-view video: 24 frames around the scene
 MLP_FLOP_PER_ROW = 1186816          # algorithmic FLOPs of one 8x256 NeRF MLP evaluation
 
 
@@ -295,6 +296,90 @@ def run_ours(args, rank, world, local_rank):
 FP32_PEAK_NOTE = "fp32 FMA: 148 SMs x 128 lanes x 2 FLOP x SM clock"
 
 
+def run_sweep(args, rank, world, local_rank):
+    """One step = the rays of a 24-frame 360-degree orbit (one batched ray
+    generation) rendered through ONE nerf_render call: 24 x 640,000 rays,
+    coarse + fine, bf16 network (the novel-view video of the NeRF page,
+    Section 3). An extra line; the headline is the single-frame workload."""
+    import torch
+    import neural_radiance_field_b200 as nb
+    from neural_radiance_field_b200 import build as nbuild
+    nbuild.build()
+    torch.cuda.set_device(local_rank)
+    wl = S.WORKLOADS[WORKLOAD]
+    if args.size:
+        import dataclasses
+        wl = dataclasses.replace(wl, H=args.size, W=args.size, focal=1.25 * args.size)
+    n_frames = SWEEP_FRAMES
+    cams = [c.ravel().tolist() for c in S.orbit_c2ws(wl.seed, n_frames)]
+    cw, _ = S.nerf_weights(wl.mlp, wl.seed, 0, wl.sigma_scale, wl.precision)
+    fw, _ = S.nerf_weights(wl.mlp, wl.seed, 1, wl.sigma_scale, wl.precision)
+    cwt = torch.from_numpy(cw).to(torch.bfloat16).cuda()
+    fwt = torch.from_numpy(fw).to(torch.bfloat16).cuda()
+    R = n_frames * wl.n_rays
+    o = torch.empty(R, 3, device="cuda")
+    d = torch.empty(R, 3, device="cuda")
+    rgb = torch.empty(R, 3, device="cuda")
+    dep = torch.empty(R, device="cuda")
+    acc = torch.empty(R, device="cuda")
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    rnd = nb.Renderer(precision=S.PREC_BF16, max_rays=R, max_samples=wl.n_coarse + wl.n_fine)
+    p = rnd.params(coarse_w=cwt, fine_w=fwt, seed=wl.seed, perturb=1)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        nb.nerf_raygen_batch(wl.H, wl.W, wl.focal, cams, o, d)
+        rnd.render(o, d, wl.near, wl.far, wl.n_coarse, wl.n_fine, p, rgb, dep, acc)
+
+    for _ in range(args.warmup):
+        flush.fill_(1)
+        step()
+    torch.cuda.synchronize()
+    rnd.sync_status()
+    rnd.timing_enable(True)
+    rnd.timing_read()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    with ClockSampler(local_rank) as clk:
+        for k in range(args.steps):
+            flush.fill_(k & 0xFF)
+            ev[k][0].record(stream)
+            step()
+            ev[k][1].record(stream)
+        torch.cuda.synchronize()
+    tot_ms = sum(a.elapsed_time(b) for a, b in ev)
+    mlp_ms, mlp_launches = rnd.timing_read()
+    rnd.timing_enable(False)
+    rnd.sync_status()
+    rows = R * (2 * wl.n_coarse + wl.n_fine)
+    flops_launch_avg = MLP_FLOP_PER_ROW * rows / 2
+    peaks, peak_kind = load_peaks()
+    peak_tf = peaks.get("bf16_tflops")
+    peak_sus = peaks.get("bf16_tflops_sustained", peak_tf)
+    avg_launch_ms = mlp_ms / max(1, mlp_launches)
+    achieved_tf = flops_launch_avg / (avg_launch_ms * 1e-3) / 1e12
+    line = {"metric": f"rays/sec, {n_frames}-frame 360-degree sweep at {wl.H}x{wl.W} coarse+fine "
+                      f"({wl.n_coarse}+{wl.n_fine} samples/ray) in one render call",
+            "value": R * args.steps / (tot_ms * 1e-3), "unit": UNIT, "n_gpus": 1,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": tot_ms / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded orbit cameras, Xavier-init weights)",
+            "config": {"workload": f"sweep{n_frames}_{wl.name}", "frames": n_frames, "H": wl.H,
+                       "W": wl.W, "rays_per_step": R, "n_coarse": wl.n_coarse, "n_fine": wl.n_fine,
+                       "l2": "flushed between timed steps (256 MiB write)"},
+            "frames_per_s": n_frames * args.steps / (tot_ms * 1e-3),
+            "mlp_rows_per_s": rows * args.steps / (tot_ms * 1e-3),
+            "roofline": {"bound": "tensor", "kernel": "scene MLP (coarse and fine launches)",
+                         "achieved": achieved_tf, "peak": peak_tf, "unit": "TFLOP/s",
+                         "frac": achieved_tf / peak_tf, "peak_kind": f"bf16 burst, {peak_kind}",
+                         "frac_of_sustained": achieved_tf / peak_sus,
+                         "traffic": traffic_per_launch(flops_launch_avg),
+                         "traffic_source": TRAFFIC_SOURCE, "avg_launch_ms": avg_launch_ms,
+                         "flop_per_launch": flops_launch_avg},
+            "gpu_launches": args.steps * (2 + 7), "clocks": clk.summary()}
+    print(json.dumps(line), flush=True)
+
+
 def run_march(args, rank, world, local_rank):
     """One step = ray generation + a full-frame march render of the KiloNeRF or
     hash-grid workload (occupancy skipping, scene function, compositing)."""
@@ -404,7 +489,8 @@ def main():
     ap.add_argument("--cpu-rays", type=int, default=1024)
     ap.add_argument("--ref-rays", type=int, default=128)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--workload", default=WORKLOAD, choices=[WORKLOAD, "kilonerf", "hashgrid"],
+    ap.add_argument("--workload", default=WORKLOAD,
+                    choices=[WORKLOAD, "kilonerf", "hashgrid", "sweep24"],
                     help="the benchmark workload (default) or a march workload (extra lines)")
     ap.add_argument("--traffic-bytes", type=float, default=0.0,
                     help="DRAM bytes per network launch from an ncu capture of this kernel")
@@ -416,6 +502,8 @@ def main():
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     if args.impl == "reference":
         run_reference(args, rank, world)
+    elif args.workload == "sweep24":
+        run_sweep(args, rank, world, local_rank)
     elif args.workload != WORKLOAD:
         run_march(args, rank, world, local_rank)
     else:

@@ -139,6 +139,21 @@ NERF_API nerf_status nerf_sync_status(nerf_ctx* ctx, void* stream);
 NERF_API nerf_status nerf_raygen(int H, int W, float focal, const float* c2w_host,
                         float* rays_o, float* rays_d, void* stream);
 
+/* The rays of n_cams cameras in one buffer, for a multi-view sweep (NeRF page,
+ * Section 3: a novel-view video of 24 frames circling the scene, every frame a
+ * new camera pose through the same network). Camera c's pixel (i, j) becomes
+ * ray c*H*W + j*W + i, and each value is bit-identical to what nerf_raygen
+ * writes for that camera alone. c2w_host: [n_cams][3][4] row-major, host
+ * memory, read before the call returns. rays_o, rays_d: device
+ * [n_cams*H*W][3] fp32, caller-owned. Enqueued on `stream` (one launch per 32
+ * cameras); does not synchronise. A whole sweep then goes through one
+ * nerf_render call whose max_rays covers n_cams*H*W.
+ * Errors: NERF_ERR_INVALID_ARG (H, W, n_cams <= 0, focal <= 0, NULL pointer,
+ * more than 2^40 rays), NERF_ERR_CUDA on a launch failure. */
+NERF_API nerf_status nerf_raygen_batch(int H, int W, float focal, int n_cams,
+                                       const float* c2w_host, float* rays_o, float* rays_d,
+                                       void* stream);
+
 /* Render n_rays rays (NeRF page, Section 2.6 render_rays):
  *  NERF_MODEL_MLP: n_coarse stratified samples on [near, far] through the coarse
  *    network; if n_fine > 0, n_fine inverse-CDF draws from the coarse weights of

@@ -138,6 +138,14 @@ def seeded_camera(seed: int):
     return az, el
 
 
+def orbit_c2ws(seed: int, n_frames: int = 24) -> list:
+    """Cameras of a 360-degree orbit (the novel-view video of the NeRF page,
+    Section 3): n_frames azimuths evenly spaced from the seeded camera's, at its
+    elevation and radius 4. Returns a list of [3x4] fp32 arrays."""
+    az0, el = seeded_camera(seed)
+    return [look_at_c2w(az0 + 360.0 * k / n_frames, el) for k in range(n_frames)]
+
+
 # Workloads -----------------------------------------------------------------
 
 @dataclasses.dataclass(frozen=True)

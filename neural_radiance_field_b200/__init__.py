@@ -14,7 +14,7 @@ from ._capi import (NERF_BF16, NERF_FP32, NERF_LAST_1E10, NERF_LAST_TO_FAR, NERF
                     NERF_MODEL_KILONERF, NERF_MODEL_MLP, NERF_SIGMA_RELU, NERF_SIGMA_SOFTPLUS,
                     NerfError, nerf_config, nerf_params)
 
-__all__ = ["Renderer", "nerf_raygen", "nerf_test_stratified", "nerf_test_pe",
+__all__ = ["Renderer", "nerf_raygen", "nerf_raygen_batch", "nerf_test_stratified", "nerf_test_pe",
            "nerf_test_composite", "nerf_test_sample_pdf", "NerfError", "nerf_config",
            "nerf_params"]
 
@@ -49,6 +49,17 @@ def nerf_raygen(H, W, focal, c2w, rays_o, rays_d, stream=None):
     c = (ctypes.c_float * 12)(*[float(v) for v in list(c2w)])
     _capi.check(_capi.lib().nerf_raygen(int(H), int(W), float(focal), c, _ptr(rays_o),
                                         _ptr(rays_d), _stream(stream)))
+
+
+def nerf_raygen_batch(H, W, focal, c2ws, rays_o, rays_d, stream=None):
+    """c2ws: n_cams x 12 host floats; rays_o, rays_d: CUDA [n_cams*H*W, 3], camera-major."""
+    flat = [float(v) for cam in c2ws for v in list(cam)]
+    n_cams = len(flat) // 12
+    if n_cams * 12 != len(flat):
+        raise ValueError("each camera needs 12 values ([3][4] row-major)")
+    c = (ctypes.c_float * len(flat))(*flat)
+    _capi.check(_capi.lib().nerf_raygen_batch(int(H), int(W), float(focal), n_cams, c,
+                                              _ptr(rays_o), _ptr(rays_d), _stream(stream)))
 
 
 def nerf_test_stratified(rays_o, rays_d, near, far, n, seed, perturb, out_t, out_x=None,

@@ -57,6 +57,7 @@ SIGNATURES = {
     "nerf_last_error": (ctypes.c_char_p, [_P]),
     "nerf_sync_status": (_I, [_P, _P]),
     "nerf_raygen": (_I, [_I, _I, _F, _P, _P, _P, _P]),
+    "nerf_raygen_batch": (_I, [_I, _I, _F, _I, _P, _P, _P, _P]),
     "nerf_render": (_I, [_P, _P, _P, _I64, _F, _F, _I, _I, ctypes.POINTER(nerf_params),
                          _P, _P, _P, _P]),
     "nerf_render_host": (_I, [_P, _P, _P, _I64, _F, _F, _I, _I, ctypes.POINTER(nerf_params),

@@ -32,6 +32,50 @@ cudaError_t launch_raygen(int H, int W, float focal, const float* c2w, float* o,
   return cudaGetLastError();
 }
 
+// Up to RAYGEN_BATCH cameras per launch, passed by value.
+constexpr int RAYGEN_BATCH = 32;
+struct C2WBatch {
+  float m[RAYGEN_BATCH][12];
+};
+
+// Rays of several cameras, camera-major: camera c's pixel p lands at
+// c * H * W + p, each value computed exactly as raygen_kernel does.
+__global__ void raygen_batch_kernel(int H, int W, float focal, int n_cams, C2WBatch cams,
+                                    float* __restrict__ o, float* __restrict__ d) {
+  const int64_t hw = (int64_t)H * W;
+  const int64_t q = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (q >= hw * n_cams) return;
+  const int cam = (int)(q / hw);
+  const int64_t p = q % hw;
+  const float* m = cams.m[cam];
+  int j = (int)(p / W), i = (int)(p % W);
+  float dx = fdiv(fsub((float)i, fmul((float)W, 0.5f)), focal);
+  float dy = -fdiv(fsub((float)j, fmul((float)H, 0.5f)), focal);
+#pragma unroll
+  for (int r = 0; r < 3; ++r) {
+    float v = fadd(fadd(fmul(dx, m[r * 4 + 0]), fmul(dy, m[r * 4 + 1])), fmul(-1.0f, m[r * 4 + 2]));
+    d[q * 3 + r] = v;
+    o[q * 3 + r] = m[r * 4 + 3];
+  }
+}
+
+cudaError_t launch_raygen_batch(int H, int W, float focal, int n_cams, const float* c2w,
+                                float* o, float* d, cudaStream_t st) {
+  const int64_t hw = (int64_t)H * W;
+  for (int c0 = 0; c0 < n_cams; c0 += RAYGEN_BATCH) {
+    const int nc = n_cams - c0 < RAYGEN_BATCH ? n_cams - c0 : RAYGEN_BATCH;
+    C2WBatch cams;
+    for (int c = 0; c < nc; ++c)
+      for (int k = 0; k < 12; ++k) cams.m[c][k] = c2w[(int64_t)(c0 + c) * 12 + k];
+    const int64_t n = hw * nc;
+    raygen_batch_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(
+        H, W, focal, nc, cams, o + c0 * hw * 3, d + c0 * hw * 3);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
+}
+
 __global__ void stratified_kernel(const float* __restrict__ o, const float* __restrict__ d,
                                   int64_t R, float near, float step, int n, uint64_t key,
                                   int perturb, float* __restrict__ out_t,

@@ -230,6 +230,18 @@ nerf_status nerf_raygen(int H, int W, float focal, const float* c2w_host, float*
   return NERF_OK;
 }
 
+nerf_status nerf_raygen_batch(int H, int W, float focal, int n_cams, const float* c2w_host,
+                              float* rays_o, float* rays_d, void* stream) {
+  if (H <= 0 || W <= 0 || n_cams <= 0 || !(focal > 0.0f) || !c2w_host || !rays_o || !rays_d)
+    return fail(nullptr, NERF_ERR_INVALID_ARG,
+                "nerf_raygen_batch: bad size, camera count, focal or NULL pointer");
+  if ((int64_t)H * W * n_cams > ((int64_t)1 << 40))
+    return fail(nullptr, NERF_ERR_INVALID_ARG, "nerf_raygen_batch: too many rays");
+  NERF_CHECK_LAUNCH(nullptr, launch_raygen_batch(H, W, focal, n_cams, c2w_host, rays_o, rays_d,
+                                                 (cudaStream_t)stream));
+  return NERF_OK;
+}
+
 }  // extern "C"
 
 // --------------------------------------------------------------------------

@@ -60,6 +60,8 @@ struct Ctx;
 // Launchers (each returns cudaGetLastError()).
 cudaError_t launch_raygen(int H, int W, float focal, const float* c2w, float* o, float* d,
                           cudaStream_t st);
+cudaError_t launch_raygen_batch(int H, int W, float focal, int n_cams, const float* c2w,
+                                float* o, float* d, cudaStream_t st);
 cudaError_t launch_stratified(const float* o, const float* d, int64_t R, float near, float far,
                               int n, uint64_t key, int perturb, float* out_t, float* out_x,
                               cudaStream_t st);
