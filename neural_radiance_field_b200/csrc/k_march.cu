@@ -166,46 +166,57 @@ cudaError_t upload_hash_grid(const HashGridInfo& h) {
 }
 
 // Encoding of one point; optionally records the corner rows.
+// Level l of the encoding of a point with unit-cube coordinates u: the
+// trilinear blend of the 8 corner rows, feature pair (a0, a1).
+__device__ __forceinline__ void hash_encode_level(const __half2* __restrict__ table, float u0,
+                                                  float u1, float u2, int l, int32_t* rows_out,
+                                                  float& a0, float& a1) {
+  const int N = c_hres[l];
+  const float fN = (float)N;
+  const float c0 = fmul(u0, fN), c1 = fmul(u1, fN), c2 = fmul(u2, fN);
+  const float f0 = floorf(c0), f1 = floorf(c1), f2 = floorf(c2);
+  const float w0 = fsub(c0, f0), w1 = fsub(c1, f1), w2 = fsub(c2, f2);
+  const int i0 = (int)f0, i1 = (int)f1, i2 = (int)f2;
+  a0 = 0.f;
+  a1 = 0.f;
+#pragma unroll
+  for (int corner = 0; corner < 8; ++corner) {
+    const int dx = corner >> 2, dy = (corner >> 1) & 1, dz = corner & 1;
+    const int ix = min(max(i0 + dx, 0), N), iy = min(max(i1 + dy, 0), N),
+              iz = min(max(i2 + dz, 0), N);
+    uint32_t idx;
+    if (c_hdirect[l]) {
+      idx = (uint32_t)((ix * (N + 1) + iy) * (N + 1) + iz);
+    } else {
+      idx = ((uint32_t)ix ^ ((uint32_t)iy * 2654435761u) ^ ((uint32_t)iz * 805459861u)) &
+            ((1u << 19) - 1u);
+    }
+    const int row = c_hoff[l] + (int)idx;
+    if (rows_out) rows_out[l * 8 + corner] = row;
+    const float2 f = __half22float2(__ldg(table + row));
+    const float wx = dx ? w0 : 1.0f - w0;
+    const float wy = dy ? w1 : 1.0f - w1;
+    const float wz = dz ? w2 : 1.0f - w2;
+    const float wt = wx * wy * wz;
+    a0 = fmaf(wt, f.x, a0);
+    a1 = fmaf(wt, f.y, a1);
+  }
+}
+
+__device__ __forceinline__ void hash_unit_coords(float x0, float x1, float x2, float& u0,
+                                                 float& u1, float& u2) {
+  u0 = fdiv(fadd(x0, 1.5f), 3.0f);
+  u1 = fdiv(fadd(x1, 1.5f), 3.0f);
+  u2 = fdiv(fadd(x2, 1.5f), 3.0f);
+}
+
 __device__ __forceinline__ void hash_encode_point(const __half2* __restrict__ table, float x0,
                                                   float x1, float x2, float* feat,
                                                   int32_t* rows_out) {
-  const float u0 = fdiv(fadd(x0, 1.5f), 3.0f);
-  const float u1 = fdiv(fadd(x1, 1.5f), 3.0f);
-  const float u2 = fdiv(fadd(x2, 1.5f), 3.0f);
+  float u0, u1, u2;
+  hash_unit_coords(x0, x1, x2, u0, u1, u2);
 #pragma unroll 4
-  for (int l = 0; l < 16; ++l) {
-    const int N = c_hres[l];
-    const float fN = (float)N;
-    const float c0 = fmul(u0, fN), c1 = fmul(u1, fN), c2 = fmul(u2, fN);
-    const float f0 = floorf(c0), f1 = floorf(c1), f2 = floorf(c2);
-    const float w0 = fsub(c0, f0), w1 = fsub(c1, f1), w2 = fsub(c2, f2);
-    const int i0 = (int)f0, i1 = (int)f1, i2 = (int)f2;
-    float a0 = 0.f, a1 = 0.f;
-#pragma unroll
-    for (int corner = 0; corner < 8; ++corner) {
-      const int dx = corner >> 2, dy = (corner >> 1) & 1, dz = corner & 1;
-      const int ix = min(max(i0 + dx, 0), N), iy = min(max(i1 + dy, 0), N),
-                iz = min(max(i2 + dz, 0), N);
-      uint32_t idx;
-      if (c_hdirect[l]) {
-        idx = (uint32_t)((ix * (N + 1) + iy) * (N + 1) + iz);
-      } else {
-        idx = ((uint32_t)ix ^ ((uint32_t)iy * 2654435761u) ^ ((uint32_t)iz * 805459861u)) &
-              ((1u << 19) - 1u);
-      }
-      const int row = c_hoff[l] + (int)idx;
-      if (rows_out) rows_out[l * 8 + corner] = row;
-      const float2 f = __half22float2(__ldg(table + row));
-      const float wx = dx ? w0 : 1.0f - w0;
-      const float wy = dy ? w1 : 1.0f - w1;
-      const float wz = dz ? w2 : 1.0f - w2;
-      const float wt = wx * wy * wz;
-      a0 = fmaf(wt, f.x, a0);
-      a1 = fmaf(wt, f.y, a1);
-    }
-    feat[2 * l] = a0;
-    feat[2 * l + 1] = a1;
-  }
+  for (int l = 0; l < 16; ++l) hash_encode_level(table, u0, u1, u2, l, rows_out, feat[2 * l], feat[2 * l + 1]);
 }
 
 __global__ void hash_encode_kernel(const float* __restrict__ x, int64_t n,
@@ -278,62 +289,172 @@ __global__ void sh_kernel(const float* __restrict__ d, int64_t n, ShConst K,
   for (int j = 0; j < 16; ++j) out[i * 16 + j] = o[j];
 }
 
-// Hash scene function for every live entry: encoding, density MLP, SH colour MLP.
-// Weights (fp32 blob of the ABI, 15,876 floats) are staged in shared memory.
-constexpr int HASH_NW = 15876;
 
-template <int K, int N>
-__device__ __forceinline__ void dense_relu(const float* __restrict__ W, const float* __restrict__ b,
-                                           const float* in, float* out, bool relu) {
+// The hash scene function as small fp32 GEMMs over tiles of 128 live points
+// (a CTA per SM, persistent): the points' activations sit k-major in shared
+// memory, the layer weights transposed (Wt[k][n]) beside them, and each of the
+// 256 threads accumulates an 8-point x 4-output block, so every k step costs
+// three 16-byte shared loads for 32 FMAs. Layers: encoding (32) -> 64 -> 64
+// (ReLU) -> sigma = ReLU(w . h + b); [h | SH16(d)] (80) -> 64 -> 64 (ReLU) ->
+// rgb = sigmoid(W h + b). All arithmetic is fp32 on the CUDA cores.
+constexpr int HASH_NW = 15876;                       // fp32 weights of the ABI blob
+#ifndef NERF_HT_P
+#define NERF_HT_P 128
+#endif
+constexpr int HT_P = NERF_HT_P;                      // points per tile (128 or 64)
+constexpr int HT_PPT = HT_P / 16;                    // points per thread in the GEMMs
+constexpr int HT_TPP = 256 / HT_P;                   // threads per point in the encoding
+constexpr int HT_AP = HT_P + 4;                      // padded row of an activation buffer
+constexpr int HT_THREADS = 256;
+constexpr int HT_CTAS_PER_SM = HT_P == 128 ? 1 : 2;
+// shared-memory layout (floats)
+constexpr int HT_D0 = 0, HT_D1 = HT_D0 + 32 * 64, HT_C0 = HT_D1 + 64 * 64, HT_C1 = HT_C0 + 80 * 64;
+constexpr int HT_VEC = HT_C1 + 64 * 64;              // d0b d1b c0b c1b sw (5 x 64), sb, pad, rw (192), rb
+constexpr int HT_ACT_A = HT_VEC + 5 * 64 + 4 + 192 + 4;
+constexpr int HT_ACT_B = HT_ACT_A + 80 * HT_AP;
+constexpr int HT_SIG = HT_ACT_B + 64 * HT_AP;
+constexpr int HT_RGB = HT_SIG + HT_P;
+constexpr int HT_FLOATS = HT_RGB + 3 * HT_P;
+constexpr size_t HT_SMEM = HT_FLOATS * sizeof(float);
+static_assert(HT_ACT_A % 4 == 0 && HT_ACT_B % 4 == 0 && HT_AP % 4 == 0, "float4 alignment");
+
+// out[n][p] = act(b[n] + sum_k W[n][k] in[k][p]) for the tile, N = 64.
+template <int K>
+__device__ __forceinline__ void tile_dense64(const float* __restrict__ Wt, const float* __restrict__ b,
+                                             const float* in, float* out) {
+  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+  const int n0 = 4 * tx, p0 = HT_PPT * ty;
+  float acc[HT_PPT][4];
+  const float4 bb = *reinterpret_cast<const float4*>(b + n0);
 #pragma unroll
-  for (int n = 0; n < N; ++n) {
-    float acc = b[n];
+  for (int i = 0; i < HT_PPT; ++i) { acc[i][0] = bb.x; acc[i][1] = bb.y; acc[i][2] = bb.z; acc[i][3] = bb.w; }
+#pragma unroll 4
+  for (int k = 0; k < K; ++k) {
+    float a[HT_PPT];
 #pragma unroll
-    for (int k = 0; k < K; ++k) acc = fmaf(W[n * K + k], in[k], acc);
-    out[n] = relu ? fmaxf(acc, 0.0f) : acc;
+    for (int v = 0; v < HT_PPT / 4; ++v) {
+      const float4 a4 = *reinterpret_cast<const float4*>(in + k * HT_AP + p0 + 4 * v);
+      a[4 * v] = a4.x; a[4 * v + 1] = a4.y; a[4 * v + 2] = a4.z; a[4 * v + 3] = a4.w;
+    }
+    const float4 w = *reinterpret_cast<const float4*>(Wt + k * 64 + n0);
+#pragma unroll
+    for (int i = 0; i < HT_PPT; ++i) {
+      acc[i][0] = fmaf(w.x, a[i], acc[i][0]);
+      acc[i][1] = fmaf(w.y, a[i], acc[i][1]);
+      acc[i][2] = fmaf(w.z, a[i], acc[i][2]);
+      acc[i][3] = fmaf(w.w, a[i], acc[i][3]);
+    }
+  }
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    float* o = out + (n0 + j) * HT_AP + p0;
+#pragma unroll
+    for (int v = 0; v < HT_PPT / 4; ++v)
+      *reinterpret_cast<float4*>(o + 4 * v) =
+          make_float4(fmaxf(acc[4 * v][j], 0.f), fmaxf(acc[4 * v + 1][j], 0.f),
+                      fmaxf(acc[4 * v + 2][j], 0.f), fmaxf(acc[4 * v + 3][j], 0.f));
   }
 }
 
-__global__ void __launch_bounds__(128)
+__global__ void __launch_bounds__(HT_THREADS, HT_CTAS_PER_SM)
 hash_eval_kernel(const float* __restrict__ o, const float* __restrict__ d, int64_t r0,
                  float near, float step, const uint32_t* __restrict__ live,
                  const int32_t* __restrict__ total, const __half2* __restrict__ table,
                  const float* __restrict__ mlp, ShConst K, float* __restrict__ out) {
-  extern __shared__ float w[];
-  for (int i = threadIdx.x; i < HASH_NW; i += blockDim.x) w[i] = mlp[i];
-  __syncthreads();
-  const float* d0 = w;            const float* d0b = d0 + 64 * 32;
-  const float* d1 = d0b + 64;     const float* d1b = d1 + 64 * 64;
-  const float* sw = d1b + 64;     const float* sb = sw + 64;
-  const float* c0 = sb + 1;       const float* c0b = c0 + 64 * 80;
-  const float* c1 = c0b + 64;     const float* c1b = c1 + 64 * 64;
-  const float* rw = c1b + 64;     const float* rb = rw + 3 * 64;
+  extern __shared__ __align__(16) float hs[];
+  float* d0t = hs + HT_D0;
+  float* d1t = hs + HT_D1;
+  float* c0t = hs + HT_C0;
+  float* c1t = hs + HT_C1;
+  float* d0b = hs + HT_VEC;
+  float* d1b = d0b + 64;
+  float* c0b = d1b + 64;
+  float* c1b = c0b + 64;
+  float* sw = c1b + 64;
+  float* sb = sw + 64;                 // [1] + pad
+  float* rw = sb + 4;                  // [3][64]
+  float* rb = rw + 192;                // [3]
+  float* act_a = hs + HT_ACT_A;        // [80][HT_AP]: encoding, then h2 | SH, then the last h
+  float* act_b = hs + HT_ACT_B;        // [64][HT_AP]
+  float* sig = hs + HT_SIG;
+  float* rgbv = hs + HT_RGB;           // [3][HT_P]
+  // weights of the ABI blob (row-major W[n][k]) -> transposed Wt[k][n]
+  for (int q = threadIdx.x; q < HASH_NW; q += HT_THREADS) {
+    const float v = mlp[q];
+    if (q < 2048) { d0t[(q % 32) * 64 + q / 32] = v; }
+    else if (q < 2112) { d0b[q - 2048] = v; }
+    else if (q < 6208) { const int z = q - 2112; d1t[(z % 64) * 64 + z / 64] = v; }
+    else if (q < 6272) { d1b[q - 6208] = v; }
+    else if (q < 6336) { sw[q - 6272] = v; }
+    else if (q < 6337) { sb[0] = v; }
+    else if (q < 11457) { const int z = q - 6337; c0t[(z % 80) * 64 + z / 80] = v; }
+    else if (q < 11521) { c0b[q - 11457] = v; }
+    else if (q < 15617) { const int z = q - 11521; c1t[(z % 64) * 64 + z / 64] = v; }
+    else if (q < 15681) { c1b[q - 15617] = v; }
+    else if (q < 15873) { rw[q - 15681] = v; }
+    else { rb[q - 15873] = v; }
+  }
   const int64_t P = *total;
-  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < P;
-       i += (int64_t)gridDim.x * blockDim.x) {
-    const uint32_t e = live[i];
-    const int64_t r = r0 + (e >> 9);
-    const int k = (int)(e & 511u);
-    float x[3], t;
-    march_point(o, d, r, near, step, k, x, &t);
-    float in[80], h[64];
-    hash_encode_point(table, x[0], x[1], x[2], in, nullptr);
-    dense_relu<32, 64>(d0, d0b, in, h, true);
-    dense_relu<64, 64>(d1, d1b, h, in, true);          // in[0..63] = h2
-    float sigma = sb[0];
+  const int p = threadIdx.x & (HT_P - 1);
+  const int part = threadIdx.x / HT_P;          // 0 .. HT_TPP - 1
+  for (int64_t i0 = (int64_t)blockIdx.x * HT_P; i0 < P; i0 += (int64_t)gridDim.x * HT_P) {
+    const int n = (int)min((int64_t)HT_P, P - i0);
+    __syncthreads();     // the previous tile's last reads (and the weight staging) are over
+    // encoding: HT_TPP threads per point, each 16 / HT_TPP of the levels; the
+    // last also writes SH16 of the unit direction into rows 64..79
+    {
+      float x[3] = {0.f, 0.f, 0.f}, t;
+      int64_t r = 0;
+      if (p < n) {
+        const uint32_t e = live[i0 + p];
+        r = r0 + (e >> 9);
+        march_point(o, d, r, near, step, (int)(e & 511u), x, &t);
+      }
+      float u0, u1, u2;
+      hash_unit_coords(x[0], x[1], x[2], u0, u1, u2);
+      constexpr int LPT = 16 / HT_TPP;
+#pragma unroll 2
+      for (int l = LPT * part; l < LPT * part + LPT; ++l) {
+        float a0 = 0.f, a1 = 0.f;
+        if (p < n) hash_encode_level(table, u0, u1, u2, l, nullptr, a0, a1);
+        act_a[(2 * l) * HT_AP + p] = a0;
+        act_a[(2 * l + 1) * HT_AP + p] = a1;
+      }
+      if (part == HT_TPP - 1) {
+        float sh[16];
+        const float dx = d[r * 3], dy = d[r * 3 + 1], dz = d[r * 3 + 2];
+        const float inv = 1.0f / sqrtf(dx * dx + dy * dy + dz * dz);
+        sh16(dx * inv, dy * inv, dz * inv, K, sh);
 #pragma unroll
-    for (int j = 0; j < 64; ++j) sigma = fmaf(sw[j], in[j], sigma);
-    sigma = fmaxf(sigma, 0.0f);
-    const float dx = d[r * 3], dy = d[r * 3 + 1], dz = d[r * 3 + 2];
-    const float inv = 1.0f / sqrtf(dx * dx + dy * dy + dz * dz);
-    sh16(dx * inv, dy * inv, dz * inv, K, in + 64);
-    dense_relu<80, 64>(c0, c0b, in, h, true);
-    dense_relu<64, 64>(c1, c1b, h, in, true);
-    float rgb[3];
-    dense_relu<64, 3>(rw, rb, in, rgb, false);
-    float4 v = make_float4(1.0f / (1.0f + expf(-rgb[0])), 1.0f / (1.0f + expf(-rgb[1])),
-                           1.0f / (1.0f + expf(-rgb[2])), sigma);
-    reinterpret_cast<float4*>(out)[i] = v;
+        for (int j = 0; j < 16; ++j) act_a[(64 + j) * HT_AP + p] = p < n ? sh[j] : 0.f;
+      }
+    }
+    __syncthreads();
+    tile_dense64<32>(d0t, d0b, act_a, act_b);          // 32 -> 64
+    __syncthreads();
+    tile_dense64<64>(d1t, d1b, act_b, act_a);          // 64 -> 64: h2 in rows 0..63
+    __syncthreads();
+    if (part == 0) {                                   // sigma = ReLU(sw . h2 + sb)
+      float s = sb[0];
+#pragma unroll 8
+      for (int j = 0; j < 64; ++j) s = fmaf(sw[j], act_a[j * HT_AP + p], s);
+      sig[p] = fmaxf(s, 0.0f);
+    }
+    tile_dense64<80>(c0t, c0b, act_a, act_b);          // [h2 | SH16] -> 64
+    __syncthreads();
+    tile_dense64<64>(c1t, c1b, act_b, act_a);          // 64 -> 64
+    __syncthreads();
+    for (int q = threadIdx.x; q < 3 * HT_P; q += HT_THREADS) {   // rgb head
+      const int c = q / HT_P, pp = q % HT_P;
+      float v = rb[c];
+#pragma unroll 8
+      for (int j = 0; j < 64; ++j) v = fmaf(rw[c * 64 + j], act_a[j * HT_AP + pp], v);
+      rgbv[c * HT_P + pp] = 1.0f / (1.0f + expf(-v));
+    }
+    __syncthreads();
+    if (part == 0 && p < n)
+      reinterpret_cast<float4*>(out)[i0 + p] =
+          make_float4(rgbv[p], rgbv[HT_P + p], rgbv[2 * HT_P + p], sig[p]);
   }
 }
 
@@ -550,7 +671,7 @@ cudaError_t march_render_chunk(const MarchArgs& a, cudaStream_t st) {
   const unsigned g = (unsigned)(a.num_sms * 8);
   if (a.model == NERF_MODEL_HASHGRID) {
     if (a.ev_start) cudaEventRecord(a.ev_start, st);
-    hash_eval_kernel<<<g, 128, HASH_NW * sizeof(float), st>>>(
+    hash_eval_kernel<<<(unsigned)(a.num_sms * HT_CTAS_PER_SM), HT_THREADS, HT_SMEM, st>>>(
         a.o, a.d, a.r0, a.near, a.step, a.ws.live, total,
         reinterpret_cast<const __half2*>(a.hash_table), a.hash_mlp, a.sh, a.ws.val);
   } else {
@@ -603,7 +724,7 @@ cudaError_t march_prepare(cudaStream_t st) {
   cudaError_t e = upload_hash_grid(hash_grid_info());
   if (e != cudaSuccess) return e;
   return cudaFuncSetAttribute(hash_eval_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              HASH_NW * (int)sizeof(float));
+                              (int)HT_SMEM);
 }
 
 }  // namespace nerfb
