@@ -504,68 +504,197 @@ __global__ void cell_scatter_kernel(const int32_t* __restrict__ cell, const int3
 
 constexpr int KILO_NP = 3317;
 
-// Per-cell tiny MLP over the cell-grouped order: consecutive threads mostly
-// share a cell, so their weight loads coalesce into broadcasts.
-__global__ void __launch_bounds__(128)
+// Work items of the per-cell evaluation: every cell's run of the cell-grouped
+// order split into tiles of at most KT_P points. One CTA of 1024 threads, four
+// cells per thread, a block scan of the tile counts.
+constexpr int KT_P = 128;
+__global__ void __launch_bounds__(1024)
+kilo_items_kernel(const int32_t* __restrict__ hist, const int32_t* __restrict__ cell_off,
+                  int4* __restrict__ items, int32_t* __restrict__ n_items) {
+  __shared__ int32_t sums[1024];
+  const int t = threadIdx.x;
+  int cnt[4], tot = 0;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    cnt[j] = (hist[4 * t + j] + KT_P - 1) / KT_P;
+    tot += cnt[j];
+  }
+  sums[t] = tot;
+  __syncthreads();
+  for (int off = 1; off < 1024; off <<= 1) {
+    const int v = t >= off ? sums[t - off] : 0;
+    __syncthreads();
+    sums[t] += v;
+    __syncthreads();
+  }
+  int pos = sums[t] - tot;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const int c = 4 * t + j, h = hist[c], base = cell_off[c];
+    for (int q = 0; q < cnt[j]; ++q)
+      items[pos++] = make_int4(c, base + q * KT_P, min(KT_P, h - q * KT_P), 0);
+  }
+  if (t == 1023) *n_items = sums[1023];
+}
+
+// The per-cell tiny MLPs as small fp32 GEMMs: a CTA stages one cell's 3,317
+// weights in shared memory (the layer matrices transposed, Wt[k][n]) and runs a
+// tile of that cell's points through them; activations sit k-major, and each
+// of 256 threads accumulates a 4-point x 4-output block (two 16-byte shared
+// loads per 16 FMAs). The accumulation order (bias, then k ascending) is the
+// per-point definition's.
+constexpr int KT_AP = KT_P + 4;
+constexpr int KT_THREADS = 256;
+constexpr int KT_W1 = 0, KT_B1 = KT_W1 + 63 * 32, KT_W2 = KT_B1 + 32, KT_B2 = KT_W2 + 32 * 32;
+constexpr int KT_WS = KT_B2 + 32, KT_BS = KT_WS + 32, KT_WC = KT_BS + 1, KT_BC = KT_WC + 3 * 59;
+constexpr int KT_ACT = 3320;                          // KILO_NP rounded up to a multiple of 4
+constexpr int KT_H1 = KT_ACT + 63 * KT_AP;            // [32][KT_AP]
+constexpr int KT_DPE = KT_H1 + 32 * KT_AP;            // [27][KT_AP]: gamma(unit d)
+constexpr int KT_SIG = KT_DPE + 27 * KT_AP;
+constexpr int KT_RGB = KT_SIG + KT_P;
+constexpr int KT_FLOATS = KT_RGB + 3 * KT_P;
+constexpr size_t KT_SMEM = KT_FLOATS * sizeof(float);
+static_assert(KT_ACT >= KILO_NP && KT_ACT % 4 == 0 && KT_H1 % 4 == 0, "layout");
+
+// out[n][p] = ReLU(b[n] + sum_k W[n][k] in[k][p]), N = 32.
+template <int K>
+__device__ __forceinline__ void tile_dense32(const float* __restrict__ Wt, const float* __restrict__ b,
+                                             const float* in, float* out) {
+  const int tx = threadIdx.x & 7, ty = threadIdx.x >> 3;
+  const int n0 = 4 * tx, p0 = 4 * ty;
+  float acc[4][4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) acc[i][j] = b[n0 + j];
+#pragma unroll 7
+  for (int k = 0; k < K; ++k) {
+    const float4 a4 = *reinterpret_cast<const float4*>(in + k * KT_AP + p0);
+    const float4 w = *reinterpret_cast<const float4*>(Wt + k * 32 + n0);
+    const float a[4] = {a4.x, a4.y, a4.z, a4.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      acc[i][0] = fmaf(w.x, a[i], acc[i][0]);
+      acc[i][1] = fmaf(w.y, a[i], acc[i][1]);
+      acc[i][2] = fmaf(w.z, a[i], acc[i][2]);
+      acc[i][3] = fmaf(w.w, a[i], acc[i][3]);
+    }
+  }
+#pragma unroll
+  for (int j = 0; j < 4; ++j)
+    *reinterpret_cast<float4*>(out + (n0 + j) * KT_AP + p0) =
+        make_float4(fmaxf(acc[0][j], 0.f), fmaxf(acc[1][j], 0.f), fmaxf(acc[2][j], 0.f),
+                    fmaxf(acc[3][j], 0.f));
+}
+
+__global__ void __launch_bounds__(KT_THREADS, 2)
 kilo_eval_kernel(const float* __restrict__ o, const float* __restrict__ d, int64_t r0, float near,
-                 float step, const uint32_t* __restrict__ live, const int32_t* __restrict__ total,
-                 const int32_t* __restrict__ order, const int32_t* __restrict__ cell,
+                 float step, const uint32_t* __restrict__ live, const int32_t* __restrict__ order,
+                 const int4* __restrict__ items, const int32_t* __restrict__ n_items,
                  const float* __restrict__ cell_w, float* __restrict__ out) {
-  const int64_t P = *total;
-  for (int64_t j = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; j < P;
-       j += (int64_t)gridDim.x * blockDim.x) {
-    const int64_t i = order[j];
-    const uint32_t e = live[i];
-    const int64_t r = r0 + (e >> 9);
-    float x[3], t;
-    march_point(o, d, r, near, step, (int)(e & 511u), x, &t);
-    const float* W = cell_w + (int64_t)cell[i] * KILO_NP;
-    const float* W1 = W;           const float* b1 = W1 + 32 * 63;
-    const float* W2 = b1 + 32;     const float* b2 = W2 + 32 * 32;
-    const float* ws = b2 + 32;     const float* bs = ws + 32;
-    const float* Wc = bs + 1;      const float* bc = Wc + 3 * 59;
-    float pe[63];
-    pe[0] = x[0]; pe[1] = x[1]; pe[2] = x[2];
-#pragma unroll
-    for (int c = 0; c < 3; ++c)
-#pragma unroll
-      for (int k = 0; k < 10; ++k) pe_sincos(x[c], k, &pe[3 + c * 10 + k], &pe[33 + c * 10 + k]);
-    float h1[32], h2[59];
-#pragma unroll 4
-    for (int n = 0; n < 32; ++n) {
-      float acc = __ldg(b1 + n);
-#pragma unroll
-      for (int k = 0; k < 63; ++k) acc = fmaf(__ldg(W1 + n * 63 + k), pe[k], acc);
-      h1[n] = fmaxf(acc, 0.0f);
+  extern __shared__ __align__(16) float ks[];
+  float* w1t = ks + KT_W1;
+  float* b1 = ks + KT_B1;
+  float* w2t = ks + KT_W2;
+  float* b2 = ks + KT_B2;
+  float* ws = ks + KT_WS;
+  float* bs = ks + KT_BS;
+  float* wc = ks + KT_WC;
+  float* bc = ks + KT_BC;
+  float* act = ks + KT_ACT;          // gamma(x) [63][KT_AP], then h2 in rows 0..31
+  float* h1 = ks + KT_H1;
+  float* dpe = ks + KT_DPE;
+  float* sig = ks + KT_SIG;
+  float* rgbv = ks + KT_RGB;
+  const int p = threadIdx.x & (KT_P - 1);
+  const int part = threadIdx.x / KT_P;          // 0: position encoding, 1: direction encoding
+  const int NI = *n_items;
+  for (int it = blockIdx.x; it < NI; it += gridDim.x) {
+    const int4 item = items[it];
+    const int n = item.z;
+    __syncthreads();     // the previous item's last reads are over
+    // this cell's weights (row-major W[n][k] in the blob) -> Wt[k][n], in two
+    // bank-conflict-free steps through the (idle) activation buffer: a
+    // coalesced copy (W2 rows padded to 33), then a transpose with lanes along n
+    const float* W = cell_w + (int64_t)item.x * KILO_NP;
+    float* tmp = act;
+    for (int q = threadIdx.x; q < KILO_NP; q += KT_THREADS) {
+      const float v = __ldg(W + q);
+      if (q < KT_B1) tmp[q] = v;
+      else if (q < KT_W2) b1[q - KT_B1] = v;
+      else if (q < KT_B2) { const int z = q - KT_W2; tmp[KT_B1 + (z / 32) * 33 + z % 32] = v; }
+      else ks[q] = v;                               // b2, ws, bs, wc, bc in place
     }
-#pragma unroll 4
-    for (int n = 0; n < 32; ++n) {
-      float acc = __ldg(b2 + n);
+    __syncthreads();
+    for (int t = threadIdx.x; t < 63 * 32; t += KT_THREADS) w1t[t] = tmp[(t % 32) * 63 + t / 32];
+    for (int t = threadIdx.x; t < 32 * 32; t += KT_THREADS)
+      w2t[t] = tmp[KT_B1 + (t % 32) * 33 + t / 32];
+    __syncthreads();     // the transpose's reads of the activation buffer are over
+    int64_t i = 0;
+    if (p < n) i = order[item.y + p];
+    {
+      float x[3] = {0.f, 0.f, 0.f}, t;
+      int64_t r = 0;
+      if (p < n) {
+        const uint32_t e = live[i];
+        r = r0 + (e >> 9);
+        march_point(o, d, r, near, step, (int)(e & 511u), x, &t);
+      }
+      if (part == 0) {
+        act[0 * KT_AP + p] = x[0];
+        act[1 * KT_AP + p] = x[1];
+        act[2 * KT_AP + p] = x[2];
 #pragma unroll
-      for (int k = 0; k < 32; ++k) acc = fmaf(__ldg(W2 + n * 32 + k), h1[k], acc);
-      h2[n] = fmaxf(acc, 0.0f);
+        for (int c = 0; c < 3; ++c)
+#pragma unroll
+          for (int k = 0; k < 10; ++k) {
+            float sn, cs;
+            pe_sincos(x[c], k, &sn, &cs);
+            act[(3 + c * 10 + k) * KT_AP + p] = sn;
+            act[(33 + c * 10 + k) * KT_AP + p] = cs;
+          }
+      } else {
+        const float dx = d[r * 3], dy = d[r * 3 + 1], dz = d[r * 3 + 2];
+        const float inv = 1.0f / sqrtf(dx * dx + dy * dy + dz * dz);
+        const float u[3] = {dx * inv, dy * inv, dz * inv};
+        dpe[0 * KT_AP + p] = u[0];
+        dpe[1 * KT_AP + p] = u[1];
+        dpe[2 * KT_AP + p] = u[2];
+#pragma unroll
+        for (int c = 0; c < 3; ++c)
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            float sn, cs;
+            pe_sincos(u[c], k, &sn, &cs);
+            dpe[(3 + c * 4 + k) * KT_AP + p] = sn;
+            dpe[(15 + c * 4 + k) * KT_AP + p] = cs;
+          }
+      }
     }
-    float sigma = __ldg(bs);
-#pragma unroll
-    for (int k = 0; k < 32; ++k) sigma = fmaf(__ldg(ws + k), h2[k], sigma);
-    sigma = fmaxf(sigma, 0.0f);
-    const float dx = d[r * 3], dy = d[r * 3 + 1], dz = d[r * 3 + 2];
-    const float inv = 1.0f / sqrtf(dx * dx + dy * dy + dz * dz);
-    const float u[3] = {dx * inv, dy * inv, dz * inv};
-    h2[32] = u[0]; h2[33] = u[1]; h2[34] = u[2];
-#pragma unroll
-    for (int c = 0; c < 3; ++c)
-#pragma unroll
-      for (int k = 0; k < 4; ++k) pe_sincos(u[c], k, &h2[35 + c * 4 + k], &h2[47 + c * 4 + k]);
-    float rgb[3];
-#pragma unroll
-    for (int n = 0; n < 3; ++n) {
-      float acc = __ldg(bc + n);
-#pragma unroll
-      for (int k = 0; k < 59; ++k) acc = fmaf(__ldg(Wc + n * 59 + k), h2[k], acc);
-      rgb[n] = 1.0f / (1.0f + expf(-acc));
+    __syncthreads();
+    tile_dense32<63>(w1t, b1, act, h1);                // gamma(x) -> h1
+    __syncthreads();
+    tile_dense32<32>(w2t, b2, h1, act);                // h1 -> h2 (rows 0..31)
+    __syncthreads();
+    if (part == 0) {
+      float s = bs[0];
+#pragma unroll 8
+      for (int k = 0; k < 32; ++k) s = fmaf(ws[k], act[k * KT_AP + p], s);
+      sig[p] = fmaxf(s, 0.0f);
     }
-    reinterpret_cast<float4*>(out)[i] = make_float4(rgb[0], rgb[1], rgb[2], sigma);
+    for (int q = threadIdx.x; q < 3 * KT_P; q += KT_THREADS) {
+      const int c = q / KT_P, pp = q % KT_P;
+      float v = bc[c];
+#pragma unroll 8
+      for (int k = 0; k < 32; ++k) v = fmaf(wc[c * 59 + k], act[k * KT_AP + pp], v);
+#pragma unroll
+      for (int k = 0; k < 27; ++k) v = fmaf(wc[c * 59 + 32 + k], dpe[k * KT_AP + pp], v);
+      rgbv[c * KT_P + pp] = 1.0f / (1.0f + expf(-v));
+    }
+    __syncthreads();
+    if (part == 0 && p < n)
+      reinterpret_cast<float4*>(out)[i] =
+          make_float4(rgbv[p], rgbv[KT_P + p], rgbv[2 * KT_P + p], sig[p]);
   }
 }
 
@@ -684,9 +813,13 @@ cudaError_t march_render_chunk(const MarchArgs& a, cudaStream_t st) {
     cell_scatter_kernel<<<g, 256, 0, st>>>(a.ws.cell, total, 0, a.ws.cell_off, a.ws.cell_fill,
                                            a.ws.order);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    kilo_items_kernel<<<1, 1024, 0, st>>>(a.ws.cell_hist, a.ws.cell_off, a.ws.items,
+                                          a.ws.n_items);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
     if (a.ev_start) cudaEventRecord(a.ev_start, st);
-    kilo_eval_kernel<<<g, 128, 0, st>>>(a.o, a.d, a.r0, a.near, a.step, a.ws.live, total,
-                                        a.ws.order, a.ws.cell, a.cell_w, a.ws.val);
+    kilo_eval_kernel<<<(unsigned)(a.num_sms * 2), KT_THREADS, KT_SMEM, st>>>(
+        a.o, a.d, a.r0, a.near, a.step, a.ws.live, a.ws.order, a.ws.items, a.ws.n_items,
+        a.cell_w, a.ws.val);
   }
   if (a.ev_stop) cudaEventRecord(a.ev_stop, st);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
@@ -723,8 +856,11 @@ cudaError_t march_prepare(cudaStream_t st) {
   (void)st;
   cudaError_t e = upload_hash_grid(hash_grid_info());
   if (e != cudaSuccess) return e;
-  return cudaFuncSetAttribute(hash_eval_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              (int)HT_SMEM);
+  cudaError_t e2 = cudaFuncSetAttribute(hash_eval_kernel,
+                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)HT_SMEM);
+  if (e2 != cudaSuccess) return e2;
+  return cudaFuncSetAttribute(kilo_eval_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              (int)KT_SMEM);
 }
 
 }  // namespace nerfb

@@ -75,7 +75,7 @@ void free_march(nerf_ctx* ctx) {
   MarchWs& w = ctx->mws;
   cudaFree(w.mask); cudaFree(w.count); cudaFree(w.off); cudaFree(w.scan_tmp);
   cudaFree(w.live); cudaFree(w.val); cudaFree(w.cell); cudaFree(w.order);
-  cudaFree(w.cell_hist); cudaFree(w.cell_off);
+  cudaFree(w.cell_hist); cudaFree(w.cell_off); cudaFree(w.items); cudaFree(w.n_items);
   w = MarchWs{};
 }
 
@@ -105,6 +105,8 @@ nerf_status create_march(const nerf_config& c, nerf_ctx** out) {
     ok &= dalloc(&w.order, (size_t)w.cap) == cudaSuccess;
     ok &= dalloc(&w.cell_hist, 2 * 4096) == cudaSuccess;
     ok &= dalloc(&w.cell_off, 4097) == cudaSuccess;
+    ok &= dalloc(&w.items, (size_t)(w.cap / 128 + 4096)) == cudaSuccess;
+    ok &= dalloc(&w.n_items, 1) == cudaSuccess;
     if (ok) w.cell_fill = w.cell_hist + 4096;
   }
   ok &= dalloc(&ctx->stage, (size_t)(c.max_rays * 11)) == cudaSuccess;

@@ -30,6 +30,8 @@ struct MarchWs {
   int32_t* cell_hist = nullptr;  // [4096] followed by cell_fill [4096]
   int32_t* cell_fill = nullptr;
   int32_t* cell_off = nullptr;   // [4097]
+  int4* items = nullptr;         // [cap / 128 + 4096]: (cell, first order index, points, 0)
+  int32_t* n_items = nullptr;    // [1]
 };
 
 struct MarchArgs {
