@@ -380,6 +380,85 @@ def run_sweep(args, rank, world, local_rank):
     print(json.dumps(line), flush=True)
 
 
+def run_compact(args, rank, world, local_rank):
+    """One step = ray generation + a coarse+fine render of the 800x800 frame with a
+    compact fp32 network (D=4, W=128, skip after layer 1: a scene-specialised
+    shape in the spirit of the NAS-NeRF page) on the CUDA-core MLP kernel. An
+    extra line; the headline is the 8x256 bf16 workload."""
+    import dataclasses
+    import torch
+    import neural_radiance_field_b200 as nb
+    from neural_radiance_field_b200 import build as nbuild
+    nbuild.build()
+    torch.cuda.set_device(local_rank)
+    shape = S.MLPShape(D=4, W=128, skip=1)
+    wl = dataclasses.replace(S.WORKLOADS[WORKLOAD], mlp=shape, precision=S.PREC_FP32)
+    if args.size:
+        wl = dataclasses.replace(wl, H=args.size, W=args.size, focal=1.25 * args.size)
+    c2w = wl.c2w().ravel().tolist()
+    cw, _ = S.nerf_weights(shape, wl.seed, 0, wl.sigma_scale, wl.precision)
+    fw, _ = S.nerf_weights(shape, wl.seed, 1, wl.sigma_scale, wl.precision)
+    cwt, fwt = torch.from_numpy(cw).cuda(), torch.from_numpy(fw).cuda()
+    R = wl.n_rays
+    o = torch.empty(R, 3, device="cuda")
+    d = torch.empty(R, 3, device="cuda")
+    rgb = torch.empty(R, 3, device="cuda")
+    dep = torch.empty(R, device="cuda")
+    acc = torch.empty(R, device="cuda")
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    rnd = nb.Renderer(D=shape.D, W=shape.W, skip=shape.skip, precision=S.PREC_FP32, max_rays=R,
+                      max_samples=wl.n_coarse + wl.n_fine)
+    p = rnd.params(coarse_w=cwt, fine_w=fwt, seed=wl.seed, perturb=1)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        nb.nerf_raygen(wl.H, wl.W, wl.focal, c2w, o, d)
+        rnd.render(o, d, wl.near, wl.far, wl.n_coarse, wl.n_fine, p, rgb, dep, acc)
+
+    for _ in range(args.warmup):
+        flush.fill_(1)
+        step()
+    torch.cuda.synchronize()
+    rnd.sync_status()
+    rnd.timing_enable(True)
+    rnd.timing_read()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    with ClockSampler(local_rank) as clk:
+        for k in range(args.steps):
+            flush.fill_(k & 0xFF)
+            ev[k][0].record(stream)
+            step()
+            ev[k][1].record(stream)
+        torch.cuda.synchronize()
+    tot_ms = sum(a.elapsed_time(b) for a, b in ev)
+    mlp_ms, mlp_launches = rnd.timing_read()
+    rnd.timing_enable(False)
+    rnd.sync_status()
+    flop_row = 2 * sum(n * k for _, n, k in shape.layer_shapes())
+    rows = R * (2 * wl.n_coarse + wl.n_fine)
+    clocks = clk.summary()
+    sm_mhz = clocks["sm_mhz"] or 1965.0
+    peak = 148 * 128 * 2 * sm_mhz * 1e6 / 1e12
+    achieved = flop_row * rows * args.steps / (mlp_ms * 1e-3) / 1e12
+    line = {"metric": f"rays/sec at {wl.H}x{wl.W} coarse+fine ({wl.n_coarse}+{wl.n_fine} samples/ray), "
+                      f"compact fp32 network D{shape.D} W{shape.W} skip@{shape.skip}",
+            "value": R * args.steps / (tot_ms * 1e-3), "unit": UNIT, "n_gpus": 1,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": tot_ms / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+            "data": "synthetic (seeded camera, Xavier-init weights)",
+            "config": {"workload": f"compact_D{shape.D}W{shape.W}_{wl.H}x{wl.W}_fp32",
+                       "mlp": f"{shape.D}x{shape.W} skip@{shape.skip}", "flop_per_row": flop_row,
+                       "l2": "flushed between timed steps (256 MiB write)"},
+            "mlp_rows_per_s": rows * args.steps / (tot_ms * 1e-3),
+            "roofline": {"bound": "alu", "kernel": "mlp_fp32_kernel (CUDA-core MLP, W=128)",
+                         "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                         "frac": achieved / peak, "peak_kind": FP32_PEAK_NOTE, "traffic": None,
+                         "avg_launch_ms": mlp_ms / max(1, mlp_launches)},
+            "gpu_launches": args.steps * 9, "clocks": clocks}
+    print(json.dumps(line), flush=True)
+
+
 def run_march(args, rank, world, local_rank):
     """One step = ray generation + a full-frame march render of the KiloNeRF or
     hash-grid workload (occupancy skipping, scene function, compositing)."""
@@ -490,7 +569,7 @@ def main():
     ap.add_argument("--ref-rays", type=int, default=128)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--workload", default=WORKLOAD,
-                    choices=[WORKLOAD, "kilonerf", "hashgrid", "sweep24"],
+                    choices=[WORKLOAD, "kilonerf", "hashgrid", "sweep24", "compact"],
                     help="the benchmark workload (default) or a march workload (extra lines)")
     ap.add_argument("--traffic-bytes", type=float, default=0.0,
                     help="DRAM bytes per network launch from an ncu capture of this kernel")
@@ -504,6 +583,8 @@ def main():
         run_reference(args, rank, world)
     elif args.workload == "sweep24":
         run_sweep(args, rank, world, local_rank)
+    elif args.workload == "compact":
+        run_compact(args, rank, world, local_rank)
     elif args.workload != WORKLOAD:
         run_march(args, rank, world, local_rank)
     else:

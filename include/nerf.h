@@ -64,9 +64,12 @@ enum { NERF_LAST_1E10 = 0, NERF_LAST_TO_FAR = 1 };
  * F_theta (Section 2.4): D layers of width W with ReLU, gamma(x) concatenated
  * after layer `skip` (skip < 0: none), sigma head Linear(W,1), feature layer
  * Linear(W,W), direction layer Linear(W + 3(1+2 L_dir), W/2) + ReLU, rgb head
- * Linear(W/2, 3). Supported: (W=256, D=8, skip=4) and (W=64, D in 1..8, no skip),
- * L_pos = 10, L_dir = 4. precision BF16 selects the tensor-core path (W=256
- * only); sigma_act and white_bkgd are applied in compositing.
+ * Linear(W/2, 3). Supported with precision FP32: W in {64, 128, 256}, D in
+ * 1..8, skip = -1 or 0 <= skip <= D-2 (the compact, scene-specialised shapes
+ * of the NAS-NeRF page; the CUDA-core kernel is compiled per width), with
+ * L_pos = 10, L_dir = 4. precision BF16 selects the tensor-core path, built
+ * for the page's (W=256, D=8, skip=4) network only (NERF_ERR_UNSUPPORTED
+ * otherwise); sigma_act and white_bkgd are applied in compositing.
  * KILONERF and HASHGRID ignore D..precision. max_rays and max_samples size
  * the context's workspace (max_samples >= n_coarse + n_fine of any render). */
 typedef struct {

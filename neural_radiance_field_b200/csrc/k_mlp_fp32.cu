@@ -260,6 +260,10 @@ cudaError_t launch_mlp_fp32(const PackedFp32& p, const float* packed, const floa
     size_t sh = sizeof(Smem<256>);
     cudaFuncSetAttribute(mlp_fp32_kernel<256>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sh);
     mlp_fp32_kernel<256><<<blocks, NT, sh, st>>>(p, packed, dir_bias, o, d, R, ss, raw);
+  } else if (p.W == 128) {
+    size_t sh = sizeof(Smem<128>);
+    cudaFuncSetAttribute(mlp_fp32_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sh);
+    mlp_fp32_kernel<128><<<blocks, NT, sh, st>>>(p, packed, dir_bias, o, d, R, ss, raw);
   } else if (p.W == 64) {
     size_t sh = sizeof(Smem<64>);
     cudaFuncSetAttribute(mlp_fp32_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sh);

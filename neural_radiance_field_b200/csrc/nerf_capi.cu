@@ -145,11 +145,14 @@ nerf_status nerf_create(const nerf_config* cfg, nerf_ctx** out) {
   if (c.model == NERF_MODEL_MLP) {
     if (c.L_pos != 10 || c.L_dir != 4)
       return fail(nullptr, NERF_ERR_UNSUPPORTED, "L_pos must be 10 and L_dir 4");
-    bool big = (c.W == 256 && c.D == 8 && c.skip == 4);
-    bool tiny = (c.W == 64 && c.D >= 1 && c.D <= 8 && c.skip < 0);
-    if (!big && !tiny)
+    // compact shapes (NAS-NeRF page): any depth 1..8, width 64/128/256, the
+    // skip concatenation after any layer but the last, or none
+    const bool big = (c.W == 256 && c.D == 8 && c.skip == 4);
+    const bool shape_ok = (c.W == 64 || c.W == 128 || c.W == 256) && c.D >= 1 && c.D <= 8 &&
+                          (c.skip == -1 || (c.skip >= 0 && c.skip <= c.D - 2));
+    if (!shape_ok)
       return fail(nullptr, NERF_ERR_UNSUPPORTED,
-                  "network must be (W=256, D=8, skip=4) or (W=64, D<=8, no skip)");
+                  "network must have W in {64, 128, 256}, D in 1..8 and skip -1 or in 0..D-2");
     if (c.precision != NERF_FP32 && c.precision != NERF_BF16)
       return fail(nullptr, NERF_ERR_INVALID_ARG, "precision must be FP32 or BF16");
     if (c.precision == NERF_BF16 && !big)

@@ -43,7 +43,11 @@ def test_create_rejects_bad_configs_without_a_device(lib):
     assert lib.nerf_create(ctypes.byref(cfg), ctypes.byref(h)) == _capi.NERF_ERR_INVALID_ARG
     assert h.value is None
     assert b"max_rays" in lib.nerf_last_error(None)
-    cfg = _capi.nerf_config(0, 8, 128, 4, 10, 4, 0, 0, 0, 0, 16, 192)     # W = 128
+    cfg = _capi.nerf_config(0, 8, 96, 4, 10, 4, 0, 0, 0, 0, 16, 192)      # W = 96
+    assert lib.nerf_create(ctypes.byref(cfg), ctypes.byref(h)) == _capi.NERF_ERR_UNSUPPORTED
+    cfg = _capi.nerf_config(0, 4, 128, 3, 10, 4, 0, 0, 0, 0, 16, 192)     # skip after the last layer
+    assert lib.nerf_create(ctypes.byref(cfg), ctypes.byref(h)) == _capi.NERF_ERR_UNSUPPORTED
+    cfg = _capi.nerf_config(0, 9, 128, -1, 10, 4, 0, 0, 0, 0, 16, 192)    # D = 9
     assert lib.nerf_create(ctypes.byref(cfg), ctypes.byref(h)) == _capi.NERF_ERR_UNSUPPORTED
     cfg = _capi.nerf_config(0, 4, 64, -1, 10, 4, 0, 1, 0, 0, 16, 192)     # bf16 tiny
     assert lib.nerf_create(ctypes.byref(cfg), ctypes.byref(h)) == _capi.NERF_ERR_UNSUPPORTED
