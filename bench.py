@@ -26,6 +26,7 @@ WORKLOAD = "full"
 METRIC = "rays/sec at 800x800 coarse+fine (64+128 samples/ray)"
 UNIT = "rays/s"
 SWEEP_FRAMES = 24                   # the novel-view video: 24 frames around the scene
+TRAIN_BATCH = 4096                  # rays per training step (NeRF page, "7. Training loop")
 MLP_FLOP_PER_ROW = 1186816          # algorithmic FLOPs of one 8x256 NeRF MLP evaluation
 
 
@@ -459,6 +460,86 @@ def run_compact(args, rank, world, local_rank):
     print(json.dumps(line), flush=True)
 
 
+def run_train(args, rank, world, local_rank):
+    """One step = the NeRF page's training step ("7. Training loop") on a batch of
+    4096 rays drawn from the 800x800 frame: coarse + fine render of the 8x256
+    network in fp32, loss = mse(coarse) + mse(fine) against seeded target colours,
+    and the gradients of both networks (nerf_loss_grad). An extra line."""
+    import dataclasses
+    import torch
+    import neural_radiance_field_b200 as nb
+    from neural_radiance_field_b200 import build as nbuild
+    nbuild.build()
+    torch.cuda.set_device(local_rank)
+    wl = dataclasses.replace(S.WORKLOADS[WORKLOAD], precision=S.PREC_FP32)
+    B = TRAIN_BATCH
+    shape = wl.mlp
+    o_all = torch.empty(wl.n_rays, 3, device="cuda")
+    d_all = torch.empty(wl.n_rays, 3, device="cuda")
+    nb.nerf_raygen(wl.H, wl.W, wl.focal, wl.c2w().ravel().tolist(), o_all, d_all)
+    gen = torch.Generator(device="cpu").manual_seed(wl.seed)
+    cw, _ = S.nerf_weights(shape, wl.seed, 0, wl.sigma_scale, S.PREC_FP32)
+    fw, _ = S.nerf_weights(shape, wl.seed, 1, wl.sigma_scale, S.PREC_FP32)
+    cwt, fwt = torch.from_numpy(cw).cuda(), torch.from_numpy(fw).cuda()
+    n_batches = max(args.steps, args.warmup)
+    idx = [torch.randperm(wl.n_rays, generator=gen)[:B].cuda() for _ in range(n_batches)]
+    batches = [(o_all[i].contiguous(), d_all[i].contiguous()) for i in idx]
+    targets = [torch.rand(B, 3, generator=gen).cuda() for _ in range(n_batches)]
+    rnd = nb.Renderer(precision=S.PREC_FP32, max_rays=B, max_samples=wl.n_coarse + wl.n_fine)
+    p = rnd.params(coarse_w=cwt, fine_w=fwt, seed=wl.seed, perturb=1)
+    loss = torch.zeros(1, device="cuda")
+    gc = torch.empty(cw.size, device="cuda")
+    gf = torch.empty(fw.size, device="cuda")
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    def step(k):
+        o, d = batches[k]
+        rnd.loss_grad(o, d, wl.near, wl.far, wl.n_coarse, wl.n_fine, p, targets[k], loss, gc, gf)
+
+    for k in range(args.warmup):
+        flush.fill_(1)
+        step(k)
+    torch.cuda.synchronize()
+    rnd.sync_status()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    with ClockSampler(local_rank) as clk:
+        for k in range(args.steps):
+            flush.fill_(k & 0xFF)
+            ev[k][0].record(stream)
+            step(k)
+            ev[k][1].record(stream)
+        torch.cuda.synchronize()
+    rnd.sync_status()
+    tot_ms = sum(a.elapsed_time(b) for a, b in ev)
+    # algorithmic FLOPs per MLP row: the forward, then the backward's weight
+    # gradients (one multiply-add per weight and row) and input gradients (all
+    # layers but the first, and not for the direction layer's gamma(d) columns)
+    fwd = MLP_FLOP_PER_ROW
+    bwd = fwd + (fwd - 2 * shape.W * shape.pos_ch - 2 * (shape.W // 2) * shape.dir_ch)
+    rows = B * (2 * wl.n_coarse + wl.n_fine)
+    clocks = clk.summary()
+    sm_mhz = clocks["sm_mhz"] or 1965.0
+    peak = 148 * 128 * 2 * sm_mhz * 1e6 / 1e12
+    achieved = (fwd + bwd) * rows * args.steps / (tot_ms * 1e-3) / 1e12
+    line = {"metric": f"training rays/sec, batches of {B} rays, {wl.H}x{wl.W} frame, coarse+fine "
+                      f"({wl.n_coarse}+{wl.n_fine}), 8x256 fp32, loss + gradients of both networks",
+            "value": B * args.steps / (tot_ms * 1e-3), "unit": UNIT, "n_gpus": 1,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": tot_ms / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+            "data": "synthetic (seeded ray batches and target colours, Xavier-init weights)",
+            "config": {"workload": f"train_batch{B}_nerf_800x800_fp32", "batch_rays": B,
+                       "mlp": "8x256 skip@4, fp32", "flop_per_row_fwd_bwd": fwd + bwd,
+                       "l2": "flushed between timed steps (256 MiB write)"},
+            "loss_last_step": float(loss.item()),
+            "roofline": {"bound": "alu", "kernel": "whole training step (fp32 CUDA-core kernels)",
+                         "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                         "frac": achieved / peak, "peak_kind": FP32_PEAK_NOTE, "traffic": None},
+            "gpu_launches": None, "clocks": clocks}
+    print(json.dumps(line), flush=True)
+
+
 def run_march(args, rank, world, local_rank):
     """One step = ray generation + a full-frame march render of the KiloNeRF or
     hash-grid workload (occupancy skipping, scene function, compositing)."""
@@ -569,7 +650,7 @@ def main():
     ap.add_argument("--ref-rays", type=int, default=128)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--workload", default=WORKLOAD,
-                    choices=[WORKLOAD, "kilonerf", "hashgrid", "sweep24", "compact"],
+                    choices=[WORKLOAD, "kilonerf", "hashgrid", "sweep24", "compact", "train"],
                     help="the benchmark workload (default) or a march workload (extra lines)")
     ap.add_argument("--traffic-bytes", type=float, default=0.0,
                     help="DRAM bytes per network launch from an ncu capture of this kernel")
@@ -585,6 +666,8 @@ def main():
         run_sweep(args, rank, world, local_rank)
     elif args.workload == "compact":
         run_compact(args, rank, world, local_rank)
+    elif args.workload == "train":
+        run_train(args, rank, world, local_rank)
     elif args.workload != WORKLOAD:
         run_march(args, rank, world, local_rank)
     else:

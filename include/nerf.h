@@ -173,6 +173,30 @@ NERF_API nerf_status nerf_render(nerf_ctx* ctx, const float* rays_o, const float
                         const nerf_params* params, float* out_rgb, float* out_depth,
                         float* out_acc, void* stream);
 
+/* Loss and parameter gradients of one training step (NeRF page, "7. Training
+ * loop"): the rays are rendered as nerf_render does (coarse pass; with n_fine >
+ * 0 the fine pass on the sorted union of positions drawn from the coarse
+ * weights, which are detached: "6. Hierarchical sampling"), and
+ *   loss = mse(rgb_coarse, target) + mse(rgb_fine, target)
+ * (each mse the mean over n_rays x 3 values; without a fine pass only the
+ * coarse term). Writes *out_loss and the gradients of the loss with respect to
+ * every parameter of the coarse and fine networks.
+ * ctx: NERF_MODEL_MLP with precision FP32 (NERF_ERR_UNSUPPORTED otherwise).
+ * target_rgb: device [n_rays][3] fp32. out_loss: device, one float.
+ * grad_coarse, grad_fine: device fp32 buffers of the network's parameter count,
+ * laid out like the weight blobs (per Linear: W row-major [N][K], then b);
+ * overwritten. grad_fine may be NULL when n_fine == 0. n_coarse >= 2 and
+ * n_coarse + n_fine <= min(max_samples, 256); the fine pass needs n_coarse = 64.
+ * The first call allocates the training workspace on the current device, about
+ * max_rays x min(max_samples, 256) x (64 + (D+1) W + 2.5 W + 4) floats
+ * (NERF_ERR_OOM if that fails). The gradients are summed with fp32 atomics, so
+ * their last bits vary between runs. Enqueued on `stream`; does not synchronise. */
+NERF_API nerf_status nerf_loss_grad(nerf_ctx* ctx, const float* rays_o, const float* rays_d,
+                                    int64_t n_rays, float near, float far, int n_coarse,
+                                    int n_fine, const nerf_params* params,
+                                    const float* target_rgb, float* out_loss, float* grad_coarse,
+                                    float* grad_fine, void* stream);
+
 /* nerf_render with HOST ray and output buffers (pinned memory recommended):
  * copies the rays into the context's staging buffers, renders, copies the
  * results back and synchronises `stream` before returning. */

@@ -165,6 +165,14 @@ class Renderer:
             int(n_coarse), int(n_fine), ctypes.byref(params), _ptr(out_rgb), _ptr(out_depth),
             _ptr(out_acc), _stream(stream)), self.ctx)
 
+    def loss_grad(self, rays_o, rays_d, near, far, n_coarse, n_fine, params, target_rgb,
+                  out_loss, grad_coarse, grad_fine=None, stream=None):
+        """Training-step loss and gradients (fp32 contexts); see nerf_loss_grad."""
+        _capi.check(_capi.lib().nerf_loss_grad(
+            self.ctx, _ptr(rays_o), _ptr(rays_d), rays_o.shape[0], float(near), float(far),
+            int(n_coarse), int(n_fine), ctypes.byref(params), _ptr(target_rgb), _ptr(out_loss),
+            _ptr(grad_coarse), _ptr(grad_fine), _stream(stream)), self.ctx)
+
     def render_host(self, rays_o, rays_d, near, far, n_coarse, n_fine, params, out_rgb, out_depth,
                     out_acc, stream=None):
         _capi.check(_capi.lib().nerf_render_host(

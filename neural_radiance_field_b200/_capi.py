@@ -60,6 +60,8 @@ SIGNATURES = {
     "nerf_raygen_batch": (_I, [_I, _I, _F, _I, _P, _P, _P, _P]),
     "nerf_render": (_I, [_P, _P, _P, _I64, _F, _F, _I, _I, ctypes.POINTER(nerf_params),
                          _P, _P, _P, _P]),
+    "nerf_loss_grad": (_I, [_P, _P, _P, _I64, _F, _F, _I, _I, ctypes.POINTER(nerf_params),
+                            _P, _P, _P, _P, _P]),
     "nerf_render_host": (_I, [_P, _P, _P, _I64, _F, _F, _I, _I, ctypes.POINTER(nerf_params),
                               _P, _P, _P, _P]),
     "nerf_timing_enable": (_I, [_P, _I]),

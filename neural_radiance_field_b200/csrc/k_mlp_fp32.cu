@@ -163,11 +163,31 @@ __device__ __forceinline__ void tile_layer(Smem<W>& sm, const float* __restrict_
   __syncthreads();
 }
 
+// Copies columns [src, src + n) of the tile's activations to columns
+// [dst, dst + n) of the training path's activation store (row-major, ld floats
+// per row; n a multiple of 4).
+template <int W>
+__device__ __forceinline__ void store_cols(const Smem<W>& sm, float* save, int64_t ld,
+                                           int64_t row0, int64_t rows, int src, int64_t dst,
+                                           int n) {
+  const int n4 = n / 4;
+  for (int q = threadIdx.x; q < BM * n4; q += NT) {
+    const int r = q / n4, c = 4 * (q % n4);
+    const int64_t row = row0 + r;
+    if (row < rows)
+      *reinterpret_cast<float4*>(save + row * ld + dst + c) =
+          *reinterpret_cast<const float4*>(&sm.act[r][src + c]);
+  }
+}
+
 template <int W>
 __global__ void __launch_bounds__(NT, 1)
 mlp_fp32_kernel(PackedFp32 p, const float* __restrict__ pk, const float* __restrict__ dir_bias,
                 const float* __restrict__ o, const float* __restrict__ d, int64_t R,
-                SampleSpec ss, float* __restrict__ raw) {
+                SampleSpec ss, float* __restrict__ raw, float* __restrict__ save) {
+  // save (training path, else NULL): per row [gamma(x) (64) | h_0 .. h_{D-1} |
+  // feature | h_dir], the layers' post-activation outputs
+  const int64_t ldc = 64 + (int64_t)(p.D + 1) * W + W / 2;
   extern __shared__ __align__(16) unsigned char smem_raw[];
   Smem<W>& sm = *reinterpret_cast<Smem<W>*>(smem_raw);
   const int64_t rows = R * ss.S;
@@ -216,11 +236,13 @@ mlp_fp32_kernel(PackedFp32 p, const float* __restrict__ pk, const float* __restr
     sm.act[r][W + j] = v;
   }
   __syncthreads();
+  if (save) store_cols<W>(sm, save, ldc, row0, rows, W, 0, 64);
 
   for (int l = 0; l < p.D; ++l) {
     int K = (l == 0) ? 64 : (l == p.skip + 1 ? W + 64 : W);
     int in_col = (l == 0) ? W : 0;
     tile_layer<W, W>(sm, pk + p.layer_w[l], pk + p.layer_b[l], nullptr, K, in_col, 0, true);
+    if (save) store_cols<W>(sm, save, ldc, row0, rows, 0, 64 + (int64_t)l * W, W);
   }
   // sigma head from h (4 threads per row)
   {
@@ -233,7 +255,9 @@ mlp_fp32_kernel(PackedFp32 p, const float* __restrict__ pk, const float* __restr
   }
   // feature layer (no activation), then the direction layer with its per-ray bias
   tile_layer<W, W>(sm, pk + p.feat_w, pk + p.feat_b, nullptr, W, 0, 0, false);
+  if (save) store_cols<W>(sm, save, ldc, row0, rows, 0, 64 + (int64_t)p.D * W, W);
   tile_layer<W, W / 2>(sm, pk + p.dir_w, nullptr, dir_bias, W, 0, 0, true);
+  if (save) store_cols<W>(sm, save, ldc, row0, rows, 0, 64 + (int64_t)(p.D + 1) * W, W / 2);
   // rgb head and output
   if (tid < BM * 3) {
     int r = tid / 3, c = tid % 3;
@@ -253,21 +277,21 @@ mlp_fp32_kernel(PackedFp32 p, const float* __restrict__ pk, const float* __restr
 
 cudaError_t launch_mlp_fp32(const PackedFp32& p, const float* packed, const float* dir_bias,
                             const float* o, const float* d, int64_t R, const SampleSpec& ss,
-                            float* raw, cudaStream_t st) {
+                            float* raw, cudaStream_t st, float* save) {
   int64_t rows = R * ss.S;
   unsigned blocks = (unsigned)((rows + BM - 1) / BM);
   if (p.W == 256) {
     size_t sh = sizeof(Smem<256>);
     cudaFuncSetAttribute(mlp_fp32_kernel<256>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sh);
-    mlp_fp32_kernel<256><<<blocks, NT, sh, st>>>(p, packed, dir_bias, o, d, R, ss, raw);
+    mlp_fp32_kernel<256><<<blocks, NT, sh, st>>>(p, packed, dir_bias, o, d, R, ss, raw, save);
   } else if (p.W == 128) {
     size_t sh = sizeof(Smem<128>);
     cudaFuncSetAttribute(mlp_fp32_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sh);
-    mlp_fp32_kernel<128><<<blocks, NT, sh, st>>>(p, packed, dir_bias, o, d, R, ss, raw);
+    mlp_fp32_kernel<128><<<blocks, NT, sh, st>>>(p, packed, dir_bias, o, d, R, ss, raw, save);
   } else if (p.W == 64) {
     size_t sh = sizeof(Smem<64>);
     cudaFuncSetAttribute(mlp_fp32_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sh);
-    mlp_fp32_kernel<64><<<blocks, NT, sh, st>>>(p, packed, dir_bias, o, d, R, ss, raw);
+    mlp_fp32_kernel<64><<<blocks, NT, sh, st>>>(p, packed, dir_bias, o, d, R, ss, raw, save);
   } else {
     return cudaErrorInvalidValue;
   }

@@ -201,6 +201,10 @@ nerf_status nerf_destroy(nerf_ctx* ctx) {
   cudaFree(ctx->t_all);
   cudaFree(ctx->stage);
   cudaFree(ctx->d_flag);
+  cudaFree(ctx->tr_save);
+  cudaFree(ctx->tr_draw);
+  cudaFree(ctx->tr_tmp);
+  cudaFree(ctx->tr_loss);
   free_march(ctx);
   if (ctx->ev) {
     for (int i = 0; i < 2 * kMaxTimed; ++i) cudaEventDestroy(ctx->ev[i]);
@@ -270,9 +274,11 @@ struct TimedScope {
   }
 };
 
-// Runs one network (coarse or fine) over R rays with S samples each.
+// Runs one network (coarse or fine) over R rays with S samples each; `save`
+// (fp32 path only) receives the activations the training path's backward reads.
 nerf_status run_network(nerf_ctx* ctx, const void* blob, const float* o, const float* d,
-                        int64_t R, const SampleSpec& ss, float* raw, cudaStream_t st) {
+                        int64_t R, const SampleSpec& ss, float* raw, cudaStream_t st,
+                        float* save = nullptr) {
   const nerf_config& c = ctx->cfg;
   int64_t w_off, b_off;
   dir_offsets(c, &w_off, &b_off);
@@ -287,7 +293,8 @@ nerf_status run_network(nerf_ctx* ctx, const void* blob, const float* o, const f
   const int dir_ch = 3 * (1 + 2 * c.L_dir);
   NERF_CHECK_LAUNCH(ctx, launch_pack_fp32(blob, c.precision, ctx->plan, dir_ch, ctx->packed, st));
   TimedScope ts(ctx, st);
-  NERF_CHECK_LAUNCH(ctx, launch_mlp_fp32(ctx->plan, ctx->packed, ctx->dir_bias, o, d, R, ss, raw, st));
+  NERF_CHECK_LAUNCH(ctx, launch_mlp_fp32(ctx->plan, ctx->packed, ctx->dir_bias, o, d, R, ss, raw, st,
+                                         save));
   return NERF_OK;
 }
 
@@ -409,6 +416,89 @@ nerf_status nerf_render(nerf_ctx* ctx, const float* rays_o, const float* rays_d,
   if (s != NERF_OK) return s;
   NERF_CHECK_LAUNCH(ctx, launch_composite(ctx->raw, fine, rays_d, R, cs, out_rgb, out_depth,
                                           out_acc, nullptr, st));
+  return NERF_OK;
+}
+
+nerf_status nerf_loss_grad(nerf_ctx* ctx, const float* rays_o, const float* rays_d,
+                           int64_t n_rays, float near, float far, int n_coarse, int n_fine,
+                           const nerf_params* params, const float* target_rgb, float* out_loss,
+                           float* grad_coarse, float* grad_fine, void* stream) {
+  if (!ctx) return fail(nullptr, NERF_ERR_INVALID_ARG, "ctx is NULL");
+  const nerf_config& c = ctx->cfg;
+  if (c.model != NERF_MODEL_MLP || c.precision != NERF_FP32)
+    return fail(ctx, NERF_ERR_UNSUPPORTED, "nerf_loss_grad needs an fp32 NERF_MODEL_MLP context");
+  if (!rays_o || !rays_d || !params || !target_rgb || !out_loss || !grad_coarse ||
+      (n_fine > 0 && !grad_fine))
+    return fail(ctx, NERF_ERR_INVALID_ARG, "NULL ray, params, target, loss or gradient pointer");
+  if (n_rays <= 0 || n_rays > c.max_rays)
+    return fail(ctx, NERF_ERR_INVALID_ARG, "n_rays=%lld outside (0, max_rays=%lld]",
+                (long long)n_rays, (long long)c.max_rays);
+  if (!(near < far)) return fail(ctx, NERF_ERR_INVALID_ARG, "near must be < far");
+  const int s_max = c.max_samples < 256 ? c.max_samples : 256;
+  if (n_coarse < 2 || n_fine < 0 || n_coarse + n_fine > s_max)
+    return fail(ctx, NERF_ERR_INVALID_ARG,
+                "n_coarse >= 2 and n_coarse + n_fine <= min(max_samples, 256) on the training path");
+  if (!params->coarse_w || (n_fine > 0 && !params->fine_w))
+    return fail(ctx, NERF_ERR_INVALID_ARG, "weight blob is NULL");
+  if (n_fine > 0 && (n_coarse != 64 || n_fine > 128))
+    return fail(ctx, NERF_ERR_UNSUPPORTED, "the fine pass needs n_coarse = 64, n_fine <= 128");
+  cudaStream_t st = (cudaStream_t)stream;
+  const int64_t R = n_rays, W = c.W;
+  const int64_t ldc = 64 + (int64_t)(c.D + 1) * W + W / 2;
+  const int dir_ch = 3 * (1 + 2 * c.L_dir);
+  if (!ctx->tr_save) {
+    const int64_t rows = c.max_rays * (int64_t)s_max;
+    bool ok = dalloc(&ctx->tr_save, (size_t)(rows * ldc)) == cudaSuccess;
+    ok &= dalloc(&ctx->tr_draw, (size_t)(rows * 4)) == cudaSuccess;
+    ok &= dalloc(&ctx->tr_tmp, (size_t)(2 * rows * W + c.max_rays * (W / 2 + dir_ch))) == cudaSuccess;
+    ok &= dalloc(&ctx->tr_loss, (size_t)(2 * c.max_rays)) == cudaSuccess;
+    if (!ok) {
+      cudaGetLastError();
+      cudaFree(ctx->tr_save); cudaFree(ctx->tr_draw); cudaFree(ctx->tr_tmp); cudaFree(ctx->tr_loss);
+      ctx->tr_save = ctx->tr_draw = ctx->tr_tmp = ctx->tr_loss = nullptr;
+      return fail(ctx, NERF_ERR_OOM, "training workspace allocation failed");
+    }
+  }
+  const size_t gbytes = (size_t)ctx->n_params * sizeof(float);
+  NERF_CHECK_LAUNCH(ctx, cudaMemsetAsync(grad_coarse, 0, gbytes, st));
+  if (n_fine > 0) NERF_CHECK_LAUNCH(ctx, cudaMemsetAsync(grad_fine, 0, gbytes, st));
+  const uint64_t key = sm64_mix(params->seed);
+  SampleSpec coarse{};
+  coarse.mode = SAMPLES_STRATIFIED;
+  coarse.S = n_coarse;
+  coarse.near = near;
+  coarse.step = (far - near) / (float)n_coarse;
+  coarse.key = key;
+  coarse.perturb = params->perturb;
+  CompositeSpec cs{c.last_delta_mode, far, 0.0f, c.sigma_act, c.white_bkgd};
+  const float inv3n = 1.0f / (3.0f * (float)R);
+  // coarse pass: forward with the activation store, the fine positions from
+  // its (detached) weights, then its backward
+  nerf_status s = run_network(ctx, params->coarse_w, rays_o, rays_d, R, coarse, ctx->raw, st,
+                              ctx->tr_save);
+  if (s != NERF_OK) return s;
+  if (n_fine > 0)
+    NERF_CHECK_LAUNCH(ctx, launch_coarse_resample(ctx->raw, coarse, rays_d, R, cs, n_fine, key,
+                                                  params->perturb, ctx->t_all, st));
+  NERF_CHECK_LAUNCH(ctx, launch_composite_bw(ctx->raw, coarse, rays_d, R, cs, target_rgb, inv3n,
+                                             ctx->tr_draw, ctx->tr_loss, st));
+  NERF_CHECK_LAUNCH(ctx, mlp_backward_fp32(ctx->plan, c.L_dir, (const float*)params->coarse_w,
+                                           ctx->tr_save, R, n_coarse, rays_d, ctx->tr_draw,
+                                           grad_coarse, ctx->tr_tmp, st));
+  if (n_fine > 0) {
+    SampleSpec fine{};
+    fine.mode = SAMPLES_GIVEN_T;
+    fine.S = n_coarse + n_fine;
+    fine.t = ctx->t_all;
+    s = run_network(ctx, params->fine_w, rays_o, rays_d, R, fine, ctx->raw, st, ctx->tr_save);
+    if (s != NERF_OK) return s;
+    NERF_CHECK_LAUNCH(ctx, launch_composite_bw(ctx->raw, fine, rays_d, R, cs, target_rgb, inv3n,
+                                               ctx->tr_draw, ctx->tr_loss + R, st));
+    NERF_CHECK_LAUNCH(ctx, mlp_backward_fp32(ctx->plan, c.L_dir, (const float*)params->fine_w,
+                                             ctx->tr_save, R, fine.S, rays_d, ctx->tr_draw,
+                                             grad_fine, ctx->tr_tmp, st));
+  }
+  NERF_CHECK_LAUNCH(ctx, launch_sum(ctx->tr_loss, n_fine > 0 ? 2 * R : R, out_loss, st));
   return NERF_OK;
 }
 

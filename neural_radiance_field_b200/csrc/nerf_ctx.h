@@ -20,6 +20,11 @@ struct nerf_ctx {
   float* t_all = nullptr;      // [max_rays][max_samples]
   float* stage = nullptr;      // host-path staging: o, d, rgb [R][3]; depth, acc [R]
   unsigned* d_flag = nullptr;  // device error flag
+  // training path (nerf_loss_grad), allocated on its first call
+  float* tr_save = nullptr;    // [max_rays * S][64 + (D+1) W + W/2] activation store
+  float* tr_draw = nullptr;    // [max_rays * S][4] d raw
+  float* tr_tmp = nullptr;     // backward scratch
+  float* tr_loss = nullptr;    // [2 max_rays] per-ray loss terms
 
   // network-kernel timing (nerf_timing_enable / nerf_timing_read)
   bool timing = false;

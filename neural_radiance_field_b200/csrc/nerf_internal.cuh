@@ -96,7 +96,8 @@ struct SampleSpec {
 
 cudaError_t launch_mlp_fp32(const PackedFp32& p, const float* packed, const float* dir_bias,
                             const float* o, const float* d, int64_t R, const SampleSpec& ss,
-                            float* raw, cudaStream_t st);
+                            float* raw, cudaStream_t st,
+                            float* save = nullptr);
 
 // Compositing of raw [R][S][4]; t from ss (stratified or given).
 struct CompositeSpec {
@@ -104,6 +105,14 @@ struct CompositeSpec {
   float far, march_step;
   int sigma_act, white;
 };
+// Training path (k_train.cu).
+cudaError_t launch_composite_bw(const float* raw, const SampleSpec& ss, const float* d, int64_t R,
+                                const CompositeSpec& cs, const float* target, float inv3n,
+                                float* d_raw, float* loss_terms, cudaStream_t st);
+cudaError_t mlp_backward_fp32(const PackedFp32& p, int L_dir, const float* w, const float* save,
+                              int64_t R, int S, const float* d, const float* d_raw,
+                              float* grad, float* tmp, cudaStream_t st);
+cudaError_t launch_sum(const float* v, int64_t n, float* out, cudaStream_t st);
 cudaError_t launch_composite(const float* raw, const SampleSpec& ss, const float* d, int64_t R,
                              const CompositeSpec& cs, float* rgb, float* depth, float* acc,
                              float* weights, cudaStream_t st);

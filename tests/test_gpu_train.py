@@ -1,0 +1,139 @@
+"""Training step (loss and parameter gradients) through nerf_loss_grad, against
+the fp64 oracle of oracle/nerf_grad.py (itself pinned by finite differences).
+
+Coarse-only steps have exact sample positions on both sides and are held to a
+strict bar. With a fine pass, the fine positions come from the coarse weights
+in fp32 (kernel) and fp64 (oracle); a random L = 10 field amplifies that
+rounding, so the fine gradient is held to max(bar, 3 x the oracle's own spread
+when its positions move by fp32 rounding), the criterion of the forward tests."""
+import dataclasses
+
+import numpy as np
+import pytest
+
+import nerf_inputs as S
+from oracle import nerf_grad as og
+
+from gpu_cases import rays_for
+
+pytestmark = pytest.mark.gpu
+
+REL = 1e-4      # gradient bar, relative to the largest gradient entry of the network
+
+
+@pytest.fixture(scope="module")
+def torch():
+    import torch
+    from neural_radiance_field_b200 import build
+    build.build()
+    return torch
+
+
+def _gpu_step(torch, wl, o, d, cw, fw, target, perturb=1):
+    import neural_radiance_field_b200 as nb
+    m = wl.mlp
+    R = o.shape[0]
+    rnd = nb.Renderer(D=m.D, W=m.W, skip=m.skip, sigma_act=wl.sigma_act, precision=S.PREC_FP32,
+                      last_delta_mode=wl.last_delta, white_bkgd=wl.white_bkgd, max_rays=R,
+                      max_samples=wl.n_coarse + wl.n_fine)
+    cwt = torch.from_numpy(cw).cuda()
+    fwt = torch.from_numpy(fw).cuda() if fw is not None else None
+    p = rnd.params(coarse_w=cwt, fine_w=fwt, seed=wl.seed, perturb=perturb)
+    tgt = torch.from_numpy(target.astype(np.float32)).cuda()
+    loss = torch.zeros(1, device="cuda")
+    gc = torch.empty(cw.size, device="cuda")
+    gf = torch.empty(cw.size, device="cuda") if fwt is not None else None
+    rnd.loss_grad(o, d, wl.near, wl.far, wl.n_coarse, wl.n_fine, p, tgt, loss, gc, gf)
+    torch.cuda.synchronize()
+    rnd.sync_status()
+    rnd.close()
+    return (float(loss.item()), gc.cpu().numpy().astype(np.float64),
+            gf.cpu().numpy().astype(np.float64) if gf is not None else None)
+
+
+def _setup(key, H, W, **kw):
+    wl = dataclasses.replace(S.WORKLOADS[key], H=H, W=W, precision=S.PREC_FP32, **kw)
+    cw, _ = S.nerf_weights(wl.mlp, wl.seed, 0, wl.sigma_scale, S.PREC_FP32)
+    fw, _ = S.nerf_weights(wl.mlp, wl.seed, 1, wl.sigma_scale, S.PREC_FP32) if wl.n_fine else (None, None)
+    target = np.random.default_rng(wl.seed + 77).uniform(0.0, 1.0, size=(wl.n_rays, 3))
+    return wl, cw, fw, target
+
+
+COARSE_CASES = [
+    dict(mlp=S.MLPShape(D=3, W=64, skip=0), last_delta=S.LAST_DELTA_TO_FAR),
+    dict(mlp=S.MLPShape(D=4, W=128, skip=1), last_delta=S.LAST_DELTA_TO_FAR, white_bkgd=1),
+    dict(mlp=S.MLPShape(D=2, W=64, skip=-1), last_delta=S.LAST_DELTA_TO_FAR,
+         sigma_act=S.SIGMA_SOFTPLUS),
+    dict(mlp=S.MLPShape(D=8, W=256, skip=4), last_delta=S.LAST_DELTA_TO_FAR),
+    dict(mlp=S.MLPShape(D=3, W=64, skip=1), last_delta=S.LAST_DELTA_PAGE,
+         sigma_act=S.SIGMA_SOFTPLUS, white_bkgd=1),
+]
+
+
+@pytest.mark.parametrize("kw", COARSE_CASES,
+                         ids=lambda kw: f"D{kw['mlp'].D}W{kw['mlp'].W}s{kw['mlp'].skip}")
+def test_coarse_step_matches_oracle(torch, kw):
+    wl, cw, fw, target = _setup("small", 5, 7, n_fine=0, **kw)
+    o, d = rays_for(wl)
+    loss, gc, _ = _gpu_step(torch, wl, o, d, cw, None, target)
+    ids = np.arange(wl.n_rays)
+    ref_loss, ref_gc, _ = og.loss_and_grad(wl, o.cpu().numpy(), d.cpu().numpy(), ids, target,
+                                           cw.astype(np.float64), None)
+    assert abs(loss - ref_loss) <= 1e-5 * ref_loss, (loss, ref_loss)
+    scale = np.abs(ref_gc).max()
+    err = np.abs(gc - ref_gc).max()
+    print(f"[train {kw['mlp']}] loss rel err {abs(loss - ref_loss) / ref_loss:.2e}, "
+          f"grad max err / max|g| {err / scale:.2e}")
+    assert err <= REL * scale + 1e-9, (err, scale, int(np.abs(gc - ref_gc).argmax()))
+
+
+def test_coarse_and_fine_step(torch):
+    wl, cw, fw, target = _setup("small", 4, 6, mlp=S.MLPShape(D=3, W=64, skip=0),
+                                last_delta=S.LAST_DELTA_TO_FAR)
+    o, d = rays_for(wl)
+    loss, gc, gf = _gpu_step(torch, wl, o, d, cw, fw, target)
+    o_np, d_np = o.cpu().numpy(), d.cpu().numpy()
+    ids = np.arange(wl.n_rays)
+    pos = og.sample_positions(wl, o_np, d_np, ids, cw)
+    ref_loss, ref_gc, ref_gf = og.loss_and_grad(wl, o_np, d_np, ids, target, cw.astype(np.float64),
+                                                fw.astype(np.float64), positions=pos)
+    # the coarse network's gradient sees exact positions
+    assert np.abs(gc - ref_gc).max() <= REL * np.abs(ref_gc).max() + 1e-9
+    # the oracle's own spread under fp32-level moves of the fine positions
+    rng = np.random.default_rng(3)
+    spread_g = np.zeros_like(ref_gf)
+    spread_l = 0.0
+    for _ in range(3):
+        t_all = pos[1].astype(np.float64)
+        t_all = (t_all * (1.0 + 1.2e-7 * rng.standard_normal(t_all.shape))).astype(np.float32)
+        t_all = np.sort(t_all, axis=-1)
+        l2, _, g2 = og.loss_and_grad(wl, o_np, d_np, ids, target, cw.astype(np.float64),
+                                     fw.astype(np.float64), positions=(pos[0], t_all))
+        spread_g = np.maximum(spread_g, np.abs(g2 - ref_gf))
+        spread_l = max(spread_l, abs(l2 - ref_loss))
+    scale = np.abs(ref_gf).max()
+    print(f"[train coarse+fine] coarse grad err {np.abs(gc - ref_gc).max() / np.abs(ref_gc).max():.2e}, "
+          f"fine grad err {np.abs(gf - ref_gf).max() / scale:.2e}, "
+          f"fine spread {spread_g.max() / scale:.2e}")
+    bound = np.maximum(REL * scale, 3.0 * spread_g) + 1e-9
+    assert (np.abs(gf - ref_gf) <= bound).all(), np.abs(gf - ref_gf).max() / scale
+    assert abs(loss - ref_loss) <= max(1e-5 * ref_loss, 3.0 * spread_l)
+
+
+def test_loss_grad_rejects_bf16_and_bad_arguments(torch):
+    import ctypes
+    import neural_radiance_field_b200 as nb
+    from neural_radiance_field_b200 import _capi
+    rnd = nb.Renderer(precision=S.PREC_BF16, max_rays=16, max_samples=192)
+    p = rnd.params()
+    fake = ctypes.c_void_p(16)
+    st = _capi.lib().nerf_loss_grad(rnd.ctx, fake, fake, 4, 2.0, 6.0, 64, 0, ctypes.byref(p),
+                                    fake, fake, fake, None, None)
+    assert st == _capi.NERF_ERR_UNSUPPORTED
+    rnd.close()
+    rnd = nb.Renderer(precision=S.PREC_FP32, max_rays=16, max_samples=192)
+    p = rnd.params()
+    st = _capi.lib().nerf_loss_grad(rnd.ctx, fake, fake, 4, 2.0, 6.0, 64, 128, ctypes.byref(p),
+                                    fake, fake, fake, None, None)
+    assert st == _capi.NERF_ERR_INVALID_ARG        # fine pass without grad_fine / weights
+    rnd.close()
