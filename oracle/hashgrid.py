@@ -112,6 +112,20 @@ class HashGrid3D:
             feats.append((wts[:, :, None] * table[rows]).sum(axis=1))
         return np.concatenate(feats, axis=1)
 
+    def encode_backward(self, x, d_feat):
+        """Gradient of sum(d_feat * encode(x, table)) with respect to the table:
+        every point adds, at each level, weight * d_feat[level] to each of its
+        8 corner rows (the encoding is linear in the table, so this is its
+        adjoint: the scatter-add that trains the grid, Instant-NGP notebook,
+        Experiment 1, made 3D). d_feat [P, L*F]; returns [n_entries, F] fp64."""
+        d_feat = np.asarray(d_feat, dtype=np.float64)
+        grad = np.zeros((self.n_entries, self.F), dtype=np.float64)
+        for level in range(self.L):
+            rows, wts = self.corners(x, level)
+            g = d_feat[:, level * self.F:(level + 1) * self.F]
+            np.add.at(grad, rows.ravel(), (wts[:, :, None] * g[:, None, :]).reshape(-1, self.F))
+        return grad
+
 
 class HashGrid2D:
     """The notebook's 2D grid over [0,1]^2 (used for the printed pins)."""
