@@ -540,6 +540,62 @@ def run_train(args, rank, world, local_rank):
     print(json.dumps(line), flush=True)
 
 
+def run_hash_backward(args, rank, world, local_rank):
+    """One step = the hash-grid encoding's backward (the scatter-add that trains
+    the grid) for 2^22 points drawn from the occupied voxels' region of the
+    hash-grid workload, in both summation modes. An extra line."""
+    import torch
+    import neural_radiance_field_b200 as nb
+    from neural_radiance_field_b200 import build as nbuild
+    nbuild.build()
+    torch.cuda.set_device(local_rank)
+    n = 1 << 22
+    gen = torch.Generator(device="cpu").manual_seed(5)
+    x = (torch.rand(n, 3, generator=gen) * 3.0 - 1.5).cuda()
+    g = torch.randn(n, 32, generator=gen).cuda()
+    grad = torch.zeros(S.HASH_ENTRIES, 2, device="cuda")
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    stream = torch.cuda.current_stream()
+    res = {}
+    with ClockSampler(local_rank) as clk:
+        for det in (False, True):
+            for _ in range(args.warmup):
+                nb.nerf_hash_encode_backward(x, g, grad, deterministic=det)
+            torch.cuda.synchronize()
+            ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                  for _ in range(args.steps)]
+            for k in range(args.steps):
+                flush.fill_(k & 0xFF)
+                ev[k][0].record(stream)
+                nb.nerf_hash_encode_backward(x, g, grad, deterministic=det)
+                ev[k][1].record(stream)
+            torch.cuda.synchronize()
+            res[det] = sum(a.elapsed_time(b) for a, b in ev) / args.steps
+    peaks, peak_kind = load_peaks()
+    # algorithmic bytes per point: x (12 B) and d_feat (128 B) read, 16 levels x
+    # 8 corners x 2 features of 4-byte read-modify-write in the gradient table
+    bytes_pt = 12 + 128 + 16 * 8 * 2 * 4 * 2
+    hbm = peaks.get("hbm_gbs")
+    achieved = n * bytes_pt / (res[False] * 1e-3) / 1e9
+    line = {"metric": "points/sec, hash-grid encoding backward (scatter-add into the tables), fp32 atomics",
+            "value": n / (res[False] * 1e-3), "unit": "points/s", "n_gpus": 1, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": res[False], "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": "hash_backward_4M_points", "points": n,
+                       "table_rows": S.HASH_ENTRIES,
+                       "l2": "flushed between timed steps (256 MiB write)"},
+            "deterministic_mode": {"ms_per_step": res[True], "points_per_s": n / (res[True] * 1e-3),
+                                   "summation": "int64 fixed point, bit-identical across runs"},
+            "roofline": {"bound": "hbm", "kernel": "hash_bw_kernel (fp32 atomics)",
+                         "achieved": achieved, "peak": hbm, "unit": "GB/s",
+                         "frac": achieved / hbm if hbm else None,
+                         "peak_kind": f"HBM copy, {peak_kind}; the 48.8 MB gradient table is "
+                                      "L2-resident, so its atomics resolve in L2",
+                         "traffic": None, "bytes_per_point": bytes_pt},
+            "gpu_launches": None, "clocks": clk.summary()}
+    print(json.dumps(line), flush=True)
+
+
 def run_march(args, rank, world, local_rank):
     """One step = ray generation + a full-frame march render of the KiloNeRF or
     hash-grid workload (occupancy skipping, scene function, compositing)."""
@@ -650,7 +706,8 @@ def main():
     ap.add_argument("--ref-rays", type=int, default=128)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--workload", default=WORKLOAD,
-                    choices=[WORKLOAD, "kilonerf", "hashgrid", "sweep24", "compact", "train"],
+                    choices=[WORKLOAD, "kilonerf", "hashgrid", "sweep24", "compact", "train",
+                             "hash_backward"],
                     help="the benchmark workload (default) or a march workload (extra lines)")
     ap.add_argument("--traffic-bytes", type=float, default=0.0,
                     help="DRAM bytes per network launch from an ncu capture of this kernel")
@@ -668,6 +725,8 @@ def main():
         run_compact(args, rank, world, local_rank)
     elif args.workload == "train":
         run_train(args, rank, world, local_rank)
+    elif args.workload == "hash_backward":
+        run_hash_backward(args, rank, world, local_rank)
     elif args.workload != WORKLOAD:
         run_march(args, rank, world, local_rank)
     else:

@@ -286,6 +286,24 @@ NERF_API nerf_status nerf_test_route_cells(const float* x, int64_t n, int32_t* o
 NERF_API nerf_status nerf_test_hash_encode(const float* x, int64_t n, const uint16_t* hash_table,
                                            float* out_feat, int32_t* out_rows, void* stream);
 
+/* Backward of the hash-grid encoding above, the scatter-add that trains the
+ * grid (Instant-NGP notebook, Experiment 1, in 3D): for every point and level,
+ * d_feat[point][2 l + f] * (corner weight) is added to grad_table[row][f] for
+ * each of the level's 8 corner rows (the same rows and trilinear weights as
+ * nerf_test_hash_encode). x [n][3] and d_feat [n][32] fp32 device;
+ * grad_table: device fp32 [6,101,902][2], ACCUMULATED into (zero it first).
+ * deterministic = 0: fp32 atomics, whose summation order (hence the last bits)
+ * varies from run to run. deterministic = 1: every term is rounded to a
+ * multiple of 2^-E, E = 62 - ceil(log2(n * max|d_feat|)), and summed as int64
+ * (associative, so bit-identical across runs; no sum can overflow since a
+ * point's 8 weights per level add to 1), then converted and added; this mode
+ * allocates 97.6 MB of stream-ordered scratch (cudaMallocAsync) per call.
+ * Enqueued on `stream`; does not synchronise. Errors: NERF_ERR_INVALID_ARG
+ * (NULL pointer, n <= 0), NERF_ERR_CUDA. */
+NERF_API nerf_status nerf_hash_encode_backward(const float* x, int64_t n, const float* d_feat,
+                                               float* grad_table, int deterministic,
+                                               void* stream);
+
 /* Real spherical harmonics of bands 0..3 (16 values, index l*l + l + m, no
  * Condon-Shortley phase) of the unit vectors d/|d|; d [P][3], out [P][16]. */
 NERF_API nerf_status nerf_test_sh(const float* d, int64_t n, float* out, void* stream);

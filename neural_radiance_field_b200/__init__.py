@@ -14,7 +14,7 @@ from ._capi import (NERF_BF16, NERF_FP32, NERF_LAST_1E10, NERF_LAST_TO_FAR, NERF
                     NERF_MODEL_KILONERF, NERF_MODEL_MLP, NERF_SIGMA_RELU, NERF_SIGMA_SOFTPLUS,
                     NerfError, nerf_config, nerf_params)
 
-__all__ = ["Renderer", "nerf_raygen", "nerf_raygen_batch", "nerf_test_stratified", "nerf_test_pe",
+__all__ = ["Renderer", "nerf_raygen", "nerf_raygen_batch", "nerf_hash_encode_backward", "nerf_test_stratified", "nerf_test_pe",
            "nerf_test_composite", "nerf_test_sample_pdf", "NerfError", "nerf_config",
            "nerf_params"]
 
@@ -107,6 +107,13 @@ def nerf_test_route_cells(x, out_cell, out_cell_count, out_cell_offset, out_orde
 def nerf_test_hash_encode(x, hash_table, out_feat, out_rows=None, stream=None):
     _capi.check(_capi.lib().nerf_test_hash_encode(
         _ptr(x), x.shape[0], _ptr(hash_table), _ptr(out_feat), _ptr(out_rows), _stream(stream)))
+
+
+def nerf_hash_encode_backward(x, d_feat, grad_table, deterministic=False, stream=None):
+    """Scatter-add of encoding gradients into grad_table (accumulated); see the header."""
+    _capi.check(_capi.lib().nerf_hash_encode_backward(_ptr(x), x.shape[0], _ptr(d_feat),
+                                                      _ptr(grad_table), int(bool(deterministic)),
+                                                      _stream(stream)))
 
 
 def nerf_test_sh(d, out, stream=None):

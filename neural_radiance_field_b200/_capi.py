@@ -74,6 +74,7 @@ SIGNATURES = {
     "nerf_test_march": (_I, [_P, _P, _I64, _F, _F, _I, _P, _P, _P, _P]),
     "nerf_test_route_cells": (_I, [_P, _I64, _P, _P, _P, _P, _P]),
     "nerf_test_hash_encode": (_I, [_P, _I64, _P, _P, _P, _P]),
+    "nerf_hash_encode_backward": (_I, [_P, _I64, _P, _P, _I, _P]),
     "nerf_test_sh": (_I, [_P, _I64, _P, _P]),
     "nerf_test_bounded_wait": (_I, [ctypes.c_uint32, _P, _P, _P]),
     "nerf_march_compact_noalloc": (_I, [_P, _P, _I64, _F, _F, _I, _P, _P, _P, _P]),

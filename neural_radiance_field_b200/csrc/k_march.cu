@@ -219,6 +219,101 @@ __device__ __forceinline__ void hash_encode_point(const __half2* __restrict__ ta
   for (int l = 0; l < 16; ++l) hash_encode_level(table, u0, u1, u2, l, rows_out, feat[2 * l], feat[2 * l + 1]);
 }
 
+// Backward of the encoding (its adjoint): every point adds, at each level,
+// weight * d_feat[level] to each of its 8 corner rows, the same rows and
+// trilinear weights as hash_encode_level computes. Two ways to sum:
+//   fp32 atomics (fast; the summation order, hence the last bits, varies), or
+//   fixed point: each term rounded to a multiple of 2^-E and added as int64 with
+//   2's-complement atomics, which are associative, so the result does not
+//   depend on the order. E = 62 - ceil(log2(n max|d_feat|)): a row's sum of
+//   |weight * g| is at most n max|g| (a point's 8 weights per level sum to 1),
+//   so no sum can overflow.
+template <bool FIXED>
+__device__ __forceinline__ void hash_level_scatter(float u0, float u1, float u2, int l, float g0,
+                                                   float g1, float* grad,
+                                                   unsigned long long* acc, double scale) {
+  const int N = c_hres[l];
+  const float fN = (float)N;
+  const float c0 = fmul(u0, fN), c1 = fmul(u1, fN), c2 = fmul(u2, fN);
+  const float f0 = floorf(c0), f1 = floorf(c1), f2 = floorf(c2);
+  const float w0 = fsub(c0, f0), w1 = fsub(c1, f1), w2 = fsub(c2, f2);
+  const int i0 = (int)f0, i1 = (int)f1, i2 = (int)f2;
+#pragma unroll
+  for (int corner = 0; corner < 8; ++corner) {
+    const int dx = corner >> 2, dy = (corner >> 1) & 1, dz = corner & 1;
+    const int ix = min(max(i0 + dx, 0), N), iy = min(max(i1 + dy, 0), N),
+              iz = min(max(i2 + dz, 0), N);
+    uint32_t idx;
+    if (c_hdirect[l]) {
+      idx = (uint32_t)((ix * (N + 1) + iy) * (N + 1) + iz);
+    } else {
+      idx = ((uint32_t)ix ^ ((uint32_t)iy * 2654435761u) ^ ((uint32_t)iz * 805459861u)) &
+            ((1u << 19) - 1u);
+    }
+    const int64_t row = (int64_t)c_hoff[l] + (int64_t)idx;
+    const float wx = dx ? w0 : 1.0f - w0;
+    const float wy = dy ? w1 : 1.0f - w1;
+    const float wz = dz ? w2 : 1.0f - w2;
+    const float wt = wx * wy * wz;
+    if (FIXED) {
+      atomicAdd(acc + 2 * row, (unsigned long long)__double2ll_rn((double)wt * (double)g0 * scale));
+      atomicAdd(acc + 2 * row + 1,
+                (unsigned long long)__double2ll_rn((double)wt * (double)g1 * scale));
+    } else {
+      atomicAdd(grad + 2 * row, wt * g0);
+      atomicAdd(grad + 2 * row + 1, wt * g1);
+    }
+  }
+}
+
+__device__ __forceinline__ double hash_fixed_scale(float max_abs, int64_t n) {
+  return ldexp(1.0, 62 - (int)ceil(log2((double)n * (double)max_abs)));
+}
+
+template <bool FIXED>
+__global__ void hash_bw_kernel(const float* __restrict__ x, int64_t n,
+                               const float* __restrict__ d_feat, float* __restrict__ grad,
+                               unsigned long long* __restrict__ acc,
+                               const unsigned* __restrict__ max_bits) {
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= n) return;
+  double scale = 0.0;
+  if (FIXED) {
+    const float mx = __uint_as_float(*max_bits);
+    if (!(mx > 0.0f)) return;
+    scale = hash_fixed_scale(mx, n);
+  }
+  float u0, u1, u2;
+  hash_unit_coords(x[i * 3], x[i * 3 + 1], x[i * 3 + 2], u0, u1, u2);
+#pragma unroll 2
+  for (int l = 0; l < 16; ++l)
+    hash_level_scatter<FIXED>(u0, u1, u2, l, d_feat[i * 32 + 2 * l], d_feat[i * 32 + 2 * l + 1],
+                              grad, acc, scale);
+}
+
+// max |v| over m values, as the bits of a non-negative float (which order like
+// unsigned integers), into *out (zeroed by the caller).
+__global__ void absmax_kernel(const float* __restrict__ v, int64_t m, unsigned* __restrict__ out) {
+  float mx = 0.0f;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < m;
+       i += (int64_t)gridDim.x * blockDim.x)
+    mx = fmaxf(mx, fabsf(v[i]));
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+  if ((threadIdx.x & 31) == 0) atomicMax(out, __float_as_uint(mx));
+}
+
+__global__ void fixed_to_grad_kernel(const unsigned long long* __restrict__ acc, int64_t m,
+                                     const unsigned* __restrict__ max_bits, int64_t n,
+                                     float* __restrict__ grad) {
+  const float mx = __uint_as_float(*max_bits);
+  if (!(mx > 0.0f)) return;
+  const double inv = 1.0 / hash_fixed_scale(mx, n);
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < m;
+       i += (int64_t)gridDim.x * blockDim.x)
+    grad[i] += (float)((double)(long long)acc[i] * inv);
+}
+
 __global__ void hash_encode_kernel(const float* __restrict__ x, int64_t n,
                                    const __half2* __restrict__ table, float* __restrict__ feat,
                                    int32_t* __restrict__ rows) {
@@ -845,6 +940,31 @@ cudaError_t launch_hash_encode(const float* x, int64_t n, const uint16_t* table,
   hash_encode_kernel<<<(unsigned)((n + 127) / 128), 128, 0, st>>>(
       x, n, reinterpret_cast<const __half2*>(table), feat, rows);
   return cudaGetLastError();
+}
+
+cudaError_t launch_hash_encode_backward(const float* x, int64_t n, const float* d_feat,
+                                       float* grad, int deterministic, cudaStream_t st) {
+  const unsigned blocks = (unsigned)((n + 127) / 128);
+  if (!deterministic) {
+    hash_bw_kernel<false><<<blocks, 128, 0, st>>>(x, n, d_feat, grad, nullptr, nullptr);
+    return cudaGetLastError();
+  }
+  const int64_t m = 2 * hash_grid_info().entries;
+  unsigned long long* acc = nullptr;
+  unsigned* mx = nullptr;
+  cudaError_t e = cudaMallocAsync((void**)&acc, m * sizeof(unsigned long long), st);
+  if (e == cudaSuccess) e = cudaMallocAsync((void**)&mx, sizeof(unsigned), st);
+  if (e == cudaSuccess) e = cudaMemsetAsync(acc, 0, m * sizeof(unsigned long long), st);
+  if (e == cudaSuccess) e = cudaMemsetAsync(mx, 0, sizeof(unsigned), st);
+  if (e == cudaSuccess) {
+    absmax_kernel<<<1024, 256, 0, st>>>(d_feat, n * 32, mx);
+    hash_bw_kernel<true><<<blocks, 128, 0, st>>>(x, n, d_feat, nullptr, acc, mx);
+    fixed_to_grad_kernel<<<2048, 256, 0, st>>>(acc, m, mx, n, grad);
+    e = cudaGetLastError();
+  }
+  if (acc) cudaFreeAsync(acc, st);
+  if (mx) cudaFreeAsync(mx, st);
+  return e;
 }
 
 cudaError_t launch_sh(const float* d, int64_t n, float* out, cudaStream_t st) {

@@ -670,6 +670,16 @@ nerf_status nerf_test_hash_encode(const float* x, int64_t n, const uint16_t* has
   return NERF_OK;
 }
 
+nerf_status nerf_hash_encode_backward(const float* x, int64_t n, const float* d_feat,
+                                      float* grad_table, int deterministic, void* stream) {
+  if (!x || !d_feat || !grad_table || n <= 0 || n > (int64_t(1) << 40))
+    return fail(nullptr, NERF_ERR_INVALID_ARG, "nerf_hash_encode_backward: bad argument");
+  NERF_CHECK_LAUNCH(nullptr, march_prepare(nullptr));
+  NERF_CHECK_LAUNCH(nullptr, launch_hash_encode_backward(x, n, d_feat, grad_table, deterministic,
+                                                         (cudaStream_t)stream));
+  return NERF_OK;
+}
+
 nerf_status nerf_test_sh(const float* d, int64_t n, float* out, void* stream) {
   if (!d || !out || n <= 0) return fail(nullptr, NERF_ERR_INVALID_ARG, "nerf_test_sh: bad argument");
   NERF_CHECK_LAUNCH(nullptr, launch_sh(d, n, out, (cudaStream_t)stream));

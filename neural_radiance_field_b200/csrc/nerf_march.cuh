@@ -66,6 +66,8 @@ cudaError_t launch_march_mask(const float* o, const float* d, int64_t R, float n
 cudaError_t launch_route_points(const float* x, int64_t n, int32_t* cell, int32_t* hist,
                                 int32_t* off, int32_t* order, int32_t* fill, int32_t* scan_tmp,
                                 unsigned* flag, cudaStream_t st);
+cudaError_t launch_hash_encode_backward(const float* x, int64_t n, const float* d_feat,
+                                       float* grad, int deterministic, cudaStream_t st);
 cudaError_t launch_hash_encode(const float* x, int64_t n, const uint16_t* table, float* feat,
                                int32_t* rows, cudaStream_t st);
 cudaError_t launch_sh(const float* d, int64_t n, float* out, cudaStream_t st);
