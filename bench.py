@@ -605,6 +605,9 @@ def run_march(args, rank, world, local_rank):
     nbuild.build()
     torch.cuda.set_device(local_rank)
     wl = S.WORKLOADS[args.workload]
+    if args.size:
+        import dataclasses
+        wl = dataclasses.replace(wl, H=args.size, W=args.size, focal=1.25 * args.size)
     c2w = wl.c2w().ravel().tolist()
     R = wl.n_rays
     packed, _ = S.occupancy_grid(wl.seed)
