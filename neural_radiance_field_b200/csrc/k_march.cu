@@ -703,28 +703,37 @@ kilo_eval_kernel(const float* __restrict__ o, const float* __restrict__ d, int64
   float* rgbv = ks + KT_RGB;
   const int p = threadIdx.x & (KT_P - 1);
   const int part = threadIdx.x / KT_P;          // 0: position encoding, 1: direction encoding
+  // a contiguous run of items per CTA: the items are in cell order, so
+  // consecutive items mostly share a cell and its weights stay staged
   const int NI = *n_items;
-  for (int it = blockIdx.x; it < NI; it += gridDim.x) {
+  const int per = (NI + (int)gridDim.x - 1) / (int)gridDim.x;
+  const int it0 = (int)blockIdx.x * per;
+  const int it1 = min(NI, it0 + per);
+  int staged = -1;
+  for (int it = it0; it < it1; ++it) {
     const int4 item = items[it];
     const int n = item.z;
     __syncthreads();     // the previous item's last reads are over
-    // this cell's weights (row-major W[n][k] in the blob) -> Wt[k][n], in two
-    // bank-conflict-free steps through the (idle) activation buffer: a
-    // coalesced copy (W2 rows padded to 33), then a transpose with lanes along n
-    const float* W = cell_w + (int64_t)item.x * KILO_NP;
-    float* tmp = act;
-    for (int q = threadIdx.x; q < KILO_NP; q += KT_THREADS) {
-      const float v = __ldg(W + q);
-      if (q < KT_B1) tmp[q] = v;
-      else if (q < KT_W2) b1[q - KT_B1] = v;
-      else if (q < KT_B2) { const int z = q - KT_W2; tmp[KT_B1 + (z / 32) * 33 + z % 32] = v; }
-      else ks[q] = v;                               // b2, ws, bs, wc, bc in place
+    if (item.x != staged) {
+      // this cell's weights (row-major W[n][k] in the blob) -> Wt[k][n], in two
+      // bank-conflict-free steps through the (idle) activation buffer: a
+      // coalesced copy (W2 rows padded to 33), then a transpose with lanes along n
+      staged = item.x;
+      const float* W = cell_w + (int64_t)item.x * KILO_NP;
+      float* tmp = act;
+      for (int q = threadIdx.x; q < KILO_NP; q += KT_THREADS) {
+        const float v = __ldg(W + q);
+        if (q < KT_B1) tmp[q] = v;
+        else if (q < KT_W2) b1[q - KT_B1] = v;
+        else if (q < KT_B2) { const int z = q - KT_W2; tmp[KT_B1 + (z / 32) * 33 + z % 32] = v; }
+        else ks[q] = v;                               // b2, ws, bs, wc, bc in place
+      }
+      __syncthreads();
+      for (int t = threadIdx.x; t < 63 * 32; t += KT_THREADS) w1t[t] = tmp[(t % 32) * 63 + t / 32];
+      for (int t = threadIdx.x; t < 32 * 32; t += KT_THREADS)
+        w2t[t] = tmp[KT_B1 + (t % 32) * 33 + t / 32];
+      __syncthreads();   // the transpose's reads of the activation buffer are over
     }
-    __syncthreads();
-    for (int t = threadIdx.x; t < 63 * 32; t += KT_THREADS) w1t[t] = tmp[(t % 32) * 63 + t / 32];
-    for (int t = threadIdx.x; t < 32 * 32; t += KT_THREADS)
-      w2t[t] = tmp[KT_B1 + (t % 32) * 33 + t / 32];
-    __syncthreads();     // the transpose's reads of the activation buffer are over
     int64_t i = 0;
     if (p < n) i = order[item.y + p];
     {
