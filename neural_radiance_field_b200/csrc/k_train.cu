@@ -13,6 +13,8 @@
 //                        split-row tiled reduction added atomically into the
 //                        gradient blob (fp32 atomics: the summation order, not
 //                        the terms, varies between runs)
+#include <algorithm>
+
 #include "nerf_internal.cuh"
 
 namespace nerfb {
@@ -156,111 +158,336 @@ __global__ void head_bw_kernel(const float* __restrict__ d_raw, const float* __r
   dz[q] = save[row * ldc + hcol + j] > 0.0f ? v : 0.0f;
 }
 
-// out[r][k] = (sum_n A[r][n] B[n][k] + ea[r] ev[k]) * (mask: save[r][mcol + k] > 0),
-// k < Kout (a multiple of 64), n < N (a multiple of 16). 64 x 64 tiles, 4 x 4 per thread.
-__global__ void __launch_bounds__(256)
-in_bw_kernel(const float* __restrict__ A, int64_t lda, const float* __restrict__ B, int64_t ldb,
-             int N, int Kout, int64_t rows, const float* __restrict__ ea, int64_t ldea,
-             const float* __restrict__ ev, const float* __restrict__ save, int64_t ldc, int mcol,
-             float* __restrict__ out, int64_t ldo) {
-  __shared__ __align__(16) float As[16][64 + 4];   // [n][row]
-  __shared__ __align__(16) float Bs[16][64];       // [n][k]
-  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
-  const int64_t r0 = (int64_t)blockIdx.x * 64;
-  const int k0 = blockIdx.y * 64;
-  float acc[4][4] = {};
-  for (int n0 = 0; n0 < N; n0 += 16) {
-    for (int q = threadIdx.x; q < 64 * 16; q += 256) {     // A tile, transposed into As[n][row]
-      const int rr = q / 16, nn = q % 16;
-      const int64_t row = r0 + rr;
-      As[nn][rr] = row < rows ? A[row * lda + n0 + nn] : 0.0f;
-    }
-    for (int q = threadIdx.x; q < 16 * 64; q += 256) {
-      const int nn = q / 64, kk = q % 64;
-      Bs[nn][kk] = __ldg(B + (int64_t)(n0 + nn) * ldb + k0 + kk);
-    }
-    __syncthreads();
+// ---------------------------------------------------------------------------
+// Register-blocked fp32 GEMM core. A CTA of 256 threads computes a 128 x 128
+// output tile; thread (ty, tx) = (tid / 16, tid % 16) owns rows
+// {4 ty + i, 64 + 4 ty + i} and columns {4 tx + j, 64 + 4 tx + j}, i, j < 4 (8 x 8
+// accumulators). The reduction runs in steps of 8 through a shared-memory
+// double buffer: the next step's operands are fetched into registers while the
+// current step computes, so a step costs one barrier. Each output accumulates
+// its terms in reduction order with fmaf.
+// ---------------------------------------------------------------------------
+constexpr int GT = 128;          // tile edge
+constexpr int GK = 8;            // reduction step
+constexpr int GLD = GT + 4;      // padded row of a shared operand tile
+
+struct GemmSmem {
+  float a[2][GK][GLD];   // [step][reduction index][tile row]
+  float b[2][GK][GLD];   // [step][reduction index][tile column]
+};
+
+__device__ __forceinline__ void gemm_step(const float (&a)[GK][GLD], const float (&b)[GK][GLD],
+                                          float (&acc)[8][8], int ty, int tx) {
 #pragma unroll
-    for (int nn = 0; nn < 16; ++nn) {
-      const float4 a = *reinterpret_cast<const float4*>(&As[nn][4 * ty]);
-      const float4 w = *reinterpret_cast<const float4*>(&Bs[nn][4 * tx]);
-      const float av[4] = {a.x, a.y, a.z, a.w}, wv[4] = {w.x, w.y, w.z, w.w};
+  for (int k = 0; k < GK; ++k) {
+    const float4 a0 = *reinterpret_cast<const float4*>(&a[k][4 * ty]);
+    const float4 a1 = *reinterpret_cast<const float4*>(&a[k][64 + 4 * ty]);
+    const float4 b0 = *reinterpret_cast<const float4*>(&b[k][4 * tx]);
+    const float4 b1 = *reinterpret_cast<const float4*>(&b[k][64 + 4 * tx]);
+    const float av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+    const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
 #pragma unroll
-      for (int i = 0; i < 4; ++i)
+    for (int i = 0; i < 8; ++i)
 #pragma unroll
-        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(av[i], wv[j], acc[i][j]);
-    }
-    __syncthreads();
-  }
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int64_t row = r0 + 4 * ty + i;
-    if (row >= rows) continue;
-    float v[4];
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int k = k0 + 4 * tx + j;
-      float x = acc[i][j];
-      if (ea) x = fmaf(ea[row * ldea], __ldg(ev + k), x);
-      if (save) x = save[row * ldc + mcol + k] > 0.0f ? x : 0.0f;
-      v[j] = x;
-    }
-    *reinterpret_cast<float4*>(out + row * ldo + k0 + 4 * tx) = make_float4(v[0], v[1], v[2], v[3]);
+      for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
   }
 }
 
-// G[n][k] += sum_r A[r][n] X(r, k) for n < N, k < K, and db[n] += sum_r A[r][n]
-// (the virtual column k = K of ones). X(r, k) = X[r * ldx + c0 + k] for k < split,
-// X[r * ldx + c1 + k - split] otherwise. Rows are cut into slices of WG_SLICE.
-constexpr int WG_SLICE = 4096;
-__global__ void __launch_bounds__(256)
-wgrad_kernel(const float* __restrict__ A, int64_t lda, int N, const float* __restrict__ X,
-             int64_t ldx, int c0, int split, int c1, int K, int64_t rows,
-             float* __restrict__ G, int64_t ldg, float* __restrict__ db) {
-  __shared__ __align__(16) float As[16][64];
-  __shared__ __align__(16) float Xs[16][64];
-  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
-  const int nb = blockIdx.x * 64, kb = blockIdx.y * 64;
-  const int64_t rs = (int64_t)blockIdx.z * WG_SLICE;
-  const int64_t re = rs + WG_SLICE < rows ? rs + WG_SLICE : rows;
-  float acc[4][4] = {};
-  for (int64_t r0 = rs; r0 < re; r0 += 16) {
-    for (int q = threadIdx.x; q < 16 * 64; q += 256) {
-      const int rr = q / 64, cc = q % 64;
-      const int64_t row = r0 + rr;
-      const int n = nb + cc, k = kb + cc;
-      As[rr][cc] = (row < re && n < N) ? A[row * lda + n] : 0.0f;
-      float xv = 0.0f;
-      if (row < re) {
-        if (k < K) xv = X[row * ldx + (k < split ? c0 + k : c1 + k - split)];
-        else if (k == K) xv = 1.0f;
+// Four consecutive floats of a row: p[0..3] with element e valid when ok[e].
+__device__ __forceinline__ float4 load4(const float* p, bool vec, bool ok0, bool ok1, bool ok2,
+                                        bool ok3) {
+  if (vec && ok3) return __ldg(reinterpret_cast<const float4*>(p));
+  return make_float4(ok0 ? __ldg(p) : 0.f, ok1 ? __ldg(p + 1) : 0.f, ok2 ? __ldg(p + 2) : 0.f,
+                     ok3 ? __ldg(p + 3) : 0.f);
+}
+
+// out[r][c] = epi( sum_k A(r, k) B[k][c] ) for r < rows, c < n_out, where
+// A(r, k) = A[r * lda + a0 + k] for k < a_split, A[r * lda + a1 + k - a_split]
+// otherwise (a row made of two column ranges, as the skip layer's [h, gamma(x)]),
+// K a multiple of 8 with a_split a multiple of 8. The epilogue, in this order:
+// + bias[c]; + row_bias[(r / rb_div) * n_out + c]; + ea[r * ldea] ev[c] (fmaf);
+// ReLU; zero where mask[r * ldm + c] <= 0.
+struct RowGemm {
+  const float* A; int64_t lda; int a0, a_split, a1;
+  const float* B; int64_t ldb;
+  int K, n_out; int64_t rows;
+  const float* bias;
+  const float* row_bias; int rb_div;
+  const float* ea; int64_t ldea; const float* ev;
+  int relu;
+  const float* mask; int64_t ldm;
+  float* out; int64_t ldo;
+  int a_vec, b_vec;
+};
+
+__global__ void __launch_bounds__(256, 2) row_gemm_kernel(RowGemm g) {
+  __shared__ __align__(16) GemmSmem sm;
+  const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
+  const int64_t m0 = (int64_t)blockIdx.x * GT;
+  const int n0 = blockIdx.y * GT;
+  // operand fetch roles: A row (tid / 2), reduction offset 4 (tid % 2); B reduction
+  // index tid / 32, columns 4 (tid % 32)
+  const int64_t ar = m0 + (tid >> 1);
+  const int ak = (tid & 1) * 4;
+  const bool a_row_ok = ar < g.rows;
+  const int bk = tid >> 5, bc = n0 + (tid & 31) * 4;
+  auto fetch_a = [&](int k0) -> float4 {
+    const int k = k0 + ak;
+    const int col = k < g.a_split ? g.a0 + k : g.a1 + k - g.a_split;
+    return a_row_ok ? load4(g.A + ar * g.lda + col, g.a_vec, true, true, true, true)
+                    : make_float4(0.f, 0.f, 0.f, 0.f);
+  };
+  auto fetch_b = [&](int k0) -> float4 {
+    const float* p = g.B + (int64_t)(k0 + bk) * g.ldb + bc;
+    return load4(p, g.b_vec, bc < g.n_out, bc + 1 < g.n_out, bc + 2 < g.n_out, bc + 3 < g.n_out);
+  };
+  auto put = [&](int buf, float4 va, float4 vb) {
+    sm.a[buf][ak + 0][tid >> 1] = va.x;
+    sm.a[buf][ak + 1][tid >> 1] = va.y;
+    sm.a[buf][ak + 2][tid >> 1] = va.z;
+    sm.a[buf][ak + 3][tid >> 1] = va.w;
+    *reinterpret_cast<float4*>(&sm.b[buf][bk][(tid & 31) * 4]) = vb;
+  };
+  float acc[8][8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+#pragma unroll
+    for (int j = 0; j < 8; ++j) acc[i][j] = 0.0f;
+  put(0, fetch_a(0), fetch_b(0));
+  __syncthreads();
+  const int steps = g.K / GK;
+  for (int s = 0; s < steps; ++s) {
+    const int cur = s & 1;
+    float4 na = make_float4(0.f, 0.f, 0.f, 0.f), nb = na;
+    if (s + 1 < steps) { na = fetch_a((s + 1) * GK); nb = fetch_b((s + 1) * GK); }
+    gemm_step(sm.a[cur], sm.b[cur], acc, ty, tx);
+    if (s + 1 < steps) put(cur ^ 1, na, nb);
+    __syncthreads();
+  }
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int64_t row = m0 + (i < 4 ? 4 * ty + i : 64 + 4 * ty + i - 4);
+    if (row >= g.rows) continue;
+    const float* rb = g.row_bias ? g.row_bias + (row / g.rb_div) * g.n_out : nullptr;
+    const float e = g.ea ? g.ea[row * g.ldea] : 0.0f;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int c = n0 + 64 * h + 4 * tx;
+      if (c >= g.n_out) continue;
+      float v[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        float x = acc[i][4 * h + j];
+        if (g.bias) x += __ldg(g.bias + c + j);
+        if (rb) x += rb[c + j];
+        if (g.ea) x = fmaf(e, __ldg(g.ev + c + j), x);
+        if (g.relu) x = fmaxf(x, 0.0f);
+        if (g.mask) x = g.mask[row * g.ldm + c + j] > 0.0f ? x : 0.0f;
+        v[j] = x;
       }
-      Xs[rr][cc] = xv;
+      *reinterpret_cast<float4*>(g.out + row * g.ldo + c) = make_float4(v[0], v[1], v[2], v[3]);
     }
-    __syncthreads();
+  }
+}
+
+// G[n][k] += sum_r A[r * lda + n] X(r, k) for n < N, k < K, rows in slices of
+// `slice` (a multiple of 8), each slice's partial sums added atomically; the
+// CTAs of the first column tile also add db[n] += sum_r A[r][n]. X(r, k) =
+// X[r * ldx + x0 + k] for k < x_split, X[r * ldx + x1 + k - x_split] otherwise.
+struct WGrad {
+  const float* A; int64_t lda; int N;
+  const float* X; int64_t ldx; int x0, x_split, x1; int K;
+  int64_t rows, slice;
+  float* G; int64_t ldg; float* db;
+  int a_vec, x_vec;   // x_vec: X, ldx, x0, x1 and x_split all 16-byte / 4-float aligned
+};
+
+template <bool XV>   // X rows 16-byte aligned and the split a multiple of 4
+__global__ void __launch_bounds__(256, 2) wgrad_gemm_kernel(WGrad g) {
+  __shared__ __align__(16) GemmSmem sm;
+  const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
+  const int nb = blockIdx.x * GT, kb = blockIdx.y * GT;
+  const int64_t rs = (int64_t)blockIdx.z * g.slice;
+  const int64_t re = rs + g.slice < g.rows ? rs + g.slice : g.rows;
+  const int fr = tid >> 5, fc = (tid & 31) * 4;          // fetch role: row, 4 columns
+  const int an = nb + fc, xk = kb + fc;
+  // with XV, a thread's four X columns lie in one of the two ranges
+  const bool x_lo = xk < g.x_split;
+  const int xcol = x_lo ? g.x0 + xk : g.x1 + xk - g.x_split;
+  // this thread's fetch row, advanced by GK rows per step
+  int64_t fr_row = rs + fr;
+  const float* pa = g.A + fr_row * g.lda + an;
+  const float* px = g.X + fr_row * g.ldx;
+  const bool a_ok0 = an < g.N, a_ok1 = an + 1 < g.N, a_ok2 = an + 2 < g.N, a_ok3 = an + 3 < g.N;
+  auto fetch = [&](float4& va, float4& vx) {
+    va = make_float4(0.f, 0.f, 0.f, 0.f);
+    vx = va;
+    if (fr_row < re) {
+      va = load4(pa, g.a_vec, a_ok0, a_ok1, a_ok2, a_ok3);
+      if (XV) {
+        vx = load4(px + xcol, true, xk < g.K, xk + 1 < g.K, xk + 2 < g.K, xk + 3 < g.K);
+      } else {
+        float t[4];
 #pragma unroll
-    for (int rr = 0; rr < 16; ++rr) {
-      const float4 a = *reinterpret_cast<const float4*>(&As[rr][4 * ty]);
-      const float4 x = *reinterpret_cast<const float4*>(&Xs[rr][4 * tx]);
-      const float av[4] = {a.x, a.y, a.z, a.w}, xv[4] = {x.x, x.y, x.z, x.w};
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(av[i], xv[j], acc[i][j]);
+        for (int e = 0; e < 4; ++e) {
+          const int k = xk + e;
+          t[e] = k < g.K ? __ldg(px + (k < g.x_split ? g.x0 + k : g.x1 + k - g.x_split)) : 0.f;
+        }
+        vx = make_float4(t[0], t[1], t[2], t[3]);
+      }
     }
+    fr_row += GK;
+    pa += GK * g.lda;
+    px += GK * g.ldx;
+  };
+  auto put = [&](int buf, float4 va, float4 vx) {
+    *reinterpret_cast<float4*>(&sm.a[buf][fr][fc]) = va;
+    *reinterpret_cast<float4*>(&sm.b[buf][fr][fc]) = vx;
+  };
+  const bool bias_cta = g.db != nullptr && blockIdx.y == 0;
+  float bsum = 0.0f;
+  float acc[8][8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+#pragma unroll
+    for (int j = 0; j < 8; ++j) acc[i][j] = 0.0f;
+  float4 va, vx;
+  fetch(va, vx);
+  put(0, va, vx);
+  __syncthreads();
+  const int steps = (int)((re - rs + GK - 1) / GK);
+  for (int s = 0; s < steps; ++s) {
+    const int cur = s & 1;
+    const bool more = s + 1 < steps;
+    if (more) fetch(va, vx);
+    gemm_step(sm.a[cur], sm.b[cur], acc, ty, tx);
+    if (bias_cta && tid < GT) {
+#pragma unroll
+      for (int k = 0; k < GK; ++k) bsum += sm.a[cur][k][tid];
+    }
+    if (more) put(cur ^ 1, va, vx);
     __syncthreads();
   }
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int n = nb + 4 * ty + i;
-    if (n >= N) continue;
+  for (int i = 0; i < 8; ++i) {
+    const int n = nb + (i < 4 ? 4 * ty + i : 64 + 4 * ty + i - 4);
+    if (n >= g.N) continue;
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int k = kb + 4 * tx + j;
-      if (k < K) atomicAdd(G + (int64_t)n * ldg + k, acc[i][j]);
-      else if (k == K && db) atomicAdd(db + n, acc[i][j]);
+    for (int j = 0; j < 8; ++j) {
+      const int k = kb + (j < 4 ? 4 * tx + j : 64 + 4 * tx + j - 4);
+      if (k < g.K) atomicAdd(g.G + (int64_t)n * g.ldg + k, acc[i][j]);
     }
   }
+  if (bias_cta && tid < GT && nb + tid < g.N) atomicAdd(g.db + nb + tid, bsum);
+}
+
+// The weight gradient of a head with N <= 4 outputs (sigma: 1, rgb: 3): one
+// thread per input column k (and k = K for the bias), summing over a slice of
+// rows; the reads of X are coalesced across the threads.
+template <int NS>
+__global__ void __launch_bounds__(128)
+wgrad_head_kernel(const float* __restrict__ A, int64_t lda, const float* __restrict__ X,
+                  int64_t ldx, int x0, int K, int64_t rows, int64_t slice, float* __restrict__ G,
+                  int64_t ldg, float* __restrict__ db) {
+  const int k = blockIdx.x * blockDim.x + threadIdx.x;
+  if (k > K) return;
+  const int64_t rs = (int64_t)blockIdx.y * slice;
+  const int64_t re = rs + slice < rows ? rs + slice : rows;
+  float acc[NS];
+#pragma unroll
+  for (int n = 0; n < NS; ++n) acc[n] = 0.0f;
+  for (int64_t r = rs; r < re; ++r) {
+    const float x = k < K ? X[r * ldx + x0 + k] : 1.0f;
+#pragma unroll
+    for (int n = 0; n < NS; ++n) acc[n] = fmaf(A[r * lda + n], x, acc[n]);
+  }
+#pragma unroll
+  for (int n = 0; n < NS; ++n) {
+    if (k < K) atomicAdd(G + (int64_t)n * ldg + k, acc[n]);
+    else atomicAdd(db + n, acc[n]);
+  }
+}
+
+// gamma(x) of every row into columns 0..63 of the activation store (the 64th
+// is zero), x = o + t d with t from the sample source: the operations and
+// rounding of the fused forward kernel's prologue.
+__global__ void encode_store_kernel(const float* __restrict__ o, const float* __restrict__ d,
+                                    int64_t R, SampleSpec ss, float* __restrict__ save,
+                                    int64_t ldc) {
+  const int64_t row = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (row >= R * ss.S) return;
+  float x[3];
+  if (ss.mode == SAMPLES_GIVEN_X) {
+    x[0] = ss.t[row * 3 + 0]; x[1] = ss.t[row * 3 + 1]; x[2] = ss.t[row * 3 + 2];
+  } else {
+    const int64_t ray = row / ss.S;
+    const int s = (int)(row % ss.S);
+    float t;
+    if (ss.mode == SAMPLES_STRATIFIED) {
+      const uint32_t m = ss.perturb ? draw_bits(ss.key, (uint64_t)ray, 0, (uint32_t)s) : 0u;
+      t = stratified_t(ss.near, ss.step, s, m, ss.perturb != 0);
+    } else {
+      t = ss.t[row];
+    }
+#pragma unroll
+    for (int c = 0; c < 3; ++c) x[c] = fadd(o[ray * 3 + c], fmul(t, d[ray * 3 + c]));
+  }
+  float v[64];
+  v[0] = x[0]; v[1] = x[1]; v[2] = x[2]; v[63] = 0.0f;
+#pragma unroll
+  for (int c = 0; c < 3; ++c)
+#pragma unroll
+    for (int k = 0; k < 10; ++k) {
+      float sn, cs;
+      pe_sincos(x[c], k, &sn, &cs);
+      v[3 + c * 10 + k] = sn;
+      v[33 + c * 10 + k] = cs;
+    }
+  float* out = save + row * ldc;
+#pragma unroll
+  for (int q = 0; q < 16; ++q)
+    *reinterpret_cast<float4*>(out + 4 * q) = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2],
+                                                          v[4 * q + 3]);
+}
+
+// raw[row] = (rgb, sigma): sigma = h_{D-1} . w_sigma + b_sigma, rgb_c = h_dir .
+// W_rgb[c] + b_rgb[c] (no activation: the raw outputs). One warp per row.
+__global__ void heads_fwd_kernel(const float* __restrict__ save, int64_t ldc, int hcol, int dcol,
+                                 int W, const float* __restrict__ pk, PackedFp32 p, int64_t rows,
+                                 float* __restrict__ raw) {
+  const int64_t row = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (row >= rows) return;
+  const float* h = save + row * ldc + hcol;
+  const float* hd = save + row * ldc + dcol;
+  float sg = 0.f, c0 = 0.f, c1 = 0.f, c2 = 0.f;
+  for (int k = 4 * lane; k < W; k += 128) {
+    const float4 a = *reinterpret_cast<const float4*>(h + k);
+    const float4 w = __ldg(reinterpret_cast<const float4*>(pk + p.sigma_w + k));
+    sg = fmaf(a.x, w.x, sg); sg = fmaf(a.y, w.y, sg); sg = fmaf(a.z, w.z, sg); sg = fmaf(a.w, w.w, sg);
+  }
+  const int Wh = W / 2;
+  for (int k = 4 * lane; k < Wh; k += 128) {
+    const float4 a = *reinterpret_cast<const float4*>(hd + k);
+    const float av[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      c0 = fmaf(av[e], __ldg(pk + p.rgb_w + k + e), c0);
+      c1 = fmaf(av[e], __ldg(pk + p.rgb_w + Wh + k + e), c1);
+      c2 = fmaf(av[e], __ldg(pk + p.rgb_w + 2 * Wh + k + e), c2);
+    }
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) {
+    sg += __shfl_xor_sync(0xffffffffu, sg, off);
+    c0 += __shfl_xor_sync(0xffffffffu, c0, off);
+    c1 += __shfl_xor_sync(0xffffffffu, c1, off);
+    c2 += __shfl_xor_sync(0xffffffffu, c2, off);
+  }
+  if (lane == 0)
+    *reinterpret_cast<float4*>(raw + row * 4) =
+        make_float4(c0 + __ldg(pk + p.rgb_b), c1 + __ldg(pk + p.rgb_b + 1),
+                    c2 + __ldg(pk + p.rgb_b + 2), sg + __ldg(pk + p.sigma_b));
 }
 
 // dz_ray[ray][j] = sum over the ray's samples of dz[ray * S + s][j].
@@ -311,6 +538,60 @@ __global__ void sum_kernel(const float* __restrict__ v, int64_t n, float* __rest
 
 unsigned blocks_for(int64_t n, int t) { return (unsigned)((n + t - 1) / t); }
 
+bool al16(const void* q) { return ((uintptr_t)q & 15u) == 0; }
+
+int sm_count() {
+  static int n = 0;
+  if (n == 0) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+      n = 148;
+  }
+  return n;
+}
+
+cudaError_t row_gemm(RowGemm g, cudaStream_t st) {
+  if (g.rows == 0) return cudaSuccess;
+  if (g.K % GK || g.a_split % GK || g.n_out % 4 || g.ldo % 4 || !al16(g.out))
+    return cudaErrorInvalidValue;
+  g.a_vec = al16(g.A) && g.lda % 4 == 0 && g.a0 % 4 == 0 && g.a1 % 4 == 0;
+  g.b_vec = al16(g.B) && g.ldb % 4 == 0;
+  row_gemm_kernel<<<dim3(blocks_for(g.rows, GT), blocks_for(g.n_out, GT)), 256, 0, st>>>(g);
+  return cudaGetLastError();
+}
+
+// Row slices sized for about two waves of two CTAs per SM, at least 512 rows each.
+int64_t slice_rows(int64_t rows, int tiles) {
+  const int64_t want = std::max<int64_t>(1, (4 * (int64_t)sm_count()) / tiles);
+  int64_t slice = (rows + want - 1) / want;
+  slice = (slice + GK - 1) / GK * GK;
+  return std::max<int64_t>(slice, 512);
+}
+
+cudaError_t wgrad(WGrad g, cudaStream_t st) {
+  if (g.rows == 0) return cudaSuccess;
+  g.a_vec = al16(g.A) && g.lda % 4 == 0;
+  g.x_vec = al16(g.X) && g.ldx % 4 == 0 && g.x0 % 4 == 0 && g.x1 % 4 == 0 && g.x_split % 4 == 0;
+  const unsigned tn = blocks_for(g.N, GT), tk = blocks_for(g.K, GT);
+  g.slice = slice_rows(g.rows, (int)(tn * tk));
+  const dim3 grid(tn, tk, blocks_for(g.rows, g.slice));
+  if (g.x_vec) wgrad_gemm_kernel<true><<<grid, 256, 0, st>>>(g);
+  else wgrad_gemm_kernel<false><<<grid, 256, 0, st>>>(g);
+  return cudaGetLastError();
+}
+
+template <int NS>
+cudaError_t wgrad_head(const float* A, int64_t lda, const float* X, int64_t ldx, int x0, int K,
+                       int64_t rows, float* G, int64_t ldg, float* db, cudaStream_t st) {
+  if (rows == 0) return cudaSuccess;
+  const unsigned bx = blocks_for(K + 1, 128);
+  const int64_t slice = slice_rows(rows, (int)bx);
+  wgrad_head_kernel<NS><<<dim3(bx, blocks_for(rows, slice)), 128, 0, st>>>(
+      A, lda, X, ldx, x0, K, rows, slice, G, ldg, db);
+  return cudaGetLastError();
+}
+
 }  // namespace
 
 cudaError_t launch_composite_bw(const float* raw, const SampleSpec& ss, const float* d, int64_t R,
@@ -319,6 +600,54 @@ cudaError_t launch_composite_bw(const float* raw, const SampleSpec& ss, const fl
   if (ss.S > CB_SMAX) return cudaErrorInvalidValue;
   composite_bw_kernel<<<blocks_for(R, CB_WARPS), CB_WARPS * 32, 0, st>>>(raw, ss, d, R, cs, target,
                                                                         inv3n, d_raw, loss_terms);
+  return cudaGetLastError();
+}
+
+// The training path's forward of one network: the activation store is written
+// layer by layer, each layer a row GEMM reading the previous layer's columns.
+// The per-output summation order (fmaf over the inputs in order, then + bias,
+// then ReLU) is that of the fused forward kernel.
+cudaError_t mlp_forward_train_fp32(const PackedFp32& p, const float* pk, const float* dir_bias,
+                                   const float* o, const float* d, int64_t R,
+                                   const SampleSpec& ss, float* raw, float* save,
+                                   cudaStream_t st) {
+  const int D = p.D, W = p.W, Wh = W / 2;
+  const int64_t rows = R * ss.S;
+  if (rows == 0) return cudaSuccess;
+  const int64_t ldc = 64 + (int64_t)(D + 1) * W + Wh;
+  auto hcol = [&](int l) { return 64 + l * W; };
+  const int feat_col = hcol(D), hdir_col = hcol(D + 1);
+  encode_store_kernel<<<blocks_for(rows, 128), 128, 0, st>>>(o, d, R, ss, save, ldc);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  for (int l = 0; l < D && e == cudaSuccess; ++l) {
+    RowGemm g{};
+    g.A = save; g.lda = ldc;
+    if (l == 0) { g.a0 = 0; g.a_split = 64; g.K = 64; }
+    else { g.a0 = hcol(l - 1); g.a_split = W; g.a1 = 0; g.K = l == p.skip + 1 ? W + 64 : W; }
+    g.B = pk + p.layer_w[l]; g.ldb = W; g.n_out = W; g.rows = rows;
+    g.bias = pk + p.layer_b[l]; g.relu = 1;
+    g.out = save + hcol(l); g.ldo = ldc;
+    e = row_gemm(g, st);
+  }
+  if (e != cudaSuccess) return e;
+  {  // feature layer (no activation)
+    RowGemm g{};
+    g.A = save; g.lda = ldc; g.a0 = hcol(D - 1); g.a_split = W; g.K = W;
+    g.B = pk + p.feat_w; g.ldb = W; g.n_out = W; g.rows = rows; g.bias = pk + p.feat_b;
+    g.out = save + feat_col; g.ldo = ldc;
+    if ((e = row_gemm(g, st)) != cudaSuccess) return e;
+  }
+  {  // direction layer: per-ray bias (b_dir + W_dir[:, W:] gamma(d)), ReLU
+    RowGemm g{};
+    g.A = save; g.lda = ldc; g.a0 = feat_col; g.a_split = W; g.K = W;
+    g.B = pk + p.dir_w; g.ldb = Wh; g.n_out = Wh; g.rows = rows;
+    g.row_bias = dir_bias; g.rb_div = ss.S; g.relu = 1;
+    g.out = save + hdir_col; g.ldo = ldc;
+    if ((e = row_gemm(g, st)) != cudaSuccess) return e;
+  }
+  heads_fwd_kernel<<<blocks_for(rows * 32, 256), 256, 0, st>>>(save, ldc, hcol(D - 1), hdir_col, W,
+                                                              pk, p, rows, raw);
   return cudaGetLastError();
 }
 
@@ -332,6 +661,7 @@ cudaError_t mlp_backward_fp32(const PackedFp32& p, int L_dir, const float* w, co
   const int D = p.D, W = p.W, Wh = W / 2, skip = p.skip;
   const int dir_ch = 3 + 6 * L_dir;
   const int64_t rows = R * S;
+  if (rows == 0) return cudaSuccess;
   const int64_t ldc = 64 + (int64_t)(D + 1) * W + Wh;
   const int feat_col = 64 + D * W, hdir_col = 64 + (D + 1) * W;
   auto hcol = [&](int l) { return 64 + l * W; };
@@ -352,57 +682,66 @@ cudaError_t mlp_backward_fp32(const PackedFp32& p, int L_dir, const float* w, co
   float* bufB = tmp + rows * W;
   float* dz_ray = bufB + rows * W;
   float* denc = dz_ray + R * Wh;
-  const unsigned zs = blocks_for(rows, WG_SLICE);
   cudaError_t e;
-#define NERF_WG(A, lda, N, X, ldx, c0, split, c1, K, nrows, G, ldg, db)                         \
-  wgrad_kernel<<<dim3(blocks_for(N, 64), blocks_for((K) + 1, 64), blocks_for(nrows, WG_SLICE)), \
-                 256, 0, st>>>(A, lda, N, X, ldx, c0, split, c1, K, nrows, G, ldg, db);          \
-  if ((e = cudaGetLastError()) != cudaSuccess) return e
-  (void)zs;
+#define NERF_TRY(x) if ((e = (x)) != cudaSuccess) return e
+  auto wg = [&](const float* A, int64_t lda, int N, int x0, int split, int x1, int K, float* G,
+                int64_t ldg, float* db) {
+    WGrad g{};
+    g.A = A; g.lda = lda; g.N = N; g.X = save; g.ldx = ldc; g.x0 = x0; g.x_split = split;
+    g.x1 = x1; g.K = K; g.rows = rows; g.G = G; g.ldg = ldg; g.db = db;
+    return wgrad(g, st);
+  };
+  auto in_grad = [&](const float* A, int64_t lda, int K, const float* B, int64_t ldb,
+                     const float* ea, const float* ev, int mcol, float* out) {
+    RowGemm g{};
+    g.A = A; g.lda = lda; g.a_split = K; g.K = K; g.B = B; g.ldb = ldb; g.n_out = W;
+    g.rows = rows; g.ea = ea; g.ldea = 4; g.ev = ev;
+    if (mcol >= 0) { g.mask = save + mcol; g.ldm = ldc; }
+    g.out = out; g.ldo = W;
+    return row_gemm(g, st);
+  };
   // rgb head: dz_dir = (d_rgb x Wr) masked by h_dir > 0; dWr, dbr
   head_bw_kernel<<<blocks_for(rows * Wh, 256), 256, 0, st>>>(d_raw, w + rgb_w, save, ldc, hdir_col,
                                                              rows, Wh, bufA);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  NERF_WG(d_raw, 4, 3, save, ldc, hdir_col, Wh, 0, Wh, rows, grad + rgb_w, Wh, grad + rgb_b);
+  NERF_TRY(cudaGetLastError());
+  NERF_TRY(wgrad_head<3>(d_raw, 4, save, ldc, hdir_col, Wh, rows, grad + rgb_w, Wh, grad + rgb_b,
+                         st));
   // direction layer: input [feature | gamma(d)]; the gamma(d) part per ray
-  NERF_WG(bufA, Wh, Wh, save, ldc, feat_col, W, 0, W, rows, grad + dir_w, W + dir_ch,
-          grad + dir_b);
+  NERF_TRY(wg(bufA, Wh, Wh, feat_col, W, 0, W, grad + dir_w, W + dir_ch, grad + dir_b));
   ray_sum_kernel<<<blocks_for(R * Wh, 256), 256, 0, st>>>(bufA, R, S, Wh, dz_ray);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  NERF_TRY(cudaGetLastError());
   dir_enc_kernel<<<blocks_for(R, 128), 128, 0, st>>>(d, R, L_dir, denc);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  NERF_WG(dz_ray, Wh, Wh, denc, dir_ch, 0, dir_ch, 0, dir_ch, R, grad + dir_w + W, W + dir_ch,
-          (float*)nullptr);
+  NERF_TRY(cudaGetLastError());
+  {
+    WGrad g{};
+    g.A = dz_ray; g.lda = Wh; g.N = Wh; g.X = denc; g.ldx = dir_ch; g.x0 = 0;
+    g.x_split = dir_ch; g.x1 = 0; g.K = dir_ch; g.rows = R; g.G = grad + dir_w + W;
+    g.ldg = W + dir_ch; g.db = nullptr;
+    NERF_TRY(wgrad(g, st));
+  }
   // d feature = dz_dir x Wd[:, :W] (no activation on the feature layer)
-  in_bw_kernel<<<dim3(blocks_for(rows, 64), W / 64), 256, 0, st>>>(
-      bufA, Wh, w + dir_w, W + dir_ch, Wh, W, rows, nullptr, 0, nullptr, nullptr, 0, 0, bufB, W);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  NERF_TRY(in_grad(bufA, Wh, Wh, w + dir_w, W + dir_ch, nullptr, nullptr, -1, bufB));
   // feature and sigma heads, both reading h_{D-1}
-  NERF_WG(bufB, W, W, save, ldc, hcol(D - 1), W, 0, W, rows, grad + feat_w, W, grad + feat_b);
-  NERF_WG(d_raw + 3, 4, 1, save, ldc, hcol(D - 1), W, 0, W, rows, grad + sig_w, W, grad + sig_b);
+  NERF_TRY(wg(bufB, W, W, hcol(D - 1), W, 0, W, grad + feat_w, W, grad + feat_b));
+  NERF_TRY(wgrad_head<1>(d_raw + 3, 4, save, ldc, hcol(D - 1), W, rows, grad + sig_w, W,
+                         grad + sig_b, st));
   // d h_{D-1} = d feature x Wf + d sigma x ws, masked by h_{D-1} > 0
-  in_bw_kernel<<<dim3(blocks_for(rows, 64), W / 64), 256, 0, st>>>(
-      bufB, W, w + feat_w, W, W, W, rows, d_raw + 3, 4, w + sig_w, save, ldc, hcol(D - 1), bufA, W);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  NERF_TRY(in_grad(bufB, W, W, w + feat_w, W, d_raw + 3, w + sig_w, hcol(D - 1), bufA));
   // the trunk, top down: bufA holds dz of layer l
   for (int l = D - 1; l >= 0; --l) {
     if (l == 0) {
-      NERF_WG(bufA, W, W, save, ldc, 0, 63, 0, 63, rows, grad + wo[0], Kl[0], grad + bo[0]);
+      NERF_TRY(wg(bufA, W, W, 0, 63, 0, 63, grad + wo[0], Kl[0], grad + bo[0]));
     } else if (l == skip + 1) {
-      NERF_WG(bufA, W, W, save, ldc, hcol(l - 1), W, 0, W + 63, rows, grad + wo[l], Kl[l],
-              grad + bo[l]);
+      NERF_TRY(wg(bufA, W, W, hcol(l - 1), W, 0, W + 63, grad + wo[l], Kl[l], grad + bo[l]));
     } else {
-      NERF_WG(bufA, W, W, save, ldc, hcol(l - 1), W, 0, W, rows, grad + wo[l], Kl[l], grad + bo[l]);
+      NERF_TRY(wg(bufA, W, W, hcol(l - 1), W, 0, W, grad + wo[l], Kl[l], grad + bo[l]));
     }
     if (l > 0) {
-      in_bw_kernel<<<dim3(blocks_for(rows, 64), W / 64), 256, 0, st>>>(
-          bufA, W, w + wo[l], Kl[l], W, W, rows, nullptr, 0, nullptr, save, ldc, hcol(l - 1), bufB,
-          W);
-      if ((e = cudaGetLastError()) != cudaSuccess) return e;
+      NERF_TRY(in_grad(bufA, W, W, w + wo[l], Kl[l], nullptr, nullptr, hcol(l - 1), bufB));
       float* t = bufA; bufA = bufB; bufB = t;
     }
   }
-#undef NERF_WG
+#undef NERF_TRY
   return cudaSuccess;
 }
 

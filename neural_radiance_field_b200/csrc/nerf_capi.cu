@@ -293,8 +293,13 @@ nerf_status run_network(nerf_ctx* ctx, const void* blob, const float* o, const f
   const int dir_ch = 3 * (1 + 2 * c.L_dir);
   NERF_CHECK_LAUNCH(ctx, launch_pack_fp32(blob, c.precision, ctx->plan, dir_ch, ctx->packed, st));
   TimedScope ts(ctx, st);
-  NERF_CHECK_LAUNCH(ctx, launch_mlp_fp32(ctx->plan, ctx->packed, ctx->dir_bias, o, d, R, ss, raw, st,
-                                         save));
+  if (save) {
+    NERF_CHECK_LAUNCH(ctx, mlp_forward_train_fp32(ctx->plan, ctx->packed, ctx->dir_bias, o, d, R,
+                                                  ss, raw, save, st));
+  } else {
+    NERF_CHECK_LAUNCH(ctx, launch_mlp_fp32(ctx->plan, ctx->packed, ctx->dir_bias, o, d, R, ss, raw,
+                                           st));
+  }
   return NERF_OK;
 }
 

@@ -109,6 +109,10 @@ struct CompositeSpec {
 cudaError_t launch_composite_bw(const float* raw, const SampleSpec& ss, const float* d, int64_t R,
                                 const CompositeSpec& cs, const float* target, float inv3n,
                                 float* d_raw, float* loss_terms, cudaStream_t st);
+cudaError_t mlp_forward_train_fp32(const PackedFp32& p, const float* packed, const float* dir_bias,
+                                   const float* o, const float* d, int64_t R,
+                                   const SampleSpec& ss, float* raw, float* save,
+                                   cudaStream_t st);
 cudaError_t mlp_backward_fp32(const PackedFp32& p, int L_dir, const float* w, const float* save,
                               int64_t R, int S, const float* d, const float* d_raw,
                               float* grad, float* tmp, cudaStream_t st);
