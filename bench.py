@@ -472,7 +472,7 @@ def run_train(args, rank, world, local_rank):
     nbuild.build()
     torch.cuda.set_device(local_rank)
     wl = dataclasses.replace(S.WORKLOADS[WORKLOAD], precision=S.PREC_FP32)
-    B = TRAIN_BATCH
+    B = args.batch or TRAIN_BATCH
     shape = wl.mlp
     o_all = torch.empty(wl.n_rays, 3, device="cuda")
     d_all = torch.empty(wl.n_rays, 3, device="cuda")
@@ -536,7 +536,11 @@ def run_train(args, rank, world, local_rank):
             "roofline": {"bound": "alu", "kernel": "whole training step (fp32 CUDA-core kernels)",
                          "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                          "frac": achieved / peak, "peak_kind": FP32_PEAK_NOTE, "traffic": None},
-            "gpu_launches": None, "clocks": clocks}
+            # per pass: weight packing, direction bias, the forward (encoding, D + 2
+            # layer GEMMs, heads), compositing backward, the backward (2 D + 9); then
+            # the resampling and the loss sum
+            "gpu_launches": args.steps * (2 * ((shape.D + 6) + 1 + (2 * shape.D + 9)) + 2),
+            "clocks": clocks}
     print(json.dumps(line), flush=True)
 
 
@@ -592,7 +596,7 @@ def run_hash_backward(args, rank, world, local_rank):
                          "peak_kind": f"HBM copy, {peak_kind}; the 48.8 MB gradient table is "
                                       "L2-resident, so its atomics resolve in L2",
                          "traffic": None, "bytes_per_point": bytes_pt},
-            "gpu_launches": None, "clocks": clk.summary()}
+            "gpu_launches": args.steps, "clocks": clk.summary()}
     print(json.dumps(line), flush=True)
 
 
@@ -680,9 +684,19 @@ def run_march(args, rank, world, local_rank):
                          "unit": "TFLOP/s", "frac": achieved / peak, "peak_kind": FP32_PEAK_NOTE,
                          "traffic": None, "kernel_ms_per_frame": per_frame_k_ms,
                          "flop_per_point": flop_per_point},
-            "gpu_launches": None, "clocks": clocks}
+            "gpu_launches": args.steps * march_launches_per_step(wl.model, R), "clocks": clocks}
     print(json.dumps(line), flush=True)
     rnd.close()
+
+
+def march_launches_per_step(model, R):
+    """The library's kernels per march step: ray generation, then per chunk of up
+    to 2^19 rays the occupancy mask, a 3-kernel scan, the emit, the scene
+    function (hash grid: 1 kernel; KiloNeRF: histogram, 3-kernel scan, scatter,
+    work items, evaluation) and compositing."""
+    chunks = -(-R // min(R, 1 << 19))
+    per_chunk = 6 + (1 if model == "hashgrid" else 7)
+    return 1 + chunks * per_chunk
 
 
 # DRAM bytes (read + write) per MLP row of the scene-MLP kernel, from the ncu
@@ -714,6 +728,8 @@ def main():
                     help="the benchmark workload (default) or a march workload (extra lines)")
     ap.add_argument("--traffic-bytes", type=float, default=0.0,
                     help="DRAM bytes per network launch from an ncu capture of this kernel")
+    ap.add_argument("--batch", type=int, default=0,
+                    help="rays per training step (train workload; default 4096)")
     ap.add_argument("--size", type=int, default=0,
                     help="render an SIZE x SIZE frame instead (profiling runs only)")
     args = ap.parse_args()

@@ -168,7 +168,7 @@ __global__ void head_bw_kernel(const float* __restrict__ d_raw, const float* __r
 // its terms in reduction order with fmaf.
 // ---------------------------------------------------------------------------
 constexpr int GT = 128;          // tile edge
-constexpr int GK = 8;            // reduction step
+constexpr int GK = 16;           // reduction step (two fetch rounds of 8)
 constexpr int GLD = GT + 4;      // padded row of a shared operand tile
 
 struct GemmSmem {
@@ -241,27 +241,32 @@ __global__ void __launch_bounds__(256, 2) row_gemm_kernel(RowGemm g) {
     const float* p = g.B + (int64_t)(k0 + bk) * g.ldb + bc;
     return load4(p, g.b_vec, bc < g.n_out, bc + 1 < g.n_out, bc + 2 < g.n_out, bc + 3 < g.n_out);
   };
-  auto put = [&](int buf, float4 va, float4 vb) {
-    sm.a[buf][ak + 0][tid >> 1] = va.x;
-    sm.a[buf][ak + 1][tid >> 1] = va.y;
-    sm.a[buf][ak + 2][tid >> 1] = va.z;
-    sm.a[buf][ak + 3][tid >> 1] = va.w;
-    *reinterpret_cast<float4*>(&sm.b[buf][bk][(tid & 31) * 4]) = vb;
+  auto put = [&](int buf, int kh, float4 va, float4 vb) {
+    sm.a[buf][kh + ak + 0][tid >> 1] = va.x;
+    sm.a[buf][kh + ak + 1][tid >> 1] = va.y;
+    sm.a[buf][kh + ak + 2][tid >> 1] = va.z;
+    sm.a[buf][kh + ak + 3][tid >> 1] = va.w;
+    *reinterpret_cast<float4*>(&sm.b[buf][kh + bk][(tid & 31) * 4]) = vb;
   };
   float acc[8][8];
 #pragma unroll
   for (int i = 0; i < 8; ++i)
 #pragma unroll
     for (int j = 0; j < 8; ++j) acc[i][j] = 0.0f;
-  put(0, fetch_a(0), fetch_b(0));
+  put(0, 0, fetch_a(0), fetch_b(0));
+  put(0, 8, fetch_a(8), fetch_b(8));
   __syncthreads();
   const int steps = g.K / GK;
   for (int s = 0; s < steps; ++s) {
     const int cur = s & 1;
-    float4 na = make_float4(0.f, 0.f, 0.f, 0.f), nb = na;
-    if (s + 1 < steps) { na = fetch_a((s + 1) * GK); nb = fetch_b((s + 1) * GK); }
+    const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
+    float4 na0 = z, nb0 = z, na1 = z, nb1 = z;
+    if (s + 1 < steps) {
+      na0 = fetch_a((s + 1) * GK); nb0 = fetch_b((s + 1) * GK);
+      na1 = fetch_a((s + 1) * GK + 8); nb1 = fetch_b((s + 1) * GK + 8);
+    }
     gemm_step(sm.a[cur], sm.b[cur], acc, ty, tx);
-    if (s + 1 < steps) put(cur ^ 1, na, nb);
+    if (s + 1 < steps) { put(cur ^ 1, 0, na0, nb0); put(cur ^ 1, 8, na1, nb1); }
     __syncthreads();
   }
 #pragma unroll
@@ -314,7 +319,7 @@ __global__ void __launch_bounds__(256, 2) wgrad_gemm_kernel(WGrad g) {
   // with XV, a thread's four X columns lie in one of the two ranges
   const bool x_lo = xk < g.x_split;
   const int xcol = x_lo ? g.x0 + xk : g.x1 + xk - g.x_split;
-  // this thread's fetch row, advanced by GK rows per step
+  // this thread's fetch row, advanced by 8 rows per fetch (two fetches per step)
   int64_t fr_row = rs + fr;
   const float* pa = g.A + fr_row * g.lda + an;
   const float* px = g.X + fr_row * g.ldx;
@@ -336,13 +341,13 @@ __global__ void __launch_bounds__(256, 2) wgrad_gemm_kernel(WGrad g) {
         vx = make_float4(t[0], t[1], t[2], t[3]);
       }
     }
-    fr_row += GK;
-    pa += GK * g.lda;
-    px += GK * g.ldx;
+    fr_row += 8;
+    pa += 8 * g.lda;
+    px += 8 * g.ldx;
   };
-  auto put = [&](int buf, float4 va, float4 vx) {
-    *reinterpret_cast<float4*>(&sm.a[buf][fr][fc]) = va;
-    *reinterpret_cast<float4*>(&sm.b[buf][fr][fc]) = vx;
+  auto put = [&](int buf, int rh, float4 va, float4 vx) {
+    *reinterpret_cast<float4*>(&sm.a[buf][rh + fr][fc]) = va;
+    *reinterpret_cast<float4*>(&sm.b[buf][rh + fr][fc]) = vx;
   };
   const bool bias_cta = g.db != nullptr && blockIdx.y == 0;
   float bsum = 0.0f;
@@ -351,21 +356,23 @@ __global__ void __launch_bounds__(256, 2) wgrad_gemm_kernel(WGrad g) {
   for (int i = 0; i < 8; ++i)
 #pragma unroll
     for (int j = 0; j < 8; ++j) acc[i][j] = 0.0f;
-  float4 va, vx;
-  fetch(va, vx);
-  put(0, va, vx);
+  float4 va0, vx0, va1, vx1;
+  fetch(va0, vx0);
+  fetch(va1, vx1);
+  put(0, 0, va0, vx0);
+  put(0, 8, va1, vx1);
   __syncthreads();
   const int steps = (int)((re - rs + GK - 1) / GK);
   for (int s = 0; s < steps; ++s) {
     const int cur = s & 1;
     const bool more = s + 1 < steps;
-    if (more) fetch(va, vx);
+    if (more) { fetch(va0, vx0); fetch(va1, vx1); }
     gemm_step(sm.a[cur], sm.b[cur], acc, ty, tx);
     if (bias_cta && tid < GT) {
 #pragma unroll
       for (int k = 0; k < GK; ++k) bsum += sm.a[cur][k][tid];
     }
-    if (more) put(cur ^ 1, va, vx);
+    if (more) { put(cur ^ 1, 0, va0, vx0); put(cur ^ 1, 8, va1, vx1); }
     __syncthreads();
   }
 #pragma unroll
@@ -382,29 +389,66 @@ __global__ void __launch_bounds__(256, 2) wgrad_gemm_kernel(WGrad g) {
 }
 
 // The weight gradient of a head with N <= 4 outputs (sigma: 1, rgb: 3): one
-// thread per input column k (and k = K for the bias), summing over a slice of
-// rows; the reads of X are coalesced across the threads.
+// thread per four input columns (the thread past the last one sums the bias),
+// over a slice of rows, four rows in flight; the reads of X are 16-byte and
+// coalesced across the threads. X rows and x0 are 4-float aligned, K % 4 == 0.
 template <int NS>
 __global__ void __launch_bounds__(128)
 wgrad_head_kernel(const float* __restrict__ A, int64_t lda, const float* __restrict__ X,
                   int64_t ldx, int x0, int K, int64_t rows, int64_t slice, float* __restrict__ G,
                   int64_t ldg, float* __restrict__ db) {
-  const int k = blockIdx.x * blockDim.x + threadIdx.x;
+  const int k = 4 * (blockIdx.x * blockDim.x + threadIdx.x);
   if (k > K) return;
+  const bool bias = k == K;
   const int64_t rs = (int64_t)blockIdx.y * slice;
   const int64_t re = rs + slice < rows ? rs + slice : rows;
-  float acc[NS];
+  float acc[NS][4];
 #pragma unroll
-  for (int n = 0; n < NS; ++n) acc[n] = 0.0f;
-  for (int64_t r = rs; r < re; ++r) {
-    const float x = k < K ? X[r * ldx + x0 + k] : 1.0f;
+  for (int n = 0; n < NS; ++n)
 #pragma unroll
-    for (int n = 0; n < NS; ++n) acc[n] = fmaf(A[r * lda + n], x, acc[n]);
+    for (int e = 0; e < 4; ++e) acc[n][e] = 0.0f;
+  const float* px = X + x0 + k;
+  int64_t r = rs;
+  for (; r + 4 <= re; r += 4) {
+    float4 x[4];
+    float a[4][NS];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      x[u] = bias ? make_float4(1.f, 0.f, 0.f, 0.f)
+                  : __ldg(reinterpret_cast<const float4*>(px + (r + u) * ldx));
+#pragma unroll
+      for (int n = 0; n < NS; ++n) a[u][n] = __ldg(A + (r + u) * lda + n);
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+#pragma unroll
+      for (int n = 0; n < NS; ++n) {
+        acc[n][0] = fmaf(a[u][n], x[u].x, acc[n][0]);
+        acc[n][1] = fmaf(a[u][n], x[u].y, acc[n][1]);
+        acc[n][2] = fmaf(a[u][n], x[u].z, acc[n][2]);
+        acc[n][3] = fmaf(a[u][n], x[u].w, acc[n][3]);
+      }
+  }
+  for (; r < re; ++r) {
+    const float4 x = bias ? make_float4(1.f, 0.f, 0.f, 0.f)
+                          : __ldg(reinterpret_cast<const float4*>(px + r * ldx));
+#pragma unroll
+    for (int n = 0; n < NS; ++n) {
+      const float a = __ldg(A + r * lda + n);
+      acc[n][0] = fmaf(a, x.x, acc[n][0]);
+      acc[n][1] = fmaf(a, x.y, acc[n][1]);
+      acc[n][2] = fmaf(a, x.z, acc[n][2]);
+      acc[n][3] = fmaf(a, x.w, acc[n][3]);
+    }
   }
 #pragma unroll
   for (int n = 0; n < NS; ++n) {
-    if (k < K) atomicAdd(G + (int64_t)n * ldg + k, acc[n]);
-    else atomicAdd(db + n, acc[n]);
+    if (bias) {
+      atomicAdd(db + n, acc[n][0]);
+    } else {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) atomicAdd(G + (int64_t)n * ldg + k + e, acc[n][e]);
+    }
   }
 }
 
@@ -585,7 +629,8 @@ template <int NS>
 cudaError_t wgrad_head(const float* A, int64_t lda, const float* X, int64_t ldx, int x0, int K,
                        int64_t rows, float* G, int64_t ldg, float* db, cudaStream_t st) {
   if (rows == 0) return cudaSuccess;
-  const unsigned bx = blocks_for(K + 1, 128);
+  if (K % 4 || x0 % 4 || ldx % 4 || !al16(X)) return cudaErrorInvalidValue;
+  const unsigned bx = blocks_for(K / 4 + 1, 128);
   const int64_t slice = slice_rows(rows, (int)bx);
   wgrad_head_kernel<NS><<<dim3(bx, blocks_for(rows, slice)), 128, 0, st>>>(
       A, lda, X, ldx, x0, K, rows, slice, G, ldg, db);
@@ -730,7 +775,8 @@ cudaError_t mlp_backward_fp32(const PackedFp32& p, int L_dir, const float* w, co
   // the trunk, top down: bufA holds dz of layer l
   for (int l = D - 1; l >= 0; --l) {
     if (l == 0) {
-      NERF_TRY(wg(bufA, W, W, 0, 63, 0, 63, grad + wo[0], Kl[0], grad + bo[0]));
+      // gamma(x) is one column range; a split past K keeps the fetches vectorised
+      NERF_TRY(wg(bufA, W, W, 0, 64, 0, 63, grad + wo[0], Kl[0], grad + bo[0]));
     } else if (l == skip + 1) {
       NERF_TRY(wg(bufA, W, W, hcol(l - 1), W, 0, W + 63, grad + wo[l], Kl[l], grad + bo[l]));
     } else {
