@@ -1,11 +1,11 @@
 // fp32 CUDA-core evaluation of the NeRF scene MLP (NeRF page, Section 2.4),
 // fused with sample placement and positional encoding.
 //
-// One CTA of 256 threads owns BM = 64 consecutive rows (samples); their
-// activations stay in shared memory for the whole network as fp32 rows of
-// [h (W columns) | gamma(x) (63 columns + 1 zero pad)], so the skip layer's input
-// [h, gamma(x)] is simply the first W + 64 columns. Each layer is a register-
-// blocked product with the packed, K-major weights read through L1.
+// One CTA of 2 W threads owns 128 consecutive rows (samples); their activations
+// stay in shared memory for the whole network, feature-major, so every layer is a
+// register-blocked product (8 x 8 outputs per thread) whose left operand is read
+// straight from the activations and whose weights (packed K-major) stream
+// through a shared-memory double buffer.
 #include "nerf_internal.cuh"
 
 namespace nerfb {
@@ -97,102 +97,134 @@ cudaError_t launch_pack_fp32(const void* blob, int precision, const PackedFp32& 
 
 namespace {
 
-// Rows r = blockIdx.x * BM + i; sample s of ray r / S.
+// Geometry for width W: a CTA of 2 W threads owns BM = 128 rows; thread (ty, tx)
+// holds 8 x 8 outputs of a layer of N columns (N = W, or W / 2 for the direction
+// layer): rows {4 ty + i, 64 + 4 ty + i} and columns {4 tx + j, N / 2 + 4 tx + j},
+// i, j < 4, for tx < N / 8. A warp covers 2 (W >= 128) or 4 (W = 64) values of ty.
 template <int W>
-struct Smem {
-  static constexpr int LD = W + 64;  // fp32 row stride of the activation tile
-  float act[BM][LD];
-  float sig[BM];
-  float x[BM][3];
-  int64_t ray[BM];
+struct Cfg {
+  static constexpr int BM = 128;
+  static constexpr int NTH = 2 * W;
+  static constexpr int BK = 8;                     // weight rows per staged slice
+  static constexpr int LDA = BM + 4;               // one feature's BM row values
+  static constexpr int LDB = W + 4;
+  static constexpr int MIN_CTAS = W == 256 ? 1 : W == 128 ? 2 : 3;
+  static constexpr int TXW = W / 8 < 16 ? W / 8 : 16;   // tx values per warp
 };
 
-// One dense layer on the tile: out[:, out_col + n] = act(act[:, in_col:in_col+K] Wt + b),
-// Wt K-major [K][N]. Thread (tx, ty) owns columns tx*8..tx*8+7 and RPT rows.
-template <int W, int N>
+// The activations are stored feature-major: actT[f][r] is feature f of row r,
+// features [h (W) | gamma(x) (63) | 0], so the skip layer's input [h, gamma(x)]
+// is features 0 .. W + 63 and layer 0's input is features W .. W + 63.
+template <int W>
+struct Smem {
+  float actT[W + 64][Cfg<W>::LDA];
+  float wb[2][Cfg<W>::BK][Cfg<W>::LDB];
+  float sig[Cfg<W>::BM];
+  float x[Cfg<W>::BM][3];
+  int64_t ray[Cfg<W>::BM];
+};
+
+// One dense layer on the tile: out[r][n] = act(sum_k actT[f0 + k][r] Wt[k][n] + bias),
+// Wt K-major [K][N] (K a multiple of BK), staged through shared memory in slices
+// of BK rows with a register prefetch of the next slice; then written back as
+// features 0 .. N - 1. bias[n], or row_bias[ray(r) * N + n] when given.
+template <int W>
 __device__ __forceinline__ void tile_layer(Smem<W>& sm, const float* __restrict__ Wt,
                                            const float* __restrict__ bias,
-                                           const float* __restrict__ row_bias, int K,
-                                           int in_col, int out_col, bool relu) {
-  constexpr int TPC = N / 8;          // threads across the columns
-  constexpr int RG = NT / TPC;        // row groups
-  constexpr int RPT = BM / RG;        // rows per thread
-  static_assert(RPT >= 1 && BM % RG == 0, "tile shape");
-  const int tx = threadIdx.x % TPC, ty = threadIdx.x / TPC;
-  const int c0 = tx * 8;
-  float acc[RPT][8];
+                                           const float* __restrict__ row_bias, int K, int f0,
+                                           int N, bool relu, int ty, int tx) {
+  using C = Cfg<W>;
+  constexpr int PF = C::BK / 8;                 // float4 fetches per thread per slice
+  const int tid = threadIdx.x;
+  const int n4 = N / 4;
+  const bool active = tx < N / 8;
+  float4 pre[PF];
+  auto fetch = [&](int k0) {
 #pragma unroll
-  for (int i = 0; i < RPT; ++i)
+    for (int i = 0; i < PF; ++i) {
+      const int q = tid + i * C::NTH;
+      const int k = q / n4, c = 4 * (q % n4);
+      pre[i] = q < C::BK * n4 ? __ldg(reinterpret_cast<const float4*>(Wt + (int64_t)(k0 + k) * N + c))
+                              : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+  };
+  auto put = [&](int buf) {
+#pragma unroll
+    for (int i = 0; i < PF; ++i) {
+      const int q = tid + i * C::NTH;
+      if (q < C::BK * n4)
+        *reinterpret_cast<float4*>(&sm.wb[buf][q / n4][4 * (q % n4)]) = pre[i];
+    }
+  };
+  float acc[8][8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
 #pragma unroll
     for (int j = 0; j < 8; ++j) acc[i][j] = 0.0f;
-  for (int k = 0; k < K; k += 4) {
-    float4 a[RPT];
+  fetch(0);
+  put(0);
+  __syncthreads();
+  const int steps = K / C::BK;
+  const int c1 = N / 2 + 4 * tx;
+  for (int s = 0; s < steps; ++s) {
+    const int cur = s & 1;
+    if (s + 1 < steps) fetch((s + 1) * C::BK);
+    if (active) {
+      const int fb = f0 + s * C::BK;
 #pragma unroll
-    for (int i = 0; i < RPT; ++i)
-      a[i] = *reinterpret_cast<const float4*>(&sm.act[ty * RPT + i][in_col + k]);
+      for (int k = 0; k < C::BK; ++k) {
+        const float4 a0 = *reinterpret_cast<const float4*>(&sm.actT[fb + k][4 * ty]);
+        const float4 a1 = *reinterpret_cast<const float4*>(&sm.actT[fb + k][64 + 4 * ty]);
+        const float4 b0 = *reinterpret_cast<const float4*>(&sm.wb[cur][k][4 * tx]);
+        const float4 b1 = *reinterpret_cast<const float4*>(&sm.wb[cur][k][c1]);
+        const float av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+        const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
 #pragma unroll
-    for (int kk = 0; kk < 4; ++kk) {
-      const float4 w0 = __ldg(reinterpret_cast<const float4*>(Wt + (int64_t)(k + kk) * N + c0));
-      const float4 w1 =
-          __ldg(reinterpret_cast<const float4*>(Wt + (int64_t)(k + kk) * N + c0 + 4));
-      const float wv[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+        for (int i = 0; i < 8; ++i)
 #pragma unroll
-      for (int i = 0; i < RPT; ++i) {
-        const float av = kk == 0 ? a[i].x : kk == 1 ? a[i].y : kk == 2 ? a[i].z : a[i].w;
-#pragma unroll
-        for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(av, wv[j], acc[i][j]);
+          for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
       }
     }
+    if (s + 1 < steps) put(cur ^ 1);
+    __syncthreads();   // the last one also ends every read of the input features
   }
-  __syncthreads();  // every read of the input columns is done
-#pragma unroll
-  for (int i = 0; i < RPT; ++i) {
-    const int r = ty * RPT + i;
-    const float* rb = row_bias ? row_bias + sm.ray[r] * N : nullptr;
-    float v[8];
+  if (active) {
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
-      float b = rb ? rb[c0 + j] : __ldg(bias + c0 + j);
-      v[j] = acc[i][j] + b;
-      if (relu) v[j] = fmaxf(v[j], 0.0f);
+      const int c = j < 4 ? 4 * tx + j : c1 + j - 4;
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int r0 = 64 * h + 4 * ty;
+        float v[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float b = row_bias ? row_bias[sm.ray[r0 + i] * N + c] : __ldg(bias + c);
+          v[i] = acc[4 * h + i][j] + b;
+          if (relu) v[i] = fmaxf(v[i], 0.0f);
+        }
+        *reinterpret_cast<float4*>(&sm.actT[c][r0]) = make_float4(v[0], v[1], v[2], v[3]);
+      }
     }
-    *reinterpret_cast<float4*>(&sm.act[r][out_col + c0]) = make_float4(v[0], v[1], v[2], v[3]);
-    *reinterpret_cast<float4*>(&sm.act[r][out_col + c0 + 4]) =
-        make_float4(v[4], v[5], v[6], v[7]);
   }
   __syncthreads();
 }
 
-// Copies columns [src, src + n) of the tile's activations to columns
-// [dst, dst + n) of the training path's activation store (row-major, ld floats
-// per row; n a multiple of 4).
 template <int W>
-__device__ __forceinline__ void store_cols(const Smem<W>& sm, float* save, int64_t ld,
-                                           int64_t row0, int64_t rows, int src, int64_t dst,
-                                           int n) {
-  const int n4 = n / 4;
-  for (int q = threadIdx.x; q < BM * n4; q += NT) {
-    const int r = q / n4, c = 4 * (q % n4);
-    const int64_t row = row0 + r;
-    if (row < rows)
-      *reinterpret_cast<float4*>(save + row * ld + dst + c) =
-          *reinterpret_cast<const float4*>(&sm.act[r][src + c]);
-  }
-}
-
-template <int W>
-__global__ void __launch_bounds__(NT, 1)
+__global__ void __launch_bounds__(Cfg<W>::NTH, Cfg<W>::MIN_CTAS)
 mlp_fp32_kernel(PackedFp32 p, const float* __restrict__ pk, const float* __restrict__ dir_bias,
                 const float* __restrict__ o, const float* __restrict__ d, int64_t R,
-                SampleSpec ss, float* __restrict__ raw, float* __restrict__ save) {
-  // save (training path, else NULL): per row [gamma(x) (64) | h_0 .. h_{D-1} |
-  // feature | h_dir], the layers' post-activation outputs
-  const int64_t ldc = 64 + (int64_t)(p.D + 1) * W + W / 2;
+                SampleSpec ss, float* __restrict__ raw) {
+  using C = Cfg<W>;
+  constexpr int BM = C::BM;
   extern __shared__ __align__(16) unsigned char smem_raw[];
   Smem<W>& sm = *reinterpret_cast<Smem<W>*>(smem_raw);
   const int64_t rows = R * ss.S;
   const int64_t row0 = (int64_t)blockIdx.x * BM;
   const int tid = threadIdx.x;
+  const int lane = tid & 31, warp = tid >> 5;
+  constexpr int NBLK = (W / 8) / C::TXW;       // warps across the columns
+  const int ty = (warp / NBLK) * (32 / C::TXW) + lane / C::TXW;
+  const int tx = (warp % NBLK) * C::TXW + lane % C::TXW;
 
   // sample positions and points (fp32, same rounded ops as the oracle)
   if (tid < BM) {
@@ -221,54 +253,47 @@ mlp_fp32_kernel(PackedFp32 p, const float* __restrict__ pk, const float* __restr
     sm.ray[tid] = ray;
   }
   __syncthreads();
-  // gamma(x) into columns W .. W+63 (last one zero)
-  for (int q = tid; q < BM * 64; q += NT) {
-    int r = q / 64, j = q % 64;
+  // gamma(x) into features W .. W + 63 (the last one zero), one row per lane
+  for (int q = tid; q < BM * 64; q += C::NTH) {
+    const int r = q % BM, j = q / BM;
     float v = 0.0f;
     if (j < 3) {
       v = sm.x[r][j];
     } else if (j < 63) {
-      int jj = (j - 3) % 30;
-      float s, c;
-      pe_sincos(sm.x[r][jj / 10], jj % 10, &s, &c);
-      v = (j - 3 < 30) ? s : c;
+      const int jj = (j - 3) % 30;
+      float sn, cs;
+      pe_sincos(sm.x[r][jj / 10], jj % 10, &sn, &cs);
+      v = (j - 3 < 30) ? sn : cs;
     }
-    sm.act[r][W + j] = v;
+    sm.actT[W + j][r] = v;
   }
   __syncthreads();
-  if (save) store_cols<W>(sm, save, ldc, row0, rows, W, 0, 64);
 
   for (int l = 0; l < p.D; ++l) {
-    int K = (l == 0) ? 64 : (l == p.skip + 1 ? W + 64 : W);
-    int in_col = (l == 0) ? W : 0;
-    tile_layer<W, W>(sm, pk + p.layer_w[l], pk + p.layer_b[l], nullptr, K, in_col, 0, true);
-    if (save) store_cols<W>(sm, save, ldc, row0, rows, 0, 64 + (int64_t)l * W, W);
+    const int K = (l == 0) ? 64 : (l == p.skip + 1 ? W + 64 : W);
+    tile_layer<W>(sm, pk + p.layer_w[l], pk + p.layer_b[l], nullptr, K, l == 0 ? W : 0, W, true,
+                  ty, tx);
   }
-  // sigma head from h (4 threads per row)
-  {
-    int r = tid / 4, part = tid % 4;
+  // sigma head from h_{D-1}
+  if (tid < BM) {
     float a = 0.0f;
-    for (int k = part; k < W; k += 4) a = fmaf(sm.act[r][k], __ldg(pk + p.sigma_w + k), a);
-    a += __shfl_xor_sync(0xffffffffu, a, 1);
-    a += __shfl_xor_sync(0xffffffffu, a, 2);
-    if (part == 0) sm.sig[r] = a + __ldg(pk + p.sigma_b);
+    for (int k = 0; k < W; ++k) a = fmaf(sm.actT[k][tid], __ldg(pk + p.sigma_w + k), a);
+    sm.sig[tid] = a + __ldg(pk + p.sigma_b);
   }
-  // feature layer (no activation), then the direction layer with its per-ray bias
-  tile_layer<W, W>(sm, pk + p.feat_w, pk + p.feat_b, nullptr, W, 0, 0, false);
-  if (save) store_cols<W>(sm, save, ldc, row0, rows, 0, 64 + (int64_t)p.D * W, W);
-  tile_layer<W, W / 2>(sm, pk + p.dir_w, nullptr, dir_bias, W, 0, 0, true);
-  if (save) store_cols<W>(sm, save, ldc, row0, rows, 0, 64 + (int64_t)(p.D + 1) * W, W / 2);
+  // (the feature layer's first barrier orders these reads before its writes)
+  tile_layer<W>(sm, pk + p.feat_w, pk + p.feat_b, nullptr, W, 0, W, false, ty, tx);
+  tile_layer<W>(sm, pk + p.dir_w, nullptr, dir_bias, W, 0, W / 2, true, ty, tx);
   // rgb head and output
-  if (tid < BM * 3) {
-    int r = tid / 3, c = tid % 3;
+  for (int q = tid; q < BM * 3; q += C::NTH) {
+    const int r = q / 3, c = q % 3;
     const float* w = pk + p.rgb_w + c * (W / 2);
     float a = __ldg(pk + p.rgb_b + c);
-    for (int k = 0; k < W / 2; ++k) a = fmaf(sm.act[r][k], __ldg(w + k), a);
-    int64_t row = row0 + r;
+    for (int k = 0; k < W / 2; ++k) a = fmaf(sm.actT[k][r], __ldg(w + k), a);
+    const int64_t row = row0 + r;
     if (row < rows) raw[row * 4 + c] = a;
   }
   if (tid < BM) {
-    int64_t row = row0 + tid;
+    const int64_t row = row0 + tid;
     if (row < rows) raw[row * 4 + 3] = sm.sig[tid];
   }
 }
@@ -277,25 +302,21 @@ mlp_fp32_kernel(PackedFp32 p, const float* __restrict__ pk, const float* __restr
 
 cudaError_t launch_mlp_fp32(const PackedFp32& p, const float* packed, const float* dir_bias,
                             const float* o, const float* d, int64_t R, const SampleSpec& ss,
-                            float* raw, cudaStream_t st, float* save) {
-  int64_t rows = R * ss.S;
-  unsigned blocks = (unsigned)((rows + BM - 1) / BM);
-  if (p.W == 256) {
-    size_t sh = sizeof(Smem<256>);
-    cudaFuncSetAttribute(mlp_fp32_kernel<256>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sh);
-    mlp_fp32_kernel<256><<<blocks, NT, sh, st>>>(p, packed, dir_bias, o, d, R, ss, raw, save);
-  } else if (p.W == 128) {
-    size_t sh = sizeof(Smem<128>);
-    cudaFuncSetAttribute(mlp_fp32_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sh);
-    mlp_fp32_kernel<128><<<blocks, NT, sh, st>>>(p, packed, dir_bias, o, d, R, ss, raw, save);
-  } else if (p.W == 64) {
-    size_t sh = sizeof(Smem<64>);
-    cudaFuncSetAttribute(mlp_fp32_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sh);
-    mlp_fp32_kernel<64><<<blocks, NT, sh, st>>>(p, packed, dir_bias, o, d, R, ss, raw, save);
-  } else {
-    return cudaErrorInvalidValue;
-  }
-  return cudaGetLastError();
+                            float* raw, cudaStream_t st) {
+  const int64_t rows = R * ss.S;
+  if (rows == 0) return cudaSuccess;
+  const unsigned blocks = (unsigned)((rows + 127) / 128);
+  cudaError_t e = cudaErrorInvalidValue;
+  auto go = [&](auto kern, int nth, size_t sh) {
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sh);
+    if (e != cudaSuccess) return;
+    kern<<<blocks, nth, sh, st>>>(p, packed, dir_bias, o, d, R, ss, raw);
+    e = cudaGetLastError();
+  };
+  if (p.W == 256) go(mlp_fp32_kernel<256>, Cfg<256>::NTH, sizeof(Smem<256>));
+  else if (p.W == 128) go(mlp_fp32_kernel<128>, Cfg<128>::NTH, sizeof(Smem<128>));
+  else if (p.W == 64) go(mlp_fp32_kernel<64>, Cfg<64>::NTH, sizeof(Smem<64>));
+  return e;
 }
 
 }  // namespace nerfb

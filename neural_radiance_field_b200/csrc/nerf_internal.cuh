@@ -96,8 +96,7 @@ struct SampleSpec {
 
 cudaError_t launch_mlp_fp32(const PackedFp32& p, const float* packed, const float* dir_bias,
                             const float* o, const float* d, int64_t R, const SampleSpec& ss,
-                            float* raw, cudaStream_t st,
-                            float* save = nullptr);
+                            float* raw, cudaStream_t st);
 
 // Compositing of raw [R][S][4]; t from ss (stratified or given).
 struct CompositeSpec {
