@@ -387,9 +387,11 @@ __global__ void sh_kernel(const float* __restrict__ d, int64_t n, ShConst K,
 
 // The hash scene function as small fp32 GEMMs over tiles of 128 live points
 // (a CTA per SM, persistent): the points' activations sit k-major in shared
-// memory, the layer weights transposed (Wt[k][n]) beside them, and each of the
+// memory, the layer weights transposed (Wt[k][n]) beside them, and each of
 // 256 threads accumulates an 8-point x 4-output block, so every k step costs
-// three 16-byte shared loads for 32 FMAs. Layers: encoding (32) -> 64 -> 64
+// three 16-byte shared loads for 32 FMAs. The CTA holds two such groups of 256
+// threads, each with its own tile and activations and its own named barrier,
+// sharing the weights: one group's table gathers overlap the other's GEMMs. Layers: encoding (32) -> 64 -> 64
 // (ReLU) -> sigma = ReLU(w . h + b); [h | SH16(d)] (80) -> 64 -> 64 (ReLU) ->
 // rgb = sigmoid(W h + b). All arithmetic is fp32 on the CUDA cores.
 constexpr int HASH_NW = 15876;                       // fp32 weights of the ABI blob
@@ -400,49 +402,70 @@ constexpr int HT_P = NERF_HT_P;                      // points per tile (128 or 
 constexpr int HT_PPT = HT_P / 16;                    // points per thread in the GEMMs
 constexpr int HT_TPP = 256 / HT_P;                   // threads per point in the encoding
 constexpr int HT_AP = HT_P + 4;                      // padded row of an activation buffer
-constexpr int HT_THREADS = 256;
-constexpr int HT_CTAS_PER_SM = HT_P == 128 ? 1 : 2;
+constexpr int HT_GROUPS = 2;                         // independent tile groups per CTA
+constexpr int HT_THREADS = 256 * HT_GROUPS;
+constexpr int HT_CTAS_PER_SM = 1;
 // shared-memory layout (floats)
 constexpr int HT_D0 = 0, HT_D1 = HT_D0 + 32 * 64, HT_C0 = HT_D1 + 64 * 64, HT_C1 = HT_C0 + 80 * 64;
 constexpr int HT_VEC = HT_C1 + 64 * 64;              // d0b d1b c0b c1b sw (5 x 64), sb, pad, rw (192), rb
-constexpr int HT_ACT_A = HT_VEC + 5 * 64 + 4 + 192 + 4;
+constexpr int HT_GRP = HT_VEC + 5 * 64 + 4 + 192 + 4;  // first group's buffers
+// per group: act_a [80][HT_AP], act_b [64][HT_AP], sig [HT_P], rgb [3][HT_P]
+constexpr int HT_ACT_A = 0;
 constexpr int HT_ACT_B = HT_ACT_A + 80 * HT_AP;
 constexpr int HT_SIG = HT_ACT_B + 64 * HT_AP;
 constexpr int HT_RGB = HT_SIG + HT_P;
-constexpr int HT_FLOATS = HT_RGB + 3 * HT_P;
+constexpr int HT_GRP_FLOATS = HT_RGB + 3 * HT_P;
+constexpr int HT_FLOATS = HT_GRP + HT_GROUPS * HT_GRP_FLOATS;
 constexpr size_t HT_SMEM = HT_FLOATS * sizeof(float);
-static_assert(HT_ACT_A % 4 == 0 && HT_ACT_B % 4 == 0 && HT_AP % 4 == 0, "float4 alignment");
+static_assert(HT_GRP % 4 == 0 && HT_ACT_B % 4 == 0 && HT_GRP_FLOATS % 4 == 0 && HT_AP % 4 == 0,
+              "float4 alignment");
 
-// out[n][p] = act(b[n] + sum_k W[n][k] in[k][p]) for the tile, N = 64.
+// Barrier of one 256-thread group (ids 1 and 2; 0 is __syncthreads).
+__device__ __forceinline__ void group_sync(int g) {
+  asm volatile("bar.sync %0, 256;" ::"r"(1 + g) : "memory");
+}
+
+// The staged weights and biases keep output n in column perm64(n), so that
+// thread tx's four columns 4 tx .. 4 tx + 3 hold outputs tx, tx + 16, tx + 32,
+// tx + 48: its epilogue then stores four feature rows 16 apart, which fall in
+// distinct shared-memory banks across the warp.
+__device__ __forceinline__ int perm64(int n) { return 4 * (n & 15) + (n >> 4); }
+
+// out[n][p] = act(b[n] + sum_k W[n][k] in[k][p]) for the tile, N = 64; the
+// operands of step k + 1 are loaded while step k computes.
 template <int K>
 __device__ __forceinline__ void tile_dense64(const float* __restrict__ Wt, const float* __restrict__ b,
-                                             const float* in, float* out) {
-  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+                                             const float* in, float* out, int lt) {
+  const int tx = lt & 15, ty = lt >> 4;
   const int n0 = 4 * tx, p0 = HT_PPT * ty;
+  static_assert(HT_PPT == 8, "two float4 of points per thread");
   float acc[HT_PPT][4];
   const float4 bb = *reinterpret_cast<const float4*>(b + n0);
 #pragma unroll
   for (int i = 0; i < HT_PPT; ++i) { acc[i][0] = bb.x; acc[i][1] = bb.y; acc[i][2] = bb.z; acc[i][3] = bb.w; }
+  float4 a0 = *reinterpret_cast<const float4*>(in + p0);
+  float4 a1 = *reinterpret_cast<const float4*>(in + p0 + 4);
+  float4 w = *reinterpret_cast<const float4*>(Wt + n0);
 #pragma unroll 4
   for (int k = 0; k < K; ++k) {
-    float a[HT_PPT];
-#pragma unroll
-    for (int v = 0; v < HT_PPT / 4; ++v) {
-      const float4 a4 = *reinterpret_cast<const float4*>(in + k * HT_AP + p0 + 4 * v);
-      a[4 * v] = a4.x; a[4 * v + 1] = a4.y; a[4 * v + 2] = a4.z; a[4 * v + 3] = a4.w;
+    const float a[HT_PPT] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+    const float4 wc = w;
+    if (k + 1 < K) {
+      a0 = *reinterpret_cast<const float4*>(in + (k + 1) * HT_AP + p0);
+      a1 = *reinterpret_cast<const float4*>(in + (k + 1) * HT_AP + p0 + 4);
+      w = *reinterpret_cast<const float4*>(Wt + (k + 1) * 64 + n0);
     }
-    const float4 w = *reinterpret_cast<const float4*>(Wt + k * 64 + n0);
 #pragma unroll
     for (int i = 0; i < HT_PPT; ++i) {
-      acc[i][0] = fmaf(w.x, a[i], acc[i][0]);
-      acc[i][1] = fmaf(w.y, a[i], acc[i][1]);
-      acc[i][2] = fmaf(w.z, a[i], acc[i][2]);
-      acc[i][3] = fmaf(w.w, a[i], acc[i][3]);
+      acc[i][0] = fmaf(wc.x, a[i], acc[i][0]);
+      acc[i][1] = fmaf(wc.y, a[i], acc[i][1]);
+      acc[i][2] = fmaf(wc.z, a[i], acc[i][2]);
+      acc[i][3] = fmaf(wc.w, a[i], acc[i][3]);
     }
   }
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
-    float* o = out + (n0 + j) * HT_AP + p0;
+    float* o = out + (tx + 16 * j) * HT_AP + p0;
 #pragma unroll
     for (int v = 0; v < HT_PPT / 4; ++v)
       *reinterpret_cast<float4*>(o + 4 * v) =
@@ -469,32 +492,36 @@ hash_eval_kernel(const float* __restrict__ o, const float* __restrict__ d, int64
   float* sb = sw + 64;                 // [1] + pad
   float* rw = sb + 4;                  // [3][64]
   float* rb = rw + 192;                // [3]
-  float* act_a = hs + HT_ACT_A;        // [80][HT_AP]: encoding, then h2 | SH, then the last h
-  float* act_b = hs + HT_ACT_B;        // [64][HT_AP]
-  float* sig = hs + HT_SIG;
-  float* rgbv = hs + HT_RGB;           // [3][HT_P]
+  const int grp = threadIdx.x >> 8, lt = threadIdx.x & 255;
+  float* gb = hs + HT_GRP + grp * HT_GRP_FLOATS;
+  float* act_a = gb + HT_ACT_A;        // [80][HT_AP]: encoding, then h2 | SH, then the last h
+  float* act_b = gb + HT_ACT_B;        // [64][HT_AP]
+  float* sig = gb + HT_SIG;
+  float* rgbv = gb + HT_RGB;           // [3][HT_P]
   // weights of the ABI blob (row-major W[n][k]) -> transposed Wt[k][n]
   for (int q = threadIdx.x; q < HASH_NW; q += HT_THREADS) {
     const float v = mlp[q];
-    if (q < 2048) { d0t[(q % 32) * 64 + q / 32] = v; }
-    else if (q < 2112) { d0b[q - 2048] = v; }
-    else if (q < 6208) { const int z = q - 2112; d1t[(z % 64) * 64 + z / 64] = v; }
-    else if (q < 6272) { d1b[q - 6208] = v; }
+    if (q < 2048) { d0t[(q % 32) * 64 + perm64(q / 32)] = v; }
+    else if (q < 2112) { d0b[perm64(q - 2048)] = v; }
+    else if (q < 6208) { const int z = q - 2112; d1t[(z % 64) * 64 + perm64(z / 64)] = v; }
+    else if (q < 6272) { d1b[perm64(q - 6208)] = v; }
     else if (q < 6336) { sw[q - 6272] = v; }
     else if (q < 6337) { sb[0] = v; }
-    else if (q < 11457) { const int z = q - 6337; c0t[(z % 80) * 64 + z / 80] = v; }
-    else if (q < 11521) { c0b[q - 11457] = v; }
-    else if (q < 15617) { const int z = q - 11521; c1t[(z % 64) * 64 + z / 64] = v; }
-    else if (q < 15681) { c1b[q - 15617] = v; }
+    else if (q < 11457) { const int z = q - 6337; c0t[(z % 80) * 64 + perm64(z / 80)] = v; }
+    else if (q < 11521) { c0b[perm64(q - 11457)] = v; }
+    else if (q < 15617) { const int z = q - 11521; c1t[(z % 64) * 64 + perm64(z / 64)] = v; }
+    else if (q < 15681) { c1b[perm64(q - 15617)] = v; }
     else if (q < 15873) { rw[q - 15681] = v; }
     else { rb[q - 15873] = v; }
   }
+  __syncthreads();       // the weights are staged
   const int64_t P = *total;
-  const int p = threadIdx.x & (HT_P - 1);
-  const int part = threadIdx.x / HT_P;          // 0 .. HT_TPP - 1
-  for (int64_t i0 = (int64_t)blockIdx.x * HT_P; i0 < P; i0 += (int64_t)gridDim.x * HT_P) {
+  const int p = lt & (HT_P - 1);
+  const int part = lt / HT_P;                   // 0 .. HT_TPP - 1
+  for (int64_t i0 = ((int64_t)blockIdx.x * HT_GROUPS + grp) * HT_P; i0 < P;
+       i0 += (int64_t)gridDim.x * HT_GROUPS * HT_P) {
     const int n = (int)min((int64_t)HT_P, P - i0);
-    __syncthreads();     // the previous tile's last reads (and the weight staging) are over
+    group_sync(grp);     // the group's previous tile's last reads are over
     // encoding: HT_TPP threads per point, each 16 / HT_TPP of the levels; the
     // last also writes SH16 of the unit direction into rows 64..79
     {
@@ -524,29 +551,29 @@ hash_eval_kernel(const float* __restrict__ o, const float* __restrict__ d, int64
         for (int j = 0; j < 16; ++j) act_a[(64 + j) * HT_AP + p] = p < n ? sh[j] : 0.f;
       }
     }
-    __syncthreads();
-    tile_dense64<32>(d0t, d0b, act_a, act_b);          // 32 -> 64
-    __syncthreads();
-    tile_dense64<64>(d1t, d1b, act_b, act_a);          // 64 -> 64: h2 in rows 0..63
-    __syncthreads();
+    group_sync(grp);
+    tile_dense64<32>(d0t, d0b, act_a, act_b, lt);          // 32 -> 64
+    group_sync(grp);
+    tile_dense64<64>(d1t, d1b, act_b, act_a, lt);          // 64 -> 64: h2 in rows 0..63
+    group_sync(grp);
     if (part == 0) {                                   // sigma = ReLU(sw . h2 + sb)
       float s = sb[0];
 #pragma unroll 8
       for (int j = 0; j < 64; ++j) s = fmaf(sw[j], act_a[j * HT_AP + p], s);
       sig[p] = fmaxf(s, 0.0f);
     }
-    tile_dense64<80>(c0t, c0b, act_a, act_b);          // [h2 | SH16] -> 64
-    __syncthreads();
-    tile_dense64<64>(c1t, c1b, act_b, act_a);          // 64 -> 64
-    __syncthreads();
-    for (int q = threadIdx.x; q < 3 * HT_P; q += HT_THREADS) {   // rgb head
+    tile_dense64<80>(c0t, c0b, act_a, act_b, lt);          // [h2 | SH16] -> 64
+    group_sync(grp);
+    tile_dense64<64>(c1t, c1b, act_b, act_a, lt);          // 64 -> 64
+    group_sync(grp);
+    for (int q = lt; q < 3 * HT_P; q += 256) {   // rgb head
       const int c = q / HT_P, pp = q % HT_P;
       float v = rb[c];
 #pragma unroll 8
       for (int j = 0; j < 64; ++j) v = fmaf(rw[c * 64 + j], act_a[j * HT_AP + pp], v);
       rgbv[c * HT_P + pp] = 1.0f / (1.0f + expf(-v));
     }
-    __syncthreads();
+    group_sync(grp);
     if (part == 0 && p < n)
       reinterpret_cast<float4*>(out)[i0 + p] =
           make_float4(rgbv[p], rgbv[HT_P + p], rgbv[2 * HT_P + p], sig[p]);
