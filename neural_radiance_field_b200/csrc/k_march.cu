@@ -677,8 +677,10 @@ constexpr int KT_RGB = KT_SIG + KT_P;
 constexpr int KT_FLOATS = KT_RGB + 3 * KT_P;
 constexpr size_t KT_SMEM = KT_FLOATS * sizeof(float);
 static_assert(KT_ACT >= KILO_NP && KT_ACT % 4 == 0 && KT_H1 % 4 == 0, "layout");
+static_assert(2 * KT_THREADS - 3 * KT_P == KT_P, "the heads' second round leaves KT_P threads for sigma");
 
-// out[n][p] = ReLU(b[n] + sum_k W[n][k] in[k][p]), N = 32.
+// out[n][p] = ReLU(b[n] + sum_k W[n][k] in[k][p]), N = 32; the operands of
+// step k + 1 are loaded while step k computes.
 template <int K>
 __device__ __forceinline__ void tile_dense32(const float* __restrict__ Wt, const float* __restrict__ b,
                                              const float* in, float* out) {
@@ -689,10 +691,16 @@ __device__ __forceinline__ void tile_dense32(const float* __restrict__ Wt, const
   for (int i = 0; i < 4; ++i)
 #pragma unroll
     for (int j = 0; j < 4; ++j) acc[i][j] = b[n0 + j];
+  float4 an = *reinterpret_cast<const float4*>(in + p0);
+  float4 wn = *reinterpret_cast<const float4*>(Wt + n0);
 #pragma unroll 7
   for (int k = 0; k < K; ++k) {
-    const float4 a4 = *reinterpret_cast<const float4*>(in + k * KT_AP + p0);
-    const float4 w = *reinterpret_cast<const float4*>(Wt + k * 32 + n0);
+    const float4 a4 = an;
+    const float4 w = wn;
+    if (k + 1 < K) {
+      an = *reinterpret_cast<const float4*>(in + (k + 1) * KT_AP + p0);
+      wn = *reinterpret_cast<const float4*>(Wt + (k + 1) * 32 + n0);
+    }
     const float a[4] = {a4.x, a4.y, a4.z, a4.w};
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
@@ -771,12 +779,14 @@ kilo_eval_kernel(const float* __restrict__ o, const float* __restrict__ d, int64
         r = r0 + (e >> 9);
         march_point(o, d, r, near, step, (int)(e & 511u), x, &t);
       }
+      // the 42 sin/cos pairs split about evenly: part 0 takes position coordinates
+      // 0 and 1 (20), part 1 coordinate 2 and the direction (10 + 12)
       if (part == 0) {
         act[0 * KT_AP + p] = x[0];
         act[1 * KT_AP + p] = x[1];
         act[2 * KT_AP + p] = x[2];
 #pragma unroll
-        for (int c = 0; c < 3; ++c)
+        for (int c = 0; c < 2; ++c)
 #pragma unroll
           for (int k = 0; k < 10; ++k) {
             float sn, cs;
@@ -785,6 +795,13 @@ kilo_eval_kernel(const float* __restrict__ o, const float* __restrict__ d, int64
             act[(33 + c * 10 + k) * KT_AP + p] = cs;
           }
       } else {
+#pragma unroll
+        for (int k = 0; k < 10; ++k) {
+          float sn, cs;
+          pe_sincos(x[2], k, &sn, &cs);
+          act[(3 + 20 + k) * KT_AP + p] = sn;
+          act[(33 + 20 + k) * KT_AP + p] = cs;
+        }
         const float dx = d[r * 3], dy = d[r * 3 + 1], dz = d[r * 3 + 2];
         const float inv = 1.0f / sqrtf(dx * dx + dy * dy + dz * dz);
         const float u[3] = {dx * inv, dy * inv, dz * inv};
@@ -807,11 +824,14 @@ kilo_eval_kernel(const float* __restrict__ o, const float* __restrict__ d, int64
     __syncthreads();
     tile_dense32<32>(w2t, b2, h1, act);                // h1 -> h2 (rows 0..31)
     __syncthreads();
-    if (part == 0) {
+    // heads: 3 KT_P rgb items and KT_P sigma items over two rounds of the 256
+    // threads (sigma on the threads the rgb items leave idle in the second round)
+    if (threadIdx.x >= 3 * KT_P - KT_THREADS) {
+      const int pp = threadIdx.x - (3 * KT_P - KT_THREADS);
       float s = bs[0];
 #pragma unroll 8
-      for (int k = 0; k < 32; ++k) s = fmaf(ws[k], act[k * KT_AP + p], s);
-      sig[p] = fmaxf(s, 0.0f);
+      for (int k = 0; k < 32; ++k) s = fmaf(ws[k], act[k * KT_AP + pp], s);
+      sig[pp] = fmaxf(s, 0.0f);
     }
     for (int q = threadIdx.x; q < 3 * KT_P; q += KT_THREADS) {
       const int c = q / KT_P, pp = q % KT_P;
