@@ -582,45 +582,72 @@ hash_eval_kernel(const float* __restrict__ o, const float* __restrict__ d, int64
 
 // ------------------------------------------------------------------ KiloNeRF
 
+// The cell routing counts and scatters with one atomic per distinct cell among
+// a warp's 32 points (__match_any_sync): consecutive live entries lie along one
+// ray and share few cells, so hot cells see far fewer contended atomics. The
+// loops step by whole warps so that every lane takes part in the match.
+__device__ __forceinline__ void warp_hist_add(int32_t* hist, int id, int lane) {
+  const unsigned peers = __match_any_sync(0xffffffffu, id);
+  if (id >= 0 && lane == __ffs(peers) - 1) atomicAdd(&hist[id], __popc(peers));
+}
+
 __global__ void cell_hist_kernel(const float* __restrict__ o, const float* __restrict__ d,
                                  int64_t r0, float near, float step,
                                  const uint32_t* __restrict__ live, const int32_t* __restrict__ total,
                                  int32_t* __restrict__ cell, int32_t* __restrict__ hist) {
   const int64_t P = *total;
-  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < P;
-       i += (int64_t)gridDim.x * blockDim.x) {
-    const uint32_t e = live[i];
-    float x[3], t;
-    march_point(o, d, r0 + (e >> 9), near, step, (int)(e & 511u), x, &t);
-    const int a = voxel_axis(x[0]), b = voxel_axis(x[1]), c = voxel_axis(x[2]);
-    const int id = ((a >> 3) * 16 + (b >> 3)) * 16 + (c >> 3);
-    cell[i] = id;
-    atomicAdd(&hist[id], 1);
+  const int lane = threadIdx.x & 31;
+  for (int64_t i0 = (int64_t)blockIdx.x * blockDim.x + (threadIdx.x & ~31); i0 < P;
+       i0 += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t i = i0 + lane;
+    int id = -1;
+    if (i < P) {
+      const uint32_t e = live[i];
+      float x[3], t;
+      march_point(o, d, r0 + (e >> 9), near, step, (int)(e & 511u), x, &t);
+      const int a = voxel_axis(x[0]), b = voxel_axis(x[1]), c = voxel_axis(x[2]);
+      id = ((a >> 3) * 16 + (b >> 3)) * 16 + (c >> 3);
+      cell[i] = id;
+    }
+    warp_hist_add(hist, id, lane);
   }
 }
 
 __global__ void cell_hist_points_kernel(const float* __restrict__ x, int64_t n,
                                         int32_t* __restrict__ cell, int32_t* __restrict__ hist,
                                         unsigned* flag) {
-  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  if (i >= n) return;
-  const int a = voxel_axis(x[i * 3]), b = voxel_axis(x[i * 3 + 1]), c = voxel_axis(x[i * 3 + 2]);
-  if (a < 0 || b < 0 || c < 0) { cell[i] = -1; atomicOr(flag, FLAG_BAD_INDEX); return; }
-  const int id = ((a >> 3) * 16 + (b >> 3)) * 16 + (c >> 3);
-  cell[i] = id;
-  atomicAdd(&hist[id], 1);
+  const int lane = threadIdx.x & 31;
+  const int64_t i0 = (int64_t)blockIdx.x * blockDim.x + (threadIdx.x & ~31);
+  if (i0 >= n) return;                         // whole warps only
+  const int64_t i = i0 + lane;
+  int id = -1;
+  if (i < n) {
+    const int a = voxel_axis(x[i * 3]), b = voxel_axis(x[i * 3 + 1]), c = voxel_axis(x[i * 3 + 2]);
+    if (a < 0 || b < 0 || c < 0) {
+      atomicOr(flag, FLAG_BAD_INDEX);
+    } else {
+      id = ((a >> 3) * 16 + (b >> 3)) * 16 + (c >> 3);
+    }
+    cell[i] = id;
+  }
+  warp_hist_add(hist, id, lane);
 }
 
 __global__ void cell_scatter_kernel(const int32_t* __restrict__ cell, const int32_t* __restrict__ total,
                                     int64_t n_fixed, const int32_t* __restrict__ cell_off,
                                     int32_t* __restrict__ fill, int32_t* __restrict__ order) {
   const int64_t P = total ? (int64_t)*total : n_fixed;
-  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < P;
-       i += (int64_t)gridDim.x * blockDim.x) {
-    const int c = cell[i];
-    if (c < 0) continue;
-    const int pos = cell_off[c] + atomicAdd(&fill[c], 1);
-    order[pos] = (int32_t)i;
+  const int lane = threadIdx.x & 31;
+  for (int64_t i0 = (int64_t)blockIdx.x * blockDim.x + (threadIdx.x & ~31); i0 < P;
+       i0 += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t i = i0 + lane;
+    const int c = i < P ? cell[i] : -1;
+    const unsigned peers = __match_any_sync(0xffffffffu, c);
+    const int leader = __ffs(peers) - 1;
+    int base = 0;
+    if (c >= 0 && lane == leader) base = atomicAdd(&fill[c], __popc(peers));
+    base = __shfl_sync(0xffffffffu, base, leader);
+    if (c >= 0) order[cell_off[c] + base + __popc(peers & ((1u << lane) - 1u))] = (int32_t)i;
   }
 }
 
