@@ -608,7 +608,8 @@ def run_march(args, rank, world, local_rank):
     from neural_radiance_field_b200 import build as nbuild
     nbuild.build()
     torch.cuda.set_device(local_rank)
-    wl = S.WORKLOADS[args.workload]
+    tc = args.workload == "hashgrid_bf16"
+    wl = S.WORKLOADS["hashgrid" if tc else args.workload]
     if args.size:
         import dataclasses
         wl = dataclasses.replace(wl, H=args.size, W=args.size, focal=1.25 * args.size)
@@ -628,13 +629,16 @@ def run_march(args, rank, world, local_rank):
         mlp = torch.from_numpy(S.hash_mlp_weights(wl.seed)).cuda()
         kw = dict(occupancy=occ, hash_table=table, hash_mlp=mlp)
         flop_per_point, kname = 2 * 15616, "hash_eval_kernel (encoding + MLPs)"
+        if tc:
+            kname = "hash_tc_kernel (fp32 encoding, MLP on the tensor cores in bf16)"
     o = torch.empty(R, 3, device="cuda")
     d = torch.empty(R, 3, device="cuda")
     rgb = torch.empty(R, 3, device="cuda")
     dep = torch.empty(R, device="cuda")
     acc = torch.empty(R, device="cuda")
     flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
-    rnd = nb.Renderer(model=model, max_rays=R, max_samples=wl.n_coarse)
+    rnd = nb.Renderer(model=model, max_rays=R, max_samples=wl.n_coarse,
+                      precision=S.PREC_BF16 if tc else S.PREC_FP32)
     p = rnd.params(march_step=wl.march_step, ert_T=wl.ert_T, **kw)
     nb.nerf_raygen(wl.H, wl.W, wl.focal, c2w, o, d)
     cnt = torch.empty(R, dtype=torch.int32, device="cuda")
@@ -671,7 +675,19 @@ def run_march(args, rank, world, local_rank):
     peak = 148 * 128 * 2 * sm_mhz * 1e6 / 1e12
     per_frame_k_ms = k_ms / args.steps
     achieved = live * flop_per_point / (per_frame_k_ms * 1e-3) / 1e12
-    line = {"metric": f"rays/sec, {wl.name} march render", "value": R * args.steps / (tot_ms * 1e-3),
+    roofline = {"bound": "alu", "kernel": kname, "achieved": achieved, "peak": peak,
+                "unit": "TFLOP/s", "frac": achieved / peak, "peak_kind": FP32_PEAK_NOTE,
+                "traffic": None, "kernel_ms_per_frame": per_frame_k_ms,
+                "flop_per_point": flop_per_point}
+    if tc:
+        # the MLP's FLOPs run on the tensor cores; the kernel is bound by the fp32
+        # encoding (128 table gathers per point), so this fraction is small
+        peaks, pk = load_peaks()
+        bf = peaks.get("bf16_tflops")
+        roofline.update({"bound": "tensor", "peak": bf, "frac": achieved / bf if bf else None,
+                         "peak_kind": f"bf16 burst, {pk}"})
+    line = {"metric": f"rays/sec, {wl.name} march render" + (", MLP in bf16 on the tensor cores" if tc else ""),
+            "value": R * args.steps / (tot_ms * 1e-3),
             "unit": UNIT, "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": tot_ms / args.steps, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f32", "data": "synthetic",
@@ -680,10 +696,7 @@ def run_march(args, rank, world, local_rank):
                        "occupied_candidates_per_frame": live,
                        "l2": "flushed between timed steps (256 MiB write)"},
             "sample_points_per_s": live * args.steps / (tot_ms * 1e-3),
-            "roofline": {"bound": "alu", "kernel": kname, "achieved": achieved, "peak": peak,
-                         "unit": "TFLOP/s", "frac": achieved / peak, "peak_kind": FP32_PEAK_NOTE,
-                         "traffic": None, "kernel_ms_per_frame": per_frame_k_ms,
-                         "flop_per_point": flop_per_point},
+            "roofline": roofline,
             "gpu_launches": args.steps * march_launches_per_step(wl.model, R), "clocks": clocks}
     print(json.dumps(line), flush=True)
     rnd.close()
@@ -723,7 +736,7 @@ def main():
     ap.add_argument("--ref-rays", type=int, default=128)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--workload", default=WORKLOAD,
-                    choices=[WORKLOAD, "kilonerf", "hashgrid", "sweep24", "compact", "train",
+                    choices=[WORKLOAD, "kilonerf", "hashgrid", "hashgrid_bf16", "sweep24", "compact", "train",
                              "hash_backward"],
                     help="the benchmark workload (default) or a march workload (extra lines)")
     ap.add_argument("--traffic-bytes", type=float, default=0.0,

@@ -4,6 +4,7 @@
 // router (KiloNeRF page, abstract), and compositing with early termination.
 #include <cmath>
 
+#include "tc_ptx.cuh"
 #include "nerf_march.cuh"
 
 namespace nerfb {
@@ -580,6 +581,253 @@ hash_eval_kernel(const float* __restrict__ o, const float* __restrict__ d, int64
   }
 }
 
+// The hash scene function with its MLP on the tensor cores (bf16 operands,
+// fp32 accumulation in tensor memory): the reading of the Instant-NGP pages'
+// tiny MLP as an optional bf16 path. The encoding and the heads stay fp32; the
+// 32 encoded features, SH16(d) and the hidden activations are rounded to bf16
+// as the MMAs' A operand, and the weights to bf16 when staged.
+//
+// One CTA per SM: warp 0 issues the MMAs (one elected thread), and four groups
+// of four warps each own a tile of 128 live points (thread = point = TMEM lane).
+// A group encodes its tile into a bf16 operand buffer in shared memory ([enc (32)
+// | h (64, overwriting enc) | SH16 at K 64..79]), then drains its 64 TMEM
+// columns after each layer (+ bias, ReLU, bf16 back into the buffer). Layers:
+// 32 -> 64 -> 64 (sigma head), [h | SH16] (80) -> 64 -> 64 (rgb head). The MMA
+// thread interleaves the four tiles layer by layer (M = 128, N = 64, K = 16
+// steps), so that one tile's epilogue overlaps the others' MMAs and encodings.
+constexpr int HC_GROUPS = 4;
+constexpr int HC_P = 128;                                   // points per tile
+constexpr int HC_THREADS = 32 + HC_GROUPS * HC_P;
+constexpr int HC_W1 = 0;                                    // bf16 weights, bytes
+constexpr int HC_W2 = HC_W1 + 64 * 32 * 2;
+constexpr int HC_W3 = HC_W2 + 64 * 64 * 2;
+constexpr int HC_W4 = HC_W3 + 64 * 80 * 2;
+constexpr int HC_VEC = HC_W4 + 64 * 64 * 2;                 // fp32: b1..b4, ws, bs, rw, rb
+constexpr int HC_NV = 4 * 64 + 64 + 4 + 3 * 64 + 4;
+constexpr int HC_A = (HC_VEC + HC_NV * 4 + 1023) / 1024 * 1024;   // per group 128 x 80 bf16
+constexpr int HC_A_BYTES = HC_P * 80 * 2;
+constexpr int HC_BARS = HC_A + HC_GROUPS * HC_A_BYTES;
+constexpr size_t HC_SMEM = HC_BARS + (2 * HC_GROUPS + 1) * 8 + 16;
+static_assert(HC_A % 128 == 0 && HC_VEC % 16 == 0, "operand alignment");
+
+// Byte offset of K-group kg (8 bf16) of row r in a 128-row operand buffer, and of
+// output n, K-group kg in a 64-row weight matrix.
+__device__ __forceinline__ uint32_t hc_a_off(int r, int kg) {
+  return (uint32_t)(kg * (HC_P * 16) + (r >> 3) * 128 + (r & 7) * 16);
+}
+__device__ __forceinline__ uint32_t hc_w_off(int n, int k) {
+  return (uint32_t)((k >> 3) * (64 * 16) + (n >> 3) * 128 + (n & 7) * 16 + (k & 7) * 2);
+}
+
+// The MMAs of one layer for one tile: KS steps of K = 16 into 64 TMEM columns.
+template <int KS>
+__device__ __forceinline__ void hc_layer_mma(uint32_t d, uint64_t a, uint64_t b) {
+  constexpr uint32_t idesc = (1u << 4) | (1u << 7) | (1u << 10) | ((64u >> 3) << 17) |
+                             ((uint32_t)(HC_P >> 4) << 24);     // M = 128, N = 64
+#pragma unroll
+  for (int s = 0; s < KS; ++s)
+    tcx::mma_bf16(d, a + (uint64_t)((s * 2 * HC_P * 16) >> 4), b + (uint64_t)((s * 2 * 64 * 16) >> 4),
+                  idesc, s != 0);
+}
+
+__global__ void __launch_bounds__(HC_THREADS, 1)
+hash_tc_kernel(const float* __restrict__ o, const float* __restrict__ d, int64_t r0, float near,
+               float step, const uint32_t* __restrict__ live, const int32_t* __restrict__ total,
+               const __half2* __restrict__ table, const float* __restrict__ mlp, ShConst K,
+               float* __restrict__ out, unsigned* flag) {
+  extern __shared__ __align__(1024) uint8_t hsm[];
+  float* vec = reinterpret_cast<float*>(hsm + HC_VEC);
+  float* b1 = vec;
+  float* ws = vec + 4 * 64;
+  float* rw = ws + 68;                                      // [3][64]
+  uint64_t* a_ready = reinterpret_cast<uint64_t*>(hsm + HC_BARS);   // [groups]
+  uint64_t* mma_done = a_ready + HC_GROUPS;                          // [groups]
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(mma_done + HC_GROUPS + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+  constexpr uint64_t kLimit = 2000000000ull;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  // weights of the blob (row-major W[n][k], layer order d0, d1, sigma, c0, c1, rgb)
+  // -> bf16 core-matrix operands; biases and head weights stay fp32
+  for (int q = threadIdx.x; q < HASH_NW; q += HC_THREADS) {
+    const float v = mlp[q];
+    auto wput = [&](int base, int K_, int z) {
+      const int n = z / K_, k = z % K_;
+      *reinterpret_cast<__nv_bfloat16*>(hsm + base + hc_w_off(n, k)) = __float2bfloat16_rn(v);
+    };
+    if (q < 2048) wput(HC_W1, 32, q);
+    else if (q < 2112) b1[q - 2048] = v;
+    else if (q < 6208) wput(HC_W2, 64, q - 2112);
+    else if (q < 6272) b1[64 + q - 6208] = v;
+    else if (q < 6336) ws[q - 6272] = v;
+    else if (q < 6337) ws[64] = v;
+    else if (q < 11457) wput(HC_W3, 80, q - 6337);
+    else if (q < 11521) b1[128 + q - 11457] = v;
+    else if (q < 15617) wput(HC_W4, 64, q - 11521);
+    else if (q < 15681) b1[192 + q - 15617] = v;
+    else if (q < 15873) rw[q - 15681] = v;
+    else rw[192 + q - 15873] = v;
+  }
+  if (threadIdx.x == 0) {
+    for (int g = 0; g < HC_GROUPS; ++g) {
+      tcx::mbar_init(&a_ready[g], 4);          // one arrival per warp of the group
+      tcx::mbar_init(&mma_done[g], 1);
+    }
+    tcx::mbar_init(&mma_done[HC_GROUPS], 1);   // final drain
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 0) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
+                 ::"r"(tcx::smem_u32(tmem_holder)), "r"(HC_GROUPS * 64));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+  tcx::fence_async_smem();                     // the staged weights, for the tensor cores
+  tcx::fence_before();
+  __syncthreads();
+  tcx::fence_after();
+  const uint32_t tmem = *tmem_holder;
+  const int64_t P = *total;
+  // tile (round k, group g): points [T * 128, T * 128 + 128), T = (k * grid + block) * groups + g
+  auto tile_of = [&](int64_t k, int g) {
+    return (k * gridDim.x + blockIdx.x) * HC_GROUPS + g;
+  };
+
+  if (warp == 0) {
+    if (lane == 0) {
+      uint32_t ph[HC_GROUPS] = {0, 0, 0, 0};
+      const uint32_t a0 = tcx::smem_u32(hsm + HC_A);
+      const uint32_t wb = tcx::smem_u32(hsm);
+      bool ok = true;
+      for (int64_t k = 0; ok; ++k) {
+        int active = 0;
+        while (active < HC_GROUPS && tile_of(k, active) * HC_P < P) ++active;
+        if (active == 0) break;
+        for (int l = 0; l < 4 && ok; ++l) {
+          for (int g = 0; g < active; ++g) {
+            if (!tcx::mbar_wait(&a_ready[g], ph[g], abort_flag, flag, kLimit)) { ok = false; break; }
+            ph[g] ^= 1;
+            tcx::fence_after();
+            const uint64_t a = tcx::sdesc(a0 + g * HC_A_BYTES, HC_P * 16, 128);
+            const uint32_t dt = tmem + 64 * g;
+            if (l == 0) hc_layer_mma<2>(dt, a, tcx::sdesc(wb + HC_W1, 64 * 16, 128));
+            else if (l == 1) hc_layer_mma<4>(dt, a, tcx::sdesc(wb + HC_W2, 64 * 16, 128));
+            else if (l == 2) hc_layer_mma<5>(dt, a, tcx::sdesc(wb + HC_W3, 64 * 16, 128));
+            else hc_layer_mma<4>(dt, a, tcx::sdesc(wb + HC_W4, 64 * 16, 128));
+            tcx::mma_commit(&mma_done[g]);
+          }
+        }
+      }
+      // drain before TMEM is freed
+      uint64_t* fin = mma_done + HC_GROUPS;
+      tcx::mma_commit(fin);
+      const uint64_t t0 = tcx::globaltimer();
+      while (!tcx::mbar_try(fin, 0) && tcx::globaltimer() - t0 < kLimit) {}
+    }
+  } else {
+    const int g = (warp - 1) >> 2;
+    const int r = (warp & 3) * 32 + lane;                  // TMEM lane = row of the tile
+    const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+    const uint32_t abase = tcx::smem_u32(hsm + HC_A + g * HC_A_BYTES);
+    uint32_t pd = 0;
+    for (int64_t k = 0;; ++k) {
+      const int64_t T = tile_of(k, g);
+      if (T * HC_P >= P) break;
+      const int64_t i = T * HC_P + r;
+      const bool valid = i < P;
+      // encoding: 16 levels x 2 features and SH16 of the unit direction, bf16
+      {
+        float x[3] = {0.f, 0.f, 0.f}, t;
+        int64_t ray = r0;
+        if (valid) {
+          const uint32_t e = live[i];
+          ray = r0 + (e >> 9);
+          march_point(o, d, ray, near, step, (int)(e & 511u), x, &t);
+        }
+        float u0, u1, u2;
+        hash_unit_coords(x[0], x[1], x[2], u0, u1, u2);
+#pragma unroll 1
+        for (int l2 = 0; l2 < 16; l2 += 4) {
+          float f[8];
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            f[2 * j] = 0.f;
+            f[2 * j + 1] = 0.f;
+            if (valid) hash_encode_level(table, u0, u1, u2, l2 + j, nullptr, f[2 * j], f[2 * j + 1]);
+          }
+          tcx::st_shared_v4(abase + hc_a_off(r, l2 / 4), tcx::pack_bf16(f[0], f[1]),
+                            tcx::pack_bf16(f[2], f[3]), tcx::pack_bf16(f[4], f[5]),
+                            tcx::pack_bf16(f[6], f[7]));
+        }
+        float sh[16];
+        const float dx = d[ray * 3], dy = d[ray * 3 + 1], dz = d[ray * 3 + 2];
+        const float inv = 1.0f / sqrtf(dx * dx + dy * dy + dz * dz);
+        sh16(dx * inv, dy * inv, dz * inv, K, sh);
+#pragma unroll
+        for (int j = 0; j < 2; ++j)
+          tcx::st_shared_v4(abase + hc_a_off(r, 8 + j), tcx::pack_bf16(sh[8 * j], sh[8 * j + 1]),
+                            tcx::pack_bf16(sh[8 * j + 2], sh[8 * j + 3]),
+                            tcx::pack_bf16(sh[8 * j + 4], sh[8 * j + 5]),
+                            tcx::pack_bf16(sh[8 * j + 6], sh[8 * j + 7]));
+        tcx::fence_async_smem();
+        __syncwarp();
+        if (lane == 0) tcx::mbar_arrive(&a_ready[g]);
+      }
+      float sig = 0.f, c0 = 0.f, c1 = 0.f, c2 = 0.f;
+      bool ok = true;
+      for (int l = 0; l < 4; ++l) {
+        if (!tcx::mbar_wait(&mma_done[g], pd, abort_flag, flag, kLimit)) { ok = false; break; }
+        pd ^= 1;
+        tcx::fence_after();
+        const float* bias = b1 + 64 * l;
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          uint32_t u[32];
+          tcx::tmem_ld32(tmem + lane_base + 64 * g + 32 * half, u);
+          tcx::tmem_ld_wait(u);
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {                   // 8 columns: one K-group
+            float v[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              const int n = 32 * half + 8 * j + e;
+              v[e] = fmaxf(__uint_as_float(u[8 * j + e]) + bias[n], 0.f);
+              if (l == 1) sig = fmaf(v[e], ws[n], sig);
+              if (l == 3) {
+                c0 = fmaf(v[e], rw[n], c0);
+                c1 = fmaf(v[e], rw[64 + n], c1);
+                c2 = fmaf(v[e], rw[128 + n], c2);
+              }
+            }
+            if (l < 3)
+              tcx::st_shared_v4(abase + hc_a_off(r, 4 * half + j), tcx::pack_bf16(v[0], v[1]),
+                                tcx::pack_bf16(v[2], v[3]), tcx::pack_bf16(v[4], v[5]),
+                                tcx::pack_bf16(v[6], v[7]));
+          }
+        }
+        tcx::fence_before();
+        if (l < 3) {
+          tcx::fence_async_smem();
+          __syncwarp();
+          if (lane == 0) tcx::mbar_arrive(&a_ready[g]);
+        }
+      }
+      if (!ok) break;
+      if (valid)
+        reinterpret_cast<float4*>(out)[i] =
+            make_float4(1.0f / (1.0f + expf(-(c0 + rw[192]))), 1.0f / (1.0f + expf(-(c1 + rw[193]))),
+                        1.0f / (1.0f + expf(-(c2 + rw[194]))), fmaxf(sig + ws[64], 0.0f));
+    }
+  }
+  tcx::fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tcx::fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
+                 "r"(HC_GROUPS * 64));
+  }
+}
+
 // ------------------------------------------------------------------ KiloNeRF
 
 // The cell routing counts and scatters with one atomic per distinct cell among
@@ -978,9 +1226,14 @@ cudaError_t march_render_chunk(const MarchArgs& a, cudaStream_t st) {
   const unsigned g = (unsigned)(a.num_sms * 8);
   if (a.model == NERF_MODEL_HASHGRID) {
     if (a.ev_start) cudaEventRecord(a.ev_start, st);
-    hash_eval_kernel<<<(unsigned)(a.num_sms * HT_CTAS_PER_SM), HT_THREADS, HT_SMEM, st>>>(
-        a.o, a.d, a.r0, a.near, a.step, a.ws.live, total,
-        reinterpret_cast<const __half2*>(a.hash_table), a.hash_mlp, a.sh, a.ws.val);
+    if (a.hash_tc)
+      hash_tc_kernel<<<(unsigned)a.num_sms, HC_THREADS, HC_SMEM, st>>>(
+          a.o, a.d, a.r0, a.near, a.step, a.ws.live, total,
+          reinterpret_cast<const __half2*>(a.hash_table), a.hash_mlp, a.sh, a.ws.val, a.flag);
+    else
+      hash_eval_kernel<<<(unsigned)(a.num_sms * HT_CTAS_PER_SM), HT_THREADS, HT_SMEM, st>>>(
+          a.o, a.d, a.r0, a.near, a.step, a.ws.live, total,
+          reinterpret_cast<const __half2*>(a.hash_table), a.hash_mlp, a.sh, a.ws.val);
   } else {
     cudaMemsetAsync(a.ws.cell_hist, 0, 2 * 4096 * sizeof(int32_t), st);
     cell_hist_kernel<<<g, 256, 0, st>>>(a.o, a.d, a.r0, a.near, a.step, a.ws.live, total,
@@ -1061,6 +1314,9 @@ cudaError_t march_prepare(cudaStream_t st) {
   if (e != cudaSuccess) return e;
   cudaError_t e2 = cudaFuncSetAttribute(hash_eval_kernel,
                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)HT_SMEM);
+  if (e2 != cudaSuccess) return e2;
+  e2 = cudaFuncSetAttribute(hash_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                            (int)HC_SMEM);
   if (e2 != cudaSuccess) return e2;
   return cudaFuncSetAttribute(kilo_eval_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                               (int)KT_SMEM);

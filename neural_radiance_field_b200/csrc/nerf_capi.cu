@@ -158,6 +158,8 @@ nerf_status nerf_create(const nerf_config* cfg, nerf_ctx** out) {
     if (c.precision == NERF_BF16 && !big)
       return fail(nullptr, NERF_ERR_UNSUPPORTED, "BF16 tensor-core path needs W=256, D=8");
   } else if (c.model == NERF_MODEL_KILONERF || c.model == NERF_MODEL_HASHGRID) {
+    if (c.model == NERF_MODEL_HASHGRID && c.precision != NERF_FP32 && c.precision != NERF_BF16)
+      return fail(nullptr, NERF_ERR_INVALID_ARG, "precision must be FP32 or BF16");
     return create_march(c, out);
   } else {
     return fail(nullptr, NERF_ERR_INVALID_ARG, "unknown model %d", c.model);
@@ -363,6 +365,7 @@ nerf_status render_march(nerf_ctx* ctx, const float* o, const float* d, int64_t 
   a.acc = acc;
   a.flag = ctx->d_flag;
   a.num_sms = ctx->num_sms;
+  a.hash_tc = ctx->cfg.model == NERF_MODEL_HASHGRID && ctx->cfg.precision == NERF_BF16;
   a.ws = ctx->mws;
   for (int64_t r0 = 0; r0 < R; r0 += ctx->chunk_rays) {
     a.r0 = r0;

@@ -51,6 +51,7 @@ struct MarchArgs {
   float* acc;
   unsigned* flag;
   int num_sms;
+  int hash_tc;                // hash model: MLP on the tensor cores (bf16 operands)
   MarchWs ws;
   cudaEvent_t ev_start = nullptr;   // recorded around the scene-function kernel
   cudaEvent_t ev_stop = nullptr;    // when timing is enabled

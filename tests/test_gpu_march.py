@@ -104,11 +104,11 @@ def test_sh_against_oracle(torch):
     np.testing.assert_allclose(out.cpu().numpy(), osh.real_sh(onerf.unit(d)), atol=2e-6)
 
 
-def _render_march(torch, wl, params_kw, o, d):
+def _render_march(torch, wl, params_kw, o, d, precision=0):
     import neural_radiance_field_b200 as nb
     R = o.shape[0]
     model = {"kilonerf": nb.NERF_MODEL_KILONERF, "hashgrid": nb.NERF_MODEL_HASHGRID}[wl.model]
-    rnd = nb.Renderer(model=model, max_rays=R, max_samples=wl.n_coarse)
+    rnd = nb.Renderer(model=model, max_rays=R, max_samples=wl.n_coarse, precision=precision)
     rgb = torch.empty(R, 3, device="cuda")
     dep = torch.empty(R, device="cuda")
     acc = torch.empty(R, device="cuda")
@@ -186,3 +186,49 @@ def test_e2e_march_ragged_small(torch):
         ids = np.arange(wl.n_rays)
         ref = omarch.render_march(wl, o.cpu().numpy(), d.cpu().numpy(), dense, ev)
         _check(gpu, ref, ids, wl)
+
+
+# The hash model with precision BF16 runs its MLP on the tensor cores (bf16
+# operands and weights, fp32 accumulation; fp32 encoding and heads): the bf16
+# bar of the headline network, 2e-2 on rgb and acc and 2e-2 * far on depth.
+def _check_bf16(gpu, ref, ids, wl):
+    err_rgb = np.abs(gpu["rgb"][ids] - ref["rgb"]).max(-1)
+    err_acc = np.abs(gpu["acc"][ids] - ref["acc"])
+    err_dep = np.abs(gpu["depth"][ids] - ref["depth"])
+    print(f"[march e2e {wl.name} bf16 MLP] max err rgb {err_rgb.max():.2e} acc {err_acc.max():.2e} "
+          f"depth {err_dep.max():.2e}")
+    assert np.all(err_rgb <= 2e-2) and np.all(err_acc <= 2e-2), (err_rgb.max(), err_acc.max())
+    assert np.all(err_dep <= 2e-2 * wl.far), err_dep.max()
+    # and it is not merely within the bar by accident: the bf16 rounding shows
+    assert err_rgb.max() > 0.0
+
+
+def _hash_case(torch, wl):
+    packed, dense = S.occupancy_grid(wl.seed)
+    grid = ohash.HashGrid3D()
+    table = S.hashgrid_table(S.HashGridShape(), grid.n_entries, wl.seed, 1.0)
+    mlp = S.hash_mlp_weights(wl.seed)
+    kw = dict(occupancy=_t(torch, packed.view(np.int32)),
+              hash_table=_t(torch, table.view(np.int16)), hash_mlp=_t(torch, mlp))
+    ev = lambda idx, x, du: omarch.hash_eval(grid, table, mlp, x, du)
+    return kw, dense, ev
+
+
+def test_e2e_hashgrid_bf16_tensor_core_full_frame(torch):
+    wl = S.WORKLOADS["hashgrid"]
+    o, d = rays_for(wl)
+    kw, dense, ev = _hash_case(torch, wl)
+    gpu = _render_march(torch, wl, kw, o, d, precision=S.PREC_BF16)
+    ids = S.ray_subset(wl.n_rays, 160, 11)
+    ref = omarch.render_march(wl, o.cpu().numpy()[ids], d.cpu().numpy()[ids], dense, ev)
+    _check_bf16(gpu, ref, ids, wl)
+
+
+def test_e2e_hashgrid_bf16_ragged_small(torch):
+    """13 x 17 rays: every tile is partial, and most CTAs have no tile at all."""
+    wl = dataclasses.replace(S.WORKLOADS["hashgrid"], H=13, W=17, focal=21.25)
+    o, d = rays_for(wl)
+    kw, dense, ev = _hash_case(torch, wl)
+    gpu = _render_march(torch, wl, kw, o, d, precision=S.PREC_BF16)
+    ref = omarch.render_march(wl, o.cpu().numpy(), d.cpu().numpy(), dense, ev)
+    _check_bf16(gpu, ref, np.arange(wl.n_rays), wl)
