@@ -70,7 +70,11 @@ enum { NERF_LAST_1E10 = 0, NERF_LAST_TO_FAR = 1 };
  * L_pos = 10, L_dir = 4. precision BF16 selects the tensor-core path, built
  * for the page's (W=256, D=8, skip=4) network only (NERF_ERR_UNSUPPORTED
  * otherwise); sigma_act and white_bkgd are applied in compositing.
- * KILONERF and HASHGRID ignore D..precision. max_rays and max_samples size
+ * KILONERF ignores D..precision; HASHGRID ignores D..sigma_act and takes
+ * precision FP32 (the whole scene function in fp32 on the CUDA cores) or BF16
+ * (the encoding and the sigma / rgb heads in fp32, the four hidden layers on the
+ * tensor cores with bf16 weights and activations and fp32 accumulation;
+ * NERF_ERR_INVALID_ARG for any other value). max_rays and max_samples size
  * the context's workspace (max_samples >= n_coarse + n_fine of any render). */
 typedef struct {
   int model;
