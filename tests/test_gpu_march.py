@@ -232,3 +232,27 @@ def test_e2e_hashgrid_bf16_ragged_small(torch):
     gpu = _render_march(torch, wl, kw, o, d, precision=S.PREC_BF16)
     ref = omarch.render_march(wl, o.cpu().numpy(), d.cpu().numpy(), dense, ev)
     _check_bf16(gpu, ref, np.arange(wl.n_rays), wl)
+
+
+def test_e2e_march_no_live_points(torch):
+    """Rays that start outside the cube and point away from it: no candidate is
+    live, every scene kernel runs on zero points, and the image is empty."""
+    g = np.random.default_rng(12)
+    R = 1000
+    o = np.tile(np.float32([4.0, 4.0, 4.0]), (R, 1)) + g.uniform(0, 1, (R, 3)).astype(np.float32)
+    d = (np.abs(g.normal(size=(R, 3))) + 0.1).astype(np.float32)       # all components > 0
+    ot, dt = _t(torch, o), _t(torch, d)
+    for key, prec in (("kilonerf", 0), ("hashgrid", 0), ("hashgrid", S.PREC_BF16)):
+        wl = S.WORKLOADS[key]
+        packed, dense = S.occupancy_grid(wl.seed)
+        if key == "kilonerf":
+            cells = S.kilonerf_weights(wl.seed)
+            kw = dict(occupancy=_t(torch, packed.view(np.int32)), cell_w=_t(torch, cells))
+            ev = lambda idx, x, du: omarch.kilonerf_eval(cells, omarch.cell_id(x), x, du)
+        else:
+            kw, dense, ev = _hash_case(torch, wl)
+        gpu = _render_march(torch, wl, kw, ot, dt, precision=prec)
+        ref = omarch.render_march(wl, o, d, dense, ev)
+        assert ref["n_live"].max() == 0
+        for k in ("rgb", "acc", "depth"):
+            assert np.all(gpu[k] == 0.0), (key, prec, k)
