@@ -47,7 +47,7 @@ typedef enum {
   NERF_OK = 0,
   NERF_ERR_INVALID_ARG = 1,   /* bad pointer, size or mode; nothing was enqueued */
   NERF_ERR_CUDA = 2,          /* CUDA runtime or launch error */
-  NERF_ERR_UNSUPPORTED = 3,   /* valid request this build does not implement */
+  NERF_ERR_UNSUPPORTED = 3,   /* valid request that this library does not implement */
   NERF_ERR_OOM = 4,           /* workspace allocation failed at create time */
   NERF_ERR_TIMEOUT = 5,       /* a bounded device wait gave up */
   NERF_ERR_DEVICE_FLAG = 6    /* a kernel reported an out-of-range input */
