@@ -1,7 +1,9 @@
 // Marching scene functions: occupancy-grid empty-space skipping, the 3D
 // multiresolution hash grid with its small MLP (Instant-NGP notebook, "A shared
-// toolkit" and Experiment 1, in 3D), the KiloNeRF grid of tiny MLPs with a cell
-// router (KiloNeRF page, abstract), and compositing with early termination.
+// toolkit" and Experiment 1, in 3D; the MLP in fp32 on the CUDA cores or in bf16
+// on the tensor cores), the hash encoding's backward, the KiloNeRF grid of tiny
+// MLPs with a cell router (KiloNeRF page, abstract), and compositing with early
+// termination.
 #include <cmath>
 
 #include "tc_ptx.cuh"

@@ -1,18 +1,24 @@
-// The training step's backward (NeRF page, "7. Training loop": loss =
+// The training step (NeRF page, "7. Training loop": loss =
 // mse(rgb_coarse, target) + mse(rgb_fine, target); the coarse weights are
 // detached before resampling, "6. Hierarchical sampling", so every pass has
 // fixed sample positions). fp32 on the CUDA cores.
 //
-// Per pass (rows = rays x samples), with the forward's activations stored
-// row-major as [gamma(x) (64) | h_0 .. h_{D-1} | feature | h_dir]:
+// Per pass (rows = rays x samples), the forward writes every layer's output to
+// an activation store, row-major [gamma(x) (64) | h_0 .. h_{D-1} | feature | h_dir]:
+//   encode_store_kernel  sample points and gamma(x)
+//   row_gemm_kernel      one launch per layer, reading the previous layer's columns
+//   heads_fwd_kernel     sigma and rgb (raw outputs)
+// and the backward reads it:
 //   composite_bw_kernel  d raw (rgb, sigma) per sample and the per-ray loss term
 //   head_bw_kernel       d h_dir through the rgb head, masked by h_dir > 0
-//   in_bw_kernel         d input = d out x W (tiled), + a rank-1 term, masked by
-//                        the ReLU of the layer below
-//   wgrad_kernel         dW = sum over rows of d out^T x input, and db, as a
-//                        split-row tiled reduction added atomically into the
-//                        gradient blob (fp32 atomics: the summation order, not
-//                        the terms, varies between runs)
+//   row_gemm_kernel      d input = d out x W, + a rank-1 term, masked by the ReLU
+//                        of the layer below
+//   wgrad_gemm_kernel    dW = sum over rows of d out^T x input, and db, in row
+//                        slices added atomically into the gradient blob (fp32
+//                        atomics: the summation order, not the terms, varies
+//                        between runs); wgrad_head_kernel for the 1- and 3-output
+//                        heads
+// All GEMMs share one register-blocked core (128 x 128 tiles, 8 x 8 per thread).
 #include <algorithm>
 
 #include "nerf_internal.cuh"
