@@ -1,4 +1,4 @@
-"""CPU oracle for the forward NeRF renderer: plain, slow, fp64 numpy.
+"""CPU oracle for the NeRF renderer, its march scene functions and its training step: plain, slow, fp64 numpy.
 
 TEST INFRASTRUCTURE ONLY. Nothing in the product path imports, links or calls
 this package; only the tests, the smoke check of the build entry point and the
