@@ -53,6 +53,9 @@ def test_create_rejects_bad_configs_without_a_device(lib):
     assert lib.nerf_create(ctypes.byref(cfg), ctypes.byref(h)) == _capi.NERF_ERR_UNSUPPORTED
     cfg = _capi.nerf_config(7, 8, 256, 4, 10, 4, 0, 0, 0, 0, 16, 192)     # unknown model
     assert lib.nerf_create(ctypes.byref(cfg), ctypes.byref(h)) == _capi.NERF_ERR_INVALID_ARG
+    cfg = _capi.nerf_config(2, 8, 256, 4, 10, 4, 0, 2, 0, 0, 16, 512)     # hash grid, precision 2
+    assert lib.nerf_create(ctypes.byref(cfg), ctypes.byref(h)) == _capi.NERF_ERR_INVALID_ARG
+    assert b"precision" in lib.nerf_last_error(None)
     assert lib.nerf_create(None, ctypes.byref(h)) == _capi.NERF_ERR_INVALID_ARG
 
 
