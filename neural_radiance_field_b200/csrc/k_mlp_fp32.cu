@@ -11,9 +11,6 @@
 namespace nerfb {
 
 namespace {
-constexpr int BM = 64;
-constexpr int NT = 256;
-
 struct PackSeg {
   int64_t src_off, dst_off;
   int N, K_take, K_pad, stride, transpose;
