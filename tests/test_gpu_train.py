@@ -137,3 +137,49 @@ def test_loss_grad_rejects_bf16_and_bad_arguments(torch):
                                     fake, fake, fake, None, None)
     assert st == _capi.NERF_ERR_INVALID_ARG        # fine pass without grad_fine / weights
     rnd.close()
+
+
+def test_full_batch_is_the_mean_of_its_halves(torch):
+    """The training step at its benchmark size (4096 rays of the 800 x 800 frame,
+    coarse 64 + fine 128, the 8 x 256 network, fp32), where the oracle would take
+    hours: with perturb = 0 every ray's samples are independent of its index, so
+    the loss and the gradients of the batch are the means of those of its two
+    halves (each term is normalised by its own 3 n). This exercises the launch
+    configuration the benchmark times (row slices, atomics, full grids)."""
+    import neural_radiance_field_b200 as nb
+    wl = dataclasses.replace(S.WORKLOADS["full"], precision=S.PREC_FP32)
+    m = wl.mlp
+    B = 4096
+    o_all, d_all = rays_for(wl)
+    idx = torch.from_numpy(np.random.default_rng(17).choice(wl.n_rays, B, replace=False)).cuda()
+    o, d = o_all[idx].contiguous(), d_all[idx].contiguous()
+    cw, _ = S.nerf_weights(m, wl.seed, 0, wl.sigma_scale, S.PREC_FP32)
+    fw, _ = S.nerf_weights(m, wl.seed, 1, wl.sigma_scale, S.PREC_FP32)
+    target = torch.from_numpy(np.random.default_rng(18).uniform(0, 1, (B, 3)).astype(np.float32)).cuda()
+    rnd = nb.Renderer(D=m.D, W=m.W, skip=m.skip, precision=S.PREC_FP32, max_rays=B,
+                      max_samples=wl.n_coarse + wl.n_fine)
+    # the context keeps raw pointers: the weight tensors must outlive every call
+    cwt, fwt = torch.from_numpy(cw).cuda(), torch.from_numpy(fw).cuda()
+    p = rnd.params(coarse_w=cwt, fine_w=fwt, seed=wl.seed, perturb=0)
+
+    def step(sl):
+        loss = torch.zeros(1, device="cuda")
+        gc = torch.empty(cw.size, device="cuda")
+        gf = torch.empty(fw.size, device="cuda")
+        rnd.loss_grad(o[sl].contiguous(), d[sl].contiguous(), wl.near, wl.far, wl.n_coarse,
+                      wl.n_fine, p, target[sl].contiguous(), loss, gc, gf)
+        torch.cuda.synchronize()
+        return float(loss.item()), gc.cpu().numpy().astype(np.float64), gf.cpu().numpy().astype(np.float64)
+
+    lf, gcf, gff = step(slice(0, B))
+    l1, gc1, gf1 = step(slice(0, B // 2))
+    l2, gc2, gf2 = step(slice(B // 2, B))
+    rnd.sync_status()
+    rnd.close()
+    assert abs(lf - 0.5 * (l1 + l2)) <= 1e-5 * lf
+    for g, a, b in ((gcf, gc1, gc2), (gff, gf1, gf2)):
+        scale = np.abs(g).max()
+        assert scale > 0
+        err = np.abs(g - 0.5 * (a + b)).max()
+        print(f"[train 4096 additivity] max err / max|g| {err / scale:.2e}")
+        assert err <= REL * scale, (err, scale)
