@@ -152,7 +152,14 @@ class Renderer:
     @staticmethod
     def params(coarse_w=None, fine_w=None, occupancy=None, cell_w=None, hash_table=None,
                hash_mlp=None, march_step=0.0, ert_T=0.0, seed=0, perturb=1):
+        """A nerf_params holding the device pointers of the given tensors. The
+        library reads the tensors through these pointers on every call, so the
+        returned object keeps references to them: they stay allocated for as long
+        as it is alive, and a temporary passed here cannot be freed and its
+        memory reused while the params are in use."""
         p = nerf_params()
+        p._tensors = tuple(t for t in (coarse_w, fine_w, occupancy, cell_w, hash_table, hash_mlp)
+                           if t is not None)
         p.coarse_w = coarse_w.data_ptr() if coarse_w is not None else None
         p.fine_w = fine_w.data_ptr() if fine_w is not None else None
         p.occupancy = occupancy.data_ptr() if occupancy is not None else None

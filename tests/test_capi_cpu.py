@@ -71,3 +71,22 @@ def test_unit_entry_points_reject_null_and_bad_sizes(lib):
     assert lib.nerf_render(None, fake, fake, 4, 2.0, 6.0, 64, 0, None, fake, fake, fake, None) \
         == _capi.NERF_ERR_INVALID_ARG
     assert lib.nerf_destroy(None) == _capi.NERF_OK
+
+
+def test_params_keep_their_tensors_alive():
+    """The context reads weights through raw pointers on every call, so the
+    params object must keep the tensors it points at: a temporary passed to
+    params() is not freed (and its memory reused) while the params are alive."""
+    import gc
+    import weakref
+    import torch
+    import neural_radiance_field_b200 as nb
+    w = torch.arange(8, dtype=torch.float32)
+    ref = weakref.ref(w)
+    p = nb.Renderer.params(coarse_w=w, fine_w=torch.ones(8), seed=1)
+    del w
+    gc.collect()
+    assert ref() is not None and p.coarse_w == ref().data_ptr()
+    del p
+    gc.collect()
+    assert ref() is None
