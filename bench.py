@@ -4,6 +4,14 @@ samples per ray, 8x256 skip MLP with bf16 weights), all in libnerf's kernels.
 
 Prints one JSON line (rank 0). `--impl reference` times the CPU oracle on the
 same workload instead (a bounded sample of rays per step).
+
+Extra lines (`--workload`):
+  kilonerf, hashgrid        march renders of the two alternative scene functions
+  hashgrid_bf16             the hash grid with its MLP in bf16 on the tensor cores
+  sweep24                   24 cameras around the scene in one render call
+  compact                   a 4x128 fp32 network on the CUDA-core MLP kernel
+  train                     the training step (loss and both networks' gradients)
+  hash_backward             the hash-grid encoding's backward (scatter-add)
 """
 from __future__ import annotations
 
