@@ -265,6 +265,7 @@ def run_ours(args, rank, world, local_rank):
     peak_tf = peaks.get("bf16_tflops")
     peak_sus = peaks.get("bf16_tflops_sustained", peak_tf)
     value = job_rays_per_s(R, world, args.steps, tot_ms)
+    frame_tf = MLP_FLOP_PER_ROW * rows * args.steps / (tot_ms * 1e-3) / 1e12
     line = None
     if rank == 0:
         cpu = None
@@ -288,7 +289,11 @@ def run_ours(args, rank, world, local_rank):
                          "traffic": args.traffic_bytes or traffic_per_launch(flops_launch_avg),
                          "traffic_source": "--traffic-bytes" if args.traffic_bytes else TRAFFIC_SOURCE,
                          "avg_launch_ms": avg_launch_ms,
-                         "flop_per_launch": flops_launch_avg},
+                         "flop_per_launch": flops_launch_avg,
+                         # the same algorithmic FLOPs over the whole frame's time
+                         # (sampling, compositing and resampling included)
+                         "frame_achieved": frame_tf,
+                         "frame_frac": frame_tf / peak_tf},
             "cpu_baseline": cpu,
             "e2e": {"value": world * R / (e2e_ms * 1e-3), "unit": UNIT,
                     "h2d_bytes_per_step": R * 24, "d2h_bytes_per_step": R * 20},
