@@ -1,5 +1,6 @@
 // Small wrappers of the sm_100a tensor-core (tcgen05), mbarrier and proxy-fence
-// instructions used by single-CTA tensor-core kernels (cta_group::1).
+// instructions shared by the tensor-core kernels. The MMA and commit wrappers
+// here are the single-CTA forms (cta_group::1); the 2-SM kernel keeps its own.
 #pragma once
 #include <cstdint>
 
