@@ -90,3 +90,30 @@ def test_params_keep_their_tensors_alive():
     del p
     gc.collect()
     assert ref() is None
+
+
+def header_prototypes():
+    """name -> (return type, parameter count) of every NERF_API declaration."""
+    text = open(os.path.join(ROOT, "include", "nerf.h")).read()
+    text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+    out = {}
+    for m in re.finditer(r"NERF_API\s+([\w\s\*]+?)\b(nerf_\w+)\s*\(([^;]*?)\)\s*;", text, flags=re.S):
+        ret, name, params = m.group(1).strip(), m.group(2), m.group(3).strip()
+        n = 0 if params in ("", "void") else len(params.split(","))
+        out[name] = (ret, n)
+    return out
+
+
+def test_binding_signatures_match_the_header():
+    """Every ctypes prototype of the binding has the header's parameter count and
+    a matching return type, so no call can shift or drop an argument."""
+    import ctypes
+    protos = header_prototypes()
+    assert set(protos) == set(_capi.SIGNATURES)
+    for name, (ret, n) in protos.items():
+        res, args = _capi.SIGNATURES[name]
+        assert len(args) == n, (name, len(args), n)
+        if "char" in ret:
+            assert res is ctypes.c_char_p, name
+        else:
+            assert ret.endswith("nerf_status") and res is ctypes.c_int, (name, ret)
