@@ -201,9 +201,11 @@ NERF_API nerf_status nerf_loss_grad(nerf_ctx* ctx, const float* rays_o, const fl
                                     const float* target_rgb, float* out_loss, float* grad_coarse,
                                     float* grad_fine, void* stream);
 
-/* nerf_render with HOST ray and output buffers (pinned memory recommended):
- * copies the rays into the context's staging buffers, renders, copies the
- * results back and synchronises `stream` before returning. */
+/* nerf_render (NeRF page, Section 2.6 render_rays) with HOST ray and output
+ * buffers (pinned memory recommended): copies the rays into the context's
+ * staging buffers, renders, copies the results back and synchronises `stream`
+ * before returning. Same argument rules and errors as nerf_render; the host
+ * buffers stay the caller's. */
 NERF_API nerf_status nerf_render_host(nerf_ctx* ctx, const float* rays_o_host, const float* rays_d_host,
                              int64_t n_rays, float near, float far, int n_coarse, int n_fine,
                              const nerf_params* params, float* out_rgb_host,
@@ -234,9 +236,10 @@ NERF_API nerf_status nerf_test_stratified(const float* rays_o, const float* rays
  * cos(2^k pi x_c)], sin and cos blocks coordinate-major. x [P][3], out [P][3+6L]. */
 NERF_API nerf_status nerf_test_pe(const float* x, int64_t n, int L, float* out, void* stream);
 
-/* The context's scene network on arbitrary points x [P][3] seen from directions
- * d [P][3] (normalised inside): raw output [P][4] = (r, g, b, sigma) before
- * activations. NERF_MODEL_MLP contexts only; P <= max_rays. */
+/* The context's scene network F_theta (NeRF page, Section 2.4) on arbitrary
+ * points x [P][3] seen from directions d [P][3] (normalised inside): raw output
+ * [P][4] = (r, g, b, sigma) before activations. NERF_MODEL_MLP contexts only;
+ * P <= max_rays (NERF_ERR_INVALID_ARG otherwise). */
 NERF_API nerf_status nerf_test_mlp(nerf_ctx* ctx, const void* weights, const float* x, const float* d,
                           int64_t n, float* out_raw, void* stream);
 
@@ -261,7 +264,9 @@ NERF_API nerf_status nerf_test_sample_pdf(const float* t_coarse, const float* we
                                  int Nc, int Nf, uint64_t seed, int perturb, float* out_t_fine,
                                  int32_t* out_below, float* out_t_all, void* stream);
 
-/* Occupancy march (empty-space skipping over the 128^3 grid of nerf_params):
+/* Occupancy march: empty-space skipping over the 128^3 grid of nerf_params (the
+ * Instant-NGP notebook, "Connection to the broader theory"; the NeRF page,
+ * Section 1.4, on uniform sampling spending most of its work on empty space):
  * candidates t_k = near + k * step (fp32, k < K <= 512), points x = o + t_k d
  * (fp32, no contraction); a point is live when it lies in [-1.5, 1.5)^3 and its
  * voxel (the exact floor of (x + 1.5) * 128 / 3 per axis) is occupied.
@@ -309,7 +314,8 @@ NERF_API nerf_status nerf_hash_encode_backward(const float* x, int64_t n, const 
                                                void* stream);
 
 /* Real spherical harmonics of bands 0..3 (16 values, index l*l + l + m, no
- * Condon-Shortley phase) of the unit vectors d/|d|; d [P][3], out [P][16]. */
+ * Condon-Shortley phase) of the unit vectors d/|d|: the hash-grid MLP's view
+ * encoding (Instant-NGP notebook, "A shared toolkit"). d [P][3], out [P][16]. */
 NERF_API nerf_status nerf_test_sh(const float* d, int64_t n, float* out, void* stream);
 
 /* Failure detection of the device waits. Every wait of the library's kernels on
