@@ -315,7 +315,9 @@ NERF_API nerf_status nerf_hash_encode_backward(const float* x, int64_t n, const 
 
 /* Real spherical harmonics of bands 0..3 (16 values, index l*l + l + m, no
  * Condon-Shortley phase) of the unit vectors d/|d|: the hash-grid MLP's view
- * encoding (Instant-NGP notebook, "A shared toolkit"). d [P][3], out [P][16]. */
+ * encoding. The pages do not describe it; degree-4 real SH with the textbook
+ * normalisation is this library's reading of the hash workload's colour input.
+ * d [P][3], out [P][16]. */
 NERF_API nerf_status nerf_test_sh(const float* d, int64_t n, float* out, void* stream);
 
 /* Failure detection of the device waits. Every wait of the library's kernels on
