@@ -288,7 +288,7 @@ def render_nerf(wl, o, d, ray_ids, coarse_flat, fine_flat=None, seed=None, pertu
     ray_ids = np.asarray(ray_ids, dtype=np.int64)
     R = len(ray_ids)
     res = {k: [] for k in ("rgb", "depth", "acc", "t_c", "w_c", "t_f", "t_all", "below",
-                           "rgb_c", "acc_c", "sigma_last_raw")}
+                           "rgb_c", "acc_c", "sigma_last_raw", "raw_final", "t_final")}
     for s in range(0, R, chunk):
         sl = slice(s, min(R, s + chunk))
         oo, dd, ids = o[sl], d[sl], ray_ids[sl]
@@ -307,6 +307,8 @@ def render_nerf(wl, o, d, ray_ids, coarse_flat, fine_flat=None, seed=None, pertu
         res["acc_c"].append(acc_c)
         if wl.n_fine == 0:
             res["sigma_last_raw"].append(raw[:, -1, 3])
+            res["raw_final"].append(raw)
+            res["t_final"].append(t_c)
             res["rgb"].append(rgb_c)
             res["depth"].append(dep_c)
             res["acc"].append(acc_c)
@@ -328,6 +330,8 @@ def render_nerf(wl, o, d, ray_ids, coarse_flat, fine_flat=None, seed=None, pertu
         delta = deltas(t_all, dn, wl.last_delta, far=wl.far)
         rgb, dep, acc, _ = composite(sig, col, t_all, delta, wl.white_bkgd)
         res["sigma_last_raw"].append(raw[:, -1, 3])
+        res["raw_final"].append(raw)
+        res["t_final"].append(t_all)
         res["rgb"].append(rgb)
         res["depth"].append(dep)
         res["acc"].append(acc)
@@ -345,3 +349,34 @@ def _eval(shape, params, o, d, t, denc):
     penc = positional_encoding(x.astype(np.float64), shape.L_pos)
     de = np.broadcast_to(denc[:, None, :], penc.shape[:-1] + (denc.shape[-1],))
     return nerf_mlp(shape, params, penc, de)
+
+
+def network_pass(wl, flat, o, d, t, chunk=256):
+    """One network pass of render_rays at given sample positions: the raw
+    outputs [R,S,4] of F_theta (parameters `flat`, the workload's shape) at the
+    points fl(o + fl(t d)) seen from d / ||d|| (NeRF page, Sections 2.3-2.4).
+    o, d fp32 [R,3]; t fp32 [R,S]. fp64."""
+    shape = wl.mlp
+    params = split_params(shape, flat)
+    o = np.asarray(o, dtype=F32)
+    d = np.asarray(d, dtype=F32)
+    t = np.asarray(t, dtype=F32)
+    out = []
+    for s in range(0, len(o), chunk):
+        sl = slice(s, s + chunk)
+        denc = positional_encoding(unit(d[sl]), shape.L_dir)
+        out.append(_eval(shape, params, o[sl], d[sl], t[sl], denc))
+    return np.concatenate(out, axis=0)
+
+
+def composite_pass(wl, raw, t, d):
+    """Volume rendering of one pass of render_rays from its raw network outputs
+    (NeRF page, Section 2.5 volume_render): sigma = act(raw_sigma), c =
+    sigmoid(raw_rgb), the workload's last interval, then `composite`.
+    raw [R,S,4], t fp32 [R,S], d [R,3]. Returns rgb, depth, acc, weights (fp64)."""
+    raw = np.asarray(raw, dtype=np.float64)
+    dn = np.linalg.norm(np.asarray(d, dtype=F32).astype(np.float64), axis=-1)
+    sig = sigma_activation(raw[..., 3], wl.sigma_act)
+    col = sigmoid(raw[..., :3])
+    delta = deltas(t, dn, wl.last_delta, far=wl.far)
+    return composite(sig, col, t, delta, wl.white_bkgd)

@@ -282,6 +282,24 @@ def test_sample_pdf_delta_weight_concentrates_samples():
     assert (below == 17).sum() == inside.sum()
 
 
+def pin_sample_pdf_ties_go_right():
+    """searchsorted(cdf, u, right=True) (the page's sample_pdf): a draw that
+    lands exactly on a CDF value takes the bin that starts there. With 62 equal
+    weights the CDF after 31 of them is exactly 1/2, so u = 1/2 (m = 2^23) has
+    below = 31; the drawn position is the bin edge either way."""
+    t = np.tile(np.arange(64, dtype=np.float32) * np.float32(0.0625) + np.float32(2.0), (3, 1))
+    w = np.full((3, 62), 0.25, dtype=np.float32)
+    m = np.array([[1 << 23], [(1 << 23) - 1], [(1 << 23) + 1]])
+    tf, below = nerf.sample_pdf(nerf.midpoints(t), w, m)
+    assert below[0, 0] == 31 and below[1, 0] == 30 and below[2, 0] == 31, below.ravel()
+    bins = nerf.midpoints(t)
+    np.testing.assert_allclose(tf[0, 0], float(bins[0, 31]), atol=1e-12)
+
+
+def test_sample_pdf_ties_go_right():
+    pin_sample_pdf_ties_go_right()
+
+
 def test_sample_pdf_bin_choice_matches_exact_rational_search():
     g = np.random.default_rng(5)
     R, nb, N = 6, 63, 128
@@ -367,20 +385,26 @@ def test_hash_encoding_partition_of_unity_and_vertices():
     x = np.random.default_rng(7).uniform(-1.5, 1.5, size=(300, 3)).astype(np.float32)
     ones = np.ones((grid.n_entries, 2), dtype=np.float16)
     np.testing.assert_allclose(grid.encode(x, ones), 1.0, atol=1e-12)
-    # a point on a vertex of a direct level reads exactly that vertex's entry
-    level = 2
-    N = grid.res[level]
+    pin_hash_vertices_read_their_entry()
+
+
+def pin_hash_vertices_read_their_entry():
+    """A point on a vertex of level 0 (N = 16) reads exactly that vertex's entry
+    (the notebook's interpolation weights are 1 at the lower corner when the
+    fractional part is 0). At level 0 the point x = 3v/16 - 1.5 maps back to c =
+    v exactly: 3v/16 and x + 1.5 are exact in fp32, and (3v/16)/3 = v/16 is
+    representable, so the correctly rounded quotient is exact."""
+    grid = hashgrid.HashGrid3D()
+    level, N = 0, grid.res[0]
+    assert N == 16
     table = np.random.default_rng(8).uniform(-1, 1, size=(grid.n_entries, 2)).astype(np.float16)
-    v = np.array([3, 7, 11])
-    x01 = np.float32(v / N)
-    # only keep vertices where x01 * N rounds back exactly in fp32
-    xv = (x01 * np.float32(3.0) - np.float32(1.5)).astype(np.float32)
-    c = ((xv + np.float32(1.5)) / np.float32(3.0)) * np.float32(N)
-    if np.all(c == v):
-        enc = grid.encode(xv[None, :], table)
-        row = grid.offsets[level] + (v[0] * (N + 1) + v[1]) * (N + 1) + v[2]
-        np.testing.assert_allclose(enc[0, 2 * level:2 * level + 2], table[row].astype(np.float64),
-                                   atol=1e-12)
+    v = np.random.default_rng(16).integers(0, N, size=(200, 3))
+    xv = (np.float32(3.0) * v.astype(np.float32) / np.float32(16.0) - np.float32(1.5)).astype(np.float32)
+    c = grid.unit_coords(xv) * np.float32(N)
+    np.testing.assert_array_equal(c, v.astype(np.float32))       # the guard holds on every point
+    enc = grid.encode(xv, table)
+    row = grid.offsets[level] + (v[:, 0] * (N + 1) + v[:, 1]) * (N + 1) + v[:, 2]
+    np.testing.assert_allclose(enc[:, 0:2], table[row].astype(np.float64), atol=1e-12)
 
 
 def test_hash_encoding_2d_bilinear_is_exact_on_linear_tables():
