@@ -6,6 +6,8 @@ Prints one JSON line (rank 0). `--impl reference` times the CPU oracle on the
 same workload instead (a bounded sample of rays per step).
 
 Extra lines (`--workload`):
+  small                     200x200 coarse + fine with the 8x256 network in fp32
+  tiny                      32x32, 64 stratified samples, a 4x64 fp32 network
   kilonerf, hashgrid        march renders of the two alternative scene functions
   hashgrid_bf16             the hash grid with its MLP in bf16 on the tensor cores
   sweep24                   24 cameras around the scene in one render call
@@ -42,10 +44,22 @@ def mlp_flops_per_row(shape):
     return 2 * sum(n * k for name, n, k in shape.layer_shapes())
 
 
+def mlp_label(wl):
+    m = wl.mlp
+    prec = "bf16" if wl.precision == S.PREC_BF16 else "fp32"
+    skip = f" skip@{m.skip}" if m.skip >= 0 else ""
+    return f"{m.D}x{m.W}{skip}, {prec} weights"
+
+
+def rows_per_frame(wl):
+    """MLP rows of one frame: the coarse samples, plus the fine pass's union."""
+    return wl.n_rays * (wl.n_coarse + (wl.n_coarse + wl.n_fine if wl.n_fine else 0))
+
+
 def config_json(wl, n_gpus, extra=None):
     c = {"workload": wl.name, "H": wl.H, "W": wl.W, "rays_per_frame": wl.n_rays,
-         "n_coarse": wl.n_coarse, "n_fine": wl.n_fine, "mlp": "8x256 skip@4, bf16 weights",
-         "mlp_rows_per_frame": wl.n_rays * (2 * wl.n_coarse + wl.n_fine),
+         "n_coarse": wl.n_coarse, "n_fine": wl.n_fine, "mlp": mlp_label(wl),
+         "mlp_rows_per_frame": rows_per_frame(wl),
          "parallelism": f"rays sharded, {n_gpus} independent frame(s) per step",
          "l2": "flushed between timed steps (256 MiB write)"}
     if extra:
@@ -137,7 +151,7 @@ def cpu_baseline(wl, n_rays_sample, seed=123):
     o, d = onerf.raygen(wl.H, wl.W, wl.focal, wl.c2w())
     ids = S.ray_subset(wl.n_rays, n_rays_sample, seed)
     cw, _ = S.nerf_weights(wl.mlp, wl.seed, 0, wl.sigma_scale, wl.precision)
-    fw, _ = S.nerf_weights(wl.mlp, wl.seed, 1, wl.sigma_scale, wl.precision)
+    fw = S.nerf_weights(wl.mlp, wl.seed, 1, wl.sigma_scale, wl.precision)[0] if wl.n_fine else None
     t0 = time.perf_counter()
     onerf.render_nerf(wl, o[ids], d[ids], ids, cw, fw)
     dt = time.perf_counter() - t0
@@ -174,7 +188,50 @@ def run_reference(args, rank, world):
     print(json.dumps(line), flush=True)
 
 
-def run_ours(args, rank, world, local_rank):
+def nerf_kernel_bytes(wl):
+    """Algorithmic DRAM bytes per frame of the bandwidth-bound kernel classes of
+    a NeRF render (each byte read or written once):
+      composite  the last pass: raw (r, g, b, sigma) 16 B and, when the positions
+                 are stored, t 4 B per sample; d 12 B in, rgb + depth + acc 20 B
+                 out per ray
+      resample   the coarse raw outputs 16 B per coarse sample and d 12 B in, the
+                 sorted union 4 B per position out, per ray
+      dir_bias   d 12 B in, W/2 fp32 out per ray, once per pass"""
+    R, Nc, Nf = wl.n_rays, wl.n_coarse, wl.n_fine
+    S_ = Nc + Nf
+    passes = 2 if Nf else 1
+    out = {"composite": R * ((S_ * 20 if Nf else Nc * 16) + 32),
+           "dir_bias": passes * R * (12 + (wl.mlp.W // 2) * 4)}
+    if Nf:
+        out["resample"] = R * (Nc * 16 + 12 + S_ * 4)
+    return out
+
+
+def bandwidth_figures(kinds, bytes_per_frame, frames, hbm, peak_kind):
+    """{class: achieved GB/s of its algorithmic bytes over its measured device
+    time, and the fraction of the HBM copy peak}."""
+    out = {}
+    for k, nbytes in bytes_per_frame.items():
+        ms, n = kinds.get(k, (0.0, 0))
+        if n == 0 or ms <= 0:
+            continue
+        gbs = nbytes * frames / (ms * 1e-3) / 1e9
+        out[k] = {"bytes_per_frame": nbytes, "ms_per_frame": ms / frames, "launches": n,
+                  "achieved_gbs": gbs, "frac": gbs / hbm if hbm else None,
+                  "peak_kind": f"HBM copy, {peak_kind}"}
+    return out
+
+
+NERF_METRICS = {
+    "full": METRIC,
+    "small": "rays/sec at 200x200 coarse+fine (64+128 samples/ray), 8x256 fp32 network",
+    "tiny": "rays/sec at 32x32, 64 stratified samples/ray, 4x64 fp32 network",
+}
+
+
+def run_nerf(args, rank, world, local_rank, key=WORKLOAD):
+    """One step = ray generation + the whole render of one frame of workload `key`
+    (full: the default bench line; small and tiny: the fp32 CUDA-core path)."""
     import torch
     import neural_radiance_field_b200 as nb
     from neural_radiance_field_b200 import build as nbuild
@@ -185,15 +242,19 @@ def run_ours(args, rank, world, local_rank):
         import torch.distributed as dist
         import datetime
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
-    wl = S.WORKLOADS[WORKLOAD]
+    wl = S.WORKLOADS[key]
     if args.size:
         import dataclasses
         wl = dataclasses.replace(wl, H=args.size, W=args.size, focal=1.25 * args.size)
+    bf16 = wl.precision == S.PREC_BF16
     c2w = rank_camera(wl, rank).ravel().tolist()
     cw, _ = S.nerf_weights(wl.mlp, wl.seed, 0, wl.sigma_scale, wl.precision)
-    fw, _ = S.nerf_weights(wl.mlp, wl.seed, 1, wl.sigma_scale, wl.precision)
-    cwt = torch.from_numpy(cw).to(torch.bfloat16).cuda()
-    fwt = torch.from_numpy(fw).to(torch.bfloat16).cuda()
+    wdt = torch.bfloat16 if bf16 else torch.float32
+    cwt = torch.from_numpy(cw).to(wdt).cuda()
+    fwt = None
+    if wl.n_fine:
+        fw, _ = S.nerf_weights(wl.mlp, wl.seed, 1, wl.sigma_scale, wl.precision)
+        fwt = torch.from_numpy(fw).to(wdt).cuda()
     R = wl.n_rays
     o = torch.empty(R, 3, device="cuda")
     d = torch.empty(R, 3, device="cuda")
@@ -201,7 +262,9 @@ def run_ours(args, rank, world, local_rank):
     dep = torch.empty(R, device="cuda")
     acc = torch.empty(R, device="cuda")
     flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
-    rnd = nb.Renderer(precision=S.PREC_BF16, max_rays=R, max_samples=wl.n_coarse + wl.n_fine)
+    m = wl.mlp
+    rnd = nb.Renderer(D=m.D, W=m.W, skip=m.skip, sigma_act=wl.sigma_act, precision=wl.precision,
+                      max_rays=R, max_samples=wl.n_coarse + wl.n_fine)
     p = rnd.params(coarse_w=cwt, fine_w=fwt, seed=wl.seed, perturb=1)
     stream = torch.cuda.current_stream()
 
@@ -215,7 +278,7 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.synchronize()
     rnd.sync_status()
     rnd.timing_enable(True)
-    rnd.timing_read()
+    rnd.timing_read_kinds()
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
           for _ in range(args.steps)]
     if dist:
@@ -231,7 +294,8 @@ def run_ours(args, rank, world, local_rank):
     if dist:
         dist.barrier()
     step_ms = [a.elapsed_time(b) for a, b in ev]
-    mlp_ms, mlp_launches = rnd.timing_read()
+    kinds = rnd.timing_read_kinds()
+    mlp_ms, mlp_launches = kinds["network"]
     rnd.timing_enable(False)
     rnd.sync_status()
     tot_ms = max_over_ranks(sum(step_ms), dist, "cuda")
@@ -254,57 +318,82 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, dist, "cuda")
 
-    rows = R * (2 * wl.n_coarse + wl.n_fine)
-    flops_launch_avg = MLP_FLOP_PER_ROW * rows / 2          # coarse + fine launches per frame
+    rows = rows_per_frame(wl)
+    flop_row = mlp_flops_per_row(wl.mlp)
+    passes = 2 if wl.n_fine else 1
+    flops_launch_avg = flop_row * rows / passes            # coarse + fine launches per frame
     peaks, peak_kind = load_peaks()
     avg_launch_ms = mlp_ms / max(1, mlp_launches)
     achieved_tf = flops_launch_avg / (avg_launch_ms * 1e-3) / 1e12
-    # The network kernel holds the top SM clock through a frame (see "clocks"),
-    # so the burst cuBLAS figure is its ceiling; the power-capped sustained figure
-    # is reported beside it.
-    peak_tf = peaks.get("bf16_tflops")
-    peak_sus = peaks.get("bf16_tflops_sustained", peak_tf)
     value = job_rays_per_s(R, world, args.steps, tot_ms)
-    frame_tf = MLP_FLOP_PER_ROW * rows * args.steps / (tot_ms * 1e-3) / 1e12
+    frame_tf = flop_row * rows * args.steps / (tot_ms * 1e-3) / 1e12
+    clocks = clk.summary()
+    if bf16:
+        # The network kernel holds the top SM clock through a frame (see "clocks"),
+        # so the burst cuBLAS figure is its ceiling; the power-capped sustained
+        # figure is reported beside it.
+        peak_tf = peaks.get("bf16_tflops")
+        peak_sus = peaks.get("bf16_tflops_sustained", peak_tf)
+        roofline = {"bound": "tensor", "kernel": "scene MLP (coarse and fine launches)",
+                    "achieved": achieved_tf, "peak": peak_tf, "unit": "TFLOP/s",
+                    "frac": achieved_tf / peak_tf, "peak_kind": f"bf16 burst, {peak_kind}",
+                    "frac_of_sustained": achieved_tf / peak_sus,
+                    "traffic": args.traffic_bytes or traffic_per_launch(flops_launch_avg),
+                    "traffic_source": "--traffic-bytes" if args.traffic_bytes else TRAFFIC_SOURCE}
+    else:
+        peak_tf = fp32_peak(clocks)
+        roofline = {"bound": "alu", "kernel": f"mlp_fp32_kernel (CUDA-core MLP, W={wl.mlp.W})",
+                    "achieved": achieved_tf, "peak": peak_tf, "unit": "TFLOP/s",
+                    "frac": achieved_tf / peak_tf, "peak_kind": FP32_PEAK_NOTE, "traffic": None}
+    roofline.update({"avg_launch_ms": avg_launch_ms, "flop_per_launch": flops_launch_avg,
+                     # the same algorithmic FLOPs over the whole frame's time
+                     # (sampling, compositing and resampling included)
+                     "frame_achieved": frame_tf, "frame_frac": frame_tf / peak_tf})
     line = None
     if rank == 0:
         cpu = None
         if world == 1 and not args.no_cpu_baseline:
-            rps, dt, n = cpu_baseline(wl, args.cpu_rays)
+            n_cpu = min(wl.n_rays, args.cpu_rays)
+            rps, dt, n = cpu_baseline(wl, n_cpu)
             cpu = {"value": rps, "unit": UNIT, "cores": n_cores(), "kind": "oracle",
-                   "sample": f"{n} seeded rays of the 800x800 frame, full coarse+fine oracle render "
-                             f"({dt:.1f} s)"}
+                   "sample": f"{n} seeded rays of the {wl.H}x{wl.W} frame, the whole oracle "
+                             f"render of each ({dt:.1f} s)"}
         line = {
-            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": tot_ms / args.steps, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "metric": NERF_METRICS[key], "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": tot_ms / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16" if bf16 else "f32",
             "data": "synthetic (seeded camera, Xavier-init weights)",
             "config": config_json(wl, world),
             "sample_points_per_s": value * (wl.n_coarse + wl.n_fine),
             "mlp_rows_per_s": world * rows * args.steps / (tot_ms * 1e-3),
-            "roofline": {"bound": "tensor", "kernel": "scene MLP (coarse and fine launches)",
-                         "achieved": achieved_tf, "peak": peak_tf, "unit": "TFLOP/s",
-                         "frac": achieved_tf / peak_tf, "peak_kind": f"bf16 burst, {peak_kind}",
-                         "frac_of_sustained": achieved_tf / peak_sus,
-                         "traffic": args.traffic_bytes or traffic_per_launch(flops_launch_avg),
-                         "traffic_source": "--traffic-bytes" if args.traffic_bytes else TRAFFIC_SOURCE,
-                         "avg_launch_ms": avg_launch_ms,
-                         "flop_per_launch": flops_launch_avg,
-                         # the same algorithmic FLOPs over the whole frame's time
-                         # (sampling, compositing and resampling included)
-                         "frame_achieved": frame_tf,
-                         "frame_frac": frame_tf / peak_tf},
+            "roofline": roofline,
+            "bandwidth_kernels": bandwidth_figures(kinds, nerf_kernel_bytes(wl), args.steps,
+                                                   peaks.get("hbm_gbs"), peak_kind),
             "cpu_baseline": cpu,
             "e2e": {"value": world * R / (e2e_ms * 1e-3), "unit": UNIT,
                     "h2d_bytes_per_step": R * 24, "d2h_bytes_per_step": R * 20},
-            "gpu_launches": args.steps * 9,
-            "clocks": clk.summary(),
+            "gpu_launches": args.steps * nerf_launches_per_step(wl),
+            "clocks": clocks,
         }
         print(json.dumps(line), flush=True)
     rnd.close()
     if dist:
         dist.barrier()
         dist.destroy_process_group()
+
+
+def nerf_launches_per_step(wl):
+    """The library's kernels per NeRF step: ray generation; per pass the weight
+    packing, the direction bias and the network; the resampling between passes;
+    the final compositing."""
+    passes = 2 if wl.n_fine else 1
+    return 1 + 3 * passes + (1 if wl.n_fine else 0) + 1
+
+
+def fp32_peak(clocks):
+    sm_mhz = clocks["sm_mhz"] or 1965.0
+    return 148 * 128 * 2 * sm_mhz * 1e6 / 1e12
 
 
 FP32_PEAK_NOTE = "fp32 FMA: 148 SMs x 128 lanes x 2 FLOP x SM clock"
@@ -613,6 +702,50 @@ def run_hash_backward(args, rank, world, local_rank):
     print(json.dumps(line), flush=True)
 
 
+def march_kernel_bytes(wl, R, live, tc):
+    """Algorithmic bytes per frame of the march kernel classes (each byte read or
+    written once; `live` occupied candidates):
+      march_mask       o, d 24 B in, 16 mask words and a count 68 B out, per ray
+                       (plus one occupancy bit per candidate from the 256 KB grid)
+      march_compact    count in and offset out 8 B, masks 64 B in, per ray; one
+                       4 B live entry out per live candidate
+      router           (KiloNeRF) live entry in, cell id out, cell id in, order
+                       out: 16 B per live candidate
+      network          (hash grid) 16 levels x 8 corners x 4 B of table gathers,
+                       the live entry 4 B and the (r, g, b, sigma) 16 B out, per
+                       live candidate
+      march_composite  offset 4 B, d 12 B in, rgb + depth + acc 20 B out per ray;
+                       live entry and (r, g, b, sigma) 20 B per live candidate"""
+    out = {"march_mask": R * 92, "march_compact": R * 72 + live * 4,
+           "march_composite": R * 36 + live * 20}
+    if wl.model == "kilonerf":
+        out["router"] = live * 16
+    else:
+        out["network"] = live * (512 + 20)
+    return out
+
+
+def march_cpu_baseline(wl, scene, n_rays_sample, seed=123):
+    """The march oracle as it stands on a bounded seeded sample of the frame's rays."""
+    from oracle import march as omarch
+    from oracle import nerf as onerf
+    o, d = onerf.raygen(wl.H, wl.W, wl.focal, wl.c2w())
+    ids = S.ray_subset(wl.n_rays, n_rays_sample, seed)
+    _, dense = S.occupancy_grid(wl.seed)
+    if wl.model == "kilonerf":
+        cells = scene
+        ev = lambda idx, x, du: omarch.kilonerf_eval(cells, omarch.cell_id(x), x, du)
+    else:
+        from oracle import hashgrid as ohash
+        grid = ohash.HashGrid3D()
+        table, mlp = scene
+        ev = lambda idx, x, du: omarch.hash_eval(grid, table, mlp, x, du)
+    t0 = time.perf_counter()
+    omarch.render_march(wl, o[ids], d[ids], dense, ev)
+    dt = time.perf_counter() - t0
+    return len(ids) / dt, dt, len(ids)
+
+
 def run_march(args, rank, world, local_rank):
     """One step = ray generation + a full-frame march render of the KiloNeRF or
     hash-grid workload (occupancy skipping, scene function, compositing)."""
@@ -632,18 +765,22 @@ def run_march(args, rank, world, local_rank):
     occ = torch.from_numpy(packed.view(np.int32)).cuda()
     if wl.model == "kilonerf":
         model = nb.NERF_MODEL_KILONERF
-        cell_w = torch.from_numpy(S.kilonerf_weights(wl.seed)).cuda()
+        cells_np = S.kilonerf_weights(wl.seed)
+        cell_w = torch.from_numpy(cells_np).cuda()
         kw = dict(occupancy=occ, cell_w=cell_w)
+        scene = cells_np
         flop_per_point, kname = 2 * 3249, "kilo_eval_kernel (per-cell tiny MLPs)"
     else:
         model = nb.NERF_MODEL_HASHGRID
-        table = torch.from_numpy(
-            S.hashgrid_table(S.HashGridShape(), S.HASH_ENTRIES, wl.seed, 1e-4).view(np.int16)).cuda()
-        mlp = torch.from_numpy(S.hash_mlp_weights(wl.seed)).cuda()
+        table_np = S.hashgrid_table(S.HashGridShape(), S.HASH_ENTRIES, wl.seed, 1e-4)
+        table = torch.from_numpy(table_np.view(np.int16)).cuda()
+        mlp_np = S.hash_mlp_weights(wl.seed)
+        mlp = torch.from_numpy(mlp_np).cuda()
         kw = dict(occupancy=occ, hash_table=table, hash_mlp=mlp)
-        flop_per_point, kname = 2 * 15616, "hash_eval_kernel (encoding + MLPs)"
-        if tc:
-            kname = "hash_tc_kernel (fp32 encoding, MLP on the tensor cores in bf16)"
+        scene = (table_np, mlp_np)
+        flop_per_point = 2 * 15616
+        kname = ("hash_tc_kernel (fp32 encoding, MLP on the tensor cores in bf16)" if tc
+                 else "hash_eval_kernel (encoding + MLPs)")
     o = torch.empty(R, 3, device="cuda")
     d = torch.empty(R, 3, device="cuda")
     rgb = torch.empty(R, 3, device="cuda")
@@ -669,7 +806,7 @@ def run_march(args, rank, world, local_rank):
     torch.cuda.synchronize()
     rnd.sync_status()
     rnd.timing_enable(True)
-    rnd.timing_read()
+    rnd.timing_read_kinds()
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
           for _ in range(args.steps)]
     with ClockSampler(local_rank) as clk:
@@ -680,36 +817,75 @@ def run_march(args, rank, world, local_rank):
             ev[k][1].record(stream)
         torch.cuda.synchronize()
     tot_ms = sum(a.elapsed_time(b) for a, b in ev)
-    k_ms, k_launches = rnd.timing_read()
+    kinds = rnd.timing_read_kinds()
+    k_ms = kinds["network"][0]
     rnd.timing_enable(False)
     rnd.sync_status()
+
+    # end to end through the host-buffer entry point (pinned host memory)
+    oh, dh = o.cpu().pin_memory(), d.cpu().pin_memory()
+    rgbh = torch.empty(R, 3).pin_memory()
+    deph = torch.empty(R).pin_memory()
+    acch = torch.empty(R).pin_memory()
+    e2e_steps = max(1, min(args.steps, 5))
+    rnd.render_host(oh, dh, wl.near, wl.far, wl.n_coarse, 0, p, rgbh, deph, acch)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        rnd.render_host(oh, dh, wl.near, wl.far, wl.n_coarse, 0, p, rgbh, deph, acch)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / e2e_steps
+
     clocks = clk.summary()
-    sm_mhz = clocks["sm_mhz"] or 1965.0
-    peak = 148 * 128 * 2 * sm_mhz * 1e6 / 1e12
+    peaks, pk = load_peaks()
+    hbm = peaks.get("hbm_gbs")
     per_frame_k_ms = k_ms / args.steps
     achieved = live * flop_per_point / (per_frame_k_ms * 1e-3) / 1e12
-    roofline = {"bound": "alu", "kernel": kname, "achieved": achieved, "peak": peak,
-                "unit": "TFLOP/s", "frac": achieved / peak, "peak_kind": FP32_PEAK_NOTE,
-                "traffic": None, "kernel_ms_per_frame": per_frame_k_ms,
-                "flop_per_point": flop_per_point}
-    if tc:
-        # the MLP's FLOPs run on the tensor cores; the kernel is bound by the fp32
-        # encoding (128 table gathers per point), so this fraction is small
-        peaks, pk = load_peaks()
-        bf = peaks.get("bf16_tflops")
-        roofline.update({"bound": "tensor", "peak": bf, "frac": achieved / bf if bf else None,
-                         "peak_kind": f"bf16 burst, {pk}"})
+    nbytes = march_kernel_bytes(wl, R, live, tc)
+    if wl.model == "kilonerf":
+        peak = fp32_peak(clocks)
+        roofline = {"bound": "alu", "kernel": kname, "achieved": achieved, "peak": peak,
+                    "unit": "TFLOP/s", "frac": achieved / peak, "peak_kind": FP32_PEAK_NOTE,
+                    "traffic": None, "kernel_ms_per_frame": per_frame_k_ms,
+                    "flop_per_point": flop_per_point}
+    else:
+        # the hash-grid scene kernel is bound by its 128 table gathers per point
+        # (the 23.3 MiB table stays in L2): its roofline is the algorithmic gather
+        # bytes against the HBM copy rate; the MLP's FLOP rate is reported beside it
+        gbs = nbytes["network"] / (per_frame_k_ms * 1e-3) / 1e9
+        roofline = {"bound": "hbm", "kernel": kname, "achieved": gbs, "peak": hbm,
+                    "unit": "GB/s", "frac": gbs / hbm if hbm else None,
+                    "peak_kind": f"HBM copy, {pk} (the table is L2-resident)",
+                    "traffic": None, "kernel_ms_per_frame": per_frame_k_ms,
+                    "bytes_per_point": 512 + 20, "mlp_tflops": achieved}
+        if tc:
+            bf = peaks.get("bf16_tflops")
+            roofline["mlp_frac_of_bf16_burst"] = achieved / bf if bf else None
+        else:
+            roofline["mlp_frac_of_fp32_fma"] = achieved / fp32_peak(clocks)
+    cpu = None
+    if not args.no_cpu_baseline:
+        rps, dt, n = march_cpu_baseline(wl, scene, args.march_cpu_rays)
+        cpu = {"value": rps, "unit": UNIT, "cores": n_cores(), "kind": "oracle",
+               "sample": f"{n} seeded rays of the {wl.H}x{wl.W} frame, the whole oracle march "
+                         f"of each ({dt:.1f} s)"}
     line = {"metric": f"rays/sec, {wl.name} march render" + (", MLP in bf16 on the tensor cores" if tc else ""),
             "value": R * args.steps / (tot_ms * 1e-3),
             "unit": UNIT, "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": tot_ms / args.steps, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-            "config": {"workload": wl.name, "H": wl.H, "W": wl.W, "candidates": wl.n_coarse,
-                       "march_step": wl.march_step, "ert_T": wl.ert_T,
+            "vs_baseline": None, "dtype": "bf16" if tc else "f32", "data": "synthetic",
+            "config": {"workload": wl.name + ("_bf16" if tc else ""), "H": wl.H, "W": wl.W,
+                       "candidates": wl.n_coarse, "march_step": wl.march_step, "ert_T": wl.ert_T,
                        "occupied_candidates_per_frame": live,
                        "l2": "flushed between timed steps (256 MiB write)"},
             "sample_points_per_s": live * args.steps / (tot_ms * 1e-3),
             "roofline": roofline,
+            "bandwidth_kernels": bandwidth_figures(kinds, nbytes, args.steps, hbm, pk),
+            "cpu_baseline": cpu,
+            "e2e": {"value": R / (e2e_ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": R * 24,
+                    "d2h_bytes_per_step": R * 20},
             "gpu_launches": args.steps * march_launches_per_step(wl.model, R), "clocks": clocks}
     print(json.dumps(line), flush=True)
     rnd.close()
@@ -725,9 +901,9 @@ def march_launches_per_step(model, R):
     return 1 + chunks * per_chunk
 
 
-# DRAM bytes (read + write) per MLP row of the scene-MLP kernel, from the ncu
-# capture summarised in profiles/mlp_tc_kernel_256x256.md: 236.75 MB for the fine
-# launch of a 256x256 frame (12,582,912 rows). The traffic is the raw output
+# DRAM bytes (read + write) per MLP row of the scene-MLP kernel, from an ncu
+# capture (dram__bytes_read.sum + dram__bytes_write.sum) of the fine launch of a
+# 256x256 frame: 236.75 MB for 12,582,912 rows. The traffic is the raw output
 # and the sample positions, so it grows in proportion to the rows; it is scaled
 # to the launch size here. Re-measure whenever the kernel changes.
 TRAFFIC_B_PER_ROW = 236.75e6 / 12582912
@@ -747,10 +923,12 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-rays", type=int, default=1024)
     ap.add_argument("--ref-rays", type=int, default=128)
+    ap.add_argument("--march-cpu-rays", type=int, default=256,
+                    help="rays of the oracle's march sample (march workloads)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--workload", default=WORKLOAD,
-                    choices=[WORKLOAD, "kilonerf", "hashgrid", "hashgrid_bf16", "sweep24", "compact", "train",
-                             "hash_backward"],
+                    choices=[WORKLOAD, "small", "tiny", "kilonerf", "hashgrid", "hashgrid_bf16",
+                             "sweep24", "compact", "train", "hash_backward"],
                     help="the benchmark workload (default) or a march workload (extra lines)")
     ap.add_argument("--traffic-bytes", type=float, default=0.0,
                     help="DRAM bytes per network launch from an ncu capture of this kernel")
@@ -772,10 +950,10 @@ def main():
         run_train(args, rank, world, local_rank)
     elif args.workload == "hash_backward":
         run_hash_backward(args, rank, world, local_rank)
-    elif args.workload != WORKLOAD:
+    elif args.workload in ("kilonerf", "hashgrid", "hashgrid_bf16"):
         run_march(args, rank, world, local_rank)
     else:
-        run_ours(args, rank, world, local_rank)
+        run_nerf(args, rank, world, local_rank, args.workload)
 
 
 if __name__ == "__main__":

@@ -99,7 +99,8 @@ typedef struct {
  *  cell_w            KILONERF: fp32 [4096][3317] per-cell parameters, cell id
  *                    (cx*16+cy)*16+cz; per cell: W1[32][63] b1[32] W2[32][32]
  *                    b2[32] w_sigma[32] b_sigma[1] Wc[3][59] bc[3].
- *  hash_table        HASHGRID: fp16 [6101902][2], all 16 levels concatenated.
+ *  hash_table        HASHGRID: fp16 [6101902][2], all 16 levels concatenated;
+ *                    16-byte aligned (rows are read in aligned groups of four).
  *  hash_mlp          HASHGRID: fp32 blob d0[64][32] b, d1[64][64] b, sigma[1][64] b,
  *                    c0[64][80] b, c1[64][64] b, rgb[3][64] b.
  *  march_step        march models: t_k = near + k * march_step, k < n_coarse.
@@ -177,6 +178,41 @@ NERF_API nerf_status nerf_render(nerf_ctx* ctx, const float* rays_o, const float
                         const nerf_params* params, float* out_rgb, float* out_depth,
                         float* out_acc, void* stream);
 
+/* Intermediates of one NERF_MODEL_MLP render, for checking every stage of the
+ * path on its own inputs. All pointers are device memory owned by the caller;
+ * any may be NULL (not written). R = n_rays, Nc = n_coarse, Nf = n_fine.
+ *  raw_coarse [R][Nc][4]      the coarse network's raw (r, g, b, sigma)
+ *  w_coarse   [R][Nc]         the coarse compositing weights w_i = T_i alpha_i
+ *                             (with n_fine > 0, those the fine positions were
+ *                             drawn from)
+ *  t_fine     [R][Nf]         the inverse-CDF draws, in draw order
+ *  below      [R][Nf] int32   the bin of each draw (searchsorted - 1, clamped)
+ *  t_all      [R][Nc+Nf]      the sorted union of coarse and fine positions
+ *  raw_fine   [R][Nc+Nf][4]   the fine network's raw outputs at t_all
+ * The fine-pass fields are ignored when n_fine == 0. */
+typedef struct {
+  float* raw_coarse;
+  float* w_coarse;
+  float* t_fine;
+  int32_t* below;
+  float* t_all;
+  float* raw_fine;
+} nerf_trace;
+
+/* nerf_render (NeRF page, Section 2.6 render_rays) of a NERF_MODEL_MLP context
+ * that also copies the render's own intermediates into `trace` (coarse network
+ * output and weights, Section 2.5; the sample_pdf draws and bins, Section 2.6;
+ * the sorted union and the fine network output). The kernels, launch shapes
+ * and outputs are those of nerf_render; only device-to-device copies of the
+ * workspace and the resampler's optional stores are added. Same argument
+ * rules and errors as nerf_render; NERF_ERR_UNSUPPORTED for the march models;
+ * NERF_ERR_INVALID_ARG if trace is NULL. Enqueued on `stream`. */
+NERF_API nerf_status nerf_render_trace(nerf_ctx* ctx, const float* rays_o, const float* rays_d,
+                                       int64_t n_rays, float near, float far, int n_coarse,
+                                       int n_fine, const nerf_params* params, float* out_rgb,
+                                       float* out_depth, float* out_acc, const nerf_trace* trace,
+                                       void* stream);
+
 /* Loss and parameter gradients of one training step (NeRF page, "7. Training
  * loop"): the rays are rendered as nerf_render does (coarse pass; with n_fine >
  * 0 the fine pass on the sorted union of positions drawn from the coarse
@@ -211,14 +247,38 @@ NERF_API nerf_status nerf_render_host(nerf_ctx* ctx, const float* rays_o_host, c
                              const nerf_params* params, float* out_rgb_host,
                              float* out_depth_host, float* out_acc_host, void* stream);
 
-/* Device timing of the scene-network kernels, for benchmarks. While enabled,
- * every network launch of nerf_render / nerf_test_mlp is bracketed by CUDA
- * events recorded on the caller's stream (at most 4096 launches between reads;
- * further launches are not timed). nerf_timing_read waits for the recorded
- * events, returns the summed kernel time in milliseconds and the number of
- * timed launches since the previous read, and starts a new count. */
+/* Device timing of the library's kernels, for benchmarks. While enabled, the
+ * launches of every kernel class below that nerf_render / nerf_test_mlp issue
+ * are bracketed by CUDA events recorded on the caller's stream (at most 4096
+ * event pairs between reads; further launches are not timed). The classes:
+ *   NETWORK          the scene-network kernel (NeRF MLP; march models: the
+ *                    hash-grid or KiloNeRF scene function)
+ *   COMPOSITE        compositing of the last NeRF pass (Section 2.5)
+ *   RESAMPLE         coarse compositing + inverse-CDF draws + sorted merge
+ *                    (Section 2.6)
+ *   DIR_BIAS         the per-ray direction-encoding bias of the direction layer
+ *   MARCH_MASK       the occupancy test of every march candidate
+ *   MARCH_COMPACT    the scan and compaction of the live candidates
+ *   ROUTER           KiloNeRF cell routing (histogram, scan, scatter, work items)
+ *   MARCH_COMPOSITE  march compositing with early termination
+ * nerf_timing_read waits for the recorded events and returns the summed time
+ * (milliseconds) and launch count of the NETWORK class; nerf_timing_read_kinds
+ * returns every class (arrays of NERF_TIMED_KINDS, indexed by the enum). Both
+ * start a new count. */
+enum {
+  NERF_TIMED_NETWORK = 0,
+  NERF_TIMED_COMPOSITE = 1,
+  NERF_TIMED_RESAMPLE = 2,
+  NERF_TIMED_DIR_BIAS = 3,
+  NERF_TIMED_MARCH_MASK = 4,
+  NERF_TIMED_MARCH_COMPACT = 5,
+  NERF_TIMED_ROUTER = 6,
+  NERF_TIMED_MARCH_COMPOSITE = 7,
+  NERF_TIMED_KINDS = 8
+};
 NERF_API nerf_status nerf_timing_enable(nerf_ctx* ctx, int enable);
 NERF_API nerf_status nerf_timing_read(nerf_ctx* ctx, double* ms, int64_t* launches);
+NERF_API nerf_status nerf_timing_read_kinds(nerf_ctx* ctx, double* ms, int64_t* launches);
 
 /* ---------------------------------------------------------------------------
  * Unit entry points: one step of the path each, same conventions as above.
@@ -291,7 +351,8 @@ NERF_API nerf_status nerf_test_route_cells(const float* x, int64_t n, int32_t* o
  * index (ix*(N+1)+iy)*(N+1)+iz while (N+1)^3 <= T, else (ix XOR iy*2654435761
  * XOR iz*805459861) mod T; trilinear weights of c = fl(fl((x + 1.5)/3) * N).
  * x [P][3]; out_feat [P][32] (level-major); out_rows [P][16][8] int32 (may be
- * NULL): global table row of every corner (dx, dy, dz loop order). */
+ * NULL): global table row of every corner (dx, dy, dz loop order). hash_table
+ * must be 16-byte aligned (NERF_ERR_INVALID_ARG otherwise). */
 NERF_API nerf_status nerf_test_hash_encode(const float* x, int64_t n, const uint16_t* hash_table,
                                            float* out_feat, int32_t* out_rows, void* stream);
 

@@ -179,6 +179,20 @@ class Renderer:
             int(n_coarse), int(n_fine), ctypes.byref(params), _ptr(out_rgb), _ptr(out_depth),
             _ptr(out_acc), _stream(stream)), self.ctx)
 
+    def render_trace(self, rays_o, rays_d, near, far, n_coarse, n_fine, params, out_rgb,
+                     out_depth, out_acc, raw_coarse=None, w_coarse=None, t_fine=None, below=None,
+                     t_all=None, raw_fine=None, stream=None):
+        """nerf_render that also copies the render's intermediates into the given
+        CUDA tensors (any may be None); see nerf_render_trace."""
+        tr = _capi.nerf_trace(*[t.data_ptr() if t is not None else None for t in
+                                (raw_coarse, w_coarse, t_fine, below, t_all, raw_fine)])
+        for t in (raw_coarse, w_coarse, t_fine, below, t_all, raw_fine):
+            _ptr(t)                                       # device and contiguous
+        _capi.check(_capi.lib().nerf_render_trace(
+            self.ctx, _ptr(rays_o), _ptr(rays_d), rays_o.shape[0], float(near), float(far),
+            int(n_coarse), int(n_fine), ctypes.byref(params), _ptr(out_rgb), _ptr(out_depth),
+            _ptr(out_acc), ctypes.byref(tr), _stream(stream)), self.ctx)
+
     def loss_grad(self, rays_o, rays_d, near, far, n_coarse, n_fine, params, target_rgb,
                   out_loss, grad_coarse, grad_fine=None, stream=None):
         """Training-step loss and gradients (fp32 contexts); see nerf_loss_grad."""
@@ -209,6 +223,15 @@ class Renderer:
         _capi.check(_capi.lib().nerf_timing_read(self.ctx, ctypes.byref(ms), ctypes.byref(n)),
                     self.ctx)
         return ms.value, n.value
+
+    def timing_read_kinds(self):
+        """{kernel class: (summed ms, launches)} since the last read, for every
+        class of nerf_timing_read_kinds."""
+        n = len(_capi.TIMED_KINDS)
+        ms = (ctypes.c_double * n)()
+        cnt = (ctypes.c_int64 * n)()
+        _capi.check(_capi.lib().nerf_timing_read_kinds(self.ctx, ms, cnt), self.ctx)
+        return {k: (ms[i], cnt[i]) for i, k in enumerate(_capi.TIMED_KINDS)}
 
     def sync_status(self, stream=None):
         _capi.check(_capi.lib().nerf_sync_status(self.ctx, _stream(stream)), self.ctx)

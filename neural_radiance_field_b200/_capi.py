@@ -23,6 +23,8 @@ NERF_MODEL_MLP, NERF_MODEL_KILONERF, NERF_MODEL_HASHGRID = 0, 1, 2
 NERF_SIGMA_RELU, NERF_SIGMA_SOFTPLUS = 0, 1
 NERF_FP32, NERF_BF16 = 0, 1
 NERF_LAST_1E10, NERF_LAST_TO_FAR = 0, 1
+TIMED_KINDS = ("network", "composite", "resample", "dir_bias", "march_mask", "march_compact",
+               "router", "march_composite")           # NERF_TIMED_* order
 
 _STATUS = {0: "NERF_OK", 1: "NERF_ERR_INVALID_ARG", 2: "NERF_ERR_CUDA", 3: "NERF_ERR_UNSUPPORTED",
            4: "NERF_ERR_OOM", 5: "NERF_ERR_TIMEOUT", 6: "NERF_ERR_DEVICE_FLAG"}
@@ -44,6 +46,12 @@ class nerf_params(ctypes.Structure):
                 ("seed", ctypes.c_uint64), ("perturb", ctypes.c_int)]
 
 
+class nerf_trace(ctypes.Structure):
+    _fields_ = [("raw_coarse", ctypes.c_void_p), ("w_coarse", ctypes.c_void_p),
+                ("t_fine", ctypes.c_void_p), ("below", ctypes.c_void_p),
+                ("t_all", ctypes.c_void_p), ("raw_fine", ctypes.c_void_p)]
+
+
 _P = ctypes.c_void_p
 _I64 = ctypes.c_int64
 _F = ctypes.c_float
@@ -60,12 +68,15 @@ SIGNATURES = {
     "nerf_raygen_batch": (_I, [_I, _I, _F, _I, _P, _P, _P, _P]),
     "nerf_render": (_I, [_P, _P, _P, _I64, _F, _F, _I, _I, ctypes.POINTER(nerf_params),
                          _P, _P, _P, _P]),
+    "nerf_render_trace": (_I, [_P, _P, _P, _I64, _F, _F, _I, _I, ctypes.POINTER(nerf_params),
+                               _P, _P, _P, ctypes.POINTER(nerf_trace), _P]),
     "nerf_loss_grad": (_I, [_P, _P, _P, _I64, _F, _F, _I, _I, ctypes.POINTER(nerf_params),
                             _P, _P, _P, _P, _P]),
     "nerf_render_host": (_I, [_P, _P, _P, _I64, _F, _F, _I, _I, ctypes.POINTER(nerf_params),
                               _P, _P, _P, _P]),
     "nerf_timing_enable": (_I, [_P, _I]),
     "nerf_timing_read": (_I, [_P, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(_I64)]),
+    "nerf_timing_read_kinds": (_I, [_P, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(_I64)]),
     "nerf_test_stratified": (_I, [_P, _P, _I64, _F, _F, _I, _U64, _I, _P, _P, _P]),
     "nerf_test_pe": (_I, [_P, _I64, _I, _P, _P]),
     "nerf_test_mlp": (_I, [_P, _P, _P, _P, _I64, _P, _P]),

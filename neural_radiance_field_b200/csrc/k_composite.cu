@@ -216,7 +216,7 @@ __device__ void resample_ray(ResampleSmem& sm, int64_t ray, int Nf, uint64_t key
 __global__ void coarse_resample_kernel(const float* __restrict__ raw_c, SampleSpec ss,
                                        const float* __restrict__ d, int64_t R, CompositeSpec cs,
                                        int Nf, uint64_t key, int perturb,
-                                       float* __restrict__ t_all) {
+                                       float* __restrict__ t_all, ResampleTrace tr) {
   __shared__ ResampleSmem smem[WARPS];
   const int wid = threadIdx.x / 32, lane = threadIdx.x & 31;
   int64_t ray = (int64_t)blockIdx.x * WARPS + wid;
@@ -226,7 +226,9 @@ __global__ void coarse_resample_kernel(const float* __restrict__ raw_c, SampleSp
   composite_ray<2>(raw_c, ss, ray, ray_norm(d, ray), cs, sm.w, res);
   for (int i = lane; i < 64; i += 32) sm.tc[i] = sample_t(ss, ray, i);
   __syncwarp();
-  resample_ray(sm, ray, Nf, key, perturb, nullptr, nullptr, t_all);
+  if (tr.w)
+    for (int i = lane; i < 64; i += 32) tr.w[ray * 64 + i] = sm.w[i];
+  resample_ray(sm, ray, Nf, key, perturb, tr.t_f, tr.below, t_all);
 }
 
 __global__ void sample_pdf_kernel(const float* __restrict__ t_c, const float* __restrict__ w,
@@ -265,11 +267,12 @@ cudaError_t launch_composite(const float* raw, const SampleSpec& ss, const float
 
 cudaError_t launch_coarse_resample(const float* raw_c, const SampleSpec& coarse, const float* d,
                                    int64_t R, const CompositeSpec& cs, int Nf, uint64_t key,
-                                   int perturb, float* t_all, cudaStream_t st) {
+                                   int perturb, float* t_all, cudaStream_t st,
+                                   const ResampleTrace& tr) {
   if (coarse.S != 64 || Nf < 1 || Nf > 128) return cudaErrorInvalidValue;
   unsigned blocks = (unsigned)((R + WARPS - 1) / WARPS);
   coarse_resample_kernel<<<blocks, WARPS * 32, 0, st>>>(raw_c, coarse, d, R, cs, Nf, key, perturb,
-                                                        t_all);
+                                                        t_all, tr);
   return cudaGetLastError();
 }
 

@@ -12,33 +12,7 @@
 namespace nerfb {
 
 // ------------------------------------------------------------------ occupancy
-
-// Voxel of one coordinate by exact comparison with the boundaries b_v = -1.5 +
-// v * 3/128 (exact in fp32): returns -1 outside [-1.5, 1.5).
-__device__ __forceinline__ int voxel_axis(float x) {
-  if (!(x >= -1.5f) || !(x < 1.5f)) return -1;
-  int v = (int)floorf(fmul(fadd(x, 1.5f), 42.666666666666664f));
-  v = v < 0 ? 0 : (v > 127 ? 127 : v);
-  if (x < fsub(fmul((float)v, 0.0234375f), 1.5f)) --v;
-  else if (v < 127 && x >= fsub(fmul((float)(v + 1), 0.0234375f), 1.5f)) ++v;
-  return v;
-}
-
-__device__ __forceinline__ bool occupied_at(const uint32_t* __restrict__ occ, float x0, float x1,
-                                            float x2, int* vox) {
-  const int a = voxel_axis(x0), b = voxel_axis(x1), c = voxel_axis(x2);
-  if (a < 0 || b < 0 || c < 0) return false;
-  const int idx = (a * 128 + b) * 128 + c;
-  if (vox) *vox = idx;
-  return (__ldg(occ + (idx >> 5)) >> (idx & 31)) & 1u;
-}
-
-__device__ __forceinline__ void march_point(const float* o, const float* d, int64_t r, float near,
-                                            float step, int k, float* x, float* t) {
-  *t = fadd(near, fmul((float)k, step));
-#pragma unroll
-  for (int c = 0; c < 3; ++c) x[c] = fadd(o[r * 3 + c], fmul(*t, d[r * 3 + c]));
-}
+// (voxel_axis, occupied_at and march_point: nerf_march.cuh)
 
 // Warp per ray: live bitmask (K <= 512 -> 16 words) and live count.
 __global__ void march_mask_kernel(const float* __restrict__ o, const float* __restrict__ d,
@@ -139,6 +113,7 @@ cudaError_t exclusive_scan(const int32_t* in, int64_t n, int32_t* out, int32_t* 
 __constant__ int c_hres[16];
 __constant__ int c_hoff[16];
 __constant__ int c_hdirect[16];
+__constant__ int c_hentries;
 
 HashGridInfo hash_grid_info() {
   HashGridInfo h{};
@@ -165,7 +140,32 @@ cudaError_t upload_hash_grid(const HashGridInfo& h) {
   cudaError_t e = cudaMemcpyToSymbol(c_hres, h.res, sizeof h.res);
   if (e == cudaSuccess) e = cudaMemcpyToSymbol(c_hoff, h.offset, sizeof h.offset);
   if (e == cudaSuccess) e = cudaMemcpyToSymbol(c_hdirect, h.direct, sizeof h.direct);
+  const int entries = (int)h.entries;
+  if (e == cudaSuccess) e = cudaMemcpyToSymbol(c_hentries, &entries, sizeof entries);
   return e;
+}
+
+__device__ __forceinline__ uint32_t pick4(const uint4& q, int k) {
+  return k == 0 ? q.x : (k == 1 ? q.y : (k == 2 ? q.z : q.w));
+}
+
+// The feature pairs (one __half2, 4 bytes, each) of table rows ga and gb, two
+// corners of one cell that usually share an aligned group of four rows (16
+// bytes): one vector load returns both, and only the lanes whose partner lies
+// in another group issue a second 4-byte load. A group that would reach past
+// the table's end is read row by row.
+__device__ __forceinline__ void load_row_pair(const __half2* __restrict__ table, int ga, int gb,
+                                              uint32_t& va, uint32_t& vb) {
+  const uint32_t* t32 = reinterpret_cast<const uint32_t*>(table);
+  const int grp = ga & ~3;
+  if (grp + 3 < c_hentries) {
+    const uint4 q = __ldg(reinterpret_cast<const uint4*>(t32 + grp));
+    va = pick4(q, ga & 3);
+    vb = (gb & ~3) == grp ? pick4(q, gb & 3) : __ldg(t32 + gb);
+  } else {
+    va = __ldg(t32 + ga);
+    vb = __ldg(t32 + gb);
+  }
 }
 
 // Encoding of one point; optionally records the corner rows.
@@ -180,23 +180,40 @@ __device__ __forceinline__ void hash_encode_level(const __half2* __restrict__ ta
   const float f0 = floorf(c0), f1 = floorf(c1), f2 = floorf(c2);
   const float w0 = fsub(c0, f0), w1 = fsub(c1, f1), w2 = fsub(c2, f2);
   const int i0 = (int)f0, i1 = (int)f1, i2 = (int)f2;
-  a0 = 0.f;
-  a1 = 0.f;
+  const bool direct = c_hdirect[l] != 0;
+  int row[8];
 #pragma unroll
   for (int corner = 0; corner < 8; ++corner) {
     const int dx = corner >> 2, dy = (corner >> 1) & 1, dz = corner & 1;
     const int ix = min(max(i0 + dx, 0), N), iy = min(max(i1 + dy, 0), N),
               iz = min(max(i2 + dz, 0), N);
     uint32_t idx;
-    if (c_hdirect[l]) {
+    if (direct) {
       idx = (uint32_t)((ix * (N + 1) + iy) * (N + 1) + iz);
     } else {
       idx = ((uint32_t)ix ^ ((uint32_t)iy * 2654435761u) ^ ((uint32_t)iz * 805459861u)) &
             ((1u << 19) - 1u);
     }
-    const int row = c_hoff[l] + (int)idx;
-    if (rows_out) rows_out[l * 8 + corner] = row;
-    const float2 f = __half22float2(__ldg(table + row));
+    row[corner] = c_hoff[l] + (int)idx;
+    if (rows_out) rows_out[l * 8 + corner] = row[corner];
+  }
+  // Paired gathers: on a direct level the corners (dz = 0, 1) are adjacent rows;
+  // on a hashed level the x prime is 1, so the corners (dx = 0, 1) differ only in
+  // the low bits ix ^ (ix + 1) of their index.
+  uint32_t v[8];
+  if (direct) {
+#pragma unroll
+    for (int p = 0; p < 4; ++p) load_row_pair(table, row[2 * p], row[2 * p + 1], v[2 * p], v[2 * p + 1]);
+  } else {
+#pragma unroll
+    for (int p = 0; p < 4; ++p) load_row_pair(table, row[p], row[p + 4], v[p], v[p + 4]);
+  }
+  a0 = 0.f;
+  a1 = 0.f;
+#pragma unroll
+  for (int corner = 0; corner < 8; ++corner) {
+    const int dx = corner >> 2, dy = (corner >> 1) & 1, dz = corner & 1;
+    const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&v[corner]));
     const float wx = dx ? w0 : 1.0f - w0;
     const float wy = dy ? w1 : 1.0f - w1;
     const float wz = dz ? w2 : 1.0f - w2;
@@ -720,11 +737,17 @@ hash_tc_kernel(const float* __restrict__ o, const float* __restrict__ d, int64_t
           }
         }
       }
-      // drain before TMEM is freed
+      // drain before TMEM is freed (not stopped by an abort: the MMAs already
+      // issued must land first); running out is reported like any other wait
       uint64_t* fin = mma_done + HC_GROUPS;
       tcx::mma_commit(fin);
       const uint64_t t0 = tcx::globaltimer();
-      while (!tcx::mbar_try(fin, 0) && tcx::globaltimer() - t0 < kLimit) {}
+      bool drained = tcx::mbar_try(fin, 0);
+      while (!drained && tcx::globaltimer() - t0 < kLimit) drained = tcx::mbar_try(fin, 0);
+      if (!drained) {
+        atomicOr(flag, FLAG_TIMEOUT);
+        *abort_flag = 1;
+      }
     }
   } else {
     const int g = (warp - 1) >> 2;
@@ -1216,18 +1239,23 @@ cudaError_t launch_march_mask(const float* o, const float* d, int64_t R, float n
 
 cudaError_t march_render_chunk(const MarchArgs& a, cudaStream_t st) {
   const int64_t R = a.R;
+  const KernelTimer& tm = a.timer;
+  int slot = tm.begin(TK_MARCH_MASK, st);
   cudaError_t e = launch_march_mask(a.o + a.r0 * 3, a.d + a.r0 * 3, R, a.near, a.step, a.K, a.occ,
                                     a.ws.mask, a.ws.count, nullptr, st);
+  tm.end(slot, st);
   if (e != cudaSuccess) return e;
+  slot = tm.begin(TK_MARCH_COMPACT, st);
   e = exclusive_scan(a.ws.count, R, a.ws.off, a.ws.scan_tmp, st);
   if (e != cudaSuccess) return e;
   march_emit_kernel<<<(unsigned)((R + 7) / 8), 256, 0, st>>>(a.ws.mask, a.ws.off, R, a.K,
                                                              a.ws.live, a.ws.cap, a.flag);
+  tm.end(slot, st);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   const int32_t* total = a.ws.off + R;
   const unsigned g = (unsigned)(a.num_sms * 8);
   if (a.model == NERF_MODEL_HASHGRID) {
-    if (a.ev_start) cudaEventRecord(a.ev_start, st);
+    slot = tm.begin(TK_NETWORK, st);
     if (a.hash_tc)
       hash_tc_kernel<<<(unsigned)a.num_sms, HC_THREADS, HC_SMEM, st>>>(
           a.o, a.d, a.r0, a.near, a.step, a.ws.live, total,
@@ -1236,7 +1264,9 @@ cudaError_t march_render_chunk(const MarchArgs& a, cudaStream_t st) {
       hash_eval_kernel<<<(unsigned)(a.num_sms * HT_CTAS_PER_SM), HT_THREADS, HT_SMEM, st>>>(
           a.o, a.d, a.r0, a.near, a.step, a.ws.live, total,
           reinterpret_cast<const __half2*>(a.hash_table), a.hash_mlp, a.sh, a.ws.val);
+    tm.end(slot, st);
   } else {
+    slot = tm.begin(TK_ROUTER, st);
     cudaMemsetAsync(a.ws.cell_hist, 0, 2 * 4096 * sizeof(int32_t), st);
     cell_hist_kernel<<<g, 256, 0, st>>>(a.o, a.d, a.r0, a.near, a.step, a.ws.live, total,
                                         a.ws.cell, a.ws.cell_hist);
@@ -1248,16 +1278,19 @@ cudaError_t march_render_chunk(const MarchArgs& a, cudaStream_t st) {
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     kilo_items_kernel<<<1, 1024, 0, st>>>(a.ws.cell_hist, a.ws.cell_off, a.ws.items,
                                           a.ws.n_items);
+    tm.end(slot, st);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    if (a.ev_start) cudaEventRecord(a.ev_start, st);
+    slot = tm.begin(TK_NETWORK, st);
     kilo_eval_kernel<<<(unsigned)(a.num_sms * 2), KT_THREADS, KT_SMEM, st>>>(
         a.o, a.d, a.r0, a.near, a.step, a.ws.live, a.ws.order, a.ws.items, a.ws.n_items,
         a.cell_w, a.ws.val);
+    tm.end(slot, st);
   }
-  if (a.ev_stop) cudaEventRecord(a.ev_stop, st);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  slot = tm.begin(TK_MARCH_COMPOSITE, st);
   march_composite_kernel<<<(unsigned)((R + 7) / 8), 256, 0, st>>>(
       a.d, a.r0, R, a.near, a.step, a.ert_T, a.ws.off, a.ws.live, a.ws.val, a.rgb, a.depth, a.acc);
+  tm.end(slot, st);
   return cudaGetLastError();
 }
 

@@ -512,10 +512,17 @@ __global__ void __launch_bounds__(NTHREADS, 1) mlp_tc_kernel(Params P, const __g
              NERF_PP_LAYER(128, 0, 8);
       }
 #undef NERF_PP_LAYER
-      // drain: everything issued so far completes before the pair frees TMEM
+      // drain: everything issued so far completes before the pair frees TMEM.
+      // The wait does not stop on an abort (the MMAs already issued must land
+      // first); if it runs out, the timeout is reported like any other wait's.
       mma_commit_pair(final_bar);
-      uint64_t t0 = globaltimer();
-      while (!mbar_try_cl(final_bar, 0) && globaltimer() - t0 < 2000000000ull) {}
+      const uint64_t t0 = globaltimer();
+      bool drained = mbar_try_cl(final_bar, 0);
+      while (!drained && globaltimer() - t0 < ctl.limit_ns) drained = mbar_try_cl(final_bar, 0);
+      if (!drained) {
+        atomicOr(ctl.flag, FLAG_TIMEOUT);
+        *ctl.abort = 1;
+      }
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------- weight loader (both CTAs)

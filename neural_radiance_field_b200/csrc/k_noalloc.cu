@@ -48,19 +48,9 @@ cudaError_t scratch_for_current_device(int32_t** out) {
   return cudaSuccess;
 }
 
-// Same voxel decision as the march kernels: exact comparison with the voxel
-// boundaries b_v = -1.5 + v * 3/128.
-__device__ __forceinline__ int voxel_axis_na(float x) {
-  if (!(x >= -1.5f) || !(x < 1.5f)) return -1;
-  int v = (int)floorf(fmul(fadd(x, 1.5f), 42.666666666666664f));
-  v = v < 0 ? 0 : (v > 127 ? 127 : v);
-  if (x < fsub(fmul((float)v, 0.0234375f), 1.5f)) --v;
-  else if (v < 127 && x >= fsub(fmul((float)(v + 1), 0.0234375f), 1.5f)) ++v;
-  return v;
-}
-
-// Warp per ray: re-tests every candidate and writes the live ones, in order,
-// from the ray's offset.
+// Warp per ray: re-tests every candidate (the same decision as the mask kernel
+// that counted them) and writes the live ones, in order, from the ray's offset.
+// Writes never pass the next ray's offset.
 __global__ void emit_recompute_kernel(const float* __restrict__ o, const float* __restrict__ d,
                                       int64_t R, float near, float step, int K,
                                       const uint32_t* __restrict__ occ,
@@ -70,23 +60,27 @@ __global__ void emit_recompute_kernel(const float* __restrict__ o, const float* 
   const int64_t r = (int64_t)blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;
   if (r >= R) return;
   int64_t base = off[r];
+  const int64_t end = off[r + 1];
   for (int w = 0; w < (K + 31) / 32; ++w) {
     const int k = w * 32 + lane;
     bool is_live = false;
     if (k < K) {
-      const float t = fadd(near, fmul((float)k, step));
-      const int a = voxel_axis_na(fadd(o[r * 3 + 0], fmul(t, d[r * 3 + 0])));
-      const int b = voxel_axis_na(fadd(o[r * 3 + 1], fmul(t, d[r * 3 + 1])));
-      const int c = voxel_axis_na(fadd(o[r * 3 + 2], fmul(t, d[r * 3 + 2])));
-      if (a >= 0 && b >= 0 && c >= 0) {
-        const int idx = (a * 128 + b) * 128 + c;
-        is_live = (__ldg(occ + (idx >> 5)) >> (idx & 31)) & 1u;
-      }
+      float x[3], t;
+      march_point(o, d, r, near, step, k, x, &t);
+      is_live = occupied_at(occ, x[0], x[1], x[2], nullptr);
     }
     const uint32_t m = __ballot_sync(0xffffffffu, is_live);
-    if (is_live) live[base + __popc(m & ((1u << lane) - 1u))] = ((uint32_t)r << 9) | (uint32_t)k;
+    const int64_t pos = base + __popc(m & ((1u << lane) - 1u));
+    if (is_live && pos < end) live[pos] = ((uint32_t)r << 9) | (uint32_t)k;
     base += __popc(m);
   }
+}
+
+nerf_status cuda_error(cudaError_t e, const char* where) {
+  char msg[200];
+  snprintf(msg, sizeof msg, "nerf_march_compact_noalloc: %s: %s", where, cudaGetErrorString(e));
+  set_global_error(msg);
+  return NERF_ERR_CUDA;
 }
 
 }  // namespace
@@ -116,20 +110,20 @@ extern "C" nerf_status nerf_march_compact_noalloc(const float* rays_o, const flo
   }
   cudaStream_t st = (cudaStream_t)stream;
   int32_t* scan = nullptr;
-  if (scratch_for_current_device(&scan) != cudaSuccess) {
-    set_global_error("nerf_march_compact_noalloc: cudaGetSymbolAddress of the scratch failed");
-    return NERF_ERR_CUDA;
-  }
+  cudaError_t e = scratch_for_current_device(&scan);
+  if (e != cudaSuccess) return cuda_error(e, "cudaGetSymbolAddress of the scratch");
   // The per-ray live counts go into the front of the caller's out_live buffer
   // (it holds n_rays * K >= n_rays entries and is overwritten by the compaction
   // below), are scanned into out_offsets, and the live entries are then written.
   int32_t* counts = reinterpret_cast<int32_t*>(out_live);
-  if (launch_march_mask(rays_o, rays_d, n_rays, near, step, K, occupancy, nullptr, counts,
-                        nullptr, st) != cudaSuccess)
-    return NERF_ERR_CUDA;
-  if (exclusive_scan(counts, n_rays, out_offsets, scan, st) != cudaSuccess)
-    return NERF_ERR_CUDA;
+  e = launch_march_mask(rays_o, rays_d, n_rays, near, step, K, occupancy, nullptr, counts,
+                        nullptr, st);
+  if (e != cudaSuccess) return cuda_error(e, "live-count launch");
+  e = exclusive_scan(counts, n_rays, out_offsets, scan, st);
+  if (e != cudaSuccess) return cuda_error(e, "scan launch");
   emit_recompute_kernel<<<(unsigned)((n_rays + 7) / 8), 256, 0, st>>>(
       rays_o, rays_d, n_rays, near, step, K, occupancy, out_offsets, out_live);
-  return cudaGetLastError() == cudaSuccess ? NERF_OK : NERF_ERR_CUDA;
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_error(e, "emit launch");
+  return NERF_OK;
 }

@@ -211,6 +211,7 @@ nerf_status nerf_destroy(nerf_ctx* ctx) {
   if (ctx->ev) {
     for (int i = 0; i < 2 * kMaxTimed; ++i) cudaEventDestroy(ctx->ev[i]);
     delete[] ctx->ev;
+    delete[] ctx->ev_kind;
   }
   tc_free(ctx);
   delete ctx;
@@ -261,19 +262,15 @@ nerf_status nerf_raygen_batch(int H, int W, float focal, int n_cams, const float
 
 namespace {
 
+// Events around the launches of one kernel class while timing is enabled.
 struct TimedScope {
-  nerf_ctx* ctx;
+  KernelTimer tm;
   cudaStream_t st;
-  int slot = -1;
-  TimedScope(nerf_ctx* c, cudaStream_t s) : ctx(c), st(s) {
-    if (ctx->timing && ctx->n_timed < kMaxTimed) {
-      slot = ctx->n_timed++;
-      cudaEventRecord(ctx->ev[2 * slot], st);
-    }
+  int slot;
+  TimedScope(nerf_ctx* c, int kind, cudaStream_t s) : tm(c->timer()), st(s) {
+    slot = tm.begin(kind, st);
   }
-  ~TimedScope() {
-    if (slot >= 0) cudaEventRecord(ctx->ev[2 * slot + 1], st);
-  }
+  ~TimedScope() { tm.end(slot, st); }
 };
 
 // Runs one network (coarse or fine) over R rays with S samples each; `save`
@@ -284,17 +281,20 @@ nerf_status run_network(nerf_ctx* ctx, const void* blob, const float* o, const f
   const nerf_config& c = ctx->cfg;
   int64_t w_off, b_off;
   dir_offsets(c, &w_off, &b_off);
-  NERF_CHECK_LAUNCH(ctx, launch_dir_bias(d, R, blob, c.precision, c.W, c.L_dir, w_off, b_off,
-                                         ctx->dir_bias, st));
+  {
+    TimedScope ts(ctx, TK_DIR_BIAS, st);
+    NERF_CHECK_LAUNCH(ctx, launch_dir_bias(d, R, blob, c.precision, c.W, c.L_dir, w_off, b_off,
+                                           ctx->dir_bias, st));
+  }
   if (c.precision == NERF_BF16 && ctx->tc_enabled) {
     NERF_CHECK_LAUNCH(ctx, tc_pack(ctx, blob, st));
-    TimedScope ts(ctx, st);
+    TimedScope ts(ctx, TK_NETWORK, st);
     NERF_CHECK_LAUNCH(ctx, tc_run(ctx, o, d, R, ss, raw, st));
     return NERF_OK;
   }
   const int dir_ch = 3 * (1 + 2 * c.L_dir);
   NERF_CHECK_LAUNCH(ctx, launch_pack_fp32(blob, c.precision, ctx->plan, dir_ch, ctx->packed, st));
-  TimedScope ts(ctx, st);
+  TimedScope ts(ctx, TK_NETWORK, st);
   if (save) {
     NERF_CHECK_LAUNCH(ctx, mlp_forward_train_fp32(ctx->plan, ctx->packed, ctx->dir_bias, o, d, R,
                                                   ss, raw, save, st));
@@ -338,8 +338,10 @@ nerf_status check_render_args(nerf_ctx* ctx, const float* o, const float* d, int
       return fail(ctx, NERF_ERR_INVALID_ARG, "ert_T must be in [0, 1)");
     if (c.model == NERF_MODEL_KILONERF && !p->cell_w)
       return fail(ctx, NERF_ERR_INVALID_ARG, "cell_w is NULL");
-    if (c.model == NERF_MODEL_HASHGRID && (!p->hash_table || !p->hash_mlp || !aligned16(p->hash_mlp)))
-      return fail(ctx, NERF_ERR_INVALID_ARG, "hash_table / hash_mlp NULL or misaligned");
+    if (c.model == NERF_MODEL_HASHGRID &&
+        (!p->hash_table || !p->hash_mlp || !aligned16(p->hash_table) || !aligned16(p->hash_mlp)))
+      return fail(ctx, NERF_ERR_INVALID_ARG,
+                  "hash_table / hash_mlp NULL or not 16-byte aligned");
   }
   return NERF_OK;
 }
@@ -370,14 +372,67 @@ nerf_status render_march(nerf_ctx* ctx, const float* o, const float* d, int64_t 
   for (int64_t r0 = 0; r0 < R; r0 += ctx->chunk_rays) {
     a.r0 = r0;
     a.R = R - r0 < ctx->chunk_rays ? R - r0 : ctx->chunk_rays;
-    a.ev_start = a.ev_stop = nullptr;
-    if (ctx->timing && ctx->n_timed < kMaxTimed) {
-      const int slot = ctx->n_timed++;
-      a.ev_start = ctx->ev[2 * slot];
-      a.ev_stop = ctx->ev[2 * slot + 1];
-    }
+    a.timer = ctx->timer();
     NERF_CHECK_LAUNCH(ctx, march_render_chunk(a, st));
   }
+  return NERF_OK;
+}
+
+// The NeRF model's render (Section 2.6 render_rays): coarse network, coarse
+// compositing fused with resampling and the sorted merge, fine network, fine
+// compositing. `tr` (may be NULL) receives copies of the intermediates.
+nerf_status render_mlp(nerf_ctx* ctx, const float* rays_o, const float* rays_d, int64_t R,
+                       float near, float far, int n_coarse, int n_fine, const nerf_params* params,
+                       float* out_rgb, float* out_depth, float* out_acc, const nerf_trace* tr,
+                       cudaStream_t st) {
+  const nerf_config& c = ctx->cfg;
+  const uint64_t key = sm64_mix(params->seed);
+  SampleSpec coarse{};
+  coarse.mode = SAMPLES_STRATIFIED;
+  coarse.S = n_coarse;
+  coarse.near = near;
+  coarse.step = (far - near) / (float)n_coarse;
+  coarse.key = key;
+  coarse.perturb = params->perturb;
+  CompositeSpec cs{c.last_delta_mode, far, 0.0f, c.sigma_act, c.white_bkgd};
+
+  nerf_status s = run_network(ctx, params->coarse_w, rays_o, rays_d, R, coarse, ctx->raw, st);
+  if (s != NERF_OK) return s;
+  if (tr && tr->raw_coarse)
+    NERF_CHECK_LAUNCH(ctx, cudaMemcpyAsync(tr->raw_coarse, ctx->raw, (size_t)R * n_coarse * 16,
+                                           cudaMemcpyDeviceToDevice, st));
+  if (n_fine == 0) {
+    TimedScope ts(ctx, TK_COMPOSITE, st);
+    NERF_CHECK_LAUNCH(ctx, launch_composite(ctx->raw, coarse, rays_d, R, cs, out_rgb, out_depth,
+                                            out_acc, tr ? tr->w_coarse : nullptr, st));
+    return NERF_OK;
+  }
+  ResampleTrace rt{};
+  if (tr) {
+    rt.w = tr->w_coarse;
+    rt.t_f = tr->t_fine;
+    rt.below = tr->below;
+  }
+  {
+    TimedScope ts(ctx, TK_RESAMPLE, st);
+    NERF_CHECK_LAUNCH(ctx, launch_coarse_resample(ctx->raw, coarse, rays_d, R, cs, n_fine, key,
+                                                  params->perturb, ctx->t_all, st, rt));
+  }
+  SampleSpec fine{};
+  fine.mode = SAMPLES_GIVEN_T;
+  fine.S = n_coarse + n_fine;
+  fine.t = ctx->t_all;
+  if (tr && tr->t_all)
+    NERF_CHECK_LAUNCH(ctx, cudaMemcpyAsync(tr->t_all, ctx->t_all, (size_t)R * fine.S * 4,
+                                           cudaMemcpyDeviceToDevice, st));
+  s = run_network(ctx, params->fine_w, rays_o, rays_d, R, fine, ctx->raw, st);
+  if (s != NERF_OK) return s;
+  if (tr && tr->raw_fine)
+    NERF_CHECK_LAUNCH(ctx, cudaMemcpyAsync(tr->raw_fine, ctx->raw, (size_t)R * fine.S * 16,
+                                           cudaMemcpyDeviceToDevice, st));
+  TimedScope ts(ctx, TK_COMPOSITE, st);
+  NERF_CHECK_LAUNCH(ctx, launch_composite(ctx->raw, fine, rays_d, R, cs, out_rgb, out_depth,
+                                          out_acc, nullptr, st));
   return NERF_OK;
 }
 
@@ -392,39 +447,25 @@ nerf_status nerf_render(nerf_ctx* ctx, const float* rays_o, const float* rays_d,
                                     params, out_rgb, out_depth, out_acc);
   if (s != NERF_OK) return s;
   cudaStream_t st = (cudaStream_t)stream;
-  const nerf_config& c = ctx->cfg;
-  const int64_t R = n_rays;
-  if (c.model != NERF_MODEL_MLP)
-    return render_march(ctx, rays_o, rays_d, R, near, n_coarse, params, out_rgb, out_depth,
+  if (ctx->cfg.model != NERF_MODEL_MLP)
+    return render_march(ctx, rays_o, rays_d, n_rays, near, n_coarse, params, out_rgb, out_depth,
                         out_acc, st);
-  const uint64_t key = sm64_mix(params->seed);
-  SampleSpec coarse{};
-  coarse.mode = SAMPLES_STRATIFIED;
-  coarse.S = n_coarse;
-  coarse.near = near;
-  coarse.step = (far - near) / (float)n_coarse;
-  coarse.key = key;
-  coarse.perturb = params->perturb;
-  CompositeSpec cs{c.last_delta_mode, far, 0.0f, c.sigma_act, c.white_bkgd};
+  return render_mlp(ctx, rays_o, rays_d, n_rays, near, far, n_coarse, n_fine, params, out_rgb,
+                    out_depth, out_acc, nullptr, st);
+}
 
-  s = run_network(ctx, params->coarse_w, rays_o, rays_d, R, coarse, ctx->raw, st);
+nerf_status nerf_render_trace(nerf_ctx* ctx, const float* rays_o, const float* rays_d,
+                              int64_t n_rays, float near, float far, int n_coarse, int n_fine,
+                              const nerf_params* params, float* out_rgb, float* out_depth,
+                              float* out_acc, const nerf_trace* trace, void* stream) {
+  nerf_status s = check_render_args(ctx, rays_o, rays_d, n_rays, near, far, n_coarse, n_fine,
+                                    params, out_rgb, out_depth, out_acc);
   if (s != NERF_OK) return s;
-  if (n_fine == 0) {
-    NERF_CHECK_LAUNCH(ctx, launch_composite(ctx->raw, coarse, rays_d, R, cs, out_rgb, out_depth,
-                                            out_acc, nullptr, st));
-    return NERF_OK;
-  }
-  NERF_CHECK_LAUNCH(ctx, launch_coarse_resample(ctx->raw, coarse, rays_d, R, cs, n_fine, key,
-                                                params->perturb, ctx->t_all, st));
-  SampleSpec fine{};
-  fine.mode = SAMPLES_GIVEN_T;
-  fine.S = n_coarse + n_fine;
-  fine.t = ctx->t_all;
-  s = run_network(ctx, params->fine_w, rays_o, rays_d, R, fine, ctx->raw, st);
-  if (s != NERF_OK) return s;
-  NERF_CHECK_LAUNCH(ctx, launch_composite(ctx->raw, fine, rays_d, R, cs, out_rgb, out_depth,
-                                          out_acc, nullptr, st));
-  return NERF_OK;
+  if (!trace) return fail(ctx, NERF_ERR_INVALID_ARG, "trace is NULL");
+  if (ctx->cfg.model != NERF_MODEL_MLP)
+    return fail(ctx, NERF_ERR_UNSUPPORTED, "nerf_render_trace needs a NERF_MODEL_MLP context");
+  return render_mlp(ctx, rays_o, rays_d, n_rays, near, far, n_coarse, n_fine, params, out_rgb,
+                    out_depth, out_acc, trace, (cudaStream_t)stream);
 }
 
 nerf_status nerf_loss_grad(nerf_ctx* ctx, const float* rays_o, const float* rays_d,
@@ -539,6 +580,7 @@ nerf_status nerf_timing_enable(nerf_ctx* ctx, int enable) {
   if (!ctx) return fail(nullptr, NERF_ERR_INVALID_ARG, "ctx is NULL");
   if (enable && !ctx->ev) {
     ctx->ev = new cudaEvent_t[2 * kMaxTimed]();
+    ctx->ev_kind = new int[kMaxTimed]();
     for (int i = 0; i < 2 * kMaxTimed; ++i) {
       cudaError_t e = cudaEventCreate(&ctx->ev[i]);
       if (e != cudaSuccess) return cuda_fail(ctx, e, "cudaEventCreate");
@@ -549,20 +591,33 @@ nerf_status nerf_timing_enable(nerf_ctx* ctx, int enable) {
   return NERF_OK;
 }
 
-nerf_status nerf_timing_read(nerf_ctx* ctx, double* ms, int64_t* launches) {
+nerf_status nerf_timing_read_kinds(nerf_ctx* ctx, double* ms, int64_t* launches) {
   if (!ctx || !ms || !launches) return fail(ctx, NERF_ERR_INVALID_ARG, "NULL argument");
-  double tot = 0.0;
+  for (int k = 0; k < NERF_TIMED_KINDS; ++k) {
+    ms[k] = 0.0;
+    launches[k] = 0;
+  }
   for (int i = 0; i < ctx->n_timed; ++i) {
     cudaError_t e = cudaEventSynchronize(ctx->ev[2 * i + 1]);
     if (e != cudaSuccess) return cuda_fail(ctx, e, "cudaEventSynchronize");
     float t = 0.0f;
     e = cudaEventElapsedTime(&t, ctx->ev[2 * i], ctx->ev[2 * i + 1]);
     if (e != cudaSuccess) return cuda_fail(ctx, e, "cudaEventElapsedTime");
-    tot += t;
+    ms[ctx->ev_kind[i]] += t;
+    launches[ctx->ev_kind[i]] += 1;
   }
-  *ms = tot;
-  *launches = ctx->n_timed;
   ctx->n_timed = 0;
+  return NERF_OK;
+}
+
+nerf_status nerf_timing_read(nerf_ctx* ctx, double* ms, int64_t* launches) {
+  if (!ctx || !ms || !launches) return fail(ctx, NERF_ERR_INVALID_ARG, "NULL argument");
+  double all_ms[NERF_TIMED_KINDS];
+  int64_t all_n[NERF_TIMED_KINDS];
+  nerf_status s = nerf_timing_read_kinds(ctx, all_ms, all_n);
+  if (s != NERF_OK) return s;
+  *ms = all_ms[NERF_TIMED_NETWORK];
+  *launches = all_n[NERF_TIMED_NETWORK];
   return NERF_OK;
 }
 
@@ -670,7 +725,7 @@ nerf_status nerf_test_route_cells(const float* x, int64_t n, int32_t* out_cell,
 
 nerf_status nerf_test_hash_encode(const float* x, int64_t n, const uint16_t* hash_table,
                                   float* out_feat, int32_t* out_rows, void* stream) {
-  if (!x || !hash_table || !out_feat || n <= 0)
+  if (!x || !hash_table || !out_feat || n <= 0 || !aligned16(hash_table))
     return fail(nullptr, NERF_ERR_INVALID_ARG, "nerf_test_hash_encode: bad argument");
   NERF_CHECK_LAUNCH(nullptr, march_prepare(nullptr));
   NERF_CHECK_LAUNCH(nullptr, launch_hash_encode(x, n, hash_table, out_feat, out_rows,

@@ -26,10 +26,12 @@ struct nerf_ctx {
   float* tr_tmp = nullptr;     // backward scratch
   float* tr_loss = nullptr;    // [2 max_rays] per-ray loss terms
 
-  // network-kernel timing (nerf_timing_enable / nerf_timing_read)
+  // kernel timing (nerf_timing_enable / nerf_timing_read / nerf_timing_read_kinds)
   bool timing = false;
   int n_timed = 0;
   cudaEvent_t* ev = nullptr;   // 2 * kMaxTimed events, created on first enable
+  int* ev_kind = nullptr;      // kernel class of each event pair
+  nerfb::KernelTimer timer();
 
   // march models (KILONERF, HASHGRID): ray chunks and their live-entry workspace
   int64_t chunk_rays = 0;
@@ -43,6 +45,20 @@ struct nerf_ctx {
 
 namespace nerfb {
 constexpr int kMaxTimed = 4096;
+}  // namespace nerfb
+
+inline nerfb::KernelTimer nerf_ctx::timer() {
+  nerfb::KernelTimer t;
+  if (timing && ev) {
+    t.ev = ev;
+    t.kind = ev_kind;
+    t.n = &n_timed;
+    t.cap = nerfb::kMaxTimed;
+  }
+  return t;
+}
+
+namespace nerfb {
 cudaError_t tc_alloc(nerf_ctx* ctx);
 void tc_free(nerf_ctx* ctx);
 cudaError_t tc_pack(nerf_ctx* ctx, const void* blob, cudaStream_t st);

@@ -57,6 +57,37 @@ __device__ __forceinline__ void pe_sincos(float xc, int k, float* s, float* c) {
 
 struct Ctx;
 
+// Kernel classes that nerf_timing_enable times (NERF_TIMED_* of the header).
+enum TimedKind : int {
+  TK_NETWORK = NERF_TIMED_NETWORK,
+  TK_COMPOSITE = NERF_TIMED_COMPOSITE,
+  TK_RESAMPLE = NERF_TIMED_RESAMPLE,
+  TK_DIR_BIAS = NERF_TIMED_DIR_BIAS,
+  TK_MARCH_MASK = NERF_TIMED_MARCH_MASK,
+  TK_MARCH_COMPACT = NERF_TIMED_MARCH_COMPACT,
+  TK_ROUTER = NERF_TIMED_ROUTER,
+  TK_MARCH_COMPOSITE = NERF_TIMED_MARCH_COMPOSITE,
+};
+
+// Records a pair of CUDA events on the launching stream around the launches of
+// one kernel class; inert when timing is off (ev == nullptr) or the slots are used up.
+struct KernelTimer {
+  cudaEvent_t* ev = nullptr;   // [2 * cap]
+  int* kind = nullptr;         // [cap]
+  int* n = nullptr;
+  int cap = 0;
+  int begin(int k, cudaStream_t st) const {
+    if (!ev || *n >= cap) return -1;
+    const int s = (*n)++;
+    kind[s] = k;
+    cudaEventRecord(ev[2 * s], st);
+    return s;
+  }
+  void end(int slot, cudaStream_t st) const {
+    if (slot >= 0) cudaEventRecord(ev[2 * slot + 1], st);
+  }
+};
+
 // Launchers (each returns cudaGetLastError()).
 cudaError_t launch_raygen(int H, int W, float focal, const float* c2w, float* o, float* d,
                           cudaStream_t st);
@@ -120,11 +151,20 @@ cudaError_t launch_composite(const float* raw, const SampleSpec& ss, const float
                              const CompositeSpec& cs, float* rgb, float* depth, float* acc,
                              float* weights, cudaStream_t st);
 
+// Optional copies of the resampler's own intermediates (device, NULL = none):
+// the coarse weights it composited [R][64], its draws in draw order [R][Nf] and
+// their bins [R][Nf].
+struct ResampleTrace {
+  float* w = nullptr;
+  float* t_f = nullptr;
+  int32_t* below = nullptr;
+};
 // Coarse compositing fused with inverse-CDF resampling and the sorted merge:
 // raw_c [R][64][4] -> t_all [R][64 + Nf].
 cudaError_t launch_coarse_resample(const float* raw_c, const SampleSpec& coarse, const float* d,
                                    int64_t R, const CompositeSpec& cs, int Nf, uint64_t key,
-                                   int perturb, float* t_all, cudaStream_t st);
+                                   int perturb, float* t_all, cudaStream_t st,
+                                   const ResampleTrace& tr = ResampleTrace{});
 // Resampling from given coarse t and weights (unit entry point).
 cudaError_t launch_sample_pdf(const float* t_c, const float* w, int64_t R, int Nc, int Nf,
                               uint64_t key, int perturb, float* t_f, int32_t* below,

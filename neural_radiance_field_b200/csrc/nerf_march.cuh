@@ -5,6 +5,37 @@
 
 namespace nerfb {
 
+// ------------------------------------------------------------------ occupancy
+// Shared by every kernel that decides whether a march candidate is live, so that
+// they all take the same decision.
+
+// Voxel of one coordinate by exact comparison with the boundaries b_v = -1.5 +
+// v * 3/128 (exact in fp32): returns -1 outside [-1.5, 1.5).
+__device__ __forceinline__ int voxel_axis(float x) {
+  if (!(x >= -1.5f) || !(x < 1.5f)) return -1;
+  int v = (int)floorf(fmul(fadd(x, 1.5f), 42.666666666666664f));
+  v = v < 0 ? 0 : (v > 127 ? 127 : v);
+  if (x < fsub(fmul((float)v, 0.0234375f), 1.5f)) --v;
+  else if (v < 127 && x >= fsub(fmul((float)(v + 1), 0.0234375f), 1.5f)) ++v;
+  return v;
+}
+
+__device__ __forceinline__ bool occupied_at(const uint32_t* __restrict__ occ, float x0, float x1,
+                                            float x2, int* vox) {
+  const int a = voxel_axis(x0), b = voxel_axis(x1), c = voxel_axis(x2);
+  if (a < 0 || b < 0 || c < 0) return false;
+  const int idx = (a * 128 + b) * 128 + c;
+  if (vox) *vox = idx;
+  return (__ldg(occ + (idx >> 5)) >> (idx & 31)) & 1u;
+}
+
+__device__ __forceinline__ void march_point(const float* o, const float* d, int64_t r, float near,
+                                            float step, int k, float* x, float* t) {
+  *t = fadd(near, fmul((float)k, step));
+#pragma unroll
+  for (int c = 0; c < 3; ++c) x[c] = fadd(o[r * 3 + c], fmul(*t, d[r * 3 + c]));
+}
+
 struct HashGridInfo {
   int res[16];
   int offset[16];
@@ -53,8 +84,7 @@ struct MarchArgs {
   int num_sms;
   int hash_tc;                // hash model: MLP on the tensor cores (bf16 operands)
   MarchWs ws;
-  cudaEvent_t ev_start = nullptr;   // recorded around the scene-function kernel
-  cudaEvent_t ev_stop = nullptr;    // when timing is enabled
+  KernelTimer timer;          // events around each kernel class (timing enabled)
 };
 
 cudaError_t march_prepare(cudaStream_t st);

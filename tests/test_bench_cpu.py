@@ -35,3 +35,35 @@ def test_traffic_scales_with_the_rows_of_a_launch():
     t = bench.traffic_per_launch(bench.MLP_FLOP_PER_ROW * rows)
     assert abs(t - 236.75e6) < 1.0
     assert abs(bench.traffic_per_launch(2 * bench.MLP_FLOP_PER_ROW * rows) - 2 * t) < 1.0
+
+
+def test_nerf_kernel_bytes_of_the_bench_frame():
+    wl = S.WORKLOADS["full"]                    # 640,000 rays, 64 + 128 samples, W = 256
+    b = bench.nerf_kernel_bytes(wl)
+    assert b["composite"] == 640000 * (192 * 20 + 32)
+    assert b["resample"] == 640000 * (64 * 16 + 12 + 192 * 4)
+    assert b["dir_bias"] == 2 * 640000 * (12 + 128 * 4)
+    tiny = bench.nerf_kernel_bytes(S.WORKLOADS["tiny"])   # coarse only: positions recomputed
+    assert tiny["composite"] == 1024 * (64 * 16 + 32) and "resample" not in tiny
+
+
+def test_nerf_launch_counts_and_rows():
+    assert bench.nerf_launches_per_step(S.WORKLOADS["full"]) == 9
+    assert bench.nerf_launches_per_step(S.WORKLOADS["tiny"]) == 5
+    assert bench.rows_per_frame(S.WORKLOADS["full"]) == 640000 * 256
+    assert bench.rows_per_frame(S.WORKLOADS["tiny"]) == 1024 * 64
+
+
+def test_bandwidth_figures():
+    kinds = {"composite": (20.0, 10), "resample": (0.0, 0)}
+    out = bench.bandwidth_figures(kinds, {"composite": 4e9, "resample": 1e9}, 10, 8000.0, "x")
+    assert set(out) == {"composite"}                     # untimed classes are left out
+    assert abs(out["composite"]["achieved_gbs"] - 4e9 * 10 / 0.020 / 1e9) < 1e-6
+    assert abs(out["composite"]["frac"] - out["composite"]["achieved_gbs"] / 8000.0) < 1e-12
+
+
+def test_march_kernel_bytes():
+    b = bench.march_kernel_bytes(S.WORKLOADS["hashgrid"], 100, 1000, False)
+    assert b["network"] == 1000 * 532 and b["march_mask"] == 100 * 92 and "router" not in b
+    k = bench.march_kernel_bytes(S.WORKLOADS["kilonerf"], 100, 1000, False)
+    assert k["router"] == 16000 and "network" not in k

@@ -10,8 +10,8 @@ import pytest
 
 import nerf_inputs as S
 
-from gpu_cases import (RAW_BOUND, compare, make_renderer, oracle_render, oracle_weights,
-                       rays_for, tolerances, weights_tensor)
+from gpu_cases import (check_rays, make_renderer, oracle_render, oracle_weights, rays_for,
+                       weights_tensor)
 
 pytestmark = pytest.mark.gpu
 
@@ -63,11 +63,7 @@ def test_render_rejects_bad_requests_then_renders_its_maximum_batch(torch):
     got = dict(rgb=rgb[:R].cpu().numpy(), depth=dep[:R].cpu().numpy(), acc=acc[:R].cpu().numpy())
     ids = np.arange(R)
     ref = oracle_render(wl, o.cpu().numpy(), d.cpu().numpy(), ids, cw, fw)
-    err, keep = compare(got, ref, wl, band=2 * RAW_BOUND[wl.precision])
-    t_rgb, t_acc, t_dep = tolerances(wl)
-    assert keep.mean() > 0.9
-    assert err["rgb"][keep].max() <= t_rgb and err["acc"][keep].max() <= t_acc
-    assert err["depth"][keep].max() <= t_dep
+    check_rays(wl, got, ref, "tiny, maximum batch")
 
 
 def test_march_render_rejects_bad_candidate_counts(torch):

@@ -3,7 +3,8 @@ for callers that cannot call cudaMalloc: a host framework that owns all device
 memory through its own allocator, or a render loop held to a fixed budget.
 
 Its output must match the allocating march test entry point (nerf_test_march)
-exactly: it is integer work (live-candidate decisions and their prefix sum).
+exactly, and the oracle's occupancy test (oracle.march.occupied) on the same
+candidates: it is integer work (live-candidate decisions and their prefix sum).
 Two calls in a row check that the shared static scratch carries nothing from
 one call into the next. The file sorts last so that a run stopping at the first
 failure has run every other test before it."""
@@ -13,6 +14,8 @@ import numpy as np
 import pytest
 
 import nerf_inputs as S
+from oracle import march as omarch
+from oracle import nerf as onerf
 
 from gpu_cases import rays_for
 
@@ -42,6 +45,17 @@ def _reference(torch, o, d, wl, K, occ):
     return offsets, entries
 
 
+def _oracle(o, d, wl, K, dense):
+    """Offsets and live entries from the oracle's voxel test of every candidate
+    x = fl(o + fl(t_k d)), t_k = fl(near + fl(k step))."""
+    x = onerf.points(o, d, np.broadcast_to(onerf.march_t(wl.near, wl.march_step, K),
+                                           (o.shape[0], K)))
+    flags = omarch.occupied(x, dense)
+    offsets = np.concatenate([[0], np.cumsum(flags.sum(1))])
+    ray, k = np.nonzero(flags)
+    return offsets, ((ray.astype(np.uint64) << 9) | k.astype(np.uint64)).astype(np.uint32)
+
+
 def _noalloc(torch, o, d, wl, K, occ):
     from neural_radiance_field_b200 import _capi
     R = o.shape[0]
@@ -65,12 +79,15 @@ def test_noalloc_compaction_matches_allocating_entry_point_twice(torch):
         o, d = rays_for(wl)
         ids = S.ray_subset(wl.n_rays, n, seed)
         o, d = o[ids].contiguous(), d[ids].contiguous()
-        packed, _ = S.occupancy_grid(wl.seed)
+        packed, dense = S.occupancy_grid(wl.seed)
         occ = torch.from_numpy(packed.view(np.int32)).cuda()
         ref_off, ref_live = _reference(torch, o, d, wl, wl.n_coarse, occ)
         off, live = _noalloc(torch, o, d, wl, wl.n_coarse, occ)
         np.testing.assert_array_equal(off, ref_off)
         np.testing.assert_array_equal(live, ref_live)
+        or_off, or_live = _oracle(o.cpu().numpy(), d.cpu().numpy(), wl, wl.n_coarse, dense)
+        np.testing.assert_array_equal(off, or_off)
+        np.testing.assert_array_equal(live, or_live)
         assert ref_off[-1] > 0
 
 
