@@ -99,8 +99,7 @@ typedef struct {
  *  cell_w            KILONERF: fp32 [4096][3317] per-cell parameters, cell id
  *                    (cx*16+cy)*16+cz; per cell: W1[32][63] b1[32] W2[32][32]
  *                    b2[32] w_sigma[32] b_sigma[1] Wc[3][59] bc[3].
- *  hash_table        HASHGRID: fp16 [6101902][2], all 16 levels concatenated;
- *                    16-byte aligned (rows are read in aligned groups of four).
+ *  hash_table        HASHGRID: fp16 [6101902][2], all 16 levels concatenated.
  *  hash_mlp          HASHGRID: fp32 blob d0[64][32] b, d1[64][64] b, sigma[1][64] b,
  *                    c0[64][80] b, c1[64][64] b, rgb[3][64] b.
  *  march_step        march models: t_k = near + k * march_step, k < n_coarse.
@@ -351,8 +350,7 @@ NERF_API nerf_status nerf_test_route_cells(const float* x, int64_t n, int32_t* o
  * index (ix*(N+1)+iy)*(N+1)+iz while (N+1)^3 <= T, else (ix XOR iy*2654435761
  * XOR iz*805459861) mod T; trilinear weights of c = fl(fl((x + 1.5)/3) * N).
  * x [P][3]; out_feat [P][32] (level-major); out_rows [P][16][8] int32 (may be
- * NULL): global table row of every corner (dx, dy, dz loop order). hash_table
- * must be 16-byte aligned (NERF_ERR_INVALID_ARG otherwise). */
+ * NULL): global table row of every corner (dx, dy, dz loop order). */
 NERF_API nerf_status nerf_test_hash_encode(const float* x, int64_t n, const uint16_t* hash_table,
                                            float* out_feat, int32_t* out_rows, void* stream);
 

@@ -113,7 +113,6 @@ cudaError_t exclusive_scan(const int32_t* in, int64_t n, int32_t* out, int32_t* 
 __constant__ int c_hres[16];
 __constant__ int c_hoff[16];
 __constant__ int c_hdirect[16];
-__constant__ int c_hentries;
 
 HashGridInfo hash_grid_info() {
   HashGridInfo h{};
@@ -140,32 +139,7 @@ cudaError_t upload_hash_grid(const HashGridInfo& h) {
   cudaError_t e = cudaMemcpyToSymbol(c_hres, h.res, sizeof h.res);
   if (e == cudaSuccess) e = cudaMemcpyToSymbol(c_hoff, h.offset, sizeof h.offset);
   if (e == cudaSuccess) e = cudaMemcpyToSymbol(c_hdirect, h.direct, sizeof h.direct);
-  const int entries = (int)h.entries;
-  if (e == cudaSuccess) e = cudaMemcpyToSymbol(c_hentries, &entries, sizeof entries);
   return e;
-}
-
-__device__ __forceinline__ uint32_t pick4(const uint4& q, int k) {
-  return k == 0 ? q.x : (k == 1 ? q.y : (k == 2 ? q.z : q.w));
-}
-
-// The feature pairs (one __half2, 4 bytes, each) of table rows ga and gb, two
-// corners of one cell that usually share an aligned group of four rows (16
-// bytes): one vector load returns both, and only the lanes whose partner lies
-// in another group issue a second 4-byte load. A group that would reach past
-// the table's end is read row by row.
-__device__ __forceinline__ void load_row_pair(const __half2* __restrict__ table, int ga, int gb,
-                                              uint32_t& va, uint32_t& vb) {
-  const uint32_t* t32 = reinterpret_cast<const uint32_t*>(table);
-  const int grp = ga & ~3;
-  if (grp + 3 < c_hentries) {
-    const uint4 q = __ldg(reinterpret_cast<const uint4*>(t32 + grp));
-    va = pick4(q, ga & 3);
-    vb = (gb & ~3) == grp ? pick4(q, gb & 3) : __ldg(t32 + gb);
-  } else {
-    va = __ldg(t32 + ga);
-    vb = __ldg(t32 + gb);
-  }
 }
 
 // Encoding of one point; optionally records the corner rows.
@@ -180,40 +154,23 @@ __device__ __forceinline__ void hash_encode_level(const __half2* __restrict__ ta
   const float f0 = floorf(c0), f1 = floorf(c1), f2 = floorf(c2);
   const float w0 = fsub(c0, f0), w1 = fsub(c1, f1), w2 = fsub(c2, f2);
   const int i0 = (int)f0, i1 = (int)f1, i2 = (int)f2;
-  const bool direct = c_hdirect[l] != 0;
-  int row[8];
+  a0 = 0.f;
+  a1 = 0.f;
 #pragma unroll
   for (int corner = 0; corner < 8; ++corner) {
     const int dx = corner >> 2, dy = (corner >> 1) & 1, dz = corner & 1;
     const int ix = min(max(i0 + dx, 0), N), iy = min(max(i1 + dy, 0), N),
               iz = min(max(i2 + dz, 0), N);
     uint32_t idx;
-    if (direct) {
+    if (c_hdirect[l]) {
       idx = (uint32_t)((ix * (N + 1) + iy) * (N + 1) + iz);
     } else {
       idx = ((uint32_t)ix ^ ((uint32_t)iy * 2654435761u) ^ ((uint32_t)iz * 805459861u)) &
             ((1u << 19) - 1u);
     }
-    row[corner] = c_hoff[l] + (int)idx;
-    if (rows_out) rows_out[l * 8 + corner] = row[corner];
-  }
-  // Paired gathers: on a direct level the corners (dz = 0, 1) are adjacent rows;
-  // on a hashed level the x prime is 1, so the corners (dx = 0, 1) differ only in
-  // the low bits ix ^ (ix + 1) of their index.
-  uint32_t v[8];
-  if (direct) {
-#pragma unroll
-    for (int p = 0; p < 4; ++p) load_row_pair(table, row[2 * p], row[2 * p + 1], v[2 * p], v[2 * p + 1]);
-  } else {
-#pragma unroll
-    for (int p = 0; p < 4; ++p) load_row_pair(table, row[p], row[p + 4], v[p], v[p + 4]);
-  }
-  a0 = 0.f;
-  a1 = 0.f;
-#pragma unroll
-  for (int corner = 0; corner < 8; ++corner) {
-    const int dx = corner >> 2, dy = (corner >> 1) & 1, dz = corner & 1;
-    const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&v[corner]));
+    const int row = c_hoff[l] + (int)idx;
+    if (rows_out) rows_out[l * 8 + corner] = row;
+    const float2 f = __half22float2(__ldg(table + row));
     const float wx = dx ? w0 : 1.0f - w0;
     const float wy = dy ? w1 : 1.0f - w1;
     const float wz = dz ? w2 : 1.0f - w2;

@@ -10,7 +10,9 @@
 // other tile's layer is computed. Each weight chunk that lands in the ring
 // serves both tiles (tile A's pass waits for it, tile B's pass frees its slot),
 // so each weight byte read from L2 serves 512 rows. Per CTA, 18 warps:
-//   warp 0       CTA 0: issues the MMAs of the pair; both CTAs: TMEM allocation
+//   warp 0       CTA 0: issues the MMAs of the pair; CTA 1: relays its epilogue's
+//                hand-offs to CTA 0 (one remote arrive per tile and layer);
+//                both CTAs: TMEM allocation
 //   warp 1       streams this CTA's half of each weight chunk into an 8-slot ring
 //                (one 256-input layer)
 //   warps 2-9    epilogue of tile A: warp w drains TMEM lane quarter (w % 4) of
@@ -397,15 +399,15 @@ __device__ __forceinline__ bool mma_pass(int g, uint32_t q0, uint64_t* full, uin
 }
 
 // The epilogue's hand-off to the MMA thread: every lane has made its stores
-// visible to the async proxy; after the warp converges, one lane arrives (on
-// CTA 0's barrier, remotely from CTA 1). 256 per-thread arrivals on one
-// barrier would serialize; 8 per CTA do not.
-__device__ __forceinline__ void warp_arrive_act(uint64_t* bar, uint32_t cta, int lane) {
+// visible to the async proxy; after the warp converges, one lane arrives on a
+// barrier of its own CTA: CTA 0's warps on the MMA thread's barrier, CTA 1's
+// on a local one that CTA 1's relay thread forwards. A remote arrive with
+// cluster-scope release costs a warp about 1,100 cycles more than a local one
+// (measured), so CTA 1 pays it once per tile and layer, off its warps' path.
+// 256 per-thread arrivals on one barrier would serialize; 8 per CTA do not.
+__device__ __forceinline__ void warp_arrive_act(uint64_t* bar, int lane) {
   __syncwarp();
-  if (lane == 0) {
-    if (cta == 0) mbar_arrive(bar);
-    else mbar_arrive_leader(bar);
-  }
+  if (lane == 0) mbar_arrive(bar);
 }
 
 __device__ __forceinline__ bool wait_act(int g, uint32_t (&ph_act)[2], uint64_t* act_ready,
@@ -462,7 +464,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) mlp_tc_kernel(Params P, const __g
   uint64_t* mma_done = bars + 2 * NSTAGE;     // [2]
   uint64_t* act_ready = bars + 2 * NSTAGE + 2;  // [2] (used in CTA 0)
   uint64_t* final_bar = bars + 2 * NSTAGE + 4;
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 2 * NSTAGE + 5);
+  uint64_t* act_local = bars + 2 * NSTAGE + 5;   // [2] (used in CTA 1)
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 2 * NSTAGE + 7);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
   const int warp = threadIdx.x >> 5;
@@ -475,7 +478,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) mlp_tc_kernel(Params P, const __g
     for (int s = 0; s < NSTAGE; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
     for (int g = 0; g < 2; ++g) {
       mbar_init(&mma_done[g], 1);
-      mbar_init(&act_ready[g], 2 * TILE_THREADS / 32);   // one arrival per epilogue warp
+      // CTA 0's epilogue warps of the tile, and CTA 1's relay
+      mbar_init(&act_ready[g], TILE_THREADS / 32 + 1);
+      mbar_init(&act_local[g], TILE_THREADS / 32);   // CTA 1's epilogue warps of the tile
     }
     mbar_init(final_bar, 1);
     *abort_flag = 0;
@@ -523,6 +528,19 @@ __global__ void __launch_bounds__(NTHREADS, 1) mlp_tc_kernel(Params P, const __g
         atomicOr(ctl.flag, FLAG_TIMEOUT);
         *ctl.abort = 1;
       }
+    } else if (lane == 0 && cta == 1) {
+      // relay: every hand-off of CTA 1's epilogue (the gamma(x) columns of each
+      // pair, then layers 0..8 of each tile) to CTA 0's barrier, in the order
+      // the MMA thread consumes them (A before B in each layer)
+      uint32_t ph[2] = {0, 0};
+      bool ok = true;
+      for (int64_t pr = cid; pr < P.n_pairs && ok; pr += ncl)
+        for (int j = 0; j < NLAYER && ok; ++j)
+          for (int g = 0; g < 2 && ok; ++g) {
+            ok = mbar_wait(&act_local[g], ph[g], ctl);
+            ph[g] ^= 1;
+            if (ok) mbar_arrive_leader(&act_ready[g]);
+          }
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------- weight loader (both CTAs)
@@ -554,6 +572,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) mlp_tc_kernel(Params P, const __g
     const int quarter = warp & 3;                 // TMEM lane quarter of this warp
     const int r = quarter * 32 + lane;            // row in this CTA's half tile = TMEM lane
     uint8_t* my_act = act + g * ACT_BYTES;
+    uint64_t* my_ready = cta == 0 ? &act_ready[g] : &act_local[g];
     const uint32_t act_base = smem_u32(my_act);
     const uint32_t t_row = tmem + (uint32_t)(g * 256) + ((uint32_t)(quarter * 32) << 16);
     const int tt = et & 255;                      // thread within the tile
@@ -590,12 +609,14 @@ __global__ void __launch_bounds__(NTHREADS, 1) mlp_tc_kernel(Params P, const __g
       if (h == 0) store_pe<0>(x[0], x[1], x[2], act_base, r);
       else store_pe<1>(x[0], x[1], x[2], act_base, r);
       fence_async_smem();
-      warp_arrive_act(&act_ready[g], cta, lane);
+      warp_arrive_act(my_ready, lane);
 
       float sigma = 0.0f;
-      for (int l = 0; l < NLAYER; ++l) {
-        // this layer's epilogue vectors: loaded now, staged after the MMA wait
-        // (all values are bf16 weights of the blob, so the bf16 staging is exact)
+      // A layer's epilogue vectors (all bf16 weights of the blob, so the bf16
+      // staging is exact) are staged while the tile waits for that layer's
+      // MMAs, so that nothing but the accumulator stands between the MMAs'
+      // completion and the epilogue.
+      auto stage_vectors = [&](int l) {
         float pre0, pre1 = 0.0f;
         if (l < 9) {
           pre0 = __ldg(vec + P.lay.bias[l] + tt);
@@ -606,15 +627,19 @@ __global__ void __launch_bounds__(NTHREADS, 1) mlp_tc_kernel(Params P, const __g
                : tt < 131 ? __ldg(vec + P.lay.b_rgb + tt - 128)
                : tt == 131 ? __ldg(vec + P.lay.b_sigma) : 0.0f;
         }
+        sb0[tt] = __bfloat16_as_ushort(__float2bfloat16_rn(pre0));
+        sb1[tt] = __bfloat16_as_ushort(__float2bfloat16_rn(pre1));
+      };
+      // the tile's threads are done with the previous pair's vectors; all
+      // agree on giving up together, so no thread is left behind at a barrier
+      if (tile_sync_or(g, *abort_flag)) break;
+      stage_vectors(0);
+      tile_sync(g);
+      bool stop = false;
+      for (int l = 0; l < NLAYER; ++l) {
         const bool waited = mbar_wait_cl(&mma_done[g], ph_md, ctl);
         ph_md ^= 1;
         tc_fence_after();
-        // every thread of the tile is done with the previous vectors; all agree
-        // on giving up together, so no thread is left behind at a barrier
-        if (tile_sync_or(g, !waited || *abort_flag)) break;
-        sb0[tt] = __bfloat16_as_ushort(__float2bfloat16_rn(pre0));
-        sb1[tt] = __bfloat16_as_ushort(__float2bfloat16_rn(pre1));
-        tile_sync(g);
         if (l < 9) {
           const int c0 = h * 128;
           if (l == 8) epi_half<false, false>(t_row, c0, sb0, sb1, act_base, r, sigma);
@@ -622,7 +647,10 @@ __global__ void __launch_bounds__(NTHREADS, 1) mlp_tc_kernel(Params P, const __g
           else epi_half<true, false>(t_row, c0, sb0, sb1, act_base, r, sigma);
           tc_fence_before();
           fence_async_smem();
-          warp_arrive_act(&act_ready[g], cta, lane);
+          warp_arrive_act(my_ready, lane);
+          if (tile_sync_or(g, !waited || *abort_flag)) { stop = true; break; }
+          stage_vectors(l + 1);
+          tile_sync(g);
         } else {
           // direction layer (N = 128): + per-ray bias, ReLU, the rgb head in fp32
           // on this half's 64 columns; the halves are summed through shared memory
@@ -665,9 +693,10 @@ __global__ void __launch_bounds__(NTHREADS, 1) mlp_tc_kernel(Params P, const __g
                             rgb2 + o2.w + bf(130), sigma + o2.x + bf(131));
           }
           tile_sync(g);
+          if (!waited) stop = true;
         }
       }
-      if (tile_sync_or(g, *abort_flag)) break;
+      if (tile_sync_or(g, stop || *abort_flag)) break;
     }
   }
 

@@ -338,10 +338,8 @@ nerf_status check_render_args(nerf_ctx* ctx, const float* o, const float* d, int
       return fail(ctx, NERF_ERR_INVALID_ARG, "ert_T must be in [0, 1)");
     if (c.model == NERF_MODEL_KILONERF && !p->cell_w)
       return fail(ctx, NERF_ERR_INVALID_ARG, "cell_w is NULL");
-    if (c.model == NERF_MODEL_HASHGRID &&
-        (!p->hash_table || !p->hash_mlp || !aligned16(p->hash_table) || !aligned16(p->hash_mlp)))
-      return fail(ctx, NERF_ERR_INVALID_ARG,
-                  "hash_table / hash_mlp NULL or not 16-byte aligned");
+    if (c.model == NERF_MODEL_HASHGRID && (!p->hash_table || !p->hash_mlp || !aligned16(p->hash_mlp)))
+      return fail(ctx, NERF_ERR_INVALID_ARG, "hash_table / hash_mlp NULL or misaligned");
   }
   return NERF_OK;
 }
@@ -725,7 +723,7 @@ nerf_status nerf_test_route_cells(const float* x, int64_t n, int32_t* out_cell,
 
 nerf_status nerf_test_hash_encode(const float* x, int64_t n, const uint16_t* hash_table,
                                   float* out_feat, int32_t* out_rows, void* stream) {
-  if (!x || !hash_table || !out_feat || n <= 0 || !aligned16(hash_table))
+  if (!x || !hash_table || !out_feat || n <= 0)
     return fail(nullptr, NERF_ERR_INVALID_ARG, "nerf_test_hash_encode: bad argument");
   NERF_CHECK_LAUNCH(nullptr, march_prepare(nullptr));
   NERF_CHECK_LAUNCH(nullptr, launch_hash_encode(x, n, hash_table, out_feat, out_rows,
