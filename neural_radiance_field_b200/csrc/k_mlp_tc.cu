@@ -10,9 +10,7 @@
 // other tile's layer is computed. Each weight chunk that lands in the ring
 // serves both tiles (tile A's pass waits for it, tile B's pass frees its slot),
 // so each weight byte read from L2 serves 512 rows. Per CTA, 18 warps:
-//   warp 0       CTA 0: issues the MMAs of the pair; CTA 1: relays its epilogue's
-//                hand-offs to CTA 0 (one remote arrive per tile and layer);
-//                both CTAs: TMEM allocation
+//   warp 0       CTA 0: issues the MMAs of the pair; both CTAs: TMEM allocation
 //   warp 1       streams this CTA's half of each weight chunk into an 8-slot ring
 //                (one 256-input layer)
 //   warps 2-9    epilogue of tile A: warp w drains TMEM lane quarter (w % 4) of
@@ -201,7 +199,15 @@ __device__ __forceinline__ void epi_block(const uint32_t* u, const uint16_t* sb_
     load_bf16x8(sb_bias + cb + 8 * j, b);
     float v[8];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(u[8 * j + i]) + b[i];
+    for (int i = 0; i < 8; i += 2)
+      asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+          "mov.b64 ra, {%2, %3};\n\t"
+          "mov.b64 rb, {%4, %5};\n\t"
+          "add.rn.f32x2 rd, ra, rb;\n\t"
+          "mov.b64 {%0, %1}, rd;\n\t}"
+          : "=f"(v[i]), "=f"(v[i + 1])
+          : "f"(__uint_as_float(u[8 * j + i])), "f"(__uint_as_float(u[8 * j + i + 1])),
+            "f"(b[i]), "f"(b[i + 1]));
     if (SIGMA) {
       float w[8];
       load_bf16x8(sb_ws + cb + 8 * j, w);
@@ -316,12 +322,17 @@ __device__ __forceinline__ bool mbar_wait_cl(uint64_t* bar, uint32_t parity, con
   return true;
 }
 
-// Arrive on the barrier at the same offset in CTA 0 of the cluster.
+// Arrive on the barrier at the same offset in CTA 0 of the cluster, releasing
+// at cluster scope this CTA's shared-memory writes (including those the calling
+// thread has acquired from other threads): a release fence restricted to
+// shared::cta operations, then a relaxed remote arrive. A full cluster-scope
+// release on the arrive itself costs about 1,100 cycles more (measured).
 __device__ __forceinline__ void mbar_arrive_leader(uint64_t* bar) {
   asm volatile(
       "{\n\t.reg .b32 ra;\n\t"
       "mapa.shared::cluster.u32 ra, %0, 0;\n\t"
-      "mbarrier.arrive.release.cluster.shared::cluster.b64 _, [ra];\n\t}"
+      "fence.release.sync_restrict::shared::cta.cluster;\n\t"
+      "mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [ra];\n\t}"
       ::"r"(smem_u32(bar))
       : "memory");
 }
@@ -399,15 +410,16 @@ __device__ __forceinline__ bool mma_pass(int g, uint32_t q0, uint64_t* full, uin
 }
 
 // The epilogue's hand-off to the MMA thread: every lane has made its stores
-// visible to the async proxy; after the warp converges, one lane arrives on a
-// barrier of its own CTA: CTA 0's warps on the MMA thread's barrier, CTA 1's
-// on a local one that CTA 1's relay thread forwards. A remote arrive with
-// cluster-scope release costs a warp about 1,100 cycles more than a local one
-// (measured), so CTA 1 pays it once per tile and layer, off its warps' path.
-// 256 per-thread arrivals on one barrier would serialize; 8 per CTA do not.
-__device__ __forceinline__ void warp_arrive_act(uint64_t* bar, int lane) {
+// visible to the async proxy; after the warp converges, one lane arrives on the
+// MMA thread's barrier in CTA 0 (remotely from CTA 1, with the restricted
+// release fence of mbar_arrive_leader). 256 per-thread arrivals on one barrier
+// would serialize; 8 per CTA do not.
+__device__ __forceinline__ void warp_arrive_act(uint64_t* bar, uint32_t cta, int lane) {
   __syncwarp();
-  if (lane == 0) mbar_arrive(bar);
+  if (lane == 0) {
+    if (cta == 0) mbar_arrive(bar);
+    else mbar_arrive_leader(bar);
+  }
 }
 
 __device__ __forceinline__ bool wait_act(int g, uint32_t (&ph_act)[2], uint64_t* act_ready,
@@ -464,8 +476,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) mlp_tc_kernel(Params P, const __g
   uint64_t* mma_done = bars + 2 * NSTAGE;     // [2]
   uint64_t* act_ready = bars + 2 * NSTAGE + 2;  // [2] (used in CTA 0)
   uint64_t* final_bar = bars + 2 * NSTAGE + 4;
-  uint64_t* act_local = bars + 2 * NSTAGE + 5;   // [2] (used in CTA 1)
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 2 * NSTAGE + 7);
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 2 * NSTAGE + 5);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
   const int warp = threadIdx.x >> 5;
@@ -478,9 +489,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) mlp_tc_kernel(Params P, const __g
     for (int s = 0; s < NSTAGE; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
     for (int g = 0; g < 2; ++g) {
       mbar_init(&mma_done[g], 1);
-      // CTA 0's epilogue warps of the tile, and CTA 1's relay
-      mbar_init(&act_ready[g], TILE_THREADS / 32 + 1);
-      mbar_init(&act_local[g], TILE_THREADS / 32);   // CTA 1's epilogue warps of the tile
+      mbar_init(&act_ready[g], 2 * TILE_THREADS / 32);   // one arrival per epilogue warp
     }
     mbar_init(final_bar, 1);
     *abort_flag = 0;
@@ -528,19 +537,6 @@ __global__ void __launch_bounds__(NTHREADS, 1) mlp_tc_kernel(Params P, const __g
         atomicOr(ctl.flag, FLAG_TIMEOUT);
         *ctl.abort = 1;
       }
-    } else if (lane == 0 && cta == 1) {
-      // relay: every hand-off of CTA 1's epilogue (the gamma(x) columns of each
-      // pair, then layers 0..8 of each tile) to CTA 0's barrier, in the order
-      // the MMA thread consumes them (A before B in each layer)
-      uint32_t ph[2] = {0, 0};
-      bool ok = true;
-      for (int64_t pr = cid; pr < P.n_pairs && ok; pr += ncl)
-        for (int j = 0; j < NLAYER && ok; ++j)
-          for (int g = 0; g < 2 && ok; ++g) {
-            ok = mbar_wait(&act_local[g], ph[g], ctl);
-            ph[g] ^= 1;
-            if (ok) mbar_arrive_leader(&act_ready[g]);
-          }
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------- weight loader (both CTAs)
@@ -572,7 +568,6 @@ __global__ void __launch_bounds__(NTHREADS, 1) mlp_tc_kernel(Params P, const __g
     const int quarter = warp & 3;                 // TMEM lane quarter of this warp
     const int r = quarter * 32 + lane;            // row in this CTA's half tile = TMEM lane
     uint8_t* my_act = act + g * ACT_BYTES;
-    uint64_t* my_ready = cta == 0 ? &act_ready[g] : &act_local[g];
     const uint32_t act_base = smem_u32(my_act);
     const uint32_t t_row = tmem + (uint32_t)(g * 256) + ((uint32_t)(quarter * 32) << 16);
     const int tt = et & 255;                      // thread within the tile
@@ -609,7 +604,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) mlp_tc_kernel(Params P, const __g
       if (h == 0) store_pe<0>(x[0], x[1], x[2], act_base, r);
       else store_pe<1>(x[0], x[1], x[2], act_base, r);
       fence_async_smem();
-      warp_arrive_act(my_ready, lane);
+      warp_arrive_act(&act_ready[g], cta, lane);
 
       float sigma = 0.0f;
       // A layer's epilogue vectors (all bf16 weights of the blob, so the bf16
@@ -647,7 +642,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) mlp_tc_kernel(Params P, const __g
           else epi_half<true, false>(t_row, c0, sb0, sb1, act_base, r, sigma);
           tc_fence_before();
           fence_async_smem();
-          warp_arrive_act(my_ready, lane);
+          warp_arrive_act(&act_ready[g], cta, lane);
           if (tile_sync_or(g, !waited || *abort_flag)) { stop = true; break; }
           stage_vectors(l + 1);
           tile_sync(g);

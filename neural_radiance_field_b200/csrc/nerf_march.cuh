@@ -36,6 +36,39 @@ __device__ __forceinline__ void march_point(const float* o, const float* d, int6
   for (int c = 0; c < 3; ++c) x[c] = fadd(o[r * 3 + c], fmul(*t, d[r * 3 + c]));
 }
 
+// Candidates [*klo, *khi] of ray r that can lie in [-1.5, 1.5)^3; every other
+// candidate's point is outside it, so the exact test above would reject it. The
+// interval comes from the slabs of the cube expanded by 1e-4 on every side (far
+// more than the fp32 error of a point, about 1e-6 here), in fp32, padded by one
+// candidate on each end. Empty (klo > khi) when the ray misses the box.
+__device__ __forceinline__ void march_window(const float* o, const float* d, int64_t r,
+                                             float near, float step, int K, int* klo, int* khi) {
+  constexpr float B = 1.5f + 1e-4f;
+  float tin = -INFINITY, tout = INFINITY;
+  bool miss = false;
+#pragma unroll
+  for (int c = 0; c < 3; ++c) {
+    const float oc = o[r * 3 + c], dc = d[r * 3 + c];
+    if (dc != 0.0f) {
+      const float t0 = (-B - oc) / dc, t1 = (B - oc) / dc;
+      tin = fmaxf(tin, fminf(t0, t1));
+      tout = fminf(tout, fmaxf(t0, t1));
+    } else if (!(oc >= -B && oc <= B)) {
+      miss = true;
+    }
+  }
+  if (miss || !(tin <= tout)) {
+    *klo = K;
+    *khi = -1;
+    return;
+  }
+  float a = (tin - near) / step, b = (tout - near) / step;
+  a = fminf(fmaxf(a, -2.0f), (float)K + 2.0f);      // also maps +-inf and keeps NaN out
+  b = fminf(fmaxf(b, -2.0f), (float)K + 2.0f);
+  *klo = max(0, (int)floorf(a) - 1);
+  *khi = min(K - 1, (int)ceilf(b) + 1);
+}
+
 struct HashGridInfo {
   int res[16];
   int offset[16];
