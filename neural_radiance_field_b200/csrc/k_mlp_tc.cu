@@ -48,11 +48,18 @@ constexpr int NTHREADS = 64 + EPI_THREADS;
 constexpr int VEC_BYTES = 2 * 512 * 2;              // per-tile staged epilogue vectors (bf16)
 constexpr size_t SMEM_BYTES = 2 * ACT_BYTES + NSTAGE * RING_BYTES + VEC_BYTES + 256;
 
-// Packed weight stream (bf16 chunks in consumption order) and fp32 vectors.
+// Packed weight stream and fp32 vectors. The stream is two half-streams, one
+// per CTA of the pair: half-stream c holds, in consumption order, every chunk's
+// rows [c N/2, (c + 1) N/2), so that a CTA's halves of two consecutive chunks
+// are contiguous and one bulk-tensor load fetches both. (Each load request
+// occupies an SM's copy path for about 400 cycles whatever its size, measured
+// from 4 to 32 KB, so one 8 KB request per chunk could not keep up with the
+// MMAs, which consume a chunk every 256 cycles.)
 struct TcLayout {
-  int64_t chunk_off[80];     // byte offset of every chunk in the stream
-  int chunk_bytes[80];
-  int n_chunks;
+  int64_t half_off[80];      // byte offset of a chunk's half within a half-stream
+  int half_bytes[80];        // bytes of one CTA's half of the chunk
+  int n_chunks;              // even: chunks are loaded in pairs
+  int64_t half_stream_bytes;
   int64_t stream_bytes;
   int64_t vec_off;           // byte offset of the fp32 vectors
   // fp32 vector block (element offsets inside it)
@@ -69,14 +76,15 @@ TcLayout make_layout() {
   int q = 0;
   for (int l = 0; l < NLAYER; ++l)
     for (int c = 0; c < kch[l]; ++c) {
-      L.chunk_off[q] = off;
-      L.chunk_bytes[q] = nout[l] * CHUNK_K * 2;
-      off += L.chunk_bytes[q];
+      L.half_off[q] = off;
+      L.half_bytes[q] = (nout[l] / 2) * CHUNK_K * 2;
+      off += L.half_bytes[q];
       ++q;
     }
   L.n_chunks = q;
-  L.stream_bytes = off;
-  L.vec_off = (off + 255) & ~int64_t(255);
+  L.half_stream_bytes = off;
+  L.stream_bytes = 2 * off;
+  L.vec_off = (L.stream_bytes + 255) & ~int64_t(255);   // the vectors follow both half-streams
   int v = 0;
   for (int l = 0; l < NLAYER; ++l) { L.bias[l] = v; v += 256; }
   L.w_sigma = v; v += 256;
@@ -388,7 +396,8 @@ __device__ __forceinline__ bool mma_pass(int g, uint32_t q0, uint64_t* full, uin
   constexpr uint64_t A_CHUNK = (4 * TM * 16) >> 4;
   constexpr uint64_t A_TILE = ACT_BYTES >> 4;
   constexpr uint64_t B_KSTEP = (2 * Nh * 16) >> 4;
-  constexpr uint64_t B_SLOT = RING_BYTES >> 4;
+  constexpr uint64_t B_PAIR = (2 * RING_BYTES) >> 4;     // a chunk pair's ring bytes
+  constexpr uint64_t B_HALF = (Nh * CHUNK_K * 2) >> 4;   // one chunk's half within the pair
   const uint64_t b0 = (b_desc & ~(0x3FFFull << 16)) | ((uint64_t)((Nh * 16) >> 4) << 16);
   const uint64_t a0 = a_desc + (uint64_t)g * A_TILE + (uint64_t)((KG0 * TM * 16) >> 4);
   const uint32_t td = tmem + (uint32_t)g * 256;
@@ -396,11 +405,11 @@ __device__ __forceinline__ bool mma_pass(int g, uint32_t q0, uint64_t* full, uin
   for (int c = C0; c < C1; ++c) {
     const uint32_t q = q0 + (uint32_t)c;
     const uint32_t slot = q & (NSTAGE - 1);
-    if (FIRST_USE) {
+    if (FIRST_USE && (q & 1) == 0) {     // a pair lands together (counted on its first slot)
       if (!mbar_wait_cl(&full[slot], (q / NSTAGE) & 1, ctl)) return false;
       tc_fence_after();
     }
-    const uint64_t b = b0 + slot * B_SLOT;
+    const uint64_t b = b0 + ((q >> 1) & (NSTAGE / 2 - 1)) * B_PAIR + (q & 1) * B_HALF;
     const uint64_t a = a0 + (uint64_t)c * A_CHUNK;
     mma_bf16_pair(td, a, b, idesc, c != 0);
     mma_bf16_pair(td, a + A_KSTEP, b + B_KSTEP, idesc, 1);
@@ -464,8 +473,8 @@ __device__ __forceinline__ bool mma_layer_pingpong(uint32_t& q, uint32_t (&ph_ac
   return true;
 }
 
-__global__ void __launch_bounds__(NTHREADS, 1) mlp_tc_kernel(Params P, const __grid_constant__ CUtensorMap tmap_h64,
-              const __grid_constant__ CUtensorMap tmap_h32) {
+__global__ void __launch_bounds__(NTHREADS, 1) mlp_tc_kernel(Params P, const __grid_constant__ CUtensorMap tmap_h128,
+              const __grid_constant__ CUtensorMap tmap_h64) {
   extern __shared__ __align__(1024) uint8_t smem[];
   uint8_t* act = smem;                                   // 2 x ACT_BYTES
   uint8_t* ring = smem + 2 * ACT_BYTES;                  // NSTAGE x RING_BYTES
@@ -540,22 +549,27 @@ __global__ void __launch_bounds__(NTHREADS, 1) mlp_tc_kernel(Params P, const __g
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------- weight loader (both CTAs)
-    // Each CTA loads its half of every chunk (rows [cta * N/2, (cta + 1) * N/2)
-    // of the layer); the bytes of both halves are counted on CTA 0's barrier.
+    // Each CTA loads its halves (rows [cta * N/2, (cta + 1) * N/2) of the layer)
+    // of two consecutive chunks with one request into two consecutive ring
+    // slots; the bytes of both CTAs are counted on CTA 0's barrier of the first.
     if (lane == 0) {
       uint32_t q = 0;
       for (int64_t pr = cid; pr < P.n_pairs; pr += ncl) {
         bool ok = true;
-        for (int j = 0; j < P.lay.n_chunks; ++j, ++q) {
+        for (int j = 0; j < P.lay.n_chunks; j += 2, q += 2) {
           const int slot = q % NSTAGE;
-          // the slot's previous chunk has served both tiles
-          if (!mbar_wait_cl(&empty[slot], ((q / NSTAGE) & 1) ^ 1, ctl)) { ok = false; break; }
-          const uint32_t bytes = (uint32_t)P.lay.chunk_bytes[j];        // both halves
-          const int64_t half_off = P.lay.chunk_off[j] + (int64_t)cta * (bytes / 2);
-          if (cta == 0) mbar_arrive_tx(&full[slot], bytes);
-          tma_load_2d_pair(ring + slot * RING_BYTES, bytes == 2 * 8192 ? (const void*)&tmap_h64
-                                                                       : (const void*)&tmap_h32,
-                           0, (int)(half_off / 128), &full[slot]);
+          // both slots' previous chunks have served both tiles
+          const uint32_t par = ((q / NSTAGE) & 1) ^ 1;
+          if (!mbar_wait_cl(&empty[slot], par, ctl) || !mbar_wait_cl(&empty[slot + 1], par, ctl)) {
+            ok = false;
+            break;
+          }
+          const uint32_t pair_bytes = (uint32_t)(P.lay.half_bytes[j] + P.lay.half_bytes[j + 1]);
+          const int64_t off = (int64_t)cta * P.lay.half_stream_bytes + P.lay.half_off[j];
+          if (cta == 0) mbar_arrive_tx(&full[slot], 2 * pair_bytes);
+          tma_load_2d_pair(ring + slot * RING_BYTES,
+                           pair_bytes == 2 * RING_BYTES ? (const void*)&tmap_h128 : (const void*)&tmap_h64,
+                           0, (int)(off / 128), &full[slot]);
         }
         if (!ok) break;
       }
@@ -756,7 +770,7 @@ __global__ void tc_pack_kernel(const __nv_bfloat16* __restrict__ blob, PackPlan 
     __nv_bfloat16 v = k < pl.K_src ? blob[pl.src_w + (int64_t)n * pl.K_src + k]
                                    : __float2bfloat16(0.0f);
     const int hh = n / Nh, nn = n % Nh;
-    const int64_t byte = lay.chunk_off[pl.chunk0 + c] + (int64_t)hh * (Nh * CHUNK_K * 2) +
+    const int64_t byte = (int64_t)hh * lay.half_stream_bytes + lay.half_off[pl.chunk0 + c] +
                          (kl >> 3) * (Nh * 16) + (nn >> 3) * 128 + (nn & 7) * 16 + (kl & 7) * 2;
     dst[byte / 2] = v;
   }
@@ -782,8 +796,8 @@ struct TcState {
   TcLayout lay;
   PackPlan plan;
   uint8_t* buf = nullptr;
-  CUtensorMap tmap_h64;     // the stream as rows of 128 B, boxes of 64 rows (8 KB halves)
-  CUtensorMap tmap_h32;     // boxes of 32 rows (4 KB halves of the direction layer)
+  CUtensorMap tmap_h128;    // the stream as rows of 128 B, boxes of 128 rows (16 KB: two 8 KB halves)
+  CUtensorMap tmap_h64;     // boxes of 64 rows (two 4 KB halves of the direction layer)
   int max_clusters = 0;     // co-resident CTA pairs of the kernel on this device
 };
 
@@ -837,9 +851,11 @@ cudaError_t tc_alloc(nerf_ctx* ctx) {
   off += (int64_t)(W / 2) * (W + dir_ch) + W / 2;
   s->plan.rgb_w = off; off += 3 * (W / 2);
   s->plan.rgb_b = off;
+  // the packed stream (both half-streams) and then the vectors, inside one allocation
+  if (s->lay.vec_off < s->lay.stream_bytes || s->lay.n_chunks % 2 != 0) { delete s; return cudaErrorInvalidValue; }
   cudaError_t e = cudaMalloc(&s->buf, s->lay.vec_off + s->lay.vec_count * sizeof(float));
+  if (e == cudaSuccess) e = make_stream_map(&s->tmap_h128, s->buf, s->lay.stream_bytes, 128);
   if (e == cudaSuccess) e = make_stream_map(&s->tmap_h64, s->buf, s->lay.stream_bytes, 64);
-  if (e == cudaSuccess) e = make_stream_map(&s->tmap_h32, s->buf, s->lay.stream_bytes, 32);
   if (e != cudaSuccess) { cudaFree(s->buf); delete s; return e; }
   int dev = 0;
   cudaGetDevice(&dev);
@@ -914,7 +930,7 @@ cudaError_t tc_run(nerf_ctx* ctx, const float* o, const float* d, int64_t R, con
   }
   const int64_t clusters = P.n_pairs < s->max_clusters ? P.n_pairs : s->max_clusters;
   cfg.gridDim = dim3((unsigned)(2 * clusters));
-  return cudaLaunchKernelEx(&cfg, mlp_tc_kernel, P, s->tmap_h64, s->tmap_h32);
+  return cudaLaunchKernelEx(&cfg, mlp_tc_kernel, P, s->tmap_h128, s->tmap_h64);
 }
 
 }  // namespace nerfb
