@@ -358,32 +358,44 @@ __device__ __forceinline__ void tma_load_2d_pair(void* dst, const void* tmap, in
 }
 
 
+// The MMA warp runs its loop converged (all 32 lanes: warp-uniform operands and
+// control), and lane 0 alone issues each tcgen05 instruction, predicated inside
+// the asm. The converged issue loop is 8 % faster than one lane running it
+// alone (measured on the 8 x 256 network).
 __device__ __forceinline__ void mma_bf16_pair(uint32_t tmem_d, uint64_t a, uint64_t b,
                                               uint32_t idesc, uint32_t accum) {
   asm volatile(
-      "{\n\t.reg .pred p;\n\t"
+      "{\n\t.reg .pred p, e;\n\t.reg .b32 ln;\n\t"
+      "mov.u32 ln, %%laneid;\n\t"
+      "setp.eq.u32 e, ln, 0;\n\t"
       "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}"
+      "@e tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}"
       ::"r"(tmem_d), "l"(a), "l"(b), "r"(idesc), "r"(accum));
 }
 
 // Arrive (once each) on the barrier at this offset in both CTAs of the pair
-// when every previously issued MMA of this thread has completed.
+// when every MMA previously issued by lane 0 of the calling warp has completed
+// (lane 0 issues the commit).
 __device__ __forceinline__ void mma_commit_pair(uint64_t* bar) {
   asm volatile(
-      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
-      " [%0], %1;"
+      "{\n\t.reg .pred e;\n\t.reg .b32 ln;\n\t"
+      "mov.u32 ln, %%laneid;\n\t"
+      "setp.eq.u32 e, ln, 0;\n\t"
+      "@e tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
+      " [%0], %1;\n\t}"
       ::"r"(smem_u32(bar)), "h"((uint16_t)3)
       : "memory");
 }
 
 // MMAs of tile g over chunks [C0, C1) of one layer, issued by CTA 0's MMA
-// thread. Every weight chunk serves both tiles: tile A's pass is its first
+// warp. Every weight chunk serves both tiles: tile A's pass is its first
 // use (it waits for the chunk to land), tile B's pass its second (it releases
-// the ring slot). A 2-SM MMA (M = 256, N = 256, K = 16) takes 128 cycles on
-// the tensor pipe and a chunk holds two, so the thread's work per chunk must
+// the ring slots). A 2-SM MMA (M = 256, N = 256, K = 16) takes 128 cycles on
+// the tensor pipe and a chunk holds two, so the warp's work per chunk must
 // stay well under 256 cycles: shapes and the instruction descriptor are
-// compile-time constants and operand descriptors advance by additions.
+// compile-time constants and operand descriptors advance by additions (the
+// loop is unrolled by two: unrolled by four or fully, it measured 15-20 %
+// slower).
 //   N: output width; KG0: first K-group of the A operand
 template <int N, int KG0, int C0, int C1, bool FIRST_USE>
 __device__ __forceinline__ bool mma_pass(int g, uint32_t q0, uint64_t* full, uint64_t* empty,
@@ -413,14 +425,16 @@ __device__ __forceinline__ bool mma_pass(int g, uint32_t q0, uint64_t* full, uin
     const uint64_t a = a0 + (uint64_t)c * A_CHUNK;
     mma_bf16_pair(td, a, b, idesc, c != 0);
     mma_bf16_pair(td, a + A_KSTEP, b + B_KSTEP, idesc, 1);
-    if (!FIRST_USE) mma_commit_pair(&empty[slot]);
+    // the ring is refilled a chunk pair at a time: the second use of a pair's
+    // second chunk releases both of its slots (MMAs complete in issue order)
+    if (!FIRST_USE && (q & 1)) mma_commit_pair(&empty[slot]);
   }
   return true;
 }
 
-// The epilogue's hand-off to the MMA thread: every lane has made its stores
+// The epilogue's hand-off to the MMA warp: every lane has made its stores
 // visible to the async proxy; after the warp converges, one lane arrives on the
-// MMA thread's barrier in CTA 0 (remotely from CTA 1, with the restricted
+// MMA warp's barrier in CTA 0 (remotely from CTA 1, with the restricted
 // release fence of mbar_arrive_leader). 256 per-thread arrivals on one barrier
 // would serialize; 8 per CTA do not.
 __device__ __forceinline__ void warp_arrive_act(uint64_t* bar, uint32_t cta, int lane) {
@@ -519,7 +533,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) mlp_tc_kernel(Params P, const __g
 
   if (warp == 0) {
     // ---------------------------------------------------------- MMA issuer (CTA 0)
-    if (lane == 0 && cta == 0) {
+    if (cta == 0) {
       uint32_t q = 0, ph_act[2] = {0, 0};
       bool ok = true;
       const uint64_t a_desc = sdesc(smem_u32(act), TM * 16, 128);
@@ -552,7 +566,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) mlp_tc_kernel(Params P, const __g
     // Each CTA loads its halves (rows [cta * N/2, (cta + 1) * N/2) of the layer)
     // of two consecutive chunks with one request into two consecutive ring
     // slots; the bytes of both CTAs are counted on CTA 0's barrier of the first.
-    if (lane == 0) {
+    // The warp runs the loop converged; lane 0 issues the requests.
+    {
       uint32_t q = 0;
       for (int64_t pr = cid; pr < P.n_pairs; pr += ncl) {
         bool ok = true;
@@ -560,16 +575,19 @@ __global__ void __launch_bounds__(NTHREADS, 1) mlp_tc_kernel(Params P, const __g
           const int slot = q % NSTAGE;
           // both slots' previous chunks have served both tiles
           const uint32_t par = ((q / NSTAGE) & 1) ^ 1;
-          if (!mbar_wait_cl(&empty[slot], par, ctl) || !mbar_wait_cl(&empty[slot + 1], par, ctl)) {
+          if (!mbar_wait_cl(&empty[slot + 1], par, ctl)) {
             ok = false;
             break;
           }
           const uint32_t pair_bytes = (uint32_t)(P.lay.half_bytes[j] + P.lay.half_bytes[j + 1]);
           const int64_t off = (int64_t)cta * P.lay.half_stream_bytes + P.lay.half_off[j];
-          if (cta == 0) mbar_arrive_tx(&full[slot], 2 * pair_bytes);
-          tma_load_2d_pair(ring + slot * RING_BYTES,
-                           pair_bytes == 2 * RING_BYTES ? (const void*)&tmap_h128 : (const void*)&tmap_h64,
-                           0, (int)(off / 128), &full[slot]);
+          if (lane == 0) {
+            if (cta == 0) mbar_arrive_tx(&full[slot], 2 * pair_bytes);
+            tma_load_2d_pair(ring + slot * RING_BYTES,
+                             pair_bytes == 2 * RING_BYTES ? (const void*)&tmap_h128 : (const void*)&tmap_h64,
+                             0, (int)(off / 128), &full[slot]);
+          }
+          __syncwarp();
         }
         if (!ok) break;
       }
