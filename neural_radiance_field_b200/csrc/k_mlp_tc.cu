@@ -39,8 +39,11 @@ constexpr int TM = 128;
 constexpr int ACT_K = 320;
 constexpr int ACT_BYTES = TM * ACT_K * 2;           // 81920
 constexpr int CHUNK_K = 32;
-constexpr int NSTAGE = 8;
+constexpr int NSTAGE = 8;                           // ring slots (chunks)
 constexpr int RING_BYTES = 128 * CHUNK_K * 2;       // 8192: one CTA's half of a chunk
+constexpr int UNIT_CHUNKS = 4;                      // chunks per load and per barrier
+constexpr int NGROUP = NSTAGE / UNIT_CHUNKS;        // slot groups, one unit each
+constexpr int GROUP_BYTES = UNIT_CHUNKS * RING_BYTES;
 constexpr int NLAYER = 10;                          // pts0..pts7, feature, dir
 constexpr int EPI_THREADS = 512;                    // 16 epilogue warps
 constexpr int TILE_THREADS = 256;                   // epilogue threads per tile
@@ -50,15 +53,20 @@ constexpr size_t SMEM_BYTES = 2 * ACT_BYTES + NSTAGE * RING_BYTES + VEC_BYTES + 
 
 // Packed weight stream and fp32 vectors. The stream is two half-streams, one
 // per CTA of the pair: half-stream c holds, in consumption order, every chunk's
-// rows [c N/2, (c + 1) N/2), so that a CTA's halves of two consecutive chunks
-// are contiguous and one bulk-tensor load fetches both. (Each load request
-// occupies an SM's copy path for about 400 cycles whatever its size, measured
-// from 4 to 32 KB, so one 8 KB request per chunk could not keep up with the
-// MMAs, which consume a chunk every 256 cycles.)
+// rows [c N/2, (c + 1) N/2), so that a CTA's halves of consecutive chunks are
+// contiguous. The chunks of a layer travel in units of four (the last unit of
+// a layer may hold two): one bulk-tensor load per CTA and unit; in the MMA
+// warp, one barrier wait (first tile) or slot release (second tile) per unit
+// around the unit's eight MMAs, which are issued back to back in straight-line
+// code. (Measured on the 8 x 256 network: units of two 0.5 % slower; a loop
+// with runtime slot arithmetic between the MMAs 5 % slower.)
 struct TcLayout {
   int64_t half_off[80];      // byte offset of a chunk's half within a half-stream
   int half_bytes[80];        // bytes of one CTA's half of the chunk
-  int n_chunks;              // even: chunks are loaded in pairs
+  int n_chunks;
+  int n_units;               // load units of one pass over the network
+  int unit_chunk0[40];       // first chunk of each unit
+  int unit_bytes[40];        // bytes of one CTA's half of each unit (a full or a half group)
   int64_t half_stream_bytes;
   int64_t stream_bytes;
   int64_t vec_off;           // byte offset of the fp32 vectors
@@ -74,14 +82,22 @@ TcLayout make_layout() {
   const int nout[NLAYER] = {256, 256, 256, 256, 256, 256, 256, 256, 256, 128};
   int64_t off = 0;
   int q = 0;
+  int u = 0;
   for (int l = 0; l < NLAYER; ++l)
     for (int c = 0; c < kch[l]; ++c) {
+      if (c % UNIT_CHUNKS == 0) {          // units of four within the layer, the rest last
+        L.unit_chunk0[u] = q;
+        L.unit_bytes[u] = 0;
+        ++u;
+      }
       L.half_off[q] = off;
       L.half_bytes[q] = (nout[l] / 2) * CHUNK_K * 2;
+      L.unit_bytes[u - 1] += L.half_bytes[q];
       off += L.half_bytes[q];
       ++q;
     }
   L.n_chunks = q;
+  L.n_units = u;
   L.half_stream_bytes = off;
   L.stream_bytes = 2 * off;
   L.vec_off = (L.stream_bytes + 255) & ~int64_t(255);   // the vectors follow both half-streams
@@ -387,20 +403,15 @@ __device__ __forceinline__ void mma_commit_pair(uint64_t* bar) {
       : "memory");
 }
 
-// MMAs of tile g over chunks [C0, C1) of one layer, issued by CTA 0's MMA
-// warp. Every weight chunk serves both tiles: tile A's pass is its first
-// use (it waits for the chunk to land), tile B's pass its second (it releases
-// the ring slots). A 2-SM MMA (M = 256, N = 256, K = 16) takes 128 cycles on
-// the tensor pipe and a chunk holds two, so the warp's work per chunk must
-// stay well under 256 cycles: shapes and the instruction descriptor are
-// compile-time constants and operand descriptors advance by additions (the
-// loop is unrolled by two: unrolled by four or fully, it measured 15-20 %
-// slower).
+// The MMAs of tile g over one unit of a layer, chunks [C0, C0 + NC), held by
+// slot group grp of the ring, issued back to back by CTA 0's MMA warp: a 2-SM
+// MMA (M = 256, N = 256, K = 16) takes 128 cycles on the tensor pipe, and the
+// unit's 2 NC MMAs run without a barrier operation or loop overhead between
+// them (shapes, offsets and the accumulate flags are compile-time constants).
 //   N: output width; KG0: first K-group of the A operand
-template <int N, int KG0, int C0, int C1, bool FIRST_USE>
-__device__ __forceinline__ bool mma_pass(int g, uint32_t q0, uint64_t* full, uint64_t* empty,
-                                         uint64_t a_desc, uint64_t b_desc, uint32_t tmem,
-                                         const Ctl& ctl) {
+template <int N, int KG0, int C0, int NC>
+__device__ __forceinline__ void mma_unit(int g, uint32_t grp, uint64_t a_desc, uint64_t b_desc,
+                                         uint32_t tmem) {
   constexpr int Nh = N / 2;                 // rows of B held by each CTA
   constexpr uint32_t idesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) |
                              (16u << 24);   // M = 256
@@ -408,28 +419,18 @@ __device__ __forceinline__ bool mma_pass(int g, uint32_t q0, uint64_t* full, uin
   constexpr uint64_t A_CHUNK = (4 * TM * 16) >> 4;
   constexpr uint64_t A_TILE = ACT_BYTES >> 4;
   constexpr uint64_t B_KSTEP = (2 * Nh * 16) >> 4;
-  constexpr uint64_t B_PAIR = (2 * RING_BYTES) >> 4;     // a chunk pair's ring bytes
-  constexpr uint64_t B_HALF = (Nh * CHUNK_K * 2) >> 4;   // one chunk's half within the pair
-  const uint64_t b0 = (b_desc & ~(0x3FFFull << 16)) | ((uint64_t)((Nh * 16) >> 4) << 16);
-  const uint64_t a0 = a_desc + (uint64_t)g * A_TILE + (uint64_t)((KG0 * TM * 16) >> 4);
+  constexpr uint64_t B_CHUNK = (Nh * CHUNK_K * 2) >> 4;   // one chunk's half, packed in the unit
+  constexpr uint64_t B_GROUP = GROUP_BYTES >> 4;
+  const uint64_t b0 = ((b_desc & ~(0x3FFFull << 16)) | ((uint64_t)((Nh * 16) >> 4) << 16)) +
+                      (uint64_t)grp * B_GROUP;
+  const uint64_t a0 = a_desc + (uint64_t)g * A_TILE + (uint64_t)((KG0 * TM * 16) >> 4) +
+                      (uint64_t)C0 * A_CHUNK;
   const uint32_t td = tmem + (uint32_t)g * 256;
-#pragma unroll 2
-  for (int c = C0; c < C1; ++c) {
-    const uint32_t q = q0 + (uint32_t)c;
-    const uint32_t slot = q & (NSTAGE - 1);
-    if (FIRST_USE && (q & 1) == 0) {     // a pair lands together (counted on its first slot)
-      if (!mbar_wait_cl(&full[slot], (q / NSTAGE) & 1, ctl)) return false;
-      tc_fence_after();
-    }
-    const uint64_t b = b0 + ((q >> 1) & (NSTAGE / 2 - 1)) * B_PAIR + (q & 1) * B_HALF;
-    const uint64_t a = a0 + (uint64_t)c * A_CHUNK;
-    mma_bf16_pair(td, a, b, idesc, c != 0);
-    mma_bf16_pair(td, a + A_KSTEP, b + B_KSTEP, idesc, 1);
-    // the ring is refilled a chunk pair at a time: the second use of a pair's
-    // second chunk releases both of its slots (MMAs complete in issue order)
-    if (!FIRST_USE && (q & 1)) mma_commit_pair(&empty[slot]);
+#pragma unroll
+  for (int c = 0; c < NC; ++c) {
+    mma_bf16_pair(td, a0 + c * A_CHUNK, b0 + c * B_CHUNK, idesc, C0 + c != 0);
+    mma_bf16_pair(td, a0 + c * A_CHUNK + A_KSTEP, b0 + c * B_CHUNK + B_KSTEP, idesc, 1);
   }
-  return true;
 }
 
 // The epilogue's hand-off to the MMA warp: every lane has made its stores
@@ -453,53 +454,74 @@ __device__ __forceinline__ bool wait_act(int g, uint32_t (&ph_act)[2], uint64_t*
   return true;
 }
 
-// One layer of both tiles, tile A first (A0 B0 A1 B1 ...): while one tile's
-// accumulator is drained by its epilogue, the other tile's layer runs. The
-// ring holds 8 chunks, one layer; the 10-chunk skip layer runs as A[0..7]
-// B[0..7] A[8, 9] B[8, 9], so that its last two chunks can reuse the slots
-// that tile B has released.
+// Units [K, KEND) of one layer for tile g, in straight-line code: tile A's
+// pass (FIRST) waits for each unit to land before its MMAs, tile B's pass
+// releases each unit's slots after its MMAs. Unit U + K of the kernel sits in
+// slot group (U + K) % NGROUP, whose barriers complete once per unit.
+template <int N, int KG0, int NCH, int K, int KEND, bool FIRST>
+__device__ __forceinline__ bool mma_units(int g, uint32_t U, uint64_t* full, uint64_t* empty,
+                                          uint64_t a_desc, uint64_t b_desc, uint32_t tmem,
+                                          const Ctl& ctl) {
+  if constexpr (K < KEND) {
+    constexpr int C0 = K * UNIT_CHUNKS;
+    constexpr int NC = NCH - C0 < UNIT_CHUNKS ? NCH - C0 : UNIT_CHUNKS;
+    const uint32_t u = U + K, grp = u % NGROUP;
+    if (FIRST) {
+      if (!mbar_wait_cl(&full[grp], (u / NGROUP) & 1, ctl)) return false;
+      tc_fence_after();
+    }
+    mma_unit<N, KG0, C0, NC>(g, grp, a_desc, b_desc, tmem);
+    if (!FIRST) mma_commit_pair(&empty[grp]);
+    return mma_units<N, KG0, NCH, K + 1, KEND, FIRST>(g, U, full, empty, a_desc, b_desc, tmem, ctl);
+  } else {
+    return true;
+  }
+}
+
+// One layer of both tiles, tile A first: while one tile's accumulator is
+// drained by its epilogue, the other tile's layer runs. Every unit serves both
+// tiles. The ring holds one 8-chunk layer; the 10-chunk skip layer runs as
+// A[0..7] B[0..7] A[8, 9] B[8, 9], its last unit reusing the slots that tile B
+// has released. U counts the units of the kernel.
 template <int N, int KG0, int NCH>
-__device__ __forceinline__ bool mma_layer_pingpong(uint32_t& q, uint32_t (&ph_act)[2],
+__device__ __forceinline__ bool mma_layer_pingpong(uint32_t& U, uint32_t (&ph_act)[2],
                                                    uint64_t* full, uint64_t* empty,
                                                    uint64_t* mma_done, uint64_t* act_ready,
                                                    uint64_t a_desc, uint64_t b_desc,
                                                    uint32_t tmem, const Ctl& ctl) {
-  static_assert(NCH <= NSTAGE || NCH == NSTAGE + 2, "chunk schedule");
-  constexpr int CA = NCH <= NSTAGE ? NCH : NSTAGE;
+  constexpr int NU = (NCH + UNIT_CHUNKS - 1) / UNIT_CHUNKS;
+  constexpr int NA = NU < NGROUP ? NU : NGROUP;          // units of the first round
+  static_assert(NU <= NA + NGROUP && NCH - NA * UNIT_CHUNKS <= NSTAGE, "unit schedule");
   if (!wait_act(0, ph_act, act_ready, ctl) ||
-      !mma_pass<N, KG0, 0, CA, true>(0, q, full, empty, a_desc, b_desc, tmem, ctl))
+      !mma_units<N, KG0, NCH, 0, NA, true>(0, U, full, empty, a_desc, b_desc, tmem, ctl))
     return false;
-  if (NCH == CA) mma_commit_pair(&mma_done[0]);
-  if (!wait_act(1, ph_act, act_ready, ctl) ||
-      !mma_pass<N, KG0, 0, CA, false>(1, q, full, empty, a_desc, b_desc, tmem, ctl))
-    return false;
-  if (NCH == CA) {
-    mma_commit_pair(&mma_done[1]);
-  } else {
-    if (!mma_pass<N, KG0, CA, NCH, true>(0, q, full, empty, a_desc, b_desc, tmem, ctl))
+  if (NU == NA) mma_commit_pair(&mma_done[0]);
+  if (!wait_act(1, ph_act, act_ready, ctl)) return false;
+  mma_units<N, KG0, NCH, 0, NA, false>(1, U, full, empty, a_desc, b_desc, tmem, ctl);
+  if (NU > NA) {
+    if (!mma_units<N, KG0, NCH, NA, NU, true>(0, U, full, empty, a_desc, b_desc, tmem, ctl))
       return false;
     mma_commit_pair(&mma_done[0]);
-    if (!mma_pass<N, KG0, CA, NCH, false>(1, q, full, empty, a_desc, b_desc, tmem, ctl))
-      return false;
-    mma_commit_pair(&mma_done[1]);
+    mma_units<N, KG0, NCH, NA, NU, false>(1, U, full, empty, a_desc, b_desc, tmem, ctl);
   }
-  q += NCH;
+  mma_commit_pair(&mma_done[1]);
+  U += NU;
   return true;
 }
 
-__global__ void __launch_bounds__(NTHREADS, 1) mlp_tc_kernel(Params P, const __grid_constant__ CUtensorMap tmap_h128,
-              const __grid_constant__ CUtensorMap tmap_h64) {
+__global__ void __launch_bounds__(NTHREADS, 1) mlp_tc_kernel(Params P, const __grid_constant__ CUtensorMap tmap_unit,
+              const __grid_constant__ CUtensorMap tmap_half) {
   extern __shared__ __align__(1024) uint8_t smem[];
   uint8_t* act = smem;                                   // 2 x ACT_BYTES
   uint8_t* ring = smem + 2 * ACT_BYTES;                  // NSTAGE x RING_BYTES
   uint16_t* svec = reinterpret_cast<uint16_t*>(ring + NSTAGE * RING_BYTES);  // 2 tiles x 512 bf16
   uint64_t* bars = reinterpret_cast<uint64_t*>(ring + NSTAGE * RING_BYTES + VEC_BYTES);
-  uint64_t* full = bars;                 // [NSTAGE] (used in CTA 0)
-  uint64_t* empty = bars + NSTAGE;       // [NSTAGE]
-  uint64_t* mma_done = bars + 2 * NSTAGE;     // [2]
-  uint64_t* act_ready = bars + 2 * NSTAGE + 2;  // [2] (used in CTA 0)
-  uint64_t* final_bar = bars + 2 * NSTAGE + 4;
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 2 * NSTAGE + 5);
+  uint64_t* full = bars;                 // [NGROUP] (used in CTA 0)
+  uint64_t* empty = bars + NGROUP;       // [NGROUP]
+  uint64_t* mma_done = bars + 2 * NGROUP;     // [2]
+  uint64_t* act_ready = bars + 2 * NGROUP + 2;  // [2] (used in CTA 0)
+  uint64_t* final_bar = bars + 2 * NGROUP + 4;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 2 * NGROUP + 5);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
   const int warp = threadIdx.x >> 5;
@@ -509,7 +531,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) mlp_tc_kernel(Params P, const __g
   Ctl ctl{abort_flag, P.flag, kWaitLimitNs};
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < NSTAGE; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
+    for (int s = 0; s < NGROUP; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
     for (int g = 0; g < 2; ++g) {
       mbar_init(&mma_done[g], 1);
       mbar_init(&act_ready[g], 2 * TILE_THREADS / 32);   // one arrival per epilogue warp
@@ -534,19 +556,24 @@ __global__ void __launch_bounds__(NTHREADS, 1) mlp_tc_kernel(Params P, const __g
   if (warp == 0) {
     // ---------------------------------------------------------- MMA issuer (CTA 0)
     if (cta == 0) {
-      uint32_t q = 0, ph_act[2] = {0, 0};
+      uint32_t U = 0, ph_act[2] = {0, 0};
       bool ok = true;
       const uint64_t a_desc = sdesc(smem_u32(act), TM * 16, 128);
       const uint64_t b_desc = sdesc(smem_u32(ring), 0, 128);
 #define NERF_PP_LAYER(N, KG0, NCH) \
-  mma_layer_pingpong<N, KG0, NCH>(q, ph_act, full, empty, mma_done, act_ready, a_desc, b_desc, tmem, ctl)
+  mma_layer_pingpong<N, KG0, NCH>(U, ph_act, full, empty, mma_done, act_ready, a_desc, b_desc, tmem, ctl)
       for (int64_t pr = cid; pr < P.n_pairs && ok; pr += ncl) {
         // layer shapes: pts0 (K = 63 -> 64, from the gamma columns), pts1..4,
-        // pts5 (skip: K = 256 + 64), pts6, pts7, feature, direction (N = 128)
-        ok = NERF_PP_LAYER(256, 32, 2) && NERF_PP_LAYER(256, 0, 8) && NERF_PP_LAYER(256, 0, 8) &&
-             NERF_PP_LAYER(256, 0, 8) && NERF_PP_LAYER(256, 0, 8) && NERF_PP_LAYER(256, 0, 10) &&
-             NERF_PP_LAYER(256, 0, 8) && NERF_PP_LAYER(256, 0, 8) && NERF_PP_LAYER(256, 0, 8) &&
-             NERF_PP_LAYER(128, 0, 8);
+        // pts5 (skip: K = 256 + 64), pts6, pts7, feature, direction (N = 128).
+        // One copy of the code per shape: the MMA warp's code stays small enough
+        // for the instruction cache (ten inlined copies measured 16 % slower).
+#pragma unroll 1
+        for (int l = 0; l < NLAYER && ok; ++l) {
+          if (l == 0) ok = NERF_PP_LAYER(256, 32, 2);
+          else if (l == 5) ok = NERF_PP_LAYER(256, 0, 10);
+          else if (l == 9) ok = NERF_PP_LAYER(128, 0, 8);
+          else ok = NERF_PP_LAYER(256, 0, 8);
+        }
       }
 #undef NERF_PP_LAYER
       // drain: everything issued so far completes before the pair frees TMEM.
@@ -564,28 +591,27 @@ __global__ void __launch_bounds__(NTHREADS, 1) mlp_tc_kernel(Params P, const __g
   } else if (warp == 1) {
     // ---------------------------------------------------------- weight loader (both CTAs)
     // Each CTA loads its halves (rows [cta * N/2, (cta + 1) * N/2) of the layer)
-    // of two consecutive chunks with one request into two consecutive ring
-    // slots; the bytes of both CTAs are counted on CTA 0's barrier of the first.
-    // The warp runs the loop converged; lane 0 issues the requests.
+    // of a unit's chunks with one request into the unit's slot group; the bytes
+    // of both CTAs are counted on CTA 0's barrier of the group. The warp runs
+    // the loop converged; lane 0 issues the requests.
     {
-      uint32_t q = 0;
+      uint32_t U = 0;
       for (int64_t pr = cid; pr < P.n_pairs; pr += ncl) {
         bool ok = true;
-        for (int j = 0; j < P.lay.n_chunks; j += 2, q += 2) {
-          const int slot = q % NSTAGE;
-          // both slots' previous chunks have served both tiles
-          const uint32_t par = ((q / NSTAGE) & 1) ^ 1;
-          if (!mbar_wait_cl(&empty[slot + 1], par, ctl)) {
+        for (int u = 0; u < P.lay.n_units; ++u, ++U) {
+          const uint32_t grp = U % NGROUP;
+          // the group's previous unit has served both tiles
+          if (!mbar_wait_cl(&empty[grp], ((U / NGROUP) & 1) ^ 1, ctl)) {
             ok = false;
             break;
           }
-          const uint32_t pair_bytes = (uint32_t)(P.lay.half_bytes[j] + P.lay.half_bytes[j + 1]);
-          const int64_t off = (int64_t)cta * P.lay.half_stream_bytes + P.lay.half_off[j];
+          const uint32_t bytes = (uint32_t)P.lay.unit_bytes[u];
+          const int64_t off = (int64_t)cta * P.lay.half_stream_bytes + P.lay.half_off[P.lay.unit_chunk0[u]];
           if (lane == 0) {
-            if (cta == 0) mbar_arrive_tx(&full[slot], 2 * pair_bytes);
-            tma_load_2d_pair(ring + slot * RING_BYTES,
-                             pair_bytes == 2 * RING_BYTES ? (const void*)&tmap_h128 : (const void*)&tmap_h64,
-                             0, (int)(off / 128), &full[slot]);
+            if (cta == 0) mbar_arrive_tx(&full[grp], 2 * bytes);
+            tma_load_2d_pair(ring + grp * GROUP_BYTES,
+                             bytes == GROUP_BYTES ? (const void*)&tmap_unit : (const void*)&tmap_half,
+                             0, (int)(off / 128), &full[grp]);
           }
           __syncwarp();
         }
@@ -814,8 +840,8 @@ struct TcState {
   TcLayout lay;
   PackPlan plan;
   uint8_t* buf = nullptr;
-  CUtensorMap tmap_h128;    // the stream as rows of 128 B, boxes of 128 rows (16 KB: two 8 KB halves)
-  CUtensorMap tmap_h64;     // boxes of 64 rows (two 4 KB halves of the direction layer)
+  CUtensorMap tmap_unit;    // the stream as rows of 128 B, boxes of one unit's half (GROUP_BYTES)
+  CUtensorMap tmap_half;    // boxes of half of that (the direction layer's units)
   int max_clusters = 0;     // co-resident CTA pairs of the kernel on this device
 };
 
@@ -870,10 +896,13 @@ cudaError_t tc_alloc(nerf_ctx* ctx) {
   s->plan.rgb_w = off; off += 3 * (W / 2);
   s->plan.rgb_b = off;
   // the packed stream (both half-streams) and then the vectors, inside one allocation
-  if (s->lay.vec_off < s->lay.stream_bytes || s->lay.n_chunks % 2 != 0) { delete s; return cudaErrorInvalidValue; }
+  bool units_ok = s->lay.n_units <= 40;
+  for (int u = 0; u < s->lay.n_units && units_ok; ++u)
+    units_ok = s->lay.unit_bytes[u] == GROUP_BYTES || s->lay.unit_bytes[u] == GROUP_BYTES / 2;
+  if (s->lay.vec_off < s->lay.stream_bytes || !units_ok) { delete s; return cudaErrorInvalidValue; }
   cudaError_t e = cudaMalloc(&s->buf, s->lay.vec_off + s->lay.vec_count * sizeof(float));
-  if (e == cudaSuccess) e = make_stream_map(&s->tmap_h128, s->buf, s->lay.stream_bytes, 128);
-  if (e == cudaSuccess) e = make_stream_map(&s->tmap_h64, s->buf, s->lay.stream_bytes, 64);
+  if (e == cudaSuccess) e = make_stream_map(&s->tmap_unit, s->buf, s->lay.stream_bytes, GROUP_BYTES / 128);
+  if (e == cudaSuccess) e = make_stream_map(&s->tmap_half, s->buf, s->lay.stream_bytes, GROUP_BYTES / 256);
   if (e != cudaSuccess) { cudaFree(s->buf); delete s; return e; }
   int dev = 0;
   cudaGetDevice(&dev);
@@ -948,7 +977,7 @@ cudaError_t tc_run(nerf_ctx* ctx, const float* o, const float* d, int64_t R, con
   }
   const int64_t clusters = P.n_pairs < s->max_clusters ? P.n_pairs : s->max_clusters;
   cfg.gridDim = dim3((unsigned)(2 * clusters));
-  return cudaLaunchKernelEx(&cfg, mlp_tc_kernel, P, s->tmap_h128, s->tmap_h64);
+  return cudaLaunchKernelEx(&cfg, mlp_tc_kernel, P, s->tmap_unit, s->tmap_half);
 }
 
 }  // namespace nerfb
