@@ -903,10 +903,11 @@ def march_launches_per_step(model, R):
 
 # DRAM bytes (read + write) per MLP row of the scene-MLP kernel, from an ncu
 # capture (dram__bytes_read.sum + dram__bytes_write.sum) of the fine launch of a
-# 256x256 frame: 236.75 MB for 12,582,912 rows. The traffic is the raw output
-# and the sample positions, so it grows in proportion to the rows; it is scaled
-# to the launch size here. Re-measure whenever the kernel changes.
-TRAFFIC_B_PER_ROW = 236.75e6 / 12582912
+# 256x256 frame: 237.21 MB (87.59 MB read, 149.63 MB written) for 12,582,912
+# rows. The traffic is the raw output and the sample positions, so it grows in
+# proportion to the rows; it is scaled to the launch size here. Re-measure
+# whenever the kernel changes.
+TRAFFIC_B_PER_ROW = 237.21e6 / 12582912
 TRAFFIC_SOURCE = ("ncu dram__bytes_read.sum + dram__bytes_write.sum of the fine launch at "
                   "256x256, scaled by rows to the average launch")
 
