@@ -922,85 +922,131 @@ kilo_items_kernel(const int32_t* __restrict__ hist, const int32_t* __restrict__ 
   if (t == 1023) *n_items = sums[1023];
 }
 
-// The per-cell tiny MLPs as small fp32 GEMMs: a CTA stages one cell's 3,317
-// weights in shared memory (the layer matrices transposed, Wt[k][n]) and runs a
-// tile of that cell's points through them; activations sit k-major, and each
-// of 256 threads accumulates a 4-point x 4-output block (two 16-byte shared
-// loads per 16 FMAs). The accumulation order (bias, then k ascending) is the
-// per-point definition's.
+// The per-cell tiny MLPs, their two 32-wide layers on the tensor cores. A CTA
+// runs a tile of up to 128 points of one cell at a time (consecutive items
+// mostly share a cell, whose weights then stay staged):
+//   gamma(x) (63 -> K 64) -> 32 -> 32 : tcgen05.mma kind::tf32, M = 128, N = 32,
+//   the heads sigma (32 -> 1) and rgb ([h2, gamma(d)] 59 -> 3) : fp32 CUDA cores.
+// fp32-level accuracy from tf32 operands: every operand value v is split into
+// hi = v rounded to tf32 and lo = v - hi (exact in fp32), and a product of two
+// operands is accumulated as hi*hi + hi*lo + lo*hi (the dropped lo*lo term is
+// below 2^-22 of it; the tensor core reads lo at tf32 precision, 2^-11 of lo).
+// The accumulation runs in fp32 in tensor memory; the bias and ReLU are applied
+// by the epilogue in fp32.
 constexpr int KT_AP = KT_P + 4;
 constexpr int KT_THREADS = 256;
-constexpr int KT_W1 = 0, KT_B1 = KT_W1 + 63 * 32, KT_W2 = KT_B1 + 32, KT_B2 = KT_W2 + 32 * 32;
-constexpr int KT_WS = KT_B2 + 32, KT_BS = KT_WS + 32, KT_WC = KT_BS + 1, KT_BC = KT_WC + 3 * 59;
-constexpr int KT_ACT = 3320;                          // KILO_NP rounded up to a multiple of 4
-constexpr int KT_H1 = KT_ACT + 63 * KT_AP;            // [32][KT_AP]
-constexpr int KT_DPE = KT_H1 + 32 * KT_AP;            // [27][KT_AP]: gamma(unit d)
-constexpr int KT_SIG = KT_DPE + 27 * KT_AP;
-constexpr int KT_RGB = KT_SIG + KT_P;
-constexpr int KT_FLOATS = KT_RGB + 3 * KT_P;
-constexpr size_t KT_SMEM = KT_FLOATS * sizeof(float);
-static_assert(KT_ACT >= KILO_NP && KT_ACT % 4 == 0 && KT_H1 % 4 == 0, "layout");
+// shared memory, bytes: operands in the no-swizzle K-major core-matrix layout
+// (8 rows x 16 bytes: 4 tf32 elements of K per row)
+constexpr int KC_B1 = 0;                               // W1 hi, lo: 32 x 64 x 4 B each
+constexpr int KC_B2 = KC_B1 + 2 * 32 * 64 * 4;         // W2 hi, lo: 32 x 32 x 4 B each
+constexpr int KC_VEC = KC_B2 + 2 * 32 * 32 * 4;        // fp32: b1, b2, ws, bs, wc, bc
+constexpr int KC_NV = 32 + 32 + 32 + 1 + 3 * 59 + 3;
+constexpr int KC_A = (KC_VEC + KC_NV * 4 + 1023) / 1024 * 1024;  // A hi, lo: 128 x 64 x 4 B each
+constexpr int KC_A_HALF = KT_P * 64 * 4;               // one of A hi / lo (32 KB)
+constexpr int KC_DPE = KC_A + 2 * KC_A_HALF;           // [27][KT_AP] fp32: gamma(unit d)
+constexpr int KC_SIG = KC_DPE + 27 * KT_AP * 4;        // [KT_P]
+constexpr int KC_RGB = KC_SIG + KT_P * 4;              // [3][KT_P]
+constexpr int KC_BAR = KC_RGB + 3 * KT_P * 4;
+constexpr size_t KT_SMEM = KC_BAR + 16 + 16;
+static_assert(KC_A % 1024 == 0 && KC_B2 % 16 == 0 && KC_DPE % 16 == 0, "operand alignment");
+static_assert(32 * KT_AP * 4 <= 2 * KC_A_HALF, "h2 fits in the A operand area");
 static_assert(2 * KT_THREADS - 3 * KT_P == KT_P, "the heads' second round leaves KT_P threads for sigma");
 
-// out[n][p] = ReLU(b[n] + sum_k W[n][k] in[k][p]), N = 32; the operands of
-// step k + 1 are loaded while step k computes.
+// Byte offset of element (r, k) in an operand of R rows, K-major core matrices.
+__device__ __forceinline__ uint32_t kc_off(int r, int k, int R) {
+  return (uint32_t)((k >> 2) * (R * 16) + (r >> 3) * 128 + (r & 7) * 16 + (k & 3) * 4);
+}
+// v = hi + lo with hi rounded to tf32 (nearest, ties away from zero) and lo exact.
+__device__ __forceinline__ void tf32_split(float v, float& hi, float& lo) {
+  uint32_t h;
+  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(h) : "f"(v));
+  hi = __uint_as_float(h);
+  lo = __fsub_rn(v, hi);
+}
+__device__ __forceinline__ void mma_tf32(uint32_t tmem_d, uint64_t a, uint64_t b, uint32_t idesc,
+                                         uint32_t accum) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}"
+      ::"r"(tmem_d), "l"(a), "l"(b), "r"(idesc), "r"(accum));
+}
+// One 32-wide layer: D[128 x 32] = A[128 x K] B[32 x K]^T in three tf32 passes
+// per K-step of 8 (issued by one thread).
 template <int K>
-__device__ __forceinline__ void tile_dense32(const float* __restrict__ Wt, const float* __restrict__ b,
-                                             const float* in, float* out) {
-  const int tx = threadIdx.x & 7, ty = threadIdx.x >> 3;
-  const int n0 = 4 * tx, p0 = 4 * ty;
-  float acc[4][4];
+__device__ __forceinline__ void kilo_layer_mma(uint32_t tmem, uint32_t a_hi, uint32_t b_hi,
+                                               int b_half_bytes) {
+  constexpr uint32_t idesc = (1u << 4) | (2u << 7) | (2u << 10) | ((32u >> 3) << 17) |
+                             ((uint32_t)(KT_P >> 4) << 24);   // f32 <- tf32 x tf32, N 32, M 128
+  const uint64_t ah = tcx::sdesc(a_hi, KT_P * 16, 128), al = tcx::sdesc(a_hi + KC_A_HALF, KT_P * 16, 128);
+  const uint64_t bh = tcx::sdesc(b_hi, 32 * 16, 128), bl = tcx::sdesc(b_hi + b_half_bytes, 32 * 16, 128);
 #pragma unroll
-  for (int i = 0; i < 4; ++i)
-#pragma unroll
-    for (int j = 0; j < 4; ++j) acc[i][j] = b[n0 + j];
-  float4 an = *reinterpret_cast<const float4*>(in + p0);
-  float4 wn = *reinterpret_cast<const float4*>(Wt + n0);
-#pragma unroll 7
-  for (int k = 0; k < K; ++k) {
-    const float4 a4 = an;
-    const float4 w = wn;
-    if (k + 1 < K) {
-      an = *reinterpret_cast<const float4*>(in + (k + 1) * KT_AP + p0);
-      wn = *reinterpret_cast<const float4*>(Wt + (k + 1) * 32 + n0);
-    }
-    const float a[4] = {a4.x, a4.y, a4.z, a4.w};
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      acc[i][0] = fmaf(w.x, a[i], acc[i][0]);
-      acc[i][1] = fmaf(w.y, a[i], acc[i][1]);
-      acc[i][2] = fmaf(w.z, a[i], acc[i][2]);
-      acc[i][3] = fmaf(w.w, a[i], acc[i][3]);
-    }
+  for (int s = 0; s < K / 8; ++s) {
+    const uint64_t da = (uint64_t)((s * 2 * KT_P * 16) >> 4), db = (uint64_t)((s * 2 * 32 * 16) >> 4);
+    mma_tf32(tmem, ah + da, bh + db, idesc, s != 0);
+    mma_tf32(tmem, ah + da, bl + db, idesc, 1);
+    mma_tf32(tmem, al + da, bh + db, idesc, 1);
   }
-#pragma unroll
-  for (int j = 0; j < 4; ++j)
-    *reinterpret_cast<float4*>(out + (n0 + j) * KT_AP + p0) =
-        make_float4(fmaxf(acc[0][j], 0.f), fmaxf(acc[1][j], 0.f), fmaxf(acc[2][j], 0.f),
-                    fmaxf(acc[3][j], 0.f));
 }
 
 __global__ void __launch_bounds__(KT_THREADS, 2)
 kilo_eval_kernel(const float* __restrict__ o, const float* __restrict__ d, int64_t r0, float near,
                  float step, const uint32_t* __restrict__ live, const int32_t* __restrict__ order,
                  const int4* __restrict__ items, const int32_t* __restrict__ n_items,
-                 const float* __restrict__ cell_w, float* __restrict__ out) {
-  extern __shared__ __align__(16) float ks[];
-  float* w1t = ks + KT_W1;
-  float* b1 = ks + KT_B1;
-  float* w2t = ks + KT_W2;
-  float* b2 = ks + KT_B2;
-  float* ws = ks + KT_WS;
-  float* bs = ks + KT_BS;
-  float* wc = ks + KT_WC;
-  float* bc = ks + KT_BC;
-  float* act = ks + KT_ACT;          // gamma(x) [63][KT_AP], then h2 in rows 0..31
-  float* h1 = ks + KT_H1;
-  float* dpe = ks + KT_DPE;
-  float* sig = ks + KT_SIG;
-  float* rgbv = ks + KT_RGB;
+                 const float* __restrict__ cell_w, float* __restrict__ out, unsigned* flag) {
+  extern __shared__ __align__(1024) uint8_t ksm[];
+  float* vecs = reinterpret_cast<float*>(ksm + KC_VEC);
+  const float* b1 = vecs;
+  const float* b2 = vecs + 32;
+  const float* ws = vecs + 64;
+  const float* bs = vecs + 96;
+  const float* wc = vecs + 97;                         // [3][59]
+  const float* bc = vecs + 97 + 3 * 59;
+  float* stage = reinterpret_cast<float*>(ksm + KC_A); // gamma(x) [64][KT_P] fp32, before the split
+  float* h2 = reinterpret_cast<float*>(ksm + KC_A);    // [32][KT_AP], after the second layer
+  float* dpe = reinterpret_cast<float*>(ksm + KC_DPE);
+  float* sig = reinterpret_cast<float*>(ksm + KC_SIG);
+  float* rgbv = reinterpret_cast<float*>(ksm + KC_RGB);
+  uint64_t* bar = reinterpret_cast<uint64_t*>(ksm + KC_BAR);
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(ksm + KC_BAR + 8);
+  const uint32_t a_hi = tcx::smem_u32(ksm + KC_A);
+  const int warp = threadIdx.x >> 5;
   const int p = threadIdx.x & (KT_P - 1);
-  const int part = threadIdx.x / KT_P;          // 0: position encoding, 1: direction encoding
+  const int part = threadIdx.x / KT_P;          // 0: position encoding, 1: the rest of it and gamma(d)
+  constexpr uint64_t kLimit = 2000000000ull;
+  __shared__ int abort_s;
+  if (threadIdx.x == 0) {
+    tcx::mbar_init(bar, 1);
+    abort_s = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 0) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
+                 ::"r"(tcx::smem_u32(tmem_holder)), "r"(32));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+  tcx::fence_before();
+  __syncthreads();
+  tcx::fence_after();
+  const uint32_t tmem = *tmem_holder;
+  uint32_t phase = 0;
+  // one thread issues a layer's MMAs and commits them; every thread waits and
+  // all take the same decision on a timeout
+  auto run_layer = [&](bool second) -> bool {
+    tcx::fence_async_smem();
+    tcx::fence_before();
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      tcx::fence_after();
+      if (second) kilo_layer_mma<32>(tmem, a_hi, tcx::smem_u32(ksm + KC_B2), 32 * 32 * 4);
+      else kilo_layer_mma<64>(tmem, a_hi, tcx::smem_u32(ksm + KC_B1), 32 * 64 * 4);
+      tcx::mma_commit(bar);
+    }
+    const bool ok = tcx::mbar_wait(bar, phase, &abort_s, flag, kLimit);
+    phase ^= 1;
+    tcx::fence_after();
+    return __syncthreads_and(ok) != 0;
+  };
   // a contiguous run of items per CTA: the items are in cell order, so
   // consecutive items mostly share a cell and its weights stay staged
   const int NI = *n_items;
@@ -1008,29 +1054,34 @@ kilo_eval_kernel(const float* __restrict__ o, const float* __restrict__ d, int64
   const int it0 = (int)blockIdx.x * per;
   const int it1 = min(NI, it0 + per);
   int staged = -1;
+  bool pending = false;          // a layer's wait gave up with its MMAs still in flight
   for (int it = it0; it < it1; ++it) {
     const int4 item = items[it];
     const int n = item.z;
     __syncthreads();     // the previous item's last reads are over
     if (item.x != staged) {
-      // this cell's weights (row-major W[n][k] in the blob) -> Wt[k][n], in two
-      // bank-conflict-free steps through the (idle) activation buffer: a
-      // coalesced copy (W2 rows padded to 33), then a transpose with lanes along n
+      // this cell's weights: W1 [32][63] and W2 [32][32] (row-major in the blob)
+      // as tf32 hi / lo operands, K-major (W1's K padded to 64 with zeros); the
+      // vectors in fp32
       staged = item.x;
       const float* W = cell_w + (int64_t)item.x * KILO_NP;
-      float* tmp = act;
-      for (int q = threadIdx.x; q < KILO_NP; q += KT_THREADS) {
-        const float v = __ldg(W + q);
-        if (q < KT_B1) tmp[q] = v;
-        else if (q < KT_W2) b1[q - KT_B1] = v;
-        else if (q < KT_B2) { const int z = q - KT_W2; tmp[KT_B1 + (z / 32) * 33 + z % 32] = v; }
-        else ks[q] = v;                               // b2, ws, bs, wc, bc in place
+      for (int q = threadIdx.x; q < 32 * 64; q += KT_THREADS) {
+        const int nn = q >> 6, k = q & 63;
+        float hi, lo;
+        tf32_split(k < 63 ? __ldg(W + nn * 63 + k) : 0.0f, hi, lo);
+        *reinterpret_cast<float*>(ksm + KC_B1 + kc_off(nn, k, 32)) = hi;
+        *reinterpret_cast<float*>(ksm + KC_B1 + 32 * 64 * 4 + kc_off(nn, k, 32)) = lo;
       }
-      __syncthreads();
-      for (int t = threadIdx.x; t < 63 * 32; t += KT_THREADS) w1t[t] = tmp[(t % 32) * 63 + t / 32];
-      for (int t = threadIdx.x; t < 32 * 32; t += KT_THREADS)
-        w2t[t] = tmp[KT_B1 + (t % 32) * 33 + t / 32];
-      __syncthreads();   // the transpose's reads of the activation buffer are over
+      for (int q = threadIdx.x; q < 32 * 32; q += KT_THREADS) {
+        const int nn = q >> 5, k = q & 31;
+        float hi, lo;
+        tf32_split(__ldg(W + 63 * 32 + 32 + q), hi, lo);
+        *reinterpret_cast<float*>(ksm + KC_B2 + kc_off(nn, k, 32)) = hi;
+        *reinterpret_cast<float*>(ksm + KC_B2 + 32 * 32 * 4 + kc_off(nn, k, 32)) = lo;
+      }
+      // blob order after W1: b1 (32), W2 (1024), b2 (32), ws (32), bs (1), wc (177), bc (3)
+      for (int q = threadIdx.x; q < KC_NV; q += KT_THREADS)
+        vecs[q] = __ldg(W + (q < 32 ? 63 * 32 + q : 63 * 32 + 32 + 32 * 32 + (q - 32)));
     }
     int64_t i = 0;
     if (p < n) i = order[item.y + p];
@@ -1042,28 +1093,30 @@ kilo_eval_kernel(const float* __restrict__ o, const float* __restrict__ d, int64
         r = r0 + (e >> 9);
         march_point(o, d, r, near, step, (int)(e & 511u), x, &t);
       }
-      // the 42 sin/cos pairs split about evenly: part 0 takes position coordinates
-      // 0 and 1 (20), part 1 coordinate 2 and the direction (10 + 12)
+      // gamma(x) in fp32, k-major; the 42 sin/cos pairs split about evenly:
+      // part 0 takes position coordinates 0 and 1 (20), part 1 coordinate 2
+      // and the direction (10 + 12)
       if (part == 0) {
-        act[0 * KT_AP + p] = x[0];
-        act[1 * KT_AP + p] = x[1];
-        act[2 * KT_AP + p] = x[2];
+        stage[0 * KT_P + p] = x[0];
+        stage[1 * KT_P + p] = x[1];
+        stage[2 * KT_P + p] = x[2];
+        stage[63 * KT_P + p] = 0.0f;
 #pragma unroll
         for (int c = 0; c < 2; ++c)
 #pragma unroll
           for (int k = 0; k < 10; ++k) {
             float sn, cs;
             pe_sincos(x[c], k, &sn, &cs);
-            act[(3 + c * 10 + k) * KT_AP + p] = sn;
-            act[(33 + c * 10 + k) * KT_AP + p] = cs;
+            stage[(3 + c * 10 + k) * KT_P + p] = sn;
+            stage[(33 + c * 10 + k) * KT_P + p] = cs;
           }
       } else {
 #pragma unroll
         for (int k = 0; k < 10; ++k) {
           float sn, cs;
           pe_sincos(x[2], k, &sn, &cs);
-          act[(3 + 20 + k) * KT_AP + p] = sn;
-          act[(33 + 20 + k) * KT_AP + p] = cs;
+          stage[(3 + 20 + k) * KT_P + p] = sn;
+          stage[(33 + 20 + k) * KT_P + p] = cs;
         }
         const float dx = d[r * 3], dy = d[r * 3 + 1], dz = d[r * 3 + 2];
         const float inv = 1.0f / sqrtf(dx * dx + dy * dy + dz * dz);
@@ -1082,10 +1135,57 @@ kilo_eval_kernel(const float* __restrict__ o, const float* __restrict__ d, int64
           }
       }
     }
-    __syncthreads();
-    tile_dense32<63>(w1t, b1, act, h1);                // gamma(x) -> h1
-    __syncthreads();
-    tile_dense32<32>(w2t, b2, h1, act);                // h1 -> h2 (rows 0..31)
+    // the A operand of the first layer: this thread's point, K columns
+    // [32 part, 32 part + 32), read from the staging area (which the operand
+    // then overwrites), split into tf32 hi / lo, four columns per 16-byte store
+    {
+      __syncthreads();
+      float g[32];
+#pragma unroll
+      for (int k = 0; k < 32; ++k) g[k] = stage[(32 * part + k) * KT_P + p];
+      __syncthreads();
+#pragma unroll
+      for (int kg = 0; kg < 8; ++kg) {
+        float hi[4], lo[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) tf32_split(g[4 * kg + j], hi[j], lo[j]);
+        const uint32_t off = kc_off(p, 32 * part + 4 * kg, KT_P);
+        tcx::st_shared_v4(a_hi + off, __float_as_uint(hi[0]), __float_as_uint(hi[1]),
+                          __float_as_uint(hi[2]), __float_as_uint(hi[3]));
+        tcx::st_shared_v4(a_hi + KC_A_HALF + off, __float_as_uint(lo[0]), __float_as_uint(lo[1]),
+                          __float_as_uint(lo[2]), __float_as_uint(lo[3]));
+      }
+    }
+    if (!run_layer(false)) { pending = true; break; }
+    // h1 = ReLU(b1 + acc) as the second layer's A operand (tf32 hi / lo): warps
+    // 0-3 read their TMEM lane quarter, 32 columns each
+    if (warp < 4) {
+      uint32_t u[32];
+      tcx::tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16), u);
+      tcx::tmem_ld_wait(u);
+#pragma unroll
+      for (int kg = 0; kg < 8; ++kg) {
+        float hi[4], lo[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          tf32_split(fmaxf(__fadd_rn(b1[4 * kg + j], __uint_as_float(u[4 * kg + j])), 0.0f), hi[j], lo[j]);
+        const uint32_t off = kc_off(p, 4 * kg, KT_P);
+        tcx::st_shared_v4(a_hi + off, __float_as_uint(hi[0]), __float_as_uint(hi[1]),
+                          __float_as_uint(hi[2]), __float_as_uint(hi[3]));
+        tcx::st_shared_v4(a_hi + KC_A_HALF + off, __float_as_uint(lo[0]), __float_as_uint(lo[1]),
+                          __float_as_uint(lo[2]), __float_as_uint(lo[3]));
+      }
+    }
+    if (!run_layer(true)) { pending = true; break; }
+    // h2 = ReLU(b2 + acc), fp32, k-major for the heads
+    if (warp < 4) {
+      uint32_t u[32];
+      tcx::tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16), u);
+      tcx::tmem_ld_wait(u);
+#pragma unroll
+      for (int k = 0; k < 32; ++k) h2[k * KT_AP + p] = fmaxf(__fadd_rn(b2[k], __uint_as_float(u[k])), 0.0f);
+    }
+    tcx::fence_before();
     __syncthreads();
     // heads: 3 KT_P rgb items and KT_P sigma items over two rounds of the 256
     // threads (sigma on the threads the rgb items leave idle in the second round)
@@ -1093,14 +1193,14 @@ kilo_eval_kernel(const float* __restrict__ o, const float* __restrict__ d, int64
       const int pp = threadIdx.x - (3 * KT_P - KT_THREADS);
       float s = bs[0];
 #pragma unroll 8
-      for (int k = 0; k < 32; ++k) s = fmaf(ws[k], act[k * KT_AP + pp], s);
+      for (int k = 0; k < 32; ++k) s = fmaf(ws[k], h2[k * KT_AP + pp], s);
       sig[pp] = fmaxf(s, 0.0f);
     }
     for (int q = threadIdx.x; q < 3 * KT_P; q += KT_THREADS) {
       const int c = q / KT_P, pp = q % KT_P;
       float v = bc[c];
 #pragma unroll 8
-      for (int k = 0; k < 32; ++k) v = fmaf(wc[c * 59 + k], act[k * KT_AP + pp], v);
+      for (int k = 0; k < 32; ++k) v = fmaf(wc[c * 59 + k], h2[k * KT_AP + pp], v);
 #pragma unroll
       for (int k = 0; k < 27; ++k) v = fmaf(wc[c * 59 + 32 + k], dpe[k * KT_AP + pp], v);
       rgbv[c * KT_P + pp] = 1.0f / (1.0f + expf(-v));
@@ -1109,6 +1209,20 @@ kilo_eval_kernel(const float* __restrict__ o, const float* __restrict__ d, int64
     if (part == 0 && p < n)
       reinterpret_cast<float4*>(out)[i] =
           make_float4(rgbv[p], rgbv[KT_P + p], rgbv[2 * KT_P + p], sig[p]);
+  }
+  // the MMAs this CTA issued complete before TMEM is freed: every layer was
+  // waited for, or a wait gave up (raising the timeout flag) and the pending
+  // MMAs get one more bounded wait here
+  if (pending && threadIdx.x == 0) {
+    const uint64_t t0 = tcx::globaltimer();
+    while (!tcx::mbar_try(bar, phase ^ 1) && tcx::globaltimer() - t0 < kLimit) {
+    }
+  }
+  tcx::fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tcx::fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(32));
   }
 }
 
@@ -1246,7 +1360,7 @@ cudaError_t march_render_chunk(const MarchArgs& a, cudaStream_t st) {
     slot = tm.begin(TK_NETWORK, st);
     kilo_eval_kernel<<<(unsigned)(a.num_sms * 2), KT_THREADS, KT_SMEM, st>>>(
         a.o, a.d, a.r0, a.near, a.step, a.ws.live, a.ws.order, a.ws.items, a.ws.n_items,
-        a.cell_w, a.ws.val);
+        a.cell_w, a.ws.val, a.flag);
     tm.end(slot, st);
   }
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
