@@ -397,6 +397,11 @@ def fp32_peak(clocks):
 
 
 FP32_PEAK_NOTE = "fp32 FMA: 148 SMs x 128 lanes x 2 FLOP x SM clock"
+# nominal dense tf32 / bf16 tensor rates of the part (1.1 and 2.25 PFLOP/s)
+TF32_PER_BF16 = 1.1 / 2.25
+# tensor-core FLOP the KiloNeRF kernel executes per point: three tf32 passes of
+# the 64 (63 + padding) -> 32 and 32 -> 32 layers
+KILO_MMA_FLOP_PER_POINT = 3 * 2 * (64 * 32 + 32 * 32)
 
 
 def run_sweep(args, rank, world, local_rank):
@@ -769,7 +774,7 @@ def run_march(args, rank, world, local_rank):
         cell_w = torch.from_numpy(cells_np).cuda()
         kw = dict(occupancy=occ, cell_w=cell_w)
         scene = cells_np
-        flop_per_point, kname = 2 * 3249, "kilo_eval_kernel (per-cell tiny MLPs)"
+        flop_per_point, kname = 2 * 3249, "kilo_eval_kernel (per-cell tiny MLPs, 32-wide layers on the tensor cores in tf32 x3)"
     else:
         model = nb.NERF_MODEL_HASHGRID
         table_np = S.hashgrid_table(S.HashGridShape(), S.HASH_ENTRIES, wl.seed, 1e-4)
@@ -845,11 +850,20 @@ def run_march(args, rank, world, local_rank):
     achieved = live * flop_per_point / (per_frame_k_ms * 1e-3) / 1e12
     nbytes = march_kernel_bytes(wl, R, live, tc)
     if wl.model == "kilonerf":
-        peak = fp32_peak(clocks)
-        roofline = {"bound": "alu", "kernel": kname, "achieved": achieved, "peak": peak,
-                    "unit": "TFLOP/s", "frac": achieved / peak, "peak_kind": FP32_PEAK_NOTE,
+        # the two 32-wide layers (6,080 of the 6,498 FLOP per point) run on the
+        # tensor cores in tf32, three passes per product (hi*hi + hi*lo + lo*hi) for
+        # fp32-level accuracy: the roofline is the tf32 dense peak (the bf16 figure
+        # times the nominal tf32 / bf16 ratio 1.1 / 2.25); the fp32 FMA rate that
+        # the CUDA-core version was measured against is reported beside it
+        bf = peaks.get("bf16_tflops")
+        peak = bf * TF32_PER_BF16 if bf else None
+        roofline = {"bound": "tensor", "kernel": kname, "achieved": achieved, "peak": peak,
+                    "unit": "TFLOP/s", "frac": achieved / peak if peak else None,
+                    "peak_kind": f"tf32 dense: bf16 {pk} x 1.1 / 2.25 (nominal ratio)",
                     "traffic": None, "kernel_ms_per_frame": per_frame_k_ms,
-                    "flop_per_point": flop_per_point}
+                    "flop_per_point": flop_per_point,
+                    "mma_flop_per_point": KILO_MMA_FLOP_PER_POINT,
+                    "frac_of_fp32_fma": achieved / fp32_peak(clocks)}
     else:
         # the hash-grid scene kernel is bound by its 128 table gathers per point
         # (the 23.3 MiB table stays in L2): its roofline is the algorithmic gather
