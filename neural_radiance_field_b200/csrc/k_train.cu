@@ -22,6 +22,7 @@
 #include <algorithm>
 
 #include "nerf_internal.cuh"
+#include "tc_ptx.cuh"
 
 namespace nerfb {
 
@@ -224,6 +225,8 @@ struct RowGemm {
   const float* mask; int64_t ldm;
   float* out; int64_t ldo;
   int a_vec, b_vec;
+  float* bsplit;   // scratch for the tensor-core path's split weights (K x n_out x 2 floats)
+  unsigned* flag;  // the context's error flag (bounded waits of the tensor-core path)
 };
 
 __global__ void __launch_bounds__(256, 2) row_gemm_kernel(RowGemm g) {
@@ -298,6 +301,289 @@ __global__ void __launch_bounds__(256, 2) row_gemm_kernel(RowGemm g) {
       }
       *reinterpret_cast<float4*>(g.out + row * g.ldo + c) = make_float4(v[0], v[1], v[2], v[3]);
     }
+  }
+}
+
+// The same row GEMM on the tensor cores (tcgen05.mma kind::tf32, M = 128 rows
+// per CTA, N = n_out, 128 or 256), with fp32-level accuracy: every operand
+// value v is split into hi = v rounded to tf32 and lo = v - hi (exact in
+// fp32), and each product accumulates hi*hi + hi*lo + lo*hi in fp32 in tensor
+// memory (the dropped lo*lo term is below 2^-22 of it). The weights B are split
+// once per call by split_b_kernel into K chunks of 32 in the MMA's K-major
+// core-matrix layout; the CTA splits its A rows chunk by chunk into shared
+// memory, double-buffered against the MMAs of the previous chunk. The epilogue
+// is row_gemm_kernel's, in the same order. Accumulation runs in the tensor
+// core's order, so results differ from the CUDA-core kernel's in the last bits.
+// A chunk's split weights (hi then lo, contiguous) arrive by one bulk copy.
+constexpr int TG_M = 128;                              // rows per CTA
+constexpr int TG_KC = 32;                              // K per chunk
+constexpr int TG_A_HALF = TG_M * TG_KC * 4;            // A hi or lo of a chunk, 16 KB
+constexpr int TG_B_HALF = 256 * TG_KC * 4;             // B hi or lo of a chunk (N <= 256), 32 KB
+constexpr int TG_STAGE = 2 * TG_A_HALF + 2 * TG_B_HALF;
+constexpr size_t TG_SMEM = 2 * TG_STAGE + 48;
+constexpr int TG_LD = 256 + 1;                          // row of the epilogue's tile (floats)
+static_assert(TG_M * TG_LD * 4 <= 2 * TG_STAGE, "the epilogue tile fits in the operand stages");
+
+// Byte offset of element (r, k) of an R-row operand chunk, K-major core matrices
+// (8 rows x 16 bytes: 4 tf32 elements of K per row).
+__device__ __forceinline__ uint32_t tg_off(int r, int k, int R) {
+  return (uint32_t)((k >> 2) * (R * 16) + (r >> 3) * 128 + (r & 7) * 16 + (k & 3) * 4);
+}
+__device__ __forceinline__ void tg_split(float v, float& hi, float& lo) {
+  uint32_t h;
+  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(h) : "f"(v));
+  hi = __uint_as_float(h);
+  lo = __fsub_rn(v, hi);
+}
+
+// B[k][c] (k < K, c < N) -> chunks of 32 K: [chunk][hi | lo][N rows x 32 K].
+__global__ void split_b_kernel(const float* __restrict__ B, int64_t ldb, int K, int N,
+                               float* __restrict__ out) {
+  const int64_t total = (int64_t)K * N;
+  for (int64_t q = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; q < total;
+       q += (int64_t)gridDim.x * blockDim.x) {
+    const int k = (int)(q / N), c = (int)(q % N);
+    float hi, lo;
+    tg_split(__ldg(B + (int64_t)k * ldb + c), hi, lo);
+    float* ch = out + (int64_t)(k / TG_KC) * 2 * N * TG_KC;
+    const uint32_t o = tg_off(c, k % TG_KC, N) >> 2;
+    ch[o] = hi;
+    ch[N * TG_KC + o] = lo;
+  }
+}
+
+__device__ __forceinline__ void tg_mma(uint32_t tmem_d, uint64_t a, uint64_t b, uint32_t idesc,
+                                       uint32_t accum) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}"
+      ::"r"(tmem_d), "l"(a), "l"(b), "r"(idesc), "r"(accum));
+}
+
+template <int N>
+__global__ void __launch_bounds__(256, 1) row_gemm_tc_kernel(RowGemm g) {
+  unsigned* flag = g.flag;
+  extern __shared__ __align__(1024) uint8_t tsm[];
+  uint64_t* done = reinterpret_cast<uint64_t*>(tsm + 2 * TG_STAGE);   // [2], MMAs of a stage
+  uint64_t* bfull = done + 2;                                           // [2], B of a stage landed
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(tsm + 2 * TG_STAGE + 32);
+  __shared__ int abort_s;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const uint32_t sbase = tcx::smem_u32(tsm);
+  constexpr uint64_t kLimit = 2000000000ull;
+  if (tid == 0) {
+    tcx::mbar_init(&done[0], 1);
+    tcx::mbar_init(&done[1], 1);
+    tcx::mbar_init(&bfull[0], 1);
+    tcx::mbar_init(&bfull[1], 1);
+    abort_s = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 0) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
+                 ::"r"(tcx::smem_u32(tmem_holder)), "r"(N));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+  tcx::fence_before();
+  __syncthreads();
+  tcx::fence_after();
+  const uint32_t tmem = *tmem_holder;
+  // A: thread tid stages row tid / 2, K columns [16 (tid % 2), +16) of a chunk
+  const int arow = tid >> 1, akh = (tid & 1) * 16;
+  const int nch = g.K / TG_KC;
+  const int64_t ntiles = (g.rows + TG_M - 1) / TG_M;
+  // A of a chunk: fetched into registers two chunks ahead (the activation
+  // store streams from DRAM), then split and stored once its stage is free
+  auto fetch_a = [&](int64_t m0, int c, float4 (&v)[4]) {
+    const int64_t ar = m0 + arow;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int k = c * TG_KC + akh + 4 * q;
+      const int col = k < g.a_split ? g.a0 + k : g.a1 + k - g.a_split;
+      v[q] = (ar < g.rows && c < nch) ? load4(g.A + ar * g.lda + col, g.a_vec, true, true, true, true)
+                                      : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+  };
+  auto put_a = [&](int stage, const float4 (&v)[4]) {
+    const uint32_t sa = sbase + stage * TG_STAGE;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      float hi[4], lo[4];
+      tg_split(v[q].x, hi[0], lo[0]);
+      tg_split(v[q].y, hi[1], lo[1]);
+      tg_split(v[q].z, hi[2], lo[2]);
+      tg_split(v[q].w, hi[3], lo[3]);
+      const uint32_t o = tg_off(arow, akh + 4 * q, TG_M);
+      tcx::st_shared_v4(sa + o, __float_as_uint(hi[0]), __float_as_uint(hi[1]),
+                        __float_as_uint(hi[2]), __float_as_uint(hi[3]));
+      tcx::st_shared_v4(sa + TG_A_HALF + o, __float_as_uint(lo[0]), __float_as_uint(lo[1]),
+                        __float_as_uint(lo[2]), __float_as_uint(lo[3]));
+    }
+  };
+  // B hi and lo of chunk c (2 N x 32 floats, contiguous) by one bulk copy
+  auto copy_b = [&](int c, int stage) {
+    constexpr uint32_t bytes = 2 * N * TG_KC * 4;
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;"
+                 ::"r"(tcx::smem_u32(&bfull[stage])), "r"(bytes) : "memory");
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+        ::"r"(sbase + stage * TG_STAGE + 2 * TG_A_HALF),
+          "l"(g.bsplit + (int64_t)c * 2 * N * TG_KC), "r"(bytes),
+          "r"(tcx::smem_u32(&bfull[stage]))
+        : "memory");
+  };
+  constexpr uint32_t idesc = (1u << 4) | (2u << 7) | (2u << 10) | ((uint32_t)(N >> 3) << 17) |
+                             ((uint32_t)(TG_M >> 4) << 24);   // f32 <- tf32 x tf32, M 128
+  bool ok = true;
+  // chunks are counted over the CTA's tiles: chunk G uses stage G % 2, and the
+  // stage's barriers complete once per chunk (parity (G / 2) % 2)
+  int64_t G = 0;
+  int64_t issued = -1;             // the last chunk whose MMAs were issued (uniform)
+  float4 va[4], vb[4];
+  // persistent: the CTA walks row tiles blockIdx.x, blockIdx.x + gridDim.x, ...
+  for (int64_t tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
+    const int64_t m0 = tile * TG_M;
+    if (tid == 0) copy_b(0, (int)(G & 1));
+    fetch_a(m0, 0, va);
+    fetch_a(m0, 1, vb);
+    put_a((int)(G & 1), va);
+    tcx::fence_async_smem();
+    __syncthreads();
+    // one chunk: its MMAs, then the next chunk's operands into the other stage
+    // (`put` holds chunk c + 1's A; chunk c + 2's A is fetched into `nxt`, two
+    // register sets alternating so that no copy waits on loads in flight)
+    auto step = [&](int c, const float4 (&put)[4], float4 (&nxt)[4]) -> bool {
+      const int stage = (int)(G & 1);
+      if (tid == 0) {
+        ok = tcx::mbar_wait(&bfull[stage], (uint32_t)((G >> 1) & 1), &abort_s, flag, kLimit) && ok;
+        tcx::fence_after();
+        const uint32_t sa = sbase + stage * TG_STAGE;
+        const uint64_t ah = tcx::sdesc(sa, TG_M * 16, 128), al = tcx::sdesc(sa + TG_A_HALF, TG_M * 16, 128);
+        const uint64_t bh = tcx::sdesc(sa + 2 * TG_A_HALF, N * 16, 128);
+        const uint64_t bl = tcx::sdesc(sa + 2 * TG_A_HALF + N * TG_KC * 4, N * 16, 128);
+#pragma unroll
+        for (int s = 0; s < TG_KC / 8; ++s) {
+          const uint64_t da = (uint64_t)((s * 2 * TG_M * 16) >> 4), db = (uint64_t)((s * 2 * N * 16) >> 4);
+          tg_mma(tmem, ah + da, bh + db, idesc, (c | s) != 0);
+          tg_mma(tmem, ah + da, bl + db, idesc, 1);
+          tg_mma(tmem, al + da, bh + db, idesc, 1);
+        }
+        tcx::mma_commit(&done[stage]);
+      }
+      issued = G;
+      if (c + 1 < nch) {
+        fetch_a(m0, c + 2, nxt);
+        // the other stage's operands were read by chunk G - 1's MMAs
+        if (c >= 1)
+          ok = tcx::mbar_wait(&done[stage ^ 1], (uint32_t)(((G - 1) >> 1) & 1), &abort_s, flag, kLimit) && ok;
+        if (tid == 0) copy_b(c + 1, stage ^ 1);
+        put_a(stage ^ 1, put);
+        tcx::fence_async_smem();
+      }
+      ++G;
+      if (__syncthreads_and(ok) == 0) { ok = false; return false; }
+      return true;
+    };
+    for (int c = 0; c < nch; c += 2) {
+      if (!step(c, vb, va)) break;
+      if (c + 1 < nch && !step(c + 1, va, vb)) break;
+    }
+    if (!ok) break;
+    // the tile's last commit covers every MMA issued so far
+    ok = tcx::mbar_wait(&done[issued & 1], (uint32_t)((issued >> 1) & 1), &abort_s, flag, kLimit);
+    tcx::fence_after();
+    if (__syncthreads_and(ok) == 0) { ok = false; break; }
+    // epilogue: the accumulator tile goes through shared memory (the operand
+    // stages are free now), so that the output, the mask and the row biases
+    // move in whole rows: warp w reads TMEM lane quarter w % 4, column half w / 4
+    // into rows of TG_LD floats, then thread t finishes columns 4 (t % (N / 4))
+    // of every (256 / (N / 4))-th row
+    float* tilebuf = reinterpret_cast<float*>(tsm);
+    {
+      const int q = warp & 3, h = warp >> 2, r = q * 32 + lane;
+#pragma unroll 1
+      for (int cb = h * (N / 2); cb < (h + 1) * (N / 2); cb += 32) {
+        uint32_t u[32];
+        tcx::tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)cb, u);
+        tcx::tmem_ld_wait(u);
+#pragma unroll
+        for (int j = 0; j < 32; ++j) tilebuf[r * TG_LD + cb + j] = __uint_as_float(u[j]);
+      }
+    }
+    tcx::fence_before();
+    __syncthreads();
+    constexpr int CPT = N / 4;                     // threads per row
+    const int c4 = 4 * (tid % CPT);
+    const bool cok = c4 < g.n_out;
+    const float4 b4 = (g.bias && cok) ? __ldg(reinterpret_cast<const float4*>(g.bias + c4))
+                                      : make_float4(0.f, 0.f, 0.f, 0.f);
+    const float4 ev4 = (g.ea && cok) ? __ldg(reinterpret_cast<const float4*>(g.ev + c4))
+                                     : make_float4(0.f, 0.f, 0.f, 0.f);
+    // rows in batches of 8 per thread: the batch's masks and row biases are all
+    // loaded before any of its outputs is stored (the compiler cannot know that
+    // the output aliases none of them)
+    constexpr int RSTEP = 256 / CPT;
+#pragma unroll 1
+    for (int r0 = tid / CPT; r0 < TG_M; r0 += 8 * RSTEP) {
+      float4 mk[8], rbv[8];
+      float ev_[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int r = r0 + i * RSTEP;
+        const int64_t row = m0 + r;
+        const bool live = cok && r < TG_M && row < g.rows;
+        mk[i] = make_float4(1.f, 1.f, 1.f, 1.f);
+        rbv[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+        ev_[i] = 0.0f;
+        if (live && g.mask) {
+          const float* mp = g.mask + row * g.ldm + c4;
+          mk[i] = make_float4(mp[0], mp[1], mp[2], mp[3]);
+        }
+        if (live && g.row_bias) {
+          const float* rp = g.row_bias + (row / g.rb_div) * g.n_out + c4;
+          rbv[i] = make_float4(rp[0], rp[1], rp[2], rp[3]);
+        }
+        if (live && g.ea) ev_[i] = g.ea[row * g.ldea];
+      }
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int r = r0 + i * RSTEP;
+        const int64_t row = m0 + r;
+        if (!cok || r >= TG_M || row >= g.rows) continue;
+        float v[4] = {tilebuf[r * TG_LD + c4], tilebuf[r * TG_LD + c4 + 1],
+                      tilebuf[r * TG_LD + c4 + 2], tilebuf[r * TG_LD + c4 + 3]};
+        const float bv[4] = {b4.x, b4.y, b4.z, b4.w}, evv[4] = {ev4.x, ev4.y, ev4.z, ev4.w};
+        const float rbb[4] = {rbv[i].x, rbv[i].y, rbv[i].z, rbv[i].w};
+        const float mkk[4] = {mk[i].x, mk[i].y, mk[i].z, mk[i].w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          float x = v[j];
+          if (g.bias) x += bv[j];
+          if (g.row_bias) x += rbb[j];
+          if (g.ea) x = fmaf(ev_[i], evv[j], x);
+          if (g.relu) x = fmaxf(x, 0.0f);
+          if (g.mask) x = mkk[j] > 0.0f ? x : 0.0f;
+          v[j] = x;
+        }
+        *reinterpret_cast<float4*>(g.out + row * g.ldo + c4) = make_float4(v[0], v[1], v[2], v[3]);
+      }
+    }
+    __syncthreads();     // the tile buffer is read before the next tile's operands overwrite it
+  }
+  if (!ok && tid == 0 && issued >= 0) {
+    // a wait gave up (timeout flag raised): one more bounded wait for the MMAs in
+    // flight before TMEM is freed
+    const uint64_t t0 = tcx::globaltimer();
+    while (!tcx::mbar_try(&done[issued & 1], (uint32_t)((issued >> 1) & 1)) &&
+           tcx::globaltimer() - t0 < kLimit) {
+    }
+  }
+  tcx::fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tcx::fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(N));
   }
 }
 
@@ -607,6 +893,31 @@ cudaError_t row_gemm(RowGemm g, cudaStream_t st) {
     return cudaErrorInvalidValue;
   g.a_vec = al16(g.A) && g.lda % 4 == 0 && g.a0 % 4 == 0 && g.a1 % 4 == 0;
   g.b_vec = al16(g.B) && g.ldb % 4 == 0;
+  // the network's layers (K a multiple of 32, 128 or 256 outputs) run on the
+  // tensor cores; other shapes on the CUDA-core kernel
+  if (g.bsplit && g.K % TG_KC == 0 && (g.n_out == 128 || g.n_out == 256) &&
+      (int64_t)g.K * g.n_out * 2 <= TRAIN_BSPLIT) {
+    static bool attr_set[2] = {false, false};
+    const int wide = g.n_out == 256;
+    if (!attr_set[wide]) {
+      cudaError_t e = wide ? cudaFuncSetAttribute(row_gemm_tc_kernel<256>,
+                                                  cudaFuncAttributeMaxDynamicSharedMemorySize, (int)TG_SMEM)
+                           : cudaFuncSetAttribute(row_gemm_tc_kernel<128>,
+                                                  cudaFuncAttributeMaxDynamicSharedMemorySize, (int)TG_SMEM);
+      if (e != cudaSuccess) return e;
+      attr_set[wide] = true;
+    }
+    const int64_t nb = (int64_t)g.K * g.n_out;
+    split_b_kernel<<<(unsigned)std::min<int64_t>(blocks_for(nb, 256), 1024), 256, 0, st>>>(
+        g.B, g.ldb, g.K, g.n_out, g.bsplit);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    // persistent: one CTA per SM walks the row tiles
+    const unsigned grid = (unsigned)std::min<int64_t>(blocks_for(g.rows, TG_M), sm_count());
+    if (wide) row_gemm_tc_kernel<256><<<grid, 256, TG_SMEM, st>>>(g);
+    else row_gemm_tc_kernel<128><<<grid, 256, TG_SMEM, st>>>(g);
+    return cudaGetLastError();
+  }
   row_gemm_kernel<<<dim3(blocks_for(g.rows, GT), blocks_for(g.n_out, GT)), 256, 0, st>>>(g);
   return cudaGetLastError();
 }
@@ -660,8 +971,8 @@ cudaError_t launch_composite_bw(const float* raw, const SampleSpec& ss, const fl
 // then ReLU) is that of the fused forward kernel.
 cudaError_t mlp_forward_train_fp32(const PackedFp32& p, const float* pk, const float* dir_bias,
                                    const float* o, const float* d, int64_t R,
-                                   const SampleSpec& ss, float* raw, float* save,
-                                   cudaStream_t st) {
+                                   const SampleSpec& ss, float* raw, float* save, float* bsplit,
+                                   unsigned* flag, cudaStream_t st) {
   const int D = p.D, W = p.W, Wh = W / 2;
   const int64_t rows = R * ss.S;
   if (rows == 0) return cudaSuccess;
@@ -679,6 +990,7 @@ cudaError_t mlp_forward_train_fp32(const PackedFp32& p, const float* pk, const f
     g.B = pk + p.layer_w[l]; g.ldb = W; g.n_out = W; g.rows = rows;
     g.bias = pk + p.layer_b[l]; g.relu = 1;
     g.out = save + hcol(l); g.ldo = ldc;
+    g.bsplit = bsplit; g.flag = flag;
     e = row_gemm(g, st);
   }
   if (e != cudaSuccess) return e;
@@ -687,6 +999,7 @@ cudaError_t mlp_forward_train_fp32(const PackedFp32& p, const float* pk, const f
     g.A = save; g.lda = ldc; g.a0 = hcol(D - 1); g.a_split = W; g.K = W;
     g.B = pk + p.feat_w; g.ldb = W; g.n_out = W; g.rows = rows; g.bias = pk + p.feat_b;
     g.out = save + feat_col; g.ldo = ldc;
+    g.bsplit = bsplit; g.flag = flag;
     if ((e = row_gemm(g, st)) != cudaSuccess) return e;
   }
   {  // direction layer: per-ray bias (b_dir + W_dir[:, W:] gamma(d)), ReLU
@@ -695,6 +1008,7 @@ cudaError_t mlp_forward_train_fp32(const PackedFp32& p, const float* pk, const f
     g.B = pk + p.dir_w; g.ldb = Wh; g.n_out = Wh; g.rows = rows;
     g.row_bias = dir_bias; g.rb_div = ss.S; g.relu = 1;
     g.out = save + hdir_col; g.ldo = ldc;
+    g.bsplit = bsplit; g.flag = flag;
     if ((e = row_gemm(g, st)) != cudaSuccess) return e;
   }
   heads_fwd_kernel<<<blocks_for(rows * 32, 256), 256, 0, st>>>(save, ldc, hcol(D - 1), hdir_col, W,
@@ -708,7 +1022,8 @@ cudaError_t mlp_forward_train_fp32(const PackedFp32& p, const float* pk, const f
 // floats of scratch.
 cudaError_t mlp_backward_fp32(const PackedFp32& p, int L_dir, const float* w, const float* save,
                               int64_t R, int S, const float* d, const float* d_raw,
-                              float* grad, float* tmp, cudaStream_t st) {
+                              float* grad, float* tmp, float* bsplit, unsigned* flag,
+                              cudaStream_t st) {
   const int D = p.D, W = p.W, Wh = W / 2, skip = p.skip;
   const int dir_ch = 3 + 6 * L_dir;
   const int64_t rows = R * S;
@@ -749,6 +1064,7 @@ cudaError_t mlp_backward_fp32(const PackedFp32& p, int L_dir, const float* w, co
     g.rows = rows; g.ea = ea; g.ldea = 4; g.ev = ev;
     if (mcol >= 0) { g.mask = save + mcol; g.ldm = ldc; }
     g.out = out; g.ldo = W;
+    g.bsplit = bsplit; g.flag = flag;
     return row_gemm(g, st);
   };
   // rgb head: dz_dir = (d_rgb x Wr) masked by h_dir > 0; dWr, dbr

@@ -206,6 +206,7 @@ nerf_status nerf_destroy(nerf_ctx* ctx) {
   cudaFree(ctx->tr_save);
   cudaFree(ctx->tr_draw);
   cudaFree(ctx->tr_tmp);
+  cudaFree(ctx->tr_bsplit);
   cudaFree(ctx->tr_loss);
   free_march(ctx);
   if (ctx->ev) {
@@ -297,7 +298,7 @@ nerf_status run_network(nerf_ctx* ctx, const void* blob, const float* o, const f
   TimedScope ts(ctx, TK_NETWORK, st);
   if (save) {
     NERF_CHECK_LAUNCH(ctx, mlp_forward_train_fp32(ctx->plan, ctx->packed, ctx->dir_bias, o, d, R,
-                                                  ss, raw, save, st));
+                                                  ss, raw, save, ctx->tr_bsplit, ctx->d_flag, st));
   } else {
     NERF_CHECK_LAUNCH(ctx, launch_mlp_fp32(ctx->plan, ctx->packed, ctx->dir_bias, o, d, R, ss, raw,
                                            st));
@@ -499,10 +500,12 @@ nerf_status nerf_loss_grad(nerf_ctx* ctx, const float* rays_o, const float* rays
     ok &= dalloc(&ctx->tr_draw, (size_t)(rows * 4)) == cudaSuccess;
     ok &= dalloc(&ctx->tr_tmp, (size_t)(2 * rows * W + c.max_rays * (W / 2 + dir_ch))) == cudaSuccess;
     ok &= dalloc(&ctx->tr_loss, (size_t)(2 * c.max_rays)) == cudaSuccess;
+    ok &= dalloc(&ctx->tr_bsplit, (size_t)TRAIN_BSPLIT) == cudaSuccess;
     if (!ok) {
       cudaGetLastError();
       cudaFree(ctx->tr_save); cudaFree(ctx->tr_draw); cudaFree(ctx->tr_tmp); cudaFree(ctx->tr_loss);
-      ctx->tr_save = ctx->tr_draw = ctx->tr_tmp = ctx->tr_loss = nullptr;
+      cudaFree(ctx->tr_bsplit);
+      ctx->tr_save = ctx->tr_draw = ctx->tr_tmp = ctx->tr_loss = ctx->tr_bsplit = nullptr;
       return fail(ctx, NERF_ERR_OOM, "training workspace allocation failed");
     }
   }
@@ -531,7 +534,8 @@ nerf_status nerf_loss_grad(nerf_ctx* ctx, const float* rays_o, const float* rays
                                              ctx->tr_draw, ctx->tr_loss, st));
   NERF_CHECK_LAUNCH(ctx, mlp_backward_fp32(ctx->plan, c.L_dir, (const float*)params->coarse_w,
                                            ctx->tr_save, R, n_coarse, rays_d, ctx->tr_draw,
-                                           grad_coarse, ctx->tr_tmp, st));
+                                           grad_coarse, ctx->tr_tmp, ctx->tr_bsplit, ctx->d_flag,
+                                           st));
   if (n_fine > 0) {
     SampleSpec fine{};
     fine.mode = SAMPLES_GIVEN_T;
@@ -543,7 +547,8 @@ nerf_status nerf_loss_grad(nerf_ctx* ctx, const float* rays_o, const float* rays
                                                ctx->tr_draw, ctx->tr_loss + R, st));
     NERF_CHECK_LAUNCH(ctx, mlp_backward_fp32(ctx->plan, c.L_dir, (const float*)params->fine_w,
                                              ctx->tr_save, R, fine.S, rays_d, ctx->tr_draw,
-                                             grad_fine, ctx->tr_tmp, st));
+                                             grad_fine, ctx->tr_tmp, ctx->tr_bsplit, ctx->d_flag,
+                                             st));
   }
   NERF_CHECK_LAUNCH(ctx, launch_sum(ctx->tr_loss, n_fine > 0 ? 2 * R : R, out_loss, st));
   return NERF_OK;

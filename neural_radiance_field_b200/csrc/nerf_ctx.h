@@ -25,6 +25,7 @@ struct nerf_ctx {
   float* tr_draw = nullptr;    // [max_rays * S][4] d raw
   float* tr_tmp = nullptr;     // backward scratch
   float* tr_loss = nullptr;    // [2 max_rays] per-ray loss terms
+  float* tr_bsplit = nullptr;  // split weights of one tensor-core row GEMM (TRAIN_BSPLIT floats)
 
   // kernel timing (nerf_timing_enable / nerf_timing_read / nerf_timing_read_kinds)
   bool timing = false;

@@ -139,13 +139,18 @@ struct CompositeSpec {
 cudaError_t launch_composite_bw(const float* raw, const SampleSpec& ss, const float* d, int64_t R,
                                 const CompositeSpec& cs, const float* target, float inv3n,
                                 float* d_raw, float* loss_terms, cudaStream_t st);
+// bsplit: scratch of TRAIN_BSPLIT floats (K x n_out x 2 for the widest layer,
+// K = 256 + 64, 256 outputs) for the tensor-core row GEMMs' split weights;
+// flag: the context's error flag.
+constexpr int64_t TRAIN_BSPLIT = (int64_t)320 * 256 * 2;
 cudaError_t mlp_forward_train_fp32(const PackedFp32& p, const float* packed, const float* dir_bias,
                                    const float* o, const float* d, int64_t R,
-                                   const SampleSpec& ss, float* raw, float* save,
-                                   cudaStream_t st);
+                                   const SampleSpec& ss, float* raw, float* save, float* bsplit,
+                                   unsigned* flag, cudaStream_t st);
 cudaError_t mlp_backward_fp32(const PackedFp32& p, int L_dir, const float* w, const float* save,
                               int64_t R, int S, const float* d, const float* d_raw,
-                              float* grad, float* tmp, cudaStream_t st);
+                              float* grad, float* tmp, float* bsplit, unsigned* flag,
+                              cudaStream_t st);
 cudaError_t launch_sum(const float* v, int64_t n, float* out, cudaStream_t st);
 cudaError_t launch_composite(const float* raw, const SampleSpec& ss, const float* d, int64_t R,
                              const CompositeSpec& cs, float* rgb, float* depth, float* acc,
