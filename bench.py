@@ -628,7 +628,10 @@ def run_train(args, rank, world, local_rank):
     rows = B * (2 * wl.n_coarse + wl.n_fine)
     clocks = clk.summary()
     sm_mhz = clocks["sm_mhz"] or 1965.0
-    peak = 148 * 128 * 2 * sm_mhz * 1e6 / 1e12
+    fma_peak = 148 * 128 * 2 * sm_mhz * 1e6 / 1e12
+    peaks, pk = load_peaks()
+    peak = peaks["bf16_tflops"] * TF32_PER_BF16
+    tf32_kind = f"tf32 dense: bf16 {pk} x 1.1 / 2.25 (nominal ratio); algorithmic FLOPs, 3 MMA passes each"
     achieved = (fwd + bwd) * rows * args.steps / (tot_ms * 1e-3) / 1e12
     line = {"metric": f"training rays/sec, batches of {B} rays, {wl.H}x{wl.W} frame, coarse+fine "
                       f"({wl.n_coarse}+{wl.n_fine}), 8x256 fp32, loss + gradients of both networks",
@@ -640,13 +643,18 @@ def run_train(args, rank, world, local_rank):
                        "mlp": "8x256 skip@4, fp32", "flop_per_row_fwd_bwd": fwd + bwd,
                        "l2": "flushed between timed steps (256 MiB write)"},
             "loss_last_step": float(loss.item()),
-            "roofline": {"bound": "alu", "kernel": "whole training step (fp32 CUDA-core kernels)",
+            "roofline": {"bound": "tensor", "kernel": "whole training step (layer GEMMs on the "
+                                                      "tensor cores in tf32 x3, heads on the CUDA cores)",
                          "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                         "frac": achieved / peak, "peak_kind": FP32_PEAK_NOTE, "traffic": None},
+                         "frac": achieved / peak, "peak_kind": tf32_kind,
+                         "frac_of_fp32_fma": achieved / fma_peak, "traffic": None},
             # per pass: weight packing, direction bias, the forward (encoding, D + 2
-            # layer GEMMs, heads), compositing backward, the backward (2 D + 9); then
-            # the resampling and the loss sum
-            "gpu_launches": args.steps * (2 * ((shape.D + 6) + 1 + (2 * shape.D + 9)) + 2),
+            # layer GEMMs, heads), compositing backward, the backward (2 D + 9); a
+            # weight split before each of the 2 D + 3 tensor-core row GEMMs, and a
+            # second column tile for the skip layer's weight gradient; then the
+            # resampling and the loss sum
+            "gpu_launches": args.steps * (2 * ((shape.D + 6) + 1 + (2 * shape.D + 9) + (2 * shape.D + 3)
+                                               + (1 if 0 <= shape.skip < shape.D - 1 else 0)) + 2),
             "clocks": clocks}
     print(json.dumps(line), flush=True)
 

@@ -310,19 +310,30 @@ __global__ void __launch_bounds__(256, 2) row_gemm_kernel(RowGemm g) {
 // fp32), and each product accumulates hi*hi + hi*lo + lo*hi in fp32 in tensor
 // memory (the dropped lo*lo term is below 2^-22 of it). The weights B are split
 // once per call by split_b_kernel into K chunks of 32 in the MMA's K-major
-// core-matrix layout; the CTA splits its A rows chunk by chunk into shared
+// core-matrix layout, and a chunk's split weights (hi then lo, contiguous)
+// arrive by one bulk copy; the CTA splits its A rows chunk by chunk into shared
 // memory, double-buffered against the MMAs of the previous chunk. The epilogue
-// is row_gemm_kernel's, in the same order. Accumulation runs in the tensor
-// core's order, so results differ from the CUDA-core kernel's in the last bits.
-// A chunk's split weights (hi then lo, contiguous) arrive by one bulk copy.
-constexpr int TG_M = 128;                              // rows per CTA
+// applies row_gemm_kernel's steps in the same order. Accumulation runs in the
+// tensor core's order, so results differ from the CUDA-core kernel's in the
+// last bits.
+constexpr int TG_M = 128;                              // rows per tile
 constexpr int TG_KC = 32;                              // K per chunk
 constexpr int TG_A_HALF = TG_M * TG_KC * 4;            // A hi or lo of a chunk, 16 KB
 constexpr int TG_B_HALF = 256 * TG_KC * 4;             // B hi or lo of a chunk (N <= 256), 32 KB
 constexpr int TG_STAGE = 2 * TG_A_HALF + 2 * TG_B_HALF;
-constexpr size_t TG_SMEM = 2 * TG_STAGE + 48;
-constexpr int TG_LD = 256 + 1;                          // row of the epilogue's tile (floats)
-static_assert(TG_M * TG_LD * 4 <= 2 * TG_STAGE, "the epilogue tile fits in the operand stages");
+constexpr int TG_WORKERS = 256;                         // the weight gradient's staging threads
+constexpr int TG_THREADS = TG_WORKERS + 32;             // + its issuer warp
+// Named barrier 1 over the worker threads; the second form returns whether any passed true.
+__device__ __forceinline__ void workers_sync() {
+  asm volatile("bar.sync 1, %0;" ::"n"(TG_WORKERS) : "memory");
+}
+__device__ __forceinline__ bool __syncthreads_or_workers(bool v) {
+  uint32_t r;
+  asm volatile("{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\t"
+               "bar.red.or.pred q, 1, %2, p;\n\tselp.u32 %0, 1, 0, q;\n\t}"
+               : "=r"(r) : "r"((uint32_t)v), "n"(TG_WORKERS) : "memory");
+  return r != 0;
+}
 
 // Byte offset of element (r, k) of an R-row operand chunk, K-major core matrices
 // (8 rows x 16 bytes: 4 tf32 elements of K per row).
@@ -361,229 +372,265 @@ __device__ __forceinline__ void tg_mma(uint32_t tmem_d, uint64_t a, uint64_t b, 
       ::"r"(tmem_d), "l"(a), "l"(b), "r"(idesc), "r"(accum));
 }
 
+// Roles of the row GEMM's CTA: warps 0-3 run the epilogue (warp w reads TMEM
+// lane quarter w: one accumulator row per thread), warps 4-11 stage the A rows,
+// warp 12 copies the weights and issues the MMAs. The accumulator is double-
+// buffered in tensor memory (2 N columns), so a tile's epilogue overlaps the
+// next tile's MMAs.
+constexpr int RG_EPI = 128;
+constexpr int RG_STG = 256;
+constexpr int RG_THREADS = RG_EPI + RG_STG + 32;
+constexpr size_t RG_SMEM = 2 * TG_STAGE + 128;
+
 template <int N>
-__global__ void __launch_bounds__(256, 1) row_gemm_tc_kernel(RowGemm g) {
+__global__ void __launch_bounds__(RG_THREADS, 1) row_gemm_tc_kernel(RowGemm g) {
   unsigned* flag = g.flag;
   extern __shared__ __align__(1024) uint8_t tsm[];
-  uint64_t* done = reinterpret_cast<uint64_t*>(tsm + 2 * TG_STAGE);   // [2], MMAs of a stage
-  uint64_t* bfull = done + 2;                                           // [2], B of a stage landed
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(tsm + 2 * TG_STAGE + 32);
+  uint64_t* done = reinterpret_cast<uint64_t*>(tsm + 2 * TG_STAGE);   // [2] MMAs of a stage done
+  uint64_t* bfull = done + 2;                                           // [2] B of a stage landed
+  uint64_t* afull = done + 4;                                           // [2] A of a stage staged
+  uint64_t* accf = done + 6;                                            // [2] accumulator ready
+  uint64_t* acce = done + 8;                                            // [2] accumulator read out
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(done + 10);
   __shared__ int abort_s;
+  __shared__ __align__(16) float s_bias[N], s_ev[N];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const uint32_t sbase = tcx::smem_u32(tsm);
   constexpr uint64_t kLimit = 2000000000ull;
   if (tid == 0) {
-    tcx::mbar_init(&done[0], 1);
-    tcx::mbar_init(&done[1], 1);
-    tcx::mbar_init(&bfull[0], 1);
-    tcx::mbar_init(&bfull[1], 1);
+    for (int i = 0; i < 2; ++i) {
+      tcx::mbar_init(&done[i], 1);
+      tcx::mbar_init(&bfull[i], 1);
+      tcx::mbar_init(&afull[i], RG_STG / 32);   // one arrival per staging warp
+      tcx::mbar_init(&accf[i], 1);
+      tcx::mbar_init(&acce[i], RG_EPI / 32);    // one arrival per epilogue warp
+    }
     abort_s = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
+  for (int i = tid; i < N; i += RG_THREADS) {
+    s_bias[i] = g.bias ? g.bias[i] : 0.0f;
+    s_ev[i] = g.ea ? g.ev[i] : 0.0f;
+  }
   if (warp == 0) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
-                 ::"r"(tcx::smem_u32(tmem_holder)), "r"(N));
+                 ::"r"(tcx::smem_u32(tmem_holder)), "r"(2 * N));
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
   }
   tcx::fence_before();
   __syncthreads();
   tcx::fence_after();
   const uint32_t tmem = *tmem_holder;
-  // A: thread tid stages row tid / 2, K columns [16 (tid % 2), +16) of a chunk
-  const int arow = tid >> 1, akh = (tid & 1) * 16;
   const int nch = g.K / TG_KC;
   const int64_t ntiles = (g.rows + TG_M - 1) / TG_M;
-  // A of a chunk: fetched into registers two chunks ahead (the activation
-  // store streams from DRAM), then split and stored once its stage is free
-  auto fetch_a = [&](int64_t m0, int c, float4 (&v)[4]) {
-    const int64_t ar = m0 + arow;
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const int k = c * TG_KC + akh + 4 * q;
-      const int col = k < g.a_split ? g.a0 + k : g.a1 + k - g.a_split;
-      v[q] = (ar < g.rows && c < nch) ? load4(g.A + ar * g.lda + col, g.a_vec, true, true, true, true)
-                                      : make_float4(0.f, 0.f, 0.f, 0.f);
-    }
-  };
-  auto put_a = [&](int stage, const float4 (&v)[4]) {
-    const uint32_t sa = sbase + stage * TG_STAGE;
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      float hi[4], lo[4];
-      tg_split(v[q].x, hi[0], lo[0]);
-      tg_split(v[q].y, hi[1], lo[1]);
-      tg_split(v[q].z, hi[2], lo[2]);
-      tg_split(v[q].w, hi[3], lo[3]);
-      const uint32_t o = tg_off(arow, akh + 4 * q, TG_M);
-      tcx::st_shared_v4(sa + o, __float_as_uint(hi[0]), __float_as_uint(hi[1]),
-                        __float_as_uint(hi[2]), __float_as_uint(hi[3]));
-      tcx::st_shared_v4(sa + TG_A_HALF + o, __float_as_uint(lo[0]), __float_as_uint(lo[1]),
-                        __float_as_uint(lo[2]), __float_as_uint(lo[3]));
-    }
-  };
-  // B hi and lo of chunk c (2 N x 32 floats, contiguous) by one bulk copy
-  auto copy_b = [&](int c, int stage) {
-    constexpr uint32_t bytes = 2 * N * TG_KC * 4;
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;"
-                 ::"r"(tcx::smem_u32(&bfull[stage])), "r"(bytes) : "memory");
-    asm volatile(
-        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
-        ::"r"(sbase + stage * TG_STAGE + 2 * TG_A_HALF),
-          "l"(g.bsplit + (int64_t)c * 2 * N * TG_KC), "r"(bytes),
-          "r"(tcx::smem_u32(&bfull[stage]))
-        : "memory");
-  };
-  constexpr uint32_t idesc = (1u << 4) | (2u << 7) | (2u << 10) | ((uint32_t)(N >> 3) << 17) |
-                             ((uint32_t)(TG_M >> 4) << 24);   // f32 <- tf32 x tf32, M 128
+  // this CTA's tiles: blockIdx.x, + gridDim.x, ...; chunk G of the CTA is chunk
+  // G % nch of its tile G / nch and uses operand stage G % 2, whose barriers
+  // complete once per chunk (parity (G / 2) % 2); tile i uses accumulator i % 2
+  const int n_my = blockIdx.x < ntiles ? (int)((ntiles - 1 - blockIdx.x) / gridDim.x + 1) : 0;
+  const int64_t total = (int64_t)n_my * nch;
   bool ok = true;
-  // chunks are counted over the CTA's tiles: chunk G uses stage G % 2, and the
-  // stage's barriers complete once per chunk (parity (G / 2) % 2)
-  int64_t G = 0;
-  int64_t issued = -1;             // the last chunk whose MMAs were issued (uniform)
-  float4 va[4], vb[4];
-  // persistent: the CTA walks row tiles blockIdx.x, blockIdx.x + gridDim.x, ...
-  for (int64_t tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
-    const int64_t m0 = tile * TG_M;
-    if (tid == 0) copy_b(0, (int)(G & 1));
-    fetch_a(m0, 0, va);
-    fetch_a(m0, 1, vb);
-    put_a((int)(G & 1), va);
-    tcx::fence_async_smem();
-    __syncthreads();
-    // one chunk: its MMAs, then the next chunk's operands into the other stage
-    // (`put` holds chunk c + 1's A; chunk c + 2's A is fetched into `nxt`, two
-    // register sets alternating so that no copy waits on loads in flight)
-    auto step = [&](int c, const float4 (&put)[4], float4 (&nxt)[4]) -> bool {
-      const int stage = (int)(G & 1);
-      if (tid == 0) {
-        ok = tcx::mbar_wait(&bfull[stage], (uint32_t)((G >> 1) & 1), &abort_s, flag, kLimit) && ok;
-        tcx::fence_after();
-        const uint32_t sa = sbase + stage * TG_STAGE;
-        const uint64_t ah = tcx::sdesc(sa, TG_M * 16, 128), al = tcx::sdesc(sa + TG_A_HALF, TG_M * 16, 128);
-        const uint64_t bh = tcx::sdesc(sa + 2 * TG_A_HALF, N * 16, 128);
-        const uint64_t bl = tcx::sdesc(sa + 2 * TG_A_HALF + N * TG_KC * 4, N * 16, 128);
-#pragma unroll
-        for (int s = 0; s < TG_KC / 8; ++s) {
-          const uint64_t da = (uint64_t)((s * 2 * TG_M * 16) >> 4), db = (uint64_t)((s * 2 * N * 16) >> 4);
-          tg_mma(tmem, ah + da, bh + db, idesc, (c | s) != 0);
-          tg_mma(tmem, ah + da, bl + db, idesc, 1);
-          tg_mma(tmem, al + da, bh + db, idesc, 1);
+  if (warp == (RG_EPI + RG_STG) / 32) {
+    // ------------------------------------------------------------- issuer warp
+    if (lane == 0) {
+      constexpr uint32_t idesc = (1u << 4) | (2u << 7) | (2u << 10) | ((uint32_t)(N >> 3) << 17) |
+                                 ((uint32_t)(TG_M >> 4) << 24);   // f32 <- tf32 x tf32, M 128
+      auto copy_b = [&](int c, int stage) {
+        constexpr uint32_t bytes = 2 * N * TG_KC * 4;
+        asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;"
+                     ::"r"(tcx::smem_u32(&bfull[stage])), "r"(bytes) : "memory");
+        asm volatile(
+            "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+            ::"r"(sbase + stage * TG_STAGE + 2 * TG_A_HALF),
+              "l"(g.bsplit + (int64_t)c * 2 * N * TG_KC), "r"(bytes),
+              "r"(tcx::smem_u32(&bfull[stage]))
+            : "memory");
+      };
+      int64_t G = 0, issued = -1, copied = -1;
+      if (total > 0) {
+        copy_b(0, 0);
+        copied = 0;
+      }
+      for (int it = 0; it < n_my && ok; ++it) {
+        const int b = it & 1;
+        if (it >= 2 && !tcx::mbar_wait(&acce[b], (uint32_t)(((it >> 1) - 1) & 1), &abort_s, flag, kLimit)) {
+          ok = false;
+          break;
         }
-        tcx::mma_commit(&done[stage]);
+        const uint32_t acc = tmem + (uint32_t)(b * N);
+        for (int c = 0; c < nch && ok; ++c, ++G) {
+          const int stage = (int)(G & 1);
+          const uint32_t par = (uint32_t)((G >> 1) & 1);
+          ok = tcx::mbar_wait(&bfull[stage], par, &abort_s, flag, kLimit) &&
+               tcx::mbar_wait(&afull[stage], par, &abort_s, flag, kLimit);
+          if (!ok) break;
+          tcx::fence_after();
+          const uint32_t sa = sbase + stage * TG_STAGE;
+          const uint64_t ah = tcx::sdesc(sa, TG_M * 16, 128), al = tcx::sdesc(sa + TG_A_HALF, TG_M * 16, 128);
+          const uint64_t bh = tcx::sdesc(sa + 2 * TG_A_HALF, N * 16, 128);
+          const uint64_t bl = tcx::sdesc(sa + 2 * TG_A_HALF + N * TG_KC * 4, N * 16, 128);
+#pragma unroll
+          for (int s = 0; s < TG_KC / 8; ++s) {
+            const uint64_t da = (uint64_t)((s * 2 * TG_M * 16) >> 4), db = (uint64_t)((s * 2 * N * 16) >> 4);
+            tg_mma(acc, ah + da, bh + db, idesc, (c | s) != 0);
+            tg_mma(acc, ah + da, bl + db, idesc, 1);
+            tg_mma(acc, al + da, bh + db, idesc, 1);
+          }
+          tcx::mma_commit(&done[stage]);
+          if (c == nch - 1) tcx::mma_commit(&accf[b]);
+          issued = G;
+          if (G + 1 < total) {
+            // the next chunk's weights (of this tile or the next) go into the
+            // stage that chunk G - 1's MMAs read
+            if (G >= 1)
+              ok = tcx::mbar_wait(&done[stage ^ 1], (uint32_t)(((G - 1) >> 1) & 1), &abort_s, flag, kLimit);
+            if (ok) {
+              copy_b(c + 1 < nch ? c + 1 : 0, stage ^ 1);
+              copied = G + 1;
+            }
+          }
+        }
       }
-      issued = G;
-      if (c + 1 < nch) {
-        fetch_a(m0, c + 2, nxt);
-        // the other stage's operands were read by chunk G - 1's MMAs
-        if (c >= 1)
-          ok = tcx::mbar_wait(&done[stage ^ 1], (uint32_t)(((G - 1) >> 1) & 1), &abort_s, flag, kLimit) && ok;
-        if (tid == 0) copy_b(c + 1, stage ^ 1);
-        put_a(stage ^ 1, put);
-        tcx::fence_async_smem();
+      // drain before TMEM and shared memory are given up (not stopped by an
+      // abort: the MMAs and the weight copy already issued must land first)
+      const uint64_t t0 = tcx::globaltimer();
+      if (issued >= 0)
+        while (!tcx::mbar_try(&done[issued & 1], (uint32_t)((issued >> 1) & 1)) &&
+               tcx::globaltimer() - t0 < kLimit) {
+        }
+      if (copied >= 0)
+        while (!tcx::mbar_try(&bfull[copied & 1], (uint32_t)((copied >> 1) & 1)) &&
+               tcx::globaltimer() - t0 < kLimit) {
+        }
+    }
+    __syncwarp();
+  } else if (warp >= RG_EPI / 32) {
+    // ------------------------------------------------------------- staging warps
+    // thread st stages row st / 2, K columns [16 (st % 2), +16) of a chunk; the
+    // rows are fetched into registers two chunks ahead (the activation store
+    // streams from DRAM), split and stored once their stage is free
+    const int st = tid - RG_EPI;
+    const int arow = st >> 1, akh = (st & 1) * 16;
+    auto fetch_a = [&](int64_t G, float4 (&v)[4]) {
+      const int64_t it = G / nch;
+      const int c = (int)(G - it * nch);
+      const int64_t ar = (blockIdx.x + it * gridDim.x) * TG_M + arow;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int k = c * TG_KC + akh + 4 * q;
+        const int col = k < g.a_split ? g.a0 + k : g.a1 + k - g.a_split;
+        v[q] = (G < total && ar < g.rows) ? load4(g.A + ar * g.lda + col, g.a_vec, true, true, true, true)
+                                          : make_float4(0.f, 0.f, 0.f, 0.f);
       }
-      ++G;
-      if (__syncthreads_and(ok) == 0) { ok = false; return false; }
+    };
+    auto put_a = [&](int stage, const float4 (&v)[4]) {
+      const uint32_t sa = sbase + stage * TG_STAGE;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        float hi[4], lo[4];
+        tg_split(v[q].x, hi[0], lo[0]);
+        tg_split(v[q].y, hi[1], lo[1]);
+        tg_split(v[q].z, hi[2], lo[2]);
+        tg_split(v[q].w, hi[3], lo[3]);
+        const uint32_t o = tg_off(arow, akh + 4 * q, TG_M);
+        tcx::st_shared_v4(sa + o, __float_as_uint(hi[0]), __float_as_uint(hi[1]),
+                          __float_as_uint(hi[2]), __float_as_uint(hi[3]));
+        tcx::st_shared_v4(sa + TG_A_HALF + o, __float_as_uint(lo[0]), __float_as_uint(lo[1]),
+                          __float_as_uint(lo[2]), __float_as_uint(lo[3]));
+      }
+    };
+    // chunk G from `cur` into stage G % 2 (free once chunk G - 2's MMAs are
+    // done), then chunk G + 2 fetched into `cur`: two register sets alternate
+    auto stage_chunk = [&](int64_t G, float4 (&cur)[4]) -> bool {
+      const int stage = (int)(G & 1);
+      const bool w = G < 2 || tcx::mbar_wait(&done[stage], (uint32_t)(((G - 2) >> 1) & 1), &abort_s, flag, kLimit);
+      if (!__all_sync(0xffffffffu, w)) return false;   // the warp leaves together
+      put_a(stage, cur);
+      tcx::fence_async_smem();
+      __syncwarp();
+      if (lane == 0) tcx::mbar_arrive(&afull[stage]);
+      fetch_a(G + 2, cur);
       return true;
     };
-    for (int c = 0; c < nch; c += 2) {
-      if (!step(c, vb, va)) break;
-      if (c + 1 < nch && !step(c + 1, va, vb)) break;
+    float4 va[4], vb[4];
+    fetch_a(0, va);
+    fetch_a(1, vb);
+    for (int64_t G = 0; G < total && ok; G += 2) {
+      ok = stage_chunk(G, va);
+      if (ok && G + 1 < total) ok = stage_chunk(G + 1, vb);
     }
-    if (!ok) break;
-    // the tile's last commit covers every MMA issued so far
-    ok = tcx::mbar_wait(&done[issued & 1], (uint32_t)((issued >> 1) & 1), &abort_s, flag, kLimit);
-    tcx::fence_after();
-    if (__syncthreads_and(ok) == 0) { ok = false; break; }
-    // epilogue: the accumulator tile goes through shared memory (the operand
-    // stages are free now), so that the output, the mask and the row biases
-    // move in whole rows: warp w reads TMEM lane quarter w % 4, column half w / 4
-    // into rows of TG_LD floats, then thread t finishes columns 4 (t % (N / 4))
-    // of every (256 / (N / 4))-th row
-    float* tilebuf = reinterpret_cast<float*>(tsm);
-    {
-      const int q = warp & 3, h = warp >> 2, r = q * 32 + lane;
+  } else {
+    // ------------------------------------------------------------- epilogue warps
+    // thread = accumulator row warp * 32 + lane; 32 columns per TMEM load, the
+    // output row written in 16-byte pieces (each thread a whole 128-byte line
+    // per column block); the next block's side input (the mask or the row
+    // biases: a launch has at most one) is loaded while the current block is
+    // finished
+    const int rl = warp * 32 + lane;
+    for (int it = 0; it < n_my && ok; ++it) {
+      const int b = it & 1;
+      const bool w = tcx::mbar_wait(&accf[b], (uint32_t)((it >> 1) & 1), &abort_s, flag, kLimit);
+      if (!__all_sync(0xffffffffu, w)) {
+        ok = false;
+        break;
+      }
+      tcx::fence_after();
+      const int64_t row = (blockIdx.x + (int64_t)it * gridDim.x) * TG_M + rl;
+      const bool live = row < g.rows;
+      const float eav = (g.ea && live) ? g.ea[row * g.ldea] : 0.0f;
+      const float* mrow = (g.mask && live) ? g.mask + row * g.ldm : nullptr;
+      const float* rrow = (g.row_bias && live) ? g.row_bias + (row / g.rb_div) * g.n_out : nullptr;
+      float* orow = g.out + row * g.ldo;
+      const float* srow = mrow ? mrow : rrow;
+      float4 sd[8];
+      auto load_side = [&](int cb, float4 (&m)[8]) {
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+          m[j] = srow ? *reinterpret_cast<const float4*>(srow + cb + 4 * j) : make_float4(0.f, 0.f, 0.f, 0.f);
+      };
+      load_side(0, sd);
 #pragma unroll 1
-      for (int cb = h * (N / 2); cb < (h + 1) * (N / 2); cb += 32) {
+      for (int cb = 0; cb < N; cb += 32) {
         uint32_t u[32];
-        tcx::tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)cb, u);
+        tcx::tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)(b * N + cb), u);
+        float4 sd2[8];
+        if (cb + 32 < N) load_side(cb + 32, sd2);
         tcx::tmem_ld_wait(u);
 #pragma unroll
-        for (int j = 0; j < 32; ++j) tilebuf[r * TG_LD + cb + j] = __uint_as_float(u[j]);
-      }
-    }
-    tcx::fence_before();
-    __syncthreads();
-    constexpr int CPT = N / 4;                     // threads per row
-    const int c4 = 4 * (tid % CPT);
-    const bool cok = c4 < g.n_out;
-    const float4 b4 = (g.bias && cok) ? __ldg(reinterpret_cast<const float4*>(g.bias + c4))
-                                      : make_float4(0.f, 0.f, 0.f, 0.f);
-    const float4 ev4 = (g.ea && cok) ? __ldg(reinterpret_cast<const float4*>(g.ev + c4))
-                                     : make_float4(0.f, 0.f, 0.f, 0.f);
-    // rows in batches of 8 per thread: the batch's masks and row biases are all
-    // loaded before any of its outputs is stored (the compiler cannot know that
-    // the output aliases none of them)
-    constexpr int RSTEP = 256 / CPT;
-#pragma unroll 1
-    for (int r0 = tid / CPT; r0 < TG_M; r0 += 8 * RSTEP) {
-      float4 mk[8], rbv[8];
-      float ev_[8];
+        for (int j = 0; j < 8; ++j) {
+          const float4 bv = *reinterpret_cast<const float4*>(s_bias + cb + 4 * j);
+          const float4 ev = *reinterpret_cast<const float4*>(s_ev + cb + 4 * j);
+          float x[4] = {__uint_as_float(u[4 * j]), __uint_as_float(u[4 * j + 1]),
+                        __uint_as_float(u[4 * j + 2]), __uint_as_float(u[4 * j + 3])};
+          const float bb[4] = {bv.x, bv.y, bv.z, bv.w}, ee[4] = {ev.x, ev.y, ev.z, ev.w};
+          const float sv[4] = {sd[j].x, sd[j].y, sd[j].z, sd[j].w};
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const int r = r0 + i * RSTEP;
-        const int64_t row = m0 + r;
-        const bool live = cok && r < TG_M && row < g.rows;
-        mk[i] = make_float4(1.f, 1.f, 1.f, 1.f);
-        rbv[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-        ev_[i] = 0.0f;
-        if (live && g.mask) {
-          const float* mp = g.mask + row * g.ldm + c4;
-          mk[i] = make_float4(mp[0], mp[1], mp[2], mp[3]);
+          for (int e = 0; e < 4; ++e) {
+            float v = x[e];
+            if (g.bias) v += bb[e];
+            if (g.row_bias) v += sv[e];
+            if (g.ea) v = fmaf(eav, ee[e], v);
+            if (g.relu) v = fmaxf(v, 0.0f);
+            if (g.mask) v = sv[e] > 0.0f ? v : 0.0f;
+            x[e] = v;
+          }
+          if (live) *reinterpret_cast<float4*>(orow + cb + 4 * j) = make_float4(x[0], x[1], x[2], x[3]);
         }
-        if (live && g.row_bias) {
-          const float* rp = g.row_bias + (row / g.rb_div) * g.n_out + c4;
-          rbv[i] = make_float4(rp[0], rp[1], rp[2], rp[3]);
-        }
-        if (live && g.ea) ev_[i] = g.ea[row * g.ldea];
-      }
+        if (cb + 32 < N) {
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const int r = r0 + i * RSTEP;
-        const int64_t row = m0 + r;
-        if (!cok || r >= TG_M || row >= g.rows) continue;
-        float v[4] = {tilebuf[r * TG_LD + c4], tilebuf[r * TG_LD + c4 + 1],
-                      tilebuf[r * TG_LD + c4 + 2], tilebuf[r * TG_LD + c4 + 3]};
-        const float bv[4] = {b4.x, b4.y, b4.z, b4.w}, evv[4] = {ev4.x, ev4.y, ev4.z, ev4.w};
-        const float rbb[4] = {rbv[i].x, rbv[i].y, rbv[i].z, rbv[i].w};
-        const float mkk[4] = {mk[i].x, mk[i].y, mk[i].z, mk[i].w};
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          float x = v[j];
-          if (g.bias) x += bv[j];
-          if (g.row_bias) x += rbb[j];
-          if (g.ea) x = fmaf(ev_[i], evv[j], x);
-          if (g.relu) x = fmaxf(x, 0.0f);
-          if (g.mask) x = mkk[j] > 0.0f ? x : 0.0f;
-          v[j] = x;
+          for (int j = 0; j < 8; ++j) sd[j] = sd2[j];
         }
-        *reinterpret_cast<float4*>(g.out + row * g.ldo + c4) = make_float4(v[0], v[1], v[2], v[3]);
       }
-    }
-    __syncthreads();     // the tile buffer is read before the next tile's operands overwrite it
-  }
-  if (!ok && tid == 0 && issued >= 0) {
-    // a wait gave up (timeout flag raised): one more bounded wait for the MMAs in
-    // flight before TMEM is freed
-    const uint64_t t0 = tcx::globaltimer();
-    while (!tcx::mbar_try(&done[issued & 1], (uint32_t)((issued >> 1) & 1)) &&
-           tcx::globaltimer() - t0 < kLimit) {
+      // this warp's rows of the accumulator are read out
+      tcx::fence_before();
+      __syncwarp();
+      if (lane == 0) tcx::mbar_arrive(&acce[b]);
     }
   }
   tcx::fence_before();
   __syncthreads();
   if (warp == 0) {
     tcx::fence_after();
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(N));
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(2 * N));
   }
 }
 
@@ -597,6 +644,7 @@ struct WGrad {
   int64_t rows, slice;
   float* G; int64_t ldg; float* db;
   int a_vec, x_vec;   // x_vec: X, ldx, x0, x1 and x_split all 16-byte / 4-float aligned
+  unsigned* flag;     // the context's error word; set: the tensor-core kernel may run
 };
 
 template <bool XV>   // X rows 16-byte aligned and the split a multiple of 4
@@ -679,6 +727,209 @@ __global__ void __launch_bounds__(256, 2) wgrad_gemm_kernel(WGrad g) {
   }
   if (bias_cta && tid < GT && nb + tid < g.N) atomicAdd(g.db + nb + tid, bsum);
 }
+
+// The same weight gradient on the tensor cores, for N = 128 or 256 and one
+// column tile [k0, k0 + nt) of X (nt a power of two, 32..256; columns past K
+// are zero): G[n][k0 + k] += sum_r A[r][n] X(r, k0 + k), and, in the tile
+// with k0 = 0, db[n] += sum_r A[r][n]. The sum runs over the rows, so the rows
+// are the MMA's K: the CTAs take equal contiguous runs of 16-row chunks, the
+// worker warps split both operands per chunk (tf32 hi + fp32 remainder, as in
+// the row GEMM) into K-major core matrices, thread t owning column t of A and
+// of X, and the issuer warp accumulates hi*hi + hi*lo + lo*hi for each 128-row
+// half of n in tensor memory (M 128, N nt). At the end the CTA's partial tile
+// goes through shared memory and is added to G with coalesced atomics.
+constexpr int WT_KC = 16;                               // rows per chunk
+constexpr int WT_NSTAGE = 3;
+constexpr int WT_PART = 256 * WT_KC * 4;                // A hi, A lo, X hi or X lo of a chunk: 16 KB
+constexpr int WT_STAGE = 4 * WT_PART;
+constexpr size_t WT_SMEM = (size_t)WT_NSTAGE * WT_STAGE + 64;
+static_assert(128 * 257 * 4 <= WT_NSTAGE * WT_STAGE, "the epilogue tile fits in the stages");
+
+__global__ void __launch_bounds__(TG_THREADS, 1) wgrad_tc_kernel(WGrad g, int k0, int nt,
+                                                                 unsigned* flag) {
+  extern __shared__ __align__(1024) uint8_t wsm[];
+  uint64_t* done = reinterpret_cast<uint64_t*>(wsm + WT_NSTAGE * WT_STAGE);   // [3] MMAs of a stage
+  uint64_t* afull = done + WT_NSTAGE;                                          // [3] stage staged
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(afull + WT_NSTAGE);
+  __shared__ int abort_s;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const uint32_t sbase = tcx::smem_u32(wsm);
+  const int mh = g.N >> 7;                                   // 128-row halves of n
+  const uint32_t ncols = (uint32_t)(mh * nt);                // a power of two, 32..512
+  constexpr uint64_t kLimit = 2000000000ull;
+  if (tid == 0) {
+    for (int i = 0; i < WT_NSTAGE; ++i) {
+      tcx::mbar_init(&done[i], 1);
+      tcx::mbar_init(&afull[i], TG_WORKERS / 32);
+    }
+    abort_s = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 0) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
+                 ::"r"(tcx::smem_u32(tmem_holder)), "r"(ncols));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+  tcx::fence_before();
+  __syncthreads();
+  tcx::fence_after();
+  const uint32_t tmem = *tmem_holder;
+  const int64_t total = (g.rows + WT_KC - 1) / WT_KC;
+  const int64_t cb = (int64_t)blockIdx.x * total / gridDim.x;
+  const int nch = (int)((int64_t)(blockIdx.x + 1) * total / gridDim.x - cb);
+  bool ok = true;
+  if (warp == TG_WORKERS / 32) {
+    // ------------------------------------------------------------- issuer warp
+    if (lane == 0) {
+      const uint32_t idesc = (1u << 4) | (2u << 7) | (2u << 10) | ((uint32_t)(nt >> 3) << 17) |
+                             ((uint32_t)(128 >> 4) << 24);   // f32 <- tf32 x tf32, M 128, N nt
+      int issued = -1;
+      for (int c = 0; c < nch; ++c) {
+        const int s = c % WT_NSTAGE;
+        if (!tcx::mbar_wait(&afull[s], (uint32_t)((c / WT_NSTAGE) & 1), &abort_s, flag, kLimit)) break;
+        tcx::fence_after();
+        const uint32_t sa = sbase + s * WT_STAGE;
+        const uint64_t xh = tcx::sdesc(sa + 2 * WT_PART, nt * 16, 128);
+        const uint64_t xl = tcx::sdesc(sa + 3 * WT_PART, nt * 16, 128);
+        for (int h = 0; h < mh; ++h) {
+          const uint64_t ah = tcx::sdesc(sa + h * (128 * WT_KC * 4), 128 * 16, 128);
+          const uint64_t al = tcx::sdesc(sa + WT_PART + h * (128 * WT_KC * 4), 128 * 16, 128);
+          const uint32_t d = tmem + (uint32_t)(h * nt);
+#pragma unroll
+          for (int ks = 0; ks < WT_KC / 8; ++ks) {
+            const uint64_t da = (uint64_t)((ks * 2 * 128 * 16) >> 4);
+            const uint64_t dx = (uint64_t)((ks * 2 * nt * 16) >> 4);
+            tg_mma(d, ah + da, xh + dx, idesc, (c | ks) != 0);
+            tg_mma(d, ah + da, xl + dx, idesc, 1);
+            tg_mma(d, al + da, xh + dx, idesc, 1);
+          }
+        }
+        tcx::mma_commit(&done[s]);
+        issued = c;
+      }
+      // the MMAs already issued land before TMEM is freed, abort or not
+      if (issued >= 0) {
+        const uint64_t t0 = tcx::globaltimer();
+        while (!tcx::mbar_try(&done[issued % WT_NSTAGE], (uint32_t)((issued / WT_NSTAGE) & 1)) &&
+               tcx::globaltimer() - t0 < kLimit) {
+        }
+      }
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------- workers
+    const bool a_on = tid < g.N;
+    const int kx = k0 + tid;
+    const bool x_on = tid < nt && kx < g.K;
+    const int64_t xcol = kx < g.x_split ? g.x0 + kx : g.x1 + kx - g.x_split;
+    const int ah_ = tid >> 7, am = tid & 127;
+    float dbs = 0.0f;
+    auto fetch = [&](int c, float (&va)[WT_KC], float (&vx)[WT_KC]) {
+      const int64_t r0 = (cb + c) * WT_KC;
+#pragma unroll
+      for (int i = 0; i < WT_KC; ++i) {
+        const int64_t r = r0 + i;
+        const bool live = c < nch && r < g.rows;
+        va[i] = (live && a_on) ? __ldg(g.A + r * g.lda + tid) : 0.0f;
+        vx[i] = (live && x_on) ? __ldg(g.X + r * g.ldx + xcol) : 0.0f;
+      }
+    };
+    auto put = [&](int s, const float (&va)[WT_KC], const float (&vx)[WT_KC]) {
+      const uint32_t sa = sbase + s * WT_STAGE;
+      if (a_on) {
+        const uint32_t base = sa + ah_ * (128 * WT_KC * 4);
+#pragma unroll
+        for (int q = 0; q < WT_KC / 4; ++q) {
+          float hi[4], lo[4];
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            tg_split(va[4 * q + j], hi[j], lo[j]);
+            dbs += va[4 * q + j];
+          }
+          const uint32_t o = tg_off(am, 4 * q, 128);
+          tcx::st_shared_v4(base + o, __float_as_uint(hi[0]), __float_as_uint(hi[1]),
+                            __float_as_uint(hi[2]), __float_as_uint(hi[3]));
+          tcx::st_shared_v4(base + WT_PART + o, __float_as_uint(lo[0]), __float_as_uint(lo[1]),
+                            __float_as_uint(lo[2]), __float_as_uint(lo[3]));
+        }
+      }
+      if (tid < nt) {
+#pragma unroll
+        for (int q = 0; q < WT_KC / 4; ++q) {
+          float hi[4], lo[4];
+#pragma unroll
+          for (int j = 0; j < 4; ++j) tg_split(vx[4 * q + j], hi[j], lo[j]);
+          const uint32_t o = tg_off(tid, 4 * q, nt);
+          tcx::st_shared_v4(sa + 2 * WT_PART + o, __float_as_uint(hi[0]), __float_as_uint(hi[1]),
+                            __float_as_uint(hi[2]), __float_as_uint(hi[3]));
+          tcx::st_shared_v4(sa + 3 * WT_PART + o, __float_as_uint(lo[0]), __float_as_uint(lo[1]),
+                            __float_as_uint(lo[2]), __float_as_uint(lo[3]));
+        }
+      }
+    };
+    // chunk c goes into stage c % 3 once chunk c - 3's MMAs are done; the rows
+    // are fetched two chunks ahead into two alternating register sets
+    auto stage_chunk = [&](int c, float (&va)[WT_KC], float (&vx)[WT_KC]) -> bool {
+      const int s = c % WT_NSTAGE;
+      const bool w = c < WT_NSTAGE ||
+                     tcx::mbar_wait(&done[s], (uint32_t)((c / WT_NSTAGE - 1) & 1), &abort_s, flag, kLimit);
+      if (!__all_sync(0xffffffffu, w)) return false;
+      put(s, va, vx);
+      tcx::fence_async_smem();
+      __syncwarp();
+      if (lane == 0) tcx::mbar_arrive(&afull[s]);
+      fetch(c + 2, va, vx);
+      return true;
+    };
+    float a0[WT_KC], x0[WT_KC], a1[WT_KC], x1[WT_KC];
+    fetch(0, a0, x0);
+    fetch(1, a1, x1);
+    for (int c = 0; c < nch && ok; c += 2) {
+      ok = stage_chunk(c, a0, x0);
+      if (ok && c + 1 < nch) ok = stage_chunk(c + 1, a1, x1);
+    }
+    if (ok && nch > 0)
+      ok = tcx::mbar_wait(&done[(nch - 1) % WT_NSTAGE], (uint32_t)(((nch - 1) / WT_NSTAGE) & 1),
+                          &abort_s, flag, kLimit);
+    ok = __all_sync(0xffffffffu, ok);
+    tcx::fence_after();
+    if (!__syncthreads_or_workers(!ok) && nch > 0) {
+      // epilogue, one 128-row half of n at a time: TMEM -> tile [128][nt + 1]
+      // (warp w reads lane quarter w % 4; warps w and w + 4 split the columns),
+      // then thread t adds column t % nt of rows t / nt, + 256 / nt, ...
+      float* tile = reinterpret_cast<float*>(wsm);
+      const int ldt = nt + 1;
+      const int q = warp & 3, nsplit = nt >= 64 ? 2 : 1, cw = nt / nsplit;
+      for (int h = 0; h < mh; ++h) {
+        if ((warp >> 2) < nsplit) {
+          const int m = q * 32 + lane;
+          for (int c0 = (warp >> 2) * cw; c0 < (warp >> 2) * cw + cw; c0 += 32) {
+            uint32_t u[32];
+            tcx::tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(h * nt + c0), u);
+            tcx::tmem_ld_wait(u);
+#pragma unroll
+            for (int j = 0; j < 32; ++j) tile[m * ldt + c0 + j] = __uint_as_float(u[j]);
+          }
+        }
+        workers_sync();
+        const int col = tid & (nt - 1), rstep = TG_WORKERS / nt;
+        if (k0 + col < g.K) {
+          float* gp = g.G + (int64_t)(h * 128) * g.ldg + k0 + col;
+          for (int m = tid / nt; m < 128; m += rstep) atomicAdd(gp + (int64_t)m * g.ldg, tile[m * ldt + col]);
+        }
+        workers_sync();
+      }
+      if (k0 == 0 && g.db && a_on) atomicAdd(g.db + tid, dbs);
+    }
+  }
+  tcx::fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tcx::fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(ncols));
+  }
+}
+
 
 // The weight gradient of a head with N <= 4 outputs (sigma: 1, rgb: 3): one
 // thread per four input columns (the thread past the last one sums the bias),
@@ -895,15 +1146,19 @@ cudaError_t row_gemm(RowGemm g, cudaStream_t st) {
   g.b_vec = al16(g.B) && g.ldb % 4 == 0;
   // the network's layers (K a multiple of 32, 128 or 256 outputs) run on the
   // tensor cores; other shapes on the CUDA-core kernel
-  if (g.bsplit && g.K % TG_KC == 0 && (g.n_out == 128 || g.n_out == 256) &&
+  // (the epilogue moves 16-byte pieces of the output, mask and row-bias rows)
+  const bool side_vec = g.ldo % 4 == 0 && !(g.mask && g.row_bias) &&
+                        (!g.mask || (al16(g.mask) && g.ldm % 4 == 0)) &&
+                        (!g.row_bias || (al16(g.row_bias) && g.n_out % 4 == 0));
+  if (g.bsplit && side_vec && g.K % TG_KC == 0 && (g.n_out == 128 || g.n_out == 256) &&
       (int64_t)g.K * g.n_out * 2 <= TRAIN_BSPLIT) {
     static bool attr_set[2] = {false, false};
     const int wide = g.n_out == 256;
     if (!attr_set[wide]) {
       cudaError_t e = wide ? cudaFuncSetAttribute(row_gemm_tc_kernel<256>,
-                                                  cudaFuncAttributeMaxDynamicSharedMemorySize, (int)TG_SMEM)
+                                                  cudaFuncAttributeMaxDynamicSharedMemorySize, (int)RG_SMEM)
                            : cudaFuncSetAttribute(row_gemm_tc_kernel<128>,
-                                                  cudaFuncAttributeMaxDynamicSharedMemorySize, (int)TG_SMEM);
+                                                  cudaFuncAttributeMaxDynamicSharedMemorySize, (int)RG_SMEM);
       if (e != cudaSuccess) return e;
       attr_set[wide] = true;
     }
@@ -914,8 +1169,8 @@ cudaError_t row_gemm(RowGemm g, cudaStream_t st) {
     if (e != cudaSuccess) return e;
     // persistent: one CTA per SM walks the row tiles
     const unsigned grid = (unsigned)std::min<int64_t>(blocks_for(g.rows, TG_M), sm_count());
-    if (wide) row_gemm_tc_kernel<256><<<grid, 256, TG_SMEM, st>>>(g);
-    else row_gemm_tc_kernel<128><<<grid, 256, TG_SMEM, st>>>(g);
+    if (wide) row_gemm_tc_kernel<256><<<grid, RG_THREADS, RG_SMEM, st>>>(g);
+    else row_gemm_tc_kernel<128><<<grid, RG_THREADS, RG_SMEM, st>>>(g);
     return cudaGetLastError();
   }
   row_gemm_kernel<<<dim3(blocks_for(g.rows, GT), blocks_for(g.n_out, GT)), 256, 0, st>>>(g);
@@ -932,6 +1187,25 @@ int64_t slice_rows(int64_t rows, int tiles) {
 
 cudaError_t wgrad(WGrad g, cudaStream_t st) {
   if (g.rows == 0) return cudaSuccess;
+  // 128 or 256 outputs on the tensor cores, one launch per 256-column tile of X
+  if (g.flag && (g.N == 128 || g.N == 256)) {
+    static bool attr_set = false;
+    if (!attr_set) {
+      cudaError_t e = cudaFuncSetAttribute(wgrad_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           (int)WT_SMEM);
+      if (e != cudaSuccess) return e;
+      attr_set = true;
+    }
+    const unsigned grid = (unsigned)std::min<int64_t>((g.rows + WT_KC - 1) / WT_KC, sm_count());
+    for (int k0 = 0; k0 < g.K; k0 += 256) {
+      int nt = 32;
+      while (nt < g.K - k0 && nt < 256) nt *= 2;
+      wgrad_tc_kernel<<<grid, TG_THREADS, WT_SMEM, st>>>(g, k0, nt, g.flag);
+      cudaError_t e = cudaGetLastError();
+      if (e != cudaSuccess) return e;
+    }
+    return cudaSuccess;
+  }
   g.a_vec = al16(g.A) && g.lda % 4 == 0;
   g.x_vec = al16(g.X) && g.ldx % 4 == 0 && g.x0 % 4 == 0 && g.x1 % 4 == 0 && g.x_split % 4 == 0;
   const unsigned tn = blocks_for(g.N, GT), tk = blocks_for(g.K, GT);
@@ -1054,7 +1328,7 @@ cudaError_t mlp_backward_fp32(const PackedFp32& p, int L_dir, const float* w, co
                 int64_t ldg, float* db) {
     WGrad g{};
     g.A = A; g.lda = lda; g.N = N; g.X = save; g.ldx = ldc; g.x0 = x0; g.x_split = split;
-    g.x1 = x1; g.K = K; g.rows = rows; g.G = G; g.ldg = ldg; g.db = db;
+    g.x1 = x1; g.K = K; g.rows = rows; g.G = G; g.ldg = ldg; g.db = db; g.flag = flag;
     return wgrad(g, st);
   };
   auto in_grad = [&](const float* A, int64_t lda, int K, const float* B, int64_t ldb,

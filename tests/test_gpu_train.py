@@ -87,6 +87,26 @@ def test_coarse_step_matches_oracle(torch, kw):
     assert err <= REL * scale + 1e-9, (err, scale, int(np.abs(gc - ref_gc).argmax()))
 
 
+def test_many_tiles_step_matches_oracle(torch):
+    """The 8 x 256 network on 800 rays x 64 samples (51,200 rows): the tensor-core
+    row GEMMs walk two or three 128-row tiles per CTA and the weight gradients
+    twenty-odd 16-row chunks per CTA through their three shared-memory stages, so
+    every stage and tensor-memory buffer is reused, at the strict bar."""
+    wl, cw, fw, target = _setup("small", 32, 25, n_fine=0, mlp=S.MLPShape(D=8, W=256, skip=4),
+                                last_delta=S.LAST_DELTA_TO_FAR)
+    o, d = rays_for(wl)
+    loss, gc, _ = _gpu_step(torch, wl, o, d, cw, None, target)
+    ids = np.arange(wl.n_rays)
+    ref_loss, ref_gc, _ = og.loss_and_grad(wl, o.cpu().numpy(), d.cpu().numpy(), ids, target,
+                                           cw.astype(np.float64), None)
+    assert abs(loss - ref_loss) <= 1e-5 * ref_loss, (loss, ref_loss)
+    scale = np.abs(ref_gc).max()
+    err = np.abs(gc - ref_gc).max()
+    print(f"[train 800 rays D8W256] loss rel err {abs(loss - ref_loss) / ref_loss:.2e}, "
+          f"grad max err / max|g| {err / scale:.2e}")
+    assert err <= REL * scale + 1e-9, (err, scale, int(np.abs(gc - ref_gc).argmax()))
+
+
 def test_coarse_and_fine_step(torch):
     wl, cw, fw, target = _setup("small", 4, 6, mlp=S.MLPShape(D=3, W=64, skip=0),
                                 last_delta=S.LAST_DELTA_TO_FAR)
