@@ -7,6 +7,8 @@ same workload instead (a bounded sample of rays per step).
 
 Extra lines (`--workload`):
   small                     200x200 coarse + fine with the 8x256 network in fp32
+  small_tf32                the same with precision TF32 (layer GEMMs on the
+                            tensor cores, three tf32 MMAs per product)
   tiny                      32x32, 64 stratified samples, a 4x64 fp32 network
   kilonerf, hashgrid        march renders of the two alternative scene functions
   hashgrid_bf16             the hash grid with its MLP in bf16 on the tensor cores
@@ -225,6 +227,8 @@ def bandwidth_figures(kinds, bytes_per_frame, frames, hbm, peak_kind):
 NERF_METRICS = {
     "full": METRIC,
     "small": "rays/sec at 200x200 coarse+fine (64+128 samples/ray), 8x256 fp32 network",
+    "small_tf32": "rays/sec at 200x200 coarse+fine (64+128 samples/ray), 8x256 network, fp32 "
+                  "weights and I/O, layer products on the tensor cores (tf32 hi/lo, 3 passes)",
     "tiny": "rays/sec at 32x32, 64 stratified samples/ray, 4x64 fp32 network",
 }
 
@@ -340,6 +344,16 @@ def run_nerf(args, rank, world, local_rank, key=WORKLOAD):
                     "frac_of_sustained": achieved_tf / peak_sus,
                     "traffic": args.traffic_bytes or traffic_per_launch(flops_launch_avg),
                     "traffic_source": "--traffic-bytes" if args.traffic_bytes else TRAFFIC_SOURCE}
+    elif wl.precision == S.PREC_TF32:
+        # layer GEMMs on the tensor cores, three tf32 MMAs per product: the
+        # roofline is the tf32 dense peak against the algorithmic FLOPs
+        peak_tf = peaks.get("bf16_tflops") * TF32_PER_BF16
+        roofline = {"bound": "tensor",
+                    "kernel": "network pass: encoding, tensor-core row GEMMs (tf32 x3), heads",
+                    "achieved": achieved_tf, "peak": peak_tf, "unit": "TFLOP/s",
+                    "frac": achieved_tf / peak_tf,
+                    "peak_kind": f"tf32 dense: bf16 {peak_kind} x 1.1 / 2.25 (nominal ratio)",
+                    "frac_of_fp32_fma": achieved_tf / fp32_peak(clocks), "traffic": None}
     else:
         peak_tf = fp32_peak(clocks)
         roofline = {"bound": "alu", "kernel": f"mlp_fp32_kernel (CUDA-core MLP, W={wl.mlp.W})",
@@ -362,7 +376,7 @@ def run_nerf(args, rank, world, local_rank, key=WORKLOAD):
             "metric": NERF_METRICS[key], "value": value, "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": tot_ms / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": "bf16" if bf16 else "f32",
+            "dtype": "bf16" if bf16 else ("tf32x3" if wl.precision == S.PREC_TF32 else "f32"),
             "data": "synthetic (seeded camera, Xavier-init weights)",
             "config": config_json(wl, world),
             "sample_points_per_s": value * (wl.n_coarse + wl.n_fine),
@@ -386,9 +400,20 @@ def run_nerf(args, rank, world, local_rank, key=WORKLOAD):
 def nerf_launches_per_step(wl):
     """The library's kernels per NeRF step: ray generation; per pass the weight
     packing, the direction bias and the network; the resampling between passes;
-    the final compositing."""
+    the final compositing. With precision TF32 the network of a pass is, per
+    sub-batch of rays (the context's activation store holds 2^20 samples), the
+    encoding, a weight split and a row GEMM per layer (D + 2 of them) and the
+    heads."""
     passes = 2 if wl.n_fine else 1
-    return 1 + 3 * passes + (1 if wl.n_fine else 0) + 1
+    if wl.precision != S.PREC_TF32:
+        return 1 + 3 * passes + (1 if wl.n_fine else 0) + 1
+    fw_rows = min(wl.n_rays * (wl.n_coarse + wl.n_fine), 1 << 20)
+    net = 0
+    for s_pass in ([wl.n_coarse, wl.n_coarse + wl.n_fine] if wl.n_fine else [wl.n_coarse]):
+        per = max(1, fw_rows // s_pass)
+        n_sub = -(-wl.n_rays // per)
+        net += n_sub * (2 + 2 * (wl.mlp.D + 2))
+    return 1 + 2 * passes + net + (1 if wl.n_fine else 0) + 1
 
 
 def fp32_peak(clocks):
@@ -950,7 +975,7 @@ def main():
                     help="rays of the oracle's march sample (march workloads)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--workload", default=WORKLOAD,
-                    choices=[WORKLOAD, "small", "tiny", "kilonerf", "hashgrid", "hashgrid_bf16",
+                    choices=[WORKLOAD, "small", "small_tf32", "tiny", "kilonerf", "hashgrid", "hashgrid_bf16",
                              "sweep24", "compact", "train", "hash_backward"],
                     help="the benchmark workload (default) or a march workload (extra lines)")
     ap.add_argument("--traffic-bytes", type=float, default=0.0,

@@ -55,7 +55,7 @@ typedef enum {
 
 enum { NERF_MODEL_MLP = 0, NERF_MODEL_KILONERF = 1, NERF_MODEL_HASHGRID = 2 };
 enum { NERF_SIGMA_RELU = 0, NERF_SIGMA_SOFTPLUS = 1 };
-enum { NERF_FP32 = 0, NERF_BF16 = 1 };
+enum { NERF_FP32 = 0, NERF_BF16 = 1, NERF_TF32 = 2 };
 /* Length of the last interval of a ray: 1e10 as in the NeRF page's volume_render
  * (Section 2.5), or up to `far` (the closed form of T(t) on [t_n, t_f]). */
 enum { NERF_LAST_1E10 = 0, NERF_LAST_TO_FAR = 1 };
@@ -70,6 +70,13 @@ enum { NERF_LAST_1E10 = 0, NERF_LAST_TO_FAR = 1 };
  * L_pos = 10, L_dir = 4. precision BF16 selects the tensor-core path, built
  * for the page's (W=256, D=8, skip=4) network only (NERF_ERR_UNSUPPORTED
  * otherwise); sigma_act and white_bkgd are applied in compositing.
+ * precision TF32 takes the fp32 blobs and evaluates the same network layer by
+ * layer on the tensor cores: every operand v is split into hi = v rounded to
+ * tf32 and lo = v - hi, each product accumulates hi*hi + hi*lo + lo*hi in
+ * fp32 (the dropped lo*lo term is below 2^-22 of it), so results agree with
+ * FP32 to fp32 rounding level; W in {128, 256}, any D and skip as for FP32
+ * (NERF_ERR_UNSUPPORTED for W = 64). The context then holds an activation
+ * store of up to 2^20 samples (64 + 2.5 W floats each) for the layer outputs.
  * KILONERF ignores D..precision; HASHGRID ignores D..sigma_act and takes
  * precision FP32 (the whole scene function in fp32 on the CUDA cores) or BF16
  * (the encoding and the sigma / rgb heads in fp32, the four hidden layers on the
@@ -220,7 +227,7 @@ NERF_API nerf_status nerf_render_trace(nerf_ctx* ctx, const float* rays_o, const
  * (each mse the mean over n_rays x 3 values; without a fine pass only the
  * coarse term). Writes *out_loss and the gradients of the loss with respect to
  * every parameter of the coarse and fine networks.
- * ctx: NERF_MODEL_MLP with precision FP32 (NERF_ERR_UNSUPPORTED otherwise).
+ * ctx: NERF_MODEL_MLP with precision FP32 or TF32 (NERF_ERR_UNSUPPORTED otherwise).
  * target_rgb: device [n_rays][3] fp32. out_loss: device, one float.
  * grad_coarse, grad_fine: device fp32 buffers of the network's parameter count,
  * laid out like the weight blobs (per Linear: W row-major [N][K], then b);

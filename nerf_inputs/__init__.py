@@ -24,6 +24,7 @@ SIGMA_RELU = 0
 SIGMA_SOFTPLUS = 1
 PREC_FP32 = 0
 PREC_BF16 = 1
+PREC_TF32 = 2   # fp32 weights, layer products on the tensor cores (tf32 hi/lo, 3 passes)
 LAST_DELTA_PAGE = 0   # last interval 1e10 (volume_render on the NeRF page)
 LAST_DELTA_TO_FAR = 1  # last interval reaches t_f
 
@@ -184,12 +185,16 @@ class Workload:
 # The five workloads. Sizes follow the pages' NeRF render (64 + 128 samples per
 # ray, 8x256 network, 800x800 views, near 2 / far 6); the tiny, KiloNeRF and
 # hash-grid shapes are the synthetic stand-ins described in the design notes.
+# small_tf32 is the small workload on the TF32 precision (same weights, camera
+# and samples).
 WORKLOADS = {
     "tiny": Workload("tiny_nerf_32x32", 32, 32, 40.0, seed=0, n_coarse=64, n_fine=0,
                      mlp=MLPShape(D=4, W=64, skip=-1), sigma_act=SIGMA_SOFTPLUS,
                      az=45.0, el=30.0),
     "small": Workload("nerf_200x200_fp32", 200, 200, 250.0, seed=1, n_coarse=64, n_fine=128,
                       mlp=MLPShape(), sigma_scale=1.0),
+    "small_tf32": Workload("nerf_200x200_tf32x3", 200, 200, 250.0, seed=1, n_coarse=64, n_fine=128,
+                           mlp=MLPShape(), sigma_scale=1.0, precision=PREC_TF32),
     "full": Workload("nerf_800x800_bf16", 800, 800, 1000.0, seed=3, n_coarse=64, n_fine=128,
                      mlp=MLPShape(), precision=PREC_BF16, sigma_scale=1.0),
     "kilonerf": Workload("kilonerf_16cubed_800x800", 800, 800, 1000.0, seed=4, model="kilonerf",

@@ -10,7 +10,7 @@ from __future__ import annotations
 import ctypes
 
 from . import _capi
-from ._capi import (NERF_BF16, NERF_FP32, NERF_LAST_1E10, NERF_LAST_TO_FAR, NERF_MODEL_HASHGRID,
+from ._capi import (NERF_BF16, NERF_FP32, NERF_TF32, NERF_LAST_1E10, NERF_LAST_TO_FAR, NERF_MODEL_HASHGRID,
                     NERF_MODEL_KILONERF, NERF_MODEL_MLP, NERF_SIGMA_RELU, NERF_SIGMA_SOFTPLUS,
                     NerfError, nerf_config, nerf_params)
 

@@ -21,7 +21,7 @@ NERF_ERR_DEVICE_FLAG = 6
 
 NERF_MODEL_MLP, NERF_MODEL_KILONERF, NERF_MODEL_HASHGRID = 0, 1, 2
 NERF_SIGMA_RELU, NERF_SIGMA_SOFTPLUS = 0, 1
-NERF_FP32, NERF_BF16 = 0, 1
+NERF_FP32, NERF_BF16, NERF_TF32 = 0, 1, 2
 NERF_LAST_1E10, NERF_LAST_TO_FAR = 0, 1
 TIMED_KINDS = ("network", "composite", "resample", "dir_bias", "march_mask", "march_compact",
                "router", "march_composite")           # NERF_TIMED_* order

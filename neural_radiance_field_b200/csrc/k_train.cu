@@ -21,6 +21,8 @@
 // All GEMMs share one register-blocked core (128 x 128 tiles, 8 x 8 per thread).
 #include <algorithm>
 
+#include <cuda.h>
+
 #include "nerf_internal.cuh"
 #include "tc_ptx.cuh"
 
@@ -317,9 +319,9 @@ __global__ void __launch_bounds__(256, 2) row_gemm_kernel(RowGemm g) {
 // tensor core's order, so results differ from the CUDA-core kernel's in the
 // last bits.
 constexpr int TG_M = 128;                              // rows per tile
-constexpr int TG_KC = 32;                              // K per chunk
-constexpr int TG_A_HALF = TG_M * TG_KC * 4;            // A hi or lo of a chunk, 16 KB
-constexpr int TG_B_HALF = 256 * TG_KC * 4;             // B hi or lo of a chunk (N <= 256), 32 KB
+constexpr int TG_KC = 16;                              // K per chunk
+constexpr int TG_A_HALF = TG_M * TG_KC * 4;            // A hi or lo of a chunk, 8 KB
+constexpr int TG_B_HALF = 256 * TG_KC * 4;             // B hi or lo of a chunk (N <= 256), 16 KB
 constexpr int TG_STAGE = 2 * TG_A_HALF + 2 * TG_B_HALF;
 constexpr int TG_WORKERS = 256;                         // the weight gradient's staging threads
 constexpr int TG_THREADS = TG_WORKERS + 32;             // + its issuer warp
@@ -373,37 +375,53 @@ __device__ __forceinline__ void tg_mma(uint32_t tmem_d, uint64_t a, uint64_t b, 
 }
 
 // Roles of the row GEMM's CTA: warps 0-3 run the epilogue (warp w reads TMEM
-// lane quarter w: one accumulator row per thread), warps 4-11 stage the A rows,
-// warp 12 copies the weights and issues the MMAs. The accumulator is double-
-// buffered in tensor memory (2 N columns), so a tile's epilogue overlaps the
-// next tile's MMAs.
+// lane quarter w: one accumulator row per thread), warps 4-11 split the A rows
+// into the operand stages, warp 12 copies the weights and issues the MMAs, and
+// warp 13 streams the raw A rows by 2-D tensor copies (16 K-columns x 128 rows
+// per chunk) into an 8-slot ring, eight chunks ahead of the MMAs. The operand
+// stages are triple-buffered; the accumulator is double-buffered in tensor
+// memory (2 N columns), so a tile's epilogue overlaps the next tile's MMAs.
 constexpr int RG_EPI = 128;
 constexpr int RG_STG = 256;
-constexpr int RG_THREADS = RG_EPI + RG_STG + 32;
-constexpr size_t RG_SMEM = 2 * TG_STAGE + 128;
+constexpr int RG_THREADS = RG_EPI + RG_STG + 64;
+constexpr int RG_NSTAGE = 3;
+constexpr int RG_RAW = TG_M * TG_KC * 4;                // one raw A chunk, 8 KB
+constexpr int RG_NRAW = 8;
+constexpr int RG_BAR = RG_NSTAGE * TG_STAGE + RG_NRAW * RG_RAW;
+constexpr size_t RG_SMEM = (size_t)RG_BAR + 256;
 
 template <int N>
-__global__ void __launch_bounds__(RG_THREADS, 1) row_gemm_tc_kernel(RowGemm g) {
+__global__ void __launch_bounds__(RG_THREADS, 1) row_gemm_tc_kernel(RowGemm g,
+                                                                    const __grid_constant__ CUtensorMap amap) {
   unsigned* flag = g.flag;
   extern __shared__ __align__(1024) uint8_t tsm[];
-  uint64_t* done = reinterpret_cast<uint64_t*>(tsm + 2 * TG_STAGE);   // [2] MMAs of a stage done
-  uint64_t* bfull = done + 2;                                           // [2] B of a stage landed
-  uint64_t* afull = done + 4;                                           // [2] A of a stage staged
-  uint64_t* accf = done + 6;                                            // [2] accumulator ready
-  uint64_t* acce = done + 8;                                            // [2] accumulator read out
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(done + 10);
+  uint64_t* done = reinterpret_cast<uint64_t*>(tsm + RG_BAR);   // [3] MMAs of a stage done
+  uint64_t* bfull = done + RG_NSTAGE;                            // [3] B of a stage landed
+  uint64_t* afull = bfull + RG_NSTAGE;                           // [3] A of a stage staged
+  uint64_t* accf = afull + RG_NSTAGE;                            // [2] accumulator ready
+  uint64_t* acce = accf + 2;                                     // [2] accumulator read out
+  uint64_t* rfull = acce + 2;                                    // [8] raw A chunk landed
+  uint64_t* rempty = rfull + RG_NRAW;                            // [8] raw A chunk read
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(rempty + RG_NRAW);
   __shared__ int abort_s;
   __shared__ __align__(16) float s_bias[N], s_ev[N];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const uint32_t sbase = tcx::smem_u32(tsm);
+  const uint32_t rawbase = sbase + RG_NSTAGE * TG_STAGE;
   constexpr uint64_t kLimit = 2000000000ull;
   if (tid == 0) {
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < RG_NSTAGE; ++i) {
       tcx::mbar_init(&done[i], 1);
       tcx::mbar_init(&bfull[i], 1);
       tcx::mbar_init(&afull[i], RG_STG / 32);   // one arrival per staging warp
+    }
+    for (int i = 0; i < 2; ++i) {
       tcx::mbar_init(&accf[i], 1);
       tcx::mbar_init(&acce[i], RG_EPI / 32);    // one arrival per epilogue warp
+    }
+    for (int i = 0; i < RG_NRAW; ++i) {
+      tcx::mbar_init(&rfull[i], 1);
+      tcx::mbar_init(&rempty[i], RG_STG / 32);
     }
     abort_s = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -424,8 +442,9 @@ __global__ void __launch_bounds__(RG_THREADS, 1) row_gemm_tc_kernel(RowGemm g) {
   const int nch = g.K / TG_KC;
   const int64_t ntiles = (g.rows + TG_M - 1) / TG_M;
   // this CTA's tiles: blockIdx.x, + gridDim.x, ...; chunk G of the CTA is chunk
-  // G % nch of its tile G / nch and uses operand stage G % 2, whose barriers
-  // complete once per chunk (parity (G / 2) % 2); tile i uses accumulator i % 2
+  // G % nch of its tile G / nch, uses operand stage G % 3 (barrier parity
+  // (G / 3) % 2) and raw slot G % 8 (parity (G / 8) % 2); tile i uses
+  // accumulator i % 2 (parity (i / 2) % 2)
   const int n_my = blockIdx.x < ntiles ? (int)((ntiles - 1 - blockIdx.x) / gridDim.x + 1) : 0;
   const int64_t total = (int64_t)n_my * nch;
   bool ok = true;
@@ -434,8 +453,9 @@ __global__ void __launch_bounds__(RG_THREADS, 1) row_gemm_tc_kernel(RowGemm g) {
     if (lane == 0) {
       constexpr uint32_t idesc = (1u << 4) | (2u << 7) | (2u << 10) | ((uint32_t)(N >> 3) << 17) |
                                  ((uint32_t)(TG_M >> 4) << 24);   // f32 <- tf32 x tf32, M 128
-      auto copy_b = [&](int c, int stage) {
+      auto copy_b = [&](int64_t G) {
         constexpr uint32_t bytes = 2 * N * TG_KC * 4;
+        const int stage = (int)(G % RG_NSTAGE), c = (int)(G % nch);
         asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;"
                      ::"r"(tcx::smem_u32(&bfull[stage])), "r"(bytes) : "memory");
         asm volatile(
@@ -446,9 +466,9 @@ __global__ void __launch_bounds__(RG_THREADS, 1) row_gemm_tc_kernel(RowGemm g) {
             : "memory");
       };
       int64_t G = 0, issued = -1, copied = -1;
-      if (total > 0) {
-        copy_b(0, 0);
-        copied = 0;
+      for (int64_t q = 0; q < 2 && q < total; ++q) {   // the first two chunks' weights
+        copy_b(q);
+        copied = q;
       }
       for (int it = 0; it < n_my && ok; ++it) {
         const int b = it & 1;
@@ -458,8 +478,8 @@ __global__ void __launch_bounds__(RG_THREADS, 1) row_gemm_tc_kernel(RowGemm g) {
         }
         const uint32_t acc = tmem + (uint32_t)(b * N);
         for (int c = 0; c < nch && ok; ++c, ++G) {
-          const int stage = (int)(G & 1);
-          const uint32_t par = (uint32_t)((G >> 1) & 1);
+          const int stage = (int)(G % RG_NSTAGE);
+          const uint32_t par = (uint32_t)((G / RG_NSTAGE) & 1);
           ok = tcx::mbar_wait(&bfull[stage], par, &abort_s, flag, kLimit) &&
                tcx::mbar_wait(&afull[stage], par, &abort_s, flag, kLimit);
           if (!ok) break;
@@ -478,85 +498,112 @@ __global__ void __launch_bounds__(RG_THREADS, 1) row_gemm_tc_kernel(RowGemm g) {
           tcx::mma_commit(&done[stage]);
           if (c == nch - 1) tcx::mma_commit(&accf[b]);
           issued = G;
-          if (G + 1 < total) {
-            // the next chunk's weights (of this tile or the next) go into the
-            // stage that chunk G - 1's MMAs read
+          if (G + 2 < total) {
+            // chunk G + 2's weights go into the stage that chunk G - 1's MMAs read
             if (G >= 1)
-              ok = tcx::mbar_wait(&done[stage ^ 1], (uint32_t)(((G - 1) >> 1) & 1), &abort_s, flag, kLimit);
+              ok = tcx::mbar_wait(&done[(G - 1) % RG_NSTAGE], (uint32_t)(((G - 1) / RG_NSTAGE) & 1),
+                                  &abort_s, flag, kLimit);
             if (ok) {
-              copy_b(c + 1 < nch ? c + 1 : 0, stage ^ 1);
-              copied = G + 1;
+              copy_b(G + 2);
+              copied = G + 2;
             }
           }
         }
       }
       // drain before TMEM and shared memory are given up (not stopped by an
-      // abort: the MMAs and the weight copy already issued must land first)
+      // abort: the MMAs and the weight copies already issued must land first)
       const uint64_t t0 = tcx::globaltimer();
       if (issued >= 0)
-        while (!tcx::mbar_try(&done[issued & 1], (uint32_t)((issued >> 1) & 1)) &&
+        while (!tcx::mbar_try(&done[issued % RG_NSTAGE], (uint32_t)((issued / RG_NSTAGE) & 1)) &&
                tcx::globaltimer() - t0 < kLimit) {
         }
-      if (copied >= 0)
-        while (!tcx::mbar_try(&bfull[copied & 1], (uint32_t)((copied >> 1) & 1)) &&
+      for (int64_t q = copied; q >= 0 && q > copied - 2; --q)
+        while (!tcx::mbar_try(&bfull[q % RG_NSTAGE], (uint32_t)((q / RG_NSTAGE) & 1)) &&
+               tcx::globaltimer() - t0 < kLimit) {
+        }
+    }
+    __syncwarp();
+  } else if (warp == (RG_EPI + RG_STG) / 32 + 1) {
+    // ------------------------------------------------------------- raw A producer
+    if (lane == 0) {
+      int64_t loaded = -1;
+      for (int64_t G = 0; G < total && ok; ++G) {
+        const int slot = (int)(G % RG_NRAW);
+        if (G >= RG_NRAW &&
+            !tcx::mbar_wait(&rempty[slot], (uint32_t)((G / RG_NRAW - 1) & 1), &abort_s, flag, kLimit)) {
+          ok = false;
+          break;
+        }
+        const int64_t it = G / nch;
+        const int c = (int)(G - it * nch);
+        const int k = c * TG_KC;
+        const int col = k < g.a_split ? g.a0 + k : g.a1 + k - g.a_split;
+        const int row = (int)((blockIdx.x + it * gridDim.x) * TG_M);
+        asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;"
+                     ::"r"(tcx::smem_u32(&rfull[slot])), "r"(RG_RAW) : "memory");
+        asm volatile(
+            "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
+            ::"r"(rawbase + slot * RG_RAW), "l"(reinterpret_cast<uint64_t>(&amap)), "r"(col), "r"(row),
+              "r"(tcx::smem_u32(&rfull[slot]))
+            : "memory");
+        loaded = G;
+      }
+      // the copies in flight land before shared memory is given up
+      const uint64_t t0 = tcx::globaltimer();
+      for (int64_t q = loaded; q >= 0 && q > loaded - RG_NRAW; --q)
+        while (!tcx::mbar_try(&rfull[q % RG_NRAW], (uint32_t)((q / RG_NRAW) & 1)) &&
                tcx::globaltimer() - t0 < kLimit) {
         }
     }
     __syncwarp();
   } else if (warp >= RG_EPI / 32) {
     // ------------------------------------------------------------- staging warps
-    // thread st stages row st / 2, K columns [16 (st % 2), +16) of a chunk; the
-    // rows are fetched into registers two chunks ahead (the activation store
-    // streams from DRAM), split and stored once their stage is free
+    // per chunk, thread st takes the 16-byte pieces i = st and st + 256 of the
+    // raw chunk (row i / 4, K columns 4 (i % 4) ..): a warp reads 512
+    // contiguous bytes and writes four 128-byte core-matrix rows. A warp that
+    // broke out on an abort never arrives again, so the other roles' waits
+    // end by the abort word.
     const int st = tid - RG_EPI;
-    const int arow = st >> 1, akh = (st & 1) * 16;
-    auto fetch_a = [&](int64_t G, float4 (&v)[4]) {
-      const int64_t it = G / nch;
-      const int c = (int)(G - it * nch);
-      const int64_t ar = (blockIdx.x + it * gridDim.x) * TG_M + arow;
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const int k = c * TG_KC + akh + 4 * q;
-        const int col = k < g.a_split ? g.a0 + k : g.a1 + k - g.a_split;
-        v[q] = (G < total && ar < g.rows) ? load4(g.A + ar * g.lda + col, g.a_vec, true, true, true, true)
-                                          : make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int64_t G = 0; G < total && ok; ++G) {
+      const int slot = (int)(G % RG_NRAW), stage = (int)(G % RG_NSTAGE);
+      bool w = tcx::mbar_wait(&rfull[slot], (uint32_t)((G / RG_NRAW) & 1), &abort_s, flag, kLimit);
+      if (!__all_sync(0xffffffffu, w)) {
+        ok = false;
+        break;
       }
-    };
-    auto put_a = [&](int stage, const float4 (&v)[4]) {
+      const float* raw = reinterpret_cast<const float*>(tsm + RG_NSTAGE * TG_STAGE + slot * RG_RAW);
+      const float4 v0 = *reinterpret_cast<const float4*>(raw + 4 * st);
+      const float4 v1 = *reinterpret_cast<const float4*>(raw + 4 * (st + 256));
+      w = G < RG_NSTAGE || tcx::mbar_wait(&done[stage], (uint32_t)((G / RG_NSTAGE - 1) & 1), &abort_s, flag, kLimit);
+      if (!__all_sync(0xffffffffu, w)) {
+        ok = false;
+        break;
+      }
       const uint32_t sa = sbase + stage * TG_STAGE;
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
+      for (int h = 0; h < 2; ++h) {
+        const int i = st + 256 * h;
+        const float4 v = h ? v1 : v0;
         float hi[4], lo[4];
-        tg_split(v[q].x, hi[0], lo[0]);
-        tg_split(v[q].y, hi[1], lo[1]);
-        tg_split(v[q].z, hi[2], lo[2]);
-        tg_split(v[q].w, hi[3], lo[3]);
-        const uint32_t o = tg_off(arow, akh + 4 * q, TG_M);
+        tg_split(v.x, hi[0], lo[0]);
+        tg_split(v.y, hi[1], lo[1]);
+        tg_split(v.z, hi[2], lo[2]);
+        tg_split(v.w, hi[3], lo[3]);
+        const uint32_t o = tg_off(i >> 2, 4 * (i & 3), TG_M);
         tcx::st_shared_v4(sa + o, __float_as_uint(hi[0]), __float_as_uint(hi[1]),
                           __float_as_uint(hi[2]), __float_as_uint(hi[3]));
         tcx::st_shared_v4(sa + TG_A_HALF + o, __float_as_uint(lo[0]), __float_as_uint(lo[1]),
                           __float_as_uint(lo[2]), __float_as_uint(lo[3]));
       }
-    };
-    // chunk G from `cur` into stage G % 2 (free once chunk G - 2's MMAs are
-    // done), then chunk G + 2 fetched into `cur`: two register sets alternate
-    auto stage_chunk = [&](int64_t G, float4 (&cur)[4]) -> bool {
-      const int stage = (int)(G & 1);
-      const bool w = G < 2 || tcx::mbar_wait(&done[stage], (uint32_t)(((G - 2) >> 1) & 1), &abort_s, flag, kLimit);
-      if (!__all_sync(0xffffffffu, w)) return false;   // the warp leaves together
-      put_a(stage, cur);
       tcx::fence_async_smem();
       __syncwarp();
-      if (lane == 0) tcx::mbar_arrive(&afull[stage]);
-      fetch_a(G + 2, cur);
-      return true;
-    };
-    float4 va[4], vb[4];
-    fetch_a(0, va);
-    fetch_a(1, vb);
-    for (int64_t G = 0; G < total && ok; G += 2) {
-      ok = stage_chunk(G, va);
-      if (ok && G + 1 < total) ok = stage_chunk(G + 1, vb);
+      // the raw slot is released only now: every lane's stores above consumed
+      // its loads of the slot, so the next tensor copy into it cannot overtake
+      // a read still in flight
+      if (lane == 0) {
+        tcx::mbar_arrive(&afull[stage]);
+        tcx::mbar_arrive(&rempty[slot]);
+      }
     }
   } else {
     // ------------------------------------------------------------- epilogue warps
@@ -1000,7 +1047,7 @@ wgrad_head_kernel(const float* __restrict__ A, int64_t lda, const float* __restr
 // rounding of the fused forward kernel's prologue.
 __global__ void encode_store_kernel(const float* __restrict__ o, const float* __restrict__ d,
                                     int64_t R, SampleSpec ss, float* __restrict__ save,
-                                    int64_t ldc) {
+                                    int64_t ldc, int64_t ray0) {
   const int64_t row = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (row >= R * ss.S) return;
   float x[3];
@@ -1011,7 +1058,7 @@ __global__ void encode_store_kernel(const float* __restrict__ o, const float* __
     const int s = (int)(row % ss.S);
     float t;
     if (ss.mode == SAMPLES_STRATIFIED) {
-      const uint32_t m = ss.perturb ? draw_bits(ss.key, (uint64_t)ray, 0, (uint32_t)s) : 0u;
+      const uint32_t m = ss.perturb ? draw_bits(ss.key, (uint64_t)(ray0 + ray), 0, (uint32_t)s) : 0u;
       t = stratified_t(ss.near, ss.step, s, m, ss.perturb != 0);
     } else {
       t = ss.t[row];
@@ -1138,6 +1185,32 @@ int sm_count() {
   return n;
 }
 
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+// fp32 matrix of `rows` rows of `ld` floats, boxes of TG_KC columns x TG_M rows
+// (rows past the end read as zero).
+cudaError_t encode_rows_map(CUtensorMap* m, const float* base, int64_t ld, int64_t rows) {
+  static EncodeTiledFn encode = nullptr;
+  if (!encode) {
+    cudaDriverEntryPointQueryResult q;
+    void* fn = nullptr;
+    cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q);
+    if (e != cudaSuccess || q != cudaDriverEntryPointSuccess || !fn) return cudaErrorNotSupported;
+    encode = reinterpret_cast<EncodeTiledFn>(fn);
+  }
+  const cuuint64_t dims[2] = {(cuuint64_t)ld, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)ld * 4};
+  const cuuint32_t box[2] = {TG_KC, TG_M};
+  const cuuint32_t estr[2] = {1, 1};
+  CUresult r = encode(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float*>(base), dims, strides,
+                      box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
 cudaError_t row_gemm(RowGemm g, cudaStream_t st) {
   if (g.rows == 0) return cudaSuccess;
   if (g.K % GK || g.a_split % GK || g.n_out % 4 || g.ldo % 4 || !al16(g.out))
@@ -1150,7 +1223,11 @@ cudaError_t row_gemm(RowGemm g, cudaStream_t st) {
   const bool side_vec = g.ldo % 4 == 0 && !(g.mask && g.row_bias) &&
                         (!g.mask || (al16(g.mask) && g.ldm % 4 == 0)) &&
                         (!g.row_bias || (al16(g.row_bias) && g.n_out % 4 == 0));
-  if (g.bsplit && side_vec && g.K % TG_KC == 0 && (g.n_out == 128 || g.n_out == 256) &&
+  // (the raw A chunks are 2-D tensor copies: 16-byte aligned rows and column
+  // offsets on whole chunks)
+  const bool a_tma = al16(g.A) && g.lda % 4 == 0 && g.a0 % TG_KC == 0 && g.a1 % TG_KC == 0 &&
+                     g.a_split % TG_KC == 0 && g.rows < (int64_t)1 << 31;
+  if (g.bsplit && side_vec && a_tma && g.K % TG_KC == 0 && (g.n_out == 128 || g.n_out == 256) &&
       (int64_t)g.K * g.n_out * 2 <= TRAIN_BSPLIT) {
     static bool attr_set[2] = {false, false};
     const int wide = g.n_out == 256;
@@ -1162,15 +1239,18 @@ cudaError_t row_gemm(RowGemm g, cudaStream_t st) {
       if (e != cudaSuccess) return e;
       attr_set[wide] = true;
     }
+    CUtensorMap amap;
+    cudaError_t e = encode_rows_map(&amap, g.A, g.lda, g.rows);
+    if (e != cudaSuccess) return e;
     const int64_t nb = (int64_t)g.K * g.n_out;
     split_b_kernel<<<(unsigned)std::min<int64_t>(blocks_for(nb, 256), 1024), 256, 0, st>>>(
         g.B, g.ldb, g.K, g.n_out, g.bsplit);
-    cudaError_t e = cudaGetLastError();
+    e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     // persistent: one CTA per SM walks the row tiles
     const unsigned grid = (unsigned)std::min<int64_t>(blocks_for(g.rows, TG_M), sm_count());
-    if (wide) row_gemm_tc_kernel<256><<<grid, RG_THREADS, RG_SMEM, st>>>(g);
-    else row_gemm_tc_kernel<128><<<grid, RG_THREADS, RG_SMEM, st>>>(g);
+    if (wide) row_gemm_tc_kernel<256><<<grid, RG_THREADS, RG_SMEM, st>>>(g, amap);
+    else row_gemm_tc_kernel<128><<<grid, RG_THREADS, RG_SMEM, st>>>(g, amap);
     return cudaGetLastError();
   }
   row_gemm_kernel<<<dim3(blocks_for(g.rows, GT), blocks_for(g.n_out, GT)), 256, 0, st>>>(g);
@@ -1246,14 +1326,16 @@ cudaError_t launch_composite_bw(const float* raw, const SampleSpec& ss, const fl
 cudaError_t mlp_forward_train_fp32(const PackedFp32& p, const float* pk, const float* dir_bias,
                                    const float* o, const float* d, int64_t R,
                                    const SampleSpec& ss, float* raw, float* save, float* bsplit,
-                                   unsigned* flag, cudaStream_t st) {
+                                   unsigned* flag, cudaStream_t st, int64_t ray0, bool compact) {
   const int D = p.D, W = p.W, Wh = W / 2;
   const int64_t rows = R * ss.S;
   if (rows == 0) return cudaSuccess;
-  const int64_t ldc = 64 + (int64_t)(D + 1) * W + Wh;
-  auto hcol = [&](int l) { return 64 + l * W; };
-  const int feat_col = hcol(D), hdir_col = hcol(D + 1);
-  encode_store_kernel<<<blocks_for(rows, 128), 128, 0, st>>>(o, d, R, ss, save, ldc);
+  const int64_t ldc = compact ? compact_ldc(W) : 64 + (int64_t)(D + 1) * W + Wh;
+  // compact: layer l writes slot l % 2 and reads slot (l - 1) % 2; the feature
+  // layer writes slot D % 2, keeping h_{D-1} (slot (D - 1) % 2) for the sigma head
+  auto hcol = [&](int l) { return compact ? 64 + (l & 1) * W : 64 + l * W; };
+  const int feat_col = hcol(D), hdir_col = compact ? 64 + 2 * W : hcol(D + 1);
+  encode_store_kernel<<<blocks_for(rows, 128), 128, 0, st>>>(o, d, R, ss, save, ldc, ray0);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   for (int l = 0; l < D && e == cudaSuccess; ++l) {

@@ -153,10 +153,12 @@ nerf_status nerf_create(const nerf_config* cfg, nerf_ctx** out) {
     if (!shape_ok)
       return fail(nullptr, NERF_ERR_UNSUPPORTED,
                   "network must have W in {64, 128, 256}, D in 1..8 and skip -1 or in 0..D-2");
-    if (c.precision != NERF_FP32 && c.precision != NERF_BF16)
-      return fail(nullptr, NERF_ERR_INVALID_ARG, "precision must be FP32 or BF16");
+    if (c.precision != NERF_FP32 && c.precision != NERF_BF16 && c.precision != NERF_TF32)
+      return fail(nullptr, NERF_ERR_INVALID_ARG, "precision must be FP32, BF16 or TF32");
     if (c.precision == NERF_BF16 && !big)
       return fail(nullptr, NERF_ERR_UNSUPPORTED, "BF16 tensor-core path needs W=256, D=8");
+    if (c.precision == NERF_TF32 && c.W == 64)
+      return fail(nullptr, NERF_ERR_UNSUPPORTED, "TF32 tensor-core layers need W in {128, 256}");
   } else if (c.model == NERF_MODEL_KILONERF || c.model == NERF_MODEL_HASHGRID) {
     if (c.model == NERF_MODEL_HASHGRID && c.precision != NERF_FP32 && c.precision != NERF_BF16)
       return fail(nullptr, NERF_ERR_INVALID_ARG, "precision must be FP32 or BF16");
@@ -184,6 +186,12 @@ nerf_status nerf_create(const nerf_config* cfg, nerf_ctx** out) {
   ok &= dalloc(&ctx->d_flag, 1) == cudaSuccess;
   if (ok) ok &= cudaMemset(ctx->d_flag, 0, sizeof(unsigned)) == cudaSuccess;
   if (ok && c.precision == NERF_BF16) ok &= tc_alloc(ctx) == cudaSuccess;
+  if (ok && c.precision == NERF_TF32) {
+    // the layer outputs of a sub-batch of up to 2^20 samples
+    ctx->fw_rows = std::min<int64_t>(R * S, (int64_t)1 << 20);
+    ok &= dalloc(&ctx->fw_save, (size_t)(ctx->fw_rows * compact_ldc(c.W))) == cudaSuccess;
+    ok &= dalloc(&ctx->tr_bsplit, (size_t)TRAIN_BSPLIT) == cudaSuccess;
+  }
   if (!ok) {
     cudaGetLastError();
     nerf_destroy(ctx);
@@ -207,6 +215,7 @@ nerf_status nerf_destroy(nerf_ctx* ctx) {
   cudaFree(ctx->tr_draw);
   cudaFree(ctx->tr_tmp);
   cudaFree(ctx->tr_bsplit);
+  cudaFree(ctx->fw_save);
   cudaFree(ctx->tr_loss);
   free_march(ctx);
   if (ctx->ev) {
@@ -299,6 +308,21 @@ nerf_status run_network(nerf_ctx* ctx, const void* blob, const float* o, const f
   if (save) {
     NERF_CHECK_LAUNCH(ctx, mlp_forward_train_fp32(ctx->plan, ctx->packed, ctx->dir_bias, o, d, R,
                                                   ss, raw, save, ctx->tr_bsplit, ctx->d_flag, st));
+  } else if (c.precision == NERF_TF32) {
+    // layer by layer on the tensor cores, in sub-batches of whole rays that fit
+    // the activation store
+    const int64_t per = std::max<int64_t>(1, ctx->fw_rows / ss.S);
+    for (int64_t r0 = 0; r0 < R; r0 += per) {
+      const int64_t n = std::min(per, R - r0);
+      SampleSpec sub = ss;
+      if (ss.mode == SAMPLES_GIVEN_T) sub.t = ss.t + r0 * ss.S;
+      if (ss.mode == SAMPLES_GIVEN_X) sub.t = ss.t + r0 * ss.S * 3;
+      NERF_CHECK_LAUNCH(ctx, mlp_forward_train_fp32(ctx->plan, ctx->packed,
+                                                    ctx->dir_bias + r0 * (c.W / 2), o + r0 * 3,
+                                                    d + r0 * 3, n, sub, raw + r0 * ss.S * 4,
+                                                    ctx->fw_save, ctx->tr_bsplit, ctx->d_flag, st,
+                                                    r0, true));
+    }
   } else {
     NERF_CHECK_LAUNCH(ctx, launch_mlp_fp32(ctx->plan, ctx->packed, ctx->dir_bias, o, d, R, ss, raw,
                                            st));
@@ -473,7 +497,7 @@ nerf_status nerf_loss_grad(nerf_ctx* ctx, const float* rays_o, const float* rays
                            float* grad_coarse, float* grad_fine, void* stream) {
   if (!ctx) return fail(nullptr, NERF_ERR_INVALID_ARG, "ctx is NULL");
   const nerf_config& c = ctx->cfg;
-  if (c.model != NERF_MODEL_MLP || c.precision != NERF_FP32)
+  if (c.model != NERF_MODEL_MLP || (c.precision != NERF_FP32 && c.precision != NERF_TF32))
     return fail(ctx, NERF_ERR_UNSUPPORTED, "nerf_loss_grad needs an fp32 NERF_MODEL_MLP context");
   if (!rays_o || !rays_d || !params || !target_rgb || !out_loss || !grad_coarse ||
       (n_fine > 0 && !grad_fine))
@@ -500,12 +524,11 @@ nerf_status nerf_loss_grad(nerf_ctx* ctx, const float* rays_o, const float* rays
     ok &= dalloc(&ctx->tr_draw, (size_t)(rows * 4)) == cudaSuccess;
     ok &= dalloc(&ctx->tr_tmp, (size_t)(2 * rows * W + c.max_rays * (W / 2 + dir_ch))) == cudaSuccess;
     ok &= dalloc(&ctx->tr_loss, (size_t)(2 * c.max_rays)) == cudaSuccess;
-    ok &= dalloc(&ctx->tr_bsplit, (size_t)TRAIN_BSPLIT) == cudaSuccess;
+    if (ok && !ctx->tr_bsplit) ok &= dalloc(&ctx->tr_bsplit, (size_t)TRAIN_BSPLIT) == cudaSuccess;
     if (!ok) {
       cudaGetLastError();
       cudaFree(ctx->tr_save); cudaFree(ctx->tr_draw); cudaFree(ctx->tr_tmp); cudaFree(ctx->tr_loss);
-      cudaFree(ctx->tr_bsplit);
-      ctx->tr_save = ctx->tr_draw = ctx->tr_tmp = ctx->tr_loss = ctx->tr_bsplit = nullptr;
+      ctx->tr_save = ctx->tr_draw = ctx->tr_tmp = ctx->tr_loss = nullptr;
       return fail(ctx, NERF_ERR_OOM, "training workspace allocation failed");
     }
   }

@@ -26,6 +26,8 @@ struct nerf_ctx {
   float* tr_tmp = nullptr;     // backward scratch
   float* tr_loss = nullptr;    // [2 max_rays] per-ray loss terms
   float* tr_bsplit = nullptr;  // split weights of one tensor-core row GEMM (TRAIN_BSPLIT floats)
+  float* fw_save = nullptr;    // precision TF32: [fw_rows][64 + 2 W + W/2] layer outputs of a sub-batch
+  int64_t fw_rows = 0;
 
   // kernel timing (nerf_timing_enable / nerf_timing_read / nerf_timing_read_kinds)
   bool timing = false;

@@ -143,10 +143,16 @@ cudaError_t launch_composite_bw(const float* raw, const SampleSpec& ss, const fl
 // K = 256 + 64, 256 outputs) for the tensor-core row GEMMs' split weights;
 // flag: the context's error flag.
 constexpr int64_t TRAIN_BSPLIT = (int64_t)320 * 256 * 2;
+// ray0: index of the first ray in the whole batch (the stratified draws are
+// keyed by it); compact: the store keeps only what the forward needs,
+// [gamma(x) 64 | two ping-pong hidden slots W | h_dir W/2] (row stride
+// compact_ldc), instead of every layer's output for the backward.
 cudaError_t mlp_forward_train_fp32(const PackedFp32& p, const float* packed, const float* dir_bias,
                                    const float* o, const float* d, int64_t R,
                                    const SampleSpec& ss, float* raw, float* save, float* bsplit,
-                                   unsigned* flag, cudaStream_t st);
+                                   unsigned* flag, cudaStream_t st, int64_t ray0 = 0,
+                                   bool compact = false);
+inline int64_t compact_ldc(int W) { return 64 + 2 * (int64_t)W + W / 2; }
 cudaError_t mlp_backward_fp32(const PackedFp32& p, int L_dir, const float* w, const float* save,
                               int64_t R, int S, const float* d, const float* d_raw,
                               float* grad, float* tmp, float* bsplit, unsigned* flag,

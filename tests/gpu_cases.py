@@ -22,7 +22,7 @@ TOL_BF16 = dict(rgb=2e-2, acc=2e-2, depth_rel=1e-3)      # depth: 1e-3 * (far - 
 # K = 256..320 fp32 dot-product chain, ~K * 2^-24 relative per layer on O(1)
 # values, with margin. bf16: operands and activations rounded to bf16 (2^-9
 # relative) through 10 layers, accumulated with random signs, with margin.
-RAW_BOUND = {S.PREC_FP32: 5e-5, S.PREC_BF16: 5e-3}
+RAW_BOUND = {S.PREC_FP32: 5e-5, S.PREC_BF16: 5e-3, S.PREC_TF32: 5e-5}
 # Unit bars of the compositing and sampling stages on identical inputs (fp32
 # exp/expm1 and a 192-term sum; two rounded operands and three operations).
 TOL_COMPOSITE = dict(rgb=1e-5, acc=1e-5, depth=1e-4)

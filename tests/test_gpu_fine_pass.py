@@ -40,6 +40,12 @@ def test_staged_fine_pass_200x200_fp32(torch):
     staged_fine_pass(S.WORKLOADS["small"], 384, 1)
 
 
+def test_staged_fine_pass_200x200_tf32(torch):
+    """The same with precision TF32: the fine network's 40,000 x 192 samples run
+    in eight sub-batches of the activation store."""
+    staged_fine_pass(S.WORKLOADS["small_tf32"], 384, 1)
+
+
 def test_staged_fine_pass_unperturbed_to_far_white(torch):
     """Evenly spaced draws and jitter-free strata, the last interval reaching
     far (the closed-form reading), white background; ragged 21x23 image."""

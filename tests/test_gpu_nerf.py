@@ -74,7 +74,7 @@ def test_positional_encoding(torch, L):
 
 # ---------------------------------------------------------------- a5 MLP
 
-@pytest.mark.parametrize("key", ["tiny", "small", "full"])
+@pytest.mark.parametrize("key", ["tiny", "small", "small_tf32", "full"])
 def test_mlp_rows(torch, key):
     wl = S.WORKLOADS[key]
     cw, _ = oracle_weights(wl)
@@ -197,6 +197,34 @@ def test_e2e_small_fp32_coarse_pass(torch):
     wl = dataclasses.replace(S.WORKLOADS["small"], n_fine=0)
     gpu, ref = _render_and_oracle(wl, 2000, 0)
     check_rays(wl, gpu, ref, "200x200 fp32 coarse pass")
+
+
+def test_e2e_small_tf32_coarse_pass(torch):
+    """The same frame with precision TF32 (the layer GEMMs on the tensor cores,
+    three tf32 MMAs per product), 2000 sampled rays at the fp32 bar. The 40,000
+    rays run in three sub-batches of 16,384 + 16,384 + 7,232 (the activation
+    store's 2^20 samples), so the stratified draws of later sub-batches are
+    keyed by their index in the whole batch."""
+    wl = dataclasses.replace(S.WORKLOADS["small_tf32"], n_fine=0)
+    gpu, ref = _render_and_oracle(wl, 2000, 0)
+    check_rays(wl, gpu, ref, "200x200 tf32x3 coarse pass")
+
+
+def test_tf32_matches_fp32_render(torch):
+    """The TF32 and FP32 precisions render the same 48x48 coarse frame (weights,
+    samples and draws shared; the last interval reaching far, so no ray sits on
+    the ReLU kink) to within the fp32 bar of each other on every ray."""
+    outs = []
+    for key in ("small", "small_tf32"):
+        wl = dataclasses.replace(S.WORKLOADS[key], H=48, W=48, n_fine=0,
+                                 last_delta=S.LAST_DELTA_TO_FAR)
+        o, d = rays_for(wl)
+        cw, fw = oracle_weights(wl)
+        outs.append(render_gpu(wl, o, d, weights_tensor(cw, wl.precision), None))
+    trgb, tacc, tdep = tolerances(S.WORKLOADS["small"])
+    err = ray_errors(outs[1], outs[0])
+    print("[tf32 vs fp32 48x48] " + ", ".join(f"{k} {v.max():.2e}" for k, v in err.items()))
+    assert within(err, dict(rgb=trgb, acc=tacc, depth=tdep)).all()
 
 
 def free_running_statistic(wl, n_check, seed_ids, perturb=1):
