@@ -374,16 +374,26 @@ __device__ __forceinline__ void tg_mma(uint32_t tmem_d, uint64_t a, uint64_t b, 
       ::"r"(tmem_d), "l"(a), "l"(b), "r"(idesc), "r"(accum));
 }
 
-// Roles of the row GEMM's CTA: warps 0-3 run the epilogue (warp w reads TMEM
-// lane quarter w: one accumulator row per thread), warps 4-11 split the A rows
-// into the operand stages, warp 12 copies the weights and issues the MMAs, and
-// warp 13 streams the raw A rows by 2-D tensor copies (16 K-columns x 128 rows
-// per chunk) into an 8-slot ring, eight chunks ahead of the MMAs. The operand
-// stages are triple-buffered; the accumulator is double-buffered in tensor
-// memory (2 N columns), so a tile's epilogue overlaps the next tile's MMAs.
+// Roles of the row GEMM's CTA (16 warps):
+//   warps 0-3    epilogue: warp w reads TMEM lane quarter w (one accumulator row
+//                per lane), 32 columns at a time, and writes each row's block
+//                as whole 128-byte lines in 16-byte pieces (a transpose
+//                through shared memory for fully coalesced rows measured four
+//                times slower);
+//   warps 4-11   split the raw A rows into the operand stages;
+//   warp 12      issues the MMAs: one barrier wait per chunk, six MMAs, a commit;
+//   warp 13      streams the raw A rows by 2-D tensor copies (16 K-columns x
+//                128 rows per chunk) into an 8-slot ring;
+//   warps 14-15  copy the split weights of the even / odd chunks (one bulk copy
+//                each; a copy takes the issuing thread about 600 cycles, so two
+//                threads share the chunk stream).
+// The operand stages are triple-buffered; a stage is full when the eight
+// staging warps and the weight copy have arrived. The accumulator is double-
+// buffered in tensor memory (2 N columns), so a tile's epilogue overlaps the
+// next tile's MMAs.
 constexpr int RG_EPI = 128;
 constexpr int RG_STG = 256;
-constexpr int RG_THREADS = RG_EPI + RG_STG + 64;
+constexpr int RG_THREADS = RG_EPI + RG_STG + 128;
 constexpr int RG_NSTAGE = 3;
 constexpr int RG_RAW = TG_M * TG_KC * 4;                // one raw A chunk, 8 KB
 constexpr int RG_NRAW = 8;
@@ -396,9 +406,8 @@ __global__ void __launch_bounds__(RG_THREADS, 1) row_gemm_tc_kernel(RowGemm g,
   unsigned* flag = g.flag;
   extern __shared__ __align__(1024) uint8_t tsm[];
   uint64_t* done = reinterpret_cast<uint64_t*>(tsm + RG_BAR);   // [3] MMAs of a stage done
-  uint64_t* bfull = done + RG_NSTAGE;                            // [3] B of a stage landed
-  uint64_t* afull = bfull + RG_NSTAGE;                           // [3] A of a stage staged
-  uint64_t* accf = afull + RG_NSTAGE;                            // [2] accumulator ready
+  uint64_t* full = done + RG_NSTAGE;                             // [3] stage staged (A and B)
+  uint64_t* accf = full + RG_NSTAGE;                             // [2] accumulator ready
   uint64_t* acce = accf + 2;                                     // [2] accumulator read out
   uint64_t* rfull = acce + 2;                                    // [8] raw A chunk landed
   uint64_t* rempty = rfull + RG_NRAW;                            // [8] raw A chunk read
@@ -412,12 +421,11 @@ __global__ void __launch_bounds__(RG_THREADS, 1) row_gemm_tc_kernel(RowGemm g,
   if (tid == 0) {
     for (int i = 0; i < RG_NSTAGE; ++i) {
       tcx::mbar_init(&done[i], 1);
-      tcx::mbar_init(&bfull[i], 1);
-      tcx::mbar_init(&afull[i], RG_STG / 32);   // one arrival per staging warp
+      tcx::mbar_init(&full[i], RG_STG / 32 + 1);   // the staging warps and the weight copy
     }
     for (int i = 0; i < 2; ++i) {
       tcx::mbar_init(&accf[i], 1);
-      tcx::mbar_init(&acce[i], RG_EPI / 32);    // one arrival per epilogue warp
+      tcx::mbar_init(&acce[i], RG_EPI / 32);       // one arrival per epilogue warp
     }
     for (int i = 0; i < RG_NRAW; ++i) {
       tcx::mbar_init(&rfull[i], 1);
@@ -448,28 +456,13 @@ __global__ void __launch_bounds__(RG_THREADS, 1) row_gemm_tc_kernel(RowGemm g,
   const int n_my = blockIdx.x < ntiles ? (int)((ntiles - 1 - blockIdx.x) / gridDim.x + 1) : 0;
   const int64_t total = (int64_t)n_my * nch;
   bool ok = true;
-  if (warp == (RG_EPI + RG_STG) / 32) {
-    // ------------------------------------------------------------- issuer warp
+  constexpr int W_ISSUE = (RG_EPI + RG_STG) / 32, W_APROD = W_ISSUE + 1, W_BPROD = W_ISSUE + 2;
+  if (warp == W_ISSUE) {
+    // ------------------------------------------------------------- MMA issuer
     if (lane == 0) {
       constexpr uint32_t idesc = (1u << 4) | (2u << 7) | (2u << 10) | ((uint32_t)(N >> 3) << 17) |
                                  ((uint32_t)(TG_M >> 4) << 24);   // f32 <- tf32 x tf32, M 128
-      auto copy_b = [&](int64_t G) {
-        constexpr uint32_t bytes = 2 * N * TG_KC * 4;
-        const int stage = (int)(G % RG_NSTAGE), c = (int)(G % nch);
-        asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;"
-                     ::"r"(tcx::smem_u32(&bfull[stage])), "r"(bytes) : "memory");
-        asm volatile(
-            "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
-            ::"r"(sbase + stage * TG_STAGE + 2 * TG_A_HALF),
-              "l"(g.bsplit + (int64_t)c * 2 * N * TG_KC), "r"(bytes),
-              "r"(tcx::smem_u32(&bfull[stage]))
-            : "memory");
-      };
-      int64_t G = 0, issued = -1, copied = -1;
-      for (int64_t q = 0; q < 2 && q < total; ++q) {   // the first two chunks' weights
-        copy_b(q);
-        copied = q;
-      }
+      int64_t G = 0, issued = -1;
       for (int it = 0; it < n_my && ok; ++it) {
         const int b = it & 1;
         if (it >= 2 && !tcx::mbar_wait(&acce[b], (uint32_t)(((it >> 1) - 1) & 1), &abort_s, flag, kLimit)) {
@@ -477,12 +470,12 @@ __global__ void __launch_bounds__(RG_THREADS, 1) row_gemm_tc_kernel(RowGemm g,
           break;
         }
         const uint32_t acc = tmem + (uint32_t)(b * N);
-        for (int c = 0; c < nch && ok; ++c, ++G) {
+        for (int c = 0; c < nch; ++c, ++G) {
           const int stage = (int)(G % RG_NSTAGE);
-          const uint32_t par = (uint32_t)((G / RG_NSTAGE) & 1);
-          ok = tcx::mbar_wait(&bfull[stage], par, &abort_s, flag, kLimit) &&
-               tcx::mbar_wait(&afull[stage], par, &abort_s, flag, kLimit);
-          if (!ok) break;
+          if (!tcx::mbar_wait(&full[stage], (uint32_t)((G / RG_NSTAGE) & 1), &abort_s, flag, kLimit)) {
+            ok = false;
+            break;
+          }
           tcx::fence_after();
           const uint32_t sa = sbase + stage * TG_STAGE;
           const uint64_t ah = tcx::sdesc(sa, TG_M * 16, 128), al = tcx::sdesc(sa + TG_A_HALF, TG_M * 16, 128);
@@ -498,32 +491,55 @@ __global__ void __launch_bounds__(RG_THREADS, 1) row_gemm_tc_kernel(RowGemm g,
           tcx::mma_commit(&done[stage]);
           if (c == nch - 1) tcx::mma_commit(&accf[b]);
           issued = G;
-          if (G + 2 < total) {
-            // chunk G + 2's weights go into the stage that chunk G - 1's MMAs read
-            if (G >= 1)
-              ok = tcx::mbar_wait(&done[(G - 1) % RG_NSTAGE], (uint32_t)(((G - 1) / RG_NSTAGE) & 1),
-                                  &abort_s, flag, kLimit);
-            if (ok) {
-              copy_b(G + 2);
-              copied = G + 2;
-            }
-          }
         }
       }
-      // drain before TMEM and shared memory are given up (not stopped by an
-      // abort: the MMAs and the weight copies already issued must land first)
+      // the MMAs already issued land before TMEM is freed, abort or not
       const uint64_t t0 = tcx::globaltimer();
       if (issued >= 0)
         while (!tcx::mbar_try(&done[issued % RG_NSTAGE], (uint32_t)((issued / RG_NSTAGE) & 1)) &&
                tcx::globaltimer() - t0 < kLimit) {
         }
-      for (int64_t q = copied; q >= 0 && q > copied - 2; --q)
-        while (!tcx::mbar_try(&bfull[q % RG_NSTAGE], (uint32_t)((q / RG_NSTAGE) & 1)) &&
-               tcx::globaltimer() - t0 < kLimit) {
-        }
     }
     __syncwarp();
-  } else if (warp == (RG_EPI + RG_STG) / 32 + 1) {
+  } else if (warp >= W_BPROD) {
+    // ------------------------------------------------------------- weight copies
+    // warp W_BPROD + q copies the weights of chunks G = q, q + 2, ... into stage
+    // G % 3 once chunk G - 3's MMAs have read it
+    if (lane == 0) {
+      constexpr uint32_t bytes = 2 * N * TG_KC * 4;
+      int64_t copied = -1;
+      for (int64_t G = warp - W_BPROD; G < total; G += 2) {
+        const int stage = (int)(G % RG_NSTAGE), c = (int)(G % nch);
+        if (G >= RG_NSTAGE &&
+            !tcx::mbar_wait(&done[stage], (uint32_t)((G / RG_NSTAGE - 1) & 1), &abort_s, flag, kLimit))
+          break;
+        asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;"
+                     ::"r"(tcx::smem_u32(&full[stage])), "r"(bytes) : "memory");
+        asm volatile(
+            "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+            ::"r"(sbase + stage * TG_STAGE + 2 * TG_A_HALF),
+              "l"(g.bsplit + (int64_t)c * 2 * N * TG_KC), "r"(bytes),
+              "r"(tcx::smem_u32(&full[stage]))
+            : "memory");
+        copied = G;
+      }
+      // the last copy lands before shared memory is given up: it has arrived on
+      // full[] once that phase completes, or, after an abort, once its bytes did
+      // (the staging warps may not have arrived); wait on the copy's bytes by
+      // the phase, bounded either way
+      const uint64_t t0 = tcx::globaltimer();
+      if (copied >= 0)
+        while (!tcx::mbar_try(&full[copied % RG_NSTAGE], (uint32_t)((copied / RG_NSTAGE) & 1)) &&
+               !abort_s && tcx::globaltimer() - t0 < kLimit) {
+        }
+      if (copied >= 0 && abort_s) {
+        const uint64_t t1 = tcx::globaltimer();
+        while (tcx::globaltimer() - t1 < 20000) {   // an aborted launch: give the copy 20 us
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp == W_APROD) {
     // ------------------------------------------------------------- raw A producer
     if (lane == 0) {
       int64_t loaded = -1;
@@ -558,12 +574,16 @@ __global__ void __launch_bounds__(RG_THREADS, 1) row_gemm_tc_kernel(RowGemm g,
     __syncwarp();
   } else if (warp >= RG_EPI / 32) {
     // ------------------------------------------------------------- staging warps
-    // per chunk, thread st takes the 16-byte pieces i = st and st + 256 of the
-    // raw chunk (row i / 4, K columns 4 (i % 4) ..): a warp reads 512
-    // contiguous bytes and writes four 128-byte core-matrix rows. A warp that
-    // broke out on an abort never arrives again, so the other roles' waits
-    // end by the abort word.
+    // per chunk, thread st reads the 16-byte pieces i = st and st + 256 of the
+    // raw chunk (row i / 4, K columns 4 (i % 4) ..), so that a warp reads 512
+    // contiguous bytes. A shuffle then hands lane l the piece of row
+    // 8 (warp) + l % 8, K group l / 8: each quarter-warp (the unit in which
+    // 16-byte shared accesses are served) stores one 128-byte core-matrix row
+    // without bank conflicts. A warp that broke out on an abort never arrives
+    // again, so the other roles' waits end by the abort word.
     const int st = tid - RG_EPI;
+    const int src = ((lane & 7) << 2) | (lane >> 3);
+    const int srow = 8 * (st >> 5) + (lane & 7), skq = lane >> 3;
     for (int64_t G = 0; G < total && ok; ++G) {
       const int slot = (int)(G % RG_NRAW), stage = (int)(G % RG_NSTAGE);
       bool w = tcx::mbar_wait(&rfull[slot], (uint32_t)((G / RG_NRAW) & 1), &abort_s, flag, kLimit);
@@ -572,8 +592,12 @@ __global__ void __launch_bounds__(RG_THREADS, 1) row_gemm_tc_kernel(RowGemm g,
         break;
       }
       const float* raw = reinterpret_cast<const float*>(tsm + RG_NSTAGE * TG_STAGE + slot * RG_RAW);
-      const float4 v0 = *reinterpret_cast<const float4*>(raw + 4 * st);
-      const float4 v1 = *reinterpret_cast<const float4*>(raw + 4 * (st + 256));
+      const float4 r0 = *reinterpret_cast<const float4*>(raw + 4 * st);
+      const float4 r1 = *reinterpret_cast<const float4*>(raw + 4 * (st + 256));
+      const float4 v0 = make_float4(__shfl_sync(0xffffffffu, r0.x, src), __shfl_sync(0xffffffffu, r0.y, src),
+                                    __shfl_sync(0xffffffffu, r0.z, src), __shfl_sync(0xffffffffu, r0.w, src));
+      const float4 v1 = make_float4(__shfl_sync(0xffffffffu, r1.x, src), __shfl_sync(0xffffffffu, r1.y, src),
+                                    __shfl_sync(0xffffffffu, r1.z, src), __shfl_sync(0xffffffffu, r1.w, src));
       w = G < RG_NSTAGE || tcx::mbar_wait(&done[stage], (uint32_t)((G / RG_NSTAGE - 1) & 1), &abort_s, flag, kLimit);
       if (!__all_sync(0xffffffffu, w)) {
         ok = false;
@@ -582,14 +606,13 @@ __global__ void __launch_bounds__(RG_THREADS, 1) row_gemm_tc_kernel(RowGemm g,
       const uint32_t sa = sbase + stage * TG_STAGE;
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
-        const int i = st + 256 * h;
         const float4 v = h ? v1 : v0;
         float hi[4], lo[4];
         tg_split(v.x, hi[0], lo[0]);
         tg_split(v.y, hi[1], lo[1]);
         tg_split(v.z, hi[2], lo[2]);
         tg_split(v.w, hi[3], lo[3]);
-        const uint32_t o = tg_off(i >> 2, 4 * (i & 3), TG_M);
+        const uint32_t o = tg_off(srow + 64 * h, 4 * skq, TG_M);
         tcx::st_shared_v4(sa + o, __float_as_uint(hi[0]), __float_as_uint(hi[1]),
                           __float_as_uint(hi[2]), __float_as_uint(hi[3]));
         tcx::st_shared_v4(sa + TG_A_HALF + o, __float_as_uint(lo[0]), __float_as_uint(lo[1]),
@@ -601,7 +624,7 @@ __global__ void __launch_bounds__(RG_THREADS, 1) row_gemm_tc_kernel(RowGemm g,
       // its loads of the slot, so the next tensor copy into it cannot overtake
       // a read still in flight
       if (lane == 0) {
-        tcx::mbar_arrive(&afull[stage]);
+        tcx::mbar_arrive(&full[stage]);
         tcx::mbar_arrive(&rempty[slot]);
       }
     }
