@@ -51,6 +51,11 @@ def test_create_rejects_bad_configs_without_a_device(lib):
     assert lib.nerf_create(ctypes.byref(cfg), ctypes.byref(h)) == _capi.NERF_ERR_UNSUPPORTED
     cfg = _capi.nerf_config(0, 4, 64, -1, 10, 4, 0, 1, 0, 0, 16, 192)     # bf16 tiny
     assert lib.nerf_create(ctypes.byref(cfg), ctypes.byref(h)) == _capi.NERF_ERR_UNSUPPORTED
+    cfg = _capi.nerf_config(0, 4, 64, -1, 10, 4, 0, 2, 0, 0, 16, 192)     # TF32 at W = 64
+    assert lib.nerf_create(ctypes.byref(cfg), ctypes.byref(h)) == _capi.NERF_ERR_UNSUPPORTED
+    assert b"TF32" in lib.nerf_last_error(None)
+    cfg = _capi.nerf_config(0, 8, 256, 4, 10, 4, 0, 3, 0, 0, 16, 192)     # precision 3
+    assert lib.nerf_create(ctypes.byref(cfg), ctypes.byref(h)) == _capi.NERF_ERR_INVALID_ARG
     cfg = _capi.nerf_config(7, 8, 256, 4, 10, 4, 0, 0, 0, 0, 16, 192)     # unknown model
     assert lib.nerf_create(ctypes.byref(cfg), ctypes.byref(h)) == _capi.NERF_ERR_INVALID_ARG
     cfg = _capi.nerf_config(2, 8, 256, 4, 10, 4, 0, 2, 0, 0, 16, 512)     # hash grid, precision 2
