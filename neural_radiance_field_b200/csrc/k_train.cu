@@ -494,11 +494,9 @@ __global__ void __launch_bounds__(RG_THREADS, 1) row_gemm_tc_kernel(RowGemm g,
         }
       }
       // the MMAs already issued land before TMEM is freed, abort or not
-      const uint64_t t0 = tcx::globaltimer();
       if (issued >= 0)
-        while (!tcx::mbar_try(&done[issued % RG_NSTAGE], (uint32_t)((issued / RG_NSTAGE) & 1)) &&
-               tcx::globaltimer() - t0 < kLimit) {
-        }
+        tcx::mbar_drain(&done[issued % RG_NSTAGE], (uint32_t)((issued / RG_NSTAGE) & 1), flag,
+                        tcx::globaltimer(), kLimit);
     }
     __syncwarp();
   } else if (warp >= W_BPROD) {
@@ -528,11 +526,15 @@ __global__ void __launch_bounds__(RG_THREADS, 1) row_gemm_tc_kernel(RowGemm g,
       // (the staging warps may not have arrived); wait on the copy's bytes by
       // the phase, bounded either way
       const uint64_t t0 = tcx::globaltimer();
-      if (copied >= 0)
-        while (!tcx::mbar_try(&full[copied % RG_NSTAGE], (uint32_t)((copied / RG_NSTAGE) & 1)) &&
-               !abort_s && tcx::globaltimer() - t0 < kLimit) {
+      bool landed = copied < 0;
+      while (!landed && !abort_s) {
+        landed = tcx::mbar_try(&full[copied % RG_NSTAGE], (uint32_t)((copied / RG_NSTAGE) & 1));
+        if (!landed && tcx::globaltimer() - t0 > kLimit) {
+          atomicOr(flag, FLAG_TIMEOUT);
+          abort_s = 1;
         }
-      if (copied >= 0 && abort_s) {
+      }
+      if (!landed) {
         const uint64_t t1 = tcx::globaltimer();
         while (tcx::globaltimer() - t1 < 20000) {   // an aborted launch: give the copy 20 us
         }
@@ -567,9 +569,7 @@ __global__ void __launch_bounds__(RG_THREADS, 1) row_gemm_tc_kernel(RowGemm g,
       // the copies in flight land before shared memory is given up
       const uint64_t t0 = tcx::globaltimer();
       for (int64_t q = loaded; q >= 0 && q > loaded - RG_NRAW; --q)
-        while (!tcx::mbar_try(&rfull[q % RG_NRAW], (uint32_t)((q / RG_NRAW) & 1)) &&
-               tcx::globaltimer() - t0 < kLimit) {
-        }
+        if (!tcx::mbar_drain(&rfull[q % RG_NRAW], (uint32_t)((q / RG_NRAW) & 1), flag, t0, kLimit)) break;
     }
     __syncwarp();
   } else if (warp >= RG_EPI / 32) {
@@ -878,12 +878,9 @@ __global__ void __launch_bounds__(TG_THREADS, 1) wgrad_tc_kernel(WGrad g, int k0
         issued = c;
       }
       // the MMAs already issued land before TMEM is freed, abort or not
-      if (issued >= 0) {
-        const uint64_t t0 = tcx::globaltimer();
-        while (!tcx::mbar_try(&done[issued % WT_NSTAGE], (uint32_t)((issued / WT_NSTAGE) & 1)) &&
-               tcx::globaltimer() - t0 < kLimit) {
-        }
-      }
+      if (issued >= 0)
+        tcx::mbar_drain(&done[issued % WT_NSTAGE], (uint32_t)((issued / WT_NSTAGE) & 1), flag,
+                        tcx::globaltimer(), kLimit);
     }
     __syncwarp();
   } else {

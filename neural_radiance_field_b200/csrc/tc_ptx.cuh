@@ -52,6 +52,20 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   return true;
 }
 
+// Drain wait before a CTA gives up shared or tensor memory: not stopped by an
+// abort (what was issued must land first); running out of time (limit_ns since
+// t0) raises FLAG_TIMEOUT like any other wait. Returns whether the phase completed.
+__device__ __forceinline__ bool mbar_drain(uint64_t* bar, uint32_t parity, unsigned* flag,
+                                           uint64_t t0, uint64_t limit_ns) {
+  while (!mbar_try(bar, parity)) {
+    if (globaltimer() - t0 > limit_ns) {
+      atomicOr(flag, FLAG_TIMEOUT);
+      return false;
+    }
+  }
+  return true;
+}
+
 __device__ __forceinline__ void fence_before() {
   asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
 }
