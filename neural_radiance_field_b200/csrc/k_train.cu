@@ -376,14 +376,17 @@ __device__ __forceinline__ void tg_mma(uint32_t tmem_d, uint64_t a, uint64_t b, 
 
 // Roles of the row GEMM's CTA (16 warps):
 //   warps 0-3    epilogue: warp w reads TMEM lane quarter w (one accumulator row
-//                per lane), 32 columns at a time, and writes each row's block
-//                as whole 128-byte lines in 16-byte pieces (a transpose
-//                through shared memory for fully coalesced rows measured four
-//                times slower);
+//                per lane), 32 columns at a time, finishes the values in
+//                registers and writes the 32 x 32 block to one of its two
+//                shared-memory tiles (128-byte swizzle: conflict-free), which
+//                lane 0 stores with one 2-D tensor copy: a store instruction
+//                costs about 64 cycles of the SM's store path whatever its
+//                width (measured), so the block leaves in one request instead
+//                of eight uncoalesced or thirty-two coalesced ones;
 //   warps 4-11   split the raw A rows into the operand stages;
 //   warp 12      issues the MMAs: one barrier wait per chunk, six MMAs, a commit;
 //   warp 13      streams the raw A rows by 2-D tensor copies (16 K-columns x
-//                128 rows per chunk) into an 8-slot ring;
+//                128 rows per chunk) into a 4-slot ring;
 //   warps 14-15  copy the split weights of the even / odd chunks (one bulk copy
 //                each; a copy takes the issuing thread about 600 cycles, so two
 //                threads share the chunk stream).
@@ -396,21 +399,24 @@ constexpr int RG_STG = 256;
 constexpr int RG_THREADS = RG_EPI + RG_STG + 128;
 constexpr int RG_NSTAGE = 3;
 constexpr int RG_RAW = TG_M * TG_KC * 4;                // one raw A chunk, 8 KB
-constexpr int RG_NRAW = 8;
-constexpr int RG_BAR = RG_NSTAGE * TG_STAGE + RG_NRAW * RG_RAW;
+constexpr int RG_NRAW = 4;
+constexpr int RG_OUTB = 32 * 32 * 4;                    // an epilogue warp's 32 x 32 output block
+constexpr int RG_OUT = RG_NSTAGE * TG_STAGE + RG_NRAW * RG_RAW;   // 4 warps x 2 blocks, 1024-aligned
+constexpr int RG_BAR = RG_OUT + 4 * 2 * RG_OUTB;
 constexpr size_t RG_SMEM = (size_t)RG_BAR + 256;
 
 template <int N>
 __global__ void __launch_bounds__(RG_THREADS, 1) row_gemm_tc_kernel(RowGemm g,
-                                                                    const __grid_constant__ CUtensorMap amap) {
+                                                                    const __grid_constant__ CUtensorMap amap,
+                                                                    const __grid_constant__ CUtensorMap omap) {
   unsigned* flag = g.flag;
   extern __shared__ __align__(1024) uint8_t tsm[];
   uint64_t* done = reinterpret_cast<uint64_t*>(tsm + RG_BAR);   // [3] MMAs of a stage done
   uint64_t* full = done + RG_NSTAGE;                             // [3] stage staged (A and B)
   uint64_t* accf = full + RG_NSTAGE;                             // [2] accumulator ready
   uint64_t* acce = accf + 2;                                     // [2] accumulator read out
-  uint64_t* rfull = acce + 2;                                    // [8] raw A chunk landed
-  uint64_t* rempty = rfull + RG_NRAW;                            // [8] raw A chunk read
+  uint64_t* rfull = acce + 2;                                    // [4] raw A chunk landed
+  uint64_t* rempty = rfull + RG_NRAW;                            // [4] raw A chunk read
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(rempty + RG_NRAW);
   __shared__ int abort_s;
   __shared__ __align__(16) float s_bias[N], s_ev[N];
@@ -451,9 +457,13 @@ __global__ void __launch_bounds__(RG_THREADS, 1) row_gemm_tc_kernel(RowGemm g,
   const int64_t ntiles = (g.rows + TG_M - 1) / TG_M;
   // this CTA's tiles: blockIdx.x, + gridDim.x, ...; chunk G of the CTA is chunk
   // G % nch of its tile G / nch, uses operand stage G % 3 (barrier parity
-  // (G / 3) % 2) and raw slot G % 8 (parity (G / 8) % 2); tile i uses
+  // (G / 3) % 2) and raw slot G % 4 (parity (G / 4) % 2); tile i uses
   // accumulator i % 2 (parity (i / 2) % 2)
-  const int n_my = blockIdx.x < ntiles ? (int)((ntiles - 1 - blockIdx.x) / gridDim.x + 1) : 0;
+  // the swizzled output tiles must sit on 1024-byte boundaries: otherwise no
+  // role runs (the error flag says why) rather than stores of permuted tiles
+  const int n_my = (blockIdx.x < ntiles && ((sbase + RG_OUT) & 1023u) == 0)
+                       ? (int)((ntiles - 1 - blockIdx.x) / gridDim.x + 1) : 0;
+  if (tid == 0 && ((sbase + RG_OUT) & 1023u) != 0) atomicOr(flag, FLAG_BAD_INDEX);
   const int64_t total = (int64_t)n_my * nch;
   bool ok = true;
   constexpr int W_ISSUE = (RG_EPI + RG_STG) / 32, W_APROD = W_ISSUE + 1, W_BPROD = W_ISSUE + 2;
@@ -630,12 +640,13 @@ __global__ void __launch_bounds__(RG_THREADS, 1) row_gemm_tc_kernel(RowGemm g,
     }
   } else {
     // ------------------------------------------------------------- epilogue warps
-    // thread = accumulator row warp * 32 + lane; 32 columns per TMEM load, the
-    // output row written in 16-byte pieces (each thread a whole 128-byte line
-    // per column block); the next block's side input (the mask or the row
-    // biases: a launch has at most one) is loaded while the current block is
-    // finished
-    const int rl = warp * 32 + lane;
+    // thread = accumulator row warp * 32 + lane; 32 columns per TMEM load; the
+    // next block's side input (the mask or the row biases: a launch has at most
+    // one) is loaded while the current block is finished; chunk j (columns
+    // 4j..4j+3) of row r sits at r * 128 + ((j ^ (r % 8)) * 16) in the tile,
+    // the layout the tensor map's 128-byte swizzle reads
+    const uint32_t obase = sbase + RG_OUT + warp * 2 * RG_OUTB;
+    int nstore = 0;
     for (int it = 0; it < n_my && ok; ++it) {
       const int b = it & 1;
       const bool w = tcx::mbar_wait(&accf[b], (uint32_t)((it >> 1) & 1), &abort_s, flag, kLimit);
@@ -644,12 +655,12 @@ __global__ void __launch_bounds__(RG_THREADS, 1) row_gemm_tc_kernel(RowGemm g,
         break;
       }
       tcx::fence_after();
-      const int64_t row = (blockIdx.x + (int64_t)it * gridDim.x) * TG_M + rl;
+      const int64_t row0 = (blockIdx.x + (int64_t)it * gridDim.x) * TG_M + warp * 32;
+      const int64_t row = row0 + lane;
       const bool live = row < g.rows;
       const float eav = (g.ea && live) ? g.ea[row * g.ldea] : 0.0f;
       const float* mrow = (g.mask && live) ? g.mask + row * g.ldm : nullptr;
       const float* rrow = (g.row_bias && live) ? g.row_bias + (row / g.rb_div) * g.n_out : nullptr;
-      float* orow = g.out + row * g.ldo;
       const float* srow = mrow ? mrow : rrow;
       float4 sd[8];
       auto load_side = [&](int cb, float4 (&m)[8]) {
@@ -659,11 +670,15 @@ __global__ void __launch_bounds__(RG_THREADS, 1) row_gemm_tc_kernel(RowGemm g,
       };
       load_side(0, sd);
 #pragma unroll 1
-      for (int cb = 0; cb < N; cb += 32) {
+      for (int cb = 0; cb < N; cb += 32, ++nstore) {
         uint32_t u[32];
         tcx::tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)(b * N + cb), u);
         float4 sd2[8];
         if (cb + 32 < N) load_side(cb + 32, sd2);
+        // the tile written two blocks ago has been read by its store
+        if (lane == 0 && nstore >= 2) asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+        __syncwarp();
+        const uint32_t ob = obase + (uint32_t)(nstore & 1) * RG_OUTB + (uint32_t)lane * 128;
         tcx::tmem_ld_wait(u);
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
@@ -683,7 +698,19 @@ __global__ void __launch_bounds__(RG_THREADS, 1) row_gemm_tc_kernel(RowGemm g,
             if (g.mask) v = sv[e] > 0.0f ? v : 0.0f;
             x[e] = v;
           }
-          if (live) *reinterpret_cast<float4*>(orow + cb + 4 * j) = make_float4(x[0], x[1], x[2], x[3]);
+          tcx::st_shared_v4(ob + (uint32_t)((j ^ (lane & 7)) * 16), __float_as_uint(x[0]),
+                            __float_as_uint(x[1]), __float_as_uint(x[2]), __float_as_uint(x[3]));
+        }
+        tcx::fence_async_smem();
+        __syncwarp();
+        if (lane == 0 && row0 < g.rows) {
+          // rows past the end of the matrix are clipped by the tensor map
+          asm volatile(
+              "cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];"
+              ::"l"(reinterpret_cast<uint64_t>(&omap)), "r"(cb), "r"((int)row0),
+                "r"(obase + (uint32_t)(nstore & 1) * RG_OUTB)
+              : "memory");
+          asm volatile("cp.async.bulk.commit_group;" ::: "memory");
         }
         if (cb + 32 < N) {
 #pragma unroll
@@ -695,6 +722,10 @@ __global__ void __launch_bounds__(RG_THREADS, 1) row_gemm_tc_kernel(RowGemm g,
       __syncwarp();
       if (lane == 0) tcx::mbar_arrive(&acce[b]);
     }
+    // every store has read its tile before the CTA gives up shared memory, and
+    // has written global memory before the kernel ends
+    if (lane == 0) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+    __syncwarp();
   }
   tcx::fence_before();
   __syncthreads();
@@ -1212,15 +1243,21 @@ using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t
 
 // fp32 matrix of `rows` rows of `ld` floats, boxes of TG_KC columns x TG_M rows
 // (rows past the end read as zero).
-cudaError_t encode_rows_map(CUtensorMap* m, const float* base, int64_t ld, int64_t rows) {
+EncodeTiledFn tiled_encoder() {
   static EncodeTiledFn encode = nullptr;
   if (!encode) {
     cudaDriverEntryPointQueryResult q;
     void* fn = nullptr;
     cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q);
-    if (e != cudaSuccess || q != cudaDriverEntryPointSuccess || !fn) return cudaErrorNotSupported;
+    if (e != cudaSuccess || q != cudaDriverEntryPointSuccess || !fn) return nullptr;
     encode = reinterpret_cast<EncodeTiledFn>(fn);
   }
+  return encode;
+}
+
+cudaError_t encode_rows_map(CUtensorMap* m, const float* base, int64_t ld, int64_t rows) {
+  EncodeTiledFn encode = tiled_encoder();
+  if (!encode) return cudaErrorNotSupported;
   const cuuint64_t dims[2] = {(cuuint64_t)ld, (cuuint64_t)rows};
   const cuuint64_t strides[1] = {(cuuint64_t)ld * 4};
   const cuuint32_t box[2] = {TG_KC, TG_M};
@@ -1228,6 +1265,22 @@ cudaError_t encode_rows_map(CUtensorMap* m, const float* base, int64_t ld, int64
   CUresult r = encode(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float*>(base), dims, strides,
                       box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
                       CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+// fp32 output matrix of `rows` rows of `ld` floats, `cols` of them written,
+// boxes of 32 columns x 32 rows with the 128-byte swizzle (rows past the end
+// are not written).
+cudaError_t encode_out_map(CUtensorMap* m, float* base, int64_t ld, int cols, int64_t rows) {
+  EncodeTiledFn encode = tiled_encoder();
+  if (!encode) return cudaErrorNotSupported;
+  const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)ld * 4};
+  const cuuint32_t box[2] = {32, 32};
+  const cuuint32_t estr[2] = {1, 1};
+  CUresult r = encode(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, base, dims, strides, box, estr,
+                      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                      CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
@@ -1259,8 +1312,9 @@ cudaError_t row_gemm(RowGemm g, cudaStream_t st) {
       if (e != cudaSuccess) return e;
       attr_set[wide] = true;
     }
-    CUtensorMap amap;
+    CUtensorMap amap, omap;
     cudaError_t e = encode_rows_map(&amap, g.A, g.lda, g.rows);
+    if (e == cudaSuccess) e = encode_out_map(&omap, g.out, g.ldo, g.n_out, g.rows);
     if (e != cudaSuccess) return e;
     const int64_t nb = (int64_t)g.K * g.n_out;
     split_b_kernel<<<(unsigned)std::min<int64_t>(blocks_for(nb, 256), 1024), 256, 0, st>>>(
@@ -1269,8 +1323,8 @@ cudaError_t row_gemm(RowGemm g, cudaStream_t st) {
     if (e != cudaSuccess) return e;
     // persistent: one CTA per SM walks the row tiles
     const unsigned grid = (unsigned)std::min<int64_t>(blocks_for(g.rows, TG_M), sm_count());
-    if (wide) row_gemm_tc_kernel<256><<<grid, RG_THREADS, RG_SMEM, st>>>(g, amap);
-    else row_gemm_tc_kernel<128><<<grid, RG_THREADS, RG_SMEM, st>>>(g, amap);
+    if (wide) row_gemm_tc_kernel<256><<<grid, RG_THREADS, RG_SMEM, st>>>(g, amap, omap);
+    else row_gemm_tc_kernel<128><<<grid, RG_THREADS, RG_SMEM, st>>>(g, amap, omap);
     return cudaGetLastError();
   }
   row_gemm_kernel<<<dim3(blocks_for(g.rows, GT), blocks_for(g.n_out, GT)), 256, 0, st>>>(g);
