@@ -735,6 +735,440 @@ __global__ void __launch_bounds__(RG_THREADS, 1) row_gemm_tc_kernel(RowGemm g,
   }
 }
 
+// ---------------------------------------------------------------------------
+// The same row GEMM on CTA pairs: a cluster of two CTAs on two SMs runs
+// tcgen05.mma.cta_group::2 (M = 256: rows [0, 128) of a 256-row tile in CTA 0,
+// [128, 256) in CTA 1). Each CTA stages its own 128 A rows and holds half of
+// the split weights (N / 2 rows of B), and CTA 0 issues the MMAs for both, so
+// per MMA each SM reads 4 KB of A and 4 KB of B from its shared memory instead
+// of 4 + 8 KB, each CTA copies 16 KB of weights per chunk instead of 32, and one
+// MMA instruction does the work of two. The roles per CTA are the single-CTA
+// kernel's; a stage is full on CTA 0's barrier when the sixteen staging warps
+// of both CTAs and the two weight copies (counted by CTA 0's expect) have
+// arrived, an accumulator is free on CTA 0's barrier when the eight epilogue
+// warps of both CTAs have read it, and the commits arrive on both CTAs.
+constexpr int RP_NSTAGE = 4;
+constexpr int RP_STAGE = 2 * TG_A_HALF + 2 * (128 * TG_KC * 4);    // A hi, lo; B half hi, lo: 32 KB
+constexpr int RP_NRAW = 4;
+constexpr int RP_OUT = RP_NSTAGE * RP_STAGE + RP_NRAW * RG_RAW;    // 1024-aligned
+constexpr int RP_VEC = RP_OUT + 4 * 2 * RG_OUTB;
+constexpr int RP_BAR = RP_VEC + 2 * 256 * 4;
+constexpr size_t RP_SMEM = (size_t)RP_BAR + 256;
+
+__device__ __forceinline__ uint32_t rp_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ uint32_t rp_cluster() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%clusterid.x;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ uint32_t rp_nclusters() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%nclusterid.x;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ void rp_cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// try_wait with cluster-scope acquire: the phase may be completed from the peer CTA
+__device__ __forceinline__ bool rp_try(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(tcx::smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// bounded, as tcx::mbar_wait
+__device__ __forceinline__ bool rp_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                        unsigned* flag, uint64_t limit_ns) {
+  if (rp_try(bar, parity)) return true;
+  const uint64_t t0 = tcx::globaltimer();
+  while (!rp_try(bar, parity)) {
+    if (*abort) return false;
+    if (tcx::globaltimer() - t0 > limit_ns) {
+      atomicOr(flag, FLAG_TIMEOUT);
+      *abort = 1;
+      return false;
+    }
+  }
+  return true;
+}
+// Arrive on CTA 0's barrier at this barrier's offset, releasing this CTA's
+// shared-memory writes at cluster scope (a release fence restricted to
+// shared::cta operations, then a relaxed remote arrive).
+__device__ __forceinline__ void rp_arrive_cta0(uint64_t* bar) {
+  asm volatile(
+      "{\n\t.reg .b32 ra;\n\t"
+      "mapa.shared::cluster.u32 ra, %0, 0;\n\t"
+      "fence.release.sync_restrict::shared::cta.cluster;\n\t"
+      "mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [ra];\n\t}"
+      ::"r"(tcx::smem_u32(bar))
+      : "memory");
+}
+// 2-D tensor load into this CTA's shared memory counted on CTA 0's barrier
+// (the barrier's shared address with the peer bit cleared); no multicast.
+__device__ __forceinline__ void rp_load_pair(uint32_t dst, const void* tmap, int x, int y,
+                                             uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4}], [%2];"
+      ::"r"(dst), "l"(reinterpret_cast<uint64_t>(tmap)),
+        "r"(tcx::smem_u32(bar) & 0xFEFFFFFFu), "r"(x), "r"(y)
+      : "memory");
+}
+__device__ __forceinline__ void rp_mma(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc,
+                                       uint32_t accum) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::tf32 [%0], %1, %2, %3, p;\n\t}"
+      ::"r"(d), "l"(a), "l"(b), "r"(idesc), "r"(accum));
+}
+// arrive (once each) on this barrier's offset in both CTAs once every MMA
+// issued so far by the calling thread has completed
+__device__ __forceinline__ void rp_commit(uint64_t* bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
+      " [%0], %1;"
+      ::"r"(tcx::smem_u32(bar)), "h"((uint16_t)3)
+      : "memory");
+}
+
+// B[k][c] -> chunks of 32 K, each [half h][hi | lo][N/2 rows x 32 K] (K-major core
+// matrices of N/2 rows): the half a CTA of the pair holds is one contiguous run.
+__global__ void split_b_pair_kernel(const float* __restrict__ B, int64_t ldb, int K, int N,
+                                    float* __restrict__ out) {
+  const int64_t total = (int64_t)K * N;
+  const int Nh = N / 2;
+  for (int64_t q = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; q < total;
+       q += (int64_t)gridDim.x * blockDim.x) {
+    const int k = (int)(q / N), c = (int)(q % N);
+    const int h = c / Nh, cl = c - h * Nh;
+    float hi, lo;
+    tg_split(__ldg(B + (int64_t)k * ldb + c), hi, lo);
+    float* ch = out + (int64_t)(k / TG_KC) * 2 * N * TG_KC + (int64_t)h * N * TG_KC;
+    const uint32_t o = tg_off(cl, k % TG_KC, Nh) >> 2;
+    ch[o] = hi;
+    ch[Nh * TG_KC + o] = lo;
+  }
+}
+
+template <int N>
+__global__ void __launch_bounds__(RG_THREADS, 1) row_gemm_pair_kernel(RowGemm g,
+                                                                      const __grid_constant__ CUtensorMap amap,
+                                                                      const __grid_constant__ CUtensorMap bmap,
+                                                                      const __grid_constant__ CUtensorMap omap) {
+  constexpr int Nh = N / 2;
+  constexpr uint32_t BH = Nh * TG_KC * 4;        // B half, hi or lo, of a chunk
+  unsigned* flag = g.flag;
+  extern __shared__ __align__(1024) uint8_t tsm[];
+  float* s_bias = reinterpret_cast<float*>(tsm + RP_VEC);
+  float* s_ev = s_bias + 256;
+  uint64_t* done = reinterpret_cast<uint64_t*>(tsm + RP_BAR);   // [4] MMAs of a stage done (both CTAs)
+  uint64_t* full = done + RP_NSTAGE;                             // [4] stage staged (CTA 0's)
+  uint64_t* accf = full + RP_NSTAGE;                             // [2] accumulator ready (both CTAs)
+  uint64_t* acce = accf + 2;                                     // [2] accumulator read out (CTA 0's)
+  uint64_t* rfull = acce + 2;                                    // [4] raw A chunk landed
+  uint64_t* rempty = rfull + RP_NRAW;                            // [4] raw A chunk read
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(rempty + RP_NRAW);
+  volatile int* abort_p = reinterpret_cast<volatile int*>(tmem_holder + 1);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int rank = (int)rp_rank();
+  const uint32_t sbase = tcx::smem_u32(tsm);
+  const uint32_t rawbase = sbase + RP_NSTAGE * RP_STAGE;
+  constexpr uint64_t kLimit = 2000000000ull;
+  if (tid == 0) {
+    for (int i = 0; i < RP_NSTAGE; ++i) {
+      tcx::mbar_init(&done[i], 1);
+      tcx::mbar_init(&full[i], 2 * (RG_STG / 32) + 1);   // both CTAs' staging warps, CTA 0's expect
+    }
+    for (int i = 0; i < 2; ++i) {
+      tcx::mbar_init(&accf[i], 1);
+      tcx::mbar_init(&acce[i], 2 * (RG_EPI / 32));       // both CTAs' epilogue warps
+    }
+    for (int i = 0; i < RP_NRAW; ++i) {
+      tcx::mbar_init(&rfull[i], 1);
+      tcx::mbar_init(&rempty[i], RG_STG / 32);
+    }
+    *abort_p = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  for (int i = tid; i < N; i += RG_THREADS) {
+    s_bias[i] = g.bias ? g.bias[i] : 0.0f;
+    s_ev[i] = g.ea ? g.ev[i] : 0.0f;
+  }
+  if (warp == 0) {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;"
+                 ::"r"(tcx::smem_u32(tmem_holder)), "r"(2 * N));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;");
+  }
+  tcx::fence_before();
+  __syncthreads();
+  rp_cluster_sync();            // both CTAs' barriers exist before any remote use
+  tcx::fence_after();
+  const uint32_t tmem = *tmem_holder;
+  const int nch = g.K / TG_KC;
+  const int64_t ntiles = (g.rows + 2 * TG_M - 1) / (2 * TG_M);   // 256-row pair tiles
+  const int64_t cid = rp_cluster(), ncl = rp_nclusters();
+  // pair tile i = cid + i * ncl; chunk G of the pair is chunk G % nch of its
+  // tile G / nch and uses stage G % 4 (parity (G / 4) % 2) and raw slot G % 4;
+  // tile i uses accumulator i % 2 (parity (i / 2) % 2). Both CTAs lay out
+  // shared memory alike, so the alignment test agrees between them.
+  const bool aligned = ((sbase + RP_OUT) & 1023u) == 0;
+  const int n_my = (cid < ntiles && aligned) ? (int)((ntiles - 1 - cid) / ncl + 1) : 0;
+  if (tid == 0 && !aligned) atomicOr(flag, FLAG_BAD_INDEX);
+  const int64_t total = (int64_t)n_my * nch;
+  auto tile_row = [&](int64_t it) { return (cid + it * ncl) * (2 * TG_M) + rank * TG_M; };
+  bool ok = true;
+  constexpr int W_ISSUE = (RG_EPI + RG_STG) / 32, W_APROD = W_ISSUE + 1, W_BPROD = W_ISSUE + 2;
+  if (warp == W_ISSUE) {
+    // ------------------------------------------------------------- MMA issuer (CTA 0)
+    if (lane == 0 && rank == 0) {
+      constexpr uint32_t idesc = (1u << 4) | (2u << 7) | (2u << 10) | ((uint32_t)(N >> 3) << 17) |
+                                 ((uint32_t)((2 * TG_M) >> 4) << 24);   // f32 <- tf32 x tf32, M 256
+      int64_t G = 0, issued = -1;
+      for (int it = 0; it < n_my && ok; ++it) {
+        const int b = it & 1;
+        if (it >= 2 && !rp_wait(&acce[b], (uint32_t)(((it >> 1) - 1) & 1), abort_p, flag, kLimit)) {
+          ok = false;
+          break;
+        }
+        const uint32_t acc = tmem + (uint32_t)(b * N);
+        for (int c = 0; c < nch; ++c, ++G) {
+          const int stage = (int)(G % RP_NSTAGE);
+          if (!rp_wait(&full[stage], (uint32_t)((G / RP_NSTAGE) & 1), abort_p, flag, kLimit)) {
+            ok = false;
+            break;
+          }
+          tcx::fence_after();
+          const uint32_t sa = sbase + stage * RP_STAGE;
+          const uint64_t ah = tcx::sdesc(sa, TG_M * 16, 128), al = tcx::sdesc(sa + TG_A_HALF, TG_M * 16, 128);
+          const uint64_t bh = tcx::sdesc(sa + 2 * TG_A_HALF, Nh * 16, 128);
+          const uint64_t bl = tcx::sdesc(sa + 2 * TG_A_HALF + BH, Nh * 16, 128);
+#pragma unroll
+          for (int s = 0; s < TG_KC / 8; ++s) {
+            const uint64_t da = (uint64_t)((s * 2 * TG_M * 16) >> 4), db = (uint64_t)((s * 2 * Nh * 16) >> 4);
+            rp_mma(acc, ah + da, bh + db, idesc, (c | s) != 0);
+            rp_mma(acc, ah + da, bl + db, idesc, 1);
+            rp_mma(acc, al + da, bh + db, idesc, 1);
+          }
+          rp_commit(&done[stage]);
+          if (c == nch - 1) rp_commit(&accf[b]);
+          issued = G;
+        }
+      }
+      // the MMAs already issued land before either CTA frees its memory, abort or not
+      if (issued >= 0) {
+        const uint64_t t0 = tcx::globaltimer();
+        while (!rp_try(&done[issued % RP_NSTAGE], (uint32_t)((issued / RP_NSTAGE) & 1))) {
+          if (tcx::globaltimer() - t0 > kLimit) {
+            atomicOr(flag, FLAG_TIMEOUT);
+            break;
+          }
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp >= W_BPROD) {
+    // ------------------------------------------------------------- weight copies
+    // warp W_BPROD + q of each CTA copies that CTA's half of the weights of
+    // chunks G = q, q + 2, ... into stage G % 4 once chunk G - 4's MMAs are done;
+    // CTA 0 expects both halves' bytes on its full[] barrier
+    if (lane == 0) {
+      constexpr uint32_t half_bytes = 2 * BH;
+      for (int64_t G = warp - W_BPROD; G < total; G += 2) {
+        const int stage = (int)(G % RP_NSTAGE), c = (int)(G % nch);
+        if (G >= RP_NSTAGE &&
+            !rp_wait(&done[stage], (uint32_t)((G / RP_NSTAGE - 1) & 1), abort_p, flag, kLimit))
+          break;
+        if (rank == 0)
+          asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;"
+                       ::"r"(tcx::smem_u32(&full[stage])), "r"(2 * half_bytes) : "memory");
+        rp_load_pair(sbase + stage * RP_STAGE + 2 * TG_A_HALF, &bmap, 0, (2 * c + rank) * Nh,
+                     &full[stage]);
+      }
+      // every copy lands before the final cluster barrier: the issuer waits
+      // for each stage it consumes, and an aborted launch pauses before it
+    }
+    __syncwarp();
+  } else if (warp == W_APROD) {
+    // ------------------------------------------------------------- raw A producer
+    if (lane == 0) {
+      int64_t loaded = -1;
+      for (int64_t G = 0; G < total && ok; ++G) {
+        const int slot = (int)(G % RP_NRAW);
+        if (G >= RP_NRAW &&
+            !tcx::mbar_wait(&rempty[slot], (uint32_t)((G / RP_NRAW - 1) & 1), abort_p, flag, kLimit)) {
+          ok = false;
+          break;
+        }
+        const int64_t it = G / nch;
+        const int c = (int)(G - it * nch);
+        const int k = c * TG_KC;
+        const int col = k < g.a_split ? g.a0 + k : g.a1 + k - g.a_split;
+        asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;"
+                     ::"r"(tcx::smem_u32(&rfull[slot])), "r"(RG_RAW) : "memory");
+        asm volatile(
+            "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
+            ::"r"(rawbase + slot * RG_RAW), "l"(reinterpret_cast<uint64_t>(&amap)), "r"(col),
+              "r"((int)tile_row(it)), "r"(tcx::smem_u32(&rfull[slot]))
+            : "memory");
+        loaded = G;
+      }
+      const uint64_t t0 = tcx::globaltimer();
+      for (int64_t q = loaded; q >= 0 && q > loaded - RP_NRAW; --q)
+        if (!tcx::mbar_drain(&rfull[q % RP_NRAW], (uint32_t)((q / RP_NRAW) & 1), flag, t0, kLimit)) break;
+    }
+    __syncwarp();
+  } else if (warp >= RG_EPI / 32) {
+    // ------------------------------------------------------------- staging warps
+    const int st = tid - RG_EPI;
+    const int src = ((lane & 7) << 2) | (lane >> 3);
+    const int srow = 8 * (st >> 5) + (lane & 7), skq = lane >> 3;
+    for (int64_t G = 0; G < total && ok; ++G) {
+      const int slot = (int)(G % RP_NRAW), stage = (int)(G % RP_NSTAGE);
+      bool w = tcx::mbar_wait(&rfull[slot], (uint32_t)((G / RP_NRAW) & 1), abort_p, flag, kLimit);
+      if (!__all_sync(0xffffffffu, w)) {
+        ok = false;
+        break;
+      }
+      const float* raw = reinterpret_cast<const float*>(tsm + RP_NSTAGE * RP_STAGE + slot * RG_RAW);
+      const float4 r0 = *reinterpret_cast<const float4*>(raw + 4 * st);
+      const float4 r1 = *reinterpret_cast<const float4*>(raw + 4 * (st + 256));
+      const float4 v0 = make_float4(__shfl_sync(0xffffffffu, r0.x, src), __shfl_sync(0xffffffffu, r0.y, src),
+                                    __shfl_sync(0xffffffffu, r0.z, src), __shfl_sync(0xffffffffu, r0.w, src));
+      const float4 v1 = make_float4(__shfl_sync(0xffffffffu, r1.x, src), __shfl_sync(0xffffffffu, r1.y, src),
+                                    __shfl_sync(0xffffffffu, r1.z, src), __shfl_sync(0xffffffffu, r1.w, src));
+      w = G < RP_NSTAGE || rp_wait(&done[stage], (uint32_t)((G / RP_NSTAGE - 1) & 1), abort_p, flag, kLimit);
+      if (!__all_sync(0xffffffffu, w)) {
+        ok = false;
+        break;
+      }
+      const uint32_t sa = sbase + stage * RP_STAGE;
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const float4 v = h ? v1 : v0;
+        float hi[4], lo[4];
+        tg_split(v.x, hi[0], lo[0]);
+        tg_split(v.y, hi[1], lo[1]);
+        tg_split(v.z, hi[2], lo[2]);
+        tg_split(v.w, hi[3], lo[3]);
+        const uint32_t o = tg_off(srow + 64 * h, 4 * skq, TG_M);
+        tcx::st_shared_v4(sa + o, __float_as_uint(hi[0]), __float_as_uint(hi[1]),
+                          __float_as_uint(hi[2]), __float_as_uint(hi[3]));
+        tcx::st_shared_v4(sa + TG_A_HALF + o, __float_as_uint(lo[0]), __float_as_uint(lo[1]),
+                          __float_as_uint(lo[2]), __float_as_uint(lo[3]));
+      }
+      tcx::fence_async_smem();
+      __syncwarp();
+      // the raw slot is released only after the stores that consumed its loads
+      if (lane == 0) {
+        rp_arrive_cta0(&full[stage]);
+        tcx::mbar_arrive(&rempty[slot]);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------- epilogue warps
+    const uint32_t obase = sbase + RP_OUT + warp * 2 * RG_OUTB;
+    int nstore = 0;
+    for (int it = 0; it < n_my && ok; ++it) {
+      const int b = it & 1;
+      const bool w = rp_wait(&accf[b], (uint32_t)((it >> 1) & 1), abort_p, flag, kLimit);
+      if (!__all_sync(0xffffffffu, w)) {
+        ok = false;
+        break;
+      }
+      tcx::fence_after();
+      const int64_t row0 = tile_row(it) + warp * 32;
+      const int64_t row = row0 + lane;
+      const bool live = row < g.rows;
+      const float eav = (g.ea && live) ? g.ea[row * g.ldea] : 0.0f;
+      const float* mrow = (g.mask && live) ? g.mask + row * g.ldm : nullptr;
+      const float* rrow = (g.row_bias && live) ? g.row_bias + (row / g.rb_div) * g.n_out : nullptr;
+      const float* srow = mrow ? mrow : rrow;
+      float4 sd[8];
+      auto load_side = [&](int cb, float4 (&m)[8]) {
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+          m[j] = srow ? *reinterpret_cast<const float4*>(srow + cb + 4 * j) : make_float4(0.f, 0.f, 0.f, 0.f);
+      };
+      load_side(0, sd);
+#pragma unroll 1
+      for (int cb = 0; cb < N; cb += 32, ++nstore) {
+        uint32_t u[32];
+        tcx::tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)(b * N + cb), u);
+        float4 sd2[8];
+        if (cb + 32 < N) load_side(cb + 32, sd2);
+        if (lane == 0 && nstore >= 2) asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+        __syncwarp();
+        const uint32_t ob = obase + (uint32_t)(nstore & 1) * RG_OUTB + (uint32_t)lane * 128;
+        tcx::tmem_ld_wait(u);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const float4 bv = *reinterpret_cast<const float4*>(s_bias + cb + 4 * j);
+          const float4 ev = *reinterpret_cast<const float4*>(s_ev + cb + 4 * j);
+          float x[4] = {__uint_as_float(u[4 * j]), __uint_as_float(u[4 * j + 1]),
+                        __uint_as_float(u[4 * j + 2]), __uint_as_float(u[4 * j + 3])};
+          const float bb[4] = {bv.x, bv.y, bv.z, bv.w}, ee[4] = {ev.x, ev.y, ev.z, ev.w};
+          const float sv[4] = {sd[j].x, sd[j].y, sd[j].z, sd[j].w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            float v = x[e];
+            if (g.bias) v += bb[e];
+            if (g.row_bias) v += sv[e];
+            if (g.ea) v = fmaf(eav, ee[e], v);
+            if (g.relu) v = fmaxf(v, 0.0f);
+            if (g.mask) v = sv[e] > 0.0f ? v : 0.0f;
+            x[e] = v;
+          }
+          tcx::st_shared_v4(ob + (uint32_t)((j ^ (lane & 7)) * 16), __float_as_uint(x[0]),
+                            __float_as_uint(x[1]), __float_as_uint(x[2]), __float_as_uint(x[3]));
+        }
+        tcx::fence_async_smem();
+        __syncwarp();
+        if (lane == 0 && row0 < g.rows) {
+          asm volatile(
+              "cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];"
+              ::"l"(reinterpret_cast<uint64_t>(&omap)), "r"(cb), "r"((int)row0),
+                "r"(obase + (uint32_t)(nstore & 1) * RG_OUTB)
+              : "memory");
+          asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+        }
+        if (cb + 32 < N) {
+#pragma unroll
+          for (int j = 0; j < 8; ++j) sd[j] = sd2[j];
+        }
+      }
+      // this warp's rows of the accumulator are read out: tell CTA 0's issuer
+      tcx::fence_before();
+      __syncwarp();
+      if (lane == 0) rp_arrive_cta0(&acce[b]);
+    }
+    if (lane == 0) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+    __syncwarp();
+  }
+  tcx::fence_before();
+  __syncthreads();
+  if (tid == 0 && *abort_p) {   // an aborted launch: copies still in flight land first
+    const uint64_t t1 = tcx::globaltimer();
+    while (tcx::globaltimer() - t1 < 50000) {
+    }
+  }
+  __syncthreads();
+  rp_cluster_sync();            // the peer's MMAs, copies and arrivals into this CTA are over
+  if (warp == 0) {
+    tcx::fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(2 * N));
+  }
+}
+
 // G[n][k] += sum_r A[r * lda + n] X(r, k) for n < N, k < K, rows in slices of
 // `slice` (a multiple of 8), each slice's partial sums added atomically; the
 // CTAs of the first column tile also add db[n] += sum_r A[r][n]. X(r, k) =
@@ -1284,6 +1718,53 @@ cudaError_t encode_out_map(CUtensorMap* m, float* base, int64_t ld, int cols, in
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
+// The split weights as rows of 128 bytes; a box is one CTA's half of a chunk
+// (N / 2 rows: 16 KB for N = 256).
+cudaError_t encode_bhalf_map(CUtensorMap* m, float* bsplit, int K, int N) {
+  EncodeTiledFn encode = tiled_encoder();
+  if (!encode) return cudaErrorNotSupported;
+  const cuuint64_t dims[2] = {32, (cuuint64_t)K * N * 2 / 32};
+  const cuuint64_t strides[1] = {128};
+  const cuuint32_t box[2] = {32, (cuuint32_t)(N / 2)};
+  const cuuint32_t estr[2] = {1, 1};
+  CUresult r = encode(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, bsplit, dims, strides, box, estr,
+                      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+template <int N>
+cudaError_t launch_row_gemm_pair(const RowGemm& g, const CUtensorMap& amap, const CUtensorMap& bmap,
+                                 const CUtensorMap& omap, cudaStream_t st) {
+  static int max_clusters = 0;
+  cudaLaunchConfig_t cfg = {};
+  cfg.blockDim = dim3(RG_THREADS);
+  cfg.dynamicSmemBytes = RP_SMEM;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (max_clusters <= 0) {
+    cudaError_t e = cudaFuncSetAttribute(row_gemm_pair_kernel<N>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)RP_SMEM);
+    if (e != cudaSuccess) return e;
+    cfg.gridDim = dim3((unsigned)sm_count() & ~1u);
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, row_gemm_pair_kernel<N>, &cfg) != cudaSuccess || n <= 0) {
+      cudaGetLastError();
+      n = sm_count() / 2;
+    }
+    max_clusters = n;
+  }
+  const int64_t pairs = (g.rows + 2 * TG_M - 1) / (2 * TG_M);
+  cfg.gridDim = dim3((unsigned)(2 * std::min<int64_t>(pairs, max_clusters)));
+  return cudaLaunchKernelEx(&cfg, row_gemm_pair_kernel<N>, g, amap, bmap, omap);
+}
+
 cudaError_t row_gemm(RowGemm g, cudaStream_t st) {
   if (g.rows == 0) return cudaSuccess;
   if (g.K % GK || g.a_split % GK || g.n_out % 4 || g.ldo % 4 || !al16(g.out))
@@ -1317,6 +1798,16 @@ cudaError_t row_gemm(RowGemm g, cudaStream_t st) {
     if (e == cudaSuccess) e = encode_out_map(&omap, g.out, g.ldo, g.n_out, g.rows);
     if (e != cudaSuccess) return e;
     const int64_t nb = (int64_t)g.K * g.n_out;
+    if (g.rows >= 2 * TG_M) {
+      // CTA pairs: each SM reads half the weights per MMA (see row_gemm_pair_kernel)
+      CUtensorMap bmap;
+      if ((e = encode_bhalf_map(&bmap, g.bsplit, g.K, g.n_out)) != cudaSuccess) return e;
+      split_b_pair_kernel<<<(unsigned)std::min<int64_t>(blocks_for(nb, 256), 1024), 256, 0, st>>>(
+          g.B, g.ldb, g.K, g.n_out, g.bsplit);
+      if ((e = cudaGetLastError()) != cudaSuccess) return e;
+      return wide ? launch_row_gemm_pair<256>(g, amap, bmap, omap, st)
+                  : launch_row_gemm_pair<128>(g, amap, bmap, omap, st);
+    }
     split_b_kernel<<<(unsigned)std::min<int64_t>(blocks_for(nb, 256), 1024), 256, 0, st>>>(
         g.B, g.ldb, g.K, g.n_out, g.bsplit);
     e = cudaGetLastError();
