@@ -747,10 +747,13 @@ __global__ void __launch_bounds__(RG_THREADS, 1) row_gemm_tc_kernel(RowGemm g,
 // of both CTAs and the two weight copies (counted by CTA 0's expect) have
 // arrived, an accumulator is free on CTA 0's barrier when the eight epilogue
 // warps of both CTAs have read it, and the commits arrive on both CTAs.
-constexpr int RP_NSTAGE = 4;
-constexpr int RP_STAGE = 2 * TG_A_HALF + 2 * (128 * TG_KC * 4);    // A hi, lo; B half hi, lo: 32 KB
+constexpr int RP_KC = 32;                                          // K per chunk
+constexpr int RP_A_HALF = TG_M * RP_KC * 4;                        // A hi or lo of a chunk: 16 KB
+constexpr int RP_NSTAGE = 2;
+constexpr int RP_STAGE = 2 * RP_A_HALF + 2 * (128 * RP_KC * 4);    // A hi, lo; B half hi, lo: 64 KB
+constexpr int RP_RAW = TG_M * RP_KC * 4;                           // one raw A chunk, 16 KB
 constexpr int RP_NRAW = 4;
-constexpr int RP_OUT = RP_NSTAGE * RP_STAGE + RP_NRAW * RG_RAW;    // 1024-aligned
+constexpr int RP_OUT = RP_NSTAGE * RP_STAGE + RP_NRAW * RP_RAW;    // 1024-aligned
 constexpr int RP_VEC = RP_OUT + 4 * 2 * RG_OUTB;
 constexpr int RP_BAR = RP_VEC + 2 * 256 * 4;
 constexpr size_t RP_SMEM = (size_t)RP_BAR + 256;
@@ -841,8 +844,8 @@ __device__ __forceinline__ void rp_commit(uint64_t* bar) {
       : "memory");
 }
 
-// B[k][c] -> chunks of 32 K, each [half h][hi | lo][N/2 rows x 32 K] (K-major core
-// matrices of N/2 rows): the half a CTA of the pair holds is one contiguous run.
+// B[k][c] -> chunks of RP_KC K, each [half h][hi | lo][N/2 rows x RP_KC K] (K-major
+// core matrices of N/2 rows): the half a CTA of the pair holds is one contiguous run.
 __global__ void split_b_pair_kernel(const float* __restrict__ B, int64_t ldb, int K, int N,
                                     float* __restrict__ out) {
   const int64_t total = (int64_t)K * N;
@@ -853,10 +856,10 @@ __global__ void split_b_pair_kernel(const float* __restrict__ B, int64_t ldb, in
     const int h = c / Nh, cl = c - h * Nh;
     float hi, lo;
     tg_split(__ldg(B + (int64_t)k * ldb + c), hi, lo);
-    float* ch = out + (int64_t)(k / TG_KC) * 2 * N * TG_KC + (int64_t)h * N * TG_KC;
-    const uint32_t o = tg_off(cl, k % TG_KC, Nh) >> 2;
+    float* ch = out + (int64_t)(k / RP_KC) * 2 * N * RP_KC + (int64_t)h * N * RP_KC;
+    const uint32_t o = tg_off(cl, k % RP_KC, Nh) >> 2;
     ch[o] = hi;
-    ch[Nh * TG_KC + o] = lo;
+    ch[Nh * RP_KC + o] = lo;
   }
 }
 
@@ -866,7 +869,7 @@ __global__ void __launch_bounds__(RG_THREADS, 1) row_gemm_pair_kernel(RowGemm g,
                                                                       const __grid_constant__ CUtensorMap bmap,
                                                                       const __grid_constant__ CUtensorMap omap) {
   constexpr int Nh = N / 2;
-  constexpr uint32_t BH = Nh * TG_KC * 4;        // B half, hi or lo, of a chunk
+  constexpr uint32_t BH = Nh * RP_KC * 4;        // B half, hi or lo, of a chunk
   unsigned* flag = g.flag;
   extern __shared__ __align__(1024) uint8_t tsm[];
   float* s_bias = reinterpret_cast<float*>(tsm + RP_VEC);
@@ -914,11 +917,11 @@ __global__ void __launch_bounds__(RG_THREADS, 1) row_gemm_pair_kernel(RowGemm g,
   rp_cluster_sync();            // both CTAs' barriers exist before any remote use
   tcx::fence_after();
   const uint32_t tmem = *tmem_holder;
-  const int nch = g.K / TG_KC;
+  const int nch = g.K / RP_KC;
   const int64_t ntiles = (g.rows + 2 * TG_M - 1) / (2 * TG_M);   // 256-row pair tiles
   const int64_t cid = rp_cluster(), ncl = rp_nclusters();
   // pair tile i = cid + i * ncl; chunk G of the pair is chunk G % nch of its
-  // tile G / nch and uses stage G % 4 (parity (G / 4) % 2) and raw slot G % 4;
+  // tile G / nch and uses stage G % 2 (parity (G / 2) % 2) and raw slot G % 4;
   // tile i uses accumulator i % 2 (parity (i / 2) % 2). Both CTAs lay out
   // shared memory alike, so the alignment test agrees between them.
   const bool aligned = ((sbase + RP_OUT) & 1023u) == 0;
@@ -949,11 +952,11 @@ __global__ void __launch_bounds__(RG_THREADS, 1) row_gemm_pair_kernel(RowGemm g,
           }
           tcx::fence_after();
           const uint32_t sa = sbase + stage * RP_STAGE;
-          const uint64_t ah = tcx::sdesc(sa, TG_M * 16, 128), al = tcx::sdesc(sa + TG_A_HALF, TG_M * 16, 128);
-          const uint64_t bh = tcx::sdesc(sa + 2 * TG_A_HALF, Nh * 16, 128);
-          const uint64_t bl = tcx::sdesc(sa + 2 * TG_A_HALF + BH, Nh * 16, 128);
+          const uint64_t ah = tcx::sdesc(sa, TG_M * 16, 128), al = tcx::sdesc(sa + RP_A_HALF, TG_M * 16, 128);
+          const uint64_t bh = tcx::sdesc(sa + 2 * RP_A_HALF, Nh * 16, 128);
+          const uint64_t bl = tcx::sdesc(sa + 2 * RP_A_HALF + BH, Nh * 16, 128);
 #pragma unroll
-          for (int s = 0; s < TG_KC / 8; ++s) {
+          for (int s = 0; s < RP_KC / 8; ++s) {
             const uint64_t da = (uint64_t)((s * 2 * TG_M * 16) >> 4), db = (uint64_t)((s * 2 * Nh * 16) >> 4);
             rp_mma(acc, ah + da, bh + db, idesc, (c | s) != 0);
             rp_mma(acc, ah + da, bl + db, idesc, 1);
@@ -979,7 +982,7 @@ __global__ void __launch_bounds__(RG_THREADS, 1) row_gemm_pair_kernel(RowGemm g,
   } else if (warp >= W_BPROD) {
     // ------------------------------------------------------------- weight copies
     // warp W_BPROD + q of each CTA copies that CTA's half of the weights of
-    // chunks G = q, q + 2, ... into stage G % 4 once chunk G - 4's MMAs are done;
+    // chunks G = q, q + 2, ... into stage G % 2 once chunk G - 2's MMAs are done;
     // CTA 0 expects both halves' bytes on its full[] barrier
     if (lane == 0) {
       constexpr uint32_t half_bytes = 2 * BH;
@@ -991,7 +994,7 @@ __global__ void __launch_bounds__(RG_THREADS, 1) row_gemm_pair_kernel(RowGemm g,
         if (rank == 0)
           asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;"
                        ::"r"(tcx::smem_u32(&full[stage])), "r"(2 * half_bytes) : "memory");
-        rp_load_pair(sbase + stage * RP_STAGE + 2 * TG_A_HALF, &bmap, 0, (2 * c + rank) * Nh,
+        rp_load_pair(sbase + stage * RP_STAGE + 2 * RP_A_HALF, &bmap, 0, (2 * c + rank) * (2 * BH / 128),
                      &full[stage]);
       }
       // every copy lands before the final cluster barrier: the issuer waits
@@ -1011,13 +1014,13 @@ __global__ void __launch_bounds__(RG_THREADS, 1) row_gemm_pair_kernel(RowGemm g,
         }
         const int64_t it = G / nch;
         const int c = (int)(G - it * nch);
-        const int k = c * TG_KC;
+        const int k = c * RP_KC;
         const int col = k < g.a_split ? g.a0 + k : g.a1 + k - g.a_split;
         asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;"
-                     ::"r"(tcx::smem_u32(&rfull[slot])), "r"(RG_RAW) : "memory");
+                     ::"r"(tcx::smem_u32(&rfull[slot])), "r"(RP_RAW) : "memory");
         asm volatile(
             "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
-            ::"r"(rawbase + slot * RG_RAW), "l"(reinterpret_cast<uint64_t>(&amap)), "r"(col),
+            ::"r"(rawbase + slot * RP_RAW), "l"(reinterpret_cast<uint64_t>(&amap)), "r"(col),
               "r"((int)tile_row(it)), "r"(tcx::smem_u32(&rfull[slot]))
             : "memory");
         loaded = G;
@@ -1029,9 +1032,13 @@ __global__ void __launch_bounds__(RG_THREADS, 1) row_gemm_pair_kernel(RowGemm g,
     __syncwarp();
   } else if (warp >= RG_EPI / 32) {
     // ------------------------------------------------------------- staging warps
+    // thread st owns row st % 128 of the chunk and its K groups kq = st / 128,
+    // + 2, + 4, + 6 (four K columns each). The raw chunk arrives by a tensor copy
+    // with the 128-byte swizzle (group kq of row r at 16 ((kq ^ (r % 8))) in the
+    // row's 128 bytes), so a quarter-warp (eight consecutive rows, one group)
+    // reads and writes without bank conflicts.
     const int st = tid - RG_EPI;
-    const int src = ((lane & 7) << 2) | (lane >> 3);
-    const int srow = 8 * (st >> 5) + (lane & 7), skq = lane >> 3;
+    const int arow = st & (TG_M - 1), kq0 = st >> 7;
     for (int64_t G = 0; G < total && ok; ++G) {
       const int slot = (int)(G % RP_NRAW), stage = (int)(G % RP_NSTAGE);
       bool w = tcx::mbar_wait(&rfull[slot], (uint32_t)((G / RP_NRAW) & 1), abort_p, flag, kLimit);
@@ -1039,13 +1046,11 @@ __global__ void __launch_bounds__(RG_THREADS, 1) row_gemm_pair_kernel(RowGemm g,
         ok = false;
         break;
       }
-      const float* raw = reinterpret_cast<const float*>(tsm + RP_NSTAGE * RP_STAGE + slot * RG_RAW);
-      const float4 r0 = *reinterpret_cast<const float4*>(raw + 4 * st);
-      const float4 r1 = *reinterpret_cast<const float4*>(raw + 4 * (st + 256));
-      const float4 v0 = make_float4(__shfl_sync(0xffffffffu, r0.x, src), __shfl_sync(0xffffffffu, r0.y, src),
-                                    __shfl_sync(0xffffffffu, r0.z, src), __shfl_sync(0xffffffffu, r0.w, src));
-      const float4 v1 = make_float4(__shfl_sync(0xffffffffu, r1.x, src), __shfl_sync(0xffffffffu, r1.y, src),
-                                    __shfl_sync(0xffffffffu, r1.z, src), __shfl_sync(0xffffffffu, r1.w, src));
+      const uint8_t* raw = tsm + RP_NSTAGE * RP_STAGE + slot * RP_RAW + arow * 128;
+      float4 v[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        v[j] = *reinterpret_cast<const float4*>(raw + (((kq0 + 2 * j) ^ (arow & 7)) * 16));
       w = G < RP_NSTAGE || rp_wait(&done[stage], (uint32_t)((G / RP_NSTAGE - 1) & 1), abort_p, flag, kLimit);
       if (!__all_sync(0xffffffffu, w)) {
         ok = false;
@@ -1053,17 +1058,16 @@ __global__ void __launch_bounds__(RG_THREADS, 1) row_gemm_pair_kernel(RowGemm g,
       }
       const uint32_t sa = sbase + stage * RP_STAGE;
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const float4 v = h ? v1 : v0;
+      for (int j = 0; j < 4; ++j) {
         float hi[4], lo[4];
-        tg_split(v.x, hi[0], lo[0]);
-        tg_split(v.y, hi[1], lo[1]);
-        tg_split(v.z, hi[2], lo[2]);
-        tg_split(v.w, hi[3], lo[3]);
-        const uint32_t o = tg_off(srow + 64 * h, 4 * skq, TG_M);
+        tg_split(v[j].x, hi[0], lo[0]);
+        tg_split(v[j].y, hi[1], lo[1]);
+        tg_split(v[j].z, hi[2], lo[2]);
+        tg_split(v[j].w, hi[3], lo[3]);
+        const uint32_t o = tg_off(arow, 4 * (kq0 + 2 * j), TG_M);
         tcx::st_shared_v4(sa + o, __float_as_uint(hi[0]), __float_as_uint(hi[1]),
                           __float_as_uint(hi[2]), __float_as_uint(hi[3]));
-        tcx::st_shared_v4(sa + TG_A_HALF + o, __float_as_uint(lo[0]), __float_as_uint(lo[1]),
+        tcx::st_shared_v4(sa + RP_A_HALF + o, __float_as_uint(lo[0]), __float_as_uint(lo[1]),
                           __float_as_uint(lo[2]), __float_as_uint(lo[3]));
       }
       tcx::fence_async_smem();
@@ -1719,16 +1723,30 @@ cudaError_t encode_out_map(CUtensorMap* m, float* base, int64_t ld, int cols, in
 }
 
 // The split weights as rows of 128 bytes; a box is one CTA's half of a chunk
-// (N / 2 rows: 16 KB for N = 256).
+// (N rows of 128 bytes: 32 KB for N = 256).
 cudaError_t encode_bhalf_map(CUtensorMap* m, float* bsplit, int K, int N) {
   EncodeTiledFn encode = tiled_encoder();
   if (!encode) return cudaErrorNotSupported;
   const cuuint64_t dims[2] = {32, (cuuint64_t)K * N * 2 / 32};
   const cuuint64_t strides[1] = {128};
-  const cuuint32_t box[2] = {32, (cuuint32_t)(N / 2)};
+  const cuuint32_t box[2] = {32, (cuuint32_t)(N * RP_KC / 32)};
   const cuuint32_t estr[2] = {1, 1};
   CUresult r = encode(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, bsplit, dims, strides, box, estr,
                       CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+// The A rows for the pairs: boxes of RP_KC columns x TG_M rows, 128-byte swizzle.
+cudaError_t encode_rows_map_sw(CUtensorMap* m, const float* base, int64_t ld, int64_t rows) {
+  EncodeTiledFn encode = tiled_encoder();
+  if (!encode) return cudaErrorNotSupported;
+  const cuuint64_t dims[2] = {(cuuint64_t)ld, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)ld * 4};
+  const cuuint32_t box[2] = {RP_KC, TG_M};
+  const cuuint32_t estr[2] = {1, 1};
+  CUresult r = encode(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float*>(base), dims, strides,
+                      box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                       CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
@@ -1798,15 +1816,17 @@ cudaError_t row_gemm(RowGemm g, cudaStream_t st) {
     if (e == cudaSuccess) e = encode_out_map(&omap, g.out, g.ldo, g.n_out, g.rows);
     if (e != cudaSuccess) return e;
     const int64_t nb = (int64_t)g.K * g.n_out;
-    if (g.rows >= 2 * TG_M) {
+    if (g.rows >= 2 * TG_M && g.K % RP_KC == 0 && g.a_split % RP_KC == 0 && g.a0 % RP_KC == 0 &&
+        g.a1 % RP_KC == 0) {
       // CTA pairs: each SM reads half the weights per MMA (see row_gemm_pair_kernel)
-      CUtensorMap bmap;
+      CUtensorMap bmap, amap2;
       if ((e = encode_bhalf_map(&bmap, g.bsplit, g.K, g.n_out)) != cudaSuccess) return e;
+      if ((e = encode_rows_map_sw(&amap2, g.A, g.lda, g.rows)) != cudaSuccess) return e;
       split_b_pair_kernel<<<(unsigned)std::min<int64_t>(blocks_for(nb, 256), 1024), 256, 0, st>>>(
           g.B, g.ldb, g.K, g.n_out, g.bsplit);
       if ((e = cudaGetLastError()) != cudaSuccess) return e;
-      return wide ? launch_row_gemm_pair<256>(g, amap, bmap, omap, st)
-                  : launch_row_gemm_pair<128>(g, amap, bmap, omap, st);
+      return wide ? launch_row_gemm_pair<256>(g, amap2, bmap, omap, st)
+                  : launch_row_gemm_pair<128>(g, amap2, bmap, omap, st);
     }
     split_b_kernel<<<(unsigned)std::min<int64_t>(blocks_for(nb, 256), 1024), 256, 0, st>>>(
         g.B, g.ldb, g.K, g.n_out, g.bsplit);
