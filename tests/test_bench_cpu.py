@@ -50,6 +50,12 @@ def test_nerf_kernel_bytes_of_the_bench_frame():
 def test_nerf_launch_counts_and_rows():
     assert bench.nerf_launches_per_step(S.WORKLOADS["full"]) == 9
     assert bench.nerf_launches_per_step(S.WORKLOADS["tiny"]) == 5
+    # precision TF32, 200x200: the 2^20-sample store takes 16,384 rays of the
+    # coarse pass and 5,461 of the fine one per sub-batch (3 and 8 sub-batches),
+    # each with the encoding, a weight split and a row GEMM per layer (10 layers)
+    # and the heads: 1 + 2 * 2 + (3 + 8) * 22 + 1 + 1 launches (the ncu launch
+    # list of that frame counts the same 249)
+    assert bench.nerf_launches_per_step(S.WORKLOADS["small_tf32"]) == 249
     assert bench.rows_per_frame(S.WORKLOADS["full"]) == 640000 * 256
     assert bench.rows_per_frame(S.WORKLOADS["tiny"]) == 1024 * 64
 
