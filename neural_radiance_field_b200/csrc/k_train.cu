@@ -1,24 +1,29 @@
 // The training step (NeRF page, "7. Training loop": loss =
 // mse(rgb_coarse, target) + mse(rgb_fine, target); the coarse weights are
 // detached before resampling, "6. Hierarchical sampling", so every pass has
-// fixed sample positions). fp32 on the CUDA cores.
+// fixed sample positions), at fp32-level accuracy: the layer GEMMs run on the
+// tensor cores as three tf32 products per fp32 product (hi*hi + hi*lo + lo*hi),
+// the rest in fp32 on the CUDA cores. The same forward, with a compact store,
+// is precision TF32's render.
 //
 // Per pass (rows = rays x samples), the forward writes every layer's output to
 // an activation store, row-major [gamma(x) (64) | h_0 .. h_{D-1} | feature | h_dir]:
-//   encode_store_kernel  sample points and gamma(x)
-//   row_gemm_kernel      one launch per layer, reading the previous layer's columns
-//   heads_fwd_kernel     sigma and rgb (raw outputs)
+//   encode_store_kernel   sample points and gamma(x)
+//   row GEMM              one launch per layer, reading the previous layer's
+//                         columns: row_gemm_pair_kernel (2-SM pairs, 256 rows or
+//                         more), row_gemm_tc_kernel (one CTA), row_gemm_kernel
+//                         (CUDA cores: 64 outputs, other K)
+//   heads_fwd_kernel      sigma and rgb (raw outputs)
 // and the backward reads it:
-//   composite_bw_kernel  d raw (rgb, sigma) per sample and the per-ray loss term
-//   head_bw_kernel       d h_dir through the rgb head, masked by h_dir > 0
-//   row_gemm_kernel      d input = d out x W, + a rank-1 term, masked by the ReLU
-//                        of the layer below
-//   wgrad_gemm_kernel    dW = sum over rows of d out^T x input, and db, in row
-//                        slices added atomically into the gradient blob (fp32
-//                        atomics: the summation order, not the terms, varies
-//                        between runs); wgrad_head_kernel for the 1- and 3-output
-//                        heads
-// All GEMMs share one register-blocked core (128 x 128 tiles, 8 x 8 per thread).
+//   composite_bw_kernel   d raw (rgb, sigma) per sample and the per-ray loss term
+//   head_bw_kernel        d h_dir through the rgb head, masked by h_dir > 0
+//   row GEMM              d input = d out x W, + a rank-1 term, masked by the ReLU
+//                         of the layer below
+//   wgrad_tc_kernel       dW = sum over rows of d out^T x input, and db (the rows as
+//                         the MMA's K; partial tiles added with fp32 atomics: the
+//                         summation order, not the terms, varies between runs);
+//                         wgrad_gemm_kernel on the CUDA cores for other shapes,
+//                         wgrad_head_kernel for the 1- and 3-output heads
 #include <algorithm>
 
 #include <cuda.h>
