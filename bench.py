@@ -14,6 +14,7 @@ Extra lines (`--workload`):
   hashgrid_bf16             the hash grid with its MLP in bf16 on the tensor cores
   sweep24                   24 cameras around the scene in one render call
   compact                   a 4x128 fp32 network on the CUDA-core MLP kernel
+  compact_tf32              the same network with precision TF32
   train                     the training step (loss and both networks' gradients)
   hash_backward             the hash-grid encoding's backward (scatter-add)
 """
@@ -412,7 +413,10 @@ def nerf_launches_per_step(wl):
     for s_pass in ([wl.n_coarse, wl.n_coarse + wl.n_fine] if wl.n_fine else [wl.n_coarse]):
         per = max(1, fw_rows // s_pass)
         n_sub = -(-wl.n_rays // per)
-        net += n_sub * (2 + 2 * (wl.mlp.D + 2))
+        # encoding and heads; a split and a row GEMM per tensor-core layer (the D
+        # trunk layers and the feature layer; the direction layer when its W / 2
+        # outputs are 128), one CUDA-core launch otherwise
+        net += n_sub * (2 + 2 * (wl.mlp.D + 1) + (2 if wl.mlp.W == 256 else 1))
     return 1 + 2 * passes + net + (1 if wl.n_fine else 0) + 1
 
 
@@ -516,7 +520,8 @@ def run_sweep(args, rank, world, local_rank):
 def run_compact(args, rank, world, local_rank):
     """One step = ray generation + a coarse+fine render of the 800x800 frame with a
     compact fp32 network (D=4, W=128, skip after layer 1: a scene-specialised
-    shape in the spirit of the NAS-NeRF page) on the CUDA-core MLP kernel. An
+    shape in the spirit of the NAS-NeRF page) on the CUDA-core MLP kernel, or with
+    precision TF32 (`compact_tf32`: the layer GEMMs on the tensor cores). An
     extra line; the headline is the 8x256 bf16 workload."""
     import dataclasses
     import torch
@@ -525,7 +530,9 @@ def run_compact(args, rank, world, local_rank):
     nbuild.build()
     torch.cuda.set_device(local_rank)
     shape = S.MLPShape(D=4, W=128, skip=1)
-    wl = dataclasses.replace(S.WORKLOADS[WORKLOAD], mlp=shape, precision=S.PREC_FP32)
+    tf32 = args.workload == "compact_tf32"
+    prec = S.PREC_TF32 if tf32 else S.PREC_FP32
+    wl = dataclasses.replace(S.WORKLOADS[WORKLOAD], mlp=shape, precision=prec)
     if args.size:
         wl = dataclasses.replace(wl, H=args.size, W=args.size, focal=1.25 * args.size)
     c2w = wl.c2w().ravel().tolist()
@@ -539,7 +546,7 @@ def run_compact(args, rank, world, local_rank):
     dep = torch.empty(R, device="cuda")
     acc = torch.empty(R, device="cuda")
     flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
-    rnd = nb.Renderer(D=shape.D, W=shape.W, skip=shape.skip, precision=S.PREC_FP32, max_rays=R,
+    rnd = nb.Renderer(D=shape.D, W=shape.W, skip=shape.skip, precision=prec, max_rays=R,
                       max_samples=wl.n_coarse + wl.n_fine)
     p = rnd.params(coarse_w=cwt, fine_w=fwt, seed=wl.seed, perturb=1)
     stream = torch.cuda.current_stream()
@@ -574,21 +581,30 @@ def run_compact(args, rank, world, local_rank):
     sm_mhz = clocks["sm_mhz"] or 1965.0
     peak = 148 * 128 * 2 * sm_mhz * 1e6 / 1e12
     achieved = flop_row * rows * args.steps / (mlp_ms * 1e-3) / 1e12
+    if tf32:
+        peak_kind_tf = load_peaks()[1]
+        roof = {"bound": "tensor", "kernel": "network pass: encoding, tensor-core row GEMMs (tf32 x3), heads",
+                "peak": load_peaks()[0]["bf16_tflops"] * TF32_PER_BF16,
+                "peak_kind": f"tf32 dense: bf16 {peak_kind_tf} x 1.1 / 2.25 (nominal ratio)",
+                "frac_of_fp32_fma": achieved / peak}
+    else:
+        roof = {"bound": "alu", "kernel": "mlp_fp32_kernel (CUDA-core MLP, W=128)", "peak": peak,
+                "peak_kind": FP32_PEAK_NOTE}
     line = {"metric": f"rays/sec at {wl.H}x{wl.W} coarse+fine ({wl.n_coarse}+{wl.n_fine} samples/ray), "
-                      f"compact fp32 network D{shape.D} W{shape.W} skip@{shape.skip}",
+                      f"compact network D{shape.D} W{shape.W} skip@{shape.skip}, "
+                      f"{'fp32 weights, layer GEMMs on the tensor cores (tf32 x3)' if tf32 else 'fp32'}",
             "value": R * args.steps / (tot_ms * 1e-3), "unit": UNIT, "n_gpus": 1,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": tot_ms / args.steps,
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "tf32x3" if tf32 else "f32",
             "data": "synthetic (seeded camera, Xavier-init weights)",
-            "config": {"workload": f"compact_D{shape.D}W{shape.W}_{wl.H}x{wl.W}_fp32",
+            "config": {"workload": f"compact_D{shape.D}W{shape.W}_{wl.H}x{wl.W}_{'tf32x3' if tf32 else 'fp32'}",
                        "mlp": f"{shape.D}x{shape.W} skip@{shape.skip}", "flop_per_row": flop_row,
                        "l2": "flushed between timed steps (256 MiB write)"},
             "mlp_rows_per_s": rows * args.steps / (tot_ms * 1e-3),
-            "roofline": {"bound": "alu", "kernel": "mlp_fp32_kernel (CUDA-core MLP, W=128)",
-                         "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                         "frac": achieved / peak, "peak_kind": FP32_PEAK_NOTE, "traffic": None,
-                         "avg_launch_ms": mlp_ms / max(1, mlp_launches)},
-            "gpu_launches": args.steps * 9, "clocks": clocks}
+            "roofline": dict(roof, achieved=achieved, unit="TFLOP/s", frac=achieved / roof["peak"],
+                             traffic=None, avg_launch_ms=mlp_ms / max(1, mlp_launches)),
+            "gpu_launches": args.steps * nerf_launches_per_step(wl), "clocks": clocks}
     print(json.dumps(line), flush=True)
 
 
@@ -975,7 +991,7 @@ def main():
                     help="rays of the oracle's march sample (march workloads)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--workload", default=WORKLOAD,
-                    choices=[WORKLOAD, "small", "small_tf32", "tiny", "kilonerf", "hashgrid", "hashgrid_bf16",
+                    choices=[WORKLOAD, "small", "small_tf32", "compact_tf32", "tiny", "kilonerf", "hashgrid", "hashgrid_bf16",
                              "sweep24", "compact", "train", "hash_backward"],
                     help="the benchmark workload (default) or a march workload (extra lines)")
     ap.add_argument("--traffic-bytes", type=float, default=0.0,
@@ -992,7 +1008,7 @@ def main():
         run_reference(args, rank, world)
     elif args.workload == "sweep24":
         run_sweep(args, rank, world, local_rank)
-    elif args.workload == "compact":
+    elif args.workload in ("compact", "compact_tf32"):
         run_compact(args, rank, world, local_rank)
     elif args.workload == "train":
         run_train(args, rank, world, local_rank)
