@@ -56,6 +56,12 @@ def test_nerf_launch_counts_and_rows():
     # and the heads: 1 + 2 * 2 + (3 + 8) * 22 + 1 + 1 launches (the ncu launch
     # list of that frame counts the same 249)
     assert bench.nerf_launches_per_step(S.WORKLOADS["small_tf32"]) == 249
+    # the compact 4x128 network at 800x800 with precision TF32: 40 + 118 sub-batches,
+    # the direction layer's 64 outputs on the CUDA-core row GEMM (one launch)
+    import dataclasses
+    compact = dataclasses.replace(S.WORKLOADS["full"], mlp=S.MLPShape(D=4, W=128, skip=1),
+                                  precision=S.PREC_TF32)
+    assert bench.nerf_launches_per_step(compact) == 1 + 2 * 2 + (40 + 118) * 13 + 1 + 1
     assert bench.rows_per_frame(S.WORKLOADS["full"]) == 640000 * 256
     assert bench.rows_per_frame(S.WORKLOADS["tiny"]) == 1024 * 64
 
