@@ -121,7 +121,11 @@ def nerf_test_sh(d, out, stream=None):
 
 
 class Renderer:
-    """Owns a nerf_ctx (nerf_create / nerf_destroy)."""
+    """Owns a nerf_ctx (nerf_create / nerf_destroy). The arguments are the fields
+    of nerf_config (include/nerf.h): precision NERF_FP32 (fused CUDA-core
+    network), NERF_BF16 (the 8x256 network on the tensor cores with bf16
+    weights) or NERF_TF32 (fp32 weights, the layers on the tensor cores as
+    three tf32 products each, at fp32-level accuracy; W of 128 or 256)."""
 
     def __init__(self, model=NERF_MODEL_MLP, D=8, W=256, skip=4, L_pos=10, L_dir=4,
                  sigma_act=NERF_SIGMA_RELU, precision=NERF_FP32, last_delta_mode=NERF_LAST_1E10,
