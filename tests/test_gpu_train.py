@@ -29,11 +29,11 @@ def torch():
     return torch
 
 
-def _gpu_step(torch, wl, o, d, cw, fw, target, perturb=1):
+def _gpu_step(torch, wl, o, d, cw, fw, target, perturb=1, precision=S.PREC_FP32):
     import neural_radiance_field_b200 as nb
     m = wl.mlp
     R = o.shape[0]
-    rnd = nb.Renderer(D=m.D, W=m.W, skip=m.skip, sigma_act=wl.sigma_act, precision=S.PREC_FP32,
+    rnd = nb.Renderer(D=m.D, W=m.W, skip=m.skip, sigma_act=wl.sigma_act, precision=precision,
                       last_delta_mode=wl.last_delta, white_bkgd=wl.white_bkgd, max_rays=R,
                       max_samples=wl.n_coarse + wl.n_fine)
     cwt = torch.from_numpy(cw).cuda()
@@ -105,6 +105,22 @@ def test_many_tiles_step_matches_oracle(torch):
     print(f"[train 800 rays D8W256] loss rel err {abs(loss - ref_loss) / ref_loss:.2e}, "
           f"grad max err / max|g| {err / scale:.2e}")
     assert err <= REL * scale + 1e-9, (err, scale, int(np.abs(gc - ref_gc).argmax()))
+
+
+def test_step_on_a_tf32_context(torch):
+    """nerf_loss_grad on a context of precision TF32 (fp32 weights): the same
+    training path and the same bar as FP32, 8 x 256 network, 35 rays."""
+    wl, cw, fw, target = _setup("small", 5, 7, n_fine=0, mlp=S.MLPShape(D=8, W=256, skip=4),
+                                last_delta=S.LAST_DELTA_TO_FAR)
+    o, d = rays_for(wl)
+    loss, gc, _ = _gpu_step(torch, wl, o, d, cw, None, target, precision=S.PREC_TF32)
+    ref_loss, ref_gc, _ = og.loss_and_grad(wl, o.cpu().numpy(), d.cpu().numpy(), np.arange(wl.n_rays),
+                                           target, cw.astype(np.float64), None)
+    assert abs(loss - ref_loss) <= 1e-5 * ref_loss, (loss, ref_loss)
+    scale = np.abs(ref_gc).max()
+    err = np.abs(gc - ref_gc).max()
+    print(f"[train tf32 context] grad max err / max|g| {err / scale:.2e}")
+    assert err <= REL * scale + 1e-9
 
 
 def test_coarse_and_fine_step(torch):
