@@ -746,12 +746,15 @@ __global__ void __launch_bounds__(RG_THREADS, 1) row_gemm_tc_kernel(RowGemm g,
 // [128, 256) in CTA 1). Each CTA stages its own 128 A rows and holds half of
 // the split weights (N / 2 rows of B), and CTA 0 issues the MMAs for both, so
 // per MMA each SM reads 4 KB of A and 4 KB of B from its shared memory instead
-// of 4 + 8 KB, each CTA copies 16 KB of weights per chunk instead of 32, and one
-// MMA instruction does the work of two. The roles per CTA are the single-CTA
-// kernel's; a stage is full on CTA 0's barrier when the sixteen staging warps
-// of both CTAs and the two weight copies (counted by CTA 0's expect) have
-// arrived, an accumulator is free on CTA 0's barrier when the eight epilogue
-// warps of both CTAs have read it, and the commits arrive on both CTAs.
+// of 4 + 8 KB, each CTA copies half the weights, and one MMA instruction does
+// the work of two. The halved weight stages make room for 32-K chunks in two
+// 64 KB stages (twelve MMAs per barrier wait and commit); the raw A chunks
+// arrive under the 128-byte swizzle, read conflict-free by the staging warps.
+// The roles per CTA are the single-CTA kernel's; a stage is full on CTA 0's
+// barrier when the sixteen staging warps of both CTAs and the two weight
+// copies (counted by CTA 0's expect) have arrived, an accumulator is free on
+// CTA 0's barrier when the eight epilogue warps of both CTAs have read it, and
+// the commits arrive on both CTAs.
 constexpr int RP_KC = 32;                                          // K per chunk
 constexpr int RP_A_HALF = TG_M * RP_KC * 4;                        // A hi or lo of a chunk: 16 KB
 constexpr int RP_NSTAGE = 2;
